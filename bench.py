@@ -1,0 +1,532 @@
+"""Benchmark of the CSA / HCA attention path on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the whole path over one batch of synthetic input:
+  csa_decode (default; batch 32 x 131072-token context, top-k 512, 64 heads x 576 dims,
+  E4M3+BF16 cache, MXFP4 indexer): prepare the query and the newest window row, compress
+  the block the newest token closed, index scores, top-k, sparse attention.
+  csa_prefill / hca_prefill / tiny_csa_prefill: the whole prefill of one sequence.
+  mixed_decode: a CSA decode layer and an HCA decode layer, batch 8, ragged 0.5M-1M.
+Metric: query tokens per second (whole job, all ranks).  Inputs are resident in HBM when
+the timed region starts; L2 is flushed (a 512 MiB write) between timed steps, outside
+the per-step CUDA events.  With N > 1 (torchrun) every rank runs its own batch: weak
+scaling, no collective on the data path.
+--impl reference times the CPU oracle (the plain float64 restatement of the method) on a
+bounded sample of the same workload on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA/HCA attention query-tokens/s at 128K-1M ctx; % of HBM/tensor-pipe roofline"
+UNIT = "query-tokens/s"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="csa_decode",
+                    choices=["csa_decode", "csa_prefill", "hca_prefill", "mixed_decode", "tiny_csa_prefill"])
+    ap.add_argument("--impl", default="lc", choices=["lc", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-s", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def peaks():
+    if os.path.exists(PEAKS_PATH):
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------------
+# algorithmic work per stage (bytes that must move / flops that must be done)
+# ------------------------------------------------------------------------------------
+def _row_bytes(fmt: int, D: int, d_r: int) -> int:
+    return {0: 4 * D, 1: 2 * D, 2: (D - d_r) + 2 * d_r}[fmt]
+
+
+def _n_vis(p, m, W_x, n_ent):
+    return max(0, min((p - W_x + 1) // m, n_ent)) if p - W_x + 1 > 0 else 0
+
+
+def stage_work(spec, inp, run):
+    """{stage: (bytes, flops)} of one step, counting only what the method must touch."""
+    import numpy as np
+    s = spec
+    raw_es = 4 if s.fp32 else 2
+    ent_b = _row_bytes(s.kv_fmt, s.D, s.d_r)
+    win_b = _row_bytes(s.win_fmt, s.D, s.d_r)
+    q_b = _row_bytes(s.q_fmt, s.D, s.d_r)
+    out_b = (4 if s.out_f32 else 2) * s.D
+    idx_key_b = (4 * s.d_I) if s.fp32 else (s.d_I // 2 + s.d_I // 32)
+    idx_q_b = s.H_I * idx_key_b
+    W = s.W
+    work = {}
+    if s.is_decode:
+        B = s.num_seqs
+        pos = [L - 1 for L in s.seq_lens]
+        n_c = list(inp["n_c"])
+        nv = [_n_vis(p, s.m, s.W, n) for p, n in zip(pos, n_c)]
+        nwin = [min(W, p + 1) for p in pos]
+        n_blk = int(sum(1 for L in s.seq_lens if L % s.m == 0))
+        work["qk_prep_q"] = (B * s.H * (s.D * raw_es + q_b), 0)
+        work["qk_prep_win"] = (B * (s.D * raw_es + win_b), 0)
+        work["compress"] = (n_blk * (s.m * (s.D * raw_es + 4) + ent_b), 0)
+        if s.is_csa:
+            K = [min(s.k, v) for v in nv]
+            work["index"] = (sum(v * (idx_key_b + 4) for v in nv) + B * idx_q_b,
+                             sum(2 * v * s.H_I * s.d_I for v in nv))
+            work["topk"] = (sum(4 * v for v in nv) + B * 4 * s.k, 0)
+            sel = K
+        else:
+            sel = nv
+        keys = [a + w for a, w in zip(sel, nwin)]
+        work["attn"] = (sum(a * ent_b + w * win_b for a, w in zip(sel, nwin)) + B * s.H * (q_b + out_b + 4),
+                        sum(4 * s.H * k * s.D for k in keys))
+        units = B
+    else:
+        L, n_c = inp["L"], inp["n_c"]
+        pos = np.arange(s.q_first, s.q_first + s.n_q)
+        nv = np.clip((pos - s.W + 1) // s.m, 0, n_c)
+        nv[pos - s.W + 1 <= 0] = 0
+        nwin = np.minimum(W, pos + 1)
+        n_win_rows = int(inp["win_pos"].numel())
+        work["qk_prep_q"] = (s.n_q * s.H * (s.D * raw_es + q_b), 0)
+        work["qk_prep_win"] = (n_win_rows * (s.D * raw_es + win_b), 0)
+        work["compress"] = (n_c * (s.m * (s.D * raw_es + 4) + ent_b), 0)
+        if s.is_csa:
+            K = np.minimum(s.k, nv)
+            work["index"] = (n_c * idx_key_b + s.n_q * idx_q_b + int(nv.sum()) * 4,
+                             int(nv.sum()) * 2 * s.H_I * s.d_I)
+            work["topk"] = (int(nv.sum()) * 4 + s.n_q * 4 * s.k, 0)
+            sel = K
+        else:
+            sel = nv
+        keys = sel + nwin
+        work["attn"] = (n_c * ent_b + n_win_rows * win_b + s.n_q * s.H * (q_b + out_b + 4),
+                        int(keys.sum()) * 4 * s.H * s.D)
+        units = s.n_q
+    return work, units
+
+
+def bound_of(stage, spec, work, pk):
+    """HBM- or tensor-bound by comparing the two roofline times."""
+    b, f = work[stage]
+    t_mem = b / (pk["hbm_gbs"] * 1e9)
+    t_math = f / (pk["bf16_tflops"] * 1e12) if f else 0.0
+    return ("tensor", t_math) if t_math > t_mem else ("hbm", t_mem)
+
+
+# ------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def kernel_traffic(stage_kernel: str):
+    """DRAM bytes per launch of a kernel from the committed ncu summary, if the kernel's
+    source is unchanged since the capture; else None."""
+    if not os.path.exists(TRAFFIC_PATH):
+        return None
+    with open(TRAFFIC_PATH) as f:
+        t = json.load(f)
+    e = t.get(stage_kernel)
+    if not e:
+        return None
+    src = os.path.join(ROOT, "long_context_sparse_softmax_b200", "csrc", e["source"])
+    if not os.path.exists(src):
+        return None
+    sha = hashlib.sha1(open(src, "rb").read()).hexdigest()
+    if sha != e.get("source_sha1"):
+        return None
+    return e.get("dram_bytes_per_launch_full")
+
+
+STAGE_SOURCE = {"qk_prep_q": "k_prep.cu", "qk_prep_win": "k_prep.cu", "compress": "k_prep.cu",
+                "index": "k_index.cu", "topk": "k_topk.cu", "attn": "k_attn.cu"}
+
+
+# ------------------------------------------------------------------------------------
+# the library arm
+# ------------------------------------------------------------------------------------
+def make_runs(name, device, rank):
+    from long_context_sparse_softmax_b200 import runner
+    from long_context_sparse_softmax_b200 import workloads as wl
+    runs = []
+    for spec in wl.WORKLOADS[name]:
+        if rank:
+            import dataclasses
+            spec = dataclasses.replace(spec, seed=spec.seed + 1000 * rank)
+        inp = (wl.make_decode if spec.is_decode else wl.make_prefill)(spec, device)
+        r = (runner.Decode if spec.is_decode else runner.Prefill)(inp, device)
+        runs.append((spec, inp, r))
+    return runs
+
+
+def host_io(runs):
+    """Per-step inputs (pinned host copies) and outputs of the e2e leg."""
+    import torch
+    io = []
+    for spec, inp, r in runs:
+        names = ["q_raw"]
+        if spec.is_decode:
+            names += ["x_new", "x_tail", "g_tail"]
+        else:
+            names += ["x", "g"]
+        ins = [(inp[n], inp[n].cpu().pin_memory()) for n in names]
+        if spec.is_csa:
+            for t in inp["qI"].values():
+                ins.append((t, t.cpu().pin_memory()))
+        outs = [(r.out, torch.empty(r.out.shape, dtype=r.out.dtype, pin_memory=True)),
+                (r.lse, torch.empty(r.lse.shape, dtype=r.lse.dtype, pin_memory=True))]
+        io.append((ins, outs))
+    return io
+
+
+def run_lc(args):
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    pk, pk_kind = peaks()
+    runs = make_runs(args.workload, dev, rank)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    work = {}
+    units = 0
+    for i, (spec, inp, r) in enumerate(runs):
+        w, u = stage_work(spec, inp, r)
+        for k, v in w.items():
+            work[f"{i}:{k}"] = v
+        units += u if i == 0 else 0  # a mixed step counts each sequence's token once
+    stage_names = [f"{i}:{n}" for i, (_, _, r) in enumerate(runs) for n, _ in r.stages()]
+    stage_fns = [f for (_, _, r) in runs for _, f in r.stages()]
+    n_launch = len(stage_fns)
+
+    for _ in range(args.warmup):
+        for f in stage_fns:
+            f(stream)
+    torch.cuda.synchronize()
+    for _, _, r in runs:
+        assert r.read_status() == 0, "device status bits set"
+
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in stage_fns]
+          for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = str(local)
+    with ClockSampler(gpu_id) as clk:
+        for s in range(args.steps):
+            flush.zero_()
+            for j, f in enumerate(stage_fns):
+                ev[s][j][0].record(stream)
+                f(stream)
+                ev[s][j][1].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    per_stage = {n: [] for n in stage_names}
+    step_ms = []
+    for s in range(args.steps):
+        tot = 0.0
+        for j, n in enumerate(stage_names):
+            t = ev[s][j][0].elapsed_time(ev[s][j][1])
+            per_stage[n].append(t)
+            tot += t
+        step_ms.append(tot)
+    # a step's time runs from its first stage's start to its last stage's end
+    span = [ev[s][0][0].elapsed_time(ev[s][-1][1]) for s in range(args.steps)]
+    total_ms = sum(span)
+    t_max = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t_max, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(t_max.item())
+    value = world * units * args.steps / (total_ms / 1e3)
+
+    # e2e: host inputs in, host outputs back, through the same C-ABI calls
+    e2e = None
+    if not args.no_e2e:
+        io = host_io(runs)
+        h2d = sum(h.numel() * h.element_size() for ins, _ in io for _, h in ins)
+        d2h = sum(h.numel() * h.element_size() for _, outs in io for _, h in outs)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e_ms = 0.0
+        for s in range(args.steps):
+            flush.zero_()
+            e0.record(stream)
+            for ins, _ in io:
+                for d, h in ins:
+                    d.copy_(h, non_blocking=True)
+            for f in stage_fns:
+                f(stream)
+            for _, outs in io:
+                for d, h in outs:
+                    h.copy_(d, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            e_ms += e0.elapsed_time(e1)
+        t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e = {"value": world * units * args.steps / (float(t.item()) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    # roofline of the dominant kernel (largest share of the step)
+    avg = {n: statistics.mean(v) for n, v in per_stage.items()}
+    dom = max(avg, key=avg.get)
+    spec0 = runs[int(dom.split(":")[0])][0]
+    bnd, _ = bound_of(dom, spec0, work, pk)
+    b, f = work[dom]
+    if bnd == "hbm":
+        achieved = b / (avg[dom] / 1e3) / 1e9
+        peak, unit = pk["hbm_gbs"], "GB/s"
+    else:
+        achieved = f / (avg[dom] / 1e3) / 1e12
+        peak, unit = pk["bf16_tflops"], "TFLOP/s"
+    traffic = kernel_traffic(dom.split(":")[1])
+    stages = {}
+    for n in stage_names:
+        bb, ff = work[n]
+        bn, t_roof = bound_of(n, runs[int(n.split(":")[0])][0], work, pk)
+        stages[n] = {"ms": round(avg[n], 5), "share": round(avg[n] / sum(avg.values()), 4),
+                     "bytes": int(bb), "flops": int(ff), "bound": bn,
+                     "roofline_frac": round(t_roof * 1e3 / avg[n], 4) if avg[n] > 0 else None}
+
+    status_ok = all(r.read_status() == 0 for _, _, r in runs)
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3+bf16 KV, mxfp4 indexer, fp32 accumulate" if not runs[0][0].fp32 else "f32",
+        "data": "synthetic",
+        "config": {"workload": runs[0][0].name if len(runs) == 1 else args.workload,
+                   "batch": runs[0][0].num_seqs if runs[0][0].is_decode else 1,
+                   "context": max(runs[0][0].seq_lens), "heads": runs[0][0].H, "dims": runs[0][0].D,
+                   "topk": runs[0][0].k, "query_tokens_per_step_per_gpu": units,
+                   "l2": "flushed between timed steps (512 MiB write outside the step events)",
+                   "parallelism": f"replicas x{world} (independent batches)"},
+        "roofline": {"bound": bnd, "kernel": dom.split(":")[1], "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": pk_kind},
+        "stages": stages,
+        "gpu_launches": n_launch * args.steps,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "status_ok": status_ok,
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        out["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_sample_s)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------------------------------------------
+# the oracle (CPU baseline / reference arm)
+# ------------------------------------------------------------------------------------
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_unit(name: str):
+    """A callable that processes ONE query token of the workload with the oracle (host
+    inputs drawn with the same generators), plus a description."""
+    import numpy as np
+    from long_context_sparse_softmax_b200 import workloads as wl
+    from oracle import lc_oracle as O
+    from oracle import pipeline as P
+    spec = wl.WORKLOADS[name][0]
+    if spec.is_decode:
+        # one sequence of the batch: index over its whole visible cache, top-k, attention
+        one = wl.shrink(spec, seq_lens=spec.seq_lens[:1])
+        inp = wl.make_decode(one, "cpu")
+        cache = inp["cache"]
+        ent = O.rows_to_f64(one.kv_fmt, cache["x"].numpy(), cache.get("rope").numpy() if "rope" in cache else None)
+        win = O.rows_to_f64(one.win_fmt, inp["win"].numpy())
+        p = one.seq_lens[0] - 1
+        qr = P.raw_rows(one.raw_fmt, inp["q_raw"].numpy())
+        sink = inp["sink"].numpy().astype(np.float64)
+
+        def unit():
+            q, _, _ = P.stored(one.q_fmt, O.qk_prep(qr, np.array([p]), one.rope_off, one.d_r), one.d_n)
+            if one.is_csa:
+                qI = P.indexer_f64(one.idx_fmt, {k: v.numpy() for k, v in inp["qI"].items()})[0]
+                kI = P.indexer_f64(one.idx_fmt, {k: v.numpy() for k, v in inp["kI"].items()})
+                idx, _, _ = P.select(qI, kI, inp["w"].numpy().astype(np.float64), p, one.m, one.W, one.k)
+            else:
+                idx = range(O.n_visible(p, one.m, one.W, ent.shape[0]))
+            return O.sparse_attn_query(q[0], ent, idx, win, max(0, p - one.W + 1), p, one.W, sink, one.scale)
+        return unit, f"{name}: one sequence (context {one.seq_lens[0]}) per unit, float64 oracle"
+    # prefill: one query of the sequence (entries compressed once, outside the timing)
+    small_n = 1
+    inp = wl.make_prefill(spec, "cpu")
+    x_bits = inp["x"].numpy()
+    xfun = lambda r0, n: P.raw_rows(spec.raw_fmt, x_bits[r0:r0 + n])
+    ent, _, _ = P.entries_from_tokens(xfun, inp["g"].numpy().astype(np.float64), spec.m, spec.rope_off, spec.d_r,
+                                      spec.kv_fmt, spec.d_n)
+    sink = inp["sink"].numpy().astype(np.float64)
+    rng = np.random.default_rng(0)
+    qs = rng.integers(0, spec.n_q, 64)
+    state = {"i": 0}
+
+    def unit():
+        i = int(qs[state["i"] % len(qs)])
+        state["i"] += 1
+        p = spec.q_first + i
+        ts = list(O.window_positions(p, spec.W))
+        raw = P.raw_rows(spec.raw_fmt, x_bits[ts])
+        win, _, _ = P.stored(spec.win_fmt, O.qk_prep(raw, np.array(ts), spec.rope_off, spec.d_r), spec.d_n)
+        qr = P.raw_rows(spec.raw_fmt, inp["q_raw"][i:i + 1].numpy())
+        q, _, _ = P.stored(spec.q_fmt, O.qk_prep(qr, np.array([p]), spec.rope_off, spec.d_r), spec.d_n)
+        if spec.is_csa:
+            qI = P.indexer_f64(spec.idx_fmt, {k: v[i:i + 1].numpy() for k, v in inp["qI"].items()})[0]
+            kI = P.indexer_f64(spec.idx_fmt, {k: v.numpy() for k, v in inp["kI"].items()})
+            idx, _, _ = P.select(qI, kI, inp["w"].numpy().astype(np.float64), p, spec.m, spec.W, spec.k)
+        else:
+            idx = range(O.n_visible(p, spec.m, spec.W, ent.shape[0]))
+        return O.sparse_attn_query(q[0], ent, idx, win, ts[0], p, spec.W, sink, spec.scale)
+    return unit, f"{name}: one query per unit (entries compressed once beforehand), float64 oracle"
+
+
+def cpu_baseline(name: str, budget_s: float):
+    unit, desc = oracle_unit(name)
+    unit()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        unit()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 10000:
+            break
+    return {"value": n / el, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{desc}; {n} units in {el:.1f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    unit, desc = oracle_unit(args.workload)
+    for _ in range(args.warmup):
+        unit()
+    t = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        unit()
+        t.append(time.perf_counter() - t0)
+    total = sum(t)
+    value = args.steps / total
+    cores = _blas_threads()
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{desc}; one unit per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_lc(a)

@@ -1,0 +1,287 @@
+/*
+ * lc.h — C ABI of the CSA / HCA long-context attention path for NVIDIA B200 (sm_100a).
+ *
+ * The method (DeepSeek-V4 hybrid attention, as described on the pages
+ * "解读 DeepSeek V4" (llm-tech.com.cn), "DeepSeek-V4 论文分析" (ai.kenelite.com) and the
+ * 10100.com technical analysis):
+ *   - Compressed Sparse Attention (CSA): every m = 4 tokens of KV are compressed into
+ *     one entry; a lightning indexer scores the entries per query; the query attends to
+ *     its top-k entries (512 / 1024), a 128-token sliding window of raw tokens and an
+ *     attention sink.
+ *   - Heavily Compressed Attention (HCA): m' = 128, dense attention over every entry
+ *     plus the same window and sink.
+ *   - RMSNorm on queries and KV entries; partial RoPE; KV entries keep the RoPE dims in
+ *     BF16 and the rest in FP8 (E4M3); the indexer runs in FP4 (MXFP4).
+ *
+ * Readings this library takes where the pages are silent:
+ *   gate:    alpha = softmax(g) over the m tokens of a block (one FP32 logit per token),
+ *            entry = RMSNorm(sum alpha_t x_t), then RoPE at the block's last position.
+ *   norm:    RMSNorm with unit weight over all D dims, eps given per call (1e-6 default).
+ *   RoPE:    interleaved pairs (2i, 2i+1) of the d_r RoPE dims, angle pos * base^(-2i/d_r).
+ *   indexer: s(p, j) = sum_h w_h * ReLU(<qI[p, h], kI[j]>), w_h >= 0.
+ *   window:  raw tokens max(0, p-W+1) .. p (prepared with RMSNorm + RoPE like queries).
+ *   visible: entry j is visible to a query at p iff (j+1)*m - 1 <= p - W_x and j < n_ent;
+ *            W_x = W keeps window and entries disjoint (default), W_x = 0 lets them overlap.
+ *   values:  V = K = the full D-dim entry (shared-KV MQA); output D dims per head.
+ *   sink:    one logit per head in the softmax denominator only (unscaled).
+ *   top-k:   K = min(k, n_vis) best scores, ties to the lower index, written in
+ *            ascending index order and padded with -1.
+ *
+ * Conventions
+ *   - Every pointer inside an args struct is a DEVICE pointer unless its comment says
+ *     host.  The caller allocates every input, output and workspace buffer and owns the
+ *     stream; the library allocates nothing, keeps no global state, never synchronises.
+ *     Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - Host-side validation failures return an LC_ERR_* code and launch nothing.
+ *     LC_ERR_LAUNCH reports a CUDA launch error (cudaGetLastError after the launch).
+ *   - Conditions only the device can see (an index out of range, a window row that is
+ *     not present, a block whose tokens are not given) are skipped by the kernel and
+ *     reported by OR-ing LC_DEV_* bits into *status when `status` is non-NULL.
+ *   - Row layouts are dense and row-major.  A query tensor [n_q, H, D] is n_q*H rows.
+ *   - Buffers must be 16-byte aligned (LC_ERR_ALIGN otherwise).
+ *   - Each operation has a _prefill and a _decode entry point taking the same struct.
+ *     Prefill: one sequence, many queries (num_seqs == 1).  Decode: one query per
+ *     sequence (q_start[b] = b).  The variant picks the kernel tiling; results agree.
+ */
+#ifndef LC_H_
+#define LC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t lc_status;
+enum {
+  LC_OK = 0,
+  LC_ERR_ARG = 1,          /* a null pointer, a size out of range, inconsistent shapes */
+  LC_ERR_ALIGN = 2,        /* a buffer not 16-byte aligned */
+  LC_ERR_UNSUPPORTED = 3,  /* a format / shape combination this build has no kernel for */
+  LC_ERR_WORKSPACE = 4,    /* workspace missing or smaller than *_workspace_bytes() */
+  LC_ERR_LAUNCH = 5        /* the CUDA launch failed */
+};
+
+/* Bits OR-ed into *status by the kernels. */
+enum {
+  LC_DEV_BAD_INDEX = 1,    /* a top-k index outside [0, n_ent(b)) other than -1: skipped */
+  LC_DEV_WINDOW_RANGE = 2, /* a window position outside the given window rows: skipped */
+  LC_DEV_BAD_BLOCK = 4,    /* a block whose tokens are not in the given token rows: skipped */
+  LC_DEV_NONVISIBLE = 8    /* a selected entry not visible to its query: skipped */
+};
+
+/* Row storage formats. */
+enum {
+  LC_FMT_F32 = 0,          /* one FP32 array [n, D] */
+  LC_FMT_BF16 = 1,         /* one BF16 array [n, D] */
+  LC_FMT_E4M3_BF16 = 2     /* nope dims E4M3 [n, D - d_r] + RoPE dims BF16 [n, d_r] */
+};
+
+/* Lightning-indexer operand formats. */
+enum {
+  LC_IDX_F32 = 0,          /* FP32 [.., d_I] */
+  LC_IDX_MXFP4 = 3         /* OCP MXFP4: E2M1 codes [.., d_I/2] (element 2i in the low
+                              nibble, 2i+1 in the high nibble) + E8M0 scales [.., d_I/32] */
+};
+
+/* Rows of D logical dims.  In LC_FMT_E4M3_BF16 the logical order is the D - d_r nope
+ * dims followed by the d_r RoPE dims, and rope_off (lc_dims) must equal D - d_r. */
+typedef struct lc_rows {
+  int32_t fmt;
+  int32_t reserved;
+  void* x;                 /* F32/BF16 rows, or the E4M3 nope part */
+  void* rope;              /* E4M3_BF16: BF16 RoPE part [n, d_r]; otherwise NULL */
+} lc_rows;
+
+typedef struct lc_dims {
+  int32_t D;               /* dims per row (multiple of 8, <= 1024) */
+  int32_t d_r;             /* RoPE dims (multiple of 8, <= D) */
+  int32_t rope_off;        /* first RoPE dim inside a row (multiple of 8) */
+  int32_t H;               /* heads per query token (rows per token) */
+} lc_dims;
+
+/* Ragged batch descriptor: device arrays, one entry per sequence. */
+typedef struct lc_batch {
+  int32_t num_seqs;
+  int32_t reserved;
+  const int32_t* q_start;   /* [num_seqs + 1] queries of b are q_start[b] .. q_start[b+1]-1 */
+  const int32_t* q_pos0;    /* [num_seqs] position of the first query of b; query i of b
+                               sits at q_pos0[b] + (i - q_start[b]) */
+  const int64_t* ent_start; /* [num_seqs] row of entry 0 (and indexer key 0) of b */
+  const int32_t* n_ent;     /* [num_seqs] entries stored for b */
+  const int64_t* win_start; /* [num_seqs] row of the first window row of b */
+  const int32_t* win_pos0;  /* [num_seqs] position of that row */
+  const int32_t* win_len;   /* [num_seqs] window rows present for b */
+} lc_batch;
+
+/* ---------------------------------------------------------------------------------
+ * qk_prep — RMSNorm over the D dims, RoPE on the RoPE dims at the token's position,
+ * cast to out.fmt.  Used for queries (H heads share a position) and for window tokens
+ * (H = 1).  Pages: 10100.com analysis §三.1 "辅助优化" (RMSNorm on queries/KV entries,
+ * partial RoPE).
+ * ------------------------------------------------------------------------------- */
+typedef struct lc_qk_prep_args {
+  lc_dims dims;
+  int32_t n_tok;           /* tokens; rows = n_tok * H */
+  int32_t in_fmt;          /* LC_FMT_F32 or LC_FMT_BF16 */
+  const void* x;           /* [n_tok, H, D] raw rows */
+  const int32_t* pos;      /* [n_tok] position of each token */
+  const int64_t* out_tok;  /* optional [n_tok]: token t writes rows out_tok[t]*H .. +H-1
+                              of `out` (e.g. its slot in a window cache); NULL: rows t*H.. */
+  lc_rows out;             /* output rows */
+  float eps;               /* RMSNorm epsilon */
+  float rope_base;         /* RoPE base (10000) */
+  int32_t* status;         /* optional */
+} lc_qk_prep_args;
+
+lc_status lc_qk_prep_prefill(const lc_qk_prep_args* a, void* stream);
+lc_status lc_qk_prep_decode(const lc_qk_prep_args* a, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * csa_compress / hca_compress — for each requested complete block j of sequence b
+ * (tokens j*m .. j*m + m - 1): alpha = softmax(g over the block), c = sum alpha_t x_t,
+ * entry = RoPE(RMSNorm(c), (j+1)*m - 1), cast to out.fmt, written to row
+ * ent_start[b] + j.  Pages: "解读 DeepSeek V4" CSA (m = 4) and HCA (m' = 128) sections;
+ * "DeepSeek-V4 论文分析" §5.2 (learned per-token contribution weights, not an average).
+ * csa_compress takes 1 <= m <= 64; hca_compress takes 64 <= m <= 1024, m % 32 == 0.
+ * Prefill: blk_first = 0, blk_count = L / m.  Decode: the block the newest token closed.
+ * ------------------------------------------------------------------------------- */
+typedef struct lc_compress_args {
+  lc_dims dims;            /* H unused */
+  int32_t m;
+  int32_t num_seqs;
+  int32_t in_fmt;          /* LC_FMT_F32 or LC_FMT_BF16 */
+  int32_t max_blocks;      /* host value: max over b of blk_count[b] */
+  const void* x;           /* raw token rows [*, D] */
+  const float* g;          /* gate logit of each token row */
+  const int64_t* tok_row0; /* [num_seqs] row of the token at position tok_pos0[b] */
+  const int32_t* tok_pos0; /* [num_seqs] */
+  const int32_t* tok_len;  /* [num_seqs] consecutive token rows present for b */
+  const int32_t* blk_first;/* [num_seqs] first block to compress */
+  const int32_t* blk_count;/* [num_seqs] blocks to compress */
+  const int64_t* ent_start;/* [num_seqs] row of entry 0 of b in `out` */
+  lc_rows out;
+  float eps;
+  float rope_base;
+  int32_t* status;
+} lc_compress_args;
+
+lc_status lc_csa_compress_prefill(const lc_compress_args* a, void* stream);
+lc_status lc_csa_compress_decode(const lc_compress_args* a, void* stream);
+lc_status lc_hca_compress_prefill(const lc_compress_args* a, void* stream);
+lc_status lc_hca_compress_decode(const lc_compress_args* a, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * csa_index_scores — lightning indexer: for each query (position p, sequence b) and
+ * each visible entry j < n_vis(p), scores[q, j] = sum_h w_h * ReLU(<qI[q,h], kI[j]>).
+ * Columns j >= n_vis(p) are not written.  Pages: "解读 DeepSeek V4" CSA section and
+ * "FP4 Quantization-Aware Training" (indexer QK path in MXFP4); "DeepSeek-V4 论文分析"
+ * §5.3 and §8.3.
+ * FP32 operands are computed with FP32 FMA (no TF32).  MXFP4 operands are exact
+ * products accumulated in FP32.
+ * ------------------------------------------------------------------------------- */
+typedef struct lc_index_args {
+  int32_t n_q;
+  int32_t H_I;             /* indexer heads (<= 128) */
+  int32_t d_I;             /* indexer dims (F32: multiple of 4, <= 256; MXFP4: 128) */
+  int32_t fmt;             /* LC_IDX_F32 or LC_IDX_MXFP4 */
+  const void* q;           /* F32 [n_q, H_I, d_I] or MXFP4 codes [n_q, H_I, d_I/2] */
+  const uint8_t* q_scale;  /* MXFP4: [n_q, H_I, d_I/32] */
+  const void* k;           /* F32 [n_keys, d_I] or MXFP4 codes [n_keys, d_I/2] */
+  const uint8_t* k_scale;  /* MXFP4: [n_keys, d_I/32] */
+  const float* w;          /* head weights, >= 0: [H_I], or [n_q, H_I] if w_qstride = H_I */
+  int32_t w_qstride;       /* 0 (shared) or H_I */
+  int32_t m;
+  int32_t W_x;
+  int32_t max_ent;         /* host value: max over b of n_ent[b] */
+  lc_batch batch;          /* q_start, q_pos0, ent_start, n_ent */
+  float* scores;           /* [n_q, score_stride] */
+  int64_t score_stride;    /* >= max_ent, multiple of 4 */
+  int32_t* status;
+} lc_index_args;
+
+lc_status lc_csa_index_scores_prefill(const lc_index_args* a, void* stream);
+lc_status lc_csa_index_scores_decode(const lc_index_args* a, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * csa_topk — per query: K = min(k, n_vis(p)) largest scores among columns
+ * 0 .. n_vis(p) - 1, ties to the lower index; idx[q, 0..K-1] ascending, the rest -1;
+ * count[q] = K.  Pages: "解读 DeepSeek V4" CSA section; "DeepSeek-V4 论文分析" §5.3
+ * (Top-512 Flash / Top-1024 Pro).  Bit-exact: the result depends only on the scores.
+ * ------------------------------------------------------------------------------- */
+typedef struct lc_topk_args {
+  int32_t n_q;
+  int32_t k;               /* 1 .. 2048 */
+  int32_t m;
+  int32_t W_x;
+  int32_t max_ent;         /* host value */
+  int32_t reserved;
+  const float* scores;     /* [n_q, score_stride] */
+  int64_t score_stride;
+  lc_batch batch;          /* q_start, q_pos0, n_ent */
+  int32_t* idx;            /* [n_q, k] */
+  int32_t* count;          /* [n_q] or NULL */
+  int32_t* status;
+} lc_topk_args;
+
+lc_status lc_csa_topk_prefill(const lc_topk_args* a, void* stream);
+lc_status lc_csa_topk_decode(const lc_topk_args* a, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * csa_sparse_attn / hca_attn — for each query at p and head h, softmax attention over
+ *   CSA: the selected entries idx[q, :] (-1 skipped), HCA: every visible entry,
+ * joined with the window rows for positions max(0, p-W+1) .. p and the sink logit
+ * sink[h]:  l = scale * <q_h, key>, M = max(sink_h, max l),
+ * Z = e^(sink_h - M) + sum e^(l - M), o = sum e^(l - M) key / Z, lse = M + ln Z.
+ * Pages: "解读 DeepSeek V4" CSA / HCA sections and "其他架构细节" (attention sink);
+ * "DeepSeek-V4 论文分析" §5.4, §六, §七 and §8.4 (sparse core attention).
+ * out: [n_q, H, D] in out_fmt (F32 or BF16); lse: [n_q, H] FP32 (optional).
+ * The decode variant splits the keys of each query across CTAs and needs a workspace
+ * of *_workspace_bytes(a) bytes (0 for prefill).
+ * ------------------------------------------------------------------------------- */
+typedef struct lc_attn_args {
+  lc_dims dims;
+  int32_t n_q;
+  int32_t k;               /* CSA: columns of idx; HCA: ignored */
+  int32_t m;
+  int32_t W;
+  int32_t W_x;
+  int32_t max_ent;         /* host value: max over b of n_ent[b] */
+  float scale;             /* softmax scale (1/sqrt(D)) */
+  int32_t out_fmt;         /* LC_FMT_F32 or LC_FMT_BF16 */
+  lc_rows q;               /* [n_q * H] prepared queries */
+  lc_rows ent;             /* compressed entries */
+  lc_rows win;             /* prepared window rows (LC_FMT_F32 or LC_FMT_BF16) */
+  const int32_t* idx;      /* CSA: [n_q, k] entry index within the sequence, -1 = none */
+  const float* sink;       /* [H] */
+  lc_batch batch;
+  void* out;               /* [n_q, H, D] */
+  float* lse;              /* [n_q, H] or NULL */
+  void* workspace;
+  size_t workspace_bytes;
+  int32_t* status;
+} lc_attn_args;
+
+lc_status lc_csa_sparse_attn_prefill(const lc_attn_args* a, void* stream);
+lc_status lc_csa_sparse_attn_decode(const lc_attn_args* a, void* stream);
+lc_status lc_hca_attn_prefill(const lc_attn_args* a, void* stream);
+lc_status lc_hca_attn_decode(const lc_attn_args* a, void* stream);
+
+size_t lc_csa_sparse_attn_workspace_bytes(const lc_attn_args* a);
+size_t lc_hca_attn_workspace_bytes(const lc_attn_args* a);
+
+/* Library version string (static storage). */
+const char* lc_version(void);
+/* Name of a status code (static storage). */
+const char* lc_status_string(lc_status s);
+/* sizeof of the args structs, for bindings to check their mirrors:
+ * 0 lc_rows, 1 lc_dims, 2 lc_batch, 3 lc_qk_prep_args, 4 lc_compress_args,
+ * 5 lc_index_args, 6 lc_topk_args, 7 lc_attn_args; other values return 0. */
+size_t lc_struct_size(int32_t which);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LC_H_ */

@@ -1,0 +1,36 @@
+// Internal launchers of the CSA / HCA attention library (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "lc_common.cuh"
+
+namespace lc {
+
+cudaError_t launch_qk_prep(const lc_qk_prep_args& a, cudaStream_t st);
+cudaError_t launch_compress(const lc_compress_args& a, bool per_cta, cudaStream_t st);
+cudaError_t launch_index_scores(const lc_index_args& a, bool decode, cudaStream_t st);
+cudaError_t launch_topk(const lc_topk_args& a, bool decode, cudaStream_t st);
+cudaError_t launch_attn(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st);
+size_t attn_workspace_bytes(const lc_attn_args& a, bool sparse, bool decode);
+
+// Sequence of query row q: the b with q_start[b] <= q < q_start[b+1] (binary search).
+__device__ __forceinline__ int seq_of_query(const int32_t* __restrict__ q_start, int num_seqs, int q) {
+  int lo = 0, hi = num_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(q_start + mid) <= q) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Entries visible to a query at p: j with (j+1)*m - 1 <= p - W_x, clamped to [0, n_ent].
+__device__ __forceinline__ int n_visible(int p, int m, int W_x, int n_ent) {
+  const int t = p - W_x + 1;
+  if (t <= 0) return 0;
+  const int v = t / m;
+  return v < n_ent ? v : n_ent;
+}
+
+}  // namespace lc

@@ -1,0 +1,246 @@
+"""Drive a workload through the C ABI: allocate the path's buffers with torch (device
+memory only) and issue the library calls in the method's order.
+
+Prefill (one sequence): prepare queries and window tokens -> compress the context ->
+[CSA: index scores -> top-k] -> attention.  Decode (one query per sequence, on a
+cache): prepare the query and the newest token's window row, compress the block the
+newest token closed, [CSA: index -> top-k] -> attention.
+
+Nothing here computes any part of the method; every step is a kernel of liblc.so.
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import torch
+
+from . import (AttnArgs, Batch, CompressArgs, Dims, IndexArgs, QkPrepArgs, Rows, TopkArgs,
+               LC_FMT_BF16, LC_FMT_E4M3_BF16, LC_FMT_F32, LC_IDX_F32, LC_IDX_MXFP4,
+               lc_csa_compress_decode, lc_csa_compress_prefill, lc_csa_index_scores_decode,
+               lc_csa_index_scores_prefill, lc_csa_sparse_attn_decode, lc_csa_sparse_attn_prefill,
+               lc_csa_sparse_attn_workspace_bytes, lc_csa_topk_decode, lc_csa_topk_prefill,
+               lc_hca_attn_decode, lc_hca_attn_prefill, lc_hca_attn_workspace_bytes,
+               lc_hca_compress_decode, lc_hca_compress_prefill, lc_qk_prep_decode, lc_qk_prep_prefill)
+from . import workloads as wl
+
+RMS_EPS = 1e-6
+ROPE_BASE = 10000.0
+
+
+def ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def alloc_rows(fmt: int, n: int, D: int, d_r: int, device) -> Dict[str, torch.Tensor]:
+    if fmt == LC_FMT_F32:
+        return {"x": torch.empty(n, D, dtype=torch.float32, device=device)}
+    if fmt == LC_FMT_BF16:
+        return {"x": torch.empty(n, D, dtype=torch.int16, device=device)}
+    return {"x": torch.empty(n, D - d_r, dtype=torch.uint8, device=device),
+            "rope": torch.empty(n, d_r, dtype=torch.int16, device=device)}
+
+
+def rows(fmt: int, r: Dict[str, torch.Tensor]) -> Rows:
+    return Rows(fmt, 0, ptr(r["x"]), ptr(r.get("rope")))
+
+
+def batch(bd: Dict[str, torch.Tensor]) -> Batch:
+    return Batch(int(bd["n_ent"].numel()), 0, ptr(bd["q_start"]), ptr(bd["q_pos0"]), ptr(bd["ent_start"]),
+                 ptr(bd["n_ent"]), ptr(bd["win_start"]), ptr(bd["win_pos0"]), ptr(bd["win_len"]))
+
+
+def _round4(n: int) -> int:
+    return max(4, (n + 3) // 4 * 4)
+
+
+class _Common:
+    def _index_args(self, n_q: int, max_ent: int, scores: torch.Tensor) -> IndexArgs:
+        s, inp = self.spec, self.inp
+        qI, kI = inp["qI"], inp["kI"]
+        mx = s.idx_fmt == wl.IDX_MXFP4
+        return IndexArgs(n_q, s.H_I, s.d_I, LC_IDX_MXFP4 if mx else LC_IDX_F32,
+                         ptr(qI["codes"] if mx else qI["f32"]), ptr(qI.get("scales")),
+                         ptr(kI["codes"] if mx else kI["f32"]), ptr(kI.get("scales")),
+                         ptr(inp["w"]), 0, s.m, self.W_x, max_ent, self.batch,
+                         ptr(scores), scores.shape[1], ptr(self.status))
+
+    def _topk_args(self, n_q: int, max_ent: int) -> TopkArgs:
+        s = self.spec
+        return TopkArgs(n_q, s.k, s.m, self.W_x, max_ent, 0, ptr(self.scores), self.scores.shape[1], self.batch,
+                        ptr(self.idx), ptr(self.count), ptr(self.status))
+
+    def _attn_args(self, n_q: int, max_ent: int, sparse: bool) -> AttnArgs:
+        s = self.spec
+        a = AttnArgs()
+        a.dims = self.dims
+        a.n_q, a.k, a.m, a.W, a.W_x, a.max_ent = n_q, (s.k if sparse else 0), s.m, s.W, self.W_x, max_ent
+        a.scale = s.scale
+        a.out_fmt = LC_FMT_F32 if s.out_f32 else LC_FMT_BF16
+        a.q = rows(s.q_fmt, self.q)
+        a.ent = rows(s.kv_fmt, self.ent)
+        a.win = rows(s.win_fmt, self.win)
+        a.idx = ptr(self.idx) if sparse else None
+        a.sink = ptr(self.inp["sink"])
+        a.batch = self.batch
+        a.out = ptr(self.out)
+        a.lse = ptr(self.lse)
+        a.status = ptr(self.status)
+        ws = (lc_csa_sparse_attn_workspace_bytes if sparse else lc_hca_attn_workspace_bytes)(a)
+        self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.device)
+        a.workspace, a.workspace_bytes = ptr(self.workspace), ws
+        return a
+
+    def read_status(self) -> int:
+        return int(self.status.item())
+
+
+class Prefill(_Common):
+    """One sequence of L raw tokens; queries at q_first .. q_first + n_q - 1."""
+
+    def __init__(self, inp: Dict[str, object], device="cuda", W_x: Optional[int] = None):
+        s: wl.Spec = inp["spec"]
+        self.spec, self.inp, self.device = s, inp, device
+        self.W_x = s.W if W_x is None else W_x
+        L, n_c = inp["L"], inp["n_c"]
+        self.dims = Dims(s.D, s.d_r, s.rope_off, s.H)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.ent = alloc_rows(s.kv_fmt, max(n_c, 1), s.D, s.d_r, device)
+        n_win = int(inp["win_pos"].numel())
+        self.win = alloc_rows(s.win_fmt, n_win, s.D, s.d_r, device)
+        self.q = alloc_rows(s.q_fmt, s.n_q * s.H, s.D, s.d_r, device)
+        self.batch = batch(inp["batch"])
+        i32 = dict(dtype=torch.int32, device=device)
+        i64 = dict(dtype=torch.int64, device=device)
+        self._cmp = {"tok_row0": torch.zeros(1, **i64), "tok_pos0": torch.zeros(1, **i32),
+                     "tok_len": torch.tensor([L], **i32), "blk_first": torch.zeros(1, **i32),
+                     "blk_count": torch.tensor([n_c], **i32), "ent_start": torch.zeros(1, **i64)}
+        c = self._cmp
+        self.a_compress = CompressArgs(Dims(s.D, s.d_r, s.rope_off, 1), s.m, 1, s.raw_fmt, n_c, ptr(inp["x"]),
+                                       ptr(inp["g"]), ptr(c["tok_row0"]), ptr(c["tok_pos0"]), ptr(c["tok_len"]),
+                                       ptr(c["blk_first"]), ptr(c["blk_count"]), ptr(c["ent_start"]),
+                                       rows(s.kv_fmt, self.ent), RMS_EPS, ROPE_BASE, ptr(self.status))
+        self.a_prep_q = QkPrepArgs(self.dims, s.n_q, s.raw_fmt, ptr(inp["q_raw"]), ptr(inp["q_pos"]), None,
+                                   rows(s.q_fmt, self.q), RMS_EPS, ROPE_BASE, ptr(self.status))
+        x_win = inp["x"][inp["win_pos0"]:]
+        self.a_prep_win = QkPrepArgs(Dims(s.D, s.d_r, s.rope_off, 1), n_win, s.raw_fmt, ptr(x_win),
+                                     ptr(inp["win_pos"]), None, rows(s.win_fmt, self.win), RMS_EPS, ROPE_BASE,
+                                     ptr(self.status))
+        self.out = torch.empty(s.n_q * s.H, s.D, dtype=torch.float32 if s.out_f32 else torch.int16, device=device)
+        self.lse = torch.empty(s.n_q * s.H, dtype=torch.float32, device=device)
+        if s.is_csa:
+            self.scores = torch.empty(s.n_q, _round4(n_c), dtype=torch.float32, device=device)
+            self.idx = torch.empty(s.n_q, s.k, dtype=torch.int32, device=device)
+            self.count = torch.empty(s.n_q, dtype=torch.int32, device=device)
+            self.a_index = self._index_args(s.n_q, n_c, self.scores)
+            self.a_topk = self._topk_args(s.n_q, n_c)
+        else:
+            self.idx = None
+        self.a_attn = self._attn_args(s.n_q, n_c, s.is_csa)
+
+    def prep_queries(self, stream=None):
+        lc_qk_prep_prefill(self.a_prep_q, stream)
+
+    def prep_window(self, stream=None):
+        lc_qk_prep_prefill(self.a_prep_win, stream)
+
+    def compress(self, stream=None):
+        (lc_csa_compress_prefill if self.spec.is_csa else lc_hca_compress_prefill)(self.a_compress, stream)
+
+    def index(self, stream=None):
+        lc_csa_index_scores_prefill(self.a_index, stream)
+
+    def topk(self, stream=None):
+        lc_csa_topk_prefill(self.a_topk, stream)
+
+    def attn(self, stream=None):
+        (lc_csa_sparse_attn_prefill if self.spec.is_csa else lc_hca_attn_prefill)(self.a_attn, stream)
+
+    def stages(self):
+        st = [("qk_prep_q", self.prep_queries), ("qk_prep_win", self.prep_window), ("compress", self.compress)]
+        if self.spec.is_csa:
+            st += [("index", self.index), ("topk", self.topk)]
+        return st + [("attn", self.attn)]
+
+    def step(self, stream=None):
+        for _, f in self.stages():
+            f(stream)
+
+
+class Decode(_Common):
+    """B sequences, one query each at L_b - 1, on an existing cache (see workloads.make_decode)."""
+
+    def __init__(self, inp: Dict[str, object], device="cuda", W_x: Optional[int] = None):
+        s: wl.Spec = inp["spec"]
+        self.spec, self.inp, self.device = s, inp, device
+        self.W_x = s.W if W_x is None else W_x
+        B = s.num_seqs
+        n_c = inp["n_c"]
+        max_ent = max(n_c)
+        self.dims = Dims(s.D, s.d_r, s.rope_off, s.H)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.ent = inp["cache"]
+        self.win = {"x": inp["win"]}
+        self.q = alloc_rows(s.q_fmt, B * s.H, s.D, s.d_r, device)
+        self.batch = batch(inp["batch"])
+        i32 = dict(dtype=torch.int32, device=device)
+        i64 = dict(dtype=torch.int64, device=device)
+        L = s.seq_lens
+        self._cmp = {"tok_row0": torch.tensor([b * s.m for b in range(B)], **i64),
+                     "tok_pos0": torch.tensor([Lb - s.m for Lb in L], **i32),
+                     "tok_len": torch.tensor([s.m] * B, **i32)}
+        c = self._cmp
+        self.a_compress = CompressArgs(Dims(s.D, s.d_r, s.rope_off, 1), s.m, B, s.raw_fmt, 1, ptr(inp["x_tail"]),
+                                       ptr(inp["g_tail"]), ptr(c["tok_row0"]), ptr(c["tok_pos0"]), ptr(c["tok_len"]),
+                                       ptr(inp["blk_first"]), ptr(inp["blk_count"]), ptr(inp["batch"]["ent_start"]),
+                                       rows(s.kv_fmt, self.ent), RMS_EPS, ROPE_BASE, ptr(self.status))
+        self.a_prep_q = QkPrepArgs(self.dims, B, s.raw_fmt, ptr(inp["q_raw"]), ptr(inp["q_pos"]), None,
+                                   rows(s.q_fmt, self.q), RMS_EPS, ROPE_BASE, ptr(self.status))
+        self.win_slot = torch.tensor([b * s.W + (Lb - 1 - max(0, Lb - s.W)) for b, Lb in enumerate(L)], **i64)
+        self.a_prep_win = QkPrepArgs(Dims(s.D, s.d_r, s.rope_off, 1), B, s.raw_fmt, ptr(inp["x_new"]),
+                                     ptr(inp["q_pos"]), ptr(self.win_slot), rows(s.win_fmt, self.win), RMS_EPS,
+                                     ROPE_BASE, ptr(self.status))
+        self.out = torch.empty(B * s.H, s.D, dtype=torch.float32 if s.out_f32 else torch.int16, device=device)
+        self.lse = torch.empty(B * s.H, dtype=torch.float32, device=device)
+        if s.is_csa:
+            self.scores = torch.empty(B, _round4(max_ent), dtype=torch.float32, device=device)
+            self.idx = torch.empty(B, s.k, dtype=torch.int32, device=device)
+            self.count = torch.empty(B, dtype=torch.int32, device=device)
+            self.a_index = self._index_args(B, max_ent, self.scores)
+            self.a_topk = self._topk_args(B, max_ent)
+        else:
+            self.idx = None
+        self.a_attn = self._attn_args(B, max_ent, s.is_csa)
+
+    def prep_queries(self, stream=None):
+        lc_qk_prep_decode(self.a_prep_q, stream)
+
+    def prep_window(self, stream=None):
+        lc_qk_prep_decode(self.a_prep_win, stream)
+
+    def compress(self, stream=None):
+        (lc_csa_compress_decode if self.spec.is_csa else lc_hca_compress_decode)(self.a_compress, stream)
+
+    def index(self, stream=None):
+        lc_csa_index_scores_decode(self.a_index, stream)
+
+    def topk(self, stream=None):
+        lc_csa_topk_decode(self.a_topk, stream)
+
+    def attn(self, stream=None):
+        (lc_csa_sparse_attn_decode if self.spec.is_csa else lc_hca_attn_decode)(self.a_attn, stream)
+
+    def stages(self):
+        st = [("qk_prep_q", self.prep_queries), ("qk_prep_win", self.prep_window), ("compress", self.compress)]
+        if self.spec.is_csa:
+            st += [("index", self.index), ("topk", self.topk)]
+        return st + [("attn", self.attn)]
+
+    def step(self, stream=None):
+        for _, f in self.stages():
+            f(stream)
+
+
+def make_run(spec: wl.Spec, device="cuda", W_x: Optional[int] = None):
+    if spec.is_decode:
+        return Decode(wl.make_decode(spec, device), device, W_x)
+    return Prefill(wl.make_prefill(spec, device), device, W_x)

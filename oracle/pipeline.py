@@ -31,13 +31,14 @@ def indexer_f64(fmt: int, op: Dict[str, np.ndarray]) -> np.ndarray:
     return O.mxfp4_to_f64(op["codes"], op["scales"])
 
 
-def entries_from_tokens(x: np.ndarray, g: np.ndarray, m: int, lo: int, d_r: int, kv_fmt: int, d_n: int,
+def entries_from_tokens(x, g: np.ndarray, m: int, lo: int, d_r: int, kv_fmt: int, d_n: int,
                         first_block: int = 0, n_blocks=None, tok_pos0: int = 0, chunk: int = 4096):
     """Compress complete blocks of raw token rows (float64), then cast to the entry format.
 
-    Processes `chunk` blocks at a time so a 1M-token context fits in memory."""
+    x is a float64 array [T, D] or a callable (r0, n) -> rows r0..r0+n-1 as float64, so a
+    1M-token context is converted `chunk` blocks at a time."""
     if n_blocks is None:
-        n_blocks = (tok_pos0 + x.shape[0]) // m - first_block
+        n_blocks = (tok_pos0 + g.shape[0]) // m - first_block
     parts_f, parts_x, parts_r = [], [], []
     for b0 in range(0, n_blocks, chunk):
         nb = min(chunk, n_blocks - b0)
@@ -49,7 +50,7 @@ def entries_from_tokens(x: np.ndarray, g: np.ndarray, m: int, lo: int, d_r: int,
         parts_f.append(f)
         parts_x.append(sx)
         parts_r.append(sr)
-    f = np.concatenate(parts_f) if parts_f else np.zeros((0, x.shape[1]))
+    f = np.concatenate(parts_f) if parts_f else np.zeros((0, 0))
     sx = np.concatenate(parts_x) if parts_x else None
     sr = np.concatenate(parts_r) if parts_r and parts_r[0] is not None else None
     return f, sx, sr

@@ -1,0 +1,209 @@
+"""Stage-by-stage and end-to-end comparison of a library run with the oracle (GPU tests).
+
+Every stage is checked twice where it makes sense:
+  * stage-wise: the stage's inputs are the oracle's own values (written into the library's
+    buffers), so the comparison isolates that kernel;
+  * end to end: the library's whole path against the oracle's whole path.
+"""
+from __future__ import annotations
+
+from typing import Sequence
+
+import numpy as np
+import torch
+
+from oracle import lc_oracle as O
+from long_context_sparse_softmax_b200 import runner
+from long_context_sparse_softmax_b200 import workloads as wl
+from tests.oracle_ref import (OracleDecode, OraclePrefill, attn_ok, np_, out_np, rows_np, stored_close,
+                              topk_sets_ok, write_rows)
+
+
+def _sync():
+    torch.cuda.synchronize()
+
+
+def check_prefill(spec: wl.Spec, q_sel: Sequence[int] = None, W_x: int = None, report=None):
+    """Run a prefill workload through the library and compare it with the oracle on the
+    queries q_sel (local indices; all queries if None)."""
+    dev = "cuda"
+    inp = wl.make_prefill(spec, dev)
+    run = runner.Prefill(inp, dev, W_x)
+    run.step()
+    _sync()
+    assert run.read_status() == 0, f"device status {run.read_status()}"
+    q_sel = list(range(spec.n_q)) if q_sel is None else list(q_sel)
+    orc = OraclePrefill(inp, q_sel, W_x)
+    d_n = spec.d_n
+    rep = {} if report is None else report
+
+    # compression
+    n_c = inp["n_c"]
+    got = rows_np(spec.kv_fmt, run.ent)[:n_c]
+    ok = stored_close(spec.kv_fmt, got, orc.ent_f, d_n)
+    rep["entries_off_grid"] = int((~ok).sum())
+    assert ok.all(), f"entries: {(~ok).sum()} elements beyond one grid step"
+
+    # window rows the sampled queries use
+    if orc.win_pos.size:
+        sel = torch.as_tensor(orc.win_pos - inp["win_pos0"], device=dev)
+        got = rows_np(spec.win_fmt, run.win, sel)
+        ok = stored_close(spec.win_fmt, got, orc.win_f, d_n)
+        assert ok.all(), f"window rows: {(~ok).sum()} elements beyond one grid step"
+
+    # queries (rows of all heads of the sampled queries)
+    qrows = torch.as_tensor([i * spec.H + h for i in q_sel for h in range(spec.H)], device=dev)
+    got = rows_np(spec.q_fmt, run.q, qrows).reshape(len(q_sel), spec.H, spec.D)
+    ok = stored_close(spec.q_fmt, got, orc.q_f, d_n)
+    assert ok.all(), f"queries: {(~ok).sum()} elements beyond one grid step"
+
+    e2e_out = out_np(run, q_sel)
+    e2e_idx = np_(run.idx)[q_sel] if spec.is_csa else None
+    sel_t = torch.as_tensor(q_sel, device=dev)
+
+    exp_idx = {}
+    if spec.is_csa:
+        scores_gpu = np_(run.scores)
+        s_or = {}
+        n_diff = 0
+        for i, q in enumerate(q_sel):
+            s, bnd = orc.scores(i)
+            s_or[i] = s
+            g = scores_gpu[q, :s.shape[0]].astype(np.float64)
+            assert np.all(np.abs(g - s) <= bnd), f"scores of query {q}: max err {np.max(np.abs(g - s))}"
+            exp_idx[i] = O.topk(s, spec.k)
+            ok_i, nd, why = topk_sets_ok(e2e_idx[i], exp_idx[i], s, spec.k, spec.fp32, bnd)
+            assert ok_i, f"top-k of query {q}: {why}"
+            n_diff += nd
+        rep["topk_e2e_set_diff"] = n_diff
+        # top-k stage-wise: identical FP32 scores on both sides -> bit-exact
+        s32 = torch.full_like(run.scores, float("nan"))
+        for i, q in enumerate(q_sel):
+            s32[q, :s_or[i].shape[0]] = torch.from_numpy(s_or[i].astype(np.float32)).to(dev)
+        run.scores.copy_(s32)
+        run.topk()
+        _sync()
+        got_idx = np_(run.idx)[q_sel]
+        for i, q in enumerate(q_sel):
+            exp = O.topk(s_or[i].astype(np.float32).astype(np.float64), spec.k)
+            e = -np.ones(spec.k, dtype=np.int64)
+            e[:exp.shape[0]] = exp
+            assert np.array_equal(got_idx[i], e), f"top-k (identical scores) of query {q} differs"
+            exp_idx[i] = exp
+        assert np.array_equal(np_(run.count)[q_sel], [len(exp_idx[i]) for i in range(len(q_sel))])
+
+    # attention, stage-wise on the oracle's inputs
+    write_rows(run.ent, spec.kv_fmt, orc.ent_f, d_n, slice(0, n_c))
+    if orc.win_pos.size:
+        write_rows(run.win, spec.win_fmt, orc.win_f, d_n,
+                   torch.as_tensor(orc.win_pos - inp["win_pos0"], device=dev))
+    write_rows(run.q, spec.q_fmt, orc.q_f.reshape(-1, spec.D), d_n, qrows)
+    if spec.is_csa:
+        idx_t = run.idx.clone()
+        for i, q in enumerate(q_sel):
+            e = -np.ones(spec.k, dtype=np.int32)
+            e[:exp_idx[i].shape[0]] = exp_idx[i]
+            idx_t[q] = torch.from_numpy(e).to(dev)
+        run.idx.copy_(idx_t)
+    run.attn()
+    _sync()
+    assert run.read_status() == 0
+    got = out_np(run, q_sel)
+    got_lse = np_(run.lse.view(-1, spec.H))[q_sel]
+    worst = 0.0
+    for i, q in enumerate(q_sel):
+        o, lse = orc.attend(i, exp_idx.get(i))
+        ok_i, err, tol = attn_ok(got[i], o, spec.out_f32)
+        worst = max(worst, err / tol)
+        assert ok_i, f"attention (oracle inputs) query {q}: err {err} > tol {tol}"
+        np.testing.assert_allclose(got_lse[i], lse, rtol=0, atol=1e-4 if spec.out_f32 else 2e-3)
+        # end to end: the library's own pipeline, where it selected the same entries
+        if not spec.is_csa or set(int(v) for v in e2e_idx[i] if v >= 0) == set(int(v) for v in exp_idx[i]):
+            ok_e, err_e, tol_e = attn_ok(e2e_out[i], o, spec.out_f32)
+            assert ok_e, f"attention (end to end) query {q}: err {err_e} > tol {tol_e}"
+    rep["attn_worst_err_over_tol"] = worst
+    return rep
+
+
+def check_decode(spec: wl.Spec, W_x: int = None, report=None):
+    dev = "cuda"
+    inp = wl.make_decode(spec, dev)
+    run = runner.Decode(inp, dev, W_x)
+    run.step()
+    _sync()
+    assert run.read_status() == 0, f"device status {run.read_status()}"
+    orc = OracleDecode(inp, W_x)
+    B = spec.num_seqs
+    d_n = spec.d_n
+    rep = {} if report is None else report
+
+    # decode-time compression of the closed block
+    for b, f in orc.new_entry.items():
+        r = orc.ent_start[b] + spec.seq_lens[b] // spec.m - 1
+        got = rows_np(spec.kv_fmt, run.ent, torch.as_tensor([r], device=dev))[0]
+        assert stored_close(spec.kv_fmt, got, f, d_n).all(), f"decode compression of sequence {b}"
+    # newest window rows
+    got = rows_np(spec.win_fmt, run.win, run.win_slot)
+    assert stored_close(spec.win_fmt, got, orc.new_win, d_n).all(), "newest window rows"
+    # queries
+    got = rows_np(spec.q_fmt, run.q).reshape(B, spec.H, spec.D)
+    assert stored_close(spec.q_fmt, got, orc.q_f, d_n).all(), "queries"
+
+    e2e_out = out_np(run, range(B))
+    exp_idx = {}
+    if spec.is_csa:
+        e2e_idx = np_(run.idx)
+        scores_gpu = np_(run.scores)
+        s_or = {}
+        n_diff = 0
+        for b in range(B):
+            s, bnd = orc.scores(b)
+            s_or[b] = s
+            g = scores_gpu[b, :s.shape[0]].astype(np.float64)
+            assert np.all(np.abs(g - s) <= bnd), f"scores of sequence {b}: max err {np.max(np.abs(g - s))}"
+            exp_idx[b] = O.topk(s, spec.k)
+            ok_b, nd, why = topk_sets_ok(e2e_idx[b], exp_idx[b], s, spec.k, spec.fp32, bnd)
+            assert ok_b, f"top-k of sequence {b}: {why}"
+            n_diff += nd
+        rep["topk_e2e_set_diff"] = n_diff
+        s32 = torch.full_like(run.scores, float("nan"))
+        for b in range(B):
+            s32[b, :s_or[b].shape[0]] = torch.from_numpy(s_or[b].astype(np.float32)).to(dev)
+        run.scores.copy_(s32)
+        run.topk()
+        _sync()
+        got_idx = np_(run.idx)
+        for b in range(B):
+            exp = O.topk(s_or[b].astype(np.float32).astype(np.float64), spec.k)
+            e = -np.ones(spec.k, dtype=np.int64)
+            e[:exp.shape[0]] = exp
+            assert np.array_equal(got_idx[b], e), f"top-k (identical scores) of sequence {b}"
+            exp_idx[b] = exp
+    # attention stage-wise: oracle's window rows, queries, indices (the cache is shared input)
+    write_rows(run.win, spec.win_fmt, orc.new_win, d_n, run.win_slot)
+    for b, f in orc.new_entry.items():
+        r = orc.ent_start[b] + spec.seq_lens[b] // spec.m - 1
+        write_rows(run.ent, spec.kv_fmt, f[None], d_n, slice(r, r + 1))
+    write_rows(run.q, spec.q_fmt, orc.q_f.reshape(-1, spec.D), d_n, slice(0, B * spec.H))
+    if spec.is_csa:
+        idx_t = torch.full_like(run.idx, -1)
+        for b in range(B):
+            idx_t[b, :exp_idx[b].shape[0]] = torch.from_numpy(exp_idx[b].astype(np.int32)).to(dev)
+        run.idx.copy_(idx_t)
+    run.attn()
+    _sync()
+    assert run.read_status() == 0
+    got = out_np(run, range(B))
+    got_lse = np_(run.lse.view(B, spec.H))
+    worst = 0.0
+    for b in range(B):
+        o, lse = orc.attend(b, exp_idx.get(b))
+        ok_b, err, tol = attn_ok(got[b], o, spec.out_f32)
+        worst = max(worst, err / tol)
+        assert ok_b, f"attention (oracle inputs) sequence {b}: err {err} > tol {tol}"
+        np.testing.assert_allclose(got_lse[b], lse, rtol=0, atol=1e-4 if spec.out_f32 else 2e-3)
+        if not spec.is_csa or set(int(v) for v in e2e_idx[b] if v >= 0) == set(int(v) for v in exp_idx[b]):
+            ok_e, err_e, tol_e = attn_ok(e2e_out[b], o, spec.out_f32)
+            assert ok_e, f"attention (end to end) sequence {b}: err {err_e} > tol {tol_e}"
+    rep["attn_worst_err_over_tol"] = worst
+    return rep

@@ -1,0 +1,242 @@
+"""Test-side glue: run the oracle on a workload's inputs (host copies of the very tensors
+the library receives) and compare library outputs with it.
+
+Acceptance (stated per workload class):
+  * stored entries / window rows / queries: within one step of the storage format's grid
+    (the library rounds an FP32 value, the oracle a float64 one; they can land on the
+    two sides of a rounding midpoint), FP32 within 1e-5;
+  * index scores: within the FP32 evaluation error bound of the score;
+  * top-k on identical scores: bit-exact; end to end, FP32 inputs: identical wherever the
+    k-th / (k+1)-th score gap exceeds the error bound; FP4 inputs: the selected sets may
+    differ only in entries whose oracle score lies within 1e-2 |s_k| of the k-th score;
+  * attention: max-abs error <= 1e-4 (FP32 outputs) or <= 2e-2 x RMS(oracle output)
+    (BF16 outputs).
+"""
+from __future__ import annotations
+
+from typing import Dict, List, Sequence
+
+import numpy as np
+import torch
+
+from oracle import lc_oracle as O
+from oracle import pipeline as P
+from long_context_sparse_softmax_b200 import workloads as wl
+
+ATTN_TOL_F32 = 1e-4
+ATTN_TOL_REL_BF16 = 2e-2
+TOPK_FP4_BAND = 1e-2
+
+
+def np_(t):
+    return None if t is None else t.detach().cpu().numpy()
+
+
+def idx_operand_np(op: Dict[str, torch.Tensor], rows=None):
+    d = {k: np_(v if rows is None else v[rows]) for k, v in op.items()}
+    return d
+
+
+def stored_close(fmt: int, got_f64: np.ndarray, exp_f64: np.ndarray, d_n: int) -> np.ndarray:
+    """Per-element acceptance of stored rows: one grid step of the storage format."""
+    if fmt == O.FMT_F32:
+        tol = np.full(exp_f64.shape, 1e-5)
+    elif fmt == O.FMT_BF16:
+        tol = O.ulp_bf16(exp_f64) * 1.0001
+    else:
+        tol = np.concatenate([O.ulp_e4m3(exp_f64[..., :d_n]), O.ulp_bf16(exp_f64[..., d_n:])], -1) * 1.0001
+    return np.abs(got_f64 - exp_f64) <= tol
+
+
+def rows_np(fmt: int, r: Dict[str, torch.Tensor], sel=None) -> np.ndarray:
+    x = r["x"] if sel is None else r["x"][sel]
+    rope = r.get("rope")
+    if rope is not None and sel is not None:
+        rope = rope[sel]
+    return O.rows_to_f64(fmt, np_(x), np_(rope))
+
+
+def write_rows(r: Dict[str, torch.Tensor], fmt: int, y: np.ndarray, d_n: int, sel) -> None:
+    """Write float64 rows (cast to the storage format) into library buffer rows `sel`."""
+    x, rope = O.rows_from_f64(fmt, y, d_n)
+    dev = r["x"].device
+    r["x"][sel] = torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+    if rope is not None:
+        r["rope"][sel] = torch.from_numpy(np.ascontiguousarray(rope)).to(dev)
+
+
+def out_np(run, q_sel: Sequence[int]) -> np.ndarray:
+    s = run.spec
+    o = run.out.view(-1, s.H, s.D)[torch.as_tensor(list(q_sel), device=run.out.device)]
+    o = np_(o)
+    return o.astype(np.float64) if s.out_f32 else O.bf16_to_f64(o)
+
+
+def attn_ok(got: np.ndarray, exp: np.ndarray, out_f32: bool):
+    err = float(np.max(np.abs(got - exp))) if got.size else 0.0
+    tol = ATTN_TOL_F32 if out_f32 else ATTN_TOL_REL_BF16 * O.rms(exp)
+    return err <= tol, err, tol
+
+
+def topk_sets_ok(got_idx: np.ndarray, exp_idx: np.ndarray, s_oracle: np.ndarray, k: int, fp32: bool,
+                 bound: np.ndarray = None):
+    """End-to-end selection check for one query.  Returns (ok, n_diff, reason)."""
+    g = set(int(v) for v in got_idx if v >= 0)
+    e = set(int(v) for v in exp_idx if v >= 0)
+    if g == e:
+        return True, 0, ""
+    diff = g ^ e
+    K = len(e)
+    if len(g) != K:
+        return False, len(diff), "count differs"
+    order = np.lexsort((np.arange(s_oracle.shape[0]), -s_oracle))
+    s_k = s_oracle[order[K - 1]]
+    if fp32:
+        # only allowed where the oracle's k-th/(k+1)-th gap is within the FP32 error bound
+        if K < s_oracle.shape[0]:
+            s_k1 = s_oracle[order[K]]
+            b = bound[order[K - 1]] + bound[order[K]]
+            if s_k - s_k1 <= b and all(abs(s_oracle[j] - s_k) <= 2 * b for j in diff):
+                return True, len(diff), "within error bound"
+        return False, len(diff), "fp32 selection differs"
+    band = TOPK_FP4_BAND * abs(s_k)
+    bad = [j for j in diff if abs(s_oracle[j] - s_k) > band]
+    return (not bad), len(diff), ("" if not bad else f"{len(bad)} entries outside band")
+
+
+class OraclePrefill:
+    """Oracle of a prefill workload, for a sample of its queries (local indices)."""
+
+    def __init__(self, inp, q_sel: Sequence[int], W_x: int = None, entries=True):
+        s: wl.Spec = inp["spec"]
+        self.s = s
+        self.sink = np_(inp["sink"]).astype(np.float64)
+        self.W_x = s.W if W_x is None else W_x
+        self.q_sel = list(q_sel)
+        self.pos = [s.q_first + i for i in self.q_sel]
+        lo, d_r, d_n = s.rope_off, s.d_r, s.d_n
+        x_bits = np_(inp["x"])
+        self.x_bits = x_bits
+        g = np_(inp["g"]).astype(np.float64)
+        if entries:
+            xfun = lambda r0, n: P.raw_rows(s.raw_fmt, x_bits[r0:r0 + n])
+            self.ent_f, self.ent_x, self.ent_r = P.entries_from_tokens(xfun, g, s.m, lo, d_r, s.kv_fmt, d_n)
+            if self.ent_f.size == 0:
+                self.ent_f = np.zeros((0, s.D))
+        # window rows needed by the sampled queries
+        need = sorted(set(t for p in self.pos for t in O.window_positions(p, s.W)))
+        self.win_pos = np.array(need, dtype=np.int64)
+        if need:
+            raw = P.raw_rows(s.raw_fmt, x_bits[self.win_pos])
+            self.win_f, _, _ = P.stored(s.win_fmt, O.qk_prep(raw, self.win_pos, lo, d_r), d_n)
+        else:
+            self.win_f = np.zeros((0, s.D))
+        self.win_row = {int(t): i for i, t in enumerate(need)}
+        # queries
+        qr = P.raw_rows(s.raw_fmt, np_(inp["q_raw"][torch.as_tensor(self.q_sel, device=inp["q_raw"].device)]))
+        self.q_f, _, _ = P.stored(s.q_fmt, O.qk_prep(qr, np.array(self.pos), lo, d_r), d_n)
+        if s.is_csa:
+            sel_t = torch.as_tensor(self.q_sel, device=inp["q_raw"].device)
+            self.qI = P.indexer_f64(s.idx_fmt, idx_operand_np(inp["qI"], sel_t))
+            self.kI = P.indexer_f64(s.idx_fmt, idx_operand_np(inp["kI"]))
+            self.w = np_(inp["w"]).astype(np.float64)
+
+    def scores(self, i: int):
+        """Visible scores of sampled query i, and their FP32 error bound."""
+        p = self.pos[i]
+        s, n_vis = P.visible_scores(self.qI[i], self.kI, self.w, p, self.s.m, self.W_x)
+        return s, O.score_error_bound(self.qI[i], self.kI[:n_vis], self.w)
+
+    def select(self, i: int, s_vis: np.ndarray = None):
+        if s_vis is None:
+            s_vis, _ = self.scores(i)
+        return O.topk(s_vis, self.s.k)
+
+    def window_rows_for(self, p: int):
+        """(positions, float64 rows) of the window of a query at p."""
+        ts = list(O.window_positions(p, self.s.W))
+        return ts, self.win_f[[self.win_row[t] for t in ts]] if ts else np.zeros((0, self.s.D))
+
+    def attend(self, i: int, idx: Sequence[int]):
+        s = self.s
+        p = self.pos[i]
+        ts, wr = self.window_rows_for(p)
+        n_vis = O.n_visible(p, s.m, self.W_x, self.ent_f.shape[0])
+        if s.is_csa:
+            sel = [int(j) for j in idx if j >= 0]
+        else:
+            sel = list(range(n_vis))
+        keys = np.concatenate([self.ent_f[sel].reshape(len(sel), s.D), wr], 0)
+        return O.attend(self.q_f[i], keys, self.sink, s.scale)
+
+
+class OracleDecode:
+    """Oracle of a decode step: one query per sequence on the given cache."""
+
+    def __init__(self, inp, W_x: int = None):
+        s: wl.Spec = inp["spec"]
+        self.s = s
+        self.W_x = s.W if W_x is None else W_x
+        self.sink = np_(inp["sink"]).astype(np.float64)
+        lo, d_r, d_n = s.rope_off, s.d_r, s.d_n
+        B = s.num_seqs
+        self.n_c = list(inp["n_c"])
+        self.ent_start = [int(v) for v in np_(inp["batch"]["ent_start"])]
+        cache = inp["cache"]
+        self.ent_f = O.rows_to_f64(s.kv_fmt, np_(cache["x"]), np_(cache.get("rope")))
+        # decode-time compression of the block the newest token closed
+        xt = np_(inp["x_tail"])
+        gt = np_(inp["g_tail"]).astype(np.float64)
+        self.blk_count = [int(v) for v in np_(inp["blk_count"])]
+        self.new_entry = {}
+        for b, L in enumerate(s.seq_lens):
+            if self.blk_count[b]:
+                j = L // s.m - 1
+                y = O.compress(P.raw_rows(s.raw_fmt, xt[b]), gt[b], s.m, lo, d_r, first_block=j,
+                               tok_pos0=L - s.m, n_blocks=1)
+                f, _, _ = P.stored(s.kv_fmt, y, d_n)
+                self.new_entry[b] = f[0]
+                self.ent_f[self.ent_start[b] + j] = f[0]
+        # window rows: the cached rows, with the newest token prepared from x_new
+        self.win_f = O.rows_to_f64(s.win_fmt, np_(inp["win"])).reshape(B, s.W, s.D)
+        xn = P.raw_rows(s.raw_fmt, np_(inp["x_new"]))
+        self.pos = [L - 1 for L in s.seq_lens]
+        newrow, _, _ = P.stored(s.win_fmt, O.qk_prep(xn, np.array(self.pos), lo, d_r), d_n)
+        self.win_pos0 = [max(0, L - s.W) for L in s.seq_lens]
+        self.win_len = [min(s.W, L) for L in s.seq_lens]
+        for b in range(B):
+            self.win_f[b, self.win_len[b] - 1] = newrow[b]
+        self.new_win = newrow
+        qr = P.raw_rows(s.raw_fmt, np_(inp["q_raw"]))
+        self.q_f, _, _ = P.stored(s.q_fmt, O.qk_prep(qr, np.array(self.pos), lo, d_r), d_n)
+        if s.is_csa:
+            self.qI = P.indexer_f64(s.idx_fmt, idx_operand_np(inp["qI"]))
+            kI_np = idx_operand_np(inp["kI"])
+            self.kI_np = kI_np
+            self.w = np_(inp["w"]).astype(np.float64)
+
+    def kI(self, b: int):
+        n0, n = self.ent_start[b], self.n_c[b]
+        s = self.s
+        if s.idx_fmt == O.IDX_F32:
+            return self.kI_np["f32"][n0:n0 + n].astype(np.float64)
+        return O.mxfp4_to_f64(self.kI_np["codes"][n0:n0 + n], self.kI_np["scales"][n0:n0 + n])
+
+    def scores(self, b: int):
+        kI = self.kI(b)
+        s, n_vis = P.visible_scores(self.qI[b], kI, self.w, self.pos[b], self.s.m, self.W_x)
+        return s, O.score_error_bound(self.qI[b], kI[:n_vis], self.w)
+
+    def entries(self, b: int):
+        return self.ent_f[self.ent_start[b]:self.ent_start[b] + self.n_c[b]]
+
+    def attend(self, b: int, idx: Sequence[int]):
+        s = self.s
+        p = self.pos[b]
+        ent = self.entries(b)
+        n_vis = O.n_visible(p, s.m, self.W_x, self.n_c[b])
+        sel = [int(j) for j in idx if j >= 0] if s.is_csa else list(range(n_vis))
+        ts = list(O.window_positions(p, s.W))
+        wr = self.win_f[b][[t - self.win_pos0[b] for t in ts]]
+        keys = np.concatenate([ent[sel].reshape(len(sel), s.D), wr.reshape(len(ts), s.D)], 0)
+        return O.attend(self.q_f[b], keys, self.sink, s.scale)

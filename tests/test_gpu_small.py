@@ -1,0 +1,75 @@
+"""GPU parity at oracle-sized shapes: every query of each case is checked, the shapes
+span several kernel tiles with ragged tails, and the edge cases of the method are
+covered (no visible entry, fewer visible entries than k, window off, overlap reading,
+sequences shorter than the window, m = 1)."""
+import pytest
+
+from long_context_sparse_softmax_b200 import workloads as wl
+from tests.gpu_checks import check_decode, check_prefill
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_fp32_csa_prefill_all_queries():
+    """The FP32 workload (L = 1024, D = 128, 8 heads, k = 64): top-k bit-exact,
+    attention within 1e-4."""
+    rep = check_prefill(wl.TINY_CSA_PREFILL)
+    assert rep["topk_e2e_set_diff"] == 0
+
+
+SMALL_CSA = wl.shrink(wl.CSA_PREFILL, name="small_csa_prefill", seed=31, seq_lens=(1100,), H=16, k=64,
+                      n_q=1100, q_first=0)
+
+
+def test_small_csa_prefill_fp8_mxfp4():
+    check_prefill(SMALL_CSA)
+
+
+def test_small_csa_prefill_128_heads_ragged():
+    s = wl.shrink(wl.CSA_PREFILL, name="small_csa_h128", seed=32, seq_lens=(613,), H=128, k=32, n_q=613)
+    check_prefill(s)
+
+
+def test_small_csa_prefill_overlap_reading():
+    check_prefill(SMALL_CSA, q_sel=range(0, 1100, 7), W_x=0)
+
+
+def test_small_csa_prefill_without_window():
+    s = wl.shrink(SMALL_CSA, name="small_csa_w0", seed=33, W=0, seq_lens=(300,), n_q=300)
+    check_prefill(s)
+
+
+def test_m1_fp32_csa_prefill():
+    s = wl.shrink(wl.TINY_CSA_PREFILL, name="tiny_m1", seed=34, m=1, seq_lens=(300,), n_q=300, k=300)
+    check_prefill(s)
+
+
+def test_small_hca_prefill():
+    s = wl.shrink(wl.HCA_PREFILL, name="small_hca_prefill", seed=35, seq_lens=(128 * 30 + 77,),
+                  q_first=128 * 30 + 77 - 300, n_q=300)
+    check_prefill(s)
+
+
+def test_small_hca_prefill_from_position_zero():
+    s = wl.shrink(wl.HCA_PREFILL, name="small_hca_from0", seed=36, seq_lens=(700,), q_first=0, n_q=700)
+    check_prefill(s)
+
+
+def test_small_csa_decode_ragged():
+    s = wl.shrink(wl.CSA_DECODE, name="small_csa_decode", seed=37, seq_lens=(1000, 2053, 517, 50, 132), k=128)
+    check_decode(s)
+
+
+def test_small_csa_decode_k1024():
+    s = wl.shrink(wl.MIXED_CSA, name="small_mixed_csa", seed=38, seq_lens=(5000, 4096, 1300))
+    check_decode(s)
+
+
+def test_small_hca_decode_ragged():
+    s = wl.shrink(wl.MIXED_HCA, name="small_hca_decode", seed=39, seq_lens=(128 * 20 + 5, 128 * 3, 1000, 64))
+    check_decode(s)
+
+
+def test_small_csa_decode_overlap_reading():
+    s = wl.shrink(wl.CSA_DECODE, name="small_csa_decode_ov", seed=40, seq_lens=(900, 1204), k=64)
+    check_decode(s, W_x=0)
