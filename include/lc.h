@@ -68,7 +68,9 @@ enum {
   LC_DEV_BAD_INDEX = 1,    /* a top-k index outside [0, n_ent(b)) other than -1: skipped */
   LC_DEV_WINDOW_RANGE = 2, /* a window position outside the given window rows: skipped */
   LC_DEV_BAD_BLOCK = 4,    /* a block whose tokens are not in the given token rows: skipped */
-  LC_DEV_NONVISIBLE = 8    /* a selected entry not visible to its query: skipped */
+  LC_DEV_NONVISIBLE = 8,   /* a selected entry not visible to its query: skipped */
+  LC_DEV_TIMEOUT = 16      /* a bounded wait on the tensor core gave up: results of that
+                              CTA are missing (never expected; reported, not hung) */
 };
 
 /* Row storage formats. */
@@ -96,7 +98,7 @@ typedef struct lc_rows {
 
 typedef struct lc_dims {
   int32_t D;               /* dims per row (multiple of 8, <= 1024) */
-  int32_t d_r;             /* RoPE dims (multiple of 8, <= D) */
+  int32_t d_r;             /* RoPE dims (multiple of 8, <= min(D, 128)) */
   int32_t rope_off;        /* first RoPE dim inside a row (multiple of 8) */
   int32_t H;               /* heads per query token (rows per token) */
 } lc_dims;
@@ -187,9 +189,9 @@ typedef struct lc_index_args {
   int32_t d_I;             /* indexer dims (F32: multiple of 4, <= 256; MXFP4: 128) */
   int32_t fmt;             /* LC_IDX_F32 or LC_IDX_MXFP4 */
   const void* q;           /* F32 [n_q, H_I, d_I] or MXFP4 codes [n_q, H_I, d_I/2] */
-  const uint8_t* q_scale;  /* MXFP4: [n_q, H_I, d_I/32] */
+  const uint8_t* q_scale;  /* MXFP4: [n_q, H_I, d_I/32], 4-byte aligned */
   const void* k;           /* F32 [n_keys, d_I] or MXFP4 codes [n_keys, d_I/2] */
-  const uint8_t* k_scale;  /* MXFP4: [n_keys, d_I/32] */
+  const uint8_t* k_scale;  /* MXFP4: [n_keys, d_I/32], 4-byte aligned */
   const float* w;          /* head weights, >= 0: [H_I], or [n_q, H_I] if w_qstride = H_I */
   int32_t w_qstride;       /* 0 (shared) or H_I */
   int32_t m;
@@ -237,8 +239,8 @@ lc_status lc_csa_topk_decode(const lc_topk_args* a, void* stream);
  * Pages: "解读 DeepSeek V4" CSA / HCA sections and "其他架构细节" (attention sink);
  * "DeepSeek-V4 论文分析" §5.4, §六, §七 and §8.4 (sparse core attention).
  * out: [n_q, H, D] in out_fmt (F32 or BF16); lse: [n_q, H] FP32 (optional).
- * The decode variant splits the keys of each query across CTAs and needs a workspace
- * of *_workspace_bytes(a) bytes (0 for prefill).
+ * The decode variant may split the keys of each query across CTAs; it then needs a
+ * workspace of lc_*_workspace_bytes(a) bytes (the prefill variant needs none).
  * ------------------------------------------------------------------------------- */
 typedef struct lc_attn_args {
   lc_dims dims;

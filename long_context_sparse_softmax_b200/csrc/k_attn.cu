@@ -56,11 +56,11 @@ __device__ __forceinline__ void attend_row(OnlineSoftmax& st, const Vec8 (&q)[kA
   }
 }
 
-// grid: (ceil(H / 8), n_q); 8 warps, one head each.
+// grid: (n_q, ceil(H / 8)); 8 warps, one head each.
 __global__ void __launch_bounds__(256) k_attn_ref(lc_attn_args a, int sparse) {
   const int lane = threadIdx.x & 31;
-  const int h = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int q = blockIdx.y;
+  const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
+  const int q = blockIdx.x;
   const int H = a.dims.H, D = a.dims.D, d_r = a.dims.d_r;
   if (h >= H) return;
   const int b = seq_of_query(a.batch.q_start, a.batch.num_seqs, q);
@@ -132,11 +132,16 @@ __global__ void __launch_bounds__(256) k_attn_ref(lc_attn_args a, int sparse) {
   if (a.lse && lane == 0) a.lse[qrow] = st.m + logf(st.z);
 }
 
-size_t attn_workspace_bytes(const lc_attn_args& /*a*/, bool /*sparse*/, bool /*decode*/) { return 0; }
+size_t attn_workspace_bytes(const lc_attn_args& a, bool sparse, bool decode) {
+  return attn_mma_supported(a) ? attn_mma_workspace(a, sparse, decode) : 0;
+}
 
-cudaError_t launch_attn(const lc_attn_args& a, bool sparse, bool /*decode*/, cudaStream_t st) {
+// 576-dim BF16/E4M3 shapes go to the tensor-core kernel (k_attn_mma.cu); FP32 and other
+// head dims use the reference kernel.
+cudaError_t launch_attn(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st) {
   if (a.n_q == 0) return cudaSuccess;
-  const dim3 grid((a.dims.H + 7) / 8, a.n_q);
+  if (attn_mma_supported(a)) return launch_attn_mma(a, sparse, decode, st);
+  const dim3 grid(a.n_q, (a.dims.H + 7) / 8);
   k_attn_ref<<<grid, 256, 0, st>>>(a, sparse ? 1 : 0);
   return cudaGetLastError();
 }

@@ -1,0 +1,446 @@
+// Tensor-core CSA sparse / HCA dense attention for 576-dim shared-KV entries (BF16 MMA).
+//
+// Same mathematics as the reference kernel in k_attn.cu ("解读 DeepSeek V4": CSA attends to
+// its top-k compressed entries, HCA to all of them, both plus a 128-token window and a
+// per-head sink; V = K = the entry).  The rows of a CTA are heads of ONE query, which all
+// share the same keys (MQA), so a key tile is gathered once and feeds every head:
+//
+//   * key tile: 64 keys gathered by index (entries: E4M3 nope + BF16 RoPE; window rows:
+//     BF16), widened to BF16 in shared memory (E4M3 -> BF16 is exact);
+//   * S = Q K^T on BF16 mma.sync; the D = 576 contraction is split across DS warps and
+//     their partial sums are added in a fixed order through shared memory, so every warp
+//     of a row tile holds the same S;
+//   * online softmax in registers (running max starts at -inf, the sink joins at the end);
+//   * O += P V with P from registers and V = the same key tile, each warp owning D/DS
+//     output dims.
+//
+// A CTA covers MT x 16 heads with MT * DS warps: prefill uses 64 heads (MT = 4, DS = 2),
+// decode 16 heads (MT = 1, DS = 4) so that a small batch still fills the GPU.  Decode
+// may split a query's keys across CTAs (n_split > 1): each writes its unnormalised O,
+// running max and sum to the workspace and k_attn_combine merges them with the sink in
+// a fixed order.  The split count depends only on the shapes, never on timing.
+#include "lc_internal.h"
+
+namespace lc {
+
+constexpr int kAD = 576;          // head dim of this kernel
+constexpr int kRS = kAD + 8;      // padded shared row stride (elements): 1168 B, ldmatrix conflict-free
+constexpr int kTK = 64;           // keys per tile
+constexpr uint32_t kWinFlag = 1u << 30;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  return static_cast<uint32_t>(f32_to_bf16_bits(lo)) | (static_cast<uint32_t>(f32_to_bf16_bits(hi)) << 16);
+}
+
+// 8 E4M3 values (8 bytes) -> 8 BF16 values (16 bytes), exact.
+__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 u) {
+  const uint32_t w[2] = {u.x, u.y};
+  uint32_t o[4];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const float2 a = e4m3x2_to_f32x2(static_cast<uint16_t>(w[j] & 0xffffu));
+    const float2 b = e4m3x2_to_f32x2(static_cast<uint16_t>(w[j] >> 16));
+    // E4M3 values have <= 4 significant bits: the upper half of the FP32 bits is exact BF16
+    o[2 * j] = (__float_as_uint(a.x) >> 16) | (__float_as_uint(a.y) & 0xffff0000u);
+    o[2 * j + 1] = (__float_as_uint(b.x) >> 16) | (__float_as_uint(b.y) & 0xffff0000u);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Row `r` of a row set (576 logical dims) widened to BF16 into shared memory; `nthr`
+// threads of index `sub` share the row, 8 dims (one 16-byte chunk) at a time.
+__device__ __forceinline__ void stage_row_bf16(const lc_rows& rs, int64_t r, int d_r, uint16_t* dst, int sub,
+                                               int nthr) {
+  const int d_n = kAD - d_r;
+  if (rs.fmt == LC_FMT_BF16) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(rs.x) + r * kAD);
+#pragma unroll 6
+    for (int c = sub; c < kAD / 8; c += nthr) reinterpret_cast<uint4*>(dst)[c] = __ldg(src + c);
+  } else {
+    const uint2* nope = reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(rs.x) + r * d_n);
+    const uint4* rope = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(rs.rope) + r * d_r);
+#pragma unroll 6
+    for (int c = sub; c < kAD / 8; c += nthr) {
+      uint4 v;
+      if (c * 8 < d_n) v = e4m3x8_to_bf16x8(__ldg(nope + c));
+      else v = __ldg(rope + (c - d_n / 8));
+      reinterpret_cast<uint4*>(dst)[c] = v;
+    }
+  }
+}
+
+__device__ __forceinline__ void zero_row(uint16_t* dst, int sub, int nthr) {
+  for (int c = sub; c < kAD / 8; c += nthr) reinterpret_cast<uint4*>(dst)[c] = make_uint4(0, 0, 0, 0);
+}
+
+struct AttnGeom {
+  int n_split;   // CTAs per (query, head group) along the keys
+  int sps;       // slots per split (multiple of kTK)
+};
+
+// grid: (n_q, n_hg * n_split); MT * DS warps.
+template <int MT, int DS>
+__global__ void __launch_bounds__(MT * DS * 32, 1)
+    k_attn_mma(lc_attn_args a, int sparse, AttnGeom geo, float* __restrict__ ws_o, float* __restrict__ ws_ml) {
+  constexpr int NW = MT * DS;
+  constexpr int NTHR = NW * 32;
+  constexpr int ROWS = MT * 16;
+  constexpr int DW = kAD / DS;        // output dims per warp
+  constexpr int KS = DW / 16;         // k16 steps of the partial S
+  constexpr int NTO = DW / 8;         // n8 tiles of O per warp
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint16_t* Qs = reinterpret_cast<uint16_t*>(smem);                 // [ROWS][kRS]
+  uint16_t* Ks = Qs + ROWS * kRS;                                    // [kTK][kRS]
+  float* Sx = reinterpret_cast<float*>(Ks + kTK * kRS);              // [NW][32][32]
+  int* kval = reinterpret_cast<int*>(Sx + NW * 32 * 32);             // [kTK] key valid
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int mt = warp / DS, ds = warp % DS;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int q = blockIdx.x;
+  const int n_hg = gridDim.y / geo.n_split;
+  const int hg = blockIdx.y / geo.n_split, split = blockIdx.y % geo.n_split;
+  const int H = a.dims.H, d_r = a.dims.d_r;
+  const int b = seq_of_query(a.batch.q_start, a.batch.num_seqs, q);
+  const int p = __ldg(a.batch.q_pos0 + b) + (q - __ldg(a.batch.q_start + b));
+  const int n_ent = __ldg(a.batch.n_ent + b);
+  const int nv = n_visible(p, a.m, a.W_x, n_ent);
+  const int64_t ent0 = __ldg(a.batch.ent_start + b);
+  const int wlo = a.W > 0 ? max(0, p - a.W + 1) : p + 1;
+  const int n_win = p + 1 - wlo;
+  const int n_first = sparse ? a.k : nv;           // slots before the window
+  const int n_slots = n_first + n_win;
+  const int s_begin = split * geo.sps;
+  const int s_end = min(n_slots, s_begin + geo.sps);
+  const int wp0 = a.W > 0 ? __ldg(a.batch.win_pos0 + b) : 0;
+  const int wl = a.W > 0 ? __ldg(a.batch.win_len + b) : 0;
+  const int64_t wr0 = a.W > 0 ? __ldg(a.batch.win_start + b) : 0;
+  const int32_t* idx_row = sparse ? a.idx + static_cast<int64_t>(q) * a.k : nullptr;
+  (void)n_hg;
+
+  // queries of this head group, widened to BF16
+  {
+    constexpr int TPR = NTHR / ROWS;  // threads per row
+    const int r = tid / TPR, sub = tid % TPR;
+    const int h = hg * ROWS + r;
+    if (h < H) stage_row_bf16(a.q, static_cast<int64_t>(q) * H + h, d_r, Qs + r * kRS, sub, TPR);
+    else zero_row(Qs + r * kRS, sub, TPR);
+  }
+
+  float o[NTO][4];
+#pragma unroll
+  for (int i = 0; i < NTO; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m_run[2] = {-INFINITY, -INFINITY};
+  float l_run[2] = {0.f, 0.f};
+  const float sl2 = a.scale * 1.4426950408889634f;  // logits in log2 units
+
+  for (int s0 = s_begin; s0 < s_end; s0 += kTK) {
+    __syncthreads();  // previous tile fully consumed
+    {
+      constexpr int TPK = NTHR / kTK;
+      const int kr = tid / TPK, sub = tid % TPK;
+      const int s = s0 + kr;
+      int code = -1;
+      if (s < s_end) {
+        if (s < n_first) {
+          const int j = sparse ? __ldg(idx_row + s) : s;
+          if (j >= 0) {
+            if (j >= n_ent) {
+              if (sub == 0) set_status(a.status, LC_DEV_BAD_INDEX);
+            } else if (j >= nv) {
+              if (sub == 0) set_status(a.status, LC_DEV_NONVISIBLE);
+            } else {
+              code = j;
+            }
+          }
+        } else {
+          const int rr = wlo + (s - n_first) - wp0;
+          if (rr < 0 || rr >= wl) {
+            if (sub == 0) set_status(a.status, LC_DEV_WINDOW_RANGE);
+          } else {
+            code = static_cast<int>(kWinFlag) | rr;
+          }
+        }
+      }
+      uint16_t* dst = Ks + kr * kRS;
+      if (code < 0) zero_row(dst, sub, TPK);
+      else if (code & kWinFlag) stage_row_bf16(a.win, wr0 + (code & ~kWinFlag), d_r, dst, sub, TPK);
+      else stage_row_bf16(a.ent, ent0 + code, d_r, dst, sub, TPK);
+      if (sub == 0) kval[kr] = code >= 0;
+    }
+    __syncthreads();
+
+    // partial S over this warp's dims: 16 rows x 64 keys
+    float sacc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.f;
+    const uint32_t qa = smem_u32(Qs + (mt * 16 + (lane & 15)) * kRS + ds * DW + (lane >> 4) * 8);
+    const uint32_t kb = smem_u32(Ks + ((lane >> 4) * 8 + (lane & 7)) * kRS + ds * DW + ((lane >> 3) & 1) * 8);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(qa + ks * 32, a0, a1, a2, a3);
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kb + np * 16 * kRS * 2 + ks * 32, b0, b1, b2, b3);
+        mma_bf16(sacc[2 * np], a0, a1, a2, a3, b0, b1);
+        mma_bf16(sacc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+    // add the DS partial sums in a fixed order (every warp of the row tile gets the same S)
+    float* mine = Sx + warp * 1024;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) mine[(i * 4 + j) * 32 + lane] = sacc[i][j];
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float v = Sx[(mt * DS + 0) * 1024 + (i * 4 + j) * 32 + lane];
+#pragma unroll
+        for (int d = 1; d < DS; ++d) v += Sx[(mt * DS + d) * 1024 + (i * 4 + j) * 32 + lane];
+        sacc[i][j] = v;
+      }
+    // online softmax (log2 units); masked keys get -inf
+    float tmax[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool v0 = kval[i * 8 + 2 * t4], v1 = kval[i * 8 + 2 * t4 + 1];
+      sacc[i][0] = v0 ? sacc[i][0] * sl2 : -INFINITY;
+      sacc[i][1] = v1 ? sacc[i][1] * sl2 : -INFINITY;
+      sacc[i][2] = v0 ? sacc[i][2] * sl2 : -INFINITY;
+      sacc[i][3] = v1 ? sacc[i][3] * sl2 : -INFINITY;
+      tmax[0] = fmaxf(tmax[0], fmaxf(sacc[i][0], sacc[i][1]));
+      tmax[1] = fmaxf(tmax[1], fmaxf(sacc[i][2], sacc[i][3]));
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 1));
+      tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 2));
+    }
+    float corr[2], mref[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float mn = fmaxf(m_run[r], tmax[r]);
+      corr[r] = (m_run[r] == -INFINITY) ? 0.f : exp2f(m_run[r] - mn);
+      mref[r] = (mn == -INFINITY) ? 0.f : mn;
+      m_run[r] = mn;
+    }
+    float rs[2] = {0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      sacc[i][0] = exp2f(sacc[i][0] - mref[0]);
+      sacc[i][1] = exp2f(sacc[i][1] - mref[0]);
+      sacc[i][2] = exp2f(sacc[i][2] - mref[1]);
+      sacc[i][3] = exp2f(sacc[i][3] - mref[1]);
+      rs[0] += sacc[i][0] + sacc[i][1];
+      rs[1] += sacc[i][2] + sacc[i][3];
+    }
+    l_run[0] = l_run[0] * corr[0] + rs[0];
+    l_run[1] = l_run[1] * corr[1] + rs[1];
+#pragma unroll
+    for (int i = 0; i < NTO; ++i) {
+      o[i][0] *= corr[0];
+      o[i][1] *= corr[0];
+      o[i][2] *= corr[1];
+      o[i][3] *= corr[1];
+    }
+    // O += P V over the 64 keys (4 k16 steps), this warp's dims
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint32_t pa0 = pack_bf16(sacc[2 * kk][0], sacc[2 * kk][1]);
+      const uint32_t pa1 = pack_bf16(sacc[2 * kk][2], sacc[2 * kk][3]);
+      const uint32_t pa2 = pack_bf16(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1]);
+      const uint32_t pa3 = pack_bf16(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3]);
+      const uint32_t vb = smem_u32(Ks + (kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7)) * kRS + ds * DW + (lane >> 4) * 8);
+#pragma unroll
+      for (int np = 0; np < NTO / 2; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vb + np * 32, b0, b1, b2, b3);
+        mma_bf16(o[2 * np], pa0, pa1, pa2, pa3, b0, b1);
+        mma_bf16(o[2 * np + 1], pa0, pa1, pa2, pa3, b2, b3);
+      }
+    }
+  }
+
+  // row sums over the 4 threads of a row
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
+    l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
+  }
+  const int hr0 = hg * ROWS + mt * 16 + g;  // head of row g (row g + 8 is hr0 + 8)
+  if (geo.n_split == 1) {
+    // join the sink and normalise: M = max(sink, m), Z = e^(sink-M) + l e^(m-M)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int h = hr0 + 8 * r;
+      if (h >= H) continue;
+      const float sk = __ldg(a.sink + h) * 1.4426950408889634f;
+      const float M = fmaxf(sk, m_run[r]);
+      const float wl_ = (m_run[r] == -INFINITY) ? 0.f : exp2f(m_run[r] - M);
+      const float Z = exp2f(sk - M) + l_run[r] * wl_;
+      const float f = wl_ / Z;
+      const int64_t orow = static_cast<int64_t>(q) * H + h;
+      if (a.out_fmt == LC_FMT_BF16) {
+        uint32_t* op = reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(a.out) + orow * kAD + ds * DW + 2 * t4);
+#pragma unroll
+        for (int i = 0; i < NTO; ++i) op[i * 4] = pack_bf16(o[i][2 * r] * f, o[i][2 * r + 1] * f);
+      } else {
+        float2* op = reinterpret_cast<float2*>(static_cast<float*>(a.out) + orow * kAD + ds * DW + 2 * t4);
+#pragma unroll
+        for (int i = 0; i < NTO; ++i) op[i * 4] = make_float2(o[i][2 * r] * f, o[i][2 * r + 1] * f);
+      }
+      if (a.lse && ds == 0 && t4 == 0) a.lse[orow] = (M + log2f(Z)) * 0.6931471805599453f;
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int h = hr0 + 8 * r;
+      if (h >= H) continue;
+      const int64_t slot = (static_cast<int64_t>(q) * H + h) * geo.n_split + split;
+      float2* op = reinterpret_cast<float2*>(ws_o + slot * kAD + ds * DW + 2 * t4);
+#pragma unroll
+      for (int i = 0; i < NTO; ++i) op[i * 4] = make_float2(o[i][2 * r], o[i][2 * r + 1]);
+      if (ds == 0 && t4 == 0) {
+        ws_ml[2 * slot] = m_run[r];
+        ws_ml[2 * slot + 1] = l_run[r];
+      }
+    }
+  }
+}
+
+// Merge the key splits of each (query, head) with the sink, in split order.
+// grid: ceil(n_q * H / 8); one warp per (query, head).
+__global__ void __launch_bounds__(256) k_attn_combine(lc_attn_args a, int n_split, const float* __restrict__ ws_o,
+                                                      const float* __restrict__ ws_ml) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= static_cast<int64_t>(a.n_q) * a.dims.H) return;
+  const int h = static_cast<int>(row % a.dims.H);
+  const float sk = __ldg(a.sink + h) * 1.4426950408889634f;
+  float M = sk;
+  for (int c = 0; c < n_split; ++c) M = fmaxf(M, __ldg(ws_ml + 2 * (row * n_split + c)));
+  float Z = exp2f(sk - M);
+  float o[kAD / 32];
+#pragma unroll
+  for (int i = 0; i < kAD / 32; ++i) o[i] = 0.f;
+  for (int c = 0; c < n_split; ++c) {
+    const float mc = __ldg(ws_ml + 2 * (row * n_split + c));
+    if (mc == -INFINITY) continue;
+    const float w = exp2f(mc - M);
+    Z = fmaf(__ldg(ws_ml + 2 * (row * n_split + c) + 1), w, Z);
+    const float* src = ws_o + (row * n_split + c) * kAD;
+#pragma unroll
+    for (int i = 0; i < kAD / 32; ++i) o[i] = fmaf(__ldg(src + i * 32 + lane), w, o[i]);
+  }
+  const float inv = 1.f / Z;
+  if (a.out_fmt == LC_FMT_BF16) {
+    uint16_t* dst = static_cast<uint16_t*>(a.out) + row * kAD;
+#pragma unroll
+    for (int i = 0; i < kAD / 32; ++i) dst[i * 32 + lane] = f32_to_bf16_bits(o[i] * inv);
+  } else {
+    float* dst = static_cast<float*>(a.out) + row * kAD;
+#pragma unroll
+    for (int i = 0; i < kAD / 32; ++i) dst[i * 32 + lane] = o[i] * inv;
+  }
+  if (a.lse && lane == 0) a.lse[row] = (M + log2f(Z)) * 0.6931471805599453f;
+}
+
+// ---------------------------------------------------------------------------------
+// launch configuration
+// ---------------------------------------------------------------------------------
+bool attn_mma_supported(const lc_attn_args& a) {
+  if (a.dims.D != kAD || a.dims.d_r % 8 || a.dims.H % 16) return false;
+  auto ok_rows = [&](const lc_rows& r) {
+    return r.fmt == LC_FMT_BF16 || (r.fmt == LC_FMT_E4M3_BF16 && a.dims.d_r > 0);
+  };
+  if (!ok_rows(a.q) || !ok_rows(a.ent) || (a.W > 0 && a.win.fmt != LC_FMT_BF16)) return false;
+  return a.out_fmt == LC_FMT_BF16 || a.out_fmt == LC_FMT_F32;
+}
+
+static int max_slots(const lc_attn_args& a, bool sparse) {
+  return (sparse ? a.k : a.max_ent) + a.W;
+}
+
+AttnGeom attn_geometry(const lc_attn_args& a, bool sparse, bool decode) {
+  AttnGeom g{1, 0};
+  const int ns = max(max_slots(a, sparse), 1);
+  const int tiles = (ns + kTK - 1) / kTK;
+  if (decode) {
+    // fill ~2 CTAs per SM, but keep >= 4 key tiles (256 keys) per split so that the
+    // partial results a split writes stay small next to the keys it reads
+    const int ctas = a.n_q * (a.dims.H / 16);
+    const int want = (2 * 148 + ctas - 1) / max(ctas, 1);
+    int n = min(want, max(1, tiles / 4));
+    n = max(1, min(n, tiles));
+    const int per = (tiles + n - 1) / n;
+    g.n_split = (tiles + per - 1) / per;
+    g.sps = per * kTK;
+  } else {
+    g.sps = tiles * kTK;
+  }
+  return g;
+}
+
+size_t attn_mma_workspace(const lc_attn_args& a, bool sparse, bool decode) {
+  const AttnGeom g = attn_geometry(a, sparse, decode);
+  if (g.n_split <= 1) return 0;
+  const size_t rows = static_cast<size_t>(a.n_q) * a.dims.H * g.n_split;
+  return rows * kAD * sizeof(float) + rows * 2 * sizeof(float);
+}
+
+template <int MT, int DS>
+static cudaError_t launch_mma(const lc_attn_args& a, bool sparse, const AttnGeom& g, cudaStream_t st) {
+  constexpr int ROWS = MT * 16;
+  const size_t sm = (ROWS + kTK) * kRS * 2 + MT * DS * 32 * 32 * 4 + kTK * 4;
+  cudaFuncSetAttribute(k_attn_mma<MT, DS>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
+  const int n_hg = (a.dims.H + ROWS - 1) / ROWS;
+  float* ws_o = static_cast<float*>(a.workspace);
+  float* ws_ml = nullptr;
+  if (g.n_split > 1) {
+    const size_t rows = static_cast<size_t>(a.n_q) * a.dims.H * g.n_split;
+    ws_ml = ws_o + rows * kAD;
+  }
+  const dim3 grid(a.n_q, n_hg * g.n_split);
+  k_attn_mma<MT, DS><<<grid, MT * DS * 32, sm, st>>>(a, sparse ? 1 : 0, g, ws_o, ws_ml);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || g.n_split == 1) return e;
+  const int64_t rows = static_cast<int64_t>(a.n_q) * a.dims.H;
+  k_attn_combine<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(a, g.n_split, ws_o, ws_ml);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_mma(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st) {
+  const AttnGeom g = attn_geometry(a, sparse, decode);
+  if (decode || a.dims.H % 64) return launch_mma<1, 4>(a, sparse, g, st);
+  return launch_mma<4, 2>(a, sparse, g, st);
+}
+
+}  // namespace lc

@@ -56,7 +56,7 @@ __device__ __forceinline__ void mma_e4m3_16x8x32(float (&d)[4], const uint32_t (
 constexpr int kIdxKeys = 128;       // keys per CTA tile (4 warps x 2 m16 tiles)
 constexpr int kIdxMaxHeads = 64;    // heads per pass (8 n8 tiles)
 
-// grid: (key tiles, query chunks); 128 threads.  KB = d_I / 32 MX blocks.
+// grid: (query chunks, key tiles); 128 threads.  KB = d_I / 32 MX blocks.
 template <int KB>
 __global__ void __launch_bounds__(128) k_index_mxfp4(lc_index_args a, int q_chunk) {
   constexpr int DI = KB * 32;
@@ -72,8 +72,8 @@ __global__ void __launch_bounds__(128) k_index_mxfp4(lc_index_args a, int q_chun
   const int g = lane >> 2, t = lane & 3;
   const int H = a.H_I;
   const int NT = H >> 3;
-  const int j0 = blockIdx.x * kIdxKeys;
-  const int qa = blockIdx.y * q_chunk;
+  const int j0 = blockIdx.y * kIdxKeys;
+  const int qa = blockIdx.x * q_chunk;
   const int qb = min(qa + q_chunk, a.n_q);
   if (qa >= qb) return;
 
@@ -202,11 +202,11 @@ __global__ void __launch_bounds__(128) k_index_mxfp4(lc_index_args a, int q_chun
 // FP32 operands: one thread per (query, key); query heads staged in shared memory.
 __global__ void __launch_bounds__(128) k_index_f32(lc_index_args a) {
   extern __shared__ float qs[];  // [H_I][d_I] then w [H_I]
-  const int q = blockIdx.y;
+  const int q = blockIdx.x;
   const int b = seq_of_query(a.batch.q_start, a.batch.num_seqs, q);
   const int p = __ldg(a.batch.q_pos0 + b) + (q - __ldg(a.batch.q_start + b));
   const int nv = n_visible(p, a.m, a.W_x, __ldg(a.batch.n_ent + b));
-  const int j0 = blockIdx.x * blockDim.x;
+  const int j0 = blockIdx.y * blockDim.x;
   if (j0 >= nv) return;
   const int H = a.H_I, DI = a.d_I;
   const float* qg = static_cast<const float*>(a.q) + static_cast<int64_t>(q) * H * DI;
@@ -237,14 +237,15 @@ __global__ void __launch_bounds__(128) k_index_f32(lc_index_args a) {
 cudaError_t launch_index_scores(const lc_index_args& a, bool decode, cudaStream_t st) {
   if (a.n_q == 0 || a.max_ent == 0) return cudaSuccess;
   if (a.fmt == LC_IDX_F32) {
-    const dim3 grid((a.max_ent + 127) / 128, a.n_q);
+    const dim3 grid(a.n_q, (a.max_ent + 127) / 128);
     const size_t sm = static_cast<size_t>(a.H_I * a.d_I + a.H_I) * sizeof(float);
     cudaFuncSetAttribute(k_index_f32, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
     k_index_f32<<<grid, 128, sm, st>>>(a);
     return cudaGetLastError();
   }
+  if (index_tc_supported(a)) return launch_index_tc(a, decode, st);
   const int q_chunk = decode ? 1 : 32;
-  const dim3 grid((a.max_ent + kIdxKeys - 1) / kIdxKeys, (a.n_q + q_chunk - 1) / q_chunk);
+  const dim3 grid((a.n_q + q_chunk - 1) / q_chunk, (a.max_ent + kIdxKeys - 1) / kIdxKeys);
   const int KB = a.d_I / 32;
   const size_t rs = static_cast<size_t>(a.d_I + 16);
   const size_t sm = (kIdxKeys + kIdxMaxHeads) * rs + (kIdxKeys + kIdxMaxHeads) * KB * 4 + kIdxMaxHeads * 4;

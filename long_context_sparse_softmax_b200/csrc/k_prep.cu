@@ -10,6 +10,8 @@
 //
 // All of them stream HBM: 16-byte vector loads of 8 dims per lane, one warp per row
 // (qk_prep), per entry (CSA compress) or one CTA per entry (HCA compress, 128 tokens).
+#include <cmath>
+
 #include "lc_internal.h"
 
 namespace lc {
@@ -18,7 +20,7 @@ constexpr int kMaxGroupsPerLane = 4;  // D <= 1024: 128 groups of 8 dims over 32
 
 // RMSNorm + RoPE + store of one row held by a warp as groups of 8 dims.
 __device__ __forceinline__ void norm_rope_store(Vec8 (&v)[kMaxGroupsPerLane], int lane, int D, int d_r,
-                                                int rope_off, float eps, int pos, float base,
+                                                int rope_off, float eps, int pos, const RopeTable& rt,
                                                 const lc_rows& out, int64_t out_row) {
   const int G = D >> 3;
   float ss = 0.f;
@@ -43,7 +45,7 @@ __device__ __forceinline__ void norm_rope_store(Vec8 (&v)[kMaxGroupsPerLane], in
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         float c, s;
-        rope_cos_sin(pos, ((d - rope_off) >> 1) + j, d_r, base, &c, &s);
+        rope_cos_sin(pos, rt.inv_freq[((d - rope_off) >> 1) + j], &c, &s);
         const float a = v[i].v[2 * j], b = v[i].v[2 * j + 1];
         v[i].v[2 * j] = a * c - b * s;
         v[i].v[2 * j + 1] = a * s + b * c;
@@ -57,7 +59,7 @@ template <bool kF32In>
 __global__ void __launch_bounds__(256) k_qk_prep(const void* __restrict__ x, const int32_t* __restrict__ pos,
                                                  const int64_t* __restrict__ out_tok, lc_rows out,
                                                  int64_t n_rows, int H, int D, int d_r, int rope_off,
-                                                 float eps, float base) {
+                                                 float eps, RopeTable rt) {
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= n_rows) return;
@@ -73,12 +75,12 @@ __global__ void __launch_bounds__(256) k_qk_prep(const void* __restrict__ x, con
   const int64_t tok = row / H;
   const int p = __ldg(pos + tok);
   const int64_t orow = out_tok ? __ldg(out_tok + tok) * H + (row - tok * H) : row;
-  norm_rope_store(v, lane, D, d_r, rope_off, eps, p, base, out, orow);
+  norm_rope_store(v, lane, D, d_r, rope_off, eps, p, rt, out, orow);
 }
 
 // One warp per entry (CSA, m <= 64).
 template <bool kF32In>
-__global__ void __launch_bounds__(256) k_compress_warp(lc_compress_args a) {
+__global__ void __launch_bounds__(256) k_compress_warp(lc_compress_args a, RopeTable rt) {
   const int lane = threadIdx.x & 31;
   const int b = blockIdx.y;
   const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -121,14 +123,14 @@ __global__ void __launch_bounds__(256) k_compress_warp(lc_compress_args a) {
       }
     }
   }
-  norm_rope_store(acc, lane, D, a.dims.d_r, a.dims.rope_off, a.eps, (j + 1) * m - 1, a.rope_base, a.out,
+  norm_rope_store(acc, lane, D, a.dims.d_r, a.dims.rope_off, a.eps, (j + 1) * m - 1, rt, a.out,
                   __ldg(a.ent_start + b) + j);
 }
 
 // One CTA (8 warps) per entry (HCA, m >= 64): warp w sums tokens w, w + 8, ...; the
 // partial sums meet in shared memory and are added in a fixed order.
 template <bool kF32In>
-__global__ void __launch_bounds__(256) k_compress_cta(lc_compress_args a) {
+__global__ void __launch_bounds__(256) k_compress_cta(lc_compress_args a, RopeTable rt) {
   extern __shared__ float smem[];  // [8][D] partial sums, then [m] gate weights
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int b = blockIdx.y;
@@ -212,41 +214,50 @@ __global__ void __launch_bounds__(256) k_compress_cta(lc_compress_args a) {
       }
     }
   }
-  norm_rope_store(acc, lane, D, a.dims.d_r, a.dims.rope_off, a.eps, (j + 1) * m - 1, a.rope_base, a.out,
+  norm_rope_store(acc, lane, D, a.dims.d_r, a.dims.rope_off, a.eps, (j + 1) * m - 1, rt, a.out,
                   __ldg(a.ent_start + b) + j);
+}
+
+RopeTable make_rope_table(int d_r, float base) {
+  RopeTable t{};
+  for (int i = 0; i < d_r / 2 && i < kMaxRopePairs; ++i)
+    t.inv_freq[i] = std::pow(static_cast<double>(base), -2.0 * i / static_cast<double>(d_r));
+  return t;
 }
 
 cudaError_t launch_qk_prep(const lc_qk_prep_args& a, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(a.n_tok) * a.dims.H;
   if (rows == 0) return cudaSuccess;
+  const RopeTable rt = make_rope_table(a.dims.d_r, a.rope_base);
   const int wpb = 8;
   const dim3 grid(static_cast<unsigned>((rows + wpb - 1) / wpb));
   if (a.in_fmt == LC_FMT_F32)
     k_qk_prep<true><<<grid, 32 * wpb, 0, st>>>(a.x, a.pos, a.out_tok, a.out, rows, a.dims.H, a.dims.D, a.dims.d_r,
-                                                a.dims.rope_off, a.eps, a.rope_base);
+                                                a.dims.rope_off, a.eps, rt);
   else
     k_qk_prep<false><<<grid, 32 * wpb, 0, st>>>(a.x, a.pos, a.out_tok, a.out, rows, a.dims.H, a.dims.D, a.dims.d_r,
-                                                 a.dims.rope_off, a.eps, a.rope_base);
+                                                 a.dims.rope_off, a.eps, rt);
   return cudaGetLastError();
 }
 
 cudaError_t launch_compress(const lc_compress_args& a, bool per_cta, cudaStream_t st) {
   if (a.max_blocks <= 0 || a.num_seqs <= 0) return cudaSuccess;
   const bool f32 = a.in_fmt == LC_FMT_F32;
+  const RopeTable rt = make_rope_table(a.dims.d_r, a.rope_base);
   if (!per_cta) {
     const int wpb = 8;
     const dim3 grid((a.max_blocks + wpb - 1) / wpb, a.num_seqs);
-    if (f32) k_compress_warp<true><<<grid, 32 * wpb, 0, st>>>(a);
-    else k_compress_warp<false><<<grid, 32 * wpb, 0, st>>>(a);
+    if (f32) k_compress_warp<true><<<grid, 32 * wpb, 0, st>>>(a, rt);
+    else k_compress_warp<false><<<grid, 32 * wpb, 0, st>>>(a, rt);
   } else {
     const dim3 grid(a.max_blocks, a.num_seqs);
     const size_t sm = static_cast<size_t>(8 * a.dims.D + a.m) * sizeof(float);
     if (f32) {
       cudaFuncSetAttribute(k_compress_cta<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
-      k_compress_cta<true><<<grid, 256, sm, st>>>(a);
+      k_compress_cta<true><<<grid, 256, sm, st>>>(a, rt);
     } else {
       cudaFuncSetAttribute(k_compress_cta<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
-      k_compress_cta<false><<<grid, 256, sm, st>>>(a);
+      k_compress_cta<false><<<grid, 256, sm, st>>>(a, rt);
     }
   }
   return cudaGetLastError();

@@ -6,7 +6,7 @@
 // passes over a shared-memory histogram find the K-th largest key T and how many of the
 // keys equal to T to take.  A final pass in index order keeps every key > T and the first
 // `need` keys == T (ties to the lower index), writing indices in ascending order through
-// block-wide prefix counts.  Rows of up to kRowCache scores are staged in shared memory
+// per-warp counts.  Rows of up to kRowCache scores are staged in shared memory
 // once; longer rows are re-read from global memory (L2) on each pass.  The result depends
 // only on the score values: it is bit-exact and independent of the launch shape.
 #include "lc_internal.h"
@@ -22,35 +22,9 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Block-wide exclusive prefix count of `flag` over the CTA's threads in thread order.
-// Returns the count before this thread; *total receives the CTA total.
-__device__ __forceinline__ int block_excl_count(bool flag, int* warp_tot, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t bal = __ballot_sync(0xffffffffu, flag);
-  const int in_warp = __popc(bal & ((1u << lane) - 1u));
-  __syncthreads();  // warp_tot free from its previous use
-  if (lane == 0) warp_tot[warp] = __popc(bal);
-  __syncthreads();
-  if (warp == 0) {
-    int v = lane < kTopkWarps ? warp_tot[lane] : 0;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += n;
-    }
-    if (lane < kTopkWarps) warp_tot[lane] = incl - v;  // exclusive
-    if (lane == 31) warp_tot[kTopkWarps] = incl;
-  }
-  __syncthreads();
-  *total = warp_tot[kTopkWarps];
-  return warp_tot[warp] + in_warp;
-}
-
 __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_cache) {
   extern __shared__ uint32_t cache[];  // [kRowCache] keys when the row fits
   __shared__ int hist[256];
-  __shared__ int warp_tot[kTopkWarps + 1];
   __shared__ uint32_t s_prefix;
   __shared__ int s_remaining;
 
@@ -78,9 +52,21 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += kTopkThreads) {
-      const uint32_t u = cached ? cache[i] : order_key(__ldg(row + i));
-      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 0xffu], 1);
+    // scores of one row share their high bits, so in the first passes whole warps often
+    // hit one bin: then a single lane adds 32
+    for (int base = 0; base < n; base += kTopkThreads) {
+      const int i = base + tid;
+      int bin = 256;  // not a candidate
+      if (i < n) {
+        const uint32_t u = cached ? cache[i] : order_key(__ldg(row + i));
+        if ((u & mask) == prefix) bin = static_cast<int>((u >> shift) & 0xffu);
+      }
+      const int b0 = __shfl_sync(0xffffffffu, bin, 0);
+      if (__all_sync(0xffffffffu, bin == b0)) {
+        if ((tid & 31) == 0 && b0 < 256) atomicAdd(&hist[b0], 32);
+      } else if (bin < 256) {
+        atomicAdd(&hist[bin], 1);
+      }
     }
     __syncthreads();
     if (tid < 32) {
@@ -118,23 +104,49 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
     remaining = s_remaining;
     mask |= 0xffu << shift;
   }
-  // keys > prefix: all taken (K - remaining of them); keys == prefix: first `remaining`
+  // keys > T are all taken (K - need of them); of the keys == T the first `need` in index
+  // order.  Warp w owns the contiguous segment [w * seg, (w + 1) * seg): it counts its keys
+  // > T and == T, the counts of the warps before it give its first tie rank and output
+  // slot, and it writes its selections in index order with warp ballots.
   const uint32_t T = prefix;
   const int need = remaining;
-  int eq_seen = 0, written = 0;
-  for (int base = 0; base < n && written < K; base += kTopkThreads) {
-    const int i = base + tid;
-    uint32_t u = 0;
-    if (i < n) u = cached ? cache[i] : order_key(__ldg(row + i));
-    const bool eq = i < n && u == T;
-    int eq_tot;
-    const int eq_rank = eq_seen + block_excl_count(eq, warp_tot, &eq_tot);
-    const bool sel = i < n && (u > T || (eq && eq_rank < need));
-    int sel_tot;
-    const int pos = written + block_excl_count(sel, warp_tot, &sel_tot);
-    if (sel) out[pos] = i;
-    eq_seen += eq_tot;
-    written += sel_tot;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int seg = (n + kTopkWarps - 1) / kTopkWarps;
+  const int lo = min(n, warp * seg), hi = min(n, lo + seg);
+  int gt_c = 0, eq_c = 0;
+  for (int i = lo + lane; i < hi; i += 32) {
+    const uint32_t u = cached ? cache[i] : order_key(__ldg(row + i));
+    gt_c += u > T;
+    eq_c += u == T;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    gt_c += __shfl_xor_sync(0xffffffffu, gt_c, o);
+    eq_c += __shfl_xor_sync(0xffffffffu, eq_c, o);
+  }
+  __shared__ int s_gt[kTopkWarps], s_eq[kTopkWarps];
+  if (lane == 0) {
+    s_gt[warp] = gt_c;
+    s_eq[warp] = eq_c;
+  }
+  __syncthreads();
+  int eq_rank = 0, pos = 0;
+  for (int w = 0; w < warp; ++w) {
+    pos += s_gt[w] + min(max(need - eq_rank, 0), s_eq[w]);
+    eq_rank += s_eq[w];
+  }
+  const uint32_t below = (1u << lane) - 1u;
+  for (int base = lo; base < hi; base += 32) {
+    const int i = base + lane;
+    const bool valid = i < hi;
+    const uint32_t u = valid ? (cached ? cache[i] : order_key(__ldg(row + i))) : 0u;
+    const bool eq = valid && u == T;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+    const bool sel = valid && (u > T || (eq && eq_rank + __popc(eqm & below) < need));
+    const uint32_t selm = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[pos + __popc(selm & below)] = i;
+    eq_rank += __popc(eqm);
+    pos += __popc(selm);
   }
 }
 

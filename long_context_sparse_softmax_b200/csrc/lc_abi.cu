@@ -10,7 +10,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 lc_status check_dims(const lc_dims& d) {
   if (d.D < 8 || d.D > 1024 || d.D % 8) return LC_ERR_ARG;
-  if (d.d_r < 0 || d.d_r > d.D || d.d_r % 8) return LC_ERR_ARG;
+  if (d.d_r < 0 || d.d_r > d.D || d.d_r % 8 || d.d_r > 2 * lc::kMaxRopePairs) return LC_ERR_ARG;
   if (d.rope_off < 0 || d.rope_off % 8 || d.rope_off + d.d_r > d.D) return LC_ERR_ARG;
   if (d.H < 1) return LC_ERR_ARG;
   return LC_OK;
@@ -89,6 +89,8 @@ lc_status index_scores(const lc_index_args* a, void* stream, bool decode) {
   LC_TRY(check_batch(a->batch, true, false));
   if (!a->q || !a->k || !a->w || !a->scores) return LC_ERR_ARG;
   if (a->fmt == LC_IDX_MXFP4 && (!a->q_scale || !a->k_scale)) return LC_ERR_ARG;
+  if (a->fmt == LC_IDX_MXFP4 && ((reinterpret_cast<uintptr_t>(a->q_scale) | reinterpret_cast<uintptr_t>(a->k_scale)) & 3u))
+    return LC_ERR_ALIGN;
   if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->scores)) return LC_ERR_ALIGN;
   return launched(lc::launch_index_scores(*a, decode, static_cast<cudaStream_t>(stream)));
 }
@@ -147,11 +149,12 @@ lc_status lc_csa_sparse_attn_decode(const lc_attn_args* a, void* stream) { retur
 lc_status lc_hca_attn_prefill(const lc_attn_args* a, void* stream) { return attn(a, stream, false, false); }
 lc_status lc_hca_attn_decode(const lc_attn_args* a, void* stream) { return attn(a, stream, false, true); }
 
+// Workspace of the decode variant (the prefill variant needs none).
 size_t lc_csa_sparse_attn_workspace_bytes(const lc_attn_args* a) {
-  return a ? lc::attn_workspace_bytes(*a, true, a->n_q == a->batch.num_seqs && a->batch.num_seqs > 1) : 0;
+  return a ? lc::attn_workspace_bytes(*a, true, true) : 0;
 }
 size_t lc_hca_attn_workspace_bytes(const lc_attn_args* a) {
-  return a ? lc::attn_workspace_bytes(*a, false, a->n_q == a->batch.num_seqs && a->batch.num_seqs > 1) : 0;
+  return a ? lc::attn_workspace_bytes(*a, false, true) : 0;
 }
 
 const char* lc_version(void) { return "lc 0.1.0 (CSA/HCA attention, sm_100a)"; }

@@ -49,11 +49,17 @@ __device__ __forceinline__ void set_status(int32_t* status, int32_t bit) {
   if (status) atomicOr(status, bit);
 }
 
-// cos / sin of pos * base^(-2i/d_r).  The angle reaches ~1e6 rad at a 1M-token
-// position, so it is formed and reduced to [-pi, pi] in double precision (two-constant
-// additive reduction, Cody & Waite 1980) before the single-precision sincosf.
-__device__ __forceinline__ void rope_cos_sin(int pos, int i, int d_r, float base, float* c, float* s) {
-  const double inv_freq = pow(static_cast<double>(base), -2.0 * static_cast<double>(i) / static_cast<double>(d_r));
+// RoPE frequencies base^(-2i/d_r), i < d_r / 2, computed once per call on the host in
+// double precision and passed by value to the kernels.
+constexpr int kMaxRopePairs = 64;
+struct RopeTable {
+  double inv_freq[kMaxRopePairs];
+};
+
+// cos / sin of pos * inv_freq.  The angle reaches ~1e6 rad at a 1M-token position, so it
+// is formed and reduced to [-pi, pi] in double precision (two-constant additive
+// reduction, Cody & Waite 1980) before the single-precision sincosf.
+__device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c, float* s) {
   const double ang = static_cast<double>(pos) * inv_freq;
   const double kTwoPiHi = 6.283185307179586232;        // nearest double to 2*pi
   const double kTwoPiLo = 2.449293598294706e-16;       // 2*pi - kTwoPiHi

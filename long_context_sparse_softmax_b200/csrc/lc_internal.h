@@ -13,6 +13,11 @@ cudaError_t launch_index_scores(const lc_index_args& a, bool decode, cudaStream_
 cudaError_t launch_topk(const lc_topk_args& a, bool decode, cudaStream_t st);
 cudaError_t launch_attn(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st);
 size_t attn_workspace_bytes(const lc_attn_args& a, bool sparse, bool decode);
+bool attn_mma_supported(const lc_attn_args& a);
+size_t attn_mma_workspace(const lc_attn_args& a, bool sparse, bool decode);
+cudaError_t launch_attn_mma(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st);
+bool index_tc_supported(const lc_index_args& a);
+cudaError_t launch_index_tc(const lc_index_args& a, bool decode, cudaStream_t st);
 
 // Sequence of query row q: the b with q_start[b] <= q < q_start[b+1] (binary search).
 __device__ __forceinline__ int seq_of_query(const int32_t* __restrict__ q_start, int num_seqs, int q) {

@@ -37,15 +37,44 @@ def idx_operand_np(op: Dict[str, torch.Tensor], rows=None):
     return d
 
 
+# Absolute error of the library's FP32 evaluation of a normalised row value (|v| <= sqrt(D)):
+# a few FP32 roundings of terms of size <= 24.  RoPE's a*c - b*s can cancel to a value
+# much smaller than its terms, so this error is absolute, not relative to the result.
+FP32_EVAL_ABS = 1e-5
+
+
 def stored_close(fmt: int, got_f64: np.ndarray, exp_f64: np.ndarray, d_n: int) -> np.ndarray:
-    """Per-element acceptance of stored rows: one grid step of the storage format."""
+    """Per-element acceptance of stored rows: the two pre-rounding values differ by at most
+    the FP32 evaluation error, so the stored values differ by at most that plus one grid
+    step of the storage format (taken at the larger magnitude)."""
+    mag = np.maximum(np.abs(got_f64), np.abs(exp_f64))
+    ev = FP32_EVAL_ABS * np.maximum(1.0, np.abs(exp_f64))
     if fmt == O.FMT_F32:
-        tol = np.full(exp_f64.shape, 1e-5)
+        tol = ev
     elif fmt == O.FMT_BF16:
-        tol = O.ulp_bf16(exp_f64) * 1.0001
+        tol = O.ulp_bf16(mag) + ev
     else:
-        tol = np.concatenate([O.ulp_e4m3(exp_f64[..., :d_n]), O.ulp_bf16(exp_f64[..., d_n:])], -1) * 1.0001
+        tol = np.concatenate([O.ulp_e4m3(mag[..., :d_n]), O.ulp_bf16(mag[..., d_n:])], -1) + ev
     return np.abs(got_f64 - exp_f64) <= tol
+
+
+# A stored value can differ from the oracle's only where the pre-rounding value lies within
+# the FP32 evaluation error (~1e-6 relative) of a rounding midpoint: a rare event.  A
+# systematic shift (a wrong scale, a wrong rounding mode) would move many values by one
+# grid step and still pass the per-element check, so the fraction of differing values is
+# bounded too.
+MAX_FLIP_FRACTION = 1e-3
+
+
+def stored_check(fmt: int, got_f64: np.ndarray, exp_f64: np.ndarray, d_n: int, what: str) -> float:
+    ok = stored_close(fmt, got_f64, exp_f64, d_n)
+    assert ok.all(), f"{what}: {(~ok).sum()} elements beyond one grid step"
+    n_diff = int(np.sum(got_f64 != exp_f64))
+    frac = n_diff / got_f64.size if got_f64.size else 0.0
+    if fmt != O.FMT_F32:
+        assert n_diff <= MAX_FLIP_FRACTION * got_f64.size + 3, \
+            f"{what}: {n_diff} of {got_f64.size} stored values differ from the oracle's"
+    return frac
 
 
 def rows_np(fmt: int, r: Dict[str, torch.Tensor], sel=None) -> np.ndarray:
@@ -73,9 +102,63 @@ def out_np(run, q_sel: Sequence[int]) -> np.ndarray:
 
 
 def attn_ok(got: np.ndarray, exp: np.ndarray, out_f32: bool):
+    """Acceptance of one query's attention output [H, D].
+
+    FP32 output: max-abs error <= 1e-4.  BF16 output: for each head, max-abs error over
+    its D-dim output vector <= 2e-2 x that vector's RMS.  (An RMS pooled over heads of
+    very different magnitude - one sharp head next to diffuse ones - would reject the
+    exact result rounded to BF16 itself, whose error reaches 2^-9 |o|.)
+    Returns (ok, worst err, its tolerance)."""
+    if got.size == 0:
+        return True, 0.0, 1.0
+    if out_f32:
+        err = float(np.max(np.abs(got - exp)))
+        return err <= ATTN_TOL_F32, err, ATTN_TOL_F32
+    err_h = np.max(np.abs(got - exp), axis=-1)
+    tol_h = ATTN_TOL_REL_BF16 * np.sqrt(np.mean(exp * exp, axis=-1))
+    ratio = np.where(tol_h > 0, err_h / np.where(tol_h > 0, tol_h, 1.0), np.where(err_h > 0, np.inf, 0.0))
+    h = int(np.argmax(ratio))
+    return bool(np.all(err_h <= tol_h)), float(err_h[h]), float(tol_h[h])
+
+
+def attn_e2e_ok(got: np.ndarray, exp: np.ndarray, out_f32: bool):
+    """End-to-end acceptance (the library's own intermediates, which may sit one storage
+    grid step away from the oracle's): max-abs error over the query's whole output
+    <= 2e-2 x the RMS of that output (FP32: <= 1e-4)."""
     err = float(np.max(np.abs(got - exp))) if got.size else 0.0
     tol = ATTN_TOL_F32 if out_f32 else ATTN_TOL_REL_BF16 * O.rms(exp)
     return err <= tol, err, tol
+
+
+# End to end, the library's stored FP8 intermediates can sit one E4M3 step (up to 12.5% of
+# an element) away from the oracle's where an FP32 and a float64 evaluation straddle a
+# rounding midpoint; such a flipped element reaches the output with its key's softmax
+# weight.  The end-to-end check therefore asks that nearly every (query, head) output
+# meets the per-head tolerance and that none is grossly off; the stage-wise check on
+# identical inputs applies the tolerance to every row.
+E2E_MIN_ROW_FRACTION = 0.99
+E2E_MAX_RATIO = 8.0
+
+
+def attn_e2e_rows(got: np.ndarray, exp: np.ndarray, out_f32: bool):
+    """(rows within tolerance, rows, worst err/tol) for one query's output [H, D]."""
+    if out_f32:
+        ok, err, tol = attn_ok(got, exp, True)
+        return int(ok) * got.shape[0], got.shape[0], err / tol
+    err_h = np.max(np.abs(got - exp), axis=-1)
+    tol_h = ATTN_TOL_REL_BF16 * np.sqrt(np.mean(exp * exp, axis=-1))
+    ratio = np.where(tol_h > 0, err_h / np.where(tol_h > 0, tol_h, 1.0), np.where(err_h > 0, np.inf, 0.0))
+    return int(np.sum(ratio <= 1.0)), got.shape[0], float(np.max(ratio))
+
+
+def attn_err_in_ulps(got: np.ndarray, exp: np.ndarray, out_f32: bool) -> float:
+    """Largest error in units of the output format's grid step at that value (reported,
+    not asserted: the tensor-core path rounds the softmax weights to BF16 before P V)."""
+    if got.size == 0:
+        return 0.0
+    mag = np.maximum(np.abs(got), np.abs(exp))
+    step = np.full(mag.shape, 2.0 ** -23) * np.maximum(mag, 1e-30) if out_f32 else O.ulp_bf16(mag)
+    return float(np.max(np.abs(got - exp) / np.maximum(step, 1e-30)))
 
 
 def topk_sets_ok(got_idx: np.ndarray, exp_idx: np.ndarray, s_oracle: np.ndarray, k: int, fp32: bool,
