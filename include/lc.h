@@ -60,7 +60,9 @@ enum {
   LC_ERR_ALIGN = 2,        /* a buffer not 16-byte aligned */
   LC_ERR_UNSUPPORTED = 3,  /* a format / shape combination this build has no kernel for */
   LC_ERR_WORKSPACE = 4,    /* workspace missing or smaller than *_workspace_bytes() */
-  LC_ERR_LAUNCH = 5        /* the CUDA launch failed */
+  LC_ERR_LAUNCH = 5,       /* the CUDA launch failed */
+  LC_ERR_TOO_LARGE = 6     /* the call needs more scratch than the allocation-free entry
+                              point's fixed array holds */
 };
 
 /* Bits OR-ed into *status by the kernels. */
@@ -272,6 +274,31 @@ lc_status lc_hca_attn_decode(const lc_attn_args* a, void* stream);
 
 size_t lc_csa_sparse_attn_workspace_bytes(const lc_attn_args* a);
 size_t lc_hca_attn_workspace_bytes(const lc_attn_args* a);
+
+/* ---------------------------------------------------------------------------------
+ * lc_csa_sparse_attn_decode_static — lc_csa_sparse_attn_decode for callers that cannot
+ * allocate device memory when they call: hosts that give all device memory to their own
+ * allocator up front and forbid any other allocation, and latency-bound serving loops
+ * that must not pay for the device-wide synchronisation cudaMalloc can imply.  The pages
+ * have no counterpart; it is a property of this library's interface.
+ *
+ * Same arguments and results as lc_csa_sparse_attn_decode, except that a->workspace and
+ * a->workspace_bytes are ignored: the scratch is a fixed array of
+ * lc_csa_sparse_attn_decode_static_capacity() bytes (16 MiB) compiled into the library,
+ * held on every device that loads the library until the process exits.  The call
+ * allocates and frees nothing.
+ *   - If the call needs more scratch than the array holds (lc_csa_sparse_attn_workspace_bytes
+ *     above the capacity), it returns LC_ERR_TOO_LARGE before touching the device.
+ *   - The first call on a device, with that device current, looks up the array's device
+ *     address (cudaGetSymbolAddress) and keeps it; make that first call before any stream
+ *     capture on the device.
+ *   - Every call on a device shares the one array.  Calls whose executions overlap on the
+ *     GPU (different streams, or other threads) race on it and give wrong results: order
+ *     them on one stream or serialise them.  Nothing carries over from one call to the
+ *     next: every scratch word a call reads, the same call has written first.
+ * ------------------------------------------------------------------------------- */
+lc_status lc_csa_sparse_attn_decode_static(const lc_attn_args* a, void* stream);
+size_t lc_csa_sparse_attn_decode_static_capacity(void);
 
 /* Library version string (static storage). */
 const char* lc_version(void);

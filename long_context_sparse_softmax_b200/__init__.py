@@ -17,7 +17,7 @@ from ctypes import c_float, c_int32, c_int64, c_size_t, c_void_p
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblc.so")
 
-LC_OK, LC_ERR_ARG, LC_ERR_ALIGN, LC_ERR_UNSUPPORTED, LC_ERR_WORKSPACE, LC_ERR_LAUNCH = range(6)
+LC_OK, LC_ERR_ARG, LC_ERR_ALIGN, LC_ERR_UNSUPPORTED, LC_ERR_WORKSPACE, LC_ERR_LAUNCH, LC_ERR_TOO_LARGE = range(7)
 LC_DEV_BAD_INDEX, LC_DEV_WINDOW_RANGE, LC_DEV_BAD_BLOCK, LC_DEV_NONVISIBLE, LC_DEV_TIMEOUT = 1, 2, 4, 8, 16
 LC_FMT_F32, LC_FMT_BF16, LC_FMT_E4M3_BF16 = 0, 1, 2
 LC_IDX_F32, LC_IDX_MXFP4 = 0, 3
@@ -86,9 +86,10 @@ ENTRY_POINTS = {
     "lc_csa_topk_prefill": TopkArgs, "lc_csa_topk_decode": TopkArgs,
     "lc_csa_sparse_attn_prefill": AttnArgs, "lc_csa_sparse_attn_decode": AttnArgs,
     "lc_hca_attn_prefill": AttnArgs, "lc_hca_attn_decode": AttnArgs,
+    "lc_csa_sparse_attn_decode_static": AttnArgs,
 }
 HELPERS = ["lc_csa_sparse_attn_workspace_bytes", "lc_hca_attn_workspace_bytes", "lc_version",
-           "lc_status_string", "lc_struct_size"]
+           "lc_status_string", "lc_struct_size", "lc_csa_sparse_attn_decode_static_capacity"]
 
 
 def _load() -> ctypes.CDLL:
@@ -103,6 +104,7 @@ def _load() -> ctypes.CDLL:
         fn = getattr(so, name)
         fn.argtypes = [ctypes.POINTER(AttnArgs)]
         fn.restype = c_size_t
+    so.lc_csa_sparse_attn_decode_static_capacity.restype = c_size_t
     so.lc_version.restype = ctypes.c_char_p
     so.lc_status_string.argtypes = [c_int32]
     so.lc_status_string.restype = ctypes.c_char_p
@@ -151,6 +153,10 @@ def lc_csa_sparse_attn_workspace_bytes(args: AttnArgs) -> int:
 
 def lc_hca_attn_workspace_bytes(args: AttnArgs) -> int:
     return int(lib.lc_hca_attn_workspace_bytes(ctypes.byref(args)))
+
+
+def lc_csa_sparse_attn_decode_static_capacity() -> int:
+    return int(lib.lc_csa_sparse_attn_decode_static_capacity())
 
 
 def lc_version() -> str:

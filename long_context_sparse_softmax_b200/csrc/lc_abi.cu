@@ -167,6 +167,7 @@ const char* lc_status_string(lc_status s) {
     case LC_ERR_UNSUPPORTED: return "LC_ERR_UNSUPPORTED: no kernel for this format/shape";
     case LC_ERR_WORKSPACE: return "LC_ERR_WORKSPACE: workspace missing or too small";
     case LC_ERR_LAUNCH: return "LC_ERR_LAUNCH: CUDA launch failed";
+    case LC_ERR_TOO_LARGE: return "LC_ERR_TOO_LARGE: needs more scratch than the static array holds";
     default: return "unknown lc_status";
   }
 }

@@ -45,7 +45,7 @@ def test_struct_layouts_match_binding():
 
 def test_version_and_status_strings():
     assert "sm_100a" in lc.lc_version()
-    for s in range(6):
+    for s in range(7):
         assert lc.lib.lc_status_string(s).decode().startswith("LC_")
 
 
