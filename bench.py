@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0)
+    ap.add_argument("--attn-impl", default="auto", choices=["auto", "mma", "tc", "ref"],
+                    help="attention kernel (auto: the fastest measured for the shape)")
     return ap.parse_args()
 
 
@@ -226,7 +228,7 @@ STAGE_SOURCE = {"qk_prep_q": "k_prep.cu", "qk_prep_win": "k_prep.cu", "compress"
 # ------------------------------------------------------------------------------------
 # the library arm
 # ------------------------------------------------------------------------------------
-def make_runs(name, device, rank):
+def make_runs(name, device, rank, impl=0):
     from long_context_sparse_softmax_b200 import runner
     from long_context_sparse_softmax_b200 import workloads as wl
     runs = []
@@ -235,7 +237,7 @@ def make_runs(name, device, rank):
             import dataclasses
             spec = dataclasses.replace(spec, seed=spec.seed + 1000 * rank)
         inp = (wl.make_decode if spec.is_decode else wl.make_prefill)(spec, device)
-        r = (runner.Decode if spec.is_decode else runner.Prefill)(inp, device)
+        r = (runner.Decode if spec.is_decode else runner.Prefill)(inp, device, None, impl)
         runs.append((spec, inp, r))
     return runs
 
@@ -270,7 +272,7 @@ def run_lc(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     pk, pk_kind = peaks()
-    runs = make_runs(args.workload, dev, rank)
+    runs = make_runs(args.workload, dev, rank, {"auto": 0, "mma": 1, "tc": 2, "ref": 3}[args.attn_impl])
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -286,18 +288,34 @@ def run_lc(args):
             work[f"{i}:{k}"] = v
         units += u if i == 0 else 0  # a mixed step counts each sequence's token once
     stage_names = [f"{i}:{n}" for i, (_, _, r) in enumerate(runs) for n, _ in r.stages()]
-    stage_fns = [f for (_, _, r) in runs for _, f in r.stages()]
-    n_launch = len(stage_fns)
+    # kernels per step: one per call, plus the combine kernel of a key-split attention
+    n_launch = len(stage_names) + sum(1 for (_, _, r) in runs if r.a_attn.workspace_bytes > 0)
+    side = torch.cuda.Stream(dev)
+
+    def one_step(stage_ev=None):
+        """The whole path once: per workload, preparation and compression on the side
+        stream next to index -> top-k on the main stream, then attention."""
+        for i, (_, _, r) in enumerate(runs):
+            def on_stage(name, st, fn, i=i):
+                if stage_ev is None:
+                    fn(st)
+                    return
+                e0, e1 = stage_ev[f"{i}:{name}"]
+                e0.record(st)
+                fn(st)
+                e1.record(st)
+            r.step_overlapped(stream, side, on_stage)
 
     for _ in range(args.warmup):
-        for f in stage_fns:
-            f(stream)
+        one_step()
     torch.cuda.synchronize()
     for _, _, r in runs:
         assert r.read_status() == 0, "device status bits set"
 
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in stage_fns]
+    ev = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in stage_names}
           for _ in range(args.steps)]
+    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     try:
@@ -307,23 +325,14 @@ def run_lc(args):
     with ClockSampler(gpu_id) as clk:
         for s in range(args.steps):
             flush.zero_()
-            for j, f in enumerate(stage_fns):
-                ev[s][j][0].record(stream)
-                f(stream)
-                ev[s][j][1].record(stream)
+            ev_step[s][0].record(stream)
+            one_step(ev[s])
+            ev_step[s][1].record(stream)
         torch.cuda.synchronize()
     barrier()
-    per_stage = {n: [] for n in stage_names}
-    step_ms = []
-    for s in range(args.steps):
-        tot = 0.0
-        for j, n in enumerate(stage_names):
-            t = ev[s][j][0].elapsed_time(ev[s][j][1])
-            per_stage[n].append(t)
-            tot += t
-        step_ms.append(tot)
-    # a step's time runs from its first stage's start to its last stage's end
-    span = [ev[s][0][0].elapsed_time(ev[s][-1][1]) for s in range(args.steps)]
+    per_stage = {n: [ev[s][n][0].elapsed_time(ev[s][n][1]) for s in range(args.steps)] for n in stage_names}
+    # a step's time runs from the fork on the main stream to the end of attention
+    span = [ev_step[s][0].elapsed_time(ev_step[s][1]) for s in range(args.steps)]
     total_ms = sum(span)
     t_max = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -347,8 +356,7 @@ def run_lc(args):
             for ins, _ in io:
                 for d, h in ins:
                     d.copy_(h, non_blocking=True)
-            for f in stage_fns:
-                f(stream)
+            one_step()
             for _, outs in io:
                 for d, h in outs:
                     h.copy_(d, non_blocking=True)

@@ -71,8 +71,10 @@ enum {
   LC_DEV_WINDOW_RANGE = 2, /* a window position outside the given window rows: skipped */
   LC_DEV_BAD_BLOCK = 4,    /* a block whose tokens are not in the given token rows: skipped */
   LC_DEV_NONVISIBLE = 8,   /* a selected entry not visible to its query: skipped */
-  LC_DEV_TIMEOUT = 16      /* a bounded wait on the tensor core gave up: results of that
+  LC_DEV_TIMEOUT = 16,     /* a bounded wait on the tensor core gave up: results of that
                               CTA are missing (never expected; reported, not hung) */
+  LC_DEV_RANGE = 32        /* an attention logit above 80: the inputs were not
+                              RMS-normalised as the method prescribes */
 };
 
 /* Row storage formats. */
@@ -221,8 +223,8 @@ typedef struct lc_topk_args {
   int32_t W_x;
   int32_t max_ent;         /* host value */
   int32_t reserved;
-  const float* scores;     /* [n_q, score_stride] */
-  int64_t score_stride;
+  const float* scores;     /* [n_q, score_stride], 16-byte aligned */
+  int64_t score_stride;    /* >= max_ent, multiple of 4 */
   lc_batch batch;          /* q_start, q_pos0, n_ent */
   int32_t* idx;            /* [n_q, k] */
   int32_t* count;          /* [n_q] or NULL */
@@ -265,7 +267,20 @@ typedef struct lc_attn_args {
   void* workspace;
   size_t workspace_bytes;
   int32_t* status;
+  int32_t impl;            /* LC_IMPL_AUTO (0) picks the fastest kernel for the shape;
+                              LC_IMPL_MMA, LC_IMPL_TC, LC_IMPL_REF force one (results agree
+                              within the BF16 tolerance; LC_ERR_UNSUPPORTED if it cannot run
+                              the shape) */
+  int32_t reserved;
 } lc_attn_args;
+
+/* Attention kernels. */
+enum {
+  LC_IMPL_AUTO = 0,
+  LC_IMPL_MMA = 1,         /* BF16 mma.sync tiles (576-dim entries) */
+  LC_IMPL_TC = 2,          /* tcgen05 tiles, accumulators in tensor memory (576-dim entries) */
+  LC_IMPL_REF = 3          /* one warp per (query, head), FP32 CUDA cores (any shape) */
+};
 
 lc_status lc_csa_sparse_attn_prefill(const lc_attn_args* a, void* stream);
 lc_status lc_csa_sparse_attn_decode(const lc_attn_args* a, void* stream);

@@ -18,7 +18,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblc.so")
 
 LC_OK, LC_ERR_ARG, LC_ERR_ALIGN, LC_ERR_UNSUPPORTED, LC_ERR_WORKSPACE, LC_ERR_LAUNCH, LC_ERR_TOO_LARGE = range(7)
-LC_DEV_BAD_INDEX, LC_DEV_WINDOW_RANGE, LC_DEV_BAD_BLOCK, LC_DEV_NONVISIBLE, LC_DEV_TIMEOUT = 1, 2, 4, 8, 16
+LC_DEV_BAD_INDEX, LC_DEV_WINDOW_RANGE, LC_DEV_BAD_BLOCK, LC_DEV_NONVISIBLE, LC_DEV_TIMEOUT, LC_DEV_RANGE = \
+    1, 2, 4, 8, 16, 32
 LC_FMT_F32, LC_FMT_BF16, LC_FMT_E4M3_BF16 = 0, 1, 2
 LC_IDX_F32, LC_IDX_MXFP4 = 0, 3
 
@@ -73,7 +74,11 @@ class AttnArgs(ctypes.Structure):
     _fields_ = [("dims", Dims), ("n_q", c_int32), ("k", c_int32), ("m", c_int32), ("W", c_int32), ("W_x", c_int32),
                 ("max_ent", c_int32), ("scale", c_float), ("out_fmt", c_int32), ("q", Rows), ("ent", Rows),
                 ("win", Rows), ("idx", c_void_p), ("sink", c_void_p), ("batch", Batch), ("out", c_void_p),
-                ("lse", c_void_p), ("workspace", c_void_p), ("workspace_bytes", c_size_t), ("status", c_void_p)]
+                ("lse", c_void_p), ("workspace", c_void_p), ("workspace_bytes", c_size_t), ("status", c_void_p),
+                ("impl", c_int32), ("reserved", c_int32)]
+
+
+LC_IMPL_AUTO, LC_IMPL_MMA, LC_IMPL_TC, LC_IMPL_REF = 0, 1, 2, 3
 
 
 STRUCTS = [Rows, Dims, Batch, QkPrepArgs, CompressArgs, IndexArgs, TopkArgs, AttnArgs]

@@ -132,18 +132,48 @@ __global__ void __launch_bounds__(256) k_attn_ref(lc_attn_args a, int sparse) {
   if (a.lse && lane == 0) a.lse[qrow] = st.m + logf(st.z);
 }
 
-size_t attn_workspace_bytes(const lc_attn_args& a, bool sparse, bool decode) {
-  return attn_mma_supported(a) ? attn_mma_workspace(a, sparse, decode) : 0;
+// The kernel a call runs (never LC_IMPL_AUTO): AUTO takes the fastest one measured for
+// 576-dim BF16 / E4M3 shapes, the BF16 mma.sync kernel; other shapes (FP32, other head
+// dims) run on the reference kernel.
+int attn_impl(const lc_attn_args& a) {
+  if (a.impl != LC_IMPL_AUTO) return a.impl;
+  return attn_mma_supported(a) ? LC_IMPL_MMA : LC_IMPL_REF;
 }
 
-// 576-dim BF16/E4M3 shapes go to the tensor-core kernel (k_attn_mma.cu); FP32 and other
-// head dims use the reference kernel.
+bool attn_impl_ok(const lc_attn_args& a) {
+  switch (attn_impl(a)) {
+    case LC_IMPL_MMA: return attn_mma_supported(a);
+    case LC_IMPL_TC: return attn_tc_supported(a);
+    case LC_IMPL_REF: return true;
+    default: return false;
+  }
+}
+
+size_t attn_workspace_bytes(const lc_attn_args& a, bool sparse, bool decode) {
+  switch (attn_impl(a)) {
+    case LC_IMPL_MMA: return attn_mma_supported(a) ? attn_mma_workspace(a, sparse, decode) : 0;
+    case LC_IMPL_TC: return attn_tc_supported(a) ? attn_tc_workspace(a, sparse, decode) : 0;
+    default: return 0;
+  }
+}
+
 cudaError_t launch_attn(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st) {
   if (a.n_q == 0) return cudaSuccess;
-  if (attn_mma_supported(a)) return launch_attn_mma(a, sparse, decode, st);
-  const dim3 grid(a.n_q, (a.dims.H + 7) / 8);
-  k_attn_ref<<<grid, 256, 0, st>>>(a, sparse ? 1 : 0);
-  return cudaGetLastError();
+  switch (attn_impl(a)) {
+    case LC_IMPL_TC: {
+      int n_split = 1;
+      cudaError_t e = launch_attn_tc(a, sparse, decode, st, &n_split);
+      if (e != cudaSuccess || n_split == 1) return e;
+      return launch_attn_combine(a, n_split, st);
+    }
+    case LC_IMPL_MMA:
+      return launch_attn_mma(a, sparse, decode, st);
+    default: {
+      const dim3 grid(a.n_q, (a.dims.H + 7) / 8);
+      k_attn_ref<<<grid, 256, 0, st>>>(a, sparse ? 1 : 0);
+      return cudaGetLastError();
+    }
+  }
 }
 
 }  // namespace lc

@@ -5,8 +5,10 @@
 // per-head sink; V = K = the entry).  The rows of a CTA are heads of ONE query, which all
 // share the same keys (MQA), so a key tile is gathered once and feeds every head:
 //
-//   * key tile: 64 keys gathered by index (entries: E4M3 nope + BF16 RoPE; window rows:
-//     BF16), widened to BF16 in shared memory (E4M3 -> BF16 is exact);
+//   * key tile: TK keys gathered by index with cp.async.  BF16 data (window rows, the
+//     RoPE part of entries) lands directly in the BF16 tile; the E4M3 nope part lands in
+//     a raw area and is widened to BF16 in a second pass (E4M3 -> BF16 is exact).  Decode
+//     double-buffers the tiles so the next tile's gather overlaps this tile's math;
 //   * S = Q K^T on BF16 mma.sync; the D = 576 contraction is split across DS warps and
 //     their partial sums are added in a fixed order through shared memory, so every warp
 //     of a row tile holds the same S;
@@ -14,18 +16,21 @@
 //   * O += P V with P from registers and V = the same key tile, each warp owning D/DS
 //     output dims.
 //
-// A CTA covers MT x 16 heads with MT * DS warps: prefill uses 64 heads (MT = 4, DS = 2),
-// decode 16 heads (MT = 1, DS = 4) so that a small batch still fills the GPU.  Decode
-// may split a query's keys across CTAs (n_split > 1): each writes its unnormalised O,
-// running max and sum to the workspace and k_attn_combine merges them with the sink in
-// a fixed order.  The split count depends only on the shapes, never on timing.
+// A CTA covers MT x 16 heads with MT * DS warps: prefill uses 64 heads (MT = 4, DS = 2,
+// 64-key tiles), decode 16 heads (MT = 1, DS = 4, 32-key tiles) so that a
+// small batch still fills the GPU.  Decode may split a query's keys across CTAs
+// (n_split > 1): each writes its unnormalised O, running max and sum to the workspace and
+// k_attn_combine merges them with the sink in a fixed order.  The split count depends
+// only on the shapes, never on timing.
 #include "lc_internal.h"
 
 namespace lc {
 
 constexpr int kAD = 576;          // head dim of this kernel
 constexpr int kRS = kAD + 8;      // padded shared row stride (elements): 1168 B, ldmatrix conflict-free
-constexpr int kTK = 64;           // keys per tile
+constexpr int kChunks = kAD / 8;  // 16-byte BF16 chunks per row
+constexpr int kRawRow = 512;      // bytes of E4M3 nope data staged per key (d_n <= 512)
+constexpr int kTileMax = 64;      // largest key tile
 constexpr uint32_t kWinFlag = 1u << 30;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -51,6 +56,16 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
+}
+__device__ __forceinline__ void cp8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(dst), "l"(src));
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return static_cast<uint32_t>(f32_to_bf16_bits(lo)) | (static_cast<uint32_t>(f32_to_bf16_bits(hi)) << 16);
 }
@@ -70,39 +85,26 @@ __device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 u) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// Row `r` of a row set (576 logical dims) widened to BF16 into shared memory; `nthr`
-// threads of index `sub` share the row, 8 dims (one 16-byte chunk) at a time.
-__device__ __forceinline__ void stage_row_bf16(const lc_rows& rs, int64_t r, int d_r, uint16_t* dst, int sub,
-                                               int nthr) {
-  const int d_n = kAD - d_r;
+// Issue the copies of chunk c (dims 8c .. 8c+7) of row r of a row set into BF16 row `dst`
+// (E4M3 nope chunks go to `raw` instead, to be widened later).
+__device__ __forceinline__ void gather_chunk(const lc_rows& rs, int64_t r, int d_r, int c, uint16_t* dst,
+                                             uint8_t* raw) {
   if (rs.fmt == LC_FMT_BF16) {
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(rs.x) + r * kAD);
-#pragma unroll 6
-    for (int c = sub; c < kAD / 8; c += nthr) reinterpret_cast<uint4*>(dst)[c] = __ldg(src + c);
+    cp16(smem_u32(dst + c * 8), static_cast<const uint16_t*>(rs.x) + r * kAD + c * 8);
   } else {
-    const uint2* nope = reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(rs.x) + r * d_n);
-    const uint4* rope = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(rs.rope) + r * d_r);
-#pragma unroll 6
-    for (int c = sub; c < kAD / 8; c += nthr) {
-      uint4 v;
-      if (c * 8 < d_n) v = e4m3x8_to_bf16x8(__ldg(nope + c));
-      else v = __ldg(rope + (c - d_n / 8));
-      reinterpret_cast<uint4*>(dst)[c] = v;
-    }
+    const int d_n = kAD - d_r;
+    if (c * 8 < d_n) cp8(smem_u32(raw + c * 8), static_cast<const uint8_t*>(rs.x) + r * d_n + c * 8);
+    else cp16(smem_u32(dst + c * 8), static_cast<const uint16_t*>(rs.rope) + r * d_r + (c * 8 - d_n));
   }
-}
-
-__device__ __forceinline__ void zero_row(uint16_t* dst, int sub, int nthr) {
-  for (int c = sub; c < kAD / 8; c += nthr) reinterpret_cast<uint4*>(dst)[c] = make_uint4(0, 0, 0, 0);
 }
 
 struct AttnGeom {
   int n_split;   // CTAs per (query, head group) along the keys
-  int sps;       // slots per split (multiple of kTK)
+  int sps;       // slots per split (multiple of the key tile)
 };
 
-// grid: (n_q, n_hg * n_split); MT * DS warps.
-template <int MT, int DS>
+// grid: (n_q, n_hg * n_split); MT * DS warps; TK keys per tile; NBUF tile buffers.
+template <int MT, int DS, int TK, int NBUF>
 __global__ void __launch_bounds__(MT * DS * 32, 1)
     k_attn_mma(lc_attn_args a, int sparse, AttnGeom geo, float* __restrict__ ws_o, float* __restrict__ ws_ml) {
   constexpr int NW = MT * DS;
@@ -111,17 +113,20 @@ __global__ void __launch_bounds__(MT * DS * 32, 1)
   constexpr int DW = kAD / DS;        // output dims per warp
   constexpr int KS = DW / 16;         // k16 steps of the partial S
   constexpr int NTO = DW / 8;         // n8 tiles of O per warp
+  constexpr int NTS = TK / 8;         // n8 tiles of S
+  constexpr int SPL = TK / 2;         // partial-S floats per lane
+  static_assert(DW % 16 == 0 && NTO % 2 == 0 && TK % 16 == 0 && TK <= kTileMax, "tile shape");
   extern __shared__ __align__(16) uint8_t smem[];
   uint16_t* Qs = reinterpret_cast<uint16_t*>(smem);                 // [ROWS][kRS]
-  uint16_t* Ks = Qs + ROWS * kRS;                                    // [kTK][kRS]
-  float* Sx = reinterpret_cast<float*>(Ks + kTK * kRS);              // [NW][32][32]
-  int* kval = reinterpret_cast<int*>(Sx + NW * 32 * 32);             // [kTK] key valid
+  uint16_t* Ks = Qs + ROWS * kRS;                                    // [NBUF][TK][kRS]
+  uint8_t* Raw = reinterpret_cast<uint8_t*>(Ks + NBUF * TK * kRS);   // [NBUF][TK][kRawRow]
+  float* Sx = reinterpret_cast<float*>(Raw + NBUF * TK * kRawRow);   // [NW][SPL][32]
+  int* kcode = reinterpret_cast<int*>(Sx + NW * SPL * 32);           // [NBUF][TK]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int mt = warp / DS, ds = warp % DS;
   const int g = lane >> 2, t4 = lane & 3;
   const int q = blockIdx.x;
-  const int n_hg = gridDim.y / geo.n_split;
   const int hg = blockIdx.y / geo.n_split, split = blockIdx.y % geo.n_split;
   const int H = a.dims.H, d_r = a.dims.d_r;
   const int b = seq_of_query(a.batch.q_start, a.batch.num_seqs, q);
@@ -139,15 +144,84 @@ __global__ void __launch_bounds__(MT * DS * 32, 1)
   const int wl = a.W > 0 ? __ldg(a.batch.win_len + b) : 0;
   const int64_t wr0 = a.W > 0 ? __ldg(a.batch.win_start + b) : 0;
   const int32_t* idx_row = sparse ? a.idx + static_cast<int64_t>(q) * a.k : nullptr;
-  (void)n_hg;
+  const int n_tiles = s_end > s_begin ? (s_end - s_begin + TK - 1) / TK : 0;
 
-  // queries of this head group, widened to BF16
+  // slot -> key code: entry index j, kWinFlag | window row, or -1 (masked)
+  auto slot_code = [&](int s) -> int {
+    if (s >= s_end) return -1;
+    if (s < n_first) {
+      const int j = sparse ? __ldg(idx_row + s) : s;
+      if (j < 0) return -1;
+      if (j >= n_ent) {
+        set_status(a.status, LC_DEV_BAD_INDEX);
+        return -1;
+      }
+      if (j >= nv) {
+        set_status(a.status, LC_DEV_NONVISIBLE);
+        return -1;
+      }
+      return j;
+    }
+    const int rr = wlo + (s - n_first) - wp0;
+    if (rr < 0 || rr >= wl) {
+      set_status(a.status, LC_DEV_WINDOW_RANGE);
+      return -1;
+    }
+    return static_cast<int>(kWinFlag) | rr;
+  };
+  // codes of tile t into kcode[buf] (call, then __syncthreads, then issue)
+  auto tile_codes = [&](int t, int buf) {
+    if (tid < TK) kcode[buf * TK + tid] = slot_code(s_begin + t * TK + tid);
+  };
+  // cp.async gather of tile t into buffer buf (codes already in kcode[buf])
+  auto tile_issue = [&](int buf) {
+    uint16_t* kb = Ks + buf * TK * kRS;
+    uint8_t* rb = Raw + buf * TK * kRawRow;
+    for (int u = tid; u < TK * kChunks; u += NTHR) {
+      const int kr = u / kChunks, c = u % kChunks;
+      const int code = kcode[buf * TK + kr];
+      uint16_t* dst = kb + kr * kRS;
+      if (code < 0) reinterpret_cast<uint4*>(dst)[c] = make_uint4(0, 0, 0, 0);
+      else if (code & kWinFlag) gather_chunk(a.win, wr0 + (code & ~kWinFlag), d_r, c, dst, rb + kr * kRawRow);
+      else gather_chunk(a.ent, ent0 + code, d_r, c, dst, rb + kr * kRawRow);
+    }
+  };
+  // widen the E4M3 nope part of buffer buf (after its copies landed)
+  auto tile_widen = [&](int buf) {
+    if (a.ent.fmt != LC_FMT_E4M3_BF16) return;
+    const int dnc = (kAD - d_r) / 8;
+    uint16_t* kb = Ks + buf * TK * kRS;
+    const uint8_t* rb = Raw + buf * TK * kRawRow;
+    for (int u = tid; u < TK * dnc; u += NTHR) {
+      const int kr = u / dnc, c = u % dnc;
+      const int code = kcode[buf * TK + kr];
+      if (code >= 0 && !(code & kWinFlag))
+        reinterpret_cast<uint4*>(kb + kr * kRS)[c] =
+            e4m3x8_to_bf16x8(*reinterpret_cast<const uint2*>(rb + kr * kRawRow + c * 8));
+    }
+  };
+
+  // queries of this head group (cp.async into Qs, E4M3 nope through Raw buffer 0)
   {
-    constexpr int TPR = NTHR / ROWS;  // threads per row
-    const int r = tid / TPR, sub = tid % TPR;
-    const int h = hg * ROWS + r;
-    if (h < H) stage_row_bf16(a.q, static_cast<int64_t>(q) * H + h, d_r, Qs + r * kRS, sub, TPR);
-    else zero_row(Qs + r * kRS, sub, TPR);
+    for (int u = tid; u < ROWS * kChunks; u += NTHR) {
+      const int r = u / kChunks, c = u % kChunks;
+      const int h = hg * ROWS + r;
+      uint16_t* dst = Qs + r * kRS;
+      if (h < H) gather_chunk(a.q, static_cast<int64_t>(q) * H + h, d_r, c, dst, Raw + r * kRawRow);
+      else reinterpret_cast<uint4*>(dst)[c] = make_uint4(0, 0, 0, 0);
+    }
+    cp_commit();
+    cp_wait<0>();
+    __syncthreads();
+    if (a.q.fmt == LC_FMT_E4M3_BF16) {
+      const int dnc = (kAD - d_r) / 8;
+      for (int u = tid; u < ROWS * dnc; u += NTHR) {
+        const int r = u / dnc, c = u % dnc;
+        if (hg * ROWS + r < H)
+          reinterpret_cast<uint4*>(Qs + r * kRS)[c] = e4m3x8_to_bf16x8(*reinterpret_cast<const uint2*>(Raw + r * kRawRow + c * 8));
+      }
+    }
+    __syncthreads();  // Raw buffer 0 is free again
   }
 
   float o[NTO][4];
@@ -157,54 +231,45 @@ __global__ void __launch_bounds__(MT * DS * 32, 1)
   float l_run[2] = {0.f, 0.f};
   const float sl2 = a.scale * 1.4426950408889634f;  // logits in log2 units
 
-  for (int s0 = s_begin; s0 < s_end; s0 += kTK) {
-    __syncthreads();  // previous tile fully consumed
-    {
-      constexpr int TPK = NTHR / kTK;
-      const int kr = tid / TPK, sub = tid % TPK;
-      const int s = s0 + kr;
-      int code = -1;
-      if (s < s_end) {
-        if (s < n_first) {
-          const int j = sparse ? __ldg(idx_row + s) : s;
-          if (j >= 0) {
-            if (j >= n_ent) {
-              if (sub == 0) set_status(a.status, LC_DEV_BAD_INDEX);
-            } else if (j >= nv) {
-              if (sub == 0) set_status(a.status, LC_DEV_NONVISIBLE);
-            } else {
-              code = j;
-            }
-          }
-        } else {
-          const int rr = wlo + (s - n_first) - wp0;
-          if (rr < 0 || rr >= wl) {
-            if (sub == 0) set_status(a.status, LC_DEV_WINDOW_RANGE);
-          } else {
-            code = static_cast<int>(kWinFlag) | rr;
-          }
-        }
+  if (n_tiles > 0) {
+    tile_codes(0, 0);
+    __syncthreads();
+    tile_issue(0);
+    cp_commit();
+  }
+  for (int t = 0; t < n_tiles; ++t) {
+    const int buf = NBUF == 2 ? (t & 1) : 0;
+    if (NBUF == 2) {
+      // prefetch tile t + 1 into the other buffer (its last reader finished at the end
+      // of the previous iteration)
+      if (t + 1 < n_tiles) {
+        tile_codes(t + 1, buf ^ 1);
+        __syncthreads();
+        tile_issue(buf ^ 1);
       }
-      uint16_t* dst = Ks + kr * kRS;
-      if (code < 0) zero_row(dst, sub, TPK);
-      else if (code & kWinFlag) stage_row_bf16(a.win, wr0 + (code & ~kWinFlag), d_r, dst, sub, TPK);
-      else stage_row_bf16(a.ent, ent0 + code, d_r, dst, sub, TPK);
-      if (sub == 0) kval[kr] = code >= 0;
+      cp_commit();
+      cp_wait<1>();
+    } else {
+      cp_wait<0>();
     }
     __syncthreads();
+    tile_widen(buf);
+    __syncthreads();
+    const uint16_t* Kb = Ks + buf * TK * kRS;
+    const int* kv = kcode + buf * TK;
 
-    // partial S over this warp's dims: 16 rows x 64 keys
-    float sacc[8][4];
+    // partial S over this warp's dims: 16 rows x TK keys
+    float sacc[NTS][4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.f;
+    for (int i = 0; i < NTS; ++i) sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.f;
     const uint32_t qa = smem_u32(Qs + (mt * 16 + (lane & 15)) * kRS + ds * DW + (lane >> 4) * 8);
-    const uint32_t kb = smem_u32(Ks + ((lane >> 4) * 8 + (lane & 7)) * kRS + ds * DW + ((lane >> 3) & 1) * 8);
+    const uint32_t kb = smem_u32(Kb + ((lane >> 4) * 8 + (lane & 7)) * kRS + ds * DW + ((lane >> 3) & 1) * 8);
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
       uint32_t a0, a1, a2, a3;
       ldsm_x4(qa + ks * 32, a0, a1, a2, a3);
 #pragma unroll
-      for (int np = 0; np < 4; ++np) {
+      for (int np = 0; np < NTS / 2; ++np) {
         uint32_t b0, b1, b2, b3;
         ldsm_x4(kb + np * 16 * kRS * 2 + ks * 32, b0, b1, b2, b3);
         mma_bf16(sacc[2 * np], a0, a1, a2, a3, b0, b1);
@@ -212,26 +277,26 @@ __global__ void __launch_bounds__(MT * DS * 32, 1)
       }
     }
     // add the DS partial sums in a fixed order (every warp of the row tile gets the same S)
-    float* mine = Sx + warp * 1024;
+    float* mine = Sx + warp * SPL * 32;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < NTS; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) mine[(i * 4 + j) * 32 + lane] = sacc[i][j];
     __syncthreads();
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < NTS; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        float v = Sx[(mt * DS + 0) * 1024 + (i * 4 + j) * 32 + lane];
+        float v = Sx[(mt * DS + 0) * SPL * 32 + (i * 4 + j) * 32 + lane];
 #pragma unroll
-        for (int d = 1; d < DS; ++d) v += Sx[(mt * DS + d) * 1024 + (i * 4 + j) * 32 + lane];
+        for (int d = 1; d < DS; ++d) v += Sx[(mt * DS + d) * SPL * 32 + (i * 4 + j) * 32 + lane];
         sacc[i][j] = v;
       }
     // online softmax (log2 units); masked keys get -inf
     float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const bool v0 = kval[i * 8 + 2 * t4], v1 = kval[i * 8 + 2 * t4 + 1];
+    for (int i = 0; i < NTS; ++i) {
+      const bool v0 = kv[i * 8 + 2 * t4] >= 0, v1 = kv[i * 8 + 2 * t4 + 1] >= 0;
       sacc[i][0] = v0 ? sacc[i][0] * sl2 : -INFINITY;
       sacc[i][1] = v1 ? sacc[i][1] * sl2 : -INFINITY;
       sacc[i][2] = v0 ? sacc[i][2] * sl2 : -INFINITY;
@@ -254,7 +319,7 @@ __global__ void __launch_bounds__(MT * DS * 32, 1)
     }
     float rs[2] = {0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < NTS; ++i) {
       sacc[i][0] = exp2f(sacc[i][0] - mref[0]);
       sacc[i][1] = exp2f(sacc[i][1] - mref[0]);
       sacc[i][2] = exp2f(sacc[i][2] - mref[1]);
@@ -271,14 +336,15 @@ __global__ void __launch_bounds__(MT * DS * 32, 1)
       o[i][2] *= corr[1];
       o[i][3] *= corr[1];
     }
-    // O += P V over the 64 keys (4 k16 steps), this warp's dims
+    // O += P V over the TK keys, this warp's dims
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
+    for (int kk = 0; kk < TK / 16; ++kk) {
       const uint32_t pa0 = pack_bf16(sacc[2 * kk][0], sacc[2 * kk][1]);
       const uint32_t pa1 = pack_bf16(sacc[2 * kk][2], sacc[2 * kk][3]);
       const uint32_t pa2 = pack_bf16(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1]);
       const uint32_t pa3 = pack_bf16(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3]);
-      const uint32_t vb = smem_u32(Ks + (kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7)) * kRS + ds * DW + (lane >> 4) * 8);
+      const uint32_t vb =
+          smem_u32(Kb + (kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7)) * kRS + ds * DW + (lane >> 4) * 8);
 #pragma unroll
       for (int np = 0; np < NTO / 2; ++np) {
         uint32_t b0, b1, b2, b3;
@@ -286,6 +352,13 @@ __global__ void __launch_bounds__(MT * DS * 32, 1)
         mma_bf16(o[2 * np], pa0, pa1, pa2, pa3, b0, b1);
         mma_bf16(o[2 * np + 1], pa0, pa1, pa2, pa3, b2, b3);
       }
+    }
+    __syncthreads();  // this tile's buffers and Sx are free
+    if (NBUF == 1 && t + 1 < n_tiles) {
+      tile_codes(t + 1, 0);
+      __syncthreads();
+      tile_issue(0);
+      cp_commit();
     }
   }
 
@@ -376,8 +449,11 @@ __global__ void __launch_bounds__(256) k_attn_combine(lc_attn_args a, int n_spli
 // ---------------------------------------------------------------------------------
 // launch configuration
 // ---------------------------------------------------------------------------------
+constexpr int kTkPrefill = 64;
+constexpr int kTkDecode = 32;
+
 bool attn_mma_supported(const lc_attn_args& a) {
-  if (a.dims.D != kAD || a.dims.d_r % 8 || a.dims.H % 16) return false;
+  if (a.dims.D != kAD || a.dims.d_r % 8 || a.dims.d_r < 64 || a.dims.H % 16) return false;
   auto ok_rows = [&](const lc_rows& r) {
     return r.fmt == LC_FMT_BF16 || (r.fmt == LC_FMT_E4M3_BF16 && a.dims.d_r > 0);
   };
@@ -391,20 +467,21 @@ static int max_slots(const lc_attn_args& a, bool sparse) {
 
 AttnGeom attn_geometry(const lc_attn_args& a, bool sparse, bool decode) {
   AttnGeom g{1, 0};
+  const int tk = decode ? kTkDecode : kTkPrefill;
   const int ns = max(max_slots(a, sparse), 1);
-  const int tiles = (ns + kTK - 1) / kTK;
+  const int tiles = (ns + tk - 1) / tk;
   if (decode) {
-    // fill ~2 CTAs per SM, but keep >= 4 key tiles (256 keys) per split so that the
+    // fill ~2 CTAs per SM, but keep >= 8 key tiles (256 keys) per split so that the
     // partial results a split writes stay small next to the keys it reads
     const int ctas = a.n_q * (a.dims.H / 16);
     const int want = (2 * 148 + ctas - 1) / max(ctas, 1);
-    int n = min(want, max(1, tiles / 4));
+    int n = min(want, max(1, tiles / 8));
     n = max(1, min(n, tiles));
     const int per = (tiles + n - 1) / n;
     g.n_split = (tiles + per - 1) / per;
-    g.sps = per * kTK;
+    g.sps = per * tk;
   } else {
-    g.sps = tiles * kTK;
+    g.sps = tiles * tk;
   }
   return g;
 }
@@ -416,11 +493,13 @@ size_t attn_mma_workspace(const lc_attn_args& a, bool sparse, bool decode) {
   return rows * kAD * sizeof(float) + rows * 2 * sizeof(float);
 }
 
-template <int MT, int DS>
+template <int MT, int DS, int TK, int NBUF>
 static cudaError_t launch_mma(const lc_attn_args& a, bool sparse, const AttnGeom& g, cudaStream_t st) {
   constexpr int ROWS = MT * 16;
-  const size_t sm = (ROWS + kTK) * kRS * 2 + MT * DS * 32 * 32 * 4 + kTK * 4;
-  cudaFuncSetAttribute(k_attn_mma<MT, DS>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
+  const size_t sm = static_cast<size_t>(ROWS + NBUF * TK) * kRS * 2 + static_cast<size_t>(NBUF) * TK * kRawRow +
+                    static_cast<size_t>(MT * DS) * (TK / 2) * 32 * 4 + NBUF * TK * 4;
+  cudaFuncSetAttribute(k_attn_mma<MT, DS, TK, NBUF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(sm));
   const int n_hg = (a.dims.H + ROWS - 1) / ROWS;
   float* ws_o = static_cast<float*>(a.workspace);
   float* ws_ml = nullptr;
@@ -429,7 +508,7 @@ static cudaError_t launch_mma(const lc_attn_args& a, bool sparse, const AttnGeom
     ws_ml = ws_o + rows * kAD;
   }
   const dim3 grid(a.n_q, n_hg * g.n_split);
-  k_attn_mma<MT, DS><<<grid, MT * DS * 32, sm, st>>>(a, sparse ? 1 : 0, g, ws_o, ws_ml);
+  k_attn_mma<MT, DS, TK, NBUF><<<grid, MT * DS * 32, sm, st>>>(a, sparse ? 1 : 0, g, ws_o, ws_ml);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || g.n_split == 1) return e;
   const int64_t rows = static_cast<int64_t>(a.n_q) * a.dims.H;
@@ -437,10 +516,22 @@ static cudaError_t launch_mma(const lc_attn_args& a, bool sparse, const AttnGeom
   return cudaGetLastError();
 }
 
+// Merge step for the key splits of the tensor-core kernel (workspace: partial O, then
+// (max, sum) pairs).
+cudaError_t launch_attn_combine(const lc_attn_args& a, int n_split, cudaStream_t st) {
+  float* ws_o = static_cast<float*>(a.workspace);
+  float* ws_ml = ws_o + static_cast<size_t>(a.n_q) * a.dims.H * n_split * kAD;
+  const int64_t rows = static_cast<int64_t>(a.n_q) * a.dims.H;
+  k_attn_combine<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(a, n_split, ws_o, ws_ml);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attn_mma(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st) {
   const AttnGeom g = attn_geometry(a, sparse, decode);
-  if (decode || a.dims.H % 64) return launch_mma<1, 4>(a, sparse, g, st);
-  return launch_mma<4, 2>(a, sparse, g, st);
+  // decode: one buffer of 32 keys keeps the CTA at 80 KB of shared memory, two per SM
+  if (decode) return launch_mma<1, 4, kTkDecode, 1>(a, sparse, g, st);
+  if (a.dims.H % 64) return launch_mma<1, 4, kTkPrefill, 1>(a, sparse, g, st);
+  return launch_mma<4, 2, kTkPrefill, 1>(a, sparse, g, st);
 }
 
 }  // namespace lc

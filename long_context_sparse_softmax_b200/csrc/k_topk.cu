@@ -45,7 +45,29 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
   const float* row = a.scores + static_cast<int64_t>(q) * a.score_stride;
   const bool cached = use_cache && n <= kRowCache;
   if (cached) {
-    for (int i = tid; i < n; i += kTopkThreads) cache[i] = order_key(__ldg(row + i));
+    // 16-byte loads, four in flight per thread (rows start 16-byte aligned: the score
+    // stride is a multiple of 4 floats)
+    const int n4 = n >> 2;
+    const float4* r4 = reinterpret_cast<const float4*>(row);
+    for (int base = 0; base < n4; base += 4 * kTopkThreads) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i4 = base + u * kTopkThreads + tid;
+        if (i4 < n4) v[u] = __ldg(r4 + i4);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i4 = base + u * kTopkThreads + tid;
+        if (i4 < n4) {
+          cache[4 * i4 + 0] = order_key(v[u].x);
+          cache[4 * i4 + 1] = order_key(v[u].y);
+          cache[4 * i4 + 2] = order_key(v[u].z);
+          cache[4 * i4 + 3] = order_key(v[u].w);
+        }
+      }
+    }
+    for (int i = 4 * n4 + tid; i < n; i += kTopkThreads) cache[i] = order_key(__ldg(row + i));
   }
   uint32_t prefix = 0, mask = 0;
   int remaining = K;

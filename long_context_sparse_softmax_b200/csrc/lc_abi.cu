@@ -98,11 +98,12 @@ lc_status index_scores(const lc_index_args* a, void* stream, bool decode) {
 lc_status topk(const lc_topk_args* a, void* stream, bool decode) {
   if (!a) return LC_ERR_ARG;
   if (a->n_q < 0 || a->k < 1 || a->max_ent < 0 || a->m < 1 || a->W_x < 0) return LC_ERR_ARG;
-  if (a->score_stride < a->max_ent) return LC_ERR_ARG;
+  if (a->score_stride < a->max_ent || a->score_stride % 4) return LC_ERR_ARG;
   if (decode && a->n_q != a->batch.num_seqs) return LC_ERR_ARG;
   if (a->n_q == 0) return LC_OK;
   LC_TRY(check_batch(a->batch, true, false));
   if (!a->scores || !a->idx) return LC_ERR_ARG;
+  if (!aligned16(a->scores)) return LC_ERR_ALIGN;
   return launched(lc::launch_topk(*a, decode, static_cast<cudaStream_t>(stream)));
 }
 
@@ -113,6 +114,8 @@ lc_status attn(const lc_attn_args* a, void* stream, bool sparse, bool decode) {
   if (a->out_fmt != LC_FMT_F32 && a->out_fmt != LC_FMT_BF16) return LC_ERR_ARG;
   if (sparse && a->k < 1) return LC_ERR_ARG;
   if (decode && a->n_q != a->batch.num_seqs) return LC_ERR_ARG;
+  if (a->impl < LC_IMPL_AUTO || a->impl > LC_IMPL_REF) return LC_ERR_ARG;
+  if (!lc::attn_impl_ok(*a)) return LC_ERR_UNSUPPORTED;
   if (a->n_q == 0) return LC_OK;
   LC_TRY(check_rows(a->q, a->dims, true));
   LC_TRY(check_rows(a->ent, a->dims, a->max_ent > 0));

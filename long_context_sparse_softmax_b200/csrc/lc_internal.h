@@ -17,6 +17,12 @@ bool attn_mma_supported(const lc_attn_args& a);
 size_t attn_mma_workspace(const lc_attn_args& a, bool sparse, bool decode);
 cudaError_t launch_attn_mma(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st);
 bool index_tc_supported(const lc_index_args& a);
+bool attn_tc_supported(const lc_attn_args& a);
+int attn_impl(const lc_attn_args& a);
+bool attn_impl_ok(const lc_attn_args& a);
+size_t attn_tc_workspace(const lc_attn_args& a, bool sparse, bool decode);
+cudaError_t launch_attn_tc(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st, int* n_split);
+cudaError_t launch_attn_combine(const lc_attn_args& a, int n_split, cudaStream_t st);
 cudaError_t launch_index_tc(const lc_index_args& a, bool decode, cudaStream_t st);
 
 // Sequence of query row q: the b with q_start[b] <= q < q_start[b+1] (binary search).

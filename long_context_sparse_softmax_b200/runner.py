@@ -54,6 +54,34 @@ def _round4(n: int) -> int:
 
 
 class _Common:
+    def dag(self):
+        """The step as three groups: (side, main, after).  `side` (query and window
+        preparation, compression) and `main` (index scores -> top-k) share no buffers and
+        may run concurrently on two streams; `after` (attention) needs both."""
+        st = dict(self.stages())
+        side = [(n, st[n]) for n in ("qk_prep_q", "qk_prep_win", "compress") if n in st]
+        main = [(n, st[n]) for n in ("index", "topk") if n in st]
+        return side, main, [("attn", st["attn"])]
+
+    def step_overlapped(self, main, side, on_stage=None):
+        """One step on two streams: fork `side` from `main`, join before attention.
+        on_stage(name, stream, fn) may wrap each launch (e.g. with timing events)."""
+        import torch
+        sd, mn, af = self.dag()
+        run = on_stage or (lambda name, stream, fn: fn(stream))
+        fork = torch.cuda.Event()
+        fork.record(main)
+        side.wait_event(fork)
+        for n, f in sd:
+            run(n, side, f)
+        for n, f in mn:
+            run(n, main, f)
+        join = torch.cuda.Event()
+        join.record(side)
+        main.wait_event(join)
+        for n, f in af:
+            run(n, main, f)
+
     def _index_args(self, n_q: int, max_ent: int, scores: torch.Tensor) -> IndexArgs:
         s, inp = self.spec, self.inp
         qI, kI = inp["qI"], inp["kI"]
@@ -85,6 +113,7 @@ class _Common:
         a.out = ptr(self.out)
         a.lse = ptr(self.lse)
         a.status = ptr(self.status)
+        a.impl = self.impl
         ws = (lc_csa_sparse_attn_workspace_bytes if sparse else lc_hca_attn_workspace_bytes)(a)
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.device)
         a.workspace, a.workspace_bytes = ptr(self.workspace), ws
@@ -97,8 +126,9 @@ class _Common:
 class Prefill(_Common):
     """One sequence of L raw tokens; queries at q_first .. q_first + n_q - 1."""
 
-    def __init__(self, inp: Dict[str, object], device="cuda", W_x: Optional[int] = None):
+    def __init__(self, inp: Dict[str, object], device="cuda", W_x: Optional[int] = None, impl: int = 0):
         s: wl.Spec = inp["spec"]
+        self.impl = impl
         self.spec, self.inp, self.device = s, inp, device
         self.W_x = s.W if W_x is None else W_x
         L, n_c = inp["L"], inp["n_c"]
@@ -169,8 +199,9 @@ class Prefill(_Common):
 class Decode(_Common):
     """B sequences, one query each at L_b - 1, on an existing cache (see workloads.make_decode)."""
 
-    def __init__(self, inp: Dict[str, object], device="cuda", W_x: Optional[int] = None):
+    def __init__(self, inp: Dict[str, object], device="cuda", W_x: Optional[int] = None, impl: int = 0):
         s: wl.Spec = inp["spec"]
+        self.impl = impl
         self.spec, self.inp, self.device = s, inp, device
         self.W_x = s.W if W_x is None else W_x
         B = s.num_seqs

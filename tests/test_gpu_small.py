@@ -73,3 +73,32 @@ def test_small_hca_decode_ragged():
 def test_small_csa_decode_overlap_reading():
     s = wl.shrink(wl.CSA_DECODE, name="small_csa_decode_ov", seed=40, seq_lens=(900, 1204), k=64)
     check_decode(s, W_x=0)
+
+
+# every attention kernel on the same shapes (the tests above use the automatic choice)
+IMPLS = [pytest.param(1, id="mma"), pytest.param(2, id="tcgen05"), pytest.param(3, id="reference")]
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_small_csa_prefill_each_attention_kernel(impl):
+    s = wl.shrink(wl.CSA_PREFILL, name="small_csa_impl", seed=41, seq_lens=(700,), H=64, k=96, n_q=700)
+    check_prefill(s, q_sel=range(0, 700, 3), impl=impl)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_small_hca_prefill_each_attention_kernel(impl):
+    s = wl.shrink(wl.HCA_PREFILL, name="small_hca_impl", seed=42, seq_lens=(128 * 24 + 50,),
+                  q_first=128 * 24 + 50 - 160, n_q=160)
+    check_prefill(s, impl=impl)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_small_csa_decode_each_attention_kernel(impl):
+    s = wl.shrink(wl.CSA_DECODE, name="small_decode_impl", seed=43, seq_lens=(3000, 1027, 8192, 200), k=256)
+    check_decode(s, impl=impl)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_small_hca_decode_each_attention_kernel(impl):
+    s = wl.shrink(wl.MIXED_HCA, name="small_hcad_impl", seed=44, seq_lens=(128 * 40 + 3, 900, 128 * 7))
+    check_decode(s, impl=impl)
