@@ -135,8 +135,12 @@ __global__ void __launch_bounds__(256) k_attn_ref(lc_attn_args a, int sparse) {
 // The kernel a call runs (never LC_IMPL_AUTO): AUTO takes the fastest one measured for
 // 576-dim BF16 / E4M3 shapes, the BF16 mma.sync kernel; other shapes (FP32, other head
 // dims) run on the reference kernel.
+// The automatic choice: the tcgen05 kernel where it applies (576-dim rows with 64 RoPE
+// dims, 64-head groups, 16-byte aligned buffers), else the mma.sync kernel, else the
+// reference kernel.
 int attn_impl(const lc_attn_args& a) {
   if (a.impl != LC_IMPL_AUTO) return a.impl;
+  if (attn_tc_supported(a)) return LC_IMPL_TC;
   return attn_mma_supported(a) ? LC_IMPL_MMA : LC_IMPL_REF;
 }
 
@@ -150,6 +154,15 @@ bool attn_impl_ok(const lc_attn_args& a) {
 }
 
 size_t attn_workspace_bytes(const lc_attn_args& a, bool sparse, bool decode) {
+  if (a.impl == LC_IMPL_AUTO) {
+    // the choice may depend on buffer alignment, which the caller may not have fixed yet
+    size_t w = attn_mma_supported(a) ? attn_mma_workspace(a, sparse, decode) : 0;
+    lc_attn_args t = a;
+    t.out = nullptr;
+    t.workspace = nullptr;
+    if (attn_tc_supported(t)) w = w > attn_tc_workspace(a, sparse, decode) ? w : attn_tc_workspace(a, sparse, decode);
+    return w;
+  }
   switch (attn_impl(a)) {
     case LC_IMPL_MMA: return attn_mma_supported(a) ? attn_mma_workspace(a, sparse, decode) : 0;
     case LC_IMPL_TC: return attn_tc_supported(a) ? attn_tc_workspace(a, sparse, decode) : 0;

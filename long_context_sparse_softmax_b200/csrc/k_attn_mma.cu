@@ -398,7 +398,8 @@ __global__ void __launch_bounds__(MT * DS * 32, 1)
       const int h = hr0 + 8 * r;
       if (h >= H) continue;
       const int64_t slot = (static_cast<int64_t>(q) * H + h) * geo.n_split + split;
-      float2* op = reinterpret_cast<float2*>(ws_o + slot * kAD + ds * DW + 2 * t4);
+      const int64_t orow = static_cast<int64_t>(split) * a.n_q * H + static_cast<int64_t>(q) * H + h;
+      float2* op = reinterpret_cast<float2*>(ws_o + orow * kAD + ds * DW + 2 * t4);
 #pragma unroll
       for (int i = 0; i < NTO; ++i) op[i * 4] = make_float2(o[i][2 * r], o[i][2 * r + 1]);
       if (ds == 0 && t4 == 0) {
@@ -409,7 +410,9 @@ __global__ void __launch_bounds__(MT * DS * 32, 1)
   }
 }
 
-// Merge the key splits of each (query, head) with the sink, in split order.
+// Merge the key splits of each (query, head) with the sink, in split order.  Split c of
+// row (q * H + h) left its unnormalised O at ws_o row c * n_q * H + q * H + h and its
+// (max, sum) at ws_ml[2 ((q * H + h) * n_split + c)].
 // grid: ceil(n_q * H / 8); one warp per (query, head).
 __global__ void __launch_bounds__(256) k_attn_combine(lc_attn_args a, int n_split, const float* __restrict__ ws_o,
                                                       const float* __restrict__ ws_ml) {
@@ -429,7 +432,7 @@ __global__ void __launch_bounds__(256) k_attn_combine(lc_attn_args a, int n_spli
     if (mc == -INFINITY) continue;
     const float w = exp2f(mc - M);
     Z = fmaf(__ldg(ws_ml + 2 * (row * n_split + c) + 1), w, Z);
-    const float* src = ws_o + (row * n_split + c) * kAD;
+    const float* src = ws_o + (static_cast<int64_t>(c) * a.n_q * a.dims.H + row) * kAD;
 #pragma unroll
     for (int i = 0; i < kAD / 32; ++i) o[i] = fmaf(__ldg(src + i * 32 + lane), w, o[i]);
   }

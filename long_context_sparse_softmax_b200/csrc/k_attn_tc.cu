@@ -2,32 +2,36 @@
 //
 // Same mathematics as k_attn.cu ("解读 DeepSeek V4": CSA attends to its top-k compressed
 // entries, HCA to all of them, both plus a 128-token window and a per-head sink; V = K =
-// the 576-dim entry; "DeepSeek-V4 论文分析" §5.4, §六, §七).  The rows of a CTA are NR heads
-// of one query, which share every key (MQA).
+// the 576-dim entry; "DeepSeek-V4 论文分析" §5.4, §六, §七).  A CTA holds 64 heads of one
+// query (they share every key: MQA) and a contiguous range of that query's key slots.
 //
 // Tiles and tensor memory:
-//   * key tile: 32 keys gathered by index with cp.async (BF16 parts straight into the tile,
-//     E4M3 nope parts into a raw area widened to BF16 - exact), laid out as 8 x 8 core
-//     matrices: key group g, dim chunk c at g * KG + c * 128.  The same bytes are the
-//     K-major B operand of S = Q K^T and the MN-major A operand V^T of O^T = V^T P^T;
-//   * S = Q K^T: M = 64 rows (a query's heads; rows past NR are ignored), N = 32, K = 576,
-//     in tensor memory (M = 64 layout: row r in lane 32 (r / 16) + r % 16), two buffers;
-//   * P = exp(scale * S): the method normalises queries and entries (RMSNorm), so
-//     |scale <q, k>| <= |q| |k| / sqrt(D) = sqrt(D) = 24 and the exponent needs no running
-//     maximum; a logit above 80 (exp would leave the FP32 range) is reported as
-//     LC_DEV_RANGE.  Masked keys get P = 0.  P goes to shared memory (two buffers) as the
-//     K-major B operand of the next MMA;
-//   * O^T = V^T P^T accumulates in tensor memory, dims on lanes: 5 chunks of 128 dims x NR
-//     columns.  Dim 576 of every key is 1, so O^T[576][row] is the row's sum of P.
-// The sink joins at the end: Z = e^sink + sum P, o = O / Z, lse = ln Z.  Decode may split
-// the keys of a query across CTAs; the splits then go through k_attn_combine.
+//   * 64-row tiles (the queries' heads, or 64 keys) in shared memory as a grid of 8 x 8
+//     BF16 core matrices, row group g and dim chunk c at g * 9216 + c * 128.  The same key
+//     bytes are the K-major B operand of S = Q K^T and the MN-major A operand V^T of
+//     O^T = V^T P^T.  Rows arrive by cp.async: BF16 parts straight into their chunk slots,
+//     the E4M3 nope part (16 dims = 16 bytes per piece) raw into the slot of the piece's
+//     second chunk, then widened to BF16 in place (exact: E4M3 has 4 significant bits);
+//   * S = Q K^T: M = 64 heads, N = 64 keys, K = 576, two tensor-memory buffers (M = 64
+//     layout: row r in lane 32 (r / 16) + r % 16; the 16x32bx2 load gives lanes 0-15 of a
+//     warp columns 0-31 and lanes 16-31 columns 32-63 of the same rows);
+//   * P = 2^(x - m_h), x = scale * log2(e) * S, with a per-head reference m_h that moves up
+//     only when a tile's maximum exceeds it by more than 8; O^T is then rescaled in tensor
+//     memory (rare after the first tile: P stays below 2^8).  Masked keys get P = 0.  The
+//     row sums add up the BF16-rounded P that the MMA multiplies;
+//   * O^T = V^T P^T accumulates in tensor memory, dims on lanes: chunks of 128 dims
+//     (M = 128) and a last chunk of 64 (M = 64), 64 head columns each.
+// The sink joins at the end: M = max(sink, m), Z = e^(sink - M) + l e^(m - M),
+// o = O e^(m - M) / Z, lse = M + ln Z.  The output block of a CTA (64 consecutive rows)
+// is staged in the freed key stages and written by one bulk copy.  A query's keys may be
+// split across CTAs; each split then writes (O, m, l) and k_attn_combine merges them.
 //
-// Warp roles (288 threads): warps 0-3 turn S into P and write the output (each reaches its
-// own quarter of the tensor-memory lanes); warps 4-7 gather and widen key tiles into a
-// two-stage ring; lane 0 of warp 8 issues the MMAs, S of tile t + 1 ahead of O of tile t
-// so that the tensor core works while P is formed.  The roles meet only at mbarriers, and
-// every wait is bounded: a role that gives up sets LC_DEV_TIMEOUT and an abort flag that
-// stops the others at their next wait.
+// Warp roles (288 threads): warps 0-3 load Q, turn S into P and write the output (each
+// reaches its own quarter of the tensor-memory lanes); warps 4-7 gather key tiles into a
+// two-stage ring; lane 0 of warp 8 issues the MMAs, whichever of S(t + 1) and O(t) is
+// ready first.  The roles meet only at mbarriers and named barriers, and every mbarrier
+// wait is bounded: a role that gives up sets LC_DEV_TIMEOUT and an abort flag that stops
+// the others at their next wait.
 #include "lc_internal.h"
 
 namespace lc {
@@ -35,16 +39,26 @@ namespace lc {
 namespace {
 
 constexpr int kD = 576;
-constexpr int kTK = 32;                      // keys per tile
-constexpr int kDC = 73;                      // dim chunks per key group: 72 + the ones chunk
-constexpr int kKG = kDC * 128;               // bytes per key group of 8
-constexpr int kKTile = (kTK / 8) * kKG;      // bytes per key tile (37,376)
-constexpr int kQG = 72 * 128;                // bytes per row group of 8 (Q)
-constexpr int kRaw = 512;                    // raw E4M3 bytes per key
-constexpr int kStages = 2;
+constexpr int kDR = 64;                   // RoPE dims of the rows this kernel takes
+constexpr int kDN = kD - kDR;             // nope dims (E4M3 in E4M3 rows)
+constexpr int kTK = 64;                   // keys per tile
+constexpr int kNR = 64;                   // heads per CTA
+constexpr int kG = 72 * 128;              // bytes per group of 8 rows (72 dim chunks)
+constexpr int kTile = 8 * kG;             // bytes of a 64-row tile (Q or keys): 73,728
+constexpr int kPBytes = kNR * kTK * 2;    // P^T tile: 8,192
+constexpr int kNP = kDN / 16 + kDR / 8;   // pieces per row: 32 nope pieces + 8 RoPE chunks
+constexpr int kPI = kNP / 4;              // warp instructions per row group (4 pieces each)
+constexpr int kWI = kDN / 16 / 4;         // widening warp instructions per row group
 constexpr long kSpin = 1L << 26;
 constexpr uint32_t kWin = 1u << 30;
 constexpr int kThreads = 288;
+constexpr float kRescale = 8.f;           // log2 headroom before the reference moves
+constexpr int kColS = 0;                  // S buffers at columns 0 and 64
+constexpr int kColO = 2 * kTK;            // O^T chunk c at 128 + 64 c
+constexpr uint32_t kTmemCols = 512;
+static_assert(kNP % 4 == 0 && (kDN / 16) % 4 == 0, "piece grouping");
+
+constexpr size_t kSmem = 3 * static_cast<size_t>(kTile) + kPBytes + 2 * kTK * 4 + kNR * 4;
 
 __device__ __forceinline__ uint32_t su32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
@@ -55,15 +69,6 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t 
   d |= static_cast<uint64_t>(1) << 46;
   return d;
 }
-
-__device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
-}
-__device__ __forceinline__ void cp8(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(dst), "l"(src));
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n"); }
-__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;\n"); }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
@@ -78,11 +83,32 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
                : "r"(bar), "r"(parity));
   return done != 0;
 }
+// non-blocking probe (try_wait may suspend the thread for a while; a thread that polls
+// several barriers must not sleep on one of them)
+__device__ __forceinline__ bool mbar_probe(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile("{\n.reg .pred p;\nmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+               : "=r"(done)
+               : "r"(bar), "r"(parity));
+  return done != 0;
+}
 
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n"); }
 __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n"); }
-__device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n)); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+__device__ __forceinline__ void named_bar(int id, int n) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
+}
+// named barrier that also ORs a predicate over the participating threads
+__device__ __forceinline__ bool named_bar_or(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n.reg .pred pi, po;\nsetp.ne.b32 pi, %1, 0;\nbar.red.or.pred po, %2, %3, pi;\nselp.u32 %0, 1, 0, po;\n}\n"
+      : "=r"(r)
+      : "r"(static_cast<int>(v)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
 
 __device__ __forceinline__ void mma_f16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
@@ -93,49 +119,154 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar));
 }
 
-template <int N>
-__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]);
-template <>
-__device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-template <>
-__device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
-      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-}
-template <>
-__device__ __forceinline__ void tmem_ld<64>(uint32_t taddr, uint32_t (&r)[64]) {
-  tmem_ld<32>(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-  tmem_ld<32>(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n"); }
+#define LC_R32(r)                                                                                                 \
+  "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),   \
+      "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),      \
+      "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),     \
+      "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+#define LC_REGS32                                                                                                 \
+  "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29," \
+  "%30,%31}"
 
-__device__ __forceinline__ uint4 e4m3x8_bf16x8(uint2 u) {
-  const uint32_t w[2] = {u.x, u.y};
+// lane i of the warp's quarter, 32 consecutive columns
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 " LC_REGS32 ", [%32];\n" : LC_R32(r) : "r"(taddr));
+}
+// lanes 0-15 of the quarter: thread i < 16 gets lane i, columns c..c+31; thread 16 + i
+// gets lane i, columns c+32..c+63
+__device__ __forceinline__ void tmem_ld16x2(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x32.b32 " LC_REGS32 ", [%32], 32;\n" : LC_R32(r) : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+// 8 E4M3 values -> 8 BF16 values, exact (an E4M3 value has <= 4 significant bits)
+__device__ __forceinline__ uint4 e4m3x8_bf16x8(uint32_t lo, uint32_t hi) {
+  const uint32_t w[2] = {lo, hi};
   uint32_t o[4];
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
     const float2 a = e4m3x2_to_f32x2(static_cast<uint16_t>(w[j] & 0xffffu));
     const float2 b = e4m3x2_to_f32x2(static_cast<uint16_t>(w[j] >> 16));
-    o[2 * j] = (__float_as_uint(a.x) >> 16) | (__float_as_uint(a.y) & 0xffff0000u);
-    o[2 * j + 1] = (__float_as_uint(b.x) >> 16) | (__float_as_uint(b.y) & 0xffff0000u);
+    o[2 * j] = __byte_perm(__float_as_uint(a.x), __float_as_uint(a.y), 0x7632);
+    o[2 * j + 1] = __byte_perm(__float_as_uint(b.x), __float_as_uint(b.y), 0x7632);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// byte offset of dim chunk c (8 dims) of row r in a core-matrix tile with group stride gs
-__device__ __forceinline__ uint32_t tile_off(int r, int c, int gs) { return (r >> 3) * gs + c * 128 + (r & 7) * 16; }
+// byte offset of dim chunk c (8 dims) of row r in a 64-row core-matrix tile
+__device__ __forceinline__ uint32_t tile_off(int r, int c) { return (r >> 3) * kG + c * 128 + (r & 7) * 16; }
+
+__device__ __forceinline__ void cp16(uint8_t* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(su32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit_wait() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_all;\n" ::: "memory");
+}
+__device__ __forceinline__ void zero16(uint8_t* dst) { *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0); }
+
+struct RowSrc {  // a row set, by value (no address of a kernel parameter is taken)
+  int fmt;
+  const uint8_t* x;
+  const uint8_t* rope;
+};
+__device__ __forceinline__ RowSrc row_src(const lc_rows& r) {
+  return RowSrc{r.fmt, static_cast<const uint8_t*>(r.x), static_cast<const uint8_t*>(r.rope)};
+}
+
+// Piece p of a row: p < 32 = nope dims 16p .. 16p + 15 (chunks 2p, 2p + 1), p >= 32 = RoPE
+// chunk p + 32.  One warp instruction covers the 8 rows of a row group and 4 consecutive
+// pieces: quarter qq, lane w takes row w and piece 2 (qq / 2) + ((w / 4) ^ qq) % 2 of the
+// four, so each quarter writes 8 x 16 bytes on distinct banks and each 32-byte sector of a
+// source row is read whole by one instruction.
+__device__ __forceinline__ int piece_off(int lane) {
+  const int qq = lane >> 3, w = lane & 7;
+  return 2 * (qq >> 1) + (((w >> 2) ^ qq) & 1);
+}
+
+// Copy phase of a 64-row tile (warp wi of nw).  A BF16 row and the RoPE chunks of an E4M3
+// row land in their chunk slots; an E4M3 nope piece lands raw in the slot of its second
+// chunk (widened by tile_widen).  row_of(r, src, row) gives row r's source (row < 0: zeros).
+template <class RowOf>
+__device__ __forceinline__ void tile_copy(uint8_t* tile, int wi, int nw, int lane, RowOf row_of) {
+  const int off = piece_off(lane), w = lane & 7;
+  for (int k = wi; k < 8 * kPI; k += nw) {
+    const int g = k / kPI, p = (k % kPI) * 4 + off, r = g * 8 + w;
+    RowSrc rs;
+    int64_t row;
+    row_of(r, rs, row);
+    if (p < kDN / 16) {
+      uint8_t* d0 = tile + tile_off(r, 2 * p);
+      if (row < 0) {
+        zero16(d0);
+        zero16(d0 + 128);
+      } else if (rs.fmt == LC_FMT_BF16) {
+        const uint8_t* src = rs.x + (row * kD + p * 16) * 2;
+        cp16(d0, src);
+        cp16(d0 + 128, src + 16);
+      } else {
+        cp16(d0 + 128, rs.x + row * kDN + p * 16);
+      }
+    } else {
+      const int c = p + kDN / 16;
+      uint8_t* d0 = tile + tile_off(r, c);
+      if (row < 0) zero16(d0);
+      else if (rs.fmt == LC_FMT_BF16) cp16(d0, rs.x + (row * kD + c * 8) * 2);
+      else cp16(d0, rs.rope + (row * kDR + (c * 8 - kDN)) * 2);
+    }
+  }
+}
+
+// Widen phase: the raw E4M3 piece in chunk slot 2p + 1 of an E4M3 row becomes BF16 chunks
+// 2p and 2p + 1 (each item reads its own slot before writing it: no hazard between items).
+// Four items per thread are loaded before any is converted.
+template <class IsE4m3>
+__device__ __forceinline__ void tile_widen(uint8_t* tile, int wi, int nw, int lane, IsE4m3 is_e4m3) {
+  const int off = piece_off(lane), w = lane & 7;
+  for (int k0 = wi; k0 < 8 * kWI; k0 += 4 * nw) {
+    uint4 raw[4];
+    uint8_t* d[4];
+    bool ok[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int k = k0 + j * nw;
+      const int g = k / kWI, p = (k % kWI) * 4 + off, r = g * 8 + w;
+      ok[j] = k < 8 * kWI && is_e4m3(r);
+      d[j] = tile + tile_off(r, 2 * p);
+      if (ok[j]) raw[j] = *reinterpret_cast<const uint4*>(d[j] + 128);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (ok[j]) {
+        *reinterpret_cast<uint4*>(d[j]) = e4m3x8_bf16x8(raw[j].x, raw[j].y);
+        *reinterpret_cast<uint4*>(d[j] + 128) = e4m3x8_bf16x8(raw[j].z, raw[j].w);
+      }
+  }
+}
+
+// 2^x on the special function unit (relative error far below the BF16 rounding of P)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(gdst), "r"(su32(ssrc)),
+               "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
+}
 
 }  // namespace
 
@@ -144,37 +275,38 @@ struct AttnTcGeom {
   int sps;  // slots per split, multiple of kTK
 };
 
-// Shared state of one CTA.
 struct TcBars {
-  uint64_t kfull[kStages];   // producers -> MMA: key stage ready (128 arrivals)
-  uint64_t kempty[kStages];  // MMA -> producers: key stage read by O (commit)
-  uint64_t sfull[2];         // MMA -> softmax: S buffer computed (commit)
-  uint64_t pfull[2];         // softmax -> MMA: P buffer written, S buffer read (128 arrivals)
-  uint64_t pempty[2];        // MMA -> softmax: P buffer read by O (commit)
-  uint64_t odone;            // MMA -> epilogue: last O complete (commit)
+  uint64_t qfull;      // Q loaded (128 arrivals)
+  uint64_t kfull[2];   // key stage ready (128 arrivals)
+  uint64_t kempty[2];  // key stage read by O (commit)
+  uint64_t sfull[2];   // S buffer computed (commit)
+  uint64_t sempty[2];  // S buffer read (128 arrivals)
+  uint64_t pfull;      // P written (128 arrivals)
+  uint64_t pempty;     // P read and O updated (commit)
+  uint64_t fin;        // every MMA complete (commit)
 };
 
-// grid: (n_q, head groups * n_split); 288 threads.  NR = heads per CTA (16 or 64).
-template <int NR>
+// grid: one CTA per (query, head group, key split), the split index fastest; 288 threads.
+// Partial results of split s go to ws_o rows s * n_q * H + q * H + h (576 floats each) and
+// ws_ml[2 ((q * H + h) * n_split + s) + {0, 1}] = (m, l).
 __global__ void __launch_bounds__(kThreads, 1)
-    k_attn_tc(lc_attn_args a, int sparse, AttnTcGeom geo, uint32_t tmem_cols, float* __restrict__ ws_o,
-              float* __restrict__ ws_ml) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* Qs = smem;                                        // (NR / 8) * kQG
-  uint8_t* Ks = Qs + (NR / 8) * kQG;                         // [kStages][kKTile]
-  uint8_t* Raw = Ks + kStages * kKTile;                      // [kStages][kTK][kRaw]
-  uint8_t* Ps = Raw + kStages * kTK * kRaw;                  // [2][NR rows][kTK keys] BF16
-  int* kcode = reinterpret_cast<int*>(Ps + 2 * NR * kTK * 2);  // [kStages][kTK]
-  float* s_l = reinterpret_cast<float*>(kcode + kStages * kTK);  // [NR]
+    k_attn_tc(lc_attn_args a, int sparse, AttnTcGeom geo, float* __restrict__ ws_o, float* __restrict__ ws_ml) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* Qs = smem;                                             // kTile
+  uint8_t* Ks = Qs + kTile;                                       // [2][kTile]
+  uint8_t* Ps = Ks + 2 * kTile;                                   // kPBytes
+  int* kcode = reinterpret_cast<int*>(Ps + kPBytes);              // [2][kTK]
+  float* s_f = reinterpret_cast<float*>(kcode + 2 * kTK);         // [kNR] per-head factors
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ __align__(8) TcBars bars;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int q = blockIdx.x;
-  const int hg = blockIdx.y / geo.n_split, split = blockIdx.y % geo.n_split;
-  const int H = a.dims.H, d_r = a.dims.d_r;
-  const int d_n = kD - d_r;
+  const int n_hg = a.dims.H / kNR;
+  const int split = blockIdx.x % geo.n_split;
+  const int hg = (blockIdx.x / geo.n_split) % n_hg;
+  const int q = blockIdx.x / (geo.n_split * n_hg);
+  const int H = a.dims.H;
   const int b = seq_of_query(a.batch.q_start, a.batch.num_seqs, q);
   const int p = __ldg(a.batch.q_pos0 + b) + (q - __ldg(a.batch.q_start + b));
   const int n_ent = __ldg(a.batch.n_ent + b);
@@ -190,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int wl = a.W > 0 ? __ldg(a.batch.win_len + b) : 0;
   const int64_t wr0 = a.W > 0 ? __ldg(a.batch.win_start + b) : 0;
   const int32_t* idx_row = sparse ? a.idx + static_cast<int64_t>(q) * a.k : nullptr;
+  const int64_t row0 = static_cast<int64_t>(q) * H + hg * kNR;  // first output row of the CTA
 
   // bounded wait; gives up (and tells the other roles) after kSpin polls
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -202,268 +335,317 @@ __global__ void __launch_bounds__(kThreads, 1)
     atomicExch(&s_abort, 1);
     return false;
   };
+  // key slot -> entry index j, kWin | window row, or -1 (masked)
+  auto slot_code = [&](int s) -> int {
+    if (s >= s_end) return -1;
+    if (s < n_first) {
+      const int j = sparse ? __ldg(idx_row + s) : s;
+      if (j < 0) return -1;
+      if (j >= n_ent) {
+        set_status(a.status, LC_DEV_BAD_INDEX);
+        return -1;
+      }
+      if (j >= nv) {
+        set_status(a.status, LC_DEV_NONVISIBLE);
+        return -1;
+      }
+      return j;
+    }
+    const int rr = wlo + (s - n_first) - wp0;
+    if (rr < 0 || rr >= wl) {
+      set_status(a.status, LC_DEV_WINDOW_RANGE);
+      return -1;
+    }
+    return static_cast<int>(kWin) | rr;
+  };
 
-  // ---- set-up (all threads): tensor memory, barriers, queries, the ones chunk ----
+  // ---- set-up: tensor memory, barriers ----
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(su32(&s_tmem)),
-                 "r"(tmem_cols));
+                 "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
   }
-  if (tid == 0) {
+  if (tid == 32) {
     s_abort = 0;
-    for (int i = 0; i < kStages; ++i) {
+    mbar_init(su32(&bars.qfull), 128);
+    for (int i = 0; i < 2; ++i) {
       mbar_init(su32(&bars.kfull[i]), 128);
       mbar_init(su32(&bars.kempty[i]), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
       mbar_init(su32(&bars.sfull[i]), 1);
-      mbar_init(su32(&bars.pfull[i]), 128);
-      mbar_init(su32(&bars.pempty[i]), 1);
+      mbar_init(su32(&bars.sempty[i]), 128);
     }
-    mbar_init(su32(&bars.odone), 1);
+    mbar_init(su32(&bars.pfull), 128);
+    mbar_init(su32(&bars.pempty), 1);
+    mbar_init(su32(&bars.fin), 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n");
   }
-  for (int u = tid; u < NR * 72; u += kThreads) {
-    const int r = u / 72, c = u % 72;
-    const int h = hg * NR + r;
-    uint8_t* dst = Qs + tile_off(r, c, kQG);
-    if (h >= H) {
-      *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-      continue;
-    }
-    const int64_t row = static_cast<int64_t>(q) * H + h;
-    if (a.q.fmt == LC_FMT_BF16) cp16(su32(dst), static_cast<const uint16_t*>(a.q.x) + row * kD + c * 8);
-    else if (c * 8 < d_n) cp8(su32(Raw + r * kRaw + c * 8), static_cast<const uint8_t*>(a.q.x) + row * d_n + c * 8);
-    else cp16(su32(dst), static_cast<const uint16_t*>(a.q.rope) + row * d_r + (c * 8 - d_n));
-  }
-  for (int u = tid; u < kStages * kTK; u += kThreads) {  // dim 576 = 1, dims 577..583 = 0
-    const int st = u / kTK, kr = u % kTK;
-    *reinterpret_cast<uint4*>(Ks + st * kKTile + tile_off(kr, 72, kKG)) = make_uint4(0x3F80u, 0, 0, 0);
-  }
-  cp_commit();
-  cp_wait_all();
-  __syncthreads();
-  if (a.q.fmt == LC_FMT_E4M3_BF16) {
-    for (int u = tid; u < NR * (d_n / 8); u += kThreads) {
-      const int r = u / (d_n / 8), c = u % (d_n / 8);
-      if (hg * NR + r < H)
-        *reinterpret_cast<uint4*>(Qs + tile_off(r, c, kQG)) =
-            e4m3x8_bf16x8(*reinterpret_cast<const uint2*>(Raw + r * kRaw + c * 8));
-    }
-  }
-  fence_async_smem();
   fence_before();
   __syncthreads();
   fence_after();
   const uint32_t tm = s_tmem;
-  const uint32_t col_o = 2 * kTK;  // S buffers at columns 0 and kTK; O^T chunk c at col_o + c * NR
 
   if (warp >= 4 && warp < 8) {
     // ================= producers: gather + widen key tiles =================
-    const int pt = tid - 128;  // 0..127
+    const int pt = tid - 128, pw = warp - 4;
+    const RowSrc src_win = row_src(a.win), src_ent = row_src(a.ent);
+    int code_next = pt < kTK ? slot_code(s_begin + pt) : -1;
     for (int t = 0; t < n_tiles; ++t) {
-      const int st = t % kStages;
-      const uint32_t ph = (t / kStages) & 1;
-      if (!wait(&bars.kempty[st], ph ^ 1)) break;
-      if (pt < kTK) {
-        const int s = s_begin + t * kTK + pt;
-        int code = -1;
-        if (s < s_end) {
-          if (s < n_first) {
-            const int j = sparse ? __ldg(idx_row + s) : s;
-            if (j >= 0) {
-              if (j >= n_ent) set_status(a.status, LC_DEV_BAD_INDEX);
-              else if (j >= nv) set_status(a.status, LC_DEV_NONVISIBLE);
-              else code = j;
-            }
-          } else {
-            const int rr = wlo + (s - n_first) - wp0;
-            if (rr < 0 || rr >= wl) set_status(a.status, LC_DEV_WINDOW_RANGE);
-            else code = static_cast<int>(kWin) | rr;
-          }
-        }
-        kcode[st * kTK + pt] = code;
-      }
-      named_bar(1, 128);
-      uint8_t* kt = Ks + st * kKTile;
-      uint8_t* rw = Raw + st * kTK * kRaw;
-      for (int u = pt; u < kTK * 72; u += 128) {
-        const int kr = u / 72, c = u % 72;
-        const int code = kcode[st * kTK + kr];
-        uint8_t* dst = kt + tile_off(kr, c, kKG);
-        if (code < 0) {
-          *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-          continue;
-        }
-        const lc_rows& rs = (code & kWin) ? a.win : a.ent;
-        const int64_t r = (code & kWin) ? wr0 + (code & ~kWin) : ent0 + code;
-        if (rs.fmt == LC_FMT_BF16) cp16(su32(dst), static_cast<const uint16_t*>(rs.x) + r * kD + c * 8);
-        else if (c * 8 < d_n) cp8(su32(rw + kr * kRaw + c * 8), static_cast<const uint8_t*>(rs.x) + r * d_n + c * 8);
-        else cp16(su32(dst), static_cast<const uint16_t*>(rs.rope) + r * d_r + (c * 8 - d_n));
-      }
-      cp_commit();
-      cp_wait_all();
-      named_bar(1, 128);
-      if (a.ent.fmt == LC_FMT_E4M3_BF16) {
-        const int dnc = d_n / 8;
-        for (int u = pt; u < kTK * dnc; u += 128) {
-          const int kr = u / dnc, c = u % dnc;
-          const int code = kcode[st * kTK + kr];
-          if (code >= 0 && !(code & kWin))
-            *reinterpret_cast<uint4*>(kt + tile_off(kr, c, kKG)) =
-                e4m3x8_bf16x8(*reinterpret_cast<const uint2*>(rw + kr * kRaw + c * 8));
-        }
-      }
+      const int st = t & 1;
+      const bool ok = t < 2 || wait(&bars.kempty[st], ((t >> 1) - 1) & 1);
+      if (ok && pt < kTK) kcode[st * kTK + pt] = code_next;
+      if (named_bar_or(2, 128, !ok)) break;  // the role stops as one
+      if (pt < kTK && t + 1 < n_tiles) code_next = slot_code(s_begin + (t + 1) * kTK + pt);
+      uint8_t* kt = Ks + st * kTile;
+      const int* kc = kcode + st * kTK;
+      tile_copy(kt, pw, 4, lane, [&](int r, RowSrc& rs, int64_t& row) {
+        const int code = kc[r];
+        rs = (code & kWin) ? src_win : src_ent;
+        row = code < 0 ? -1 : (code & kWin) ? wr0 + (code & ~kWin) : ent0 + code;
+      });
+      cp_commit_wait();
+      named_bar(2, 128);
+      if (src_ent.fmt == LC_FMT_E4M3_BF16)
+        tile_widen(kt, pw, 4, lane, [&](int r) { return kc[r] >= 0 && !(kc[r] & kWin); });
       fence_async_smem();
       mbar_arrive(su32(&bars.kfull[st]));
     }
   } else if (warp == 8) {
     // ================= MMA issue (one lane) =================
     if (lane == 0) {
+      // S: M = 64, N = 64, both K-major; O^T: M = 128 (or 64), N = 64, A (V^T) MN-major
       const uint32_t id_s = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kTK >> 3) << 17) |
-                            (static_cast<uint32_t>(64 >> 4) << 24);
-      const uint32_t id_o = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) |
-                            (static_cast<uint32_t>(NR >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
-      const uint32_t qa = su32(Qs);
-      auto issue_o = [&](int u) -> bool {  // O^T += V^T P^T for tile u
-        const int st = u % kStages, pb = u & 1;
-        if (!wait(&bars.pfull[pb], (u >> 1) & 1)) return false;
-        fence_after();
-        const uint32_t kb = su32(Ks + st * kKTile), pp = su32(Ps + pb * NR * kTK * 2);
+                            (static_cast<uint32_t>(kNR >> 4) << 24);
+      const uint32_t id_o128 = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) |
+                               (static_cast<uint32_t>(kNR >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+      const uint32_t id_o64 = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) |
+                              (static_cast<uint32_t>(kNR >> 3) << 17) | (static_cast<uint32_t>(64 >> 4) << 24);
+      const uint64_t dq = sdesc(su32(Qs), 128, kG);
+      const uint64_t dp = sdesc(su32(Ps), 128, (kTK / 8) * 128);
+      // Issue whichever group is ready: S(ns) once its key stage is full and its S buffer
+      // read, O(no) once P(no) is written.  S runs at most two tiles ahead of O (the key
+      // stage of S(no + 2) is released by O(no)).
+      int ns = 0, no = 0;
+      long idle = 0;
+      bool ok = n_tiles == 0 || wait(&bars.qfull, 0);
+      while (ok && no < n_tiles) {
+        bool progressed = false;
+        if (ns < n_tiles) {
+          const int st = ns & 1;
+          if (mbar_probe(su32(&bars.kfull[st]), (ns >> 1) & 1) &&
+              (ns < 2 || mbar_probe(su32(&bars.sempty[st]), ((ns >> 1) - 1) & 1))) {
+            fence_after();
+            const uint64_t dk = sdesc(su32(Ks + st * kTile), 128, kG);
 #pragma unroll
-        for (int c = 0; c < 5; ++c)
+            for (int k = 0; k < kD / 16; ++k)
+              mma_f16(tm + kColS + st * kTK, dq + k * 16, dk + k * 16, id_s, k > 0);
+            mma_commit(su32(&bars.sfull[st]));
+            ++ns;
+            progressed = true;
+          }
+        }
+        if (no < ns && mbar_probe(su32(&bars.pfull), no & 1)) {
+          fence_after();
+          // V^T: M = dims (chunk stride 128 B), K = keys (group stride kG); P^T: K-major
+          const uint64_t dv = sdesc(su32(Ks + (no & 1) * kTile), kG, 128);
 #pragma unroll
-          for (int k = 0; k < kTK / 16; ++k)
-            mma_f16(tm + col_o + c * NR, sdesc(kb + c * 16 * 128 + k * 2 * kKG, kKG, 128),
-                    sdesc(pp + k * 256, 128, (kTK / 8) * 128), id_o, (u > 0) || (k > 0));
-        mma_commit(su32(&bars.kempty[st]));
-        mma_commit(su32(&bars.pempty[pb]));
-        return true;
-      };
-      bool ok = true;
-      for (int t = 0; t < n_tiles && ok; ++t) {
-        const int st = t % kStages, sb = t & 1;
-        ok = wait(&bars.kfull[st], (t / kStages) & 1);
-        if (!ok) break;
-        fence_after();
-        // S buffer sb was last read by the softmax of tile t - 2, which the issue of O(t - 2)
-        // waited for
-        const uint32_t kb = su32(Ks + st * kKTile);
-#pragma unroll 4
-        for (int k = 0; k < kD / 16; ++k)
-          mma_f16(tm + sb * kTK, sdesc(qa + k * 256, 128, kQG), sdesc(kb + k * 256, 128, kKG), id_s, k > 0);
-        mma_commit(su32(&bars.sfull[sb]));
-        if (t > 0) ok = issue_o(t - 1);
+          for (int kk = 0; kk < kTK / 16; ++kk)
+#pragma unroll
+            for (int c = 0; c < 5; ++c)
+              mma_f16(tm + kColO + c * kNR, dv + (c * 2048 + kk * 2 * kG) / 16, dp + kk * 16, c < 4 ? id_o128 : id_o64,
+                      (no > 0) || (kk > 0));
+          mma_commit(su32(&bars.kempty[no & 1]));
+          mma_commit(su32(&bars.pempty));
+          ++no;
+          progressed = true;
+        }
+        if (progressed) {
+          idle = 0;
+        } else if (++idle >= kSpin) {
+          set_status(a.status, LC_DEV_TIMEOUT);
+          atomicExch(&s_abort, 1);
+          ok = false;
+        } else if ((idle & 1023) == 0 && *reinterpret_cast<volatile int*>(&s_abort)) {
+          ok = false;
+        }
       }
-      if (ok && n_tiles > 0) ok = issue_o(n_tiles - 1);
-      mma_commit(su32(&bars.odone));
+      mma_commit(su32(&bars.fin));
+      wait(&bars.fin, 0);
     }
   } else {
-    // ================= softmax: S -> P =================
-    const int r = warp * 16 + lane;  // row held by this lane (lanes 0..15 of each quadrant)
+    // ================= warps 0-3: Q, softmax, epilogue =================
+    const int r = warp * 16 + (lane & 15);  // head row (tensor-memory lane 32 w + lane % 16)
+    const int hf = lane >> 4;               // which 32 of a tile's 64 keys this thread takes
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const float sl2 = a.scale * 1.4426950408889634f;
-    bool range_bad = false;
+    if (n_tiles > 0) {
+      const RowSrc src_q = row_src(a.q);
+      tile_copy(Qs, warp, 4, lane, [&](int rr, RowSrc& rs, int64_t& row) {
+        rs = src_q;
+        row = row0 + rr;
+      });
+      cp_commit_wait();
+      named_bar(1, 128);
+      if (src_q.fmt == LC_FMT_E4M3_BF16) tile_widen(Qs, warp, 4, lane, [](int) { return true; });
+      fence_async_smem();
+      mbar_arrive(su32(&bars.qfull));
+    }
+    float m_ref = -INFINITY, l_sum = 0.f;  // m_ref is the same in both halves of a row
+    bool good = true;
     for (int t = 0; t < n_tiles; ++t) {
-      const int sb = t & 1, st = t % kStages;
-      if (!wait(&bars.sfull[sb], (t >> 1) & 1)) break;
-      if (!wait(&bars.pempty[sb], ((t >> 1) & 1) ^ 1)) break;
-      // acquire the producers' key codes of this stage (the stage cannot have been refilled:
-      // that waits for O of this tile, which waits for this P)
-      if (!wait(&bars.kfull[st], (t / kStages) & 1)) break;
+      const int st = t & 1;
+      const bool okw = wait(&bars.sfull[st], (t >> 1) & 1) && wait(&bars.kfull[st], (t >> 1) & 1);
+      if (named_bar_or(1, 128, !okw)) {  // the role stops as one
+        good = false;
+        break;
+      }
       fence_after();
-      uint32_t sv[kTK];
-      tmem_ld<kTK>(tm + lane_off + sb * kTK, sv);
+      uint32_t sv[32];
+      tmem_ld16x2(tm + lane_off + kColS + st * kTK, sv);
       tmem_wait_ld();
-      if (lane < 16 && r < NR) {
-        const int* kc = kcode + st * kTK;
-        uint32_t pk[kTK / 2];
+      fence_before();
+      mbar_arrive(su32(&bars.sempty[st]));
+      const int* kc = kcode + st * kTK + 32 * hf;
+      float mx = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < kTK; j += 2) {
-          const float l0 = __uint_as_float(sv[j]) * sl2, l1 = __uint_as_float(sv[j + 1]) * sl2;
-          range_bad |= (l0 > 115.f) | (l1 > 115.f);  // 80 in natural-log units
-          const float p0 = kc[j] >= 0 ? exp2f(l0) : 0.f;
-          const float p1 = kc[j + 1] >= 0 ? exp2f(l1) : 0.f;
-          pk[j / 2] = static_cast<uint32_t>(f32_to_bf16_bits(p0)) | (static_cast<uint32_t>(f32_to_bf16_bits(p1)) << 16);
+      for (int j = 0; j < 32; ++j) {
+        const float x = kc[j] >= 0 ? __uint_as_float(sv[j]) * sl2 : -INFINITY;
+        sv[j] = __float_as_uint(x);
+        mx = fmaxf(mx, x);
+      }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const bool need = mx > m_ref + kRescale;
+      // P (single buffer) and O are free once O of the previous tile is done
+      const bool okp = t == 0 || wait(&bars.pempty, (t - 1) & 1);
+      if (named_bar_or(1, 128, !okp)) {
+        good = false;
+        break;
+      }
+      const bool any = named_bar_or(1, 128, need && t > 0);
+      float f = 1.f;
+      if (need) {
+        f = m_ref == -INFINITY ? 0.f : exp2f(m_ref - mx);
+        l_sum *= f;
+        m_ref = mx;
+      }
+      if (any) {
+        // rescale O^T columns (heads) in tensor memory: every lane of all 5 chunks
+        if (hf == 0) s_f[r] = f;
+        named_bar(1, 128);
+        fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 5; ++c)
+#pragma unroll 1
+          for (int hh = 0; hh < kNR; hh += 32) {
+            uint32_t ov[32];
+            const uint32_t ta = tm + lane_off + kColO + c * kNR + hh;
+            tmem_ld32(ta, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * s_f[hh + i]);
+            tmem_st32(ta, ov);
+          }
+        tmem_wait_st();
+        named_bar(1, 128);  // s_f is rewritten only after every lane used it
+      }
+      {
+        uint32_t pk[16];
+        const float mr = m_ref == -INFINITY ? 0.f : m_ref;  // a row with no key yet: all x = -inf
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          // masked keys: x = -inf, 2^-inf = 0
+          const __nv_bfloat162 pb =
+              __floats2bfloat162_rn(ex2(__uint_as_float(sv[j]) - mr), ex2(__uint_as_float(sv[j + 1]) - mr));
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(&pb);
+          l_sum += __uint_as_float(w << 16) + __uint_as_float(w & 0xffff0000u);
+          pk[j / 2] = w;
         }
-        uint8_t* pbuf = Ps + sb * NR * kTK * 2;
+        // P^T tile, K-major: head group (r / 8) stride 1024 B, key chunk stride 128 B
 #pragma unroll
-        for (int c = 0; c < kTK / 8; ++c)
-          *reinterpret_cast<uint4*>(pbuf + tile_off(r, c, (kTK / 8) * 128)) =
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(Ps + (r >> 3) * 1024 + (4 * hf + c) * 128 + (r & 7) * 16) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
       fence_async_smem();
       fence_before();
-      mbar_arrive(su32(&bars.pfull[sb]));
+      mbar_arrive(su32(&bars.pfull));
     }
-    if (range_bad) set_status(a.status, LC_DEV_RANGE);
-  }
-
-  // ---- epilogue (warps 0-3): chunk c, lane L -> dim 128 c + L; columns -> rows ----
-  if (warp < 4) {
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const bool good = n_tiles > 0 && wait(&bars.odone, 0);
+    // ---- epilogue ----
+    if (good && n_tiles > 0) good = wait(&bars.pempty, (n_tiles - 1) & 1);
+    good = !named_bar_or(1, 128, !good);  // uniform: the tensor-memory loads below are warp-wide
     fence_after();
-    // row sums: dim 576 = chunk 4, lane 64 (warp 2, lane 0)
-    if (warp == 2) {
-      uint32_t v[NR];
-      if (good) {
-        tmem_ld<NR>(tm + lane_off + col_o + 4 * NR, v);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int i = 0; i < NR; ++i) v[i] = 0;
+    const float l_row = l_sum + __shfl_xor_sync(0xffffffffu, l_sum, 16);
+    if (hf == 0) {
+      const int h = hg * kNR + r;
+      if (geo.n_split == 1) {
+        const float sk = __ldg(a.sink + h) * 1.4426950408889634f;
+        const float M = fmaxf(sk, m_ref);
+        const float w = m_ref == -INFINITY ? 0.f : exp2f(m_ref - M);
+        const float Z = exp2f(sk - M) + l_row * w;
+        s_f[r] = w / Z;
+        if (a.lse && good) a.lse[row0 + r] = (M + log2f(Z)) * 0.6931471805599453f;
+      } else if (good) {
+        const int64_t slot = (row0 + r) * geo.n_split + split;
+        ws_ml[2 * slot] = m_ref;
+        ws_ml[2 * slot + 1] = l_row;
       }
-      if (lane == 0)
-#pragma unroll
-        for (int i = 0; i < NR; ++i) s_l[i] = __uint_as_float(v[i]);
     }
-    named_bar(2, 128);
+    named_bar(1, 128);
+    if (good) {
+      // O rows -> the key stages (free: every MMA is complete), row-major [head][dim]
+      const bool f32 = geo.n_split > 1 || a.out_fmt == LC_FMT_F32;
+      float* stf = reinterpret_cast<float*>(Ks);
+      uint16_t* sth = reinterpret_cast<uint16_t*>(Ks);
 #pragma unroll 1
-    for (int c = 0; c < 5; ++c) {
-      const int dim = c * 128 + warp * 32 + lane;
-      uint32_t v[NR];
-      if (good) {
-        tmem_ld<NR>(tm + lane_off + col_o + c * NR, v);
-        tmem_wait_ld();
-      } else {
+      for (int c = 0; c < 5; ++c) {
+        // chunk c < 4: lane L -> dim 128 c + L; chunk 4 (M = 64): lane 32 w + i -> dim 512 + 16 w + i
+        const int dim = c < 4 ? c * 128 + warp * 32 + lane : (lane < 16 ? 512 + warp * 16 + lane : -1);
+#pragma unroll 1
+        for (int hh = 0; hh < kNR; hh += 32) {
+          uint32_t ov[32];
+          if (n_tiles > 0) {
+            tmem_ld32(tm + lane_off + kColO + c * kNR + hh, ov);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-        for (int i = 0; i < NR; ++i) v[i] = 0;
-      }
-      if (dim >= kD) continue;
+            for (int i = 0; i < 32; ++i) ov[i] = 0;
+          }
+          if (dim < 0) continue;
 #pragma unroll
-      for (int i = 0; i < NR; ++i) {
-        const int h = hg * NR + i;
-        if (h >= H) continue;
-        const int64_t orow = static_cast<int64_t>(q) * H + h;
-        const float ov = __uint_as_float(v[i]);
-        if (geo.n_split == 1) {
-          const float Z = expf(__ldg(a.sink + h)) + s_l[i];
-          const float o = ov / Z;
-          if (a.out_fmt == LC_FMT_BF16) static_cast<uint16_t*>(a.out)[orow * kD + dim] = f32_to_bf16_bits(o);
-          else static_cast<float*>(a.out)[orow * kD + dim] = o;
-          if (dim == 0 && a.lse) a.lse[orow] = logf(Z);
-        } else {
-          const int64_t slot = orow * geo.n_split + split;
-          ws_o[slot * kD + dim] = ov;
-          if (dim == 0) {
-            ws_ml[2 * slot] = 0.f;  // the exponent reference of every split is 0
-            ws_ml[2 * slot + 1] = s_l[i];
+          for (int i = 0; i < 32; ++i) {
+            float v = __uint_as_float(ov[i]);
+            if (geo.n_split == 1) v *= s_f[hh + i];
+            if (f32) stf[(hh + i) * kD + dim] = v;
+            else sth[(hh + i) * kD + dim] = f32_to_bf16_bits(v);
           }
         }
+      }
+      fence_async_smem();
+      named_bar(1, 128);
+      if (tid == 0) {
+        const uint32_t bytes = kNR * kD * (f32 ? 4 : 2);
+        void* dst;
+        if (geo.n_split > 1) dst = ws_o + (static_cast<int64_t>(split) * a.n_q * H + row0) * kD;
+        else if (a.out_fmt == LC_FMT_F32) dst = static_cast<float*>(a.out) + row0 * kD;
+        else dst = static_cast<uint16_t*>(a.out) + row0 * kD;
+        bulk_store(dst, Ks, bytes);
       }
     }
   }
   fence_before();
   __syncthreads();
-  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tm), "r"(tmem_cols));
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tm), "r"(kTmemCols));
 }
 
 // ---------------------------------------------------------------------------------
 bool attn_tc_supported(const lc_attn_args& a) {
-  if (a.dims.D != kD || a.dims.d_r < 64 || a.dims.d_r % 8 || a.dims.H % 16) return false;
-  auto ok = [&](const lc_rows& r) { return r.fmt == LC_FMT_BF16 || r.fmt == LC_FMT_E4M3_BF16; };
-  if (!ok(a.q) || !ok(a.ent) || (a.W > 0 && a.win.fmt != LC_FMT_BF16)) return false;
+  if (a.dims.D != kD || a.dims.d_r != kDR || a.dims.H % kNR) return false;
+  auto ok = [&](const lc_rows& r) {
+    if (r.fmt != LC_FMT_BF16 && r.fmt != LC_FMT_E4M3_BF16) return false;
+    if (reinterpret_cast<uintptr_t>(r.x) % 16) return false;
+    return r.fmt == LC_FMT_BF16 || reinterpret_cast<uintptr_t>(r.rope) % 16 == 0;
+  };
+  if (!ok(a.q) || !ok(a.ent) || (a.W > 0 && (a.win.fmt != LC_FMT_BF16 || !ok(a.win)))) return false;
+  if (reinterpret_cast<uintptr_t>(a.out) % 16 || reinterpret_cast<uintptr_t>(a.workspace) % 16) return false;
   return a.out_fmt == LC_FMT_BF16 || a.out_fmt == LC_FMT_F32;
 }
 
@@ -472,11 +654,10 @@ static AttnTcGeom tc_geometry(const lc_attn_args& a, bool sparse, bool decode) {
   const int ns = max((sparse ? a.k : a.max_ent) + a.W, 1);
   const int tiles = (ns + kTK - 1) / kTK;
   g.sps = tiles * kTK;
-  if (decode) {
-    // one CTA per SM: split the keys only when the (query, head group) pairs leave SMs idle
-    const int ctas = a.n_q * (a.dims.H / 16);
-    const int want = max(1, 148 / max(ctas, 1));
-    const int n = max(1, min(want, tiles / 8));
+  const int ctas = a.n_q * (a.dims.H / kNR);
+  if (decode && ctas < 148) {
+    // one CTA per SM: split the keys when the (query, head group) pairs leave SMs idle
+    const int n = max(1, min(148 / max(ctas, 1), tiles));
     const int per = (tiles + n - 1) / n;
     g.n_split = (tiles + per - 1) / per;
     g.sps = per * kTK;
@@ -491,27 +672,17 @@ size_t attn_tc_workspace(const lc_attn_args& a, bool sparse, bool decode) {
   return rows * kD * sizeof(float) + rows * 2 * sizeof(float);
 }
 
-template <int NR>
-static cudaError_t launch_tc(const lc_attn_args& a, bool sparse, const AttnTcGeom& g, cudaStream_t st) {
-  // the S MMA reads 64 query rows: with NR < 64 the extra rows are the key stages behind Q
-  const size_t sm = static_cast<size_t>((NR / 8) * kQG) + kStages * kKTile + kStages * kTK * kRaw +
-                    2 * NR * kTK * 2 + kStages * kTK * 4 + NR * 4 + 1024;
-  cudaFuncSetAttribute(k_attn_tc<NR>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
-  uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(2 * kTK + 5 * NR)) cols <<= 1;
-  float* ws_o = static_cast<float*>(a.workspace);
-  float* ws_ml = nullptr;
-  if (g.n_split > 1) ws_ml = ws_o + static_cast<size_t>(a.n_q) * a.dims.H * g.n_split * kD;
-  const dim3 grid(a.n_q, (a.dims.H / NR) * g.n_split);
-  k_attn_tc<NR><<<grid, kThreads, sm, st>>>(a, sparse ? 1 : 0, g, cols, ws_o, ws_ml);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_attn_tc(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st, int* n_split_out) {
   const AttnTcGeom g = tc_geometry(a, sparse, decode);
   *n_split_out = g.n_split;
-  if (decode || a.dims.H % 64) return launch_tc<16>(a, sparse, g, st);
-  return launch_tc<64>(a, sparse, g, st);
+  cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
+  float* ws_o = static_cast<float*>(a.workspace);
+  float* ws_ml = nullptr;
+  if (g.n_split > 1) ws_ml = ws_o + static_cast<size_t>(a.n_q) * a.dims.H * g.n_split * kD;
+  const int64_t ctas = static_cast<int64_t>(a.n_q) * (a.dims.H / kNR) * g.n_split;
+  if (ctas > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  k_attn_tc<<<static_cast<unsigned>(ctas), kThreads, kSmem, st>>>(a, sparse ? 1 : 0, g, ws_o, ws_ml);
+  return cudaGetLastError();
 }
 
 }  // namespace lc
