@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0)
     ap.add_argument("--attn-impl", default="auto", choices=["auto", "mma", "tc", "ref"],
-                    help="attention kernel (auto: the fastest measured for the shape)")
+                    help="attention kernel (auto: tcgen05 where it applies, else mma.sync, else reference)")
     return ap.parse_args()
 
 
@@ -202,9 +202,10 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def kernel_traffic(stage_kernel: str):
-    """DRAM bytes per launch of a kernel from the committed ncu summary, if the kernel's
-    source is unchanged since the capture; else None."""
+def kernel_traffic(stage_kernel: str, attn_impl: str):
+    """DRAM bytes per launch of a stage's kernels from the committed ncu summary, if every
+    source file of those kernels is unchanged since the capture (and, for attention, the
+    same kernel choice ran); else None."""
     if not os.path.exists(TRAFFIC_PATH):
         return None
     with open(TRAFFIC_PATH) as f:
@@ -212,17 +213,15 @@ def kernel_traffic(stage_kernel: str):
     e = t.get(stage_kernel)
     if not e:
         return None
-    src = os.path.join(ROOT, "long_context_sparse_softmax_b200", "csrc", e["source"])
-    if not os.path.exists(src):
+    if "attn_impl" in e and attn_impl not in e["attn_impl"]:
         return None
-    sha = hashlib.sha1(open(src, "rb").read()).hexdigest()
-    if sha != e.get("source_sha1"):
-        return None
+    for name, sha in e["sources"].items():
+        src = os.path.join(ROOT, "long_context_sparse_softmax_b200", "csrc", name)
+        if not os.path.exists(src) or hashlib.sha1(open(src, "rb").read()).hexdigest() != sha:
+            return None
     return e.get("dram_bytes_per_launch_full")
 
 
-STAGE_SOURCE = {"qk_prep_q": "k_prep.cu", "qk_prep_win": "k_prep.cu", "compress": "k_prep.cu",
-                "index": "k_index.cu", "topk": "k_topk.cu", "attn": "k_attn.cu"}
 
 
 # ------------------------------------------------------------------------------------
@@ -381,7 +380,7 @@ def run_lc(args):
     else:
         achieved = f / (avg[dom] / 1e3) / 1e12
         peak, unit = pk["bf16_tflops"], "TFLOP/s"
-    traffic = kernel_traffic(dom.split(":")[1])
+    traffic = kernel_traffic(dom.split(":")[1], args.attn_impl)
     stages = {}
     for n in stage_names:
         bb, ff = work[n]

@@ -1,4 +1,5 @@
-// CSA sparse / HCA dense attention on the 5th-generation tensor cores (tcgen05, BF16).
+// CSA sparse / HCA dense attention on the 5th-generation tensor cores (tcgen05, F16 operands,
+// FP32 accumulators).
 //
 // Same mathematics as k_attn.cu ("解读 DeepSeek V4": CSA attends to its top-k compressed
 // entries, HCA to all of them, both plus a 128-token window and a per-head sink; V = K =
@@ -7,18 +8,21 @@
 //
 // Tiles and tensor memory:
 //   * 64-row tiles (the queries' heads, or 64 keys) in shared memory as a grid of 8 x 8
-//     BF16 core matrices, row group g and dim chunk c at g * 9216 + c * 128.  The same key
+//     F16 core matrices, row group g and dim chunk c at g * 9216 + c * 128.  The same key
 //     bytes are the K-major B operand of S = Q K^T and the MN-major A operand V^T of
 //     O^T = V^T P^T.  Rows arrive by cp.async: BF16 parts straight into their chunk slots,
 //     the E4M3 nope part (16 dims = 16 bytes per piece) raw into the slot of the piece's
-//     second chunk, then widened to BF16 in place (exact: E4M3 has 4 significant bits);
+//     second chunk.  A conversion pass then widens E4M3 to F16 in place (exact) and rounds
+//     BF16 to F16 in place (exact for magnitudes in [2^-14, 65504], which RMS-normalised
+//     rows stay within; a value beyond 65504 is reported as LC_DEV_RANGE).  F16 rather than
+//     BF16 operands give P 11 significant bits instead of 8;
 //   * S = Q K^T: M = 64 heads, N = 64 keys, K = 576, two tensor-memory buffers (M = 64
 //     layout: row r in lane 32 (r / 16) + r % 16; the 16x32bx2 load gives lanes 0-15 of a
 //     warp columns 0-31 and lanes 16-31 columns 32-63 of the same rows);
 //   * P = 2^(x - m_h), x = scale * log2(e) * S, with a per-head reference m_h that moves up
 //     only when a tile's maximum exceeds it by more than 8; O^T is then rescaled in tensor
 //     memory (rare after the first tile: P stays below 2^8).  Masked keys get P = 0.  The
-//     row sums add up the BF16-rounded P that the MMA multiplies;
+//     row sums add up the F16-rounded P that the MMA multiplies;
 //   * O^T = V^T P^T accumulates in tensor memory, dims on lanes: chunks of 128 dims
 //     (M = 128) and a last chunk of 64 (M = 64), 64 head columns each.
 // The sink joins at the end: M = max(sink, m), Z = e^(sink - M) + l e^(m - M),
@@ -48,7 +52,8 @@ constexpr int kTile = 8 * kG;             // bytes of a 64-row tile (Q or keys):
 constexpr int kPBytes = kNR * kTK * 2;    // P^T tile: 8,192
 constexpr int kNP = kDN / 16 + kDR / 8;   // pieces per row: 32 nope pieces + 8 RoPE chunks
 constexpr int kPI = kNP / 4;              // warp instructions per row group (4 pieces each)
-constexpr int kWI = kDN / 16 / 4;         // widening warp instructions per row group
+constexpr int kNPair = kD / 16;           // chunk pairs per row (36)
+constexpr int kWI = kNPair / 4;           // conversion warp instructions per row group
 constexpr long kSpin = 1L << 26;
 constexpr uint32_t kWin = 1u << 30;
 constexpr int kThreads = 288;
@@ -56,7 +61,7 @@ constexpr float kRescale = 8.f;           // log2 headroom before the reference 
 constexpr int kColS = 0;                  // S buffers at columns 0 and 64
 constexpr int kColO = 2 * kTK;            // O^T chunk c at 128 + 64 c
 constexpr uint32_t kTmemCols = 512;
-static_assert(kNP % 4 == 0 && (kDN / 16) % 4 == 0, "piece grouping");
+static_assert(kNP % 4 == 0 && kNPair % 4 == 0 && (kDN / 16) % 4 == 0, "piece grouping");
 
 constexpr size_t kSmem = 3 * static_cast<size_t>(kTile) + kPBytes + 2 * kTK * 4 + kNR * 4;
 
@@ -149,16 +154,31 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
-// 8 E4M3 values -> 8 BF16 values, exact (an E4M3 value has <= 4 significant bits)
-__device__ __forceinline__ uint4 e4m3x8_bf16x8(uint32_t lo, uint32_t hi) {
-  const uint32_t w[2] = {lo, hi};
+// 8 E4M3 values -> 8 F16 values, exact (E4M3 is a subset of F16)
+__device__ __forceinline__ uint4 e4m3x8_f16x8(uint32_t lo, uint32_t hi) {
   uint32_t o[4];
+  const uint32_t w[2] = {lo, hi};
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
-    const float2 a = e4m3x2_to_f32x2(static_cast<uint16_t>(w[j] & 0xffffu));
-    const float2 b = e4m3x2_to_f32x2(static_cast<uint16_t>(w[j] >> 16));
-    o[2 * j] = __byte_perm(__float_as_uint(a.x), __float_as_uint(a.y), 0x7632);
-    o[2 * j + 1] = __byte_perm(__float_as_uint(b.x), __float_as_uint(b.y), 0x7632);
+    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[j] & 0xffffu), __NV_E4M3);
+    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[j] >> 16), __NV_E4M3);
+    o[2 * j] = static_cast<uint32_t>(a.x) | (static_cast<uint32_t>(a.y) << 16);
+    o[2 * j + 1] = static_cast<uint32_t>(b.x) | (static_cast<uint32_t>(b.y) << 16);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// 8 BF16 values -> 8 F16 values (round to nearest; exact for magnitudes in [2^-14, 65504]
+// with at most 11 significant bits, which covers every BF16 value there).  `big` is set
+// when a value leaves the F16 range.
+__device__ __forceinline__ uint4 bf16x8_f16x8(uint4 v, bool& big) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const __half2 h = __floats2half2_rn(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u));
+    o[j] = *reinterpret_cast<const uint32_t*>(&h);
+    big |= ((o[j] & 0x7c00u) == 0x7c00u) | ((o[j] & 0x7c000000u) == 0x7c000000u);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -226,34 +246,49 @@ __device__ __forceinline__ void tile_copy(uint8_t* tile, int wi, int nw, int lan
   }
 }
 
-// Widen phase: the raw E4M3 piece in chunk slot 2p + 1 of an E4M3 row becomes BF16 chunks
-// 2p and 2p + 1 (each item reads its own slot before writing it: no hazard between items).
-// Four items per thread are loaded before any is converted.
-template <class IsE4m3>
-__device__ __forceinline__ void tile_widen(uint8_t* tile, int wi, int nw, int lane, IsE4m3 is_e4m3) {
+// Conversion phase, pair p of a row (chunks 2p, 2p + 1; pairs 32..35 hold the RoPE dims).
+// kind(r): 0 = nothing (masked row), 1 = E4M3 row (pairs < 32 are raw E4M3 in the slot of
+// their second chunk: widened in place; RoPE pairs are BF16: rounded to F16 in place),
+// 2 = BF16 row (every pair rounded to F16 in place).  Each item reads its own slots before
+// writing them: no hazard between items.  Four items per thread are loaded before any is
+// converted.  Returns whether a BF16 value left the F16 range.
+template <class KindOf>
+__device__ __forceinline__ bool tile_convert(uint8_t* tile, int wi, int nw, int lane, KindOf kind_of) {
   const int off = piece_off(lane), w = lane & 7;
+  bool big = false;
   for (int k0 = wi; k0 < 8 * kWI; k0 += 4 * nw) {
-    uint4 raw[4];
+    uint4 v0[4], v1[4];
     uint8_t* d[4];
-    bool ok[4];
+    int kd[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int k = k0 + j * nw;
       const int g = k / kWI, p = (k % kWI) * 4 + off, r = g * 8 + w;
-      ok[j] = k < 8 * kWI && is_e4m3(r);
+      const int kr = k < 8 * kWI ? kind_of(r) : 0;
+      // 1: widen raw E4M3, 2: round two BF16 chunks
+      kd[j] = kr == 0 ? 0 : (kr == 1 && p < kDN / 16) ? 1 : 2;
       d[j] = tile + tile_off(r, 2 * p);
-      if (ok[j]) raw[j] = *reinterpret_cast<const uint4*>(d[j] + 128);
+      if (kd[j] == 1) v1[j] = *reinterpret_cast<const uint4*>(d[j] + 128);
+      if (kd[j] == 2) {
+        v0[j] = *reinterpret_cast<const uint4*>(d[j]);
+        v1[j] = *reinterpret_cast<const uint4*>(d[j] + 128);
+      }
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (ok[j]) {
-        *reinterpret_cast<uint4*>(d[j]) = e4m3x8_bf16x8(raw[j].x, raw[j].y);
-        *reinterpret_cast<uint4*>(d[j] + 128) = e4m3x8_bf16x8(raw[j].z, raw[j].w);
+    for (int j = 0; j < 4; ++j) {
+      if (kd[j] == 1) {
+        *reinterpret_cast<uint4*>(d[j]) = e4m3x8_f16x8(v1[j].x, v1[j].y);
+        *reinterpret_cast<uint4*>(d[j] + 128) = e4m3x8_f16x8(v1[j].z, v1[j].w);
+      } else if (kd[j] == 2) {
+        *reinterpret_cast<uint4*>(d[j]) = bf16x8_f16x8(v0[j], big);
+        *reinterpret_cast<uint4*>(d[j] + 128) = bf16x8_f16x8(v1[j], big);
       }
+    }
   }
+  return big;
 }
 
-// 2^x on the special function unit (relative error far below the BF16 rounding of P)
+// 2^x on the special function unit (relative error far below the F16 rounding of P)
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
@@ -404,20 +439,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       });
       cp_commit_wait();
       named_bar(2, 128);
-      if (src_ent.fmt == LC_FMT_E4M3_BF16)
-        tile_widen(kt, pw, 4, lane, [&](int r) { return kc[r] >= 0 && !(kc[r] & kWin); });
+      if (tile_convert(kt, pw, 4, lane, [&](int r) {
+            const int code = kc[r];
+            return code < 0 ? 0 : (!(code & kWin) && src_ent.fmt == LC_FMT_E4M3_BF16) ? 1 : 2;
+          }))
+        set_status(a.status, LC_DEV_RANGE);
       fence_async_smem();
       mbar_arrive(su32(&bars.kfull[st]));
     }
   } else if (warp == 8) {
     // ================= MMA issue (one lane) =================
     if (lane == 0) {
-      // S: M = 64, N = 64, both K-major; O^T: M = 128 (or 64), N = 64, A (V^T) MN-major
-      const uint32_t id_s = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kTK >> 3) << 17) |
+      // F16 operands, FP32 accumulator.  S: M = 64, N = 64, both K-major; O^T: M = 128 (or
+      // 64), N = 64, A (V^T) MN-major
+      const uint32_t id_s = (1u << 4) | (static_cast<uint32_t>(kTK >> 3) << 17) |
                             (static_cast<uint32_t>(kNR >> 4) << 24);
-      const uint32_t id_o128 = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) |
+      const uint32_t id_o128 = (1u << 4) | (1u << 15) |
                                (static_cast<uint32_t>(kNR >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
-      const uint32_t id_o64 = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) |
+      const uint32_t id_o64 = (1u << 4) | (1u << 15) |
                               (static_cast<uint32_t>(kNR >> 3) << 17) | (static_cast<uint32_t>(64 >> 4) << 24);
       const uint64_t dq = sdesc(su32(Qs), 128, kG);
       const uint64_t dp = sdesc(su32(Ps), 128, (kTK / 8) * 128);
@@ -485,7 +524,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       });
       cp_commit_wait();
       named_bar(1, 128);
-      if (src_q.fmt == LC_FMT_E4M3_BF16) tile_widen(Qs, warp, 4, lane, [](int) { return true; });
+      const int qkind = src_q.fmt == LC_FMT_E4M3_BF16 ? 1 : 2;
+      if (tile_convert(Qs, warp, 4, lane, [&](int) { return qkind; })) set_status(a.status, LC_DEV_RANGE);
       fence_async_smem();
       mbar_arrive(su32(&bars.qfull));
     }
@@ -553,11 +593,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           // masked keys: x = -inf, 2^-inf = 0
-          const __nv_bfloat162 pb =
-              __floats2bfloat162_rn(ex2(__uint_as_float(sv[j]) - mr), ex2(__uint_as_float(sv[j + 1]) - mr));
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(&pb);
-          l_sum += __uint_as_float(w << 16) + __uint_as_float(w & 0xffff0000u);
-          pk[j / 2] = w;
+          const __half2 ph = __floats2half2_rn(ex2(__uint_as_float(sv[j]) - mr), ex2(__uint_as_float(sv[j + 1]) - mr));
+          const float2 pf = __half22float2(ph);
+          l_sum += pf.x + pf.y;
+          pk[j / 2] = *reinterpret_cast<const uint32_t*>(&ph);
         }
         // P^T tile, K-major: head group (r / 8) stride 1024 B, key chunk stride 128 B
 #pragma unroll

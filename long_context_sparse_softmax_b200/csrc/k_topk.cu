@@ -2,20 +2,31 @@
 // the lightning indexer picks the top-k compressed entries; "DeepSeek-V4 论文分析" §5.3:
 // Top-512 (Flash) / Top-1024 (Pro)).
 //
-// One CTA per query row.  Scores map to order-preserving 32-bit keys; four 8-bit radix
-// passes over a shared-memory histogram find the K-th largest key T and how many of the
-// keys equal to T to take.  A final pass in index order keeps every key > T and the first
-// `need` keys == T (ties to the lower index), writing indices in ascending order through
-// per-warp counts.  Rows of up to kRowCache scores are staged in shared memory
-// once; longer rows are re-read from global memory (L2) on each pass.  The result depends
-// only on the score values: it is bit-exact and independent of the launch shape.
+// A thread-block cluster of C CTAs takes one query row; CTA r holds the r-th of C equal
+// segments of the row.  Scores map to order-preserving 32-bit keys.  Three radix passes
+// (11, 11 and 10 bits) find the K-th largest key T and how many keys equal to T to take:
+// each CTA builds a 2048-bin histogram of its candidates in shared memory, the cluster
+// barrier publishes it, and every CTA sums the C histograms over distributed shared memory
+// in rank order, so all CTAs reach the same bin.  The selection is then every key > T and
+// the first `need` keys == T in index order (ties to the lower index), written in ascending
+// index order: the CTAs exchange their counts of keys > T and == T the same way, and
+// within a CTA each warp owns a contiguous piece of the segment.  Segments of up to
+// kRowCache keys are staged in shared memory once; longer ones are re-read from global
+// memory (L2) on each pass.  The result depends only on the score values: it is bit-exact
+// and independent of C and of the launch shape.
+#include <cooperative_groups.h>
+
 #include "lc_internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace lc {
 
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kRowCache = 48 * 1024;  // scores held in shared memory (192 KB)
+constexpr int kRowCache = 48 * 1024;  // keys held in shared memory per CTA (192 KB)
+constexpr int kBins = 2048;
+constexpr int kMaxCluster = 8;
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f);
@@ -23,31 +34,43 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 }
 
 __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_cache) {
-  extern __shared__ uint32_t cache[];  // [kRowCache] keys when the row fits
-  __shared__ int hist[256];
+  extern __shared__ uint32_t cache[];  // [kRowCache] keys of this CTA's segment
+  __shared__ int hist[2][kBins];
+  __shared__ int s_wsum[kTopkWarps];
   __shared__ uint32_t s_prefix;
   __shared__ int s_remaining;
+  __shared__ int s_cnt[2];  // this CTA's keys > T and == T
+  __shared__ int s_gt[kTopkWarps], s_eq[kTopkWarps];
+  __shared__ uint32_t s_wmin[kTopkWarps], s_wmax[kTopkWarps];
+  __shared__ uint32_t s_range[2];  // this CTA's smallest and largest key
 
-  const int q = blockIdx.x;
-  const int tid = threadIdx.x;
+  cg::cluster_group cl = cg::this_cluster();
+  const int C = static_cast<int>(cl.num_blocks());
+  const int rank = static_cast<int>(cl.block_rank());
+  const int q = blockIdx.x / C;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b = seq_of_query(a.batch.q_start, a.batch.num_seqs, q);
   const int p = __ldg(a.batch.q_pos0 + b) + (q - __ldg(a.batch.q_start + b));
   const int n = n_visible(p, a.m, a.W_x, __ldg(a.batch.n_ent + b));
   const int K = min(a.k, n);
   int32_t* out = a.idx + static_cast<int64_t>(q) * a.k;
-  if (tid == 0 && a.count) a.count[q] = K;
-  for (int i = K + tid; i < a.k; i += kTopkThreads) out[i] = -1;
-  if (K == 0) return;
-  if (K == n) {  // every visible entry is selected
-    for (int i = tid; i < n; i += kTopkThreads) out[i] = i;
+  if (rank == 0 && tid == 0 && a.count) a.count[q] = K;
+  for (int i = K + rank * kTopkThreads + tid; i < a.k; i += C * kTopkThreads) out[i] = -1;
+  if (K == 0) return;  // the whole cluster returns here (K depends on the row only)
+  if (K == n) {        // every visible entry is selected
+    for (int i = rank * kTopkThreads + tid; i < n; i += C * kTopkThreads) out[i] = i;
     return;
   }
-  const float* row = a.scores + static_cast<int64_t>(q) * a.score_stride;
-  const bool cached = use_cache && n <= kRowCache;
+  // this CTA's segment [s0, s1): multiples of 4 keys, so float4 loads stay aligned
+  const int segl = ((n + C - 1) / C + 3) & ~3;
+  const int s0 = min(n, rank * segl), s1 = min(n, s0 + segl), ns = s1 - s0;
+  const float* row = a.scores + static_cast<int64_t>(q) * a.score_stride + s0;
+  const bool cached = use_cache != 0;
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
   if (cached) {
-    // 16-byte loads, four in flight per thread (rows start 16-byte aligned: the score
-    // stride is a multiple of 4 floats)
-    const int n4 = n >> 2;
+    // 16-byte loads, four in flight per thread (row and segment starts are 16-byte
+    // aligned: the score stride and the segment length are multiples of 4 floats)
+    const int n4 = ns >> 2;
     const float4* r4 = reinterpret_cast<const float4*>(row);
     for (int base = 0; base < n4; base += 4 * kTopkThreads) {
       float4 v[4];
@@ -60,125 +83,269 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
       for (int u = 0; u < 4; ++u) {
         const int i4 = base + u * kTopkThreads + tid;
         if (i4 < n4) {
-          cache[4 * i4 + 0] = order_key(v[u].x);
-          cache[4 * i4 + 1] = order_key(v[u].y);
-          cache[4 * i4 + 2] = order_key(v[u].z);
-          cache[4 * i4 + 3] = order_key(v[u].w);
+          const uint32_t k0 = order_key(v[u].x), k1 = order_key(v[u].y), k2 = order_key(v[u].z),
+                         k3 = order_key(v[u].w);
+          cache[4 * i4 + 0] = k0;
+          cache[4 * i4 + 1] = k1;
+          cache[4 * i4 + 2] = k2;
+          cache[4 * i4 + 3] = k3;
+          kmin = min(kmin, min(min(k0, k1), min(k2, k3)));
+          kmax = max(kmax, max(max(k0, k1), max(k2, k3)));
         }
       }
     }
-    for (int i = 4 * n4 + tid; i < n; i += kTopkThreads) cache[i] = order_key(__ldg(row + i));
+    for (int i = 4 * n4 + tid; i < ns; i += kTopkThreads) {
+      const uint32_t k0 = order_key(__ldg(row + i));
+      cache[i] = k0;
+      kmin = min(kmin, k0);
+      kmax = max(kmax, k0);
+    }
+  } else {
+    for (int i = tid; i < ns; i += kTopkThreads) {
+      const uint32_t k0 = order_key(__ldg(row + i));
+      kmin = min(kmin, k0);
+      kmax = max(kmax, k0);
+    }
   }
-  uint32_t prefix = 0, mask = 0;
+  // keys 4 i4 .. 4 i4 + 3 (past ns: don't-cares that the callers mask; they stay inside the
+  // cache and inside the score row, whose stride is a multiple of 4)
+  auto key4 = [&](int i4) -> uint4 {
+    if (cached) return reinterpret_cast<const uint4*>(cache)[i4];
+    const float4 f = __ldg(reinterpret_cast<const float4*>(row) + i4);
+    return make_uint4(order_key(f.x), order_key(f.y), order_key(f.z), order_key(f.w));
+  };
+  const int n4 = (ns + 3) >> 2;
+
+  // key range of the whole row (every CTA of the cluster gets the same one)
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) {
+    s_wmin[warp] = kmin;
+    s_wmax[warp] = kmax;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t a0 = 0xffffffffu, b0 = 0u;
+    for (int w = 0; w < kTopkWarps; ++w) {
+      a0 = min(a0, s_wmin[w]);
+      b0 = max(b0, s_wmax[w]);
+    }
+    s_range[0] = a0;
+    s_range[1] = b0;
+  }
+  cl.sync();
+  uint32_t umin = 0xffffffffu, umax = 0u;
+  for (int r = 0; r < C; ++r) {
+    const uint32_t* rr = cl.map_shared_rank(s_range, r);
+    umin = min(umin, rr[0]);
+    umax = max(umax, rr[1]);
+  }
+
+  // Radix passes over rel = key - umin, < 2^L with L = bit length of the row's key range,
+  // 11 bits at a time from the top: the first pass spreads the row over the whole
+  // histogram whatever its range, and a row whose keys are all equal needs no pass.
+  // pfx holds the bits of rel found so far; `remaining` counts the keys still to take
+  // inside the bin they select.
+  uint32_t pfx = 0;
   int remaining = K;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
+  int shift = 32 - __clz(static_cast<int>(umax - umin));
+  int pass = 0;
+#pragma unroll 1
+  while (shift > 0) {
+    const int w = min(11, shift);
+    const int hi_shift = shift;  // candidates: rel >> hi_shift == pfx
+    shift -= w;
+    const uint32_t bmask = (1u << w) - 1u;
+    int* h = hist[pass & 1];
+    for (int i = tid; i < kBins; i += kTopkThreads) h[i] = 0;
     __syncthreads();
-    // scores of one row share their high bits, so in the first passes whole warps often
-    // hit one bin: then a single lane adds 32
-    for (int base = 0; base < n; base += kTopkThreads) {
-      const int i = base + tid;
-      int bin = 256;  // not a candidate
-      if (i < n) {
-        const uint32_t u = cached ? cache[i] : order_key(__ldg(row + i));
-        if ((u & mask) == prefix) bin = static_cast<int>((u >> shift) & 0xffu);
-      }
-      const int b0 = __shfl_sync(0xffffffffu, bin, 0);
-      if (__all_sync(0xffffffffu, bin == b0)) {
-        if ((tid & 31) == 0 && b0 < 256) atomicAdd(&hist[b0], 32);
-      } else if (bin < 256) {
-        atomicAdd(&hist[bin], 1);
+    for (int i4 = tid; i4 < n4; i4 += kTopkThreads) {
+      const uint4 v = key4(i4);
+      const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t rel = kk[j] - umin;
+        const uint32_t top = hi_shift >= 32 ? 0u : rel >> hi_shift;
+        if (4 * i4 + j < ns && top == pfx) atomicAdd(&h[(rel >> shift) & bmask], 1);
       }
     }
-    __syncthreads();
-    if (tid < 32) {
-      // lane l owns bins 255-8l .. 248-8l (descending); find the bin where the count
-      // from the top reaches `remaining`
-      int c[8];
-      int sum = 0;
+    cl.sync();  // every CTA's histogram of this pass is complete
+    // thread t owns bins 2047 - 2t and 2046 - 2t (descending); sum them over the cluster
+    // in rank order
+    int v0[kMaxCluster], v1[kMaxCluster];  // every remote load in flight before the sums
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        c[i] = hist[255 - 8 * tid - i];
-        sum += c[i];
+    for (int r = 0; r < kMaxCluster; ++r) {
+      v0[r] = v1[r] = 0;
+      if (r < C) {
+        const int* hr = cl.map_shared_rank(h, r);
+        v0[r] = hr[kBins - 1 - 2 * tid];
+        v1[r] = hr[kBins - 2 - 2 * tid];
       }
-      int incl = sum;
+    }
+    int c0 = 0, c1 = 0;
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      c0 += v0[r];
+      c1 += v1[r];
+    }
+    // exclusive prefix over the threads (= over the bins from the top)
+    const int sm = c0 + c1;
+    int incl = sm;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int wv = s_wsum[lane], wi = wv;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (tid >= o) incl += v;
+        const int v = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += v;
       }
-      const int excl = incl - sum;
-      if (excl < remaining && incl >= remaining) {
-        int acc = excl;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (acc + c[i] >= remaining) {
-            s_prefix = prefix | (static_cast<uint32_t>(255 - 8 * tid - i) << shift);
-            s_remaining = remaining - acc;
-            break;
-          }
-          acc += c[i];
-        }
-      }
+      s_wsum[lane] = wi - wv;  // exclusive over the warps
     }
     __syncthreads();
-    prefix = s_prefix;
+    const int excl = s_wsum[warp] + incl - sm;
+    if (excl < remaining && excl + sm >= remaining) {
+      const bool hi = excl + c0 >= remaining;
+      const uint32_t bin = static_cast<uint32_t>(hi ? kBins - 1 - 2 * tid : kBins - 2 - 2 * tid);
+      s_prefix = (pfx << w) | bin;
+      s_remaining = hi ? remaining - excl : remaining - excl - c0;
+    }
+    __syncthreads();
+    pfx = s_prefix;
     remaining = s_remaining;
-    mask |= 0xffu << shift;
+    ++pass;
   }
-  // keys > T are all taken (K - need of them); of the keys == T the first `need` in index
-  // order.  Warp w owns the contiguous segment [w * seg, (w + 1) * seg): it counts its keys
-  // > T and == T, the counts of the warps before it give its first tie rank and output
-  // slot, and it writes its selections in index order with warp ballots.
-  const uint32_t T = prefix;
+  const uint32_t T = umin + pfx;
   const int need = remaining;
-  const int lane = tid & 31, warp = tid >> 5;
-  const int seg = (n + kTopkWarps - 1) / kTopkWarps;
-  const int lo = min(n, warp * seg), hi = min(n, lo + seg);
+  // keys > T are all taken (K - need of them); of the keys == T the first `need` in index
+  // order.  Counts of the CTAs before this one give its first tie rank and output slot;
+  // within the CTA, warp w owns the contiguous piece [w * wseg, (w + 1) * wseg).
+  const int wseg4 = (n4 + kTopkWarps - 1) / kTopkWarps;  // in groups of 4 keys
+  const int lo4 = min(n4, warp * wseg4), hi4 = min(n4, lo4 + wseg4);
   int gt_c = 0, eq_c = 0;
-  for (int i = lo + lane; i < hi; i += 32) {
-    const uint32_t u = cached ? cache[i] : order_key(__ldg(row + i));
-    gt_c += u > T;
-    eq_c += u == T;
+  for (int i4 = lo4 + lane; i4 < hi4; i4 += 32) {
+    const uint4 v = key4(i4);
+    const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const bool valid = 4 * i4 + j < ns;
+      gt_c += valid && kk[j] > T;
+      eq_c += valid && kk[j] == T;
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     gt_c += __shfl_xor_sync(0xffffffffu, gt_c, o);
     eq_c += __shfl_xor_sync(0xffffffffu, eq_c, o);
   }
-  __shared__ int s_gt[kTopkWarps], s_eq[kTopkWarps];
   if (lane == 0) {
     s_gt[warp] = gt_c;
     s_eq[warp] = eq_c;
   }
   __syncthreads();
+  if (tid == 0) {
+    int g = 0, e = 0;
+    for (int w = 0; w < kTopkWarps; ++w) {
+      g += s_gt[w];
+      e += s_eq[w];
+    }
+    s_cnt[0] = g;
+    s_cnt[1] = e;
+  }
+  cl.sync();  // every CTA's counts are published
   int eq_rank = 0, pos = 0;
+  for (int r = 0; r < rank; ++r) {
+    const int* cr = cl.map_shared_rank(s_cnt, r);
+    pos += cr[0] + min(max(need - eq_rank, 0), cr[1]);
+    eq_rank += cr[1];
+  }
   for (int w = 0; w < warp; ++w) {
     pos += s_gt[w] + min(max(need - eq_rank, 0), s_eq[w]);
     eq_rank += s_eq[w];
   }
-  const uint32_t below = (1u << lane) - 1u;
-  for (int base = lo; base < hi; base += 32) {
-    const int i = base + lane;
-    const bool valid = i < hi;
-    const uint32_t u = valid ? (cached ? cache[i] : order_key(__ldg(row + i))) : 0u;
-    const bool eq = valid && u == T;
-    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-    const bool sel = valid && (u > T || (eq && eq_rank + __popc(eqm & below) < need));
-    const uint32_t selm = __ballot_sync(0xffffffffu, sel);
-    if (sel) out[pos + __popc(selm & below)] = i;
-    eq_rank += __popc(eqm);
-    pos += __popc(selm);
+  cl.sync();  // no CTA leaves while another still reads its counts
+  // 128 keys per step, 4 consecutive ones per lane: ties are ranked in index order within
+  // the lane, then across the lanes (exclusive warp scans), then across the steps
+  for (int base4 = lo4; base4 < hi4; base4 += 32) {
+    const int i4 = base4 + lane;
+    const uint4 v = i4 < hi4 ? key4(i4) : make_uint4(0, 0, 0, 0);
+    const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+    bool gt[4], eq[4];
+    int ne = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const bool valid = i4 < hi4 && 4 * i4 + j < ns;
+      gt[j] = valid && kk[j] > T;
+      eq[j] = valid && kk[j] == T;
+      ne += eq[j];
+    }
+    int eb = ne;  // inclusive scan of the lanes' tie counts
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, eb, o);
+      if (lane >= o) eb += t;
+    }
+    const int eq_all = __shfl_sync(0xffffffffu, eb, 31);
+    eb -= ne;
+    bool sel[4];
+    int nsel = 0, er = eq_rank + eb;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      sel[j] = gt[j] || (eq[j] && er < need);
+      er += eq[j];
+      nsel += sel[j];
+    }
+    int sb = nsel;  // inclusive scan of the lanes' selection counts
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, sb, o);
+      if (lane >= o) sb += t;
+    }
+    const int sel_all = __shfl_sync(0xffffffffu, sb, 31);
+    int at = pos + sb - nsel;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (sel[j]) out[at++] = s0 + 4 * i4 + j;
+    eq_rank += eq_all;
+    pos += sel_all;
   }
 }
 
 cudaError_t launch_topk(const lc_topk_args& a, bool /*decode*/, cudaStream_t st) {
   if (a.n_q == 0) return cudaSuccess;
-  const int use_cache = a.max_ent <= kRowCache ? 1 : 0;
-  const size_t sm = use_cache ? static_cast<size_t>(a.max_ent) * 4 : 0;
+  // the largest cluster that keeps the rows within one wave (one 1024-thread CTA per SM),
+  // and at least the one whose segments fit the key cache
+  int C = 1;
+  while (C < kMaxCluster &&
+         (static_cast<int64_t>(a.n_q) * 2 * C <= 148 || (a.max_ent + C - 1) / C > kRowCache))
+    C <<= 1;
+  const int segl = ((a.max_ent + C - 1) / C + 3) & ~3;
+  const int use_cache = segl <= kRowCache ? 1 : 0;
+  const size_t sm = use_cache ? static_cast<size_t>(segl) * 4 : 0;
   cudaFuncSetAttribute(k_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kRowCache * 4));
-  k_topk<<<a.n_q, kTopkThreads, sm, st>>>(a, use_cache);
-  return cudaGetLastError();
+  const int64_t ctas = static_cast<int64_t>(a.n_q) * C;
+  if (ctas > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+  cfg.blockDim = dim3(kTopkThreads);
+  cfg.dynamicSmemBytes = sm;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_topk, a, use_cache);
 }
 
 }  // namespace lc
