@@ -412,41 +412,55 @@ __global__ void __launch_bounds__(MT * DS * 32, 1)
 
 // Merge the key splits of each (query, head) with the sink, in split order.  Split c of
 // row (q * H + h) left its unnormalised O at ws_o row c * n_q * H + q * H + h and its
-// (max, sum) at ws_ml[2 ((q * H + h) * n_split + c)].
-// grid: ceil(n_q * H / 8); one warp per (query, head).
-__global__ void __launch_bounds__(256) k_attn_combine(lc_attn_args a, int n_split, const float* __restrict__ ws_o,
-                                                      const float* __restrict__ ws_ml) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  if (row >= static_cast<int64_t>(a.n_q) * a.dims.H) return;
+// (max, sum) at ws_ml[2 ((q * H + h) * n_split + c)].  One thread per (row, 4 dims): the
+// loads of all splits are independent, so they are in flight together.
+constexpr int kCombineThreads = 256;
+constexpr int kQuads = kAD / 4;  // float4 groups per row
+
+__global__ void __launch_bounds__(kCombineThreads) k_attn_combine(lc_attn_args a, int n_split,
+                                                                  const float* __restrict__ ws_o,
+                                                                  const float* __restrict__ ws_ml) {
+  const int64_t rows = static_cast<int64_t>(a.n_q) * a.dims.H;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kCombineThreads + threadIdx.x;
+  if (t >= rows * kQuads) return;
+  const int64_t row = t / kQuads;
+  const int c4 = static_cast<int>(t % kQuads);
   const int h = static_cast<int>(row % a.dims.H);
   const float sk = __ldg(a.sink + h) * 1.4426950408889634f;
+  const float2* ml = reinterpret_cast<const float2*>(ws_ml) + row * n_split;
   float M = sk;
-  for (int c = 0; c < n_split; ++c) M = fmaxf(M, __ldg(ws_ml + 2 * (row * n_split + c)));
+  for (int c = 0; c < n_split; ++c) M = fmaxf(M, __ldg(ml + c).x);
   float Z = exp2f(sk - M);
-  float o[kAD / 32];
-#pragma unroll
-  for (int i = 0; i < kAD / 32; ++i) o[i] = 0.f;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4* src = reinterpret_cast<const float4*>(ws_o) + row * kQuads + c4;
+  const int64_t split_stride = rows * kQuads;
+#pragma unroll 4
   for (int c = 0; c < n_split; ++c) {
-    const float mc = __ldg(ws_ml + 2 * (row * n_split + c));
-    if (mc == -INFINITY) continue;
-    const float w = exp2f(mc - M);
-    Z = fmaf(__ldg(ws_ml + 2 * (row * n_split + c) + 1), w, Z);
-    const float* src = ws_o + (static_cast<int64_t>(c) * a.n_q * a.dims.H + row) * kAD;
-#pragma unroll
-    for (int i = 0; i < kAD / 32; ++i) o[i] = fmaf(__ldg(src + i * 32 + lane), w, o[i]);
+    const float2 mc = __ldg(ml + c);
+    const float4 v = __ldg(src + c * split_stride);
+    const float w = mc.x == -INFINITY ? 0.f : exp2f(mc.x - M);
+    Z = fmaf(mc.y, w, Z);
+    o.x = fmaf(v.x, w, o.x);
+    o.y = fmaf(v.y, w, o.y);
+    o.z = fmaf(v.z, w, o.z);
+    o.w = fmaf(v.w, w, o.w);
   }
   const float inv = 1.f / Z;
   if (a.out_fmt == LC_FMT_BF16) {
-    uint16_t* dst = static_cast<uint16_t*>(a.out) + row * kAD;
-#pragma unroll
-    for (int i = 0; i < kAD / 32; ++i) dst[i * 32 + lane] = f32_to_bf16_bits(o[i] * inv);
+    uint2 pk;
+    pk.x = pack_bf16(o.x * inv, o.y * inv);
+    pk.y = pack_bf16(o.z * inv, o.w * inv);
+    reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + row * kAD)[c4] = pk;
   } else {
-    float* dst = static_cast<float*>(a.out) + row * kAD;
-#pragma unroll
-    for (int i = 0; i < kAD / 32; ++i) dst[i * 32 + lane] = o[i] * inv;
+    reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * kAD)[c4] =
+        make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
   }
-  if (a.lse && lane == 0) a.lse[row] = (M + log2f(Z)) * 0.6931471805599453f;
+  if (a.lse && c4 == 0) a.lse[row] = (M + log2f(Z)) * 0.6931471805599453f;
+}
+
+static unsigned combine_blocks(const lc_attn_args& a) {
+  const int64_t n = static_cast<int64_t>(a.n_q) * a.dims.H * kQuads;
+  return static_cast<unsigned>((n + kCombineThreads - 1) / kCombineThreads);
 }
 
 // ---------------------------------------------------------------------------------
@@ -514,8 +528,7 @@ static cudaError_t launch_mma(const lc_attn_args& a, bool sparse, const AttnGeom
   k_attn_mma<MT, DS, TK, NBUF><<<grid, MT * DS * 32, sm, st>>>(a, sparse ? 1 : 0, g, ws_o, ws_ml);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || g.n_split == 1) return e;
-  const int64_t rows = static_cast<int64_t>(a.n_q) * a.dims.H;
-  k_attn_combine<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(a, g.n_split, ws_o, ws_ml);
+  k_attn_combine<<<combine_blocks(a), kCombineThreads, 0, st>>>(a, g.n_split, ws_o, ws_ml);
   return cudaGetLastError();
 }
 
@@ -524,8 +537,7 @@ static cudaError_t launch_mma(const lc_attn_args& a, bool sparse, const AttnGeom
 cudaError_t launch_attn_combine(const lc_attn_args& a, int n_split, cudaStream_t st) {
   float* ws_o = static_cast<float*>(a.workspace);
   float* ws_ml = ws_o + static_cast<size_t>(a.n_q) * a.dims.H * n_split * kAD;
-  const int64_t rows = static_cast<int64_t>(a.n_q) * a.dims.H;
-  k_attn_combine<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(a, n_split, ws_o, ws_ml);
+  k_attn_combine<<<combine_blocks(a), kCombineThreads, 0, st>>>(a, n_split, ws_o, ws_ml);
   return cudaGetLastError();
 }
 
