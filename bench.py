@@ -273,7 +273,11 @@ def run_lc(args):
     pk, pk_kind = peaks()
     runs = make_runs(args.workload, dev, rank, {"auto": 0, "mma": 1, "tc": 2, "ref": 3}[args.attn_impl])
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
+    # the critical path (index -> top-k -> attention) on a high-priority stream, made current
+    # so that the L2 flush and the host copies stay ordered with it; the side stream fills
+    # the SMs it leaves idle
+    stream = torch.cuda.Stream(dev, priority=-100)
+    torch.cuda.set_stream(stream)
 
     def barrier():
         if world > 1:
@@ -289,7 +293,7 @@ def run_lc(args):
     stage_names = [f"{i}:{n}" for i, (_, _, r) in enumerate(runs) for n, _ in r.stages()]
     # kernels per step: one per call, plus the combine kernel of a key-split attention
     n_launch = len(stage_names) + sum(1 for (_, _, r) in runs if r.a_attn.workspace_bytes > 0)
-    side = torch.cuda.Stream(dev)
+    side = torch.cuda.Stream(dev, priority=0)
 
     def one_step(stage_ev=None):
         """The whole path once: per workload, preparation and compression on the side

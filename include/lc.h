@@ -196,6 +196,9 @@ typedef struct lc_index_args {
   const uint8_t* q_scale;  /* MXFP4: [n_q, H_I, d_I/32], 4-byte aligned */
   const void* k;           /* F32 [n_keys, d_I] or MXFP4 codes [n_keys, d_I/2] */
   const uint8_t* k_scale;  /* MXFP4: [n_keys, d_I/32], 4-byte aligned */
+  int64_t n_keys;          /* rows of k and k_scale (every ent_start[b] + n_ent[b] <= n_keys);
+                              MXFP4 requires it: the tensor-core path reads whole 128-key
+                              tiles by bulk copy and must not read past the arrays */
   const float* w;          /* head weights, >= 0: [H_I], or [n_q, H_I] if w_qstride = H_I */
   int32_t w_qstride;       /* 0 (shared) or H_I */
   int32_t m;

@@ -426,6 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int code_next = pt < kTK ? slot_code(s_begin + pt) : -1;
     for (int t = 0; t < n_tiles; ++t) {
       const int st = t & 1;
+      // stage st (and its key codes) is free once O(t - 2) is done: that also means the
+      // softmax of tile t - 2 has read the codes
       const bool ok = t < 2 || wait(&bars.kempty[st], ((t >> 1) - 1) & 1);
       if (ok && pt < kTK) kcode[st * kTK + pt] = code_next;
       if (named_bar_or(2, 128, !ok)) break;  // the role stops as one
@@ -638,24 +640,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 5; ++c) {
         // chunk c < 4: lane L -> dim 128 c + L; chunk 4 (M = 64): lane 32 w + i -> dim 512 + 16 w + i
         const int dim = c < 4 ? c * 128 + warp * 32 + lane : (lane < 16 ? 512 + warp * 16 + lane : -1);
-#pragma unroll 1
-        for (int hh = 0; hh < kNR; hh += 32) {
-          uint32_t ov[32];
-          if (n_tiles > 0) {
-            tmem_ld32(tm + lane_off + kColO + c * kNR + hh, ov);
-            tmem_wait_ld();
-          } else {
+        uint32_t ov[kNR];  // the chunk's 64 head columns, one wait
+        if (n_tiles > 0) {
+          tmem_ld32(tm + lane_off + kColO + c * kNR, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
+          tmem_ld32(tm + lane_off + kColO + c * kNR + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = 0;
-          }
-          if (dim < 0) continue;
+          for (int i = 0; i < kNR; ++i) ov[i] = 0;
+        }
+        if (dim < 0) continue;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float v = __uint_as_float(ov[i]);
-            if (geo.n_split == 1) v *= s_f[hh + i];
-            if (f32) stf[(hh + i) * kD + dim] = v;
-            else sth[(hh + i) * kD + dim] = f32_to_bf16_bits(v);
-          }
+        for (int i = 0; i < kNR; ++i) {
+          float v = __uint_as_float(ov[i]);
+          if (geo.n_split == 1) v *= s_f[i];
+          if (f32) stf[i * kD + dim] = v;
+          else sth[i * kD + dim] = f32_to_bf16_bits(v);
         }
       }
       fence_async_smem();

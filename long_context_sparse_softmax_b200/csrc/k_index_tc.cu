@@ -4,22 +4,31 @@
 // p ("解读 DeepSeek V4", CSA section and "FP4 Quantization-Aware Training": the indexer QK
 // path runs in MXFP4; "DeepSeek-V4 论文分析" §5.3, §8.3).
 //
-// One MMA tile: A = 128 keys x d_I (K-major E2M1, 2 per byte) in shared memory, B = the H_I
-// heads of QPC queries (N = QPC * H_I <= 256), block scales (E8M0, one per 32 elements) in
-// tensor memory, D = 128 x N FP32 in tensor memory.  The tensor core applies the block
-// scales; the operands are the caller's bytes, never widened or converted.
+// One MMA tile: A = 128 keys x 128 dims (E2M1, 2 per byte: 64 bytes per key), B = the H_I
+// heads of QPC queries (N = QPC * H_I), block scales (E8M0, one per 32 elements) in tensor
+// memory, D = 128 x N FP32 in tensor memory.  The tensor core applies the block scales;
+// the operands are the caller's bytes, never widened or converted.
 //
-//   * shared layout: no-swizzle K-major core matrices, 8 rows x 16 bytes each, 128 bytes
-//     apart along K (LBO) and 512 bytes apart along rows (SBO); a 128 x 128 FP4 tile is 8 KB;
-//   * scale factors in tensor memory: column c holds, in lane L (all four lane quadrants),
-//     the four E8M0 bytes (K blocks 0..3) of row (L % 32) + 32 c; the k-th K = 64 MMA reads
-//     bytes 2k, 2k+1 (sf_id = 2k);
-//   * key tiles stream through three shared buffers with cp.async, two tiles ahead;
-//   * epilogue: thread t of the 128 owns key row t of D (tcgen05.ld 32x32b), so the
-//     ReLU-weighted head sum stays in registers, in a fixed order.
+//   * A tile of 128 consecutive keys is one 2-D bulk tensor copy (TMA) of 8 KB, written
+//     with the 64-byte swizzle that is the MMA's K-major SWIZZLE_64B layout (8-row groups
+//     512 bytes apart; the second K = 64 step starts 32 bytes into the rows).  The query
+//     operand is copied once per CTA into the same layout;
+//   * block scales in tensor memory: column c holds, in lane L of every lane quadrant, the
+//     four E8M0 bytes (K blocks 0..3) of row (L % 32) + 32 c; the k-th K = 64 MMA reads
+//     bytes 2k, 2k + 1 (sf_id = 2k);
+//   * warp roles (192 threads): warp 0 loads key tiles (TMA) and their scale words (one
+//     tile ahead, into registers; stored as 32 rows x 16 bytes, row L holding the words
+//     of keys L, L + 32, L + 64, L + 96) into a 4-stage ring; lane 0 of warp 1 copies a
+//     tile's scales into tensor memory (tcgen05.cp 32x128b.warpx4, which fills every
+//     lane quadrant) and issues its MMAs into one of three accumulators; warps 2-5 run the
+//     epilogue: thread t owns key row t of D (tcgen05.ld 32x32b), so the ReLU-weighted
+//     head sum stays in registers (8 partial sums of heads h = k mod 8, added in a fixed
+//     order).
 //
-// Every wait on the tensor core is bounded: after ~2^26 polls the kernel records
-// LC_DEV_TIMEOUT in the status word, stops issuing work, and releases its tensor memory.
+// The roles meet only at mbarriers.  Every wait is bounded: after ~2^26 polls a role
+// records LC_DEV_TIMEOUT in the status word and sets an abort flag that stops the others.
+#include <cuda.h>
+
 #include "lc_internal.h"
 
 namespace lc {
@@ -30,44 +39,56 @@ constexpr int kKeys = 128;          // keys per tile (MMA M)
 constexpr int kDI = 128;            // indexer dims handled here (2 MMAs of K = 64)
 constexpr int kRowB = kDI / 2;      // bytes per row
 constexpr int kTileB = kKeys * kRowB;
-constexpr int kStages = 3;
-constexpr long kSpinLimit = 1L << 26;
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr long kSpin = 1L << 26;
+constexpr int kDBuf = 3;            // tensor-memory accumulators
+constexpr uint32_t kColSfa = 0;     // offsets past the accumulators
+constexpr uint32_t kColSfb = 16;
 
 __device__ __forceinline__ uint32_t su32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
-// byte offset of (row, byte) in the core-matrix layout
-__device__ __forceinline__ uint32_t cm_off(int r, int b) {
-  return (r >> 3) * 512 + (b >> 4) * 128 + (r & 7) * 16 + (b & 15);
-}
-
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+// K-major SWIZZLE_64B operand: 64-byte rows, 8-row groups 512 bytes apart
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t addr) {
   uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFF);
-  d |= static_cast<uint64_t>(128 >> 4) << 16;   // LBO: next core matrix along K
-  d |= static_cast<uint64_t>(512 >> 4) << 32;   // SBO: next 8-row group
-  d |= static_cast<uint64_t>(1) << 46;          // descriptor version for sm_100
-  return d;                                     // base offset 0, no swizzle
+  d |= static_cast<uint64_t>(1) << 16;               // LBO (unused by swizzled K-major)
+  d |= static_cast<uint64_t>(512 >> 4) << 32;        // SBO: next 8-row group
+  d |= static_cast<uint64_t>(1) << 46;               // descriptor version for sm_100
+  d |= static_cast<uint64_t>(4) << 61;               // layout: SWIZZLE_64B
+  return d;
 }
+// byte offset of 16-byte chunk c of row r in a SWIZZLE_64B tile (512-byte aligned base)
+__device__ __forceinline__ uint32_t sw64_off(int r, int c) { return r * 64 + ((c ^ ((r >> 1) & 3)) << 4); }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
 }
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst), "l"(src), "r"(valid ? 4 : 0));
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  uint32_t done = 0;
-  for (long it = 0; it < kSpinLimit; ++it) {
-    asm volatile(
-        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(bar), "r"(parity));
-    if (done) return true;
-  }
-  return false;
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile("{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+               : "=r"(done)
+               : "r"(bar), "r"(parity)
+               : "memory");
+  return done != 0;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n"); }
@@ -78,8 +99,8 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b,
                "r"(d));
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
+// 32 columns of this warp's lanes, without waiting (tcgen05.wait::ld before use)
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
       "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
@@ -88,26 +109,36 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
         "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+
+
+struct IdxBars {
+  uint64_t kfull[kStages];   // key tile (expect-tx arrival) and its scale words (32 arrivals) landed
+  uint64_t kempty[kStages];  // MMAs of the tile done (commit)
+  uint64_t dfull[kDBuf];     // accumulator written (commit)
+  uint64_t dempty[kDBuf];    // accumulator read (128 arrivals)
+  uint64_t bfull;            // query operand, its scales and the head weights ready (128 arrivals)
+  uint64_t fin;              // every MMA complete (commit)
+};
 
 }  // namespace
 
-// grid: (query chunks of QPC queries, key-range chunks); 128 threads.
-// TMEM columns: D [0, N), SFA [N, N + 4), SFB [N + 8, N + 8 + N / 32).
+// grid: (query chunks of QPC queries, key-range chunks); 192 threads.
+// Tensor memory: accumulators at columns [k N, (k + 1) N), k < 3; key scales at 3N + {0, 8};
+// query scales at 3N + 16 (N / 32 columns).
 template <int QPC>
-__global__ void __launch_bounds__(128) k_index_tc(lc_index_args a, int tiles_per_cta, uint32_t tmem_cols) {
+__global__ void __launch_bounds__(kThreads, 1)
+    k_index_tc(const __grid_constant__ CUtensorMap tk, lc_index_args a, int tiles_per_cta, uint32_t tmem_cols) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int H = a.H_I;
   const int N = QPC * H;
-  uint8_t* As = smem;                                               // [kStages][kTileB]
-  uint8_t* Bs = As + kStages * kTileB;                              // [N rows][64 B] core matrices
+  uint8_t* As = smem;                                               // [kStages][kTileB], SWIZZLE_64B
+  uint8_t* Bs = As + kStages * kTileB;                              // [N rows][64 B], SWIZZLE_64B
   uint32_t* SFs = reinterpret_cast<uint32_t*>(Bs + N * kRowB);      // [kStages][128] key scale words
   float* ws = reinterpret_cast<float*>(SFs + kStages * kKeys);      // [N] head weights
   __shared__ uint32_t s_tmem;
-  __shared__ __align__(8) uint64_t s_mbar;
+  __shared__ int s_abort;
+  __shared__ __align__(8) IdxBars bars;
   __shared__ int s_nv[QPC];
   __shared__ int s_q[QPC];
 
@@ -119,7 +150,6 @@ __global__ void __launch_bounds__(128) k_index_tc(lc_index_args a, int tiles_per
   const int n_ent = __ldg(a.batch.n_ent + b);
   // queries of this chunk: they must belong to sequence b (prefill: one sequence;
   // decode: QPC = 1)
-  int nv_max = 0;
   if (tid < QPC) {
     const int q = qa + tid;
     int nv = 0;
@@ -131,193 +161,273 @@ __global__ void __launch_bounds__(128) k_index_tc(lc_index_args a, int tiles_per
     s_q[tid] = q;
   }
   __syncthreads();
+  int nv_max = 0;
 #pragma unroll
   for (int i = 0; i < QPC; ++i) nv_max = max(nv_max, s_nv[i]);
   const int t_begin = blockIdx.y * tiles_per_cta;
   const int t_end = min(t_begin + tiles_per_cta, (nv_max + kKeys - 1) / kKeys);
-  if (t_begin >= t_end) return;
+  if (t_begin >= t_end) return;  // uniform over the CTA: nothing allocated yet
+  const int n_tiles = t_end - t_begin;
 
-  // query operand B (rows n = i * H + h), its scales, head weights
-  for (int c = tid; c < N * 4; c += 128) {
-    const int n = c >> 2, seg = c & 3;
-    const int i = n / H, h = n % H;
-    const int q = s_q[i];
-    const bool ok = q < a.n_q && s_nv[i] > 0;
-    const uint8_t* src = static_cast<const uint8_t*>(a.q) + (static_cast<int64_t>(ok ? q : 0) * H + h) * kRowB + seg * 16;
-    cp_async16(su32(Bs + cm_off(n, seg * 16)), src, ok);
-  }
-  for (int u = tid; u < N; u += 128) {
-    const int i = u / H, h = u % H;
-    ws[u] = __ldg(a.w + static_cast<int64_t>(s_q[i] < a.n_q ? s_q[i] : 0) * a.w_qstride + h);
-  }
-  cp_async_commit();
-
-  auto load_tile = [&](int t, int stage) {
-    const int j0 = t * kKeys;
-    uint8_t* dst = As + stage * kTileB;
-    for (int c = tid; c < kKeys * 4; c += 128) {
-      const int r = c >> 2, seg = c & 3;
-      const int j = j0 + r;
-      const bool ok = j < n_ent;
-      const uint8_t* src = static_cast<const uint8_t*>(a.k) + (kbase + (ok ? j : 0)) * kRowB + seg * 16;
-      cp_async16(su32(dst + cm_off(r, seg * 16)), src, ok);
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    const uint32_t addr = su32(bar);
+    for (long it = 0; it < kSpin; ++it) {
+      if (mbar_test(addr, parity)) return true;
+      if ((it & 1023) == 1023 && *reinterpret_cast<volatile int*>(&s_abort)) return false;
     }
-    {  // the 4 scale bytes of key row tid (4-byte aligned: a sequence may start anywhere)
-      const int j = j0 + tid;
-      const bool ok = j < n_ent;
-      const uint8_t* src = a.k_scale + (kbase + (ok ? j : 0)) * 4;
-      cp_async4(su32(SFs + stage * kKeys + tid), src, ok);
-    }
+    set_status(a.status, LC_DEV_TIMEOUT);
+    atomicExch(&s_abort, 1);
+    return false;
   };
 
-  // tensor memory
-  if (warp == 0) {
+  if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(su32(&s_tmem)),
                  "r"(tmem_cols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
   }
   if (tid == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(su32(&s_mbar)));
+    s_abort = 0;
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(su32(&bars.kfull[i]), 1 + 32);
+      mbar_init(su32(&bars.kempty[i]), 1);
+    }
+    for (int i = 0; i < kDBuf; ++i) {
+      mbar_init(su32(&bars.dfull[i]), 1);
+      mbar_init(su32(&bars.dempty[i]), 128);
+    }
+    mbar_init(su32(&bars.bfull), 128);
+    mbar_init(su32(&bars.fin), 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n");
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tk)) : "memory");
   }
-  load_tile(t_begin, 0);
-  cp_async_commit();
-  if (t_begin + 1 < t_end) load_tile(t_begin + 1, 1);
-  cp_async_commit();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = s_tmem;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t col_sfa = static_cast<uint32_t>(N), col_sfb = static_cast<uint32_t>(N + 8);
+  const uint32_t col_sfa = kDBuf * N + kColSfa, col_sfb = kDBuf * N + kColSfb;
 
-  // query scales -> tensor memory (lane L of every quadrant, column c: row (L % 32) + 32 c)
-  {
-    uint32_t v[8];
+  if (warp == 0) {
+    // ================= loads: key tiles (TMA) and their scale words =================
+    // words of tile it: keys lane + 32 c (4-byte aligned: a sequence may start anywhere)
+    auto sf_load = [&](int it, uint32_t (&w)[4]) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int n = lane + 32 * c;
-      uint32_t w = 0x7f7f7f7fu;
-      if (n < N) {
-        const int i = n / H, h = n % H;
-        const int q = s_q[i];
-        if (q < a.n_q) w = __ldg(reinterpret_cast<const uint32_t*>(a.q_scale) + static_cast<int64_t>(q) * H + h);
+      for (int c = 0; c < 4; ++c) {
+        const int j = (t_begin + it) * kKeys + lane + 32 * c;
+        w[c] = j < n_ent ? __ldg(reinterpret_cast<const uint32_t*>(a.k_scale + (kbase + j) * 4)) : 0u;
       }
-      v[c] = w;
+    };
+    uint32_t sfw[4];
+    sf_load(0, sfw);
+    for (int it = 0; it < n_tiles; ++it) {
+      const int s = it % kStages;
+      const int t = t_begin + it;
+      if (it >= kStages && !__all_sync(0xffffffffu, wait(&bars.kempty[s], ((it / kStages) - 1) & 1))) break;
+      const uint32_t full = su32(&bars.kfull[s]);
+      if (lane == 0) {
+        mbar_expect_tx(full, kTileB);
+        tma_load_2d(su32(As + s * kTileB), &tk, 0, static_cast<int>(kbase + static_cast<int64_t>(t) * kKeys), full);
+      }
+      *reinterpret_cast<uint4*>(SFs + s * kKeys + 4 * lane) = make_uint4(sfw[0], sfw[1], sfw[2], sfw[3]);
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // the tensor core reads them
+      mbar_arrive(full);
+      if (it + 1 < n_tiles) sf_load(it + 1, sfw);
     }
-    tmem_st4(tm + lane_off + col_sfb, v[0], v[1], v[2], v[3]);
-    if (N > 128) tmem_st4(tm + lane_off + col_sfb + 4, v[4], v[5], v[6], v[7]);
-  }
-
-  // instruction descriptor: E2M1 x E2M1, E8M0 scales, FP32 accumulate, M = 128, N
-  const uint32_t idesc0 = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
-                          (static_cast<uint32_t>(kKeys >> 4) << 24);
-  bool alive = true;
-  uint32_t phase = 0;
-  for (int t = t_begin; t < t_end; ++t) {
-    const int it = t - t_begin;
-    const int stage = it % kStages;
-    if (t + 2 < t_end) load_tile(t + 2, (it + 2) % kStages);
-    cp_async_commit();
-    cp_async_wait<2>();  // tile t (and B) landed
-    asm volatile("fence.proxy.async.shared::cta;\n");
-    __syncthreads();
-    // key scales of this tile -> tensor memory
-    {
-      const uint32_t* sf = SFs + stage * kKeys;
-      tmem_st4(tm + lane_off + col_sfa, sf[lane], sf[lane + 32], sf[lane + 64], sf[lane + 96]);
-      asm volatile("tcgen05.wait::st.sync.aligned;\n");
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (tid == 0 && alive) {
-      const uint32_t a_base = su32(As + stage * kTileB), b_base = su32(Bs);
+  } else if (warp == 1) {
+    // ================= MMA issue (one lane) =================
+    if (lane == 0) {
+      // E2M1 x E2M1, E8M0 scales, FP32 accumulate, M = 128, N
+      const uint32_t idesc0 = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+                              (static_cast<uint32_t>(kKeys >> 4) << 24);
+      bool ok = wait(&bars.bfull, 0);
+      for (int it = 0; ok && it < n_tiles; ++it) {
+        const int s = it % kStages, slot = it % kDBuf, sfs = it & 1;
+        ok = wait(&bars.kfull[s], (it / kStages) & 1) &&
+             (it < kDBuf || wait(&bars.dempty[slot], ((it / kDBuf) - 1) & 1));
+        if (!ok) break;
+        tc_fence_after();
+        // the tile's key scales: 32 rows of 16 bytes -> lanes 0..31 of every quadrant,
+        // columns col_sfa + 8 sfs .. + 3
+        {
+          uint64_t d = static_cast<uint64_t>((su32(SFs + s * kKeys) >> 4) & 0x3FFF);
+          d |= static_cast<uint64_t>(16 >> 4) << 16;   // LBO (one 16-byte column)
+          d |= static_cast<uint64_t>(128 >> 4) << 32;  // SBO: next 8 rows
+          d |= static_cast<uint64_t>(1) << 46;
+          asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n" ::"r"(tm + col_sfa + 8u * sfs), "l"(d));
+        }
+        const uint32_t a_base = su32(As + s * kTileB), b_base = su32(Bs);
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const uint32_t sfid = 2u * k;
-        const uint32_t idesc = idesc0 | (sfid << 29) | (sfid << 4);
-        const uint64_t da = smem_desc(a_base + k * 256), db = smem_desc(b_base + k * 256);
-        asm volatile(
-            "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
-            "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(tm),
-            "l"(da), "l"(db), "r"(idesc), "r"(k), "r"((tm + col_sfa) | (sfid << 30)), "r"((tm + col_sfb) | (sfid << 30)));
+        for (int k = 0; k < 2; ++k) {
+          const uint32_t sfid = 2u * k;
+          const uint32_t idesc = idesc0 | (sfid << 29) | (sfid << 4);
+          asm volatile(
+              "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+              "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(
+                  tm + static_cast<uint32_t>(slot * N)),
+              "l"(sw64_desc(a_base + k * 32)), "l"(sw64_desc(b_base + k * 32)), "r"(idesc), "r"(k),
+              "r"((tm + col_sfa + 8u * sfs) | (sfid << 30)), "r"((tm + col_sfb) | (sfid << 30)));
+        }
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+            su32(&bars.dfull[slot])));
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+            su32(&bars.kempty[s])));
       }
       asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
-          su32(&s_mbar)));
+          su32(&bars.fin)));
+      wait(&bars.fin, 0);
     }
-    if (alive && !mbar_wait(su32(&s_mbar), phase)) {
-      alive = false;
-      set_status(a.status, LC_DEV_TIMEOUT);
+  } else {
+    // ================= warps 2-5: key scales into tensor memory, epilogue =================
+    const int et = tid - 64;                          // 0..127
+    const int quad = warp & 3;                        // tensor-memory lane quadrant of this warp
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const int row = quad * 32 + lane;                 // key row of D this thread reads
+    // query operand (rows n = i * H + h), head weights, query scales
+    for (int c = et; c < N * 4; c += 128) {
+      const int n = c >> 2, seg = c & 3;
+      const int i = n / H, h = n % H;
+      const int q = s_q[i];
+      const bool ok = q < a.n_q && s_nv[i] > 0;
+      const uint8_t* src = static_cast<const uint8_t*>(a.q) + (static_cast<int64_t>(ok ? q : 0) * H + h) * kRowB + seg * 16;
+      cp_async16(su32(Bs + sw64_off(n, seg)), src, ok);
     }
-    phase ^= 1u;
-    tc_fence_after();
-    if (alive) {
-      // epilogue: this thread's key row, the H columns of each query
-      const int j = t * kKeys + tid;
+    for (int u = et; u < N; u += 128) {
+      const int i = u / H, h = u % H;
+      ws[u] = __ldg(a.w + static_cast<int64_t>(s_q[i] < a.n_q ? s_q[i] : 0) * a.w_qstride + h);
+    }
+    {
+      uint32_t v[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int n = lane + 32 * c;
+        uint32_t w = 0x7f7f7f7fu;
+        if (n < N) {
+          const int i = n / H, h = n % H;
+          const int q = s_q[i];
+          if (q < a.n_q) w = __ldg(reinterpret_cast<const uint32_t*>(a.q_scale) + static_cast<int64_t>(q) * H + h);
+        }
+        v[c] = w;
+      }
+      tmem_st4(tm + lane_off + col_sfb, v[0], v[1], v[2], v[3]);
+      if (N > 128) tmem_st4(tm + lane_off + col_sfb + 4, v[4], v[5], v[6], v[7]);
+      asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+    }
+    asm volatile("cp.async.wait_all;\n" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    tc_fence_before();
+    mbar_arrive(su32(&bars.bfull));
+    __syncwarp();
+
+    // head weights in registers when one query's heads fill the accumulator (H <= 64);
+    // the other epilogue warps wrote part of them: wait for all 128 arrivals first
+    const bool weights_ok = __all_sync(0xffffffffu, wait(&bars.bfull, 0));
+    float wr[64];
+    if (QPC == 1) {
+#pragma unroll
+      for (int k = 0; k < 64; ++k) wr[k] = k < H ? ws[k] : 0.f;
+    }
+    auto epilogue = [&](int u) -> bool {
+      const int slot = u % kDBuf;
+      if (!__all_sync(0xffffffffu, wait(&bars.dfull[slot], (u / kDBuf) & 1))) return false;
+      tc_fence_after();
+      const int j = (t_begin + u) * kKeys + row;
 #pragma unroll
       for (int i = 0; i < QPC; ++i) {
-        float s = 0.f;
-        for (int h0 = 0; h0 < H; h0 += 32) {
-          float v[32];
-          tmem_ld32(tm + lane_off + static_cast<uint32_t>(i * H + h0), v);
+        // 8 partial sums (independent FMA chains), added in a fixed order
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int h0 = 0; h0 < H; h0 += 64) {  // H is a multiple of 32, at most 64 here
+          uint32_t v[64];
+          const uint32_t ta = tm + lane_off + static_cast<uint32_t>(slot * N + i * H + h0);
+          const int nh = min(64, H - h0);
+          tmem_ld32_async(ta, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+          if (nh > 32) tmem_ld32_async(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 #pragma unroll
-          for (int u = 0; u < 32; ++u) s = fmaf(ws[i * H + h0 + u], fmaxf(v[u], 0.f), s);
+          for (int k = 0; k < 64; ++k)
+            if (k < nh) {
+              const float w = QPC == 1 ? wr[k] : ws[i * H + h0 + k];
+              acc[k & 7] = fmaf(w, fmaxf(__uint_as_float(v[k]), 0.f), acc[k & 7]);
+            }
         }
+        const float s = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
         if (j < s_nv[i]) a.scores[static_cast<int64_t>(s_q[i]) * a.score_stride + j] = s;
       }
-    }
-    tc_fence_before();
-    __syncthreads();  // D and the tile's buffers are free again
+      tc_fence_before();
+      mbar_arrive(su32(&bars.dempty[slot]));
+      return true;
+    };
+    for (int u = 0; weights_ok && u < n_tiles; ++u)
+      if (!epilogue(u)) break;
   }
-  cp_async_wait<0>();
+  tc_fence_before();
+  __syncthreads();
   tc_fence_after();
-  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tm), "r"(tmem_cols));
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tm), "r"(tmem_cols));
 }
 
 bool index_tc_supported(const lc_index_args& a) {
-  return a.fmt == LC_IDX_MXFP4 && a.d_I == kDI && a.H_I % 32 == 0 && a.H_I <= 256;
+  return a.fmt == LC_IDX_MXFP4 && a.d_I == kDI && a.H_I % 32 == 0 && a.H_I <= 128 && a.n_keys > 0 &&
+         a.n_keys < (int64_t{1} << 31) && reinterpret_cast<uintptr_t>(a.k) % 16 == 0;
 }
 
+namespace {
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_tiled() {
+  static EncodeTiled fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiled>(nullptr);
+    return reinterpret_cast<EncodeTiled>(f);
+  }();
+  return fn;
+}
+
+}  // namespace
+
 cudaError_t launch_index_tc(const lc_index_args& a, bool decode, cudaStream_t st) {
+  const EncodeTiled enc = encode_tiled();
+  if (!enc) return cudaErrorNotSupported;
+  // the key codes as a [n_keys, 64 B] tensor; 128-row boxes, 64-byte swizzle; rows past
+  // n_keys read as zeros
+  CUtensorMap tk;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kRowB), static_cast<cuuint64_t>(a.n_keys)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kRowB)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kRowB), static_cast<cuuint32_t>(kKeys)};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a.k), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   const int H = a.H_I;
-  int qpc = 1;
-  if (!decode && a.batch.num_seqs == 1) qpc = (H <= 64) ? 2 : 1;
+  const int qpc = 1;  // three 64-column accumulators and the scales fit 256 columns: 2 CTAs per SM
   const int N = qpc * H;
   uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(N + 16)) cols <<= 1;
+  while (cols < static_cast<uint32_t>(kDBuf * N + 24)) cols <<= 1;
   const int tiles = (a.max_ent + kKeys - 1) / kKeys;
   const int n_qc = (a.n_q + qpc - 1) / qpc;
-  // decode: split each query's keys so that ~4 CTAs run per SM
+  const int per_sm = static_cast<int>(512 / cols);
   int tpc = tiles;
   if (decode) {
-    const int want = max(1, (4 * 148 + n_qc - 1) / n_qc);
+    // split each query's keys so that the CTAs fill the SMs once
+    const int want = max(1, (per_sm * 148) / n_qc);
     tpc = max(4, (tiles + want - 1) / want);
   } else {
-    tpc = max(1, min(tiles, 16));
+    tpc = max(1, min(tiles, 32));
   }
   const dim3 grid(n_qc, (tiles + tpc - 1) / tpc);
   size_t sm = static_cast<size_t>(kStages) * kTileB + static_cast<size_t>(N) * kRowB + kStages * kKeys * 4 +
-              static_cast<size_t>(N) * 4;
-  // ask for enough shared memory that no more CTAs share an SM than its 512 tensor-memory
-  // columns hold, so tcgen05.alloc never has to wait for another CTA
-  const size_t per_sm = 227 * 1024;
-  const size_t cap = per_sm / (512 / cols) - 2048;
+              static_cast<size_t>(N) * 4 + 1024;
+  // no more CTAs per SM than its 512 tensor-memory columns hold, so tcgen05.alloc never
+  // waits for another CTA
+  const size_t cap = 227 * 1024 / per_sm - 2048;
   if (sm < cap) sm = cap;
-  switch (qpc) {
-    case 1:
-      cudaFuncSetAttribute(k_index_tc<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
-      k_index_tc<1><<<grid, 128, sm, st>>>(a, tpc, cols);
-      break;
-    case 2:
-      cudaFuncSetAttribute(k_index_tc<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
-      k_index_tc<2><<<grid, 128, sm, st>>>(a, tpc, cols);
-      break;
-    default:
-      cudaFuncSetAttribute(k_index_tc<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
-      k_index_tc<4><<<grid, 128, sm, st>>>(a, tpc, cols);
-      break;
-  }
+  cudaFuncSetAttribute(k_index_tc<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
+  k_index_tc<1><<<grid, kThreads, sm, st>>>(tk, a, tpc, cols);
   return cudaGetLastError();
 }
 

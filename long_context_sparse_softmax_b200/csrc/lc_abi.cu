@@ -88,7 +88,7 @@ lc_status index_scores(const lc_index_args* a, void* stream, bool decode) {
   if (a->n_q == 0 || a->max_ent == 0) return LC_OK;
   LC_TRY(check_batch(a->batch, true, false));
   if (!a->q || !a->k || !a->w || !a->scores) return LC_ERR_ARG;
-  if (a->fmt == LC_IDX_MXFP4 && (!a->q_scale || !a->k_scale)) return LC_ERR_ARG;
+  if (a->fmt == LC_IDX_MXFP4 && (!a->q_scale || !a->k_scale || a->n_keys < 1)) return LC_ERR_ARG;
   if (a->fmt == LC_IDX_MXFP4 && ((reinterpret_cast<uintptr_t>(a->q_scale) | reinterpret_cast<uintptr_t>(a->k_scale)) & 3u))
     return LC_ERR_ALIGN;
   if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->scores)) return LC_ERR_ALIGN;

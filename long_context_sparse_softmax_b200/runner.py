@@ -89,7 +89,7 @@ class _Common:
         return IndexArgs(n_q, s.H_I, s.d_I, LC_IDX_MXFP4 if mx else LC_IDX_F32,
                          ptr(qI["codes"] if mx else qI["f32"]), ptr(qI.get("scales")),
                          ptr(kI["codes"] if mx else kI["f32"]), ptr(kI.get("scales")),
-                         ptr(inp["w"]), 0, s.m, self.W_x, max_ent, self.batch,
+                         (kI["codes"] if mx else kI["f32"]).shape[0], ptr(inp["w"]), 0, s.m, self.W_x, max_ent, self.batch,
                          ptr(scores), scores.shape[1], ptr(self.status))
 
     def _topk_args(self, n_q: int, max_ent: int) -> TopkArgs:
