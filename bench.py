@@ -48,8 +48,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0)
-    ap.add_argument("--attn-impl", default="auto", choices=["auto", "mma", "tc", "ref"],
-                    help="attention kernel (auto: tcgen05 where it applies, else mma.sync, else reference)")
+    ap.add_argument("--attn-impl", default="auto", choices=["auto", "mma", "tc", "ref", "tc16"],
+                    help="attention kernel (auto: tcgen05 where it applies, else mma.sync, else reference; tc16: the F16-score tcgen05 kernel)")
     return ap.parse_args()
 
 
@@ -271,7 +271,7 @@ def run_lc(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     pk, pk_kind = peaks()
-    runs = make_runs(args.workload, dev, rank, {"auto": 0, "mma": 1, "tc": 2, "ref": 3}[args.attn_impl])
+    runs = make_runs(args.workload, dev, rank, {"auto": 0, "mma": 1, "tc": 2, "ref": 3, "tc16": 4}[args.attn_impl])
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
     # the critical path (index -> top-k -> attention) on a high-priority stream, made current
     # so that the L2 flush and the host copies stay ordered with it; the side stream fills

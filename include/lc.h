@@ -271,18 +271,23 @@ typedef struct lc_attn_args {
   size_t workspace_bytes;
   int32_t* status;
   int32_t impl;            /* LC_IMPL_AUTO (0) picks the fastest kernel for the shape;
-                              LC_IMPL_MMA, LC_IMPL_TC, LC_IMPL_REF force one (results agree
+                              LC_IMPL_MMA, LC_IMPL_TC, LC_IMPL_REF, LC_IMPL_TC_F16 force one (results agree
                               within the BF16 tolerance; LC_ERR_UNSUPPORTED if it cannot run
                               the shape) */
-  int32_t reserved;
+  int32_t n_ent_rows;      /* rows of ent (every ent_start[b] + n_ent[b] <= n_ent_rows), or 0 if
+                              unknown; the FP8 tensor-core kernel reads entries by bulk tensor
+                              copies and needs it */
 } lc_attn_args;
 
 /* Attention kernels. */
 enum {
   LC_IMPL_AUTO = 0,
   LC_IMPL_MMA = 1,         /* BF16 mma.sync tiles (576-dim entries) */
-  LC_IMPL_TC = 2,          /* tcgen05 tiles, accumulators in tensor memory (576-dim entries) */
-  LC_IMPL_REF = 3          /* one warp per (query, head), FP32 CUDA cores (any shape) */
+  LC_IMPL_TC = 2,          /* tcgen05 tiles, accumulators in tensor memory (576-dim entries):
+                              E4M3 scores from bulk-copied tiles where queries and entries are
+                              E4M3 + BF16 RoPE and n_ent_rows is set, else the F16 kernel */
+  LC_IMPL_REF = 3,         /* one warp per (query, head), FP32 CUDA cores (any shape) */
+  LC_IMPL_TC_F16 = 4       /* tcgen05 tiles with every operand widened to F16 */
 };
 
 lc_status lc_csa_sparse_attn_prefill(const lc_attn_args* a, void* stream);

@@ -135,19 +135,23 @@ __global__ void __launch_bounds__(256) k_attn_ref(lc_attn_args a, int sparse) {
 // The kernel a call runs (never LC_IMPL_AUTO): AUTO takes the fastest one measured for
 // 576-dim BF16 / E4M3 shapes, the BF16 mma.sync kernel; other shapes (FP32, other head
 // dims) run on the reference kernel.
-// The automatic choice: the tcgen05 kernel where it applies (576-dim rows with 64 RoPE
+// The automatic choice: the tcgen05 kernels where they apply (576-dim rows with 64 RoPE
 // dims, 64-head groups, 16-byte aligned buffers), else the mma.sync kernel, else the
-// reference kernel.
+// reference kernel.  LC_IMPL_TC takes the E4M3-score kernel where queries and entries are
+// E4M3 + BF16 RoPE, else the F16 one.
+static bool tc_any(const lc_attn_args& a) { return attn_tc8_supported(a) || attn_tc_supported(a); }
+
 int attn_impl(const lc_attn_args& a) {
   if (a.impl != LC_IMPL_AUTO) return a.impl;
-  if (attn_tc_supported(a)) return LC_IMPL_TC;
+  if (tc_any(a)) return LC_IMPL_TC;
   return attn_mma_supported(a) ? LC_IMPL_MMA : LC_IMPL_REF;
 }
 
 bool attn_impl_ok(const lc_attn_args& a) {
   switch (attn_impl(a)) {
     case LC_IMPL_MMA: return attn_mma_supported(a);
-    case LC_IMPL_TC: return attn_tc_supported(a);
+    case LC_IMPL_TC: return tc_any(a);
+    case LC_IMPL_TC_F16: return attn_tc_supported(a);
     case LC_IMPL_REF: return true;
     default: return false;
   }
@@ -160,12 +164,18 @@ size_t attn_workspace_bytes(const lc_attn_args& a, bool sparse, bool decode) {
     lc_attn_args t = a;
     t.out = nullptr;
     t.workspace = nullptr;
-    if (attn_tc_supported(t)) w = w > attn_tc_workspace(a, sparse, decode) ? w : attn_tc_workspace(a, sparse, decode);
+    if (tc_any(t)) {
+      w = w > attn_tc_workspace(a, sparse, decode) ? w : attn_tc_workspace(a, sparse, decode);
+      w = w > attn_tc8_workspace(a, sparse, decode) ? w : attn_tc8_workspace(a, sparse, decode);
+    }
     return w;
   }
   switch (attn_impl(a)) {
     case LC_IMPL_MMA: return attn_mma_supported(a) ? attn_mma_workspace(a, sparse, decode) : 0;
-    case LC_IMPL_TC: return attn_tc_supported(a) ? attn_tc_workspace(a, sparse, decode) : 0;
+    case LC_IMPL_TC:
+      if (attn_tc8_supported(a)) return attn_tc8_workspace(a, sparse, decode);
+      return attn_tc_supported(a) ? attn_tc_workspace(a, sparse, decode) : 0;
+    case LC_IMPL_TC_F16: return attn_tc_supported(a) ? attn_tc_workspace(a, sparse, decode) : 0;
     default: return 0;
   }
 }
@@ -173,9 +183,11 @@ size_t attn_workspace_bytes(const lc_attn_args& a, bool sparse, bool decode) {
 cudaError_t launch_attn(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st) {
   if (a.n_q == 0) return cudaSuccess;
   switch (attn_impl(a)) {
-    case LC_IMPL_TC: {
+    case LC_IMPL_TC:
+    case LC_IMPL_TC_F16: {
       int n_split = 1;
-      cudaError_t e = launch_attn_tc(a, sparse, decode, st, &n_split);
+      const bool fp8 = attn_impl(a) == LC_IMPL_TC && attn_tc8_supported(a);
+      cudaError_t e = fp8 ? launch_attn_tc8(a, sparse, decode, st, &n_split) : launch_attn_tc(a, sparse, decode, st, &n_split);
       if (e != cudaSuccess || n_split == 1) return e;
       return launch_attn_combine(a, n_split, st);
     }

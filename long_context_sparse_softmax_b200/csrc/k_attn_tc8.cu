@@ -1,0 +1,832 @@
+// CSA sparse / HCA dense attention on the 5th-generation tensor cores with FP8 scores
+// (tcgen05; for E4M3 + BF16-RoPE queries and entries, 576 dims, 64 RoPE dims).
+//
+// Same mathematics as k_attn.cu ("解读 DeepSeek V4": CSA attends to its top-k compressed
+// entries, HCA to all of them, both plus a 128-token window and a per-head sink; V = K =
+// the 576-dim entry; "DeepSeek-V4 论文分析" §5.4, §六, §七), and the same per-CTA split
+// into (query, 64-head group, key range) as k_attn_tc.cu.  What differs is how keys reach
+// the tensor core:
+//   * entry tiles (64 keys) are gathered by bulk tensor copies (TMA tile::gather4, four rows
+//     per copy) into 128-byte-swizzled shared tiles: the E4M3 nope part (4 blocks of 128
+//     dims) and the BF16 RoPE part.  The scores of an entry tile need no conversion:
+//     S = Qn Kn^T with E4M3 x E4M3 MMAs (kind::f8f6f4; each product is exact in FP32) plus
+//     Qr Kr^T with BF16 x BF16 MMAs, both accumulating into one FP32 tensor-memory tile;
+//   * V (= K) must be 16-bit for O += P V: converter warps widen each gathered tile to F16
+//     (E4M3 -> F16 exact; BF16 -> F16 exact in [2^-14, 65504], else LC_DEV_RANGE) into a
+//     core-matrix tile, the MN-major A operand of O^T = V^T P^T (M = 128 dims, a last chunk
+//     of 64, N = 64 heads), while the scores of the next tile run;
+//   * the window rows are BF16, so the last (window) tiles run in F16: the raw stages, free
+//     by then, hold Q converted to F16, the window tile is copied into the V tile and
+//     serves both S = Q K^T and O^T = V^T P^T.
+// Softmax, the per-head exponent reference, the sink and the outputs are those of
+// k_attn_tc.cu (P in F16, 11 significant bits; row sums of the rounded P).
+//
+// Warp roles (320 threads): warps 0-3 turn S into P and write the output; warps 4-7
+// convert tiles; lane 0 of warp 8 issues the MMAs; warp 9 computes the key codes and
+// issues the bulk copies.  Every mbarrier wait is bounded: a role that gives up sets
+// LC_DEV_TIMEOUT and an abort flag that stops the others at their next wait.
+#include <cuda.h>
+
+#include "lc_internal.h"
+
+namespace lc {
+
+namespace {
+
+constexpr int kD = 576;
+constexpr int kDR = 64;
+constexpr int kDN = kD - kDR;
+constexpr int kTK = 64;                   // keys per tile
+constexpr int kNR = 64;                   // heads per CTA
+constexpr int kG = 72 * 128;              // F16 core-matrix tile: bytes per group of 8 rows
+constexpr int kTile = 8 * kG;             // F16 tile of 64 rows: 73,728 bytes
+constexpr int kBlk = kTK * 128;           // one 128-byte column block of 64 rows (SW128): 8 KB
+constexpr int kRawN = 4 * kBlk;           // E4M3 nope part of a tile: 32 KB
+constexpr int kRawStage = kRawN + kBlk;   // + BF16 RoPE part: 40 KB
+constexpr int kPBytes = kNR * kTK * 2;
+constexpr long kSpin = 1L << 26;
+constexpr uint32_t kWin = 1u << 30;
+constexpr int kThreads = 320;
+constexpr float kRescale = 8.f;
+constexpr int kColS = 0;                  // S buffers at columns 0 and 64
+constexpr int kColO = 2 * kTK;            // O^T chunk c at 128 + 64 c
+constexpr uint32_t kTmemCols = 512;
+
+// shared memory (dynamic, 1024-byte aligned)
+constexpr int kOffQn = 0;                         // Q nope, E4M3, 4 SW128 blocks
+constexpr int kOffQr = kOffQn + kRawN;            // Q RoPE, BF16, SW128
+constexpr int kOffRaw = kOffQr + kBlk;            // 2 raw stages (window phase: Q in F16)
+constexpr int kOffV = kOffRaw + 2 * kRawStage;    // F16 core-matrix tile
+constexpr int kOffP = kOffV + kTile;
+constexpr int kOffCode = kOffP + kPBytes;         // [4][kTK] key codes
+constexpr int kOffF = kOffCode + 4 * kTK * 4;     // [kNR] per-head factors
+constexpr size_t kSmem = kOffF + kNR * 4 + 1024;  // + alignment slack
+static_assert(2 * kRawStage >= kTile, "Q in F16 fits the raw stages");
+
+__device__ __forceinline__ uint32_t su32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+
+// no-swizzle core-matrix operand
+__device__ __forceinline__ uint64_t cm_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+// K-major SWIZZLE_128B operand: 128-byte rows, 8-row groups 1024 bytes apart
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+  uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>(1) << 16;
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile("{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+               : "=r"(done)
+               : "r"(bar), "r"(parity)
+               : "memory");
+  return done != 0;
+}
+__device__ __forceinline__ bool mbar_probe(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile("{\n.reg .pred p;\nmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+               : "=r"(done)
+               : "r"(bar), "r"(parity)
+               : "memory");
+  return done != 0;
+}
+
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+__device__ __forceinline__ void named_bar(int id, int n) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ bool named_bar_or(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n.reg .pred pi, po;\nsetp.ne.b32 pi, %1, 0;\nbar.red.or.pred po, %2, %3, pi;\nselp.u32 %0, 1, 0, po;\n}\n"
+      : "=r"(r)
+      : "r"(static_cast<int>(v)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+template <int KIND>  // 0: kind::f16, 1: kind::f8f6f4
+__device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if (KIND == 0)
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+            d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+  else
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+            d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar));
+}
+
+#define LC8_R32(r)                                                                                                \
+  "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),   \
+      "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),      \
+      "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),     \
+      "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+#define LC8_REGS32                                                                                                \
+  "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29," \
+  "%30,%31}"
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 " LC8_REGS32 ", [%32];\n" : LC8_R32(r) : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld16x2(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x32.b32 " LC8_REGS32 ", [%32], 32;\n" : LC8_R32(r) : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int r0, int r1, int r2, int r3,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4, %5, %6}], [%7];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_tile2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// 16 E4M3 values -> 16 F16 values (exact)
+__device__ __forceinline__ void e4m3x16_f16(uint4 v, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[j] & 0xffffu), __NV_E4M3);
+    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[j] >> 16), __NV_E4M3);
+    o[2 * j] = static_cast<uint32_t>(a.x) | (static_cast<uint32_t>(a.y) << 16);
+    o[2 * j + 1] = static_cast<uint32_t>(b.x) | (static_cast<uint32_t>(b.y) << 16);
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+// 8 BF16 values -> 8 F16 values; |value| accumulated (as F16) into `amax`
+__device__ __forceinline__ uint4 bf16x8_f16(uint4 v, __half2& amax) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const __half2 h = __floats2half2_rn(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u));
+    amax = __hmax2(amax, __habs2(h));
+    o[j] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+__device__ __forceinline__ bool f16_inf(__half2 a) {
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(&a);
+  return ((u & 0x7c00u) == 0x7c00u) | ((u & 0x7c000000u) == 0x7c000000u);
+}
+
+// byte offset of dim chunk c (8 dims) of row r in the F16 core-matrix tile
+__device__ __forceinline__ uint32_t tile_off(int r, int c) { return (r >> 3) * kG + c * 128 + (r & 7) * 16; }
+// byte offset of 16-byte chunk j of row r in a SWIZZLE_128B block of 128-byte rows
+__device__ __forceinline__ uint32_t sw128_off(int r, int j) { return r * 128 + ((j ^ (r & 7)) << 4); }
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void cp16(uint8_t* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(su32(dst)), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(gdst), "r"(su32(ssrc)),
+               "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
+}
+
+struct Bars {
+  uint64_t qfull;      // Q nope + RoPE landed (expect-tx)
+  uint64_t kfull[2];   // raw stage landed (expect-tx)
+  uint64_t kempty[2];  // raw stage read by S (commit) and by the converter (1 arrival)
+  uint64_t cready[4];  // key codes of a tile written (1 arrival)
+  uint64_t cfree[4];   // key codes of a tile read by the softmax (128 arrivals)
+  uint64_t vfull;      // F16 tile ready (1 arrival)
+  uint64_t vempty;     // F16 tile read by O (commit)
+  uint64_t q16full;    // Q in F16 ready for the window tiles (1 arrival)
+  uint64_t sfull[2];   // S buffer computed (commit)
+  uint64_t sempty[2];  // S buffer read (128 arrivals)
+  uint64_t pfull;      // P written (128 arrivals)
+  uint64_t pempty;     // P read and O updated (commit)
+  uint64_t fin;        // every MMA complete (commit)
+};
+
+}  // namespace
+
+struct AttnTc8Geom {
+  int n_split;
+  int sps;  // slots per split, multiple of kTK
+};
+
+// grid: one CTA per (query, head group, key split), the split index fastest; 320 threads.
+// Partial results of split s go to ws_o rows s * n_q * H + q * H + h (576 floats each) and
+// ws_ml[2 ((q * H + h) * n_split + s) + {0, 1}] = (m, l).
+__global__ void __launch_bounds__(kThreads, 1)
+    k_attn_tc8(const __grid_constant__ CUtensorMap tqn, const __grid_constant__ CUtensorMap tqr,
+               const __grid_constant__ CUtensorMap tkn, const __grid_constant__ CUtensorMap tkr, lc_attn_args a,
+               int sparse, AttnTc8Geom geo, float* __restrict__ ws_o, float* __restrict__ ws_ml) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Qn = smem + kOffQn;
+  uint8_t* Qr = smem + kOffQr;
+  uint8_t* Raw = smem + kOffRaw;
+  uint8_t* Vt = smem + kOffV;
+  uint8_t* Ps = smem + kOffP;
+  int* kcode = reinterpret_cast<int*>(smem + kOffCode);
+  float* s_f = reinterpret_cast<float*>(smem + kOffF);
+  uint8_t* Q16 = Raw;  // window phase
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ __align__(8) Bars bars;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_hg = a.dims.H / kNR;
+  const int split = blockIdx.x % geo.n_split;
+  const int hg = (blockIdx.x / geo.n_split) % n_hg;
+  const int q = blockIdx.x / (geo.n_split * n_hg);
+  const int H = a.dims.H;
+  const int b = seq_of_query(a.batch.q_start, a.batch.num_seqs, q);
+  const int p = __ldg(a.batch.q_pos0 + b) + (q - __ldg(a.batch.q_start + b));
+  const int n_ent = __ldg(a.batch.n_ent + b);
+  const int nv = n_visible(p, a.m, a.W_x, n_ent);
+  const int64_t ent0 = __ldg(a.batch.ent_start + b);
+  const int wlo = a.W > 0 ? max(0, p - a.W + 1) : p + 1;
+  const int n_first = sparse ? a.k : nv;
+  const int n_slots = n_first + (p + 1 - wlo);
+  const int s_begin = split * geo.sps;
+  const int s_end = min(n_slots, s_begin + geo.sps);
+  // entry tiles cover [s_begin, min(s_end, n_first)), window tiles the rest of the range
+  const int e_end = min(s_end, n_first);
+  const int n_et = e_end > s_begin ? (e_end - s_begin + kTK - 1) / kTK : 0;
+  const int w_begin = max(s_begin, n_first);
+  const int n_wt = s_end > w_begin ? (s_end - w_begin + kTK - 1) / kTK : 0;
+  const int n_tiles = n_et + n_wt;
+  const int wp0 = a.W > 0 ? __ldg(a.batch.win_pos0 + b) : 0;
+  const int wl = a.W > 0 ? __ldg(a.batch.win_len + b) : 0;
+  const int64_t wr0 = a.W > 0 ? __ldg(a.batch.win_start + b) : 0;
+  const int32_t* idx_row = sparse ? a.idx + static_cast<int64_t>(q) * a.k : nullptr;
+  const int64_t row0 = static_cast<int64_t>(q) * H + hg * kNR;
+
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    const uint32_t addr = su32(bar);
+    for (long it = 0; it < kSpin; ++it) {
+      if (mbar_test(addr, parity)) return true;
+      if ((it & 1023) == 1023 && *reinterpret_cast<volatile int*>(&s_abort)) return false;
+    }
+    set_status(a.status, LC_DEV_TIMEOUT);
+    atomicExch(&s_abort, 1);
+    return false;
+  };
+  // first slot of tile t
+  auto tile_slot0 = [&](int t) { return t < n_et ? s_begin + t * kTK : w_begin + (t - n_et) * kTK; };
+  auto tile_slot_end = [&](int t) { return t < n_et ? e_end : s_end; };
+  // key slot -> entry index j, kWin | window row, or -1 (masked)
+  auto slot_code = [&](int s, int s_lim) -> int {
+    if (s >= s_lim) return -1;
+    if (s < n_first) {
+      const int j = sparse ? __ldg(idx_row + s) : s;
+      if (j < 0) return -1;
+      if (j >= n_ent) {
+        set_status(a.status, LC_DEV_BAD_INDEX);
+        return -1;
+      }
+      if (j >= nv) {
+        set_status(a.status, LC_DEV_NONVISIBLE);
+        return -1;
+      }
+      return j;
+    }
+    const int rr = wlo + (s - n_first) - wp0;
+    if (rr < 0 || rr >= wl) {
+      set_status(a.status, LC_DEV_WINDOW_RANGE);
+      return -1;
+    }
+    return static_cast<int>(kWin) | rr;
+  };
+
+  // ---- set-up ----
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(su32(&s_tmem)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
+  }
+  if (tid == 32) {
+    s_abort = 0;
+    mbar_init(su32(&bars.qfull), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(su32(&bars.kfull[i]), 1);
+      mbar_init(su32(&bars.kempty[i]), 2);
+      mbar_init(su32(&bars.sfull[i]), 1);
+      mbar_init(su32(&bars.sempty[i]), 128);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(su32(&bars.cready[i]), 1);
+      mbar_init(su32(&bars.cfree[i]), 128);
+    }
+    mbar_init(su32(&bars.vfull), 1);
+    mbar_init(su32(&bars.vempty), 1);
+    mbar_init(su32(&bars.q16full), 1);
+    mbar_init(su32(&bars.pfull), 128);
+    mbar_init(su32(&bars.pempty), 1);
+    mbar_init(su32(&bars.fin), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tm = s_tmem;
+
+  if (warp == 9) {
+    // ================= key codes and bulk copies =================
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t qb = su32(&bars.qfull);
+      mbar_expect_tx(qb, kRawN + kBlk);
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) tma_tile2d(su32(Qn + cb * kBlk), &tqn, cb * 128, static_cast<int>(row0), qb);
+      tma_tile2d(su32(Qr), &tqr, 0, static_cast<int>(row0), qb);
+    }
+    for (int t = 0; t < n_tiles; ++t) {
+      const int cb4 = t & 3;
+      // the code buffer of tile t - 4 has been read by its softmax
+      bool ok = t < 4 || wait(&bars.cfree[cb4], ((t >> 2) - 1) & 1);
+      // raw stage of entry tile t: free once S and the conversion of tile t - 2 are done
+      if (ok && t < n_et && t >= 2) ok = wait(&bars.kempty[t & 1], ((t >> 1) - 1) & 1);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int s0 = tile_slot0(t), s_lim = tile_slot_end(t);
+      int* kc = kcode + cb4 * kTK;
+      const int c0 = slot_code(s0 + lane, s_lim), c1 = slot_code(s0 + 32 + lane, s_lim);
+      kc[lane] = c0;
+      kc[32 + lane] = c1;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(su32(&bars.cready[cb4]));
+      if (t < n_et) {
+        const int st = t & 1;
+        const uint32_t kb = su32(&bars.kfull[st]);
+        if (lane == 0) mbar_expect_tx(kb, kRawStage);
+        __syncwarp();
+        if (lane < kTK / 4) {
+          // rows 4 lane .. 4 lane + 3; a masked key reads row 0 (its P is 0)
+          int rr[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int code = kc[4 * lane + u];
+            rr[u] = code < 0 ? 0 : static_cast<int>(ent0 + code);
+          }
+          uint8_t* stage = Raw + st * kRawStage;
+#pragma unroll
+          for (int cb = 0; cb < 4; ++cb)
+            tma_gather4(su32(stage + cb * kBlk + lane * 512), &tkn, cb * 128, rr[0], rr[1], rr[2], rr[3], kb);
+          tma_gather4(su32(stage + kRawN + lane * 512), &tkr, 0, rr[0], rr[1], rr[2], rr[3], kb);
+        }
+      }
+    }
+  } else if (warp == 8) {
+    // ================= MMA issue (one lane) =================
+    if (lane == 0) {
+      // S entry: M = 64, N = 64, K-major SW128, E4M3 (kind::f8f6f4) and BF16 (kind::f16)
+      const uint32_t id_s8 = (1u << 4) | (static_cast<uint32_t>(kTK >> 3) << 17) | (static_cast<uint32_t>(kNR >> 4) << 24);
+      const uint32_t id_sbf = id_s8 | (1u << 7) | (1u << 10);
+      // S window: F16 core-matrix operands; O^T: M = 128 (or 64), N = 64, A MN-major, F16
+      const uint32_t id_sf16 = id_s8;
+      const uint32_t id_o128 = (1u << 4) | (1u << 15) | (static_cast<uint32_t>(kNR >> 3) << 17) |
+                               (static_cast<uint32_t>(128 >> 4) << 24);
+      const uint32_t id_o64 = (1u << 4) | (1u << 15) | (static_cast<uint32_t>(kNR >> 3) << 17) |
+                              (static_cast<uint32_t>(64 >> 4) << 24);
+      const uint64_t dp = cm_desc(su32(Ps), 128, (kTK / 8) * 128);
+      const uint64_t dv = cm_desc(su32(Vt), kG, 128);
+      int ns = 0, no = 0;
+      long idle = 0;
+      bool ok = n_tiles == 0 || wait(&bars.qfull, 0);
+      while (ok && no < n_tiles) {
+        bool progressed = false;
+        if (ns < n_tiles && ns <= no + 1) {
+          const int sb = ns & 1;
+          bool ready = ns < 2 || mbar_probe(su32(&bars.sempty[sb]), ((ns >> 1) - 1) & 1);
+          if (ns < n_et) ready = ready && mbar_probe(su32(&bars.kfull[ns & 1]), (ns >> 1) & 1);
+          else ready = ready && mbar_probe(su32(&bars.q16full), 0) && mbar_probe(su32(&bars.vfull), ns & 1);
+          if (ready) {
+            fence_after();
+            const uint32_t d = tm + kColS + sb * kTK;
+            if (ns < n_et) {
+              const uint32_t st = su32(Raw + (ns & 1) * kRawStage);
+#pragma unroll
+              for (int cb = 0; cb < 4; ++cb)
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  mma<1>(d, sw128_desc(su32(Qn) + cb * kBlk + k * 32), sw128_desc(st + cb * kBlk + k * 32), id_s8,
+                         cb > 0 || k > 0);
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                mma<0>(d, sw128_desc(su32(Qr) + k * 32), sw128_desc(st + kRawN + k * 32), id_sbf, 1);
+              mma_commit(su32(&bars.kempty[ns & 1]));
+            } else {
+              const uint64_t dq = cm_desc(su32(Q16), 128, kG), dk = cm_desc(su32(Vt), 128, kG);
+#pragma unroll
+              for (int k = 0; k < kD / 16; ++k) mma<0>(d, dq + k * 16, dk + k * 16, id_sf16, k > 0);
+            }
+            mma_commit(su32(&bars.sfull[sb]));
+            ++ns;
+            progressed = true;
+          }
+        }
+        if (no < ns && mbar_probe(su32(&bars.pfull), no & 1) && mbar_probe(su32(&bars.vfull), no & 1)) {
+          fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTK / 16; ++kk)
+#pragma unroll
+            for (int c = 0; c < 5; ++c)
+              mma<0>(tm + kColO + c * kNR, dv + (c * 2048 + kk * 2 * kG) / 16, dp + kk * 16, c < 4 ? id_o128 : id_o64,
+                     (no > 0) || (kk > 0));
+          mma_commit(su32(&bars.vempty));
+          mma_commit(su32(&bars.pempty));
+          ++no;
+          progressed = true;
+        }
+        if (progressed) {
+          idle = 0;
+        } else if (++idle >= kSpin) {
+          set_status(a.status, LC_DEV_TIMEOUT);
+          atomicExch(&s_abort, 1);
+          ok = false;
+        } else if ((idle & 1023) == 0 && *reinterpret_cast<volatile int*>(&s_abort)) {
+          ok = false;
+        }
+      }
+      mma_commit(su32(&bars.fin));
+      wait(&bars.fin, 0);
+    }
+  } else if (warp >= 4) {
+    // ================= converters: raw or window rows -> F16 tile =================
+    const int ct = tid - 128;  // 0..127
+    const int r8 = ct & 7;     // row within a group of 8 (one quarter warp: 8 rows, one chunk)
+    __half2 amax = __float2half2_rn(0.f);
+    bool ok = true;
+    for (int t = 0; ok && t < n_tiles; ++t) {
+      if (t == n_et) {
+        // window phase: Q to F16 in the raw stages, once S and the conversion of every
+        // entry tile are done (the raw stages are free)
+        bool okq = wait(&bars.qfull, 0);
+        if (okq && n_et >= 1) okq = wait(&bars.kempty[(n_et - 1) & 1], ((n_et - 1) >> 1) & 1);
+        if (okq && n_et >= 2) okq = wait(&bars.kempty[(n_et - 2) & 1], ((n_et - 2) >> 1) & 1);
+        if (named_bar_or(2, 128, !okq)) {
+          ok = false;
+          break;
+        }
+        // 64 rows x (64 E4M3 chunks of 8 + 8 BF16 chunks)
+        for (int i = ct; i < kNR * 36; i += 128) {
+          const int g = i >> 3, pc = g % 36, r = (g / 36) * 8 + (i & 7);
+          if (pc < 32) {  // 16 E4M3 dims: block pc / 8, 16-byte chunk pc % 8 of row r
+            const uint4 v = *reinterpret_cast<const uint4*>(Qn + (pc >> 3) * kBlk + sw128_off(r, pc & 7));
+            uint4 lo, hi;
+            e4m3x16_f16(v, lo, hi);
+            *reinterpret_cast<uint4*>(Q16 + tile_off(r, 2 * pc)) = lo;
+            *reinterpret_cast<uint4*>(Q16 + tile_off(r, 2 * pc + 1)) = hi;
+          } else {  // 16 RoPE dims: chunks 2 (pc - 32), +1 of the SW128 row
+            const int j = 2 * (pc - 32);
+            const uint4 v0 = *reinterpret_cast<const uint4*>(Qr + sw128_off(r, j));
+            const uint4 v1 = *reinterpret_cast<const uint4*>(Qr + sw128_off(r, j + 1));
+            *reinterpret_cast<uint4*>(Q16 + tile_off(r, 64 + j)) = bf16x8_f16(v0, amax);
+            *reinterpret_cast<uint4*>(Q16 + tile_off(r, 64 + j + 1)) = bf16x8_f16(v1, amax);
+          }
+        }
+        fence_async_smem();
+        named_bar(2, 128);
+        if (ct == 0) mbar_arrive(su32(&bars.q16full));
+      }
+      // the F16 tile is free once O of the previous tile is done; this tile's codes or
+      // raw rows have landed
+      bool okw = t == 0 || wait(&bars.vempty, (t - 1) & 1);
+      if (t < n_et) okw = okw && wait(&bars.kfull[t & 1], (t >> 1) & 1);
+      else okw = okw && wait(&bars.cready[t & 3], (t >> 2) & 1);
+      if (named_bar_or(2, 128, !okw)) {
+        ok = false;
+        break;
+      }
+      if (t < n_et) {
+        const uint8_t* st = Raw + (t & 1) * kRawStage;
+        // 64 keys x (32 E4M3 pieces of 16 dims + 8 BF16 chunks); a quarter warp takes 8
+        // rows of one piece: its SW128 reads and its core-matrix writes hit distinct banks
+        for (int i = ct; i < kTK * 40; i += 128) {
+          const int g = i >> 3, pc = g % 40, r = (g / 40) * 8 + r8;
+          if (pc < 32) {
+            const uint4 v = *reinterpret_cast<const uint4*>(st + (pc >> 3) * kBlk + sw128_off(r, pc & 7));
+            uint4 lo, hi;
+            e4m3x16_f16(v, lo, hi);
+            *reinterpret_cast<uint4*>(Vt + tile_off(r, 2 * pc)) = lo;
+            *reinterpret_cast<uint4*>(Vt + tile_off(r, 2 * pc + 1)) = hi;
+          } else {
+            const int j = pc - 32;
+            const uint4 v = *reinterpret_cast<const uint4*>(st + kRawN + sw128_off(r, j));
+            *reinterpret_cast<uint4*>(Vt + tile_off(r, 64 + j)) = bf16x8_f16(v, amax);
+          }
+        }
+      } else {
+        // window rows (BF16, 72 chunks each) straight into the tile, then rounded to F16
+        const int* kc = kcode + (t & 3) * kTK;
+        for (int i = ct; i < kTK * 72; i += 128) {
+          const int g = i >> 3, c = g % 72, r = (g / 72) * 8 + r8;
+          const int code = kc[r];
+          uint8_t* dst = Vt + tile_off(r, c);
+          if (code < 0 || !(code & kWin)) *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+          else cp16(dst, static_cast<const uint8_t*>(a.win.x) + ((wr0 + (code & ~kWin)) * kD + c * 8) * 2);
+        }
+        asm volatile("cp.async.commit_group;\ncp.async.wait_all;\n" ::: "memory");
+        named_bar(2, 128);
+        for (int i = ct; i < kTK * 72; i += 128) {
+          const int g = i >> 3, c = g % 72, r = (g / 72) * 8 + r8;
+          uint4* d = reinterpret_cast<uint4*>(Vt + tile_off(r, c));
+          *d = bf16x8_f16(*d, amax);
+        }
+      }
+      fence_async_smem();
+      named_bar(2, 128);
+      if (ct == 0) {
+        mbar_arrive(su32(&bars.vfull));
+        if (t < n_et) mbar_arrive(su32(&bars.kempty[t & 1]));
+      }
+    }
+    if (f16_inf(amax)) set_status(a.status, LC_DEV_RANGE);
+  } else {
+    // ================= warps 0-3: softmax, epilogue =================
+    const int r = warp * 16 + (lane & 15);
+    const int hf = lane >> 4;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = a.scale * 1.4426950408889634f;
+    float m_ref = -INFINITY, l_sum = 0.f;
+    bool good = true;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int sb = t & 1;
+      const bool okw = wait(&bars.sfull[sb], (t >> 1) & 1) && wait(&bars.cready[t & 3], (t >> 2) & 1);
+      if (named_bar_or(1, 128, !okw)) {
+        good = false;
+        break;
+      }
+      fence_after();
+      uint32_t sv[32];
+      tmem_ld16x2(tm + lane_off + kColS + sb * kTK, sv);
+      uint32_t live = 0;  // bit j: key 32 hf + j is not masked
+      const int* kc = kcode + (t & 3) * kTK + 32 * hf;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) live |= static_cast<uint32_t>(kc[j] >= 0) << j;
+      mbar_arrive(su32(&bars.cfree[t & 3]));
+      tmem_wait_ld();
+      fence_before();
+      mbar_arrive(su32(&bars.sempty[sb]));
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float x = (live >> j) & 1u ? __uint_as_float(sv[j]) * sl2 : -INFINITY;
+        sv[j] = __float_as_uint(x);
+        mx = fmaxf(mx, x);
+      }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const bool need = mx > m_ref + kRescale;
+      const bool okp = t == 0 || wait(&bars.pempty, (t - 1) & 1);
+      if (named_bar_or(1, 128, !okp)) {
+        good = false;
+        break;
+      }
+      const bool any = named_bar_or(1, 128, need && t > 0);
+      float f = 1.f;
+      if (need) {
+        f = m_ref == -INFINITY ? 0.f : exp2f(m_ref - mx);
+        l_sum *= f;
+        m_ref = mx;
+      }
+      if (any) {
+        if (hf == 0) s_f[r] = f;
+        named_bar(1, 128);
+        fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 5; ++c)
+#pragma unroll 1
+          for (int hh = 0; hh < kNR; hh += 32) {
+            uint32_t ov[32];
+            const uint32_t ta = tm + lane_off + kColO + c * kNR + hh;
+            tmem_ld32(ta, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * s_f[hh + i]);
+            tmem_st32(ta, ov);
+          }
+        tmem_wait_st();
+        named_bar(1, 128);
+      }
+      {
+        uint32_t pk[16];
+        const float mr = m_ref == -INFINITY ? 0.f : m_ref;
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const __half2 ph = __floats2half2_rn(ex2(__uint_as_float(sv[j]) - mr), ex2(__uint_as_float(sv[j + 1]) - mr));
+          const float2 pf = __half22float2(ph);
+          l_sum += pf.x + pf.y;
+          pk[j / 2] = *reinterpret_cast<const uint32_t*>(&ph);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(Ps + (r >> 3) * 1024 + (4 * hf + c) * 128 + (r & 7) * 16) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      fence_async_smem();
+      fence_before();
+      mbar_arrive(su32(&bars.pfull));
+    }
+    // ---- epilogue ----
+    if (good && n_tiles > 0) good = wait(&bars.pempty, (n_tiles - 1) & 1);
+    good = !named_bar_or(1, 128, !good);
+    fence_after();
+    const float l_row = l_sum + __shfl_xor_sync(0xffffffffu, l_sum, 16);
+    if (hf == 0) {
+      const int h = hg * kNR + r;
+      if (geo.n_split == 1) {
+        const float sk = __ldg(a.sink + h) * 1.4426950408889634f;
+        const float M = fmaxf(sk, m_ref);
+        const float w = m_ref == -INFINITY ? 0.f : exp2f(m_ref - M);
+        const float Z = exp2f(sk - M) + l_row * w;
+        s_f[r] = w / Z;
+        if (a.lse && good) a.lse[row0 + r] = (M + log2f(Z)) * 0.6931471805599453f;
+      } else if (good) {
+        const int64_t slot = (row0 + r) * geo.n_split + split;
+        ws_ml[2 * slot] = m_ref;
+        ws_ml[2 * slot + 1] = l_row;
+      }
+    }
+    named_bar(1, 128);
+    if (good) {
+      // O rows -> the raw stages (free: every MMA is complete), row-major [head][dim]
+      const bool f32 = geo.n_split > 1 || a.out_fmt == LC_FMT_F32;
+      uint8_t* stage_out = Raw;  // 2 raw stages (80 KB) + the F16 tile (72 KB) are contiguous
+      float* stf = reinterpret_cast<float*>(stage_out);
+      uint16_t* sth = reinterpret_cast<uint16_t*>(stage_out);
+#pragma unroll 1
+      for (int c = 0; c < 5; ++c) {
+        const int dim = c < 4 ? c * 128 + warp * 32 + lane : (lane < 16 ? 512 + warp * 16 + lane : -1);
+        uint32_t ov[kNR];
+        if (n_tiles > 0) {
+          tmem_ld32(tm + lane_off + kColO + c * kNR, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
+          tmem_ld32(tm + lane_off + kColO + c * kNR + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < kNR; ++i) ov[i] = 0;
+        }
+        if (dim < 0) continue;
+#pragma unroll
+        for (int i = 0; i < kNR; ++i) {
+          float v = __uint_as_float(ov[i]);
+          if (geo.n_split == 1) v *= s_f[i];
+          if (f32) stf[i * kD + dim] = v;
+          else sth[i * kD + dim] = f32_to_bf16_bits(v);
+        }
+      }
+      fence_async_smem();
+      named_bar(1, 128);
+      if (tid == 0) {
+        const uint32_t bytes = kNR * kD * (f32 ? 4 : 2);
+        void* dst;
+        if (geo.n_split > 1) dst = ws_o + (static_cast<int64_t>(split) * a.n_q * H + row0) * kD;
+        else if (a.out_fmt == LC_FMT_F32) dst = static_cast<float*>(a.out) + row0 * kD;
+        else dst = static_cast<uint16_t*>(a.out) + row0 * kD;
+        bulk_store(dst, stage_out, bytes);
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tm), "r"(kTmemCols));
+}
+
+// ---------------------------------------------------------------------------------
+bool attn_tc8_supported(const lc_attn_args& a) {
+  if (a.dims.D != kD || a.dims.d_r != kDR || a.dims.H % kNR || a.n_ent_rows < 1) return false;
+  if (a.q.fmt != LC_FMT_E4M3_BF16 || a.ent.fmt != LC_FMT_E4M3_BF16) return false;
+  if (a.W > 0 && a.win.fmt != LC_FMT_BF16) return false;
+  auto al = [](const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; };
+  if (!al(a.q.x) || !al(a.q.rope) || !al(a.ent.x) || !al(a.ent.rope) || (a.W > 0 && !al(a.win.x))) return false;
+  if (!al(a.out) || !al(a.workspace)) return false;
+  if (static_cast<int64_t>(a.n_q) * a.dims.H > 0x7fffffff) return false;
+  return a.out_fmt == LC_FMT_BF16 || a.out_fmt == LC_FMT_F32;
+}
+
+static AttnTc8Geom tc8_geometry(const lc_attn_args& a, bool sparse, bool decode) {
+  AttnTc8Geom g{1, 0};
+  const int ns = max((sparse ? a.k : a.max_ent) + a.W, 1);
+  const int tiles = (ns + kTK - 1) / kTK;
+  g.sps = tiles * kTK;
+  const int ctas = a.n_q * (a.dims.H / kNR);
+  if (decode && ctas < 148) {
+    const int n = max(1, min(148 / max(ctas, 1), tiles));
+    const int per = (tiles + n - 1) / n;
+    g.n_split = (tiles + per - 1) / per;
+    g.sps = per * kTK;
+  }
+  return g;
+}
+
+size_t attn_tc8_workspace(const lc_attn_args& a, bool sparse, bool decode) {
+  const AttnTc8Geom g = tc8_geometry(a, sparse, decode);
+  if (g.n_split <= 1) return 0;
+  const size_t rows = static_cast<size_t>(a.n_q) * a.dims.H * g.n_split;
+  return rows * kD * sizeof(float) + rows * 2 * sizeof(float);
+}
+
+namespace {
+
+using EncodeTiled8 = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled8 encode8() {
+  static EncodeTiled8 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiled8>(nullptr);
+    return reinterpret_cast<EncodeTiled8>(f);
+  }();
+  return fn;
+}
+
+// a [rows, cols] row-major tensor of `esize`-byte elements, SW128 boxes of box_rows rows
+bool make_map(CUtensorMap* m, CUtensorMapDataType ty, const void* base, int64_t rows, int cols, int esize,
+              int box_cols, int box_rows) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * esize};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t es[2] = {1, 1};
+  return encode8()(m, ty, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_attn_tc8(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st, int* n_split_out) {
+  if (!encode8()) return cudaErrorNotSupported;
+  const AttnTc8Geom g = tc8_geometry(a, sparse, decode);
+  *n_split_out = g.n_split;
+  const int64_t qrows = static_cast<int64_t>(a.n_q) * a.dims.H;
+  CUtensorMap tqn, tqr, tkn, tkr;
+  if (!make_map(&tqn, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q.x, qrows, kDN, 1, 128, kNR) ||
+      !make_map(&tqr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.q.rope, qrows, kDR, 2, 64, kNR) ||
+      !make_map(&tkn, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.ent.x, a.n_ent_rows, kDN, 1, 128, 1) ||
+      !make_map(&tkr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.ent.rope, a.n_ent_rows, kDR, 2, 64, 1))
+    return cudaErrorInvalidValue;
+  cudaFuncSetAttribute(k_attn_tc8, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
+  float* ws_o = static_cast<float*>(a.workspace);
+  float* ws_ml = nullptr;
+  if (g.n_split > 1) ws_ml = ws_o + static_cast<size_t>(a.n_q) * a.dims.H * g.n_split * kD;
+  const int64_t ctas = static_cast<int64_t>(a.n_q) * (a.dims.H / kNR) * g.n_split;
+  if (ctas > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  k_attn_tc8<<<static_cast<unsigned>(ctas), kThreads, kSmem, st>>>(tqn, tqr, tkn, tkr, a, sparse ? 1 : 0, g, ws_o,
+                                                                  ws_ml);
+  return cudaGetLastError();
+}
+
+}  // namespace lc

@@ -114,7 +114,7 @@ lc_status attn(const lc_attn_args* a, void* stream, bool sparse, bool decode) {
   if (a->out_fmt != LC_FMT_F32 && a->out_fmt != LC_FMT_BF16) return LC_ERR_ARG;
   if (sparse && a->k < 1) return LC_ERR_ARG;
   if (decode && a->n_q != a->batch.num_seqs) return LC_ERR_ARG;
-  if (a->impl < LC_IMPL_AUTO || a->impl > LC_IMPL_REF) return LC_ERR_ARG;
+  if (a->impl < LC_IMPL_AUTO || a->impl > LC_IMPL_TC_F16) return LC_ERR_ARG;
   if (!lc::attn_impl_ok(*a)) return LC_ERR_UNSUPPORTED;
   if (a->n_q == 0) return LC_OK;
   LC_TRY(check_rows(a->q, a->dims, true));

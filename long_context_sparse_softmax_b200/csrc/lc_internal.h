@@ -23,6 +23,9 @@ bool attn_impl_ok(const lc_attn_args& a);
 size_t attn_tc_workspace(const lc_attn_args& a, bool sparse, bool decode);
 cudaError_t launch_attn_tc(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st, int* n_split);
 cudaError_t launch_attn_combine(const lc_attn_args& a, int n_split, cudaStream_t st);
+bool attn_tc8_supported(const lc_attn_args& a);
+size_t attn_tc8_workspace(const lc_attn_args& a, bool sparse, bool decode);
+cudaError_t launch_attn_tc8(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st, int* n_split);
 cudaError_t launch_index_tc(const lc_index_args& a, bool decode, cudaStream_t st);
 
 // Sequence of query row q: the b with q_start[b] <= q < q_start[b+1] (binary search).
