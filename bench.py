@@ -9,8 +9,9 @@ A step is one pass of the whole path over one batch of synthetic input:
   csa_prefill / hca_prefill / tiny_csa_prefill: the whole prefill of one sequence.
   mixed_decode: a CSA decode layer and an HCA decode layer, batch 8, ragged 0.5M-1M.
 Metric: query tokens per second (whole job, all ranks).  Inputs are resident in HBM when
-the timed region starts; L2 is flushed (a 512 MiB write) between timed steps, outside
-the per-step CUDA events.  With N > 1 (torchrun) every rank runs its own batch: weak
+the timed region starts; L2 is flushed (a 512 MiB write, then a 256 MiB read that leaves
+the cache clean) between timed steps, outside the per-step CUDA events.  The step is
+captured once as a CUDA graph and replayed (--no-graph: every call launched from Python).  With N > 1 (torchrun) every rank runs its own batch: weak
 scaling, no collective on the data path.
 --impl reference times the CPU oracle (the plain float64 restatement of the method) on a
 bounded sample of the same workload on the host cores (rank 0 only).
@@ -46,6 +47,8 @@ def parse():
                     choices=["csa_decode", "csa_prefill", "hca_prefill", "mixed_decode", "tiny_csa_prefill"])
     ap.add_argument("--impl", default="lc", choices=["lc", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch every call from Python each step "
+                    "instead of replaying the step's CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0)
     ap.add_argument("--attn-impl", default="auto", choices=["auto", "mma", "tc", "ref", "tc16"],
@@ -272,7 +275,15 @@ def run_lc(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     pk, pk_kind = peaks()
     runs = make_runs(args.workload, dev, rank, {"auto": 0, "mma": 1, "tc": 2, "ref": 3, "tc16": 4}[args.attn_impl])
+    # L2 flush: a 512 MiB write, then a 256 MiB read so that the lines the step evicts are
+    # clean (the write alone would leave L2 full of dirty lines whose write-back lands on
+    # the first kernel of the step)
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        flush.zero_()
+        flush_r.sum()
     # the critical path (index -> top-k -> attention) on a high-priority stream, made current
     # so that the L2 flush and the host copies stay ordered with it; the side stream fills
     # the SMs it leaves idle
@@ -295,25 +306,38 @@ def run_lc(args):
     n_launch = len(stage_names) + sum(1 for (_, _, r) in runs if r.a_attn.workspace_bytes > 0)
     side = torch.cuda.Stream(dev, priority=0)
 
+    def timed(stage_ev):
+        """on_stage hook that brackets each launch with the stage's event pair."""
+        def on_stage(i, name, st, fn):
+            e0, e1 = stage_ev[f"{i}:{name}"]
+            e0.record(st)
+            fn(st)
+            e1.record(st)
+        return on_stage
+
     def one_step(stage_ev=None):
         """The whole path once: per workload, preparation and compression on the side
         stream next to index -> top-k on the main stream, then attention."""
+        hook = None if stage_ev is None else timed(stage_ev)
         for i, (_, _, r) in enumerate(runs):
-            def on_stage(name, st, fn, i=i):
-                if stage_ev is None:
-                    fn(st)
-                    return
-                e0, e1 = stage_ev[f"{i}:{name}"]
-                e0.record(st)
-                fn(st)
-                e1.record(st)
-            r.step_overlapped(stream, side, on_stage)
+            r.step_overlapped(stream, side, None if hook is None else
+                              (lambda name, st, fn, i=i: hook(i, name, st, fn)))
 
     for _ in range(args.warmup):
         one_step()
     torch.cuda.synchronize()
     for _, _, r in runs:
         assert r.read_status() == 0, "device status bits set"
+    graph = None
+    if not args.no_graph:
+        # the step as one CUDA graph; its stage events are graph nodes that record on replay
+        g_ev = {n: (torch.cuda.Event(enable_timing=True, external=True),
+                    torch.cuda.Event(enable_timing=True, external=True)) for n in stage_names}
+        from long_context_sparse_softmax_b200.runner import capture_step
+        graph = capture_step([r for _, _, r in runs], stream, side, timed(g_ev))
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
 
     ev = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in stage_names}
           for _ in range(args.steps)]
@@ -325,15 +349,35 @@ def run_lc(args):
         gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         gpu_id = str(local)
+    per_stage = {n: [] for n in stage_names}
+    stage_src = "eager" if graph is None else "graph"
     with ClockSampler(gpu_id) as clk:
         for s in range(args.steps):
-            flush.zero_()
+            flush_l2()
             ev_step[s][0].record(stream)
-            one_step(ev[s])
+            if graph is None:
+                one_step(ev[s])
+            else:
+                graph.replay()
             ev_step[s][1].record(stream)
+            if graph is not None and stage_src == "graph":
+                # the graph's stage events are re-recorded by every replay: read them now
+                ev_step[s][1].synchronize()
+                try:
+                    for n in stage_names:
+                        per_stage[n].append(g_ev[n][0].elapsed_time(g_ev[n][1]))
+                except RuntimeError:
+                    stage_src = "eager"
         torch.cuda.synchronize()
     barrier()
-    per_stage = {n: [ev[s][n][0].elapsed_time(ev[s][n][1]) for s in range(args.steps)] for n in stage_names}
+    if stage_src == "eager":
+        if graph is not None:
+            # per-stage times from eager steps (same flush) when graph event nodes give none
+            for s in range(args.steps):
+                flush_l2()
+                one_step(ev[s])
+            torch.cuda.synchronize()
+        per_stage = {n: [ev[s][n][0].elapsed_time(ev[s][n][1]) for s in range(args.steps)] for n in stage_names}
     # a step's time runs from the fork on the main stream to the end of attention
     span = [ev_step[s][0].elapsed_time(ev_step[s][1]) for s in range(args.steps)]
     total_ms = sum(span)
@@ -354,12 +398,15 @@ def run_lc(args):
         torch.cuda.synchronize()
         e_ms = 0.0
         for s in range(args.steps):
-            flush.zero_()
+            flush_l2()
             e0.record(stream)
             for ins, _ in io:
                 for d, h in ins:
                     d.copy_(h, non_blocking=True)
-            one_step()
+            if graph is None:
+                one_step()
+            else:
+                graph.replay()
             for _, outs in io:
                 for d, h in outs:
                     h.copy_(d, non_blocking=True)
@@ -404,7 +451,10 @@ def run_lc(args):
                    "batch": runs[0][0].num_seqs if runs[0][0].is_decode else 1,
                    "context": max(runs[0][0].seq_lens), "heads": runs[0][0].H, "dims": runs[0][0].D,
                    "topk": runs[0][0].k, "query_tokens_per_step_per_gpu": units,
-                   "l2": "flushed between timed steps (512 MiB write outside the step events)",
+                   "l2": "flushed between timed steps, outside the step events (512 MiB write, then a "
+                         "256 MiB read so that evicted lines are clean)",
+                   "launch": "eager" if graph is None else "cuda graph of the step",
+                   "stage_times": stage_src,
                    "parallelism": f"replicas x{world} (independent batches)"},
         "roofline": {"bound": bnd, "kernel": dom.split(":")[1], "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic, "peak_source": pk_kind},

@@ -72,10 +72,12 @@ class _Common:
         fork = torch.cuda.Event()
         fork.record(main)
         side.wait_event(fork)
-        for n, f in sd:
-            run(n, side, f)
+        # the critical path is enqueued first, so its CTAs take the SMs before the side
+        # stream's do
         for n, f in mn:
             run(n, main, f)
+        for n, f in sd:
+            run(n, side, f)
         join = torch.cuda.Event()
         join.record(side)
         main.wait_event(join)
@@ -270,6 +272,24 @@ class Decode(_Common):
     def step(self, stream=None):
         for _, f in self.stages():
             f(stream)
+
+
+def capture_step(runs, main, side, on_stage=None):
+    """Record one overlapped step of every run in `runs` as a CUDA graph (on_stage, if
+    given, is called as on_stage(run index, stage name, stream, launch)).
+
+    The library calls are made once, during capture; `graph.replay()` then launches the
+    same kernels with the same arguments on the current stream, with the fork onto `side`
+    and the join before attention kept as graph edges.  Each run's buffers and arguments
+    are fixed at capture: refill the input tensors in place between replays.  Make one
+    eager step first, so that one-time set-up (kernel attributes, the no-allocation
+    scratch address) happens outside the capture."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=main):
+        for i, r in enumerate(runs):
+            r.step_overlapped(main, side, None if on_stage is None else
+                              (lambda name, st, fn, i=i: on_stage(i, name, st, fn)))
+    return g
 
 
 def make_run(spec: wl.Spec, device="cuda", W_x: Optional[int] = None):
