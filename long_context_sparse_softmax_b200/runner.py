@@ -64,23 +64,29 @@ class _Common:
         return side, main, [("attn", st["attn"])]
 
     def step_overlapped(self, main, side, on_stage=None):
-        """One step on two streams: fork `side` from `main`, join before attention.
-        on_stage(name, stream, fn) may wrap each launch (e.g. with timing events)."""
+        """One step on several streams: the side stages fork from `main` (stage i on
+        side[i % len(side)]; `side` is one stream or a list) and join it before
+        attention.  on_stage(name, stream, fn) may wrap each launch (e.g. with timing
+        events)."""
         import torch
         sd, mn, af = self.dag()
+        sides = list(side) if isinstance(side, (list, tuple)) else [side]
         run = on_stage or (lambda name, stream, fn: fn(stream))
         fork = torch.cuda.Event()
         fork.record(main)
-        side.wait_event(fork)
+        used = sides[:len(sd)]
+        for st in used:
+            st.wait_event(fork)
         # the critical path is enqueued first, so its CTAs take the SMs before the side
-        # stream's do
+        # streams' do
         for n, f in mn:
             run(n, main, f)
-        for n, f in sd:
-            run(n, side, f)
-        join = torch.cuda.Event()
-        join.record(side)
-        main.wait_event(join)
+        for i, (n, f) in enumerate(sd):
+            run(n, sides[i % len(sides)], f)
+        for st in used:
+            join = torch.cuda.Event()
+            join.record(st)
+            main.wait_event(join)
         for n, f in af:
             run(n, main, f)
 
