@@ -277,6 +277,9 @@ typedef struct lc_attn_args {
   int32_t n_ent_rows;      /* rows of ent (every ent_start[b] + n_ent[b] <= n_ent_rows), or 0 if
                               unknown; the FP8 tensor-core kernel reads entries by bulk tensor
                               copies and needs it */
+  int32_t n_win_rows;      /* rows of win (every win_start[b] + win_len[b] <= n_win_rows), or 0
+                              if unknown; with W > 0 the FP8 tensor-core kernel reads window
+                              rows by bulk tensor copies and needs it */
 } lc_attn_args;
 
 /* Attention kernels. */
@@ -285,7 +288,8 @@ enum {
   LC_IMPL_MMA = 1,         /* BF16 mma.sync tiles (576-dim entries) */
   LC_IMPL_TC = 2,          /* tcgen05 tiles, accumulators in tensor memory (576-dim entries):
                               E4M3 scores from bulk-copied tiles where queries and entries are
-                              E4M3 + BF16 RoPE and n_ent_rows is set, else the F16 kernel */
+                              E4M3 + BF16 RoPE and n_ent_rows (and, with W > 0, n_win_rows)
+                              is set, else the F16 kernel */
   LC_IMPL_REF = 3,         /* one warp per (query, head), FP32 CUDA cores (any shape) */
   LC_IMPL_TC_F16 = 4       /* tcgen05 tiles with every operand widened to F16 */
 };

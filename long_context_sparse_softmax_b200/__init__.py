@@ -75,7 +75,8 @@ class AttnArgs(ctypes.Structure):
                 ("max_ent", c_int32), ("scale", c_float), ("out_fmt", c_int32), ("q", Rows), ("ent", Rows),
                 ("win", Rows), ("idx", c_void_p), ("sink", c_void_p), ("batch", Batch), ("out", c_void_p),
                 ("lse", c_void_p), ("workspace", c_void_p), ("workspace_bytes", c_size_t), ("status", c_void_p),
-                ("impl", c_int32), ("n_ent_rows", c_int32)]
+                ("impl", c_int32), ("n_ent_rows", c_int32),
+                ("n_win_rows", c_int32)]
 
 
 LC_IMPL_AUTO, LC_IMPL_MMA, LC_IMPL_TC, LC_IMPL_REF, LC_IMPL_TC_F16 = 0, 1, 2, 3, 4

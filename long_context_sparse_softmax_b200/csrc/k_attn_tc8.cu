@@ -21,9 +21,11 @@
 // Softmax, the per-head exponent reference, the sink and the outputs are those of
 // k_attn_tc.cu (P in F16, 11 significant bits; row sums of the rounded P).
 //
-// Warp roles (320 threads): warps 0-3 turn S into P and write the output; warps 4-7
-// convert tiles; lane 0 of warp 8 issues the MMAs; warp 9 computes the key codes and
-// issues the bulk copies.  Every mbarrier wait is bounded: a role that gives up sets
+// Warp roles (416 threads): warps 0-3 turn S into P and write the output; warps 4-7
+// convert tiles and bring in the window tiles; lane 0 of warp 8 issues the MMAs; warps
+// 9-12 compute the key codes and issue the entry-tile gathers, a quarter of each tile per
+// warp (a warp issues bulk copies one lane at a time, so four warps issue a tile about
+// four times as fast as one).  Every mbarrier wait is bounded: a role that gives up sets
 // LC_DEV_TIMEOUT and an abort flag that stops the others at their next wait.
 #include <cuda.h>
 
@@ -46,7 +48,8 @@ constexpr int kRawStage = kRawN + kBlk;   // + BF16 RoPE part: 40 KB
 constexpr int kPBytes = kNR * kTK * 2;
 constexpr long kSpin = 1L << 26;
 constexpr uint32_t kWin = 1u << 30;
-constexpr int kThreads = 320;
+constexpr int kThreads = 416;
+constexpr int kCopyWarps = 4;            // warps 9 .. 12: key codes and bulk copies
 constexpr float kRescale = 8.f;
 constexpr int kColS = 0;                  // S buffers at columns 0 and 64
 constexpr int kColO = 2 * kTK;            // O^T chunk c at 128 + 64 c
@@ -77,6 +80,17 @@ __device__ __forceinline__ uint64_t cm_desc(uint32_t addr, uint32_t lbo, uint32_
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
   uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFF);
   d |= static_cast<uint64_t>(1) << 16;
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+// MN-major SWIZZLE_128B operand: 128-byte rows run along M (64 16-bit values), one row per
+// K index, 8-row groups 1024 bytes apart (SBO); the next 64 values of M start kBlk bytes
+// further (LBO)
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t addr) {
+  uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>(kBlk >> 4) << 16;
   d |= static_cast<uint64_t>(1024 >> 4) << 32;
   d |= static_cast<uint64_t>(1) << 46;
   d |= static_cast<uint64_t>(2) << 61;
@@ -228,24 +242,13 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-__device__ __forceinline__ void cp16(uint8_t* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(su32(dst)), "l"(src) : "memory");
-}
-
-__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(gdst), "r"(su32(ssrc)),
-               "r"(bytes)
-               : "memory");
-  asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
-  asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
-}
-
 struct Bars {
   uint64_t qfull;      // Q nope + RoPE landed (expect-tx)
-  uint64_t kfull[2];   // raw stage landed (expect-tx)
+  uint64_t kfull[2];   // raw stage landed (expect-tx; one arrival per copy warp)
   uint64_t kempty[2];  // raw stage read by S (commit) and by the converter (1 arrival)
-  uint64_t cready[4];  // key codes of a tile written (1 arrival)
+  uint64_t cready[4];  // key codes of a tile written (one arrival per copy warp)
   uint64_t cfree[4];   // key codes of a tile read by the softmax (128 arrivals)
+  uint64_t wfull;      // window tile landed in the F16 tile area (expect-tx)
   uint64_t vfull;      // F16 tile ready (1 arrival)
   uint64_t vempty;     // F16 tile read by O (commit)
   uint64_t q16full;    // Q in F16 ready for the window tiles (1 arrival)
@@ -260,7 +263,8 @@ struct Bars {
 
 struct AttnTc8Geom {
   int n_split;
-  int sps;  // slots per split, multiple of kTK
+  int sps;       // slots per split, multiple of kTK
+  int win_own;   // 1: the last split takes every window slot, the others the entry slots
 };
 
 // grid: one CTA per (query, head group, key split), the split index fastest; 320 threads.
@@ -268,8 +272,9 @@ struct AttnTc8Geom {
 // ws_ml[2 ((q * H + h) * n_split + s) + {0, 1}] = (m, l).
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_tc8(const __grid_constant__ CUtensorMap tqn, const __grid_constant__ CUtensorMap tqr,
-               const __grid_constant__ CUtensorMap tkn, const __grid_constant__ CUtensorMap tkr, lc_attn_args a,
-               int sparse, AttnTc8Geom geo, float* __restrict__ ws_o, float* __restrict__ ws_ml) {
+               const __grid_constant__ CUtensorMap tkn, const __grid_constant__ CUtensorMap tkr,
+               const __grid_constant__ CUtensorMap twin, lc_attn_args a,
+               int sparse, int decode, AttnTc8Geom geo, float* __restrict__ ws_o, float* __restrict__ ws_ml) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* Qn = smem + kOffQn;
@@ -290,16 +295,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int hg = (blockIdx.x / geo.n_split) % n_hg;
   const int q = blockIdx.x / (geo.n_split * n_hg);
   const int H = a.dims.H;
-  const int b = seq_of_query(a.batch.q_start, a.batch.num_seqs, q);
-  const int p = __ldg(a.batch.q_pos0 + b) + (q - __ldg(a.batch.q_start + b));
+  // decode: one query per sequence (q_start[b] = b), so the per-sequence loads below are
+  // independent of one another
+  const int b = decode ? q : seq_of_query(a.batch.q_start, a.batch.num_seqs, q);
+  const int p = __ldg(a.batch.q_pos0 + b) + (decode ? 0 : q - __ldg(a.batch.q_start + b));
   const int n_ent = __ldg(a.batch.n_ent + b);
   const int nv = n_visible(p, a.m, a.W_x, n_ent);
   const int64_t ent0 = __ldg(a.batch.ent_start + b);
   const int wlo = a.W > 0 ? max(0, p - a.W + 1) : p + 1;
   const int n_first = sparse ? a.k : nv;
   const int n_slots = n_first + (p + 1 - wlo);
-  const int s_begin = split * geo.sps;
-  const int s_end = min(n_slots, s_begin + geo.sps);
+  int s_begin, s_end;
+  if (!geo.win_own) {
+    s_begin = split * geo.sps;
+    s_end = min(n_slots, s_begin + geo.sps);
+  } else if (split == geo.n_split - 1) {
+    s_begin = n_first;
+    s_end = n_slots;
+  } else {
+    s_begin = min(split * geo.sps, n_first);
+    s_end = min(s_begin + geo.sps, n_first);
+  }
   // entry tiles cover [s_begin, min(s_end, n_first)), window tiles the rest of the range
   const int e_end = min(s_end, n_first);
   const int n_et = e_end > s_begin ? (e_end - s_begin + kTK - 1) / kTK : 0;
@@ -359,15 +375,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_abort = 0;
     mbar_init(su32(&bars.qfull), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(su32(&bars.kfull[i]), 1);
+      mbar_init(su32(&bars.kfull[i]), kCopyWarps);
       mbar_init(su32(&bars.kempty[i]), 2);
       mbar_init(su32(&bars.sfull[i]), 1);
       mbar_init(su32(&bars.sempty[i]), 128);
     }
     for (int i = 0; i < 4; ++i) {
-      mbar_init(su32(&bars.cready[i]), 1);
+      mbar_init(su32(&bars.cready[i]), kCopyWarps);
       mbar_init(su32(&bars.cfree[i]), 128);
     }
+    mbar_init(su32(&bars.wfull), 1);
     mbar_init(su32(&bars.vfull), 1);
     mbar_init(su32(&bars.vempty), 1);
     mbar_init(su32(&bars.q16full), 1);
@@ -381,9 +398,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   fence_after();
   const uint32_t tm = s_tmem;
 
-  if (warp == 9) {
+  if (warp >= 9) {
     // ================= key codes and bulk copies =================
-    if (lane == 0 && n_tiles > 0) {
+    // Four warps share each tile: a warp issues its bulk copies one lane after another, so
+    // the copies of a tile go out about four times faster from four warps than from one.
+    // Copy warp cw owns keys 16 cw .. 16 cw + 15 of every tile.
+    const int cw = warp - 9;
+    if (cw == 0 && lane == 0 && n_tiles > 0) {
       const uint32_t qb = su32(&bars.qfull);
       mbar_expect_tx(qb, kRawN + kBlk);
 #pragma unroll
@@ -398,19 +419,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && t < n_et && t >= 2) ok = wait(&bars.kempty[t & 1], ((t >> 1) - 1) & 1);
       if (!__all_sync(0xffffffffu, ok)) break;
       const int s0 = tile_slot0(t), s_lim = tile_slot_end(t);
-      int* kc = kcode + cb4 * kTK;
-      const int c0 = slot_code(s0 + lane, s_lim), c1 = slot_code(s0 + 32 + lane, s_lim);
-      kc[lane] = c0;
-      kc[32 + lane] = c1;
+      int* kc = kcode + cb4 * kTK + 16 * cw;
+      if (lane < 16) kc[lane] = slot_code(s0 + 16 * cw + lane, s_lim);
       __syncwarp();
       if (lane == 0) mbar_arrive(su32(&bars.cready[cb4]));
       if (t < n_et) {
         const int st = t & 1;
         const uint32_t kb = su32(&bars.kfull[st]);
-        if (lane == 0) mbar_expect_tx(kb, kRawStage);
+        if (lane == 0) mbar_expect_tx(kb, kRawStage / kCopyWarps);
         __syncwarp();
-        if (lane < kTK / 4) {
-          // rows 4 lane .. 4 lane + 3; a masked key reads row 0 (its P is 0)
+        if (lane < 4) {
+          // rows 4 g .. 4 g + 3 of the tile, g = 4 cw + lane; a masked key reads row 0 (its
+          // P is 0)
+          const int g = 4 * cw + lane;
           int rr[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -420,8 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* stage = Raw + st * kRawStage;
 #pragma unroll
           for (int cb = 0; cb < 4; ++cb)
-            tma_gather4(su32(stage + cb * kBlk + lane * 512), &tkn, cb * 128, rr[0], rr[1], rr[2], rr[3], kb);
-          tma_gather4(su32(stage + kRawN + lane * 512), &tkr, 0, rr[0], rr[1], rr[2], rr[3], kb);
+            tma_gather4(su32(stage + cb * kBlk + g * 512), &tkn, cb * 128, rr[0], rr[1], rr[2], rr[3], kb);
+          tma_gather4(su32(stage + kRawN + g * 512), &tkr, 0, rr[0], rr[1], rr[2], rr[3], kb);
         }
       }
     }
@@ -465,9 +486,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma<0>(d, sw128_desc(su32(Qr) + k * 32), sw128_desc(st + kRawN + k * 32), id_sbf, 1);
               mma_commit(su32(&bars.kempty[ns & 1]));
             } else {
-              const uint64_t dq = cm_desc(su32(Q16), 128, kG), dk = cm_desc(su32(Vt), 128, kG);
+              // A: Q in F16 (core matrices); B: the window tile, SW128, 64 dims per block
+              const uint64_t dq = cm_desc(su32(Q16), 128, kG);
 #pragma unroll
-              for (int k = 0; k < kD / 16; ++k) mma<0>(d, dq + k * 16, dk + k * 16, id_sf16, k > 0);
+              for (int k = 0; k < kD / 16; ++k)
+                mma<0>(d, dq + k * 16, sw128_desc(su32(Vt) + (k >> 2) * kBlk + (k & 3) * 32), id_sf16, k > 0);
             }
             mma_commit(su32(&bars.sfull[sb]));
             ++ns;
@@ -476,12 +499,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (no < ns && mbar_probe(su32(&bars.pfull), no & 1) && mbar_probe(su32(&bars.vfull), no & 1)) {
           fence_after();
+          if (no < n_et) {
 #pragma unroll
-          for (int kk = 0; kk < kTK / 16; ++kk)
+            for (int kk = 0; kk < kTK / 16; ++kk)
 #pragma unroll
-            for (int c = 0; c < 5; ++c)
-              mma<0>(tm + kColO + c * kNR, dv + (c * 2048 + kk * 2 * kG) / 16, dp + kk * 16, c < 4 ? id_o128 : id_o64,
-                     (no > 0) || (kk > 0));
+              for (int c = 0; c < 5; ++c)
+                mma<0>(tm + kColO + c * kNR, dv + (c * 2048 + kk * 2 * kG) / 16, dp + kk * 16,
+                       c < 4 ? id_o128 : id_o64, (no > 0) || (kk > 0));
+          } else {
+            // window tile: V^T straight from the SW128 tile (dims along M, 16 keys per step)
+#pragma unroll
+            for (int kk = 0; kk < kTK / 16; ++kk)
+#pragma unroll
+              for (int c = 0; c < 5; ++c)
+                mma<0>(tm + kColO + c * kNR, sw128_mn_desc(su32(Vt) + c * 2 * kBlk + kk * 2048), dp + kk * 16,
+                       c < 4 ? id_o128 : id_o64, (no > 0) || (kk > 0));
+          }
           mma_commit(su32(&bars.vempty));
           mma_commit(su32(&bars.pempty));
           ++no;
@@ -495,6 +528,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
         } else if ((idle & 1023) == 0 && *reinterpret_cast<volatile int*>(&s_abort)) {
           ok = false;
+        } else {
+          // nothing ready: yield the issue slots this polling loop would take from the
+          // converter and softmax warps
+          __nanosleep(32);
         }
       }
       mma_commit(su32(&bars.fin));
@@ -507,6 +544,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     __half2 amax = __float2half2_rn(0.f);
     bool ok = true;
     for (int t = 0; ok && t < n_tiles; ++t) {
+      if (t >= n_et) {
+        // window tile: its rows are consecutive, so it comes as one 64 x 64 BF16 box per 64
+        // dims (SW128) straight into the F16 tile area, once O of tile t - 1 is done (these
+        // warps wait for every phase of vempty in order; rows past the window are masked by
+        // their codes)
+        const bool okv = t == 0 || wait(&bars.vempty, (t - 1) & 1);
+        if (named_bar_or(2, 128, !okv)) {
+          ok = false;
+          break;
+        }
+        if (ct == 0) {
+          const uint32_t wb = su32(&bars.wfull);
+          mbar_expect_tx(wb, kTile);
+          const int y = static_cast<int>(wr0) + wlo + (tile_slot0(t) - n_first) - wp0;
+#pragma unroll
+          for (int cb = 0; cb < kD / 64; ++cb) tma_tile2d(su32(Vt + cb * kBlk), &twin, cb * 64, y, wb);
+        }
+      }
       if (t == n_et) {
         // window phase: Q to F16 in the raw stages, once S and the conversion of every
         // entry tile are done (the raw stages are free)
@@ -542,45 +597,62 @@ __global__ void __launch_bounds__(kThreads, 1)
       // raw rows have landed
       bool okw = t == 0 || wait(&bars.vempty, (t - 1) & 1);
       if (t < n_et) okw = okw && wait(&bars.kfull[t & 1], (t >> 1) & 1);
-      else okw = okw && wait(&bars.cready[t & 3], (t >> 2) & 1);
+      else okw = okw && wait(&bars.cready[t & 3], (t >> 2) & 1) && wait(&bars.wfull, (t - n_et) & 1);
       if (named_bar_or(2, 128, !okw)) {
         ok = false;
         break;
       }
       if (t < n_et) {
         const uint8_t* st = Raw + (t & 1) * kRawStage;
-        // 64 keys x (32 E4M3 pieces of 16 dims + 8 BF16 chunks); a quarter warp takes 8
-        // rows of one piece: its SW128 reads and its core-matrix writes hit distinct banks
-        for (int i = ct; i < kTK * 40; i += 128) {
-          const int g = i >> 3, pc = g % 40, r = (g / 40) * 8 + r8;
-          if (pc < 32) {
-            const uint4 v = *reinterpret_cast<const uint4*>(st + (pc >> 3) * kBlk + sw128_off(r, pc & 7));
+        // 64 keys x 32 E4M3 pieces of 16 dims, then 64 keys x 8 BF16 chunks; a quarter warp
+        // takes 8 rows of one piece (its SW128 reads and its core-matrix writes hit
+        // distinct banks); the loads of four pieces are issued before any is converted
+#pragma unroll 1
+        for (int k0 = 0; k0 < kTK * 32 / 128; k0 += 4) {
+          uint4 v[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int g = (ct + 128 * (k0 + u)) >> 3, pc = g & 31, r = (g >> 5) * 8 + r8;
+            v[u] = *reinterpret_cast<const uint4*>(st + (pc >> 3) * kBlk + sw128_off(r, pc & 7));
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int g = (ct + 128 * (k0 + u)) >> 3, pc = g & 31, r = (g >> 5) * 8 + r8;
             uint4 lo, hi;
-            e4m3x16_f16(v, lo, hi);
+            e4m3x16_f16(v[u], lo, hi);
             *reinterpret_cast<uint4*>(Vt + tile_off(r, 2 * pc)) = lo;
             *reinterpret_cast<uint4*>(Vt + tile_off(r, 2 * pc + 1)) = hi;
-          } else {
-            const int j = pc - 32;
-            const uint4 v = *reinterpret_cast<const uint4*>(st + kRawN + sw128_off(r, j));
-            *reinterpret_cast<uint4*>(Vt + tile_off(r, 64 + j)) = bf16x8_f16(v, amax);
+          }
+        }
+        {
+          uint4 v[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int g = (ct + 128 * u) >> 3, j = g & 7, r = (g >> 3) * 8 + r8;
+            v[u] = *reinterpret_cast<const uint4*>(st + kRawN + sw128_off(r, j));
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int g = (ct + 128 * u) >> 3, j = g & 7, r = (g >> 3) * 8 + r8;
+            *reinterpret_cast<uint4*>(Vt + tile_off(r, 64 + j)) = bf16x8_f16(v[u], amax);
           }
         }
       } else {
-        // window rows (BF16, 72 chunks each) straight into the tile, then rounded to F16
+        // window tile (SW128 BF16: 16-byte chunk i holds 8 dims of row (i / 8) % 64) rounded
+        // to F16 in place; rows of masked keys are zeroed
         const int* kc = kcode + (t & 3) * kTK;
-        for (int i = ct; i < kTK * 72; i += 128) {
-          const int g = i >> 3, c = g % 72, r = (g / 72) * 8 + r8;
-          const int code = kc[r];
-          uint8_t* dst = Vt + tile_off(r, c);
-          if (code < 0 || !(code & kWin)) *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-          else cp16(dst, static_cast<const uint8_t*>(a.win.x) + ((wr0 + (code & ~kWin)) * kD + c * 8) * 2);
-        }
-        asm volatile("cp.async.commit_group;\ncp.async.wait_all;\n" ::: "memory");
-        named_bar(2, 128);
-        for (int i = ct; i < kTK * 72; i += 128) {
-          const int g = i >> 3, c = g % 72, r = (g / 72) * 8 + r8;
-          uint4* d = reinterpret_cast<uint4*>(Vt + tile_off(r, c));
-          *d = bf16x8_f16(*d, amax);
+#pragma unroll 1
+        for (int k0 = 0; k0 < kTile / 16 / 128; k0 += 4) {
+          uint4 v[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const uint4*>(Vt + (ct + 128 * (k0 + u)) * 16);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = ct + 128 * (k0 + u);
+            const int code = kc[(i >> 3) & (kTK - 1)];
+            *reinterpret_cast<uint4*>(Vt + i * 16) =
+                code < 0 || !(code & kWin) ? make_uint4(0, 0, 0, 0) : bf16x8_f16(v[u], amax);
+          }
         }
       }
       fence_async_smem();
@@ -698,11 +770,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     named_bar(1, 128);
     if (good) {
-      // O rows -> the raw stages (free: every MMA is complete), row-major [head][dim]
+      // O^T (dims on tensor-memory lanes, heads on columns) straight to global memory:
+      // for each head a warp writes 32 consecutive dims, 128 bytes in FP32
       const bool f32 = geo.n_split > 1 || a.out_fmt == LC_FMT_F32;
-      uint8_t* stage_out = Raw;  // 2 raw stages (80 KB) + the F16 tile (72 KB) are contiguous
-      float* stf = reinterpret_cast<float*>(stage_out);
-      uint16_t* sth = reinterpret_cast<uint16_t*>(stage_out);
+      float* of = nullptr;
+      uint16_t* oh = nullptr;
+      if (geo.n_split > 1) of = ws_o + (static_cast<int64_t>(split) * a.n_q * H + row0) * kD;
+      else if (f32) of = static_cast<float*>(a.out) + row0 * kD;
+      else oh = static_cast<uint16_t*>(a.out) + row0 * kD;
 #pragma unroll 1
       for (int c = 0; c < 5; ++c) {
         const int dim = c < 4 ? c * 128 + warp * 32 + lane : (lane < 16 ? 512 + warp * 16 + lane : -1);
@@ -720,19 +795,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kNR; ++i) {
           float v = __uint_as_float(ov[i]);
           if (geo.n_split == 1) v *= s_f[i];
-          if (f32) stf[i * kD + dim] = v;
-          else sth[i * kD + dim] = f32_to_bf16_bits(v);
+          if (f32) of[i * kD + dim] = v;
+          else oh[i * kD + dim] = f32_to_bf16_bits(v);
         }
-      }
-      fence_async_smem();
-      named_bar(1, 128);
-      if (tid == 0) {
-        const uint32_t bytes = kNR * kD * (f32 ? 4 : 2);
-        void* dst;
-        if (geo.n_split > 1) dst = ws_o + (static_cast<int64_t>(split) * a.n_q * H + row0) * kD;
-        else if (a.out_fmt == LC_FMT_F32) dst = static_cast<float*>(a.out) + row0 * kD;
-        else dst = static_cast<uint16_t*>(a.out) + row0 * kD;
-        bulk_store(dst, stage_out, bytes);
       }
     }
   }
@@ -745,7 +810,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 bool attn_tc8_supported(const lc_attn_args& a) {
   if (a.dims.D != kD || a.dims.d_r != kDR || a.dims.H % kNR || a.n_ent_rows < 1) return false;
   if (a.q.fmt != LC_FMT_E4M3_BF16 || a.ent.fmt != LC_FMT_E4M3_BF16) return false;
-  if (a.W > 0 && a.win.fmt != LC_FMT_BF16) return false;
+  if (a.W > 0 && (a.win.fmt != LC_FMT_BF16 || a.n_win_rows < 1)) return false;
   auto al = [](const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; };
   if (!al(a.q.x) || !al(a.q.rope) || !al(a.ent.x) || !al(a.ent.rope) || (a.W > 0 && !al(a.win.x))) return false;
   if (!al(a.out) || !al(a.workspace)) return false;
@@ -753,9 +818,14 @@ bool attn_tc8_supported(const lc_attn_args& a) {
   return a.out_fmt == LC_FMT_BF16 || a.out_fmt == LC_FMT_F32;
 }
 
+// Decode splits the keys of each (query, head group) over up to 148 / CTAs splits.  A
+// window tile costs about two entry tiles (72 KB of BF16 rows against 40 KB, plus its
+// conversion in place), so when the window tiles fit one split that is no longer than the
+// entry splits, they get a split of their own.
 static AttnTc8Geom tc8_geometry(const lc_attn_args& a, bool sparse, bool decode) {
-  AttnTc8Geom g{1, 0};
-  const int ns = max((sparse ? a.k : a.max_ent) + a.W, 1);
+  AttnTc8Geom g{1, 0, 0};
+  const int ne = sparse ? a.k : a.max_ent;
+  const int ns = max(ne + a.W, 1);
   const int tiles = (ns + kTK - 1) / kTK;
   g.sps = tiles * kTK;
   const int ctas = a.n_q * (a.dims.H / kNR);
@@ -764,6 +834,17 @@ static AttnTc8Geom tc8_geometry(const lc_attn_args& a, bool sparse, bool decode)
     const int per = (tiles + n - 1) / n;
     g.n_split = (tiles + per - 1) / per;
     g.sps = per * kTK;
+    const int te = (ne + kTK - 1) / kTK, tw = (a.W + kTK - 1) / kTK;
+    if (a.W > 0 && n >= 2 && te >= 1) {
+      const int per_e = (te + n - 2) / (n - 1);
+      // cost in entry-tile units: uniform splits put up to one window tile next to `per`
+      // tiles; the own-split layout costs max(per_e, 2 tw)
+      if (max(per_e, 2 * tw) < per + 1) {
+        g.win_own = 1;
+        g.sps = per_e * kTK;
+        g.n_split = (te + per_e - 1) / per_e + 1;
+      }
+    }
   }
   return g;
 }
@@ -812,19 +893,25 @@ cudaError_t launch_attn_tc8(const lc_attn_args& a, bool sparse, bool decode, cud
   const AttnTc8Geom g = tc8_geometry(a, sparse, decode);
   *n_split_out = g.n_split;
   const int64_t qrows = static_cast<int64_t>(a.n_q) * a.dims.H;
-  CUtensorMap tqn, tqr, tkn, tkr;
+  CUtensorMap tqn, tqr, tkn, tkr, twin;
   if (!make_map(&tqn, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q.x, qrows, kDN, 1, 128, kNR) ||
       !make_map(&tqr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.q.rope, qrows, kDR, 2, 64, kNR) ||
       !make_map(&tkn, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.ent.x, a.n_ent_rows, kDN, 1, 128, 1) ||
       !make_map(&tkr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.ent.rope, a.n_ent_rows, kDR, 2, 64, 1))
     return cudaErrorInvalidValue;
+  if (a.W > 0) {
+    if (!make_map(&twin, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.win.x, a.n_win_rows, kD, 2, 64, kTK))
+      return cudaErrorInvalidValue;
+  } else {
+    twin = tkr;  // no window tiles: never read
+  }
   cudaFuncSetAttribute(k_attn_tc8, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
   float* ws_o = static_cast<float*>(a.workspace);
   float* ws_ml = nullptr;
   if (g.n_split > 1) ws_ml = ws_o + static_cast<size_t>(a.n_q) * a.dims.H * g.n_split * kD;
   const int64_t ctas = static_cast<int64_t>(a.n_q) * (a.dims.H / kNR) * g.n_split;
   if (ctas > 0x7fffffff) return cudaErrorInvalidConfiguration;
-  k_attn_tc8<<<static_cast<unsigned>(ctas), kThreads, kSmem, st>>>(tqn, tqr, tkn, tkr, a, sparse ? 1 : 0, g, ws_o,
+  k_attn_tc8<<<static_cast<unsigned>(ctas), kThreads, kSmem, st>>>(tqn, tqr, tkn, tkr, twin, a, sparse ? 1 : 0, decode ? 1 : 0, g, ws_o,
                                                                   ws_ml);
   return cudaGetLastError();
 }

@@ -123,6 +123,7 @@ class _Common:
         a.status = ptr(self.status)
         a.impl = self.impl
         a.n_ent_rows = int(next(iter(self.ent.values())).shape[0])
+        a.n_win_rows = int(self.win["x"].shape[0])
         ws = (lc_csa_sparse_attn_workspace_bytes if sparse else lc_hca_attn_workspace_bytes)(a)
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.device)
         a.workspace, a.workspace_bytes = ptr(self.workspace), ws
