@@ -39,7 +39,7 @@ constexpr int kKeys = 128;          // keys per tile (MMA M)
 constexpr int kDI = 128;            // indexer dims handled here (2 MMAs of K = 64)
 constexpr int kRowB = kDI / 2;      // bytes per row
 constexpr int kTileB = kKeys * kRowB;
-constexpr int kStages = 4;
+constexpr int kStages = 8;            // key tiles in flight per CTA (2 CTAs per SM: 128 KB)
 constexpr int kThreads = 192;
 constexpr long kSpin = 1L << 26;
 constexpr int kDBuf = 3;            // tensor-memory accumulators
@@ -128,7 +128,8 @@ struct IdxBars {
 // query scales at 3N + 16 (N / 32 columns).
 template <int QPC>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_index_tc(const __grid_constant__ CUtensorMap tk, lc_index_args a, int tiles_per_cta, uint32_t tmem_cols) {
+    k_index_tc(const __grid_constant__ CUtensorMap tk, lc_index_args a, int tiles_per_cta, uint32_t tmem_cols,
+               int decode) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int H = a.H_I;
   const int N = QPC * H;
@@ -145,7 +146,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qa = blockIdx.x * QPC;
   if (qa >= a.n_q) return;
-  const int b = seq_of_query(a.batch.q_start, a.batch.num_seqs, qa);
+  // decode: one query per sequence (q_start[b] = b), no search
+  const int b = decode ? qa : seq_of_query(a.batch.q_start, a.batch.num_seqs, qa);
   const int64_t kbase = __ldg(a.batch.ent_start + b);
   const int n_ent = __ldg(a.batch.n_ent + b);
   // queries of this chunk: they must belong to sequence b (prefill: one sequence;
@@ -153,8 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid < QPC) {
     const int q = qa + tid;
     int nv = 0;
-    if (q < a.n_q && q < __ldg(a.batch.q_start + b + 1)) {
-      const int p = __ldg(a.batch.q_pos0 + b) + (q - __ldg(a.batch.q_start + b));
+    if (q < a.n_q && (decode || q < __ldg(a.batch.q_start + b + 1))) {
+      const int p = __ldg(a.batch.q_pos0 + b) + (decode ? 0 : q - __ldg(a.batch.q_start + b));
       nv = n_visible(p, a.m, a.W_x, n_ent);
     }
     s_nv[tid] = nv;
@@ -216,21 +218,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         w[c] = j < n_ent ? __ldg(reinterpret_cast<const uint32_t*>(a.k_scale + (kbase + j) * 4)) : 0u;
       }
     };
-    uint32_t sfw[4];
-    sf_load(0, sfw);
-    for (int it = 0; it < n_tiles; ++it) {
-      const int s = it % kStages;
-      const int t = t_begin + it;
-      if (it >= kStages && !__all_sync(0xffffffffu, wait(&bars.kempty[s], ((it / kStages) - 1) & 1))) break;
-      const uint32_t full = su32(&bars.kfull[s]);
-      if (lane == 0) {
-        mbar_expect_tx(full, kTileB);
-        tma_load_2d(su32(As + s * kTileB), &tk, 0, static_cast<int>(kbase + static_cast<int64_t>(t) * kKeys), full);
+    // the scale words travel four tiles ahead of their key tile, in a register ring (slot
+    // = tile % 4), so no iteration waits for a load it has just issued
+    uint32_t sfw[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (u < n_tiles) sf_load(u, sfw[u]);
+    bool go = true;
+    for (int it0 = 0; go && it0 < n_tiles; it0 += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int it = it0 + u;
+        if (it >= n_tiles) break;
+        const int s = it % kStages;
+        const int t = t_begin + it;
+        if (it >= kStages && !__all_sync(0xffffffffu, wait(&bars.kempty[s], ((it / kStages) - 1) & 1))) {
+          go = false;
+          break;
+        }
+        const uint32_t full = su32(&bars.kfull[s]);
+        if (lane == 0) {
+          mbar_expect_tx(full, kTileB);
+          tma_load_2d(su32(As + s * kTileB), &tk, 0, static_cast<int>(kbase + static_cast<int64_t>(t) * kKeys), full);
+        }
+        *reinterpret_cast<uint4*>(SFs + s * kKeys + 4 * lane) = make_uint4(sfw[u][0], sfw[u][1], sfw[u][2], sfw[u][3]);
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // the tensor core reads them
+        mbar_arrive(full);
+        if (it + 4 < n_tiles) sf_load(it + 4, sfw[u]);
       }
-      *reinterpret_cast<uint4*>(SFs + s * kKeys + 4 * lane) = make_uint4(sfw[0], sfw[1], sfw[2], sfw[3]);
-      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // the tensor core reads them
-      mbar_arrive(full);
-      if (it + 1 < n_tiles) sf_load(it + 1, sfw);
     }
   } else if (warp == 1) {
     // ================= MMA issue (one lane) =================
@@ -427,7 +442,7 @@ cudaError_t launch_index_tc(const lc_index_args& a, bool decode, cudaStream_t st
   const size_t cap = 227 * 1024 / per_sm - 2048;
   if (sm < cap) sm = cap;
   cudaFuncSetAttribute(k_index_tc<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
-  k_index_tc<1><<<grid, kThreads, sm, st>>>(tk, a, tpc, cols);
+  k_index_tc<1><<<grid, kThreads, sm, st>>>(tk, a, tpc, cols, decode ? 1 : 0);
   return cudaGetLastError();
 }
 

@@ -33,7 +33,7 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_cache) {
+__global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_cache, int decode) {
   extern __shared__ uint32_t cache[];  // [kRowCache] keys of this CTA's segment
   __shared__ int hist[2][kBins];
   __shared__ int s_wsum[kTopkWarps];
@@ -49,8 +49,9 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
   const int rank = static_cast<int>(cl.block_rank());
   const int q = blockIdx.x / C;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b = seq_of_query(a.batch.q_start, a.batch.num_seqs, q);
-  const int p = __ldg(a.batch.q_pos0 + b) + (q - __ldg(a.batch.q_start + b));
+  // decode: one query per sequence (q_start[b] = b), no search
+  const int b = decode ? q : seq_of_query(a.batch.q_start, a.batch.num_seqs, q);
+  const int p = __ldg(a.batch.q_pos0 + b) + (decode ? 0 : q - __ldg(a.batch.q_start + b));
   const int n = n_visible(p, a.m, a.W_x, __ldg(a.batch.n_ent + b));
   const int K = min(a.k, n);
   int32_t* out = a.idx + static_cast<int64_t>(q) * a.k;
@@ -319,7 +320,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
   }
 }
 
-cudaError_t launch_topk(const lc_topk_args& a, bool /*decode*/, cudaStream_t st) {
+cudaError_t launch_topk(const lc_topk_args& a, bool decode, cudaStream_t st) {
   if (a.n_q == 0) return cudaSuccess;
   // the largest cluster that keeps the rows within one wave (one 1024-thread CTA per SM),
   // and at least the one whose segments fit the key cache
@@ -345,7 +346,7 @@ cudaError_t launch_topk(const lc_topk_args& a, bool /*decode*/, cudaStream_t st)
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_topk, a, use_cache);
+  return cudaLaunchKernelEx(&cfg, k_topk, a, use_cache, decode ? 1 : 0);
 }
 
 }  // namespace lc
