@@ -27,6 +27,7 @@ constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kRowCache = 48 * 1024;  // keys held in shared memory per CTA (192 KB)
 constexpr int kBins = 2048;
 constexpr int kMaxCluster = 8;
+constexpr int kCand = kBins;          // candidates gathered after the first pass, at most
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f);
@@ -43,6 +44,11 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
   __shared__ int s_gt[kTopkWarps], s_eq[kTopkWarps];
   __shared__ uint32_t s_wmin[kTopkWarps], s_wmax[kTopkWarps];
   __shared__ uint32_t s_range[2];  // this CTA's smallest and largest key
+  __shared__ int hist2[kBins];     // histograms of the gathered candidates
+  __shared__ int s_bin_total;      // keys of the whole row in the bin just selected
+  __shared__ int s_ncand;          // this CTA's keys in the first selected bin
+  __shared__ int s_red[kTopkWarps][kMaxCluster];
+  __shared__ int s_above[kMaxCluster], s_gtr[kMaxCluster], s_eqr[kMaxCluster];
 
   cg::cluster_group cl = cg::this_cluster();
   const int C = static_cast<int>(cl.num_blocks());
@@ -145,6 +151,58 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
     umax = max(umax, rr[1]);
   }
 
+  // Descending prefix over 2048 bins held two per thread (thread t: bins 2047 - 2t and
+  // 2046 - 2t, counts c0 and c1): the bin holding the rem-th largest candidate becomes the
+  // next w bits of the prefix; s_prefix / s_remaining / s_bin_total carry the result.
+  auto pick_bin = [&](int c0, int c1, int w, uint32_t pf, int rem) {
+    const int sm = c0 + c1;
+    int incl = sm;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int wv = s_wsum[lane], wi = wv;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += v;
+      }
+      s_wsum[lane] = wi - wv;  // exclusive over the warps
+    }
+    __syncthreads();
+    const int excl = s_wsum[warp] + incl - sm;
+    if (excl < rem && excl + sm >= rem) {
+      const bool hi = excl + c0 >= rem;
+      const uint32_t bin = static_cast<uint32_t>(hi ? kBins - 1 - 2 * tid : kBins - 2 - 2 * tid);
+      s_prefix = (pf << w) | bin;
+      s_remaining = hi ? rem - excl : rem - excl - c0;
+      s_bin_total = hi ? c0 : c1;
+    }
+    __syncthreads();
+  };
+  // sums over the CTA of up to kMaxCluster per-thread counters (result in out[0 .. C))
+  auto block_sum = [&](const int (&v)[kMaxCluster], int* out) {
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      if (r >= C) break;
+      int x = v[r];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+      if (lane == 0) s_red[warp][r] = x;
+    }
+    __syncthreads();
+    if (tid < C) {
+      int t = 0;
+      for (int w2 = 0; w2 < kTopkWarps; ++w2) t += s_red[w2][tid];
+      out[tid] = t;
+    }
+    __syncthreads();
+  };
+
   // Radix passes over rel = key - umin, < 2^L with L = bit length of the row's key range,
   // 11 bits at a time from the top: the first pass spreads the row over the whole
   // histogram whatever its range, and a row whose keys are all equal needs no pass.
@@ -154,6 +212,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
   int remaining = K;
   int shift = 32 - __clz(static_cast<int>(umax - umin));
   int pass = 0;
+  bool fast = false;  // the candidate path below took over after the first pass
 #pragma unroll 1
   while (shift > 0) {
     const int w = min(11, shift);
@@ -192,37 +251,94 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
       c0 += v0[r];
       c1 += v1[r];
     }
-    // exclusive prefix over the threads (= over the bins from the top)
-    const int sm = c0 + c1;
-    int incl = sm;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    if (lane == 31) s_wsum[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      int wv = s_wsum[lane], wi = wv;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, wi, o);
-        if (lane >= o) wi += v;
-      }
-      s_wsum[lane] = wi - wv;  // exclusive over the warps
-    }
-    __syncthreads();
-    const int excl = s_wsum[warp] + incl - sm;
-    if (excl < remaining && excl + sm >= remaining) {
-      const bool hi = excl + c0 >= remaining;
-      const uint32_t bin = static_cast<uint32_t>(hi ? kBins - 1 - 2 * tid : kBins - 2 - 2 * tid);
-      s_prefix = (pfx << w) | bin;
-      s_remaining = hi ? remaining - excl : remaining - excl - c0;
-    }
-    __syncthreads();
+    pick_bin(c0, c1, w, pfx, remaining);
+    const uint32_t sel = s_prefix & bmask;
     pfx = s_prefix;
     remaining = s_remaining;
     ++pass;
+    if (pass == 1 && shift > 0 && s_bin_total <= kCand) {
+      // Few keys share the selected bin: every CTA gathers them and finishes the
+      // selection alone, with no further cluster-wide histograms.  What each rank holds
+      // above the bin comes from this pass's histograms.
+      int ab[kMaxCluster];
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r)
+        ab[r] = (static_cast<uint32_t>(kBins - 1 - 2 * tid) > sel ? v0[r] : 0) +
+                (static_cast<uint32_t>(kBins - 2 - 2 * tid) > sel ? v1[r] : 0);
+      block_sum(ab, s_above);
+      fast = true;
+      break;
+    }
+  }
+
+  if (fast) {
+    // this CTA's keys in the selected bin -> hist[1] (the other ranks read it)
+    int* cand = hist[1];
+    if (tid == 0) s_ncand = 0;
+    __syncthreads();
+    for (int i4 = tid; i4 < n4; i4 += kTopkThreads) {
+      const uint4 v = key4(i4);
+      const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t rel = kk[j] - umin;
+        if (4 * i4 + j < ns && (rel >> shift) == pfx) cand[atomicAdd(&s_ncand, 1)] = static_cast<int>(kk[j]);
+      }
+    }
+    cl.sync();  // every rank's candidates are written; every rank has read the histograms
+    // all ranks' candidates, in rank order, into hist[0]
+    int* allc = hist[0];
+    int cnt[kMaxCluster], off[kMaxCluster];
+    int n_all = 0;
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      cnt[r] = r < C ? *cl.map_shared_rank(&s_ncand, r) : 0;
+      off[r] = n_all;
+      n_all += cnt[r];
+    }
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      if (r >= C) break;
+      const int* rc = cl.map_shared_rank(cand, r);
+      for (int i = tid; i < cnt[r]; i += kTopkThreads) allc[off[r] + i] = rc[i];
+    }
+    // no more reads of other ranks' shared memory; the matching wait comes before exit,
+    // so no rank leaves while another still reads its candidates
+    asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+    __syncthreads();
+    // the remaining-th largest candidate: radix passes over the bits below the prefix
+    while (shift > 0) {
+      const int w = min(11, shift);
+      const int hi_shift = shift;
+      shift -= w;
+      const uint32_t bmask = (1u << w) - 1u;
+      for (int i = tid; i < kBins; i += kTopkThreads) hist2[i] = 0;
+      __syncthreads();
+      for (int i = tid; i < n_all; i += kTopkThreads) {
+        const uint32_t rel = static_cast<uint32_t>(allc[i]) - umin;
+        if ((rel >> hi_shift) == pfx) atomicAdd(&hist2[(rel >> shift) & bmask], 1);
+      }
+      __syncthreads();
+      pick_bin(hist2[kBins - 1 - 2 * tid], hist2[kBins - 2 - 2 * tid], w, pfx, remaining);
+      pfx = s_prefix;
+      remaining = s_remaining;
+    }
+    // every rank's keys > T and == T: those above the first bin plus its candidates
+    const uint32_t Tc = umin + pfx;
+    int gtc[kMaxCluster], eqc[kMaxCluster];
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) gtc[r] = eqc[r] = 0;
+    for (int i = tid; i < n_all; i += kTopkThreads) {
+      const uint32_t k0 = static_cast<uint32_t>(allc[i]);
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r) {
+        const bool in = i >= off[r] && i < off[r] + cnt[r];
+        gtc[r] += in && k0 > Tc;
+        eqc[r] += in && k0 == Tc;
+      }
+    }
+    block_sum(gtc, s_gtr);
+    block_sum(eqc, s_eqr);
   }
   const uint32_t T = umin + pfx;
   const int need = remaining;
@@ -252,27 +368,35 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
     s_eq[warp] = eq_c;
   }
   __syncthreads();
-  if (tid == 0) {
-    int g = 0, e = 0;
-    for (int w = 0; w < kTopkWarps; ++w) {
-      g += s_gt[w];
-      e += s_eq[w];
-    }
-    s_cnt[0] = g;
-    s_cnt[1] = e;
-  }
-  cl.sync();  // every CTA's counts are published
   int eq_rank = 0, pos = 0;
-  for (int r = 0; r < rank; ++r) {
-    const int* cr = cl.map_shared_rank(s_cnt, r);
-    pos += cr[0] + min(max(need - eq_rank, 0), cr[1]);
-    eq_rank += cr[1];
+  if (fast) {
+    for (int r = 0; r < rank; ++r) {
+      const int gr = s_above[r] + s_gtr[r];
+      pos += gr + min(max(need - eq_rank, 0), s_eqr[r]);
+      eq_rank += s_eqr[r];
+    }
+  } else {
+    if (tid == 0) {
+      int g = 0, e = 0;
+      for (int w = 0; w < kTopkWarps; ++w) {
+        g += s_gt[w];
+        e += s_eq[w];
+      }
+      s_cnt[0] = g;
+      s_cnt[1] = e;
+    }
+    cl.sync();  // every CTA's counts are published
+    for (int r = 0; r < rank; ++r) {
+      const int* cr = cl.map_shared_rank(s_cnt, r);
+      pos += cr[0] + min(max(need - eq_rank, 0), cr[1]);
+      eq_rank += cr[1];
+    }
   }
   for (int w = 0; w < warp; ++w) {
     pos += s_gt[w] + min(max(need - eq_rank, 0), s_eq[w]);
     eq_rank += s_eq[w];
   }
-  cl.sync();  // no CTA leaves while another still reads its counts
+  if (!fast) cl.sync();  // no CTA leaves while another still reads its counts
   // 128 keys per step, 4 consecutive ones per lane: ties are ranked in index order within
   // the lane, then across the lanes (exclusive warp scans), then across the steps
   for (int base4 = lo4; base4 < hi4; base4 += 32) {
@@ -318,6 +442,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
     eq_rank += eq_all;
     pos += sel_all;
   }
+  if (fast) asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
 
 cudaError_t launch_topk(const lc_topk_args& a, bool decode, cudaStream_t st) {
