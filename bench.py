@@ -302,6 +302,9 @@ def run_lc(args):
             work[f"{i}:{k}"] = v
         units += u if i == 0 else 0  # a mixed step counts each sequence's token once
     stage_names = [f"{i}:{n}" for i, (_, _, r) in enumerate(runs) for n, _ in r.stages()]
+    # the critical path: stages on the main stream (the side stages overlap them, and their
+    # event times include the wait for SMs the critical path holds)
+    crit_names = [f"{i}:{n}" for i, (_, _, r) in enumerate(runs) for part in r.dag()[1:] for n, _ in part]
     # kernels per step: one per call, plus the combine kernel of a key-split attention
     n_launch = len(stage_names) + sum(1 for (_, _, r) in runs if r.a_attn.workspace_bytes > 0)
     # one stream per side stage: they share no buffers, so none waits for another
@@ -329,8 +332,9 @@ def run_lc(args):
     torch.cuda.synchronize()
     for _, _, r in runs:
         assert r.read_status() == 0, "device status bits set"
-    graph = None       # the timed step: a CUDA graph with only the dominant stage bracketed
-    graph_all = None   # the same step with every stage bracketed, for the per-stage breakdown
+    graph = None       # the timed step: a CUDA graph of the step, no event nodes
+    graph_dom = None   # the same step with the dominant stage bracketed (its kernel time)
+    graph_all = None   # the same step with every stage bracketed (per-stage breakdown)
     dom_key = None
     rl = [r for _, _, r in runs]
     if not args.no_graph:
@@ -349,9 +353,10 @@ def run_lc(args):
             torch.cuda.synchronize()
             for n in stage_names:
                 warm[n].append(g_ev[n][0].elapsed_time(g_ev[n][1]))
-        # every event node costs the step about a microsecond, so the timed graph brackets
-        # only the stage whose kernel the roofline reports
-        dom_key = max(stage_names, key=lambda n: statistics.mean(warm[n]))
+        # an event node on the critical path lengthens the step by microseconds, so the
+        # headline graph has none; the roofline's kernel time comes from a graph that
+        # brackets only that stage, timed in a pass of its own
+        dom_key = max(crit_names, key=lambda n: statistics.mean(warm[n]))
         d_ev = ext_pair()
 
         def timed_dom(i, name, st, fn):
@@ -361,8 +366,11 @@ def run_lc(args):
             d_ev[0].record(st)
             fn(st)
             d_ev[1].record(st)
-        graph = capture_step(rl, stream, side, timed_dom)
+        graph_dom = capture_step(rl, stream, side, timed_dom)
+        graph = capture_step(rl, stream, side, None)
         for _ in range(args.warmup):
+            flush_l2()
+            graph_dom.replay()
             flush_l2()
             graph.replay()
         torch.cuda.synchronize()
@@ -387,16 +395,20 @@ def run_lc(args):
             else:
                 graph.replay()
             ev_step[s][1].record(stream)
-            if graph is not None:
-                # the graph's events are re-recorded by every replay: read them now
-                ev_step[s][1].synchronize()
-                dom_ms.append(d_ev[0].elapsed_time(d_ev[1]))
         torch.cuda.synchronize()
     barrier()
+    if graph_dom is not None:
+        # the dominant kernel's time: the same steps again, that stage bracketed (the
+        # graph's events are re-recorded by every replay: read them after each)
+        for s in range(args.steps):
+            flush_l2()
+            graph_dom.replay()
+            torch.cuda.synchronize()
+            dom_ms.append(d_ev[0].elapsed_time(d_ev[1]))
     if graph is None:
         per_stage = {n: [ev[s][n][0].elapsed_time(ev[s][n][1]) for s in range(args.steps)] for n in stage_names}
     else:
-        # per-stage breakdown: a second timed pass of the graph with every stage bracketed
+        # per-stage breakdown: a third timed pass, the graph with every stage bracketed
         per_stage = {n: [] for n in stage_names}
         for s in range(args.steps):
             flush_l2()
@@ -448,7 +460,7 @@ def run_lc(args):
     # roofline of the dominant kernel (largest share of the step); its duration comes from
     # the headline pass when that pass bracketed it
     avg = {n: statistics.mean(v) for n, v in per_stage.items()}
-    dom = max(avg, key=avg.get)
+    dom = max(crit_names, key=lambda n: avg[n])
     dom_t = statistics.mean(dom_ms) if dom == dom_key and dom_ms else avg[dom]
     spec0 = runs[int(dom.split(":")[0])][0]
     bnd, _ = bound_of(dom, spec0, work, pk)
@@ -483,7 +495,9 @@ def run_lc(args):
                          "256 MiB read so that evicted lines are clean)",
                    "launch": "eager" if graph is None else "cuda graph of the step",
                    "stage_times": "eager steps" if graph is None else
-                   "second timed pass, every stage bracketed by graph event nodes",
+                   "third timed pass, every stage bracketed by graph event nodes",
+                   "kernel_time": "eager steps" if graph is None else
+                   "second timed pass, the dominant stage bracketed by graph event nodes",
                    "parallelism": f"replicas x{world} (independent batches)"},
         "roofline": {"bound": bnd, "kernel": dom.split(":")[1], "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic, "peak_source": pk_kind,

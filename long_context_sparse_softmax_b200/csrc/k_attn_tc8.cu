@@ -15,9 +15,11 @@
 //     (E4M3 -> F16 exact; BF16 -> F16 exact in [2^-14, 65504], else LC_DEV_RANGE) into a
 //     core-matrix tile, the MN-major A operand of O^T = V^T P^T (M = 128 dims, a last chunk
 //     of 64, N = 64 heads), while the scores of the next tile run;
-//   * the window rows are BF16, so the last (window) tiles run in F16: the raw stages, free
-//     by then, hold Q converted to F16, the window tile is copied into the V tile and
-//     serves both S = Q K^T and O^T = V^T P^T.
+//   * window tiles come first: their rows are consecutive, so each arrives by nine 2-D bulk
+//     tensor copies into the V tile area while the raw stages hold Q converted to BF16;
+//     S = Q K^T reads the landed BF16 tile (exact products in FP32), then the tile is
+//     widened to F16 in place for O^T = V^T P^T, and the entry gathers begin once every
+//     window S is done.
 // Softmax, the per-head exponent reference, the sink and the outputs are those of
 // k_attn_tc.cu (P in F16, 11 significant bits; row sums of the rounded P).
 //
@@ -58,13 +60,13 @@ constexpr uint32_t kTmemCols = 512;
 // shared memory (dynamic, 1024-byte aligned)
 constexpr int kOffQn = 0;                         // Q nope, E4M3, 4 SW128 blocks
 constexpr int kOffQr = kOffQn + kRawN;            // Q RoPE, BF16, SW128
-constexpr int kOffRaw = kOffQr + kBlk;            // 2 raw stages (window phase: Q in F16)
+constexpr int kOffRaw = kOffQr + kBlk;            // 2 raw stages (window phase: Q in BF16)
 constexpr int kOffV = kOffRaw + 2 * kRawStage;    // F16 core-matrix tile
 constexpr int kOffP = kOffV + kTile;
 constexpr int kOffCode = kOffP + kPBytes;         // [4][kTK] key codes
 constexpr int kOffF = kOffCode + 4 * kTK * 4;     // [kNR] per-head factors
 constexpr size_t kSmem = kOffF + kNR * 4 + 1024;  // + alignment slack
-static_assert(2 * kRawStage >= kTile, "Q in F16 fits the raw stages");
+static_assert(2 * kRawStage >= kTile, "Q in BF16 fits the raw stages");
 
 __device__ __forceinline__ uint32_t su32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
@@ -214,6 +216,23 @@ __device__ __forceinline__ void e4m3x16_f16(uint4 v, uint4& lo, uint4& hi) {
   lo = make_uint4(o[0], o[1], o[2], o[3]);
   hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
+// 16 E4M3 values -> 16 BF16 values (exact: an E4M3 value has at most 4 significant bits,
+// so the upper half of its FP32 bits is its BF16 encoding)
+__device__ __forceinline__ void e4m3x16_bf16(uint4 v, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[j] & 0xffffu), __NV_E4M3);
+    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[j] >> 16), __NV_E4M3);
+    const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&a));
+    const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&b));
+    o[2 * j] = (__float_as_uint(fa.x) >> 16) | (__float_as_uint(fa.y) & 0xffff0000u);
+    o[2 * j + 1] = (__float_as_uint(fb.x) >> 16) | (__float_as_uint(fb.y) & 0xffff0000u);
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
 // 8 BF16 values -> 8 F16 values; |value| accumulated (as F16) into `amax`
 __device__ __forceinline__ uint4 bf16x8_f16(uint4 v, __half2& amax) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -249,9 +268,11 @@ struct Bars {
   uint64_t cready[4];  // key codes of a tile written (one arrival per copy warp)
   uint64_t cfree[4];   // key codes of a tile read by the softmax (128 arrivals)
   uint64_t wfull;      // window tile landed in the F16 tile area (expect-tx)
+  uint64_t wsdone;     // S of a window tile complete: the tile may be widened in place (commit)
   uint64_t vfull;      // F16 tile ready (1 arrival)
   uint64_t vempty;     // F16 tile read by O (commit)
-  uint64_t q16full;    // Q in F16 ready for the window tiles (1 arrival)
+  uint64_t q16full;    // Q in BF16 ready for the window tiles (1 arrival)
+  uint64_t q16free;    // every S that reads Q in BF16 is complete: the raw stages are free (commit)
   uint64_t sfull[2];   // S buffer computed (commit)
   uint64_t sempty[2];  // S buffer read (128 arrivals)
   uint64_t pfull;      // P written (128 arrivals)
@@ -284,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* Ps = smem + kOffP;
   int* kcode = reinterpret_cast<int*>(smem + kOffCode);
   float* s_f = reinterpret_cast<float*>(smem + kOffF);
-  uint8_t* Q16 = Raw;  // window phase
+  uint8_t* Q16 = Raw;  // window phase: Q in BF16, core matrices
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ __align__(8) Bars bars;
@@ -339,8 +360,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     return false;
   };
   // first slot of tile t
-  auto tile_slot0 = [&](int t) { return t < n_et ? s_begin + t * kTK : w_begin + (t - n_et) * kTK; };
-  auto tile_slot_end = [&](int t) { return t < n_et ? e_end : s_end; };
+  // window tiles come first (their rows are on hand while the entry gathers start): tile t
+  // is window tile t for t < n_wt, entry tile t - n_wt after that
+  auto tile_slot0 = [&](int t) { return t < n_wt ? w_begin + t * kTK : s_begin + (t - n_wt) * kTK; };
+  auto tile_slot_end = [&](int t) { return t < n_wt ? s_end : e_end; };
   // key slot -> entry index j, kWin | window row, or -1 (masked)
   auto slot_code = [&](int s, int s_lim) -> int {
     if (s >= s_lim) return -1;
@@ -385,9 +408,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(su32(&bars.cfree[i]), 128);
     }
     mbar_init(su32(&bars.wfull), 1);
+    mbar_init(su32(&bars.wsdone), 1);
     mbar_init(su32(&bars.vfull), 1);
     mbar_init(su32(&bars.vempty), 1);
     mbar_init(su32(&bars.q16full), 1);
+    mbar_init(su32(&bars.q16free), 1);
     mbar_init(su32(&bars.pfull), 128);
     mbar_init(su32(&bars.pempty), 1);
     mbar_init(su32(&bars.fin), 1);
@@ -415,16 +440,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int cb4 = t & 3;
       // the code buffer of tile t - 4 has been read by its softmax
       bool ok = t < 4 || wait(&bars.cfree[cb4], ((t >> 2) - 1) & 1);
-      // raw stage of entry tile t: free once S and the conversion of tile t - 2 are done
-      if (ok && t < n_et && t >= 2) ok = wait(&bars.kempty[t & 1], ((t >> 1) - 1) & 1);
+      // raw stage of entry tile e: free once S and the conversion of entry tile e - 2 are
+      // done; before the first two entry tiles it holds Q in BF16 for the window tiles
+      const int e = t - n_wt;
+      if (ok && e >= 2) ok = wait(&bars.kempty[e & 1], ((e >> 1) - 1) & 1);
+      if (ok && e >= 0 && e < 2 && n_wt > 0) ok = wait(&bars.q16free, 0);
       if (!__all_sync(0xffffffffu, ok)) break;
       const int s0 = tile_slot0(t), s_lim = tile_slot_end(t);
       int* kc = kcode + cb4 * kTK + 16 * cw;
       if (lane < 16) kc[lane] = slot_code(s0 + 16 * cw + lane, s_lim);
       __syncwarp();
       if (lane == 0) mbar_arrive(su32(&bars.cready[cb4]));
-      if (t < n_et) {
-        const int st = t & 1;
+      if (e >= 0) {
+        const int st = e & 1;
         const uint32_t kb = su32(&bars.kfull[st]);
         if (lane == 0) mbar_expect_tx(kb, kRawStage / kCopyWarps);
         __syncwarp();
@@ -452,8 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // S entry: M = 64, N = 64, K-major SW128, E4M3 (kind::f8f6f4) and BF16 (kind::f16)
       const uint32_t id_s8 = (1u << 4) | (static_cast<uint32_t>(kTK >> 3) << 17) | (static_cast<uint32_t>(kNR >> 4) << 24);
       const uint32_t id_sbf = id_s8 | (1u << 7) | (1u << 10);
-      // S window: F16 core-matrix operands; O^T: M = 128 (or 64), N = 64, A MN-major, F16
-      const uint32_t id_sf16 = id_s8;
+      // S window: BF16 (id_sbf); O^T: M = 128 (or 64), N = 64, A MN-major, F16
       const uint32_t id_o128 = (1u << 4) | (1u << 15) | (static_cast<uint32_t>(kNR >> 3) << 17) |
                                (static_cast<uint32_t>(128 >> 4) << 24);
       const uint32_t id_o64 = (1u << 4) | (1u << 15) | (static_cast<uint32_t>(kNR >> 3) << 17) |
@@ -468,13 +495,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ns < n_tiles && ns <= no + 1) {
           const int sb = ns & 1;
           bool ready = ns < 2 || mbar_probe(su32(&bars.sempty[sb]), ((ns >> 1) - 1) & 1);
-          if (ns < n_et) ready = ready && mbar_probe(su32(&bars.kfull[ns & 1]), (ns >> 1) & 1);
-          else ready = ready && mbar_probe(su32(&bars.q16full), 0) && mbar_probe(su32(&bars.vfull), ns & 1);
+          const int e = ns - n_wt;
+          if (e >= 0) ready = ready && mbar_probe(su32(&bars.kfull[e & 1]), (e >> 1) & 1);
+          else ready = ready && mbar_probe(su32(&bars.q16full), 0) && mbar_probe(su32(&bars.wfull), ns & 1);
           if (ready) {
             fence_after();
             const uint32_t d = tm + kColS + sb * kTK;
-            if (ns < n_et) {
-              const uint32_t st = su32(Raw + (ns & 1) * kRawStage);
+            if (e >= 0) {
+              const uint32_t st = su32(Raw + (e & 1) * kRawStage);
 #pragma unroll
               for (int cb = 0; cb < 4; ++cb)
 #pragma unroll
@@ -484,13 +512,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int k = 0; k < 4; ++k)
                 mma<0>(d, sw128_desc(su32(Qr) + k * 32), sw128_desc(st + kRawN + k * 32), id_sbf, 1);
-              mma_commit(su32(&bars.kempty[ns & 1]));
+              mma_commit(su32(&bars.kempty[e & 1]));
             } else {
-              // A: Q in F16 (core matrices); B: the window tile, SW128, 64 dims per block
+              // A: Q in BF16 (core matrices); B: the window tile as it landed, BF16, SW128, 64
+              // dims per block (each product is exact in FP32, as with F16 operands); the
+              // tile is widened to F16 for O only after this S is complete
               const uint64_t dq = cm_desc(su32(Q16), 128, kG);
 #pragma unroll
               for (int k = 0; k < kD / 16; ++k)
-                mma<0>(d, dq + k * 16, sw128_desc(su32(Vt) + (k >> 2) * kBlk + (k & 3) * 32), id_sf16, k > 0);
+                mma<0>(d, dq + k * 16, sw128_desc(su32(Vt) + (k >> 2) * kBlk + (k & 3) * 32), id_sbf, k > 0);
+              mma_commit(su32(&bars.wsdone));
+              if (ns == n_wt - 1) mma_commit(su32(&bars.q16free));
             }
             mma_commit(su32(&bars.sfull[sb]));
             ++ns;
@@ -499,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (no < ns && mbar_probe(su32(&bars.pfull), no & 1) && mbar_probe(su32(&bars.vfull), no & 1)) {
           fence_after();
-          if (no < n_et) {
+          if (no >= n_wt) {
 #pragma unroll
             for (int kk = 0; kk < kTK / 16; ++kk)
 #pragma unroll
@@ -544,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __half2 amax = __float2half2_rn(0.f);
     bool ok = true;
     for (int t = 0; ok && t < n_tiles; ++t) {
-      if (t >= n_et) {
+      if (t < n_wt) {
         // window tile: its rows are consecutive, so it comes as one 64 x 64 BF16 box per 64
         // dims (SW128) straight into the F16 tile area, once O of tile t - 1 is done (these
         // warps wait for every phase of vempty in order; rows past the window are masked by
@@ -562,12 +594,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int cb = 0; cb < kD / 64; ++cb) tma_tile2d(su32(Vt + cb * kBlk), &twin, cb * 64, y, wb);
         }
       }
-      if (t == n_et) {
-        // window phase: Q to F16 in the raw stages, once S and the conversion of every
-        // entry tile are done (the raw stages are free)
-        bool okq = wait(&bars.qfull, 0);
-        if (okq && n_et >= 1) okq = wait(&bars.kempty[(n_et - 1) & 1], ((n_et - 1) >> 1) & 1);
-        if (okq && n_et >= 2) okq = wait(&bars.kempty[(n_et - 2) & 1], ((n_et - 2) >> 1) & 1);
+      if (t == 0 && n_wt > 0) {
+        // Q to F16 in the raw stages for the window tiles (the entry gathers wait for
+        // q16free before they use the raw stages)
+        const bool okq = wait(&bars.qfull, 0);
         if (named_bar_or(2, 128, !okq)) {
           ok = false;
           break;
@@ -578,15 +608,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (pc < 32) {  // 16 E4M3 dims: block pc / 8, 16-byte chunk pc % 8 of row r
             const uint4 v = *reinterpret_cast<const uint4*>(Qn + (pc >> 3) * kBlk + sw128_off(r, pc & 7));
             uint4 lo, hi;
-            e4m3x16_f16(v, lo, hi);
+            e4m3x16_bf16(v, lo, hi);
             *reinterpret_cast<uint4*>(Q16 + tile_off(r, 2 * pc)) = lo;
             *reinterpret_cast<uint4*>(Q16 + tile_off(r, 2 * pc + 1)) = hi;
-          } else {  // 16 RoPE dims: chunks 2 (pc - 32), +1 of the SW128 row
+          } else {  // 16 RoPE dims (already BF16): chunks 2 (pc - 32), +1 of the SW128 row
             const int j = 2 * (pc - 32);
-            const uint4 v0 = *reinterpret_cast<const uint4*>(Qr + sw128_off(r, j));
-            const uint4 v1 = *reinterpret_cast<const uint4*>(Qr + sw128_off(r, j + 1));
-            *reinterpret_cast<uint4*>(Q16 + tile_off(r, 64 + j)) = bf16x8_f16(v0, amax);
-            *reinterpret_cast<uint4*>(Q16 + tile_off(r, 64 + j + 1)) = bf16x8_f16(v1, amax);
+            *reinterpret_cast<uint4*>(Q16 + tile_off(r, 64 + j)) = *reinterpret_cast<const uint4*>(Qr + sw128_off(r, j));
+            *reinterpret_cast<uint4*>(Q16 + tile_off(r, 64 + j + 1)) =
+                *reinterpret_cast<const uint4*>(Qr + sw128_off(r, j + 1));
           }
         }
         fence_async_smem();
@@ -596,14 +625,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the F16 tile is free once O of the previous tile is done; this tile's codes or
       // raw rows have landed
       bool okw = t == 0 || wait(&bars.vempty, (t - 1) & 1);
-      if (t < n_et) okw = okw && wait(&bars.kfull[t & 1], (t >> 1) & 1);
-      else okw = okw && wait(&bars.cready[t & 3], (t >> 2) & 1) && wait(&bars.wfull, (t - n_et) & 1);
+      const int e = t - n_wt;
+      if (e >= 0) okw = okw && wait(&bars.kfull[e & 1], (e >> 1) & 1);
+      else  // the window tile is widened in place once its S has read it
+        okw = okw && wait(&bars.cready[t & 3], (t >> 2) & 1) && wait(&bars.wsdone, t & 1);
       if (named_bar_or(2, 128, !okw)) {
         ok = false;
         break;
       }
-      if (t < n_et) {
-        const uint8_t* st = Raw + (t & 1) * kRawStage;
+      if (e >= 0) {
+        const uint8_t* st = Raw + (e & 1) * kRawStage;
         // 64 keys x 32 E4M3 pieces of 16 dims, then 64 keys x 8 BF16 chunks; a quarter warp
         // takes 8 rows of one piece (its SW128 reads and its core-matrix writes hit
         // distinct banks); the loads of four pieces are issued before any is converted
@@ -659,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar(2, 128);
       if (ct == 0) {
         mbar_arrive(su32(&bars.vfull));
-        if (t < n_et) mbar_arrive(su32(&bars.kempty[t & 1]));
+        if (e >= 0) mbar_arrive(su32(&bars.kempty[e & 1]));
       }
     }
     if (f16_inf(amax)) set_status(a.status, LC_DEV_RANGE);
