@@ -142,11 +142,30 @@ def stage_work(spec, inp, run):
     return work, units
 
 
-def bound_of(stage, spec, work, pk):
+# Dense tensor-core rates relative to BF16 (the nominal ratios; a tcgen05 probe that ran
+# M128 x N128 MMAs on every SM measured 2221, 4448 and 8899 TFLOP/s for BF16, E4M3 and
+# MXFP4, the same 1 : 2 : 4)
+TENSOR_RATIO = {"bf16": 1.0, "e4m3": 2.0, "mxf4": 4.0}
+
+
+def tensor_mix(stage, spec, attn_impl="auto"):
+    """(peak factor over the BF16 peak, label) for a tensor-bound stage: the indexer runs
+    MXFP4 MMAs; the E4M3-score attention kernel does half its flops (S) in E4M3 and half
+    (P V) in F16."""
+    from long_context_sparse_softmax_b200 import workloads as wl
+    if stage.endswith("index") and spec.idx_fmt == wl.IDX_MXFP4:
+        return TENSOR_RATIO["mxf4"], "MXFP4"
+    if (stage.endswith("attn") and attn_impl in ("auto", "tc") and spec.q_fmt == wl.FMT_E4M3_BF16
+            and spec.kv_fmt == wl.FMT_E4M3_BF16):
+        return 1.0 / (0.5 / TENSOR_RATIO["e4m3"] + 0.5 / TENSOR_RATIO["bf16"]), "E4M3 S + F16 PV"
+    return 1.0, "BF16/F16"
+
+
+def bound_of(stage, spec, work, pk, attn_impl="auto"):
     """HBM- or tensor-bound by comparing the two roofline times."""
     b, f = work[stage]
     t_mem = b / (pk["hbm_gbs"] * 1e9)
-    t_math = f / (pk["bf16_tflops"] * 1e12) if f else 0.0
+    t_math = f / (pk["bf16_tflops"] * tensor_mix(stage, spec, attn_impl)[0] * 1e12) if f else 0.0
     return ("tensor", t_math) if t_math > t_mem else ("hbm", t_mem)
 
 
@@ -463,19 +482,21 @@ def run_lc(args):
     dom = max(crit_names, key=lambda n: avg[n])
     dom_t = statistics.mean(dom_ms) if dom == dom_key and dom_ms else avg[dom]
     spec0 = runs[int(dom.split(":")[0])][0]
-    bnd, _ = bound_of(dom, spec0, work, pk)
+    bnd, _ = bound_of(dom, spec0, work, pk, args.attn_impl)
     b, f = work[dom]
     if bnd == "hbm":
         achieved = b / (dom_t / 1e3) / 1e9
         peak, unit = pk["hbm_gbs"], "GB/s"
     else:
         achieved = f / (dom_t / 1e3) / 1e12
-        peak, unit = pk["bf16_tflops"], "TFLOP/s"
+        factor, mix = tensor_mix(dom, spec0, args.attn_impl)
+        peak, unit = pk["bf16_tflops"] * factor, "TFLOP/s"
+        pk_kind = f"{pk_kind} bf16 x {factor:.3g} ({mix}; nominal dtype ratio)"
     traffic = kernel_traffic(dom.split(":")[1], args.attn_impl)
     stages = {}
     for n in stage_names:
         bb, ff = work[n]
-        bn, t_roof = bound_of(n, runs[int(n.split(":")[0])][0], work, pk)
+        bn, t_roof = bound_of(n, runs[int(n.split(":")[0])][0], work, pk, args.attn_impl)
         stages[n] = {"ms": round(avg[n], 5), "share": round(avg[n] / sum(avg.values()), 4),
                      "bytes": int(bb), "flops": int(ff), "bound": bn,
                      "roofline_frac": round(t_roof * 1e3 / avg[n], 4) if avg[n] > 0 else None}
