@@ -595,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (t == 0 && n_wt > 0) {
-        // Q to F16 in the raw stages for the window tiles (the entry gathers wait for
+        // Q to BF16 in the raw stages for the window tiles (the entry gathers wait for
         // q16free before they use the raw stages)
         const bool okq = wait(&bars.qfull, 0);
         if (named_bar_or(2, 128, !okq)) {
