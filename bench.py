@@ -264,22 +264,15 @@ def make_runs(name, device, rank, impl=0):
 
 
 def host_io(runs):
-    """Per-step inputs (pinned host copies) and outputs of the e2e leg."""
+    """Per run, the e2e leg's host copies: (h2d, d2h).  h2d maps the stage that first reads
+    a per-step input (the runner's host_inputs) to (device, pinned host) pairs; d2h holds
+    (pinned host, device) pairs of the results."""
     import torch
     io = []
-    for spec, inp, r in runs:
-        names = ["q_raw"]
-        if spec.is_decode:
-            names += ["x_new", "x_tail", "g_tail"]
-        else:
-            names += ["x", "g"]
-        ins = [(inp[n], inp[n].cpu().pin_memory()) for n in names]
-        if spec.is_csa:
-            for t in inp["qI"].values():
-                ins.append((t, t.cpu().pin_memory()))
-        outs = [(r.out, torch.empty(r.out.shape, dtype=r.out.dtype, pin_memory=True)),
-                (r.lse, torch.empty(r.lse.shape, dtype=r.lse.dtype, pin_memory=True))]
-        io.append((ins, outs))
+    for _, _, r in runs:
+        h2d = {st: [(d, d.cpu().pin_memory()) for d in ts] for st, ts in r.host_inputs().items()}
+        d2h = [(torch.empty(d.shape, dtype=d.dtype, pin_memory=True), d) for d in r.host_outputs()]
+        io.append((h2d, d2h))
     return io
 
 
@@ -338,13 +331,14 @@ def run_lc(args):
             e1.record(st)
         return on_stage
 
-    def one_step(stage_ev=None):
+    def one_step(stage_ev=None, io=None):
         """The whole path once: per workload, preparation and compression on the side
         stream next to index -> top-k on the main stream, then attention."""
         hook = None if stage_ev is None else timed(stage_ev)
         for i, (_, _, r) in enumerate(runs):
             r.step_overlapped(stream, side, None if hook is None else
-                              (lambda name, st, fn, i=i: hook(i, name, st, fn)))
+                              (lambda name, st, fn, i=i: hook(i, name, st, fn)),
+                              None if io is None else io[i])
 
     for _ in range(args.warmup):
         one_step()
@@ -448,8 +442,24 @@ def run_lc(args):
     e2e = None
     if not args.no_e2e:
         io = host_io(runs)
-        h2d = sum(h.numel() * h.element_size() for ins, _ in io for _, h in ins)
-        d2h = sum(h.numel() * h.element_size() for _, outs in io for _, h in outs)
+        h2d = sum(h.numel() * h.element_size() for hd, _ in io for pairs in hd.values() for _, h in pairs)
+        d2h = sum(h.numel() * h.element_size() for _, dl in io for h, _ in dl)
+        # each upload on the stream of the stage that first reads it, inside the step's
+        # graph, so that it overlaps the stages before it; the results come back after
+        # attention.  If copies cannot be captured, they run eagerly around the graph.
+        graph_io = None
+        e2e_mode = "eager copies, step launched from Python" if graph is None else "eager copies around the step graph"
+        if graph is not None:
+            try:
+                graph_io = capture_step(rl, stream, side, None, io)
+                for _ in range(args.warmup):
+                    graph_io.replay()
+                torch.cuda.synchronize()
+                e2e_mode = "copies inside the step graph, each on its stage's stream"
+            except Exception as ex:  # noqa: BLE001 - any capture failure falls back
+                graph_io = None
+                print(f"e2e: host copies not capturable ({ex}); timing eager copies", file=sys.stderr)
+                torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         torch.cuda.synchronize()
@@ -457,16 +467,19 @@ def run_lc(args):
         for s in range(args.steps):
             flush_l2()
             e0.record(stream)
-            for ins, _ in io:
-                for d, h in ins:
-                    d.copy_(h, non_blocking=True)
-            if graph is None:
-                one_step()
+            if graph_io is not None:
+                graph_io.replay()
+            elif graph is None:
+                one_step(None, io)
             else:
+                for hd, _ in io:
+                    for pairs in hd.values():
+                        for d, h in pairs:
+                            d.copy_(h, non_blocking=True)
                 graph.replay()
-            for _, outs in io:
-                for d, h in outs:
-                    h.copy_(d, non_blocking=True)
+                for _, dl in io:
+                    for h, d in dl:
+                        h.copy_(d, non_blocking=True)
             e1.record(stream)
             e1.synchronize()
             e_ms += e0.elapsed_time(e1)
@@ -474,7 +487,7 @@ def run_lc(args):
         if world > 1:
             torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e = {"value": world * units * args.steps / (float(t.item()) / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "copies": e2e_mode}
 
     # roofline of the dominant kernel (largest share of the step); its duration comes from
     # the headline pass when that pass bracketed it

@@ -63,15 +63,49 @@ class _Common:
         main = [(n, st[n]) for n in ("index", "topk") if n in st]
         return side, main, [("attn", st["attn"])]
 
-    def step_overlapped(self, main, side, on_stage=None):
+    def host_inputs(self):
+        """The device tensors a step reads that a caller refills from the host each step,
+        by the stage that first reads them: {stage: [tensors]}.  Tensors that stages on
+        different streams share are listed under "_fork" (copied before the fork)."""
+        inp = self.inp
+        qI = list(inp["qI"].values()) if self.spec.is_csa else []
+        if self.spec.is_decode:
+            h = {"qk_prep_q": [inp["q_raw"]], "qk_prep_win": [inp["x_new"]],
+                 "compress": [inp["x_tail"], inp["g_tail"]]}
+        else:
+            h = {"qk_prep_q": [inp["q_raw"]], "_fork": [inp["x"], inp["g"]]}
+        if qI:
+            h["index"] = qI
+        return h
+
+    def host_outputs(self):
+        """The step's results a caller reads back: attention output and lse."""
+        return [self.out, self.lse]
+
+    def step_overlapped(self, main, side, on_stage=None, io=None):
         """One step on several streams: the side stages fork from `main` (stage i on
         side[i % len(side)]; `side` is one stream or a list) and join it before
         attention.  on_stage(name, stream, fn) may wrap each launch (e.g. with timing
-        events)."""
+        events).  io = (h2d, d2h) adds the host copies: h2d maps a stage (or "_fork") to
+        (device, pinned host) pairs copied on that stage's stream just before it, so an
+        upload overlaps the stages before it; d2h holds (pinned host, device) pairs copied
+        on `main` after attention."""
         import torch
         sd, mn, af = self.dag()
         sides = list(side) if isinstance(side, (list, tuple)) else [side]
-        run = on_stage or (lambda name, stream, fn: fn(stream))
+        launch = on_stage or (lambda name, stream, fn: fn(stream))
+        h2d, d2h = io if io is not None else ({}, [])
+
+        def run(name, stream, fn):
+            if h2d.get(name):
+                with torch.cuda.stream(stream):
+                    for d, h in h2d[name]:
+                        d.copy_(h, non_blocking=True)
+            launch(name, stream, fn)
+        if h2d.get("_fork"):
+            with torch.cuda.stream(main):
+                for d, h in h2d["_fork"]:
+                    d.copy_(h, non_blocking=True)
         fork = torch.cuda.Event()
         fork.record(main)
         used = sides[:len(sd)]
@@ -89,6 +123,10 @@ class _Common:
             main.wait_event(join)
         for n, f in af:
             run(n, main, f)
+        if d2h:
+            with torch.cuda.stream(main):
+                for h, d in d2h:
+                    h.copy_(d, non_blocking=True)
 
     def _index_args(self, n_q: int, max_ent: int, scores: torch.Tensor) -> IndexArgs:
         s, inp = self.spec, self.inp
@@ -281,9 +319,10 @@ class Decode(_Common):
             f(stream)
 
 
-def capture_step(runs, main, side, on_stage=None):
+def capture_step(runs, main, side, on_stage=None, io=None):
     """Record one overlapped step of every run in `runs` as a CUDA graph (on_stage, if
-    given, is called as on_stage(run index, stage name, stream, launch)).
+    given, is called as on_stage(run index, stage name, stream, launch); io, if given,
+    holds each run's (h2d, d2h) host copies, see step_overlapped).
 
     The library calls are made once, during capture; `graph.replay()` then launches the
     same kernels with the same arguments on the current stream, with the fork onto `side`
@@ -295,7 +334,8 @@ def capture_step(runs, main, side, on_stage=None):
     with torch.cuda.graph(g, stream=main):
         for i, r in enumerate(runs):
             r.step_overlapped(main, side, None if on_stage is None else
-                              (lambda name, st, fn, i=i: on_stage(i, name, st, fn)))
+                              (lambda name, st, fn, i=i: on_stage(i, name, st, fn)),
+                              None if io is None else io[i])
     return g
 
 
