@@ -57,10 +57,33 @@ def parse():
 
 
 def dist_env():
+    """(rank, world size, local rank) from the launcher's environment (1 process: 0, 1, 0)."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return rank, world, local
+
+
+def rank_spec(spec, rank: int):
+    """The workload a rank runs: the same shapes, its own seed (independent batches, weak
+    scaling)."""
+    import dataclasses
+    return spec if rank == 0 else dataclasses.replace(spec, seed=spec.seed + 1000 * rank)
+
+
+def max_over_ranks(x: float, device, world: int) -> float:
+    """The largest of the ranks' values (the job's time is its slowest rank's)."""
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_throughput(world: int, units_per_step: int, steps: int, total_ms: float) -> float:
+    """Query tokens per second of the whole job: every rank processes its own batch of
+    units_per_step tokens per step, and the job takes total_ms (the slowest rank)."""
+    return world * units_per_step * steps / (total_ms / 1e3)
 
 
 def peaks():
@@ -254,9 +277,7 @@ def make_runs(name, device, rank, impl=0):
     from long_context_sparse_softmax_b200 import workloads as wl
     runs = []
     for spec in wl.WORKLOADS[name]:
-        if rank:
-            import dataclasses
-            spec = dataclasses.replace(spec, seed=spec.seed + 1000 * rank)
+        spec = rank_spec(spec, rank)
         inp = (wl.make_decode if spec.is_decode else wl.make_prefill)(spec, device)
         r = (runner.Decode if spec.is_decode else runner.Prefill)(inp, device, None, impl)
         runs.append((spec, inp, r))
@@ -432,11 +453,8 @@ def run_lc(args):
     # a step's time runs from the fork on the main stream to the end of attention
     span = [ev_step[s][0].elapsed_time(ev_step[s][1]) for s in range(args.steps)]
     total_ms = sum(span)
-    t_max = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t_max, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(t_max.item())
-    value = world * units * args.steps / (total_ms / 1e3)
+    total_ms = max_over_ranks(total_ms, dev, world)
+    value = weak_throughput(world, units, args.steps, total_ms)
 
     # e2e: host inputs in, host outputs back, through the same C-ABI calls
     e2e = None
@@ -483,10 +501,7 @@ def run_lc(args):
             e1.record(stream)
             e1.synchronize()
             e_ms += e0.elapsed_time(e1)
-        t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e = {"value": world * units * args.steps / (float(t.item()) / 1e3), "unit": UNIT,
+        e2e = {"value": weak_throughput(world, units, args.steps, max_over_ranks(e_ms, dev, world)), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "copies": e2e_mode}
 
     # roofline of the dominant kernel (largest share of the step); its duration comes from
