@@ -64,6 +64,17 @@ def dist_env():
     return rank, world, local
 
 
+def workload_config(name: str) -> dict:
+    """The config keys both arms report for a workload: its name and shape."""
+    from long_context_sparse_softmax_b200 import workloads as wl
+    specs = wl.WORKLOADS[name]
+    s = specs[0]
+    return {"workload": s.name if len(specs) == 1 else name,
+            "batch": s.num_seqs if s.is_decode else 1,
+            "context": max(s.seq_lens), "heads": s.H, "dims": s.D, "topk": s.k,
+            "query_tokens_per_step_per_gpu": s.num_seqs if s.is_decode else s.n_q}
+
+
 def rank_spec(spec, rank: int):
     """The workload a rank runs: the same shapes, its own seed (independent batches, weak
     scaling)."""
@@ -536,10 +547,7 @@ def run_lc(args):
         "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3+bf16 KV, mxfp4 indexer, fp32 accumulate" if not runs[0][0].fp32 else "f32",
         "data": "synthetic",
-        "config": {"workload": runs[0][0].name if len(runs) == 1 else args.workload,
-                   "batch": runs[0][0].num_seqs if runs[0][0].is_decode else 1,
-                   "context": max(runs[0][0].seq_lens), "heads": runs[0][0].H, "dims": runs[0][0].D,
-                   "topk": runs[0][0].k, "query_tokens_per_step_per_gpu": units,
+        "config": {**workload_config(args.workload), "query_tokens_per_step_per_gpu": units,
                    "l2": "flushed between timed steps, outside the step events (512 MiB write, then a "
                          "256 MiB read so that evicted lines are clean)",
                    "launch": "eager" if graph is None else "cuda graph of the step",
@@ -671,7 +679,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "sample": desc},
+        "config": {**workload_config(args.workload), "sample": desc},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"{desc}; one unit per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
