@@ -16,9 +16,9 @@
 //   * block scales in tensor memory: column c holds, in lane L of every lane quadrant, the
 //     four E8M0 bytes (K blocks 0..3) of row (L % 32) + 32 c; the k-th K = 64 MMA reads
 //     bytes 2k, 2k + 1 (sf_id = 2k);
-//   * warp roles (192 threads): warp 0 loads key tiles (TMA) and their scale words (one
-//     tile ahead, into registers; stored as 32 rows x 16 bytes, row L holding the words
-//     of keys L, L + 32, L + 64, L + 96) into a 4-stage ring; lane 0 of warp 1 copies a
+//   * warp roles (192 threads): warp 0 loads key tiles (TMA) and their scale words (four
+//     tiles ahead, into a register ring; stored as 32 rows x 16 bytes, row L holding the
+//     words of keys L, L + 32, L + 64, L + 96) into an 8-stage ring; lane 0 of warp 1 copies a
 //     tile's scales into tensor memory (tcgen05.cp 32x128b.warpx4, which fills every
 //     lane quadrant) and issues its MMAs into one of three accumulators; warps 2-5 run the
 //     epilogue: thread t owns key row t of D (tcgen05.ld 32x32b), so the ReLU-weighted

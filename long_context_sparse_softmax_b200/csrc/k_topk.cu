@@ -3,14 +3,18 @@
 // Top-512 (Flash) / Top-1024 (Pro)).
 //
 // A thread-block cluster of C CTAs takes one query row; CTA r holds the r-th of C equal
-// segments of the row.  Scores map to order-preserving 32-bit keys.  Three radix passes
-// (11, 11 and 10 bits) find the K-th largest key T and how many keys equal to T to take:
-// each CTA builds a 2048-bin histogram of its candidates in shared memory, the cluster
-// barrier publishes it, and every CTA sums the C histograms over distributed shared memory
-// in rank order, so all CTAs reach the same bin.  The selection is then every key > T and
-// the first `need` keys == T in index order (ties to the lower index), written in ascending
-// index order: the CTAs exchange their counts of keys > T and == T the same way, and
-// within a CTA each warp owns a contiguous piece of the segment.  Segments of up to
+// segments of the row.  Scores map to order-preserving 32-bit keys, taken relative to the
+// row's smallest key.  Radix passes of up to 11 bits find the K-th largest key T and how
+// many keys equal to T to take: each CTA builds a 2048-bin histogram of its candidates in
+// shared memory, the cluster barrier publishes it, and every CTA sums the C histograms
+// over distributed shared memory in rank order, so all CTAs reach the same bin.  When the
+// bin the first pass selects holds at most kCand keys of the whole row (the usual case),
+// every CTA gathers those keys from the cluster and finishes the selection alone, and each
+// rank's counts above and at T follow from the first pass's histograms; otherwise the
+// cluster-wide passes continue.  The selection is then every key > T and the first `need`
+// keys == T in index order (ties to the lower index), written in ascending index order:
+// the CTAs' counts of keys > T and == T give each one its first output slot, and within a
+// CTA each warp owns a contiguous piece of the segment.  Segments of up to
 // kRowCache keys are staged in shared memory once; longer ones are re-read from global
 // memory (L2) on each pass.  The result depends only on the score values: it is bit-exact
 // and independent of C and of the launch shape.
