@@ -1,0 +1,48 @@
+"""Host-side pieces of the bench and the runner that need no GPU: the tensor peaks per
+stage, the config both bench arms report, and which per-step inputs each stage reads."""
+import pytest
+
+import bench
+from long_context_sparse_softmax_b200 import runner
+from long_context_sparse_softmax_b200 import workloads as wl
+
+
+def test_tensor_peak_factors_follow_the_operand_types():
+    csa_p, hca_p = wl.WORKLOADS["csa_prefill"][0], wl.WORKLOADS["hca_prefill"][0]
+    # the MXFP4 indexer runs at 4x the BF16 rate
+    assert bench.tensor_mix("0:index", csa_p)[0] == 4.0
+    # E4M3 scores + F16 P V: half the flops at 2x, half at 1x
+    assert bench.tensor_mix("0:attn", csa_p)[0] == pytest.approx(4.0 / 3.0)
+    assert bench.tensor_mix("0:attn", csa_p, "tc16")[0] == 1.0  # every operand widened to F16
+    assert bench.tensor_mix("0:attn", hca_p)[0] == 1.0          # BF16 queries: the F16 kernel
+    # a tensor-bound stage's roofline time uses that factor
+    work = {"0:index": (1.0, 4.0e12)}
+    pk = {"hbm_gbs": 1e9, "bf16_tflops": 1000.0}
+    bnd, t = bench.bound_of("0:index", csa_p, work, pk)
+    assert bnd == "tensor" and t == pytest.approx(4.0e12 / (4000.0e12))
+
+
+def test_both_arms_report_one_config():
+    c = bench.workload_config("csa_decode")
+    assert c == {"workload": "csa_decode_b32_L131072_k512", "batch": 32, "context": 131072, "heads": 64,
+                 "dims": 576, "topk": 512, "query_tokens_per_step_per_gpu": 32}
+    assert bench.workload_config("mixed_decode")["workload"] == "mixed_decode"
+
+
+def test_host_inputs_name_the_stage_that_reads_them():
+    s = wl.shrink(wl.CSA_DECODE, name="host_io_decode", seq_lens=(512, 700), k=64)
+    inp = wl.make_decode(s, "cpu")
+    r = runner.Decode(inp, "cpu")
+    h = r.host_inputs()
+    assert h["qk_prep_q"][0] is inp["q_raw"]
+    assert h["qk_prep_win"][0] is inp["x_new"]
+    assert h["compress"][0] is inp["x_tail"] and h["compress"][1] is inp["g_tail"]
+    assert set(map(id, h["index"])) == set(map(id, inp["qI"].values()))
+    assert r.host_outputs() == [r.out, r.lse]
+    # prefill: the raw tokens feed both window preparation and compression (two side
+    # streams), so they are copied before the fork
+    p = wl.shrink(wl.CSA_PREFILL, name="host_io_prefill", seq_lens=(600,), H=16, k=32, n_q=600)
+    ip = wl.make_prefill(p, "cpu")
+    hp = runner.Prefill(ip, "cpu").host_inputs()
+    assert hp["_fork"][0] is ip["x"] and hp["_fork"][1] is ip["g"]
+    assert "qk_prep_win" not in hp and "compress" not in hp
