@@ -134,3 +134,28 @@ def test_mxfp4_saturation_and_zero_block():
     assert scales.tolist() == [[127, 127]]
     d = O.mxfp4_to_f64(codes.numpy(), scales.numpy())
     assert d[0, 32] == 6.0 and d[0, 33] == -6.0 and np.all(d[0, :32] == 0)
+
+
+def test_e2m1_values_match_ml_dtypes():
+    """The 16 E2M1 codes against ml_dtypes' float4_e2m1fn (an independent decoder of the
+    OCP MX v1.0 element type)."""
+    ml_dtypes = pytest.importorskip("ml_dtypes")
+    ref = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    assert np.array_equal(O.e2m1_to_f64(np.arange(16)), ref)
+
+
+def test_mxfp4_decode_matches_an_independent_dequantizer_on_every_byte_and_scale():
+    """Nibble order, element values and block scaling of the oracle's MXFP4 decoder
+    against OpenAI's triton_kernels MXFP4 upcast (pure torch; vendored by vllm): all 256
+    byte codes (16 blocks of 32 elements) under every E8M0 scale code 1..252.  Scale code
+    0 is left out because that upcast maps it to 0 rather than 2^-127; codes 253 and 254
+    overflow its FP32 output (6 * 2^126 > FP32 max); code 255 is NaN in OCP MX."""
+    mx = pytest.importorskip("vllm.third_party.triton_kernels.numerics_details.mxfp")
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8).reshape(16, 16)
+    for s0 in range(1, 253, 16):
+        sc = torch.clamp(torch.arange(s0, s0 + 16), max=252).to(torch.uint8).reshape(16, 1)
+        ref = mx.upcast_from_mxfp_torch(codes, sc, torch.float32, axis=-1).double().numpy()
+        mine = O.mxfp4_to_f64(codes.numpy(), sc.numpy())
+        assert np.array_equal(mine, ref), f"scales {s0}..{s0 + 15}"
+    # element 2i in the low nibble: byte 0x61 holds 0.5 (code 1) then 4.0 (code 6)
+    assert np.array_equal(O.mxfp4_to_f64(np.full((1, 16), 0x61, np.uint8), np.array([[127]]))[0, :2], [0.5, 4.0])

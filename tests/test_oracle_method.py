@@ -84,6 +84,23 @@ def test_gate_weights_closed_form():
     np.testing.assert_allclose(O.pool_block(x, g), np.array([1, 2, 3, 4]) / 10.0, rtol=1e-14)
 
 
+def test_pooling_comes_before_rmsnorm():
+    """The entry is RMSNorm of the gated pool, not the pool of normalised tokens: two
+    tokens of different norms with equal gates (closed form, no RoPE dims).  With
+    x1 = 2 e0 and x2 = 6 e1 the pool is e0 + 3 e1, whose RMS over D dims is sqrt(10 / D);
+    normalising each token first would give equal weights on e0 and e1 instead."""
+    D = 64
+    x = np.zeros((2, D))
+    x[0, 0] = 2.0
+    x[1, 1] = 6.0
+    e = O.compress(x, np.zeros(2), 2, 0, 0)
+    r = np.sqrt(10.0 / D + O.RMS_EPS)
+    expect = np.zeros(D)
+    expect[0], expect[1] = 1.0 / r, 3.0 / r
+    np.testing.assert_allclose(e[0], expect, rtol=1e-14, atol=0)
+    assert abs(e[0, 1] / e[0, 0] - 3.0) < 1e-12
+
+
 def test_block_entry_is_roped_at_its_last_position():
     """A block of identical tokens pools to that token; its entry equals the token
     prepared at position (j+1)m - 1."""
