@@ -14,7 +14,7 @@ the cache clean) between timed steps, outside the per-step CUDA events.  The ste
 captured once as a CUDA graph and replayed (--no-graph: every call launched from Python).  With N > 1 (torchrun) every rank runs its own batch: weak
 scaling, no collective on the data path.
 --impl reference times the CPU oracle (the plain float64 restatement of the method) on a
-bounded sample of the same workload on the host cores (rank 0 only).
+bounded sample of the same workload on one host core (rank 0 only).
 """
 from __future__ import annotations
 
@@ -51,8 +51,8 @@ def parse():
                     "instead of replaying the step's CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0)
-    ap.add_argument("--attn-impl", default="auto", choices=["auto", "mma", "tc", "ref", "tc16"],
-                    help="attention kernel (auto: tcgen05 where it applies, else mma.sync, else reference; tc16: the F16-score tcgen05 kernel)")
+    ap.add_argument("--attn-impl", default="auto", choices=["auto", "tc", "ref"],
+                    help="attention kernel (auto: tcgen05 where it applies, else the FP32 reference kernel)")
     return ap.parse_args()
 
 
@@ -258,15 +258,16 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def kernel_traffic(stage_kernel: str, attn_impl: str):
-    """DRAM bytes per launch of a stage's kernels from the committed ncu summary, if every
-    source file of those kernels is unchanged since the capture (and, for attention, the
-    same kernel choice ran); else None."""
+def kernel_traffic(workload: str, stage: str, attn_impl: str):
+    """DRAM bytes per launch of a stage's kernels on this workload from the committed ncu
+    summary (keyed "<workload>:<stage>"), if that workload was captured and every source
+    file of those kernels is unchanged since the capture (and, for attention, the same
+    kernel choice ran); else None."""
     if not os.path.exists(TRAFFIC_PATH):
         return None
     with open(TRAFFIC_PATH) as f:
         t = json.load(f)
-    e = t.get(stage_kernel)
+    e = t.get(f"{workload}:{stage}")
     if not e:
         return None
     if "attn_impl" in e and attn_impl not in e["attn_impl"]:
@@ -318,7 +319,7 @@ def run_lc(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     pk, pk_kind = peaks()
-    runs = make_runs(args.workload, dev, rank, {"auto": 0, "mma": 1, "tc": 2, "ref": 3, "tc16": 4}[args.attn_impl])
+    runs = make_runs(args.workload, dev, rank, {"auto": 0, "tc": 2, "ref": 3}[args.attn_impl])
     # L2 flush: a 512 MiB write, then a 256 MiB read so that the lines the step evicts are
     # clean (the write alone would leave L2 full of dirty lines whose write-back lands on
     # the first kernel of the step)
@@ -531,7 +532,7 @@ def run_lc(args):
         factor, mix = tensor_mix(dom, spec0, args.attn_impl)
         peak, unit = pk["bf16_tflops"] * factor, "TFLOP/s"
         pk_kind = f"{pk_kind} bf16 x {factor:.3g} ({mix}; nominal dtype ratio)"
-    traffic = kernel_traffic(dom.split(":")[1], args.attn_impl)
+    traffic = kernel_traffic(args.workload, dom.split(":")[1], args.attn_impl)
     stages = {}
     for n in stage_names:
         bb, ff = work[n]
@@ -577,13 +578,20 @@ def run_lc(args):
 # ------------------------------------------------------------------------------------
 # the oracle (CPU baseline / reference arm)
 # ------------------------------------------------------------------------------------
-def _blas_threads():
+def _one_thread():
+    """Context that limits numpy's BLAS to one thread: the oracle is timed single-threaded
+    on one host core."""
+    from threadpoolctl import threadpool_limits
+    return threadpool_limits(limits=1)
+
+
+def _lc_libs_mapped():
+    """Shared objects of this library mapped into the process (the oracle legs load none)."""
     try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:
-        return os.cpu_count() or 1
+        with open("/proc/self/maps") as f:
+            return sorted({ln.split()[-1] for ln in f if ln.rstrip().endswith("liblc.so")})
+    except OSError:
+        return []
 
 
 def oracle_unit(name: str):
@@ -648,16 +656,17 @@ def oracle_unit(name: str):
 
 def cpu_baseline(name: str, budget_s: float):
     unit, desc = oracle_unit(name)
-    unit()
-    n, t0 = 0, time.perf_counter()
-    while True:
+    with _one_thread():
         unit()
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s or n >= 10000:
-            break
-    return {"value": n / el, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{desc}; {n} units in {el:.1f} s"}
+        n, t0 = 0, time.perf_counter()
+        while True:
+            unit()
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s or n >= 10000:
+                break
+    return {"value": n / el, "unit": UNIT, "cores": 1, "host_cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{desc}; {n} units in {el:.1f} s, one thread"}
 
 
 def run_reference(args):
@@ -665,24 +674,25 @@ def run_reference(args):
     if rank != 0:
         return
     unit, desc = oracle_unit(args.workload)
-    for _ in range(args.warmup):
-        unit()
     t = []
-    for _ in range(args.steps):
-        t0 = time.perf_counter()
-        unit()
-        t.append(time.perf_counter() - t0)
+    with _one_thread():
+        for _ in range(args.warmup):
+            unit()
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            unit()
+            t.append(time.perf_counter() - t0)
     total = sum(t)
     value = args.steps / total
-    cores = _blas_threads()
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {**workload_config(args.workload), "sample": desc},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"{desc}; one unit per step"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "host_cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"{desc}; one unit per step, one thread"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "native_libs_loaded": _lc_libs_mapped(),
     }), flush=True)
 
 

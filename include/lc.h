@@ -189,7 +189,7 @@ lc_status lc_hca_compress_decode(const lc_compress_args* a, void* stream);
  * ------------------------------------------------------------------------------- */
 typedef struct lc_index_args {
   int32_t n_q;
-  int32_t H_I;             /* indexer heads (<= 128) */
+  int32_t H_I;             /* indexer heads (F32: H_I * d_I <= 16384; MXFP4: 32 or 64) */
   int32_t d_I;             /* indexer dims (F32: multiple of 4, <= 256; MXFP4: 128) */
   int32_t fmt;             /* LC_IDX_F32 or LC_IDX_MXFP4 */
   const void* q;           /* F32 [n_q, H_I, d_I] or MXFP4 codes [n_q, H_I, d_I/2] */
@@ -270,10 +270,10 @@ typedef struct lc_attn_args {
   void* workspace;
   size_t workspace_bytes;
   int32_t* status;
-  int32_t impl;            /* LC_IMPL_AUTO (0) picks the fastest kernel for the shape;
-                              LC_IMPL_MMA, LC_IMPL_TC, LC_IMPL_REF, LC_IMPL_TC_F16 force one (results agree
-                              within the BF16 tolerance; LC_ERR_UNSUPPORTED if it cannot run
-                              the shape) */
+  int32_t impl;            /* LC_IMPL_AUTO (0): the tensor-core kernels where they apply,
+                              else the reference kernel; LC_IMPL_TC or LC_IMPL_REF force one
+                              (LC_ERR_UNSUPPORTED if it cannot run the shape); other values
+                              are LC_ERR_ARG */
   int32_t n_ent_rows;      /* rows of ent (every ent_start[b] + n_ent[b] <= n_ent_rows), or 0 if
                               unknown; the FP8 tensor-core kernel reads entries by bulk tensor
                               copies and needs it */
@@ -285,13 +285,13 @@ typedef struct lc_attn_args {
 /* Attention kernels. */
 enum {
   LC_IMPL_AUTO = 0,
-  LC_IMPL_MMA = 1,         /* BF16 mma.sync tiles (576-dim entries) */
-  LC_IMPL_TC = 2,          /* tcgen05 tiles, accumulators in tensor memory (576-dim entries):
-                              E4M3 scores from bulk-copied tiles where queries and entries are
-                              E4M3 + BF16 RoPE and n_ent_rows (and, with W > 0, n_win_rows)
-                              is set, else the F16 kernel */
-  LC_IMPL_REF = 3,         /* one warp per (query, head), FP32 CUDA cores (any shape) */
-  LC_IMPL_TC_F16 = 4       /* tcgen05 tiles with every operand widened to F16 */
+  LC_IMPL_TC = 2,          /* tcgen05 tiles, accumulators in tensor memory (576-dim entries,
+                              64 RoPE dims, heads in groups of 64): E4M3 scores from
+                              bulk-copied tiles where queries and entries are E4M3 + BF16 RoPE
+                              and n_ent_rows (and, with W > 0, n_win_rows) is set, else every
+                              operand widened to F16 (BF16 queries) */
+  LC_IMPL_REF = 3          /* one warp per (query, head), FP32 CUDA cores (any shape; the
+                              FP32 workload) */
 };
 
 lc_status lc_csa_sparse_attn_prefill(const lc_attn_args* a, void* stream);
@@ -322,7 +322,9 @@ size_t lc_hca_attn_workspace_bytes(const lc_attn_args* a);
  *   - Every call on a device shares the one array.  Calls whose executions overlap on the
  *     GPU (different streams, or other threads) race on it and give wrong results: order
  *     them on one stream or serialise them.  Nothing carries over from one call to the
- *     next: every scratch word a call reads, the same call has written first.
+ *     next: every scratch word a call reads, the same call has written first, except
+ *     after a bounded wait gave up (LC_DEV_TIMEOUT in *status): the outputs of that call
+ *     are then undefined and may mix in an earlier call's partial results.
  * ------------------------------------------------------------------------------- */
 lc_status lc_csa_sparse_attn_decode_static(const lc_attn_args* a, void* stream);
 size_t lc_csa_sparse_attn_decode_static_capacity(void);

@@ -1,8 +1,11 @@
 """CSA / HCA long-context sparse attention for NVIDIA B200 — Python binding of liblc.so.
 
 The binding only marshals arguments: every step of the path runs in the library's CUDA
-kernels.  There is no CPU fallback; importing the package fails if liblc.so is missing
-(build it with ``python long_context_sparse_softmax_b200/build_lib.py``).
+kernels.  There is no CPU fallback.  liblc.so is loaded on first use (the first call, or
+the first access to ``lib``), and that use raises ImportError if the library is missing
+(build it with ``python long_context_sparse_softmax_b200/build_lib.py``).  Importing the
+package alone loads nothing, so its input generators (``workloads``) can be used by a
+process that never touches the GPU library.
 
 Each C entry point ``lc_<op>_<variant>(const args*, stream)`` is exposed under the same
 name; it takes the ctypes mirror of the args struct and an optional torch stream and
@@ -26,7 +29,7 @@ LC_IDX_F32, LC_IDX_MXFP4 = 0, 3
 
 class LcError(RuntimeError):
     def __init__(self, status: int, where: str):
-        super().__init__(f"{where}: {lib.lc_status_string(status).decode()} (status {status})")
+        super().__init__(f"{where}: {load().lc_status_string(status).decode()} (status {status})")
         self.status = status
 
 
@@ -79,7 +82,7 @@ class AttnArgs(ctypes.Structure):
                 ("n_win_rows", c_int32)]
 
 
-LC_IMPL_AUTO, LC_IMPL_MMA, LC_IMPL_TC, LC_IMPL_REF, LC_IMPL_TC_F16 = 0, 1, 2, 3, 4
+LC_IMPL_AUTO, LC_IMPL_TC, LC_IMPL_REF = 0, 2, 3
 
 
 STRUCTS = [Rows, Dims, Batch, QkPrepArgs, CompressArgs, IndexArgs, TopkArgs, AttnArgs]
@@ -122,7 +125,21 @@ def _load() -> ctypes.CDLL:
     return so
 
 
-lib = _load()
+_LIB = None
+
+
+def load() -> ctypes.CDLL:
+    """The loaded liblc.so (loaded and checked on the first call)."""
+    global _LIB
+    if _LIB is None:
+        _LIB = _load()
+    return _LIB
+
+
+def __getattr__(name):
+    if name == "lib":
+        return load()
+    raise AttributeError(name)
 
 
 def _stream_handle(stream) -> c_void_p:
@@ -135,12 +152,10 @@ def _stream_handle(stream) -> c_void_p:
 
 
 def _make_call(name: str, st):
-    fn = getattr(lib, name)
-
     def call(args, stream=None):
         if not isinstance(args, st):
             raise TypeError(f"{name} takes {st.__name__}")
-        s = fn(ctypes.byref(args), _stream_handle(stream))
+        s = getattr(load(), name)(ctypes.byref(args), _stream_handle(stream))
         if s != LC_OK:
             raise LcError(s, name)
 
@@ -154,16 +169,16 @@ for _n, _st in ENTRY_POINTS.items():
 
 
 def lc_csa_sparse_attn_workspace_bytes(args: AttnArgs) -> int:
-    return int(lib.lc_csa_sparse_attn_workspace_bytes(ctypes.byref(args)))
+    return int(load().lc_csa_sparse_attn_workspace_bytes(ctypes.byref(args)))
 
 
 def lc_hca_attn_workspace_bytes(args: AttnArgs) -> int:
-    return int(lib.lc_hca_attn_workspace_bytes(ctypes.byref(args)))
+    return int(load().lc_hca_attn_workspace_bytes(ctypes.byref(args)))
 
 
 def lc_csa_sparse_attn_decode_static_capacity() -> int:
-    return int(lib.lc_csa_sparse_attn_decode_static_capacity())
+    return int(load().lc_csa_sparse_attn_decode_static_capacity())
 
 
 def lc_version() -> str:
-    return lib.lc_version().decode()
+    return load().lc_version().decode()

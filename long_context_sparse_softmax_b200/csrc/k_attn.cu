@@ -132,73 +132,49 @@ __global__ void __launch_bounds__(256) k_attn_ref(lc_attn_args a, int sparse) {
   if (a.lse && lane == 0) a.lse[qrow] = st.m + logf(st.z);
 }
 
-// The kernel a call runs (never LC_IMPL_AUTO): AUTO takes the fastest one measured for
-// 576-dim BF16 / E4M3 shapes, the BF16 mma.sync kernel; other shapes (FP32, other head
-// dims) run on the reference kernel.
-// The automatic choice: the tcgen05 kernels where they apply (576-dim rows with 64 RoPE
-// dims, 64-head groups, 16-byte aligned buffers), else the mma.sync kernel, else the
-// reference kernel.  LC_IMPL_TC takes the E4M3-score kernel where queries and entries are
-// E4M3 + BF16 RoPE, else the F16 one.
+// The kernel a call runs.  AUTO (and TC) take the tcgen05 kernels where they apply
+// (576-dim rows with 64 RoPE dims, 64-head groups, 16-byte aligned buffers): the
+// E4M3-score kernel where queries and entries are E4M3 + BF16 RoPE, else the F16-operand
+// kernel (BF16 queries).  Every other shape (the FP32 workload, other head dims) runs on
+// the reference kernel above, which REF also forces.
 static bool tc_any(const lc_attn_args& a) { return attn_tc8_supported(a) || attn_tc_supported(a); }
 
 int attn_impl(const lc_attn_args& a) {
-  if (a.impl != LC_IMPL_AUTO) return a.impl;
-  if (tc_any(a)) return LC_IMPL_TC;
-  return attn_mma_supported(a) ? LC_IMPL_MMA : LC_IMPL_REF;
+  if (a.impl == LC_IMPL_REF) return LC_IMPL_REF;
+  if (a.impl == LC_IMPL_TC) return LC_IMPL_TC;
+  return tc_any(a) ? LC_IMPL_TC : LC_IMPL_REF;
 }
 
-bool attn_impl_ok(const lc_attn_args& a) {
-  switch (attn_impl(a)) {
-    case LC_IMPL_MMA: return attn_mma_supported(a);
-    case LC_IMPL_TC: return tc_any(a);
-    case LC_IMPL_TC_F16: return attn_tc_supported(a);
-    case LC_IMPL_REF: return true;
-    default: return false;
-  }
-}
+bool attn_impl_ok(const lc_attn_args& a) { return attn_impl(a) == LC_IMPL_REF || tc_any(a); }
 
 size_t attn_workspace_bytes(const lc_attn_args& a, bool sparse, bool decode) {
+  if (attn_impl(a) != LC_IMPL_TC) return 0;
   if (a.impl == LC_IMPL_AUTO) {
-    // the choice may depend on buffer alignment, which the caller may not have fixed yet
-    size_t w = attn_mma_supported(a) ? attn_mma_workspace(a, sparse, decode) : 0;
+    // the choice between the two tcgen05 kernels may depend on buffer alignment, which
+    // the caller may not have fixed yet: the larger of the two
     lc_attn_args t = a;
     t.out = nullptr;
     t.workspace = nullptr;
-    if (tc_any(t)) {
-      w = w > attn_tc_workspace(a, sparse, decode) ? w : attn_tc_workspace(a, sparse, decode);
-      w = w > attn_tc8_workspace(a, sparse, decode) ? w : attn_tc8_workspace(a, sparse, decode);
-    }
-    return w;
+    if (!tc_any(t)) return 0;
+    const size_t w0 = attn_tc_workspace(a, sparse, decode), w1 = attn_tc8_workspace(a, sparse, decode);
+    return w0 > w1 ? w0 : w1;
   }
-  switch (attn_impl(a)) {
-    case LC_IMPL_MMA: return attn_mma_supported(a) ? attn_mma_workspace(a, sparse, decode) : 0;
-    case LC_IMPL_TC:
-      if (attn_tc8_supported(a)) return attn_tc8_workspace(a, sparse, decode);
-      return attn_tc_supported(a) ? attn_tc_workspace(a, sparse, decode) : 0;
-    case LC_IMPL_TC_F16: return attn_tc_supported(a) ? attn_tc_workspace(a, sparse, decode) : 0;
-    default: return 0;
-  }
+  if (attn_tc8_supported(a)) return attn_tc8_workspace(a, sparse, decode);
+  return attn_tc_supported(a) ? attn_tc_workspace(a, sparse, decode) : 0;
 }
 
 cudaError_t launch_attn(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st) {
   if (a.n_q == 0) return cudaSuccess;
-  switch (attn_impl(a)) {
-    case LC_IMPL_TC:
-    case LC_IMPL_TC_F16: {
-      int n_split = 1;
-      const bool fp8 = attn_impl(a) == LC_IMPL_TC && attn_tc8_supported(a);
-      cudaError_t e = fp8 ? launch_attn_tc8(a, sparse, decode, st, &n_split) : launch_attn_tc(a, sparse, decode, st, &n_split);
-      if (e != cudaSuccess || n_split == 1) return e;
-      return launch_attn_combine(a, n_split, st);
-    }
-    case LC_IMPL_MMA:
-      return launch_attn_mma(a, sparse, decode, st);
-    default: {
-      const dim3 grid(a.n_q, (a.dims.H + 7) / 8);
-      k_attn_ref<<<grid, 256, 0, st>>>(a, sparse ? 1 : 0);
-      return cudaGetLastError();
-    }
+  if (attn_impl(a) == LC_IMPL_TC) {
+    int n_split = 1;
+    const bool fp8 = attn_tc8_supported(a);
+    cudaError_t e = fp8 ? launch_attn_tc8(a, sparse, decode, st, &n_split) : launch_attn_tc(a, sparse, decode, st, &n_split);
+    if (e != cudaSuccess || n_split == 1) return e;
+    return launch_attn_combine(a, n_split, st);
   }
+  const dim3 grid(a.n_q, (a.dims.H + 7) / 8);
+  k_attn_ref<<<grid, 256, 0, st>>>(a, sparse ? 1 : 0);
+  return cudaGetLastError();
 }
 
 }  // namespace lc

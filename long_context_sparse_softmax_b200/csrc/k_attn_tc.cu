@@ -37,6 +37,7 @@
 // wait is bounded: a role that gives up sets LC_DEV_TIMEOUT and an abort flag that stops
 // the others at their next wait.
 #include "lc_internal.h"
+#include "lc_ptx.cuh"
 
 namespace lc {
 
@@ -64,95 +65,6 @@ constexpr uint32_t kTmemCols = 512;
 static_assert(kNP % 4 == 0 && kNPair % 4 == 0 && (kDN / 16) % 4 == 0, "piece grouping");
 
 constexpr size_t kSmem = 3 * static_cast<size_t>(kTile) + kPBytes + 2 * kTK * 4 + kNR * 4;
-
-__device__ __forceinline__ uint32_t su32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
-
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFF);
-  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16;
-  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32;
-  d |= static_cast<uint64_t>(1) << 46;
-  return d;
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(bar));
-}
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile("{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-               : "=r"(done)
-               : "r"(bar), "r"(parity));
-  return done != 0;
-}
-// non-blocking probe (try_wait may suspend the thread for a while; a thread that polls
-// several barriers must not sleep on one of them)
-__device__ __forceinline__ bool mbar_probe(uint32_t bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile("{\n.reg .pred p;\nmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-               : "=r"(done)
-               : "r"(bar), "r"(parity));
-  return done != 0;
-}
-
-__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n"); }
-__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
-__device__ __forceinline__ void named_bar(int id, int n) {
-  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
-}
-// named barrier that also ORs a predicate over the participating threads
-__device__ __forceinline__ bool named_bar_or(int id, int n, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n.reg .pred pi, po;\nsetp.ne.b32 pi, %1, 0;\nbar.red.or.pred po, %2, %3, pi;\nselp.u32 %0, 1, 0, po;\n}\n"
-      : "=r"(r)
-      : "r"(static_cast<int>(v)), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
-
-__device__ __forceinline__ void mma_f16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc));
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar));
-}
-
-#define LC_R32(r)                                                                                                 \
-  "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),   \
-      "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),      \
-      "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),     \
-      "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-#define LC_REGS32                                                                                                 \
-  "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29," \
-  "%30,%31}"
-
-// lane i of the warp's quarter, 32 consecutive columns
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 " LC_REGS32 ", [%32];\n" : LC_R32(r) : "r"(taddr));
-}
-// lanes 0-15 of the quarter: thread i < 16 gets lane i, columns c..c+31; thread 16 + i
-// gets lane i, columns c+32..c+63
-__device__ __forceinline__ void tmem_ld16x2(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x32.b32 " LC_REGS32 ", [%32], 32;\n" : LC_R32(r) : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
-      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
-      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
-      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]));
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
 // 8 E4M3 values -> 8 F16 values, exact (E4M3 is a subset of F16)
 __device__ __forceinline__ uint4 e4m3x8_f16x8(uint32_t lo, uint32_t hi) {
@@ -286,13 +198,6 @@ __device__ __forceinline__ bool tile_convert(uint8_t* tile, int wi, int nw, int 
     }
   }
   return big;
-}
-
-// 2^x on the special function unit (relative error far below the F16 rounding of P)
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
-  return y;
 }
 
 __device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
@@ -460,8 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                (static_cast<uint32_t>(kNR >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
       const uint32_t id_o64 = (1u << 4) | (1u << 15) |
                               (static_cast<uint32_t>(kNR >> 3) << 17) | (static_cast<uint32_t>(64 >> 4) << 24);
-      const uint64_t dq = sdesc(su32(Qs), 128, kG);
-      const uint64_t dp = sdesc(su32(Ps), 128, (kTK / 8) * 128);
+      const uint64_t dq = cm_desc(su32(Qs), 128, kG);
+      const uint64_t dp = cm_desc(su32(Ps), 128, (kTK / 8) * 128);
       // Issue whichever group is ready: S(ns) once its key stage is full and its S buffer
       // read, O(no) once P(no) is written.  S runs at most two tiles ahead of O (the key
       // stage of S(no + 2) is released by O(no)).
@@ -475,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (mbar_probe(su32(&bars.kfull[st]), (ns >> 1) & 1) &&
               (ns < 2 || mbar_probe(su32(&bars.sempty[st]), ((ns >> 1) - 1) & 1))) {
             fence_after();
-            const uint64_t dk = sdesc(su32(Ks + st * kTile), 128, kG);
+            const uint64_t dk = cm_desc(su32(Ks + st * kTile), 128, kG);
 #pragma unroll
             for (int k = 0; k < kD / 16; ++k)
               mma_f16(tm + kColS + st * kTK, dq + k * 16, dk + k * 16, id_s, k > 0);
@@ -487,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (no < ns && mbar_probe(su32(&bars.pfull), no & 1)) {
           fence_after();
           // V^T: M = dims (chunk stride 128 B), K = keys (group stride kG); P^T: K-major
-          const uint64_t dv = sdesc(su32(Ks + (no & 1) * kTile), kG, 128);
+          const uint64_t dv = cm_desc(su32(Ks + (no & 1) * kTile), kG, 128);
 #pragma unroll
           for (int kk = 0; kk < kTK / 16; ++kk)
 #pragma unroll
@@ -694,9 +599,10 @@ static AttnTcGeom tc_geometry(const lc_attn_args& a, bool sparse, bool decode) {
   const int tiles = (ns + kTK - 1) / kTK;
   g.sps = tiles * kTK;
   const int ctas = a.n_q * (a.dims.H / kNR);
-  if (decode && ctas < 148) {
+  const int n_sm = sm_count();
+  if (decode && ctas < n_sm) {
     // one CTA per SM: split the keys when the (query, head group) pairs leave SMs idle
-    const int n = max(1, min(148 / max(ctas, 1), tiles));
+    const int n = max(1, min(n_sm / max(ctas, 1), tiles));
     const int per = (tiles + n - 1) / n;
     g.n_split = (tiles + per - 1) / per;
     g.sps = per * kTK;

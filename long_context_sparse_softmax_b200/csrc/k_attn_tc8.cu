@@ -32,6 +32,7 @@
 #include <cuda.h>
 
 #include "lc_internal.h"
+#include "lc_ptx.cuh"
 
 namespace lc {
 
@@ -67,140 +68,6 @@ constexpr int kOffCode = kOffP + kPBytes;         // [4][kTK] key codes
 constexpr int kOffF = kOffCode + 4 * kTK * 4;     // [kNR] per-head factors
 constexpr size_t kSmem = kOffF + kNR * 4 + 1024;  // + alignment slack
 static_assert(2 * kRawStage >= kTile, "Q in BF16 fits the raw stages");
-
-__device__ __forceinline__ uint32_t su32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
-
-// no-swizzle core-matrix operand
-__device__ __forceinline__ uint64_t cm_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFF);
-  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16;
-  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32;
-  d |= static_cast<uint64_t>(1) << 46;
-  return d;
-}
-// K-major SWIZZLE_128B operand: 128-byte rows, 8-row groups 1024 bytes apart
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
-  uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFF);
-  d |= static_cast<uint64_t>(1) << 16;
-  d |= static_cast<uint64_t>(1024 >> 4) << 32;
-  d |= static_cast<uint64_t>(1) << 46;
-  d |= static_cast<uint64_t>(2) << 61;
-  return d;
-}
-// MN-major SWIZZLE_128B operand: 128-byte rows run along M (64 16-bit values), one row per
-// K index, 8-row groups 1024 bytes apart (SBO); the next 64 values of M start kBlk bytes
-// further (LBO)
-__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t addr) {
-  uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFF);
-  d |= static_cast<uint64_t>(kBlk >> 4) << 16;
-  d |= static_cast<uint64_t>(1024 >> 4) << 32;
-  d |= static_cast<uint64_t>(1) << 46;
-  d |= static_cast<uint64_t>(2) << 61;
-  return d;
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile("{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-               : "=r"(done)
-               : "r"(bar), "r"(parity)
-               : "memory");
-  return done != 0;
-}
-__device__ __forceinline__ bool mbar_probe(uint32_t bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile("{\n.reg .pred p;\nmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-               : "=r"(done)
-               : "r"(bar), "r"(parity)
-               : "memory");
-  return done != 0;
-}
-
-__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n"); }
-__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
-__device__ __forceinline__ void named_bar(int id, int n) {
-  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
-}
-__device__ __forceinline__ bool named_bar_or(int id, int n, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n.reg .pred pi, po;\nsetp.ne.b32 pi, %1, 0;\nbar.red.or.pred po, %2, %3, pi;\nselp.u32 %0, 1, 0, po;\n}\n"
-      : "=r"(r)
-      : "r"(static_cast<int>(v)), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
-
-template <int KIND>  // 0: kind::f16, 1: kind::f8f6f4
-__device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  if (KIND == 0)
-    asm volatile(
-        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
-            d),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc));
-  else
-    asm volatile(
-        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(
-            d),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc));
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar));
-}
-
-#define LC8_R32(r)                                                                                                \
-  "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),   \
-      "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),      \
-      "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),     \
-      "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-#define LC8_REGS32                                                                                                \
-  "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29," \
-  "%30,%31}"
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 " LC8_REGS32 ", [%32];\n" : LC8_R32(r) : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld16x2(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x32.b32 " LC8_REGS32 ", [%32], 32;\n" : LC8_R32(r) : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
-      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
-      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
-      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]));
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
-
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int r0, int r1, int r2, int r3,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
-      "%4, %5, %6}], [%7];\n" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tma_tile2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::
-          "r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
 
 // 16 E4M3 values -> 16 F16 values (exact)
 __device__ __forceinline__ void e4m3x16_f16(uint4 v, uint4& lo, uint4& hi) {
@@ -252,14 +119,7 @@ __device__ __forceinline__ bool f16_inf(__half2 a) {
 
 // byte offset of dim chunk c (8 dims) of row r in the F16 core-matrix tile
 __device__ __forceinline__ uint32_t tile_off(int r, int c) { return (r >> 3) * kG + c * 128 + (r & 7) * 16; }
-// byte offset of 16-byte chunk j of row r in a SWIZZLE_128B block of 128-byte rows
-__device__ __forceinline__ uint32_t sw128_off(int r, int j) { return r * 128 + ((j ^ (r & 7)) << 4); }
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
-  return y;
-}
 
 struct Bars {
   uint64_t qfull;      // Q nope + RoPE landed (expect-tx)
@@ -507,11 +367,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int cb = 0; cb < 4; ++cb)
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                  mma<1>(d, sw128_desc(su32(Qn) + cb * kBlk + k * 32), sw128_desc(st + cb * kBlk + k * 32), id_s8,
+                  mma_f8(d, sw128_desc(su32(Qn) + cb * kBlk + k * 32), sw128_desc(st + cb * kBlk + k * 32), id_s8,
                          cb > 0 || k > 0);
 #pragma unroll
               for (int k = 0; k < 4; ++k)
-                mma<0>(d, sw128_desc(su32(Qr) + k * 32), sw128_desc(st + kRawN + k * 32), id_sbf, 1);
+                mma_f16(d, sw128_desc(su32(Qr) + k * 32), sw128_desc(st + kRawN + k * 32), id_sbf, 1);
               mma_commit(su32(&bars.kempty[e & 1]));
             } else {
               // A: Q in BF16 (core matrices); B: the window tile as it landed, BF16, SW128, 64
@@ -520,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint64_t dq = cm_desc(su32(Q16), 128, kG);
 #pragma unroll
               for (int k = 0; k < kD / 16; ++k)
-                mma<0>(d, dq + k * 16, sw128_desc(su32(Vt) + (k >> 2) * kBlk + (k & 3) * 32), id_sbf, k > 0);
+                mma_f16(d, dq + k * 16, sw128_desc(su32(Vt) + (k >> 2) * kBlk + (k & 3) * 32), id_sbf, k > 0);
               mma_commit(su32(&bars.wsdone));
               if (ns == n_wt - 1) mma_commit(su32(&bars.q16free));
             }
@@ -536,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < kTK / 16; ++kk)
 #pragma unroll
               for (int c = 0; c < 5; ++c)
-                mma<0>(tm + kColO + c * kNR, dv + (c * 2048 + kk * 2 * kG) / 16, dp + kk * 16,
+                mma_f16(tm + kColO + c * kNR, dv + (c * 2048 + kk * 2 * kG) / 16, dp + kk * 16,
                        c < 4 ? id_o128 : id_o64, (no > 0) || (kk > 0));
           } else {
             // window tile: V^T straight from the SW128 tile (dims along M, 16 keys per step)
@@ -544,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < kTK / 16; ++kk)
 #pragma unroll
               for (int c = 0; c < 5; ++c)
-                mma<0>(tm + kColO + c * kNR, sw128_mn_desc(su32(Vt) + c * 2 * kBlk + kk * 2048), dp + kk * 16,
+                mma_f16(tm + kColO + c * kNR, sw128_mn_desc(su32(Vt) + c * 2 * kBlk + kk * 2048, kBlk), dp + kk * 16,
                        c < 4 ? id_o128 : id_o64, (no > 0) || (kk > 0));
           }
           mma_commit(su32(&bars.vempty));
@@ -849,7 +709,7 @@ bool attn_tc8_supported(const lc_attn_args& a) {
   return a.out_fmt == LC_FMT_BF16 || a.out_fmt == LC_FMT_F32;
 }
 
-// Decode splits the keys of each (query, head group) over up to 148 / CTAs splits.  A
+// Decode splits the keys of each (query, head group) over up to SMs / CTAs splits.  A
 // window tile costs about two entry tiles (72 KB of BF16 rows against 40 KB, plus its
 // conversion in place), so when the window tiles fit one split that is no longer than the
 // entry splits, they get a split of their own.
@@ -860,8 +720,9 @@ static AttnTc8Geom tc8_geometry(const lc_attn_args& a, bool sparse, bool decode)
   const int tiles = (ns + kTK - 1) / kTK;
   g.sps = tiles * kTK;
   const int ctas = a.n_q * (a.dims.H / kNR);
-  if (decode && ctas < 148) {
-    const int n = max(1, min(148 / max(ctas, 1), tiles));
+  const int n_sm = sm_count();
+  if (decode && ctas < n_sm) {
+    const int n = max(1, min(n_sm / max(ctas, 1), tiles));
     const int per = (tiles + n - 1) / n;
     g.n_split = (tiles + per - 1) / per;
     g.sps = per * kTK;

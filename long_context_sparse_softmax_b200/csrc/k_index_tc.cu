@@ -30,6 +30,7 @@
 #include <cuda.h>
 
 #include "lc_internal.h"
+#include "lc_ptx.cuh"
 
 namespace lc {
 
@@ -45,72 +46,6 @@ constexpr long kSpin = 1L << 26;
 constexpr int kDBuf = 3;            // tensor-memory accumulators
 constexpr uint32_t kColSfa = 0;     // offsets past the accumulators
 constexpr uint32_t kColSfb = 16;
-
-__device__ __forceinline__ uint32_t su32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
-
-// K-major SWIZZLE_64B operand: 64-byte rows, 8-row groups 512 bytes apart
-__device__ __forceinline__ uint64_t sw64_desc(uint32_t addr) {
-  uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFF);
-  d |= static_cast<uint64_t>(1) << 16;               // LBO (unused by swizzled K-major)
-  d |= static_cast<uint64_t>(512 >> 4) << 32;        // SBO: next 8-row group
-  d |= static_cast<uint64_t>(1) << 46;               // descriptor version for sm_100
-  d |= static_cast<uint64_t>(4) << 61;               // layout: SWIZZLE_64B
-  return d;
-}
-// byte offset of 16-byte chunk c of row r in a SWIZZLE_64B tile (512-byte aligned base)
-__device__ __forceinline__ uint32_t sw64_off(int r, int c) { return r * 64 + ((c ^ ((r >> 1) & 3)) << 4); }
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile("{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-               : "=r"(done)
-               : "r"(bar), "r"(parity)
-               : "memory");
-  return done != 0;
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::
-          "r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n"); }
-
-__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
-               "r"(d));
-}
-
-// 32 columns of this warp's lanes, without waiting (tcgen05.wait::ld before use)
-__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
-      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-}
-
 
 struct IdxBars {
   uint64_t kfull[kStages];   // key tile (expect-tx arrival) and its scale words (32 arrivals) landed
@@ -202,9 +137,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;\n");
     asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tk)) : "memory");
   }
-  tc_fence_before();
+  fence_before();
   __syncthreads();
-  tc_fence_after();
+  fence_after();
   const uint32_t tm = s_tmem;
   const uint32_t col_sfa = kDBuf * N + kColSfa, col_sfb = kDBuf * N + kColSfb;
 
@@ -239,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t full = su32(&bars.kfull[s]);
         if (lane == 0) {
           mbar_expect_tx(full, kTileB);
-          tma_load_2d(su32(As + s * kTileB), &tk, 0, static_cast<int>(kbase + static_cast<int64_t>(t) * kKeys), full);
+          tma_tile2d(su32(As + s * kTileB), &tk, 0, static_cast<int>(kbase + static_cast<int64_t>(t) * kKeys), full);
         }
         *reinterpret_cast<uint4*>(SFs + s * kKeys + 4 * lane) = make_uint4(sfw[u][0], sfw[u][1], sfw[u][2], sfw[u][3]);
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // the tensor core reads them
@@ -259,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait(&bars.kfull[s], (it / kStages) & 1) &&
              (it < kDBuf || wait(&bars.dempty[slot], ((it / kDBuf) - 1) & 1));
         if (!ok) break;
-        tc_fence_after();
+        fence_after();
         // the tile's key scales: 32 rows of 16 bytes -> lanes 0..31 of every quadrant,
         // columns col_sfa + 8 sfs .. + 3
         {
@@ -328,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     asm volatile("cp.async.wait_all;\n" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-    tc_fence_before();
+    fence_before();
     mbar_arrive(su32(&bars.bfull));
     __syncwarp();
 
@@ -343,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto epilogue = [&](int u) -> bool {
       const int slot = u % kDBuf;
       if (!__all_sync(0xffffffffu, wait(&bars.dfull[slot], (u / kDBuf) & 1))) return false;
-      tc_fence_after();
+      fence_after();
       const int j = (t_begin + u) * kKeys + row;
 #pragma unroll
       for (int i = 0; i < QPC; ++i) {
@@ -353,8 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t v[64];
           const uint32_t ta = tm + lane_off + static_cast<uint32_t>(slot * N + i * H + h0);
           const int nh = min(64, H - h0);
-          tmem_ld32_async(ta, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-          if (nh > 32) tmem_ld32_async(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+          if (nh > 32) tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
           asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 #pragma unroll
           for (int k = 0; k < 64; ++k)
@@ -366,22 +301,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float s = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
         if (j < s_nv[i]) a.scores[static_cast<int64_t>(s_q[i]) * a.score_stride + j] = s;
       }
-      tc_fence_before();
+      fence_before();
       mbar_arrive(su32(&bars.dempty[slot]));
       return true;
     };
     for (int u = 0; weights_ok && u < n_tiles; ++u)
       if (!epilogue(u)) break;
   }
-  tc_fence_before();
+  fence_before();
   __syncthreads();
-  tc_fence_after();
+  fence_after();
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tm), "r"(tmem_cols));
-}
-
-bool index_tc_supported(const lc_index_args& a) {
-  return a.fmt == LC_IDX_MXFP4 && a.d_I == kDI && a.H_I % 32 == 0 && a.H_I <= 128 && a.n_keys > 0 &&
-         a.n_keys < (int64_t{1} << 31) && reinterpret_cast<uintptr_t>(a.k) % 16 == 0;
 }
 
 namespace {
@@ -429,7 +359,7 @@ cudaError_t launch_index_tc(const lc_index_args& a, bool decode, cudaStream_t st
   int tpc = tiles;
   if (decode) {
     // split each query's keys so that the CTAs fill the SMs once
-    const int want = max(1, (per_sm * 148) / n_qc);
+    const int want = max(1, (per_sm * sm_count()) / n_qc);
     tpc = max(4, (tiles + want - 1) / want);
   } else {
     tpc = max(1, min(tiles, 32));

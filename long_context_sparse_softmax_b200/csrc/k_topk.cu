@@ -33,8 +33,11 @@ constexpr int kBins = 2048;
 constexpr int kMaxCluster = 8;
 constexpr int kCand = kBins;          // candidates gathered after the first pass, at most
 
+// Order-preserving key of a score: larger scores get larger keys.  -0.0 maps to the key
+// of +0.0, since the two compare equal (ties between them go to the lower index).
 __device__ __forceinline__ uint32_t order_key(float f) {
-  const uint32_t u = __float_as_uint(f);
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
@@ -455,7 +458,7 @@ cudaError_t launch_topk(const lc_topk_args& a, bool decode, cudaStream_t st) {
   // and at least the one whose segments fit the key cache
   int C = 1;
   while (C < kMaxCluster &&
-         (static_cast<int64_t>(a.n_q) * 2 * C <= 148 || (a.max_ent + C - 1) / C > kRowCache))
+         (static_cast<int64_t>(a.n_q) * 2 * C <= sm_count() || (a.max_ent + C - 1) / C > kRowCache))
     C <<= 1;
   const int segl = ((a.max_ent + C - 1) / C + 3) & ~3;
   const int use_cache = segl <= kRowCache ? 1 : 0;

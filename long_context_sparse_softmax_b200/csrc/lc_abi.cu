@@ -1,8 +1,26 @@
 // C ABI of the CSA / HCA attention library: host-side validation, then one launch (or a
 // short fixed sequence of launches) on the caller's stream.  See include/lc.h.
+#include <atomic>
 #include <cstdint>
 
 #include "lc_internal.h"
+
+namespace lc {
+
+int sm_count() {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    cache[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+}  // namespace lc
 
 namespace {
 
@@ -78,7 +96,8 @@ lc_status index_scores(const lc_index_args* a, void* stream, bool decode) {
   if (a->fmt == LC_IDX_F32) {
     if (a->d_I < 4 || a->d_I % 4 || a->d_I > 256 || a->H_I * a->d_I > 16384) return LC_ERR_UNSUPPORTED;
   } else if (a->fmt == LC_IDX_MXFP4) {
-    if ((a->d_I != 64 && a->d_I != 128 && a->d_I != 256) || a->H_I % 8 || a->H_I > 64) return LC_ERR_UNSUPPORTED;
+    // the tensor-core kernel: 128 dims (two K = 64 block-scaled MMAs), 32 or 64 heads
+    if (a->d_I != 128 || (a->H_I != 32 && a->H_I != 64)) return LC_ERR_UNSUPPORTED;
   } else {
     return LC_ERR_ARG;
   }
@@ -88,7 +107,8 @@ lc_status index_scores(const lc_index_args* a, void* stream, bool decode) {
   if (a->n_q == 0 || a->max_ent == 0) return LC_OK;
   LC_TRY(check_batch(a->batch, true, false));
   if (!a->q || !a->k || !a->w || !a->scores) return LC_ERR_ARG;
-  if (a->fmt == LC_IDX_MXFP4 && (!a->q_scale || !a->k_scale || a->n_keys < 1)) return LC_ERR_ARG;
+  if (a->fmt == LC_IDX_MXFP4 && (!a->q_scale || !a->k_scale || a->n_keys < 1 || a->n_keys >= (int64_t{1} << 31)))
+    return LC_ERR_ARG;
   if (a->fmt == LC_IDX_MXFP4 && ((reinterpret_cast<uintptr_t>(a->q_scale) | reinterpret_cast<uintptr_t>(a->k_scale)) & 3u))
     return LC_ERR_ALIGN;
   if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->scores)) return LC_ERR_ALIGN;
@@ -114,7 +134,7 @@ lc_status attn(const lc_attn_args* a, void* stream, bool sparse, bool decode) {
   if (a->out_fmt != LC_FMT_F32 && a->out_fmt != LC_FMT_BF16) return LC_ERR_ARG;
   if (sparse && a->k < 1) return LC_ERR_ARG;
   if (decode && a->n_q != a->batch.num_seqs) return LC_ERR_ARG;
-  if (a->impl < LC_IMPL_AUTO || a->impl > LC_IMPL_TC_F16) return LC_ERR_ARG;
+  if (a->impl != LC_IMPL_AUTO && a->impl != LC_IMPL_TC && a->impl != LC_IMPL_REF) return LC_ERR_ARG;
   if (!lc::attn_impl_ok(*a)) return LC_ERR_UNSUPPORTED;
   if (a->n_q == 0) return LC_OK;
   LC_TRY(check_rows(a->q, a->dims, true));

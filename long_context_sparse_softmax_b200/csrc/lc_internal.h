@@ -7,16 +7,15 @@
 
 namespace lc {
 
+// Streaming multiprocessors of the current device (queried once per device; 148 on B200).
+int sm_count();
+
 cudaError_t launch_qk_prep(const lc_qk_prep_args& a, cudaStream_t st);
 cudaError_t launch_compress(const lc_compress_args& a, bool per_cta, cudaStream_t st);
 cudaError_t launch_index_scores(const lc_index_args& a, bool decode, cudaStream_t st);
 cudaError_t launch_topk(const lc_topk_args& a, bool decode, cudaStream_t st);
 cudaError_t launch_attn(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st);
 size_t attn_workspace_bytes(const lc_attn_args& a, bool sparse, bool decode);
-bool attn_mma_supported(const lc_attn_args& a);
-size_t attn_mma_workspace(const lc_attn_args& a, bool sparse, bool decode);
-cudaError_t launch_attn_mma(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st);
-bool index_tc_supported(const lc_index_args& a);
 bool attn_tc_supported(const lc_attn_args& a);
 int attn_impl(const lc_attn_args& a);
 bool attn_impl_ok(const lc_attn_args& a);

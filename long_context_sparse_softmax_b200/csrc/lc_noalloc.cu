@@ -50,11 +50,13 @@ size_t lc_csa_sparse_attn_decode_static_capacity(void) { return kStaticScratchBy
 
 lc_status lc_csa_sparse_attn_decode_static(const lc_attn_args* a, void* stream) {
   if (!a) return LC_ERR_ARG;
-  const size_t need = lc::attn_workspace_bytes(*a, true, true);
-  if (need > kStaticScratchBytes) return LC_ERR_TOO_LARGE;  // checked before touching the device
+  // the caller's workspace fields are ignored; the kernel choice (and so the scratch it
+  // needs) is made for the 256-byte-aligned array the call will pass
   lc_attn_args b = *a;
   b.workspace = nullptr;
   b.workspace_bytes = 0;
+  const size_t need = lc::attn_workspace_bytes(b, true, true);
+  if (need > kStaticScratchBytes) return LC_ERR_TOO_LARGE;  // checked before touching the device
   if (need > 0) {
     void* p = nullptr;
     const lc_status s = scratch_address(&p);

@@ -25,7 +25,9 @@ def test_reference_arm_prints_the_contract_line():
     assert d["data"] == "synthetic"
     assert d["config"]["workload"] == bench.workload_config("csa_decode")["workload"]
     cb = d["cpu_baseline"]
-    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["host_cores"] >= 1 and cb["value"] == d["value"]
+    assert cb["sample"]
+    assert d["native_libs_loaded"] == [], "the oracle arm must not load the GPU library"
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0

@@ -13,7 +13,6 @@ def test_tensor_peak_factors_follow_the_operand_types():
     assert bench.tensor_mix("0:index", csa_p)[0] == 4.0
     # E4M3 scores + F16 P V: half the flops at 2x, half at 1x
     assert bench.tensor_mix("0:attn", csa_p)[0] == pytest.approx(4.0 / 3.0)
-    assert bench.tensor_mix("0:attn", csa_p, "tc16")[0] == 1.0  # every operand widened to F16
     assert bench.tensor_mix("0:attn", hca_p)[0] == 1.0          # BF16 queries: the F16 kernel
     # a tensor-bound stage's roofline time uses that factor
     work = {"0:index": (1.0, 4.0e12)}

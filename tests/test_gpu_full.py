@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 
 from long_context_sparse_softmax_b200 import workloads as wl
-from tests.gpu_checks import check_decode, check_prefill
+from tests.gpu_checks import check_decode, check_prefill, save_report
 
 pytestmark = [pytest.mark.gpu]
 
@@ -27,19 +27,23 @@ def sample_queries(spec: wl.Spec, n: int = 64):
 
 def test_full_csa_decode_b32_128k():
     rep = check_decode(wl.CSA_DECODE)
+    save_report("full_csa_decode_b32_128k", rep)
     print(rep)
 
 
 def test_full_csa_prefill_64k():
     rep = check_prefill(wl.CSA_PREFILL, q_sel=sample_queries(wl.CSA_PREFILL))
+    save_report("full_csa_prefill_64k", rep)
     print(rep)
 
 
 def test_full_hca_prefill_1m():
     rep = check_prefill(wl.HCA_PREFILL, q_sel=sample_queries(wl.HCA_PREFILL))
+    save_report("full_hca_prefill_1m", rep)
     print(rep)
 
 
 def test_full_mixed_decode_1m():
-    print(check_decode(wl.MIXED_CSA))
-    print(check_decode(wl.MIXED_HCA))
+    rep = {"csa": check_decode(wl.MIXED_CSA), "hca": check_decode(wl.MIXED_HCA)}
+    save_report("full_mixed_decode_1m", rep)
+    print(rep)

@@ -92,3 +92,18 @@ def test_topk_mixed_and_ragged_rows():
     rows = [_rows(kinds[i % 4], n, rng) for i, n in enumerate(lens)]
     _check(rows, 512)
     _check(rows, 1024)
+
+
+def test_topk_signed_zeros_tie_by_index():
+    """-0.0 and +0.0 compare equal: at the threshold they are ties, taken by lower index
+    whatever their sign bits."""
+    rng = np.random.default_rng(13)
+    n = 5000
+    r = np.zeros(n, dtype=np.float32)
+    r[rng.random(n) < 0.5] = np.float32(-0.0)
+    pos = rng.choice(n, 200, replace=False)
+    r[pos] = np.abs(rng.standard_normal(200)).astype(np.float32) + 0.5
+    neg = rng.choice(np.setdiff1d(np.arange(n), pos), 300, replace=False)
+    r[neg] = -np.abs(rng.standard_normal(300)).astype(np.float32) - 0.5
+    assert np.signbit(r[r == 0]).any() and (~np.signbit(r[r == 0])).any()
+    _check([r, r[::-1].copy()], 512)
