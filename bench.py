@@ -144,6 +144,9 @@ def stage_work(spec, inp, run):
             work["index"] = (sum(v * (idx_key_b + 4) for v in nv) + B * idx_q_b,
                              sum(2 * v * s.H_I * s.d_I for v in nv))
             work["topk"] = (sum(4 * v for v in nv) + B * 4 * s.k, 0)
+            # fused: the keys and queries in, the selection out; no score matrix
+            work["index_topk"] = (sum(v * idx_key_b for v in nv) + B * idx_q_b + B * 4 * s.k,
+                                  sum(2 * v * s.H_I * s.d_I for v in nv))
             sel = K
         else:
             sel = nv
@@ -166,6 +169,8 @@ def stage_work(spec, inp, run):
             work["index"] = (n_c * idx_key_b + s.n_q * idx_q_b + int(nv.sum()) * 4,
                              int(nv.sum()) * 2 * s.H_I * s.d_I)
             work["topk"] = (int(nv.sum()) * 4 + s.n_q * 4 * s.k, 0)
+            work["index_topk"] = (n_c * idx_key_b + s.n_q * idx_q_b + s.n_q * 4 * s.k,
+                                  int(nv.sum()) * 2 * s.H_I * s.d_I)
             sel = K
         else:
             sel = nv
@@ -187,7 +192,7 @@ def tensor_mix(stage, spec, attn_impl="auto"):
     MXFP4 MMAs; the E4M3-score attention kernel does half its flops (S) in E4M3 and half
     (P V) in F16."""
     from long_context_sparse_softmax_b200 import workloads as wl
-    if stage.endswith("index") and spec.idx_fmt == wl.IDX_MXFP4:
+    if stage.split(":")[-1] in ("index", "index_topk") and spec.idx_fmt == wl.IDX_MXFP4:
         return TENSOR_RATIO["mxf4"], "MXFP4"
     if (stage.endswith("attn") and attn_impl in ("auto", "tc") and spec.q_fmt == wl.FMT_E4M3_BF16
             and spec.kv_fmt == wl.FMT_E4M3_BF16):
@@ -350,8 +355,11 @@ def run_lc(args):
     # the critical path: stages on the main stream (the side stages overlap them, and their
     # event times include the wait for SMs the critical path holds)
     crit_names = [f"{i}:{n}" for i, (_, _, r) in enumerate(runs) for part in r.dag()[1:] for n, _ in part]
-    # kernels per step: one per call, plus the combine kernel of a key-split attention
-    n_launch = len(stage_names) + sum(1 for (_, _, r) in runs if r.a_attn.workspace_bytes > 0)
+    # kernels per step: one per call, plus the combine kernel of an attention whose key
+    # splits leave partials in a workspace, plus the merge kernel of a fused index + top-k
+    # whose queries span several indexer CTAs (it then has a candidate workspace)
+    n_launch = len(stage_names) + sum(1 for (_, _, r) in runs if r.a_attn.workspace_bytes > 0) + \
+        sum(1 for (_, _, r) in runs if getattr(r, "fused", False) and r.a_index_topk.workspace_bytes > 0)
     # one stream per side stage: they share no buffers, so none waits for another
     side = [torch.cuda.Stream(dev, priority=0) for _ in range(3)]
 

@@ -238,6 +238,34 @@ lc_status lc_csa_topk_prefill(const lc_topk_args* a, void* stream);
 lc_status lc_csa_topk_decode(const lc_topk_args* a, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * csa_index_topk — the lightning indexer and the top-k selection fused: the same
+ * scores as csa_index_scores and the same selection as csa_topk (K = min(k, n_vis(p))
+ * largest, ties to the lower index, idx ascending and padded with -1, count[q] = K), but
+ * the score matrix is never written.  Pages: "解读 DeepSeek V4" CSA section (the indexer
+ * exists to pick the top-k entries); "DeepSeek-V4 论文分析" §5.3.
+ * Each indexer CTA keeps the scores of its key range on chip and selects its own top K
+ * exactly (every entry of the global top K is in the top K of its range); when a
+ * query's keys span several CTAs, a merge kernel selects the final K from the ranges'
+ * candidates.  The result is bit-identical to csa_index_scores followed by csa_topk.
+ * MXFP4 operands only (d_I = 128, H_I = 32 or 64); k <= 2048.  The workspace holds the
+ * candidates: lc_csa_index_topk_workspace_bytes(a) bytes, 16-byte aligned (0 when every
+ * query's keys fit one CTA).
+ * ------------------------------------------------------------------------------- */
+typedef struct lc_index_topk_args {
+  lc_index_args index;     /* scores and score_stride are ignored (nothing is written) */
+  int32_t k;               /* 1 .. 2048 */
+  int32_t reserved;
+  int32_t* idx;            /* [n_q, k] */
+  int32_t* count;          /* [n_q] or NULL */
+  void* workspace;
+  size_t workspace_bytes;
+} lc_index_topk_args;
+
+lc_status lc_csa_index_topk_prefill(const lc_index_topk_args* a, void* stream);
+lc_status lc_csa_index_topk_decode(const lc_index_topk_args* a, void* stream);
+size_t lc_csa_index_topk_workspace_bytes(const lc_index_topk_args* a, int32_t decode);
+
+/* ---------------------------------------------------------------------------------
  * csa_sparse_attn / hca_attn — for each query at p and head h, softmax attention over
  *   CSA: the selected entries idx[q, :] (-1 skipped), HCA: every visible entry,
  * joined with the window rows for positions max(0, p-W+1) .. p and the sink logit
@@ -335,7 +363,8 @@ const char* lc_version(void);
 const char* lc_status_string(lc_status s);
 /* sizeof of the args structs, for bindings to check their mirrors:
  * 0 lc_rows, 1 lc_dims, 2 lc_batch, 3 lc_qk_prep_args, 4 lc_compress_args,
- * 5 lc_index_args, 6 lc_topk_args, 7 lc_attn_args; other values return 0. */
+ * 5 lc_index_args, 6 lc_topk_args, 7 lc_attn_args, 8 lc_index_topk_args; other values
+ * return 0. */
 size_t lc_struct_size(int32_t which);
 
 #ifdef __cplusplus

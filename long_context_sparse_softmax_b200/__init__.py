@@ -73,6 +73,11 @@ class TopkArgs(ctypes.Structure):
                 ("idx", c_void_p), ("count", c_void_p), ("status", c_void_p)]
 
 
+class IndexTopkArgs(ctypes.Structure):
+    _fields_ = [("index", IndexArgs), ("k", c_int32), ("reserved", c_int32), ("idx", c_void_p), ("count", c_void_p),
+                ("workspace", c_void_p), ("workspace_bytes", c_size_t)]
+
+
 class AttnArgs(ctypes.Structure):
     _fields_ = [("dims", Dims), ("n_q", c_int32), ("k", c_int32), ("m", c_int32), ("W", c_int32), ("W_x", c_int32),
                 ("max_ent", c_int32), ("scale", c_float), ("out_fmt", c_int32), ("q", Rows), ("ent", Rows),
@@ -85,7 +90,7 @@ class AttnArgs(ctypes.Structure):
 LC_IMPL_AUTO, LC_IMPL_TC, LC_IMPL_REF = 0, 2, 3
 
 
-STRUCTS = [Rows, Dims, Batch, QkPrepArgs, CompressArgs, IndexArgs, TopkArgs, AttnArgs]
+STRUCTS = [Rows, Dims, Batch, QkPrepArgs, CompressArgs, IndexArgs, TopkArgs, AttnArgs, IndexTopkArgs]
 
 ENTRY_POINTS = {
     "lc_qk_prep_prefill": QkPrepArgs, "lc_qk_prep_decode": QkPrepArgs,
@@ -93,11 +98,13 @@ ENTRY_POINTS = {
     "lc_hca_compress_prefill": CompressArgs, "lc_hca_compress_decode": CompressArgs,
     "lc_csa_index_scores_prefill": IndexArgs, "lc_csa_index_scores_decode": IndexArgs,
     "lc_csa_topk_prefill": TopkArgs, "lc_csa_topk_decode": TopkArgs,
+    "lc_csa_index_topk_prefill": IndexTopkArgs, "lc_csa_index_topk_decode": IndexTopkArgs,
     "lc_csa_sparse_attn_prefill": AttnArgs, "lc_csa_sparse_attn_decode": AttnArgs,
     "lc_hca_attn_prefill": AttnArgs, "lc_hca_attn_decode": AttnArgs,
     "lc_csa_sparse_attn_decode_static": AttnArgs,
 }
-HELPERS = ["lc_csa_sparse_attn_workspace_bytes", "lc_hca_attn_workspace_bytes", "lc_version",
+HELPERS = ["lc_csa_sparse_attn_workspace_bytes", "lc_hca_attn_workspace_bytes", "lc_csa_index_topk_workspace_bytes",
+           "lc_version",
            "lc_status_string", "lc_struct_size", "lc_csa_sparse_attn_decode_static_capacity"]
 
 
@@ -113,6 +120,8 @@ def _load() -> ctypes.CDLL:
         fn = getattr(so, name)
         fn.argtypes = [ctypes.POINTER(AttnArgs)]
         fn.restype = c_size_t
+    so.lc_csa_index_topk_workspace_bytes.argtypes = [ctypes.POINTER(IndexTopkArgs), c_int32]
+    so.lc_csa_index_topk_workspace_bytes.restype = c_size_t
     so.lc_csa_sparse_attn_decode_static_capacity.restype = c_size_t
     so.lc_version.restype = ctypes.c_char_p
     so.lc_status_string.argtypes = [c_int32]
@@ -174,6 +183,10 @@ def lc_csa_sparse_attn_workspace_bytes(args: AttnArgs) -> int:
 
 def lc_hca_attn_workspace_bytes(args: AttnArgs) -> int:
     return int(load().lc_hca_attn_workspace_bytes(ctypes.byref(args)))
+
+
+def lc_csa_index_topk_workspace_bytes(args: IndexTopkArgs, decode: bool) -> int:
+    return int(load().lc_csa_index_topk_workspace_bytes(ctypes.byref(args), 1 if decode else 0))
 
 
 def lc_csa_sparse_attn_decode_static_capacity() -> int:

@@ -149,18 +149,13 @@ bool attn_impl_ok(const lc_attn_args& a) { return attn_impl(a) == LC_IMPL_REF ||
 
 size_t attn_workspace_bytes(const lc_attn_args& a, bool sparse, bool decode) {
   if (attn_impl(a) != LC_IMPL_TC) return 0;
-  if (a.impl == LC_IMPL_AUTO) {
-    // the choice between the two tcgen05 kernels may depend on buffer alignment, which
-    // the caller may not have fixed yet: the larger of the two
-    lc_attn_args t = a;
-    t.out = nullptr;
-    t.workspace = nullptr;
-    if (!tc_any(t)) return 0;
-    const size_t w0 = attn_tc_workspace(a, sparse, decode), w1 = attn_tc8_workspace(a, sparse, decode);
-    return w0 > w1 ? w0 : w1;
-  }
-  if (attn_tc8_supported(a)) return attn_tc8_workspace(a, sparse, decode);
-  return attn_tc_supported(a) ? attn_tc_workspace(a, sparse, decode) : 0;
+  // the formats decide between the two tcgen05 kernels (buffer alignment is validated
+  // separately), so the size is known before the buffers are
+  lc_attn_args t = a;
+  t.out = nullptr;
+  t.workspace = nullptr;
+  if (attn_tc8_supported(t)) return attn_tc8_workspace(a, sparse, decode);
+  return attn_tc_supported(t) ? attn_tc_workspace(a, sparse, decode) : 0;
 }
 
 cudaError_t launch_attn(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st) {

@@ -31,8 +31,12 @@
 // LC_DEV_TIMEOUT and an abort flag that stops the others at their next wait.
 #include <cuda.h>
 
+#include <cooperative_groups.h>
+
 #include "lc_internal.h"
 #include "lc_ptx.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace lc {
 
@@ -146,7 +150,11 @@ struct AttnTc8Geom {
   int n_split;
   int sps;       // slots per split, multiple of kTK
   int win_own;   // 1: the last split takes every window slot, the others the entry slots
+  int cluster;   // 1: the splits of a (query, head group) are one thread-block cluster and
+                 // merge their partial results over distributed shared memory
 };
+
+constexpr int kMaxClusterSplits = 8;
 
 // grid: one CTA per (query, head group, key split), the split index fastest; 320 threads.
 // Partial results of split s go to ws_o rows s * n_q * H + q * H + h (576 floats each) and
@@ -169,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ __align__(8) Bars bars;
+  __shared__ float2 s_ml[kNR];  // cluster merge: this split's (max, sum) per head
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_hg = a.dims.H / kNR;
@@ -644,7 +653,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     good = !named_bar_or(1, 128, !good);
     fence_after();
     const float l_row = l_sum + __shfl_xor_sync(0xffffffffu, l_sum, 16);
-    if (hf == 0) {
+    if (geo.cluster) {
+      // this split's (max, sum) per head, for the merge over the cluster below
+      if (hf == 0) s_ml[r] = make_float2(good ? m_ref : -INFINITY, good ? l_row : 0.f);
+    } else if (hf == 0) {
       const int h = hg * kNR + r;
       if (geo.n_split == 1) {
         const float sk = __ldg(a.sink + h) * 1.4426950408889634f;
@@ -660,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     named_bar(1, 128);
-    if (good) {
+    if (good && !geo.cluster) {
       // O^T (dims on tensor-memory lanes, heads on columns) straight to global memory:
       // for each head a warp writes 32 consecutive dims, 128 bytes in FP32
       const bool f32 = geo.n_split > 1 || a.out_fmt == LC_FMT_F32;
@@ -692,6 +704,80 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
+  if (geo.cluster) {
+    // ================= merge of the key splits over the cluster (every thread) =================
+    // M = max(sink, max_s m_s), Z = e^(sink - M) + sum_s l_s e^(m_s - M) per head; split s
+    // scales its O by e^(m_s - M) / Z into its own shared memory; then split s sums dims
+    // [d0, d1) of every split's scaled O, in split order, and writes them out.
+    cg::cluster_group cl = cg::this_cluster();
+    fence_before();
+    cl.sync();  // every split's (m, l) is published; every role of every split is done
+    fence_after();
+    float* Osm = reinterpret_cast<float*>(smem + kOffRaw);  // [kNR heads][kD dims]
+    if (warp < 4) {
+      const int r = warp * 16 + (lane & 15);
+      if ((lane >> 4) == 0) {
+        const float sk = __ldg(a.sink + hg * kNR + r) * 1.4426950408889634f;
+        float M = sk;
+        for (int sp = 0; sp < geo.n_split; ++sp) M = fmaxf(M, cl.map_shared_rank(s_ml, sp)[r].x);
+        float Z = exp2f(sk - M);
+        for (int sp = 0; sp < geo.n_split; ++sp) {
+          const float2 v = cl.map_shared_rank(s_ml, sp)[r];
+          if (v.x != -INFINITY) Z = fmaf(v.y, exp2f(v.x - M), Z);
+        }
+        const float mo = s_ml[r].x;
+        s_f[r] = mo == -INFINITY ? 0.f : exp2f(mo - M) / Z;
+        if (split == 0 && a.lse) a.lse[row0 + r] = (M + log2f(Z)) * 0.6931471805599453f;
+      }
+      named_bar(1, 128);
+      const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+#pragma unroll 1
+      for (int c = 0; c < 5; ++c) {
+        const int dim = c < 4 ? c * 128 + warp * 32 + lane : (lane < 16 ? 512 + warp * 16 + lane : -1);
+        uint32_t ov[kNR];
+        if (n_tiles > 0) {
+          tmem_ld32(tm + lane_off + kColO + c * kNR, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
+          tmem_ld32(tm + lane_off + kColO + c * kNR + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < kNR; ++i) ov[i] = 0;
+        }
+        if (dim < 0) continue;
+#pragma unroll
+        for (int i = 0; i < kNR; ++i) Osm[i * kD + dim] = __uint_as_float(ov[i]) * s_f[i];
+      }
+    }
+    cl.sync();  // every split's scaled O is in its shared memory
+    const int dpc = ((kD + geo.n_split - 1) / geo.n_split + 3) & ~3;
+    const int d0 = min(kD, split * dpc), d1 = min(kD, d0 + dpc);
+    const int nq4 = (d1 - d0) / 4;
+    const float* src[kMaxClusterSplits];
+#pragma unroll
+    for (int sp = 0; sp < kMaxClusterSplits; ++sp) src[sp] = sp < geo.n_split ? cl.map_shared_rank(Osm, sp) : Osm;
+    for (int it = tid; it < kNR * nq4; it += kThreads) {
+      const int h = it / nq4, d = d0 + 4 * (it % nq4);
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int sp = 0; sp < kMaxClusterSplits; ++sp)
+        if (sp < geo.n_split) {
+          const float4 v = *reinterpret_cast<const float4*>(src[sp] + h * kD + d);
+          o.x += v.x;
+          o.y += v.y;
+          o.z += v.z;
+          o.w += v.w;
+        }
+      const int64_t e = (row0 + h) * kD + d;
+      if (a.out_fmt == LC_FMT_F32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(a.out) + e) = o;
+      } else {
+        const uint32_t lo = static_cast<uint32_t>(f32_to_bf16_bits(o.x)) | (static_cast<uint32_t>(f32_to_bf16_bits(o.y)) << 16);
+        const uint32_t hi = static_cast<uint32_t>(f32_to_bf16_bits(o.z)) | (static_cast<uint32_t>(f32_to_bf16_bits(o.w)) << 16);
+        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + e) = make_uint2(lo, hi);
+      }
+    }
+    cl.sync();  // no split leaves while another still reads its shared memory
+  }
   fence_before();
   __syncthreads();
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tm), "r"(kTmemCols));
@@ -713,8 +799,10 @@ bool attn_tc8_supported(const lc_attn_args& a) {
 // window tile costs about two entry tiles (72 KB of BF16 rows against 40 KB, plus its
 // conversion in place), so when the window tiles fit one split that is no longer than the
 // entry splits, they get a split of their own.
+// Up to kMaxClusterSplits splits form one thread-block cluster and merge over distributed
+// shared memory; more splits (few queries) leave partials for k_attn_combine.
 static AttnTc8Geom tc8_geometry(const lc_attn_args& a, bool sparse, bool decode) {
-  AttnTc8Geom g{1, 0, 0};
+  AttnTc8Geom g{1, 0, 0, 0};
   const int ne = sparse ? a.k : a.max_ent;
   const int ns = max(ne + a.W, 1);
   const int tiles = (ns + kTK - 1) / kTK;
@@ -737,13 +825,14 @@ static AttnTc8Geom tc8_geometry(const lc_attn_args& a, bool sparse, bool decode)
         g.n_split = (te + per_e - 1) / per_e + 1;
       }
     }
+    g.cluster = g.n_split > 1 && g.n_split <= kMaxClusterSplits;
   }
   return g;
 }
 
 size_t attn_tc8_workspace(const lc_attn_args& a, bool sparse, bool decode) {
   const AttnTc8Geom g = tc8_geometry(a, sparse, decode);
-  if (g.n_split <= 1) return 0;
+  if (g.n_split <= 1 || g.cluster) return 0;
   const size_t rows = static_cast<size_t>(a.n_q) * a.dims.H * g.n_split;
   return rows * kD * sizeof(float) + rows * 2 * sizeof(float);
 }
@@ -783,7 +872,7 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType ty, const void* base, int64_t 
 cudaError_t launch_attn_tc8(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st, int* n_split_out) {
   if (!encode8()) return cudaErrorNotSupported;
   const AttnTc8Geom g = tc8_geometry(a, sparse, decode);
-  *n_split_out = g.n_split;
+  *n_split_out = g.cluster ? 1 : g.n_split;  // a cluster merges its splits itself
   const int64_t qrows = static_cast<int64_t>(a.n_q) * a.dims.H;
   CUtensorMap tqn, tqr, tkn, tkr, twin;
   if (!make_map(&tqn, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q.x, qrows, kDN, 1, 128, kNR) ||
@@ -798,14 +887,25 @@ cudaError_t launch_attn_tc8(const lc_attn_args& a, bool sparse, bool decode, cud
     twin = tkr;  // no window tiles: never read
   }
   cudaFuncSetAttribute(k_attn_tc8, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
-  float* ws_o = static_cast<float*>(a.workspace);
+  float* ws_o = g.cluster ? nullptr : static_cast<float*>(a.workspace);
   float* ws_ml = nullptr;
-  if (g.n_split > 1) ws_ml = ws_o + static_cast<size_t>(a.n_q) * a.dims.H * g.n_split * kD;
+  if (g.n_split > 1 && !g.cluster) ws_ml = ws_o + static_cast<size_t>(a.n_q) * a.dims.H * g.n_split * kD;
   const int64_t ctas = static_cast<int64_t>(a.n_q) * (a.dims.H / kNR) * g.n_split;
   if (ctas > 0x7fffffff) return cudaErrorInvalidConfiguration;
-  k_attn_tc8<<<static_cast<unsigned>(ctas), kThreads, kSmem, st>>>(tqn, tqr, tkn, tkr, twin, a, sparse ? 1 : 0, decode ? 1 : 0, g, ws_o,
-                                                                  ws_ml);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = g.cluster ? g.n_split : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g.cluster ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_attn_tc8, tqn, tqr, tkn, tkr, twin, a, sparse ? 1 : 0, decode ? 1 : 0, g, ws_o,
+                            ws_ml);
 }
 
 }  // namespace lc

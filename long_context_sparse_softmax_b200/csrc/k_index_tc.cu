@@ -27,6 +27,18 @@
 //
 // The roles meet only at mbarriers.  Every wait is bounded: after ~2^26 polls a role
 // records LC_DEV_TIMEOUT in the status word and sets an abort flag that stops the others.
+//
+// Fused selection (SELECT, lc_csa_index_topk_*): the epilogue keeps the scores of the
+// CTA's key range in shared memory instead of writing them out, and after the last tile
+// its 128 threads select the range's top K = min(k, keys in range) exactly, ties to the
+// lower index: radix passes of 11 bits over the order-preserving keys (relative to the
+// range's smallest) find the K-th largest key T and how many keys equal to T to take;
+// keys equal to T are ranked in index order with warp ballots.  The selection is a
+// bitmap in index order.  With one CTA per query it is the answer (indices written
+// ascending); otherwise the CTA writes its K (key, index) candidates in index order and
+// k_topk_merge picks the final K among every range's candidates.  Every entry of the
+// query's top K is in the top K of its own range, so the result equals csa_topk on the
+// scores this kernel computes.
 #include <cuda.h>
 
 #include "lc_internal.h"
@@ -47,6 +59,9 @@ constexpr int kDBuf = 3;            // tensor-memory accumulators
 constexpr uint32_t kColSfa = 0;     // offsets past the accumulators
 constexpr uint32_t kColSfb = 16;
 
+constexpr int kSelMaxTiles = 64;    // tiles per CTA in the fused-selection mode (32 KB of scores)
+constexpr int kSelBins = 2048;
+
 struct IdxBars {
   uint64_t kfull[kStages];   // key tile (expect-tx arrival) and its scale words (32 arrivals) landed
   uint64_t kempty[kStages];  // MMAs of the tile done (commit)
@@ -56,15 +71,55 @@ struct IdxBars {
   uint64_t fin;              // every MMA complete (commit)
 };
 
+// Order-preserving key of a score: larger scores get larger keys; -0.0 maps to +0.0's key.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive prefix of v over the 128 epilogue threads in row order (row = quad * 32 + lane),
+// and the total.  Uses named barrier 1; tmp holds 4 ints.
+__device__ __forceinline__ int scan128(int v, int quad, int lane, int* tmp, int* total) {
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) tmp[quad] = incl;
+  named_bar(1, 128);
+  int before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    before += w < quad ? tmp[w] : 0;
+    all += tmp[w];
+  }
+  named_bar(1, 128);
+  *total = all;
+  return before + incl - v;
+}
+
 }  // namespace
+
+// Outputs of the fused selection (k > 0).
+struct IdxSelect {
+  int k;            // 0: write the score matrix instead
+  int n_chunks;     // key-range CTAs per query (gridDim.y)
+  uint2* cand;      // n_chunks > 1: [n_q][n_chunks][k] (order key, entry index)
+  int* cand_cnt;    // n_chunks > 1: [n_q][n_chunks] candidates written
+  int32_t* idx;     // n_chunks == 1: [n_q][k]
+  int32_t* count;   // n_chunks == 1: [n_q] or null
+};
 
 // grid: (query chunks of QPC queries, key-range chunks); 192 threads.
 // Tensor memory: accumulators at columns [k N, (k + 1) N), k < 3; key scales at 3N + {0, 8};
 // query scales at 3N + 16 (N / 32 columns).
-template <int QPC>
+template <int QPC, bool SELECT>
 __global__ void __launch_bounds__(kThreads, 1)
     k_index_tc(const __grid_constant__ CUtensorMap tk, lc_index_args a, int tiles_per_cta, uint32_t tmem_cols,
-               int decode) {
+               int decode, IdxSelect sel) {
+  static_assert(!SELECT || QPC == 1, "fused selection takes one query per CTA");
   extern __shared__ __align__(1024) uint8_t smem[];
   const int H = a.H_I;
   const int N = QPC * H;
@@ -72,6 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* Bs = As + kStages * kTileB;                              // [N rows][64 B], SWIZZLE_64B
   uint32_t* SFs = reinterpret_cast<uint32_t*>(Bs + N * kRowB);      // [kStages][128] key scale words
   float* ws = reinterpret_cast<float*>(SFs + kStages * kKeys);      // [N] head weights
+  float* sc = ws + N;                                               // SELECT: [tiles_per_cta][128] scores
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ __align__(8) IdxBars bars;
@@ -103,7 +159,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = 0; i < QPC; ++i) nv_max = max(nv_max, s_nv[i]);
   const int t_begin = blockIdx.y * tiles_per_cta;
   const int t_end = min(t_begin + tiles_per_cta, (nv_max + kKeys - 1) / kKeys);
-  if (t_begin >= t_end) return;  // uniform over the CTA: nothing allocated yet
+  if (t_begin >= t_end) {  // uniform over the CTA: nothing allocated yet
+    if constexpr (SELECT) {
+      // an empty key range: no candidates (or, alone, an empty selection)
+      if (sel.n_chunks > 1) {
+        if (tid == 0) sel.cand_cnt[static_cast<int64_t>(qa) * sel.n_chunks + blockIdx.y] = 0;
+      } else {
+        for (int i = tid; i < sel.k; i += kThreads) sel.idx[static_cast<int64_t>(qa) * sel.k + i] = -1;
+        if (tid == 0 && sel.count) sel.count[qa] = 0;
+      }
+    }
+    return;
+  }
   const int n_tiles = t_end - t_begin;
 
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -299,7 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         const float s = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-        if (j < s_nv[i]) a.scores[static_cast<int64_t>(s_q[i]) * a.score_stride + j] = s;
+        if constexpr (SELECT) sc[u * kKeys + row] = s;
+        else if (j < s_nv[i]) a.scores[static_cast<int64_t>(s_q[i]) * a.score_stride + j] = s;
       }
       fence_before();
       mbar_arrive(su32(&bars.dempty[slot]));
@@ -307,6 +375,137 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     for (int u = 0; weights_ok && u < n_tiles; ++u)
       if (!epilogue(u)) break;
+
+    if constexpr (SELECT) {
+      // ================= the range's top K (128 threads; the key ring is idle) =================
+      __shared__ uint32_t s_rng[2][4];
+      __shared__ int s_tmp[4];
+      __shared__ int s_pick[2];
+      __shared__ int s_wcnt[kSelMaxTiles][4];
+      uint32_t* hist = reinterpret_cast<uint32_t*>(As);   // [kSelBins]
+      uint32_t* bits = hist + kSelBins;                   // [n_tiles * 4] selection words
+      const int q = s_q[0];
+      const int jbase = t_begin * kKeys;
+      const int n_valid = max(0, min(s_nv[0] - jbase, n_tiles * kKeys));
+      const int K = min(sel.k, n_valid);
+      auto valid = [&](int u) { return u * kKeys + row < n_valid; };
+      // key range of the valid scores
+      uint32_t kmin = 0xffffffffu, kmax = 0u;
+      for (int u = 0; u < n_tiles; ++u)
+        if (valid(u)) {
+          const uint32_t key = order_key(sc[u * kKeys + row]);
+          kmin = min(kmin, key);
+          kmax = max(kmax, key);
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+      }
+      if (lane == 0) {
+        s_rng[0][quad] = kmin;
+        s_rng[1][quad] = kmax;
+      }
+      named_bar(1, 128);
+      const uint32_t umin = min(min(s_rng[0][0], s_rng[0][1]), min(s_rng[0][2], s_rng[0][3]));
+      const uint32_t umax = max(max(s_rng[1][0], s_rng[1][1]), max(s_rng[1][2], s_rng[1][3]));
+      // radix passes over rel = key - umin from the top, 11 bits at a time: pfx holds the
+      // bits of the K-th largest rel found so far, rem the keys still to take inside the
+      // bin they select
+      const bool take_all = K == n_valid;
+      uint32_t pfx = 0;
+      int rem = K;
+      int shift = take_all ? 0 : 32 - __clz(static_cast<int>(umax - umin));
+#pragma unroll 1
+      while (shift > 0) {
+        const int w = min(11, shift);
+        const int hi = shift;
+        shift -= w;
+        const uint32_t bmask = (1u << w) - 1u;
+        for (int i = row; i < kSelBins; i += 128) hist[i] = 0;
+        named_bar(1, 128);
+        for (int u = 0; u < n_tiles; ++u)
+          if (valid(u)) {
+            const uint32_t rel = order_key(sc[u * kKeys + row]) - umin;
+            const uint32_t top = hi >= 32 ? 0u : rel >> hi;
+            if (top == pfx) atomicAdd(&hist[(rel >> shift) & bmask], 1u);
+          }
+        named_bar(1, 128);
+        // descending: thread `row` owns bins 2047 - 16 row - i, i < 16
+        int c[16], sum = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          c[i] = static_cast<int>(hist[kSelBins - 1 - 16 * row - i]);
+          sum += c[i];
+        }
+        int tot;
+        int run = scan128(sum, quad, lane, s_tmp, &tot);
+        if (run < rem && run + sum >= rem) {
+#pragma unroll 1
+          for (int i = 0; i < 16; ++i) {
+            if (run + c[i] >= rem) {
+              s_pick[0] = kSelBins - 1 - 16 * row - i;
+              s_pick[1] = rem - run;
+              break;
+            }
+            run += c[i];
+          }
+        }
+        named_bar(1, 128);
+        pfx = (pfx << w) | static_cast<uint32_t>(s_pick[0]);
+        rem = s_pick[1];
+      }
+      const uint32_t T = umin + pfx;
+      // keys equal to T, ranked in index order (u, then row): per-tile warp counts first
+      for (int u = 0; u < n_tiles; ++u) {
+        const bool eq = !take_all && valid(u) && order_key(sc[u * kKeys + row]) == T;
+        const uint32_t bal = __ballot_sync(0xffffffffu, eq);
+        if (lane == 0) s_wcnt[u][quad] = __popc(bal);
+      }
+      named_bar(1, 128);
+      int eq_before = 0;
+      for (int u = 0; u < n_tiles; ++u) {
+        const bool v = valid(u);
+        const uint32_t key = v ? order_key(sc[u * kKeys + row]) : 0u;
+        const bool eq = !take_all && v && key == T;
+        // rank among the keys equal to T: earlier tiles, earlier quadrants, earlier lanes
+        int rank = eq_before + __popc(__ballot_sync(0xffffffffu, eq) & ((1u << lane) - 1u));
+#pragma unroll
+        for (int w = 0; w < 4; ++w) rank += w < quad ? s_wcnt[u][w] : 0;
+        const bool pick = v && (take_all || key > T || (eq && rank < rem));
+        const uint32_t word = __ballot_sync(0xffffffffu, pick);
+        if (lane == 0) bits[u * 4 + quad] = word;
+        eq_before += s_wcnt[u][0] + s_wcnt[u][1] + s_wcnt[u][2] + s_wcnt[u][3];
+      }
+      named_bar(1, 128);
+      // the selected keys in index order: word w holds keys jbase + 32 w .. + 31
+      const int n_words = n_tiles * 4;
+      const bool alone = sel.n_chunks == 1;
+      int32_t* out_idx = alone ? sel.idx + static_cast<int64_t>(q) * sel.k : nullptr;
+      uint2* out_c = alone ? nullptr : sel.cand + (static_cast<int64_t>(q) * sel.n_chunks + blockIdx.y) * sel.k;
+      int base = 0;
+      for (int w0 = 0; w0 < n_words; w0 += 128) {
+        const int w = w0 + row;
+        uint32_t word = w < n_words ? bits[w] : 0u;
+        int tot;
+        int pos = base + scan128(__popc(word), quad, lane, s_tmp, &tot);
+        while (word) {
+          const int bpos = __ffs(word) - 1;
+          word &= word - 1;
+          const int off = w * 32 + bpos;  // key u * 128 + row' of the range
+          if (alone) out_idx[pos] = jbase + off;
+          else out_c[pos] = make_uint2(order_key(sc[off]), static_cast<uint32_t>(jbase + off));
+          ++pos;
+        }
+        base += tot;
+      }
+      if (alone) {
+        for (int i = K + row; i < sel.k; i += 128) out_idx[i] = -1;
+        if (row == 0 && sel.count) sel.count[q] = K;
+      } else if (row == 0) {
+        sel.cand_cnt[static_cast<int64_t>(q) * sel.n_chunks + blockIdx.y] = K;
+      }
+    }
   }
   fence_before();
   __syncthreads();
@@ -334,46 +533,90 @@ EncodeTiled encode_tiled() {
 
 }  // namespace
 
-cudaError_t launch_index_tc(const lc_index_args& a, bool decode, cudaStream_t st) {
+// Launch shape of the indexer: one query per CTA, each query's keys split into ranges of
+// tpc tiles so that the CTAs fill the SMs once in decode (prefill: ranges of 32 tiles).
+IndexGeom index_geometry(const lc_index_args& a, bool decode, bool select) {
+  IndexGeom g{};
+  const int N = a.H_I;
+  g.tmem_cols = 32;
+  while (g.tmem_cols < static_cast<uint32_t>(kDBuf * N + 24)) g.tmem_cols <<= 1;
+  g.tiles = (a.max_ent + kKeys - 1) / kKeys;
+  const int per_sm = static_cast<int>(512 / g.tmem_cols);
+  if (decode) {
+    const int want = max(1, (per_sm * sm_count()) / max(a.n_q, 1));
+    g.tpc = max(4, (g.tiles + want - 1) / want);
+  } else {
+    g.tpc = max(1, min(g.tiles, 32));
+  }
+  if (select) g.tpc = min(g.tpc, kSelMaxTiles);
+  g.tpc = max(g.tpc, 1);
+  g.n_chunks = max(1, (g.tiles + g.tpc - 1) / g.tpc);
+  size_t sm = static_cast<size_t>(kStages) * kTileB + static_cast<size_t>(N) * kRowB + kStages * kKeys * 4 +
+              static_cast<size_t>(N) * 4 + 1024;
+  if (select) sm += static_cast<size_t>(g.tpc) * kKeys * 4;
+  // no more CTAs per SM than its 512 tensor-memory columns hold, so tcgen05.alloc never
+  // waits for another CTA
+  const size_t cap = 227 * 1024 / per_sm - 2048;
+  g.smem = sm < cap ? cap : sm;
+  return g;
+}
+
+namespace {
+
+bool make_key_map(CUtensorMap* tk, const lc_index_args& a) {
   const EncodeTiled enc = encode_tiled();
-  if (!enc) return cudaErrorNotSupported;
+  if (!enc) return false;
   // the key codes as a [n_keys, 64 B] tensor; 128-row boxes, 64-byte swizzle; rows past
   // n_keys read as zeros
-  CUtensorMap tk;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kRowB), static_cast<cuuint64_t>(a.n_keys)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kRowB)};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(kRowB), static_cast<cuuint32_t>(kKeys)};
   const cuuint32_t estr[2] = {1, 1};
-  if (enc(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a.k), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  const int H = a.H_I;
-  const int qpc = 1;  // three 64-column accumulators and the scales fit 256 columns: 2 CTAs per SM
-  const int N = qpc * H;
-  uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(kDBuf * N + 24)) cols <<= 1;
-  const int tiles = (a.max_ent + kKeys - 1) / kKeys;
-  const int n_qc = (a.n_q + qpc - 1) / qpc;
-  const int per_sm = static_cast<int>(512 / cols);
-  int tpc = tiles;
-  if (decode) {
-    // split each query's keys so that the CTAs fill the SMs once
-    const int want = max(1, (per_sm * sm_count()) / n_qc);
-    tpc = max(4, (tiles + want - 1) / want);
-  } else {
-    tpc = max(1, min(tiles, 32));
-  }
-  const dim3 grid(n_qc, (tiles + tpc - 1) / tpc);
-  size_t sm = static_cast<size_t>(kStages) * kTileB + static_cast<size_t>(N) * kRowB + kStages * kKeys * 4 +
-              static_cast<size_t>(N) * 4 + 1024;
-  // no more CTAs per SM than its 512 tensor-memory columns hold, so tcgen05.alloc never
-  // waits for another CTA
-  const size_t cap = 227 * 1024 / per_sm - 2048;
-  if (sm < cap) sm = cap;
-  cudaFuncSetAttribute(k_index_tc<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
-  k_index_tc<1><<<grid, kThreads, sm, st>>>(tk, a, tpc, cols, decode ? 1 : 0);
+  return enc(tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a.k), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_index_tc(const lc_index_args& a, bool decode, cudaStream_t st) {
+  CUtensorMap tk;
+  if (!make_key_map(&tk, a)) return cudaErrorInvalidValue;
+  const IndexGeom g = index_geometry(a, decode, false);
+  const dim3 grid(a.n_q, g.n_chunks);
+  IdxSelect none{};
+  cudaFuncSetAttribute(k_index_tc<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(g.smem));
+  k_index_tc<1, false><<<grid, kThreads, g.smem, st>>>(tk, a, g.tpc, g.tmem_cols, decode ? 1 : 0, none);
   return cudaGetLastError();
+}
+
+size_t index_topk_workspace(const lc_index_topk_args& a, bool decode) {
+  const IndexGeom g = index_geometry(a.index, decode, true);
+  if (g.n_chunks <= 1) return 0;
+  const size_t rows = static_cast<size_t>(a.index.n_q) * g.n_chunks;
+  return (rows * 4 + 15) / 16 * 16 + rows * a.k * sizeof(uint2);
+}
+
+cudaError_t launch_index_topk(const lc_index_topk_args& a, bool decode, cudaStream_t st) {
+  CUtensorMap tk;
+  if (!make_key_map(&tk, a.index)) return cudaErrorInvalidValue;
+  const IndexGeom g = index_geometry(a.index, decode, true);
+  IdxSelect sel{};
+  sel.k = a.k;
+  sel.n_chunks = g.n_chunks;
+  sel.idx = a.idx;
+  sel.count = a.count;
+  if (g.n_chunks > 1) {
+    const size_t rows = static_cast<size_t>(a.index.n_q) * g.n_chunks;
+    sel.cand_cnt = static_cast<int*>(a.workspace);
+    sel.cand = reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.workspace) + (rows * 4 + 15) / 16 * 16);
+  }
+  const dim3 grid(a.index.n_q, g.n_chunks);
+  cudaFuncSetAttribute(k_index_tc<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(g.smem));
+  k_index_tc<1, true><<<grid, kThreads, g.smem, st>>>(tk, a.index, g.tpc, g.tmem_cols, decode ? 1 : 0, sel);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || g.n_chunks == 1) return e;
+  return launch_topk_merge(a, g.n_chunks, sel.cand, sel.cand_cnt, decode, st);
 }
 
 }  // namespace lc

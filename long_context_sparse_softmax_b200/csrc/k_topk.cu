@@ -452,6 +452,208 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
   if (fast) asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
 
+// ---------------------------------------------------------------------------------
+// Merge of the fused indexer's candidates (lc_csa_index_topk_* when a query's keys span
+// several CTAs).  Range c of query q left cnt[q][c] candidates (order key, entry index)
+// in ascending index order, at least the range's own top K; the ranges are disjoint and
+// ascending, so the concatenation of their lists is in ascending index order.  One CTA
+// per query selects the K largest keys of the list, ties to the earlier position (the
+// lower index), by radix passes of 11 bits over the keys (held in shared memory when
+// they fit), and writes the selected indices in list order.  Each thread owns a
+// contiguous segment of positions, so the order survives the block-wide scans.
+constexpr int kMergeThreads = 1024;
+constexpr int kMergeWarps = kMergeThreads / 32;
+constexpr int kMergeCache = 48 * 1024;  // keys held in shared memory (192 KB)
+constexpr int kMergeMaxChunks = kMergeThreads;
+
+// exclusive prefix of v over the CTA in thread order; *total gets the sum
+__device__ __forceinline__ int scan_cta(int v, int* s_w, int* s_total, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) s_w[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int x = s_w[lane];
+    int xi = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, xi, o);
+      if (lane >= o) xi += t;
+    }
+    s_w[lane] = xi - x;
+    if (lane == 31) *s_total = xi;
+  }
+  __syncthreads();
+  const int r = s_w[warp] + incl - v;
+  *total = *s_total;
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kMergeThreads) k_topk_merge(int k, int m, int W_x, lc_batch batch,
+                                                              const uint2* __restrict__ cand,
+                                                              const int* __restrict__ cand_cnt, int n_chunks,
+                                                              int32_t* idx, int32_t* count, int decode,
+                                                              int cached) {
+  static_assert(kMergeWarps == 32, "one warp scans the warp totals");
+  extern __shared__ uint32_t kc[];  // [n] candidate keys (cached)
+  __shared__ int s_off[kMergeMaxChunks + 1];
+  __shared__ int s_hist[kBins];
+  __shared__ int s_w[kMergeWarps];
+  __shared__ int s_total;
+  __shared__ int s_pick[2];
+  __shared__ uint32_t s_rng[2][kMergeWarps];
+  const int q = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = decode ? q : seq_of_query(batch.q_start, batch.num_seqs, q);
+  const int p = __ldg(batch.q_pos0 + b) + (decode ? 0 : q - __ldg(batch.q_start + b));
+  const int nv = n_visible(p, m, W_x, __ldg(batch.n_ent + b));
+  const int K = min(k, nv);
+  int32_t* out = idx + static_cast<int64_t>(q) * k;
+  for (int i = K + tid; i < k; i += kMergeThreads) out[i] = -1;
+  if (tid == 0 && count) count[q] = K;
+  if (K == 0) return;
+  // offsets of the ranges' lists in the concatenation
+  int n = 0;
+  {
+    const int v = tid < n_chunks ? __ldg(cand_cnt + static_cast<int64_t>(q) * n_chunks + tid) : 0;
+    const int ex = scan_cta(v, s_w, &s_total, &n);
+    if (tid < n_chunks) s_off[tid] = ex;
+    if (tid == 0) s_off[n_chunks] = n;
+  }
+  __syncthreads();
+  const uint2* cq = cand + static_cast<int64_t>(q) * n_chunks * k;
+  const int seg = (n + kMergeThreads - 1) / kMergeThreads;
+  const int i0 = min(n, tid * seg), i1 = min(n, i0 + seg);
+  int c0 = 0;  // range of position i0: the last c with s_off[c] <= i0
+  {
+    int lo = 0, hi = n_chunks - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_off[mid] <= i0) lo = mid;
+      else hi = mid - 1;
+    }
+    c0 = lo;
+  }
+  // visit the own segment in order: fn(position, candidate)
+  auto each = [&](auto fn) {
+    int c = c0;
+    for (int i = i0; i < i1; ++i) {
+      while (i >= s_off[c + 1]) ++c;
+      fn(i, cq + static_cast<int64_t>(c) * k + (i - s_off[c]));
+    }
+  };
+  const bool take_all = n <= K;
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  each([&](int i, const uint2* e) {
+    const uint32_t key = __ldg(&e->x);
+    if (cached) kc[i] = key;
+    kmin = min(kmin, key);
+    kmax = max(kmax, key);
+  });
+  auto key_at = [&](int i, const uint2* e) -> uint32_t { return cached ? kc[i] : __ldg(&e->x); };
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) {
+    s_rng[0][warp] = kmin;
+    s_rng[1][warp] = kmax;
+  }
+  __syncthreads();
+  uint32_t umin = 0xffffffffu, umax = 0u;
+#pragma unroll 4
+  for (int w = 0; w < kMergeWarps; ++w) {
+    umin = min(umin, s_rng[0][w]);
+    umax = max(umax, s_rng[1][w]);
+  }
+  // radix passes (see k_topk): pfx = bits of the K-th largest rel = key - umin so far,
+  // rem = keys still to take inside the bin they select
+  uint32_t pfx = 0;
+  int rem = K;
+  int shift = take_all ? 0 : 32 - __clz(static_cast<int>(umax - umin));
+#pragma unroll 1
+  while (shift > 0) {
+    const int w = min(11, shift);
+    const int hi = shift;
+    shift -= w;
+    const uint32_t bmask = (1u << w) - 1u;
+    for (int i = tid; i < kBins; i += kMergeThreads) s_hist[i] = 0;
+    __syncthreads();
+    each([&](int i, const uint2* e) {
+      const uint32_t rel = key_at(i, e) - umin;
+      const uint32_t top = hi >= 32 ? 0u : rel >> hi;
+      if (top == pfx) atomicAdd(&s_hist[(rel >> shift) & bmask], 1);
+    });
+    __syncthreads();
+    // thread t owns bins 2047 - 2t and 2046 - 2t (descending)
+    const int h0 = s_hist[kBins - 1 - 2 * tid], h1 = s_hist[kBins - 2 - 2 * tid];
+    int tot;
+    const int ex = scan_cta(h0 + h1, s_w, &s_total, &tot);
+    if (ex < rem && ex + h0 + h1 >= rem) {
+      const bool upper = ex + h0 >= rem;
+      s_pick[0] = upper ? kBins - 1 - 2 * tid : kBins - 2 - 2 * tid;
+      s_pick[1] = upper ? rem - ex : rem - ex - h0;
+    }
+    __syncthreads();
+    pfx = (pfx << w) | static_cast<uint32_t>(s_pick[0]);
+    rem = s_pick[1];
+  }
+  const uint32_t T = umin + pfx;
+  // keys equal to T, ranked by position; then the selection's output positions
+  int n_eq = 0;
+  each([&](int i, const uint2* e) { n_eq += !take_all && key_at(i, e) == T; });
+  int tot;
+  int eq_rank = scan_cta(n_eq, s_w, &s_total, &tot);
+  int n_sel = 0;
+  {
+    int r = eq_rank;
+    each([&](int i, const uint2* e) {
+      const uint32_t key = key_at(i, e);
+      const bool eq = !take_all && key == T;
+      n_sel += take_all || key > T || (eq && r < rem);
+      r += eq;
+    });
+  }
+  int pos = scan_cta(n_sel, s_w, &s_total, &tot);
+  each([&](int i, const uint2* e) {
+    const uint32_t key = key_at(i, e);
+    const bool eq = !take_all && key == T;
+    if (take_all || key > T || (eq && eq_rank < rem)) out[pos++] = static_cast<int32_t>(__ldg(&e->y));
+    eq_rank += eq;
+  });
+}
+
+cudaError_t launch_topk_merge(const lc_index_topk_args& a, int n_chunks, const uint2* cand, const int* cand_cnt,
+                              bool decode, cudaStream_t st) {
+  if (n_chunks > kMergeMaxChunks) return cudaErrorInvalidConfiguration;
+  const int64_t n_max = static_cast<int64_t>(n_chunks) * a.k;
+  const int cached = n_max <= kMergeCache ? 1 : 0;
+  const size_t sm = cached ? static_cast<size_t>(n_max) * 4 : 0;
+  cudaFuncSetAttribute(k_topk_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, kMergeCache * 4);
+  k_topk_merge<<<a.index.n_q, kMergeThreads, sm, st>>>(a.k, a.index.m, a.index.W_x, a.index.batch, cand, cand_cnt,
+                                                        n_chunks, a.idx, a.count, decode ? 1 : 0, cached);
+  return cudaGetLastError();
+}
+
+__global__ void k_empty_selection(int32_t* idx, int32_t* count, int n_q, int k) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < static_cast<int64_t>(n_q) * k) idx[i] = -1;
+  if (count && i < n_q) count[i] = 0;
+}
+
+cudaError_t launch_empty_selection(int32_t* idx, int32_t* count, int n_q, int k, cudaStream_t st) {
+  const int64_t n = static_cast<int64_t>(n_q) * k;
+  k_empty_selection<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(idx, count, n_q, k);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_topk(const lc_topk_args& a, bool decode, cudaStream_t st) {
   if (a.n_q == 0) return cudaSuccess;
   // the largest cluster that keeps the rows within one wave (one 1024-thread CTA per SM),

@@ -89,7 +89,8 @@ lc_status compress(const lc_compress_args* a, void* stream, bool hca) {
   return launched(lc::launch_compress(*a, hca, static_cast<cudaStream_t>(stream)));
 }
 
-lc_status index_scores(const lc_index_args* a, void* stream, bool decode) {
+// Validation shared by the indexer calls; `scores` says whether a score matrix is written.
+lc_status check_index(const lc_index_args* a, bool decode, bool scores) {
   if (!a) return LC_ERR_ARG;
   if (a->n_q < 0 || a->max_ent < 0 || a->m < 1 || a->W_x < 0) return LC_ERR_ARG;
   if (a->H_I < 1) return LC_ERR_ARG;
@@ -102,17 +103,41 @@ lc_status index_scores(const lc_index_args* a, void* stream, bool decode) {
     return LC_ERR_ARG;
   }
   if (a->w_qstride != 0 && a->w_qstride != a->H_I) return LC_ERR_ARG;
-  if (a->score_stride < a->max_ent || a->score_stride % 4) return LC_ERR_ARG;
+  if (scores && (a->score_stride < a->max_ent || a->score_stride % 4)) return LC_ERR_ARG;
   if (decode && a->n_q != a->batch.num_seqs) return LC_ERR_ARG;
   if (a->n_q == 0 || a->max_ent == 0) return LC_OK;
   LC_TRY(check_batch(a->batch, true, false));
-  if (!a->q || !a->k || !a->w || !a->scores) return LC_ERR_ARG;
+  if (!a->q || !a->k || !a->w || (scores && !a->scores)) return LC_ERR_ARG;
   if (a->fmt == LC_IDX_MXFP4 && (!a->q_scale || !a->k_scale || a->n_keys < 1 || a->n_keys >= (int64_t{1} << 31)))
     return LC_ERR_ARG;
   if (a->fmt == LC_IDX_MXFP4 && ((reinterpret_cast<uintptr_t>(a->q_scale) | reinterpret_cast<uintptr_t>(a->k_scale)) & 3u))
     return LC_ERR_ALIGN;
-  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->scores)) return LC_ERR_ALIGN;
+  if (!aligned16(a->q) || !aligned16(a->k) || (scores && !aligned16(a->scores))) return LC_ERR_ALIGN;
+  return LC_OK;
+}
+
+lc_status index_scores(const lc_index_args* a, void* stream, bool decode) {
+  LC_TRY(check_index(a, decode, true));
+  if (a->n_q == 0 || a->max_ent == 0) return LC_OK;
   return launched(lc::launch_index_scores(*a, decode, static_cast<cudaStream_t>(stream)));
+}
+
+lc_status index_topk(const lc_index_topk_args* a, void* stream, bool decode) {
+  if (!a) return LC_ERR_ARG;
+  if (a->k < 1 || a->k > 2048) return LC_ERR_ARG;
+  LC_TRY(check_index(&a->index, decode, false));
+  if (a->index.fmt != LC_IDX_MXFP4) return LC_ERR_UNSUPPORTED;
+  if (a->index.n_q == 0) return LC_OK;
+  if (!a->idx) return LC_ERR_ARG;
+  if (a->index.max_ent > 0 && lc::index_geometry(a->index, decode, true).n_chunks > 1024) return LC_ERR_UNSUPPORTED;
+  const size_t need = a->index.max_ent > 0 ? lc::index_topk_workspace(*a, decode) : 0;
+  if (need > 0 && (!a->workspace || a->workspace_bytes < need)) return LC_ERR_WORKSPACE;
+  if (need > 0 && !aligned16(a->workspace)) return LC_ERR_ALIGN;
+  if (a->index.max_ent == 0) {
+    // no entries anywhere: every query selects nothing
+    return launched(lc::launch_empty_selection(a->idx, a->count, a->index.n_q, a->k, static_cast<cudaStream_t>(stream)));
+  }
+  return launched(lc::launch_index_topk(*a, decode, static_cast<cudaStream_t>(stream)));
 }
 
 lc_status topk(const lc_topk_args* a, void* stream, bool decode) {
@@ -164,6 +189,13 @@ lc_status lc_hca_compress_decode(const lc_compress_args* a, void* stream) { retu
 lc_status lc_csa_index_scores_prefill(const lc_index_args* a, void* stream) { return index_scores(a, stream, false); }
 lc_status lc_csa_index_scores_decode(const lc_index_args* a, void* stream) { return index_scores(a, stream, true); }
 
+lc_status lc_csa_index_topk_prefill(const lc_index_topk_args* a, void* stream) { return index_topk(a, stream, false); }
+lc_status lc_csa_index_topk_decode(const lc_index_topk_args* a, void* stream) { return index_topk(a, stream, true); }
+size_t lc_csa_index_topk_workspace_bytes(const lc_index_topk_args* a, int32_t decode) {
+  if (!a || a->index.n_q <= 0 || a->index.max_ent <= 0 || a->k < 1) return 0;
+  return lc::index_topk_workspace(*a, decode != 0);
+}
+
 lc_status lc_csa_topk_prefill(const lc_topk_args* a, void* stream) { return topk(a, stream, false); }
 lc_status lc_csa_topk_decode(const lc_topk_args* a, void* stream) { return topk(a, stream, true); }
 
@@ -205,6 +237,7 @@ size_t lc_struct_size(int32_t which) {
     case 5: return sizeof(lc_index_args);
     case 6: return sizeof(lc_topk_args);
     case 7: return sizeof(lc_attn_args);
+    case 8: return sizeof(lc_index_topk_args);
     default: return 0;
   }
 }

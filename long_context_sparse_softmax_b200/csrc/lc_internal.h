@@ -14,6 +14,8 @@ cudaError_t launch_qk_prep(const lc_qk_prep_args& a, cudaStream_t st);
 cudaError_t launch_compress(const lc_compress_args& a, bool per_cta, cudaStream_t st);
 cudaError_t launch_index_scores(const lc_index_args& a, bool decode, cudaStream_t st);
 cudaError_t launch_topk(const lc_topk_args& a, bool decode, cudaStream_t st);
+// idx[q, :] = -1 and count[q] = 0 for every query
+cudaError_t launch_empty_selection(int32_t* idx, int32_t* count, int n_q, int k, cudaStream_t st);
 cudaError_t launch_attn(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st);
 size_t attn_workspace_bytes(const lc_attn_args& a, bool sparse, bool decode);
 bool attn_tc_supported(const lc_attn_args& a);
@@ -26,6 +28,19 @@ bool attn_tc8_supported(const lc_attn_args& a);
 size_t attn_tc8_workspace(const lc_attn_args& a, bool sparse, bool decode);
 cudaError_t launch_attn_tc8(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st, int* n_split);
 cudaError_t launch_index_tc(const lc_index_args& a, bool decode, cudaStream_t st);
+
+// Indexer launch shape: key tiles, tiles per CTA, CTAs per query, tensor-memory columns,
+// dynamic shared memory.
+struct IndexGeom {
+  int tiles, tpc, n_chunks;
+  uint32_t tmem_cols;
+  size_t smem;
+};
+IndexGeom index_geometry(const lc_index_args& a, bool decode, bool select);
+size_t index_topk_workspace(const lc_index_topk_args& a, bool decode);
+cudaError_t launch_index_topk(const lc_index_topk_args& a, bool decode, cudaStream_t st);
+cudaError_t launch_topk_merge(const lc_index_topk_args& a, int n_chunks, const uint2* cand, const int* cand_cnt,
+                              bool decode, cudaStream_t st);
 
 // Sequence of query row q: the b with q_start[b] <= q < q_start[b+1] (binary search).
 __device__ __forceinline__ int seq_of_query(const int32_t* __restrict__ q_start, int num_seqs, int q) {

@@ -4,7 +4,9 @@ memory only) and issue the library calls in the method's order.
 Prefill (one sequence): prepare queries and window tokens -> compress the context ->
 [CSA: index scores -> top-k] -> attention.  Decode (one query per sequence, on a
 cache): prepare the query and the newest token's window row, compress the block the
-newest token closed, [CSA: index -> top-k] -> attention.
+newest token closed, [CSA: index -> top-k] -> attention.  With MXFP4 indexer operands the
+index and top-k stages run fused (lc_csa_index_topk_*: no score matrix) unless the run is
+built with fused=False; the separate calls stay available as index() and topk().
 
 Nothing here computes any part of the method; every step is a kernel of liblc.so.
 """
@@ -14,10 +16,11 @@ from typing import Dict, Optional
 
 import torch
 
-from . import (AttnArgs, Batch, CompressArgs, Dims, IndexArgs, QkPrepArgs, Rows, TopkArgs,
+from . import (AttnArgs, Batch, CompressArgs, Dims, IndexArgs, IndexTopkArgs, QkPrepArgs, Rows, TopkArgs,
                LC_FMT_BF16, LC_FMT_E4M3_BF16, LC_FMT_F32, LC_IDX_F32, LC_IDX_MXFP4,
                lc_csa_compress_decode, lc_csa_compress_prefill, lc_csa_index_scores_decode,
-               lc_csa_index_scores_prefill, lc_csa_sparse_attn_decode, lc_csa_sparse_attn_prefill,
+               lc_csa_index_scores_prefill, lc_csa_index_topk_decode, lc_csa_index_topk_prefill,
+               lc_csa_index_topk_workspace_bytes, lc_csa_sparse_attn_decode, lc_csa_sparse_attn_prefill,
                lc_csa_sparse_attn_workspace_bytes, lc_csa_topk_decode, lc_csa_topk_prefill,
                lc_hca_attn_decode, lc_hca_attn_prefill, lc_hca_attn_workspace_bytes,
                lc_hca_compress_decode, lc_hca_compress_prefill, lc_qk_prep_decode, lc_qk_prep_prefill)
@@ -60,7 +63,7 @@ class _Common:
         may run concurrently on two streams; `after` (attention) needs both."""
         st = dict(self.stages())
         side = [(n, st[n]) for n in ("qk_prep_q", "qk_prep_win", "compress") if n in st]
-        main = [(n, st[n]) for n in ("index", "topk") if n in st]
+        main = [(n, st[n]) for n in ("index", "topk", "index_topk") if n in st]
         return side, main, [("attn", st["attn"])]
 
     def host_inputs(self):
@@ -75,7 +78,7 @@ class _Common:
         else:
             h = {"qk_prep_q": [inp["q_raw"]], "_fork": [inp["x"], inp["g"]]}
         if qI:
-            h["index"] = qI
+            h["index_topk" if self.fused else "index"] = qI
         return h
 
     def host_outputs(self):
@@ -138,6 +141,20 @@ class _Common:
                          (kI["codes"] if mx else kI["f32"]).shape[0], ptr(inp["w"]), 0, s.m, self.W_x, max_ent, self.batch,
                          ptr(scores), scores.shape[1], ptr(self.status))
 
+    def _index_topk_args(self, n_q: int, max_ent: int, decode: bool) -> IndexTopkArgs:
+        """Fused index + top-k into idx / count (the buffers the separate top-k call writes
+        and attention reads)."""
+        s = self.spec
+        a = IndexTopkArgs()
+        a.index = self._index_args(n_q, max_ent, self.scores)
+        a.index.scores, a.index.score_stride = None, 0
+        a.k = s.k
+        a.idx, a.count = ptr(self.idx), ptr(self.count)
+        ws = lc_csa_index_topk_workspace_bytes(a, decode)
+        self.ws_topk = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.device)
+        a.workspace, a.workspace_bytes = ptr(self.ws_topk), ws
+        return a
+
     def _topk_args(self, n_q: int, max_ent: int) -> TopkArgs:
         s = self.spec
         return TopkArgs(n_q, s.k, s.m, self.W_x, max_ent, 0, ptr(self.scores), self.scores.shape[1], self.batch,
@@ -174,10 +191,12 @@ class _Common:
 class Prefill(_Common):
     """One sequence of L raw tokens; queries at q_first .. q_first + n_q - 1."""
 
-    def __init__(self, inp: Dict[str, object], device="cuda", W_x: Optional[int] = None, impl: int = 0):
+    def __init__(self, inp: Dict[str, object], device="cuda", W_x: Optional[int] = None, impl: int = 0,
+                 fused: Optional[bool] = None):
         s: wl.Spec = inp["spec"]
         self.impl = impl
         self.spec, self.inp, self.device = s, inp, device
+        self.fused = s.is_csa and s.idx_fmt == wl.IDX_MXFP4 if fused is None else fused
         self.W_x = s.W if W_x is None else W_x
         L, n_c = inp["L"], inp["n_c"]
         self.dims = Dims(s.D, s.d_r, s.rope_off, s.H)
@@ -211,6 +230,8 @@ class Prefill(_Common):
             self.count = torch.empty(s.n_q, dtype=torch.int32, device=device)
             self.a_index = self._index_args(s.n_q, n_c, self.scores)
             self.a_topk = self._topk_args(s.n_q, n_c)
+            if self.fused:
+                self.a_index_topk = self._index_topk_args(s.n_q, n_c, False)
         else:
             self.idx = None
         self.a_attn = self._attn_args(s.n_q, n_c, s.is_csa)
@@ -230,13 +251,16 @@ class Prefill(_Common):
     def topk(self, stream=None):
         lc_csa_topk_prefill(self.a_topk, stream)
 
+    def index_topk(self, stream=None):
+        lc_csa_index_topk_prefill(self.a_index_topk, stream)
+
     def attn(self, stream=None):
         (lc_csa_sparse_attn_prefill if self.spec.is_csa else lc_hca_attn_prefill)(self.a_attn, stream)
 
     def stages(self):
         st = [("qk_prep_q", self.prep_queries), ("qk_prep_win", self.prep_window), ("compress", self.compress)]
         if self.spec.is_csa:
-            st += [("index", self.index), ("topk", self.topk)]
+            st += [("index_topk", self.index_topk)] if self.fused else [("index", self.index), ("topk", self.topk)]
         return st + [("attn", self.attn)]
 
     def step(self, stream=None):
@@ -247,10 +271,12 @@ class Prefill(_Common):
 class Decode(_Common):
     """B sequences, one query each at L_b - 1, on an existing cache (see workloads.make_decode)."""
 
-    def __init__(self, inp: Dict[str, object], device="cuda", W_x: Optional[int] = None, impl: int = 0):
+    def __init__(self, inp: Dict[str, object], device="cuda", W_x: Optional[int] = None, impl: int = 0,
+                 fused: Optional[bool] = None):
         s: wl.Spec = inp["spec"]
         self.impl = impl
         self.spec, self.inp, self.device = s, inp, device
+        self.fused = s.is_csa and s.idx_fmt == wl.IDX_MXFP4 if fused is None else fused
         self.W_x = s.W if W_x is None else W_x
         B = s.num_seqs
         n_c = inp["n_c"]
@@ -286,6 +312,8 @@ class Decode(_Common):
             self.count = torch.empty(B, dtype=torch.int32, device=device)
             self.a_index = self._index_args(B, max_ent, self.scores)
             self.a_topk = self._topk_args(B, max_ent)
+            if self.fused:
+                self.a_index_topk = self._index_topk_args(B, max_ent, True)
         else:
             self.idx = None
         self.a_attn = self._attn_args(B, max_ent, s.is_csa)
@@ -305,13 +333,16 @@ class Decode(_Common):
     def topk(self, stream=None):
         lc_csa_topk_decode(self.a_topk, stream)
 
+    def index_topk(self, stream=None):
+        lc_csa_index_topk_decode(self.a_index_topk, stream)
+
     def attn(self, stream=None):
         (lc_csa_sparse_attn_decode if self.spec.is_csa else lc_hca_attn_decode)(self.a_attn, stream)
 
     def stages(self):
         st = [("qk_prep_q", self.prep_queries), ("qk_prep_win", self.prep_window), ("compress", self.compress)]
         if self.spec.is_csa:
-            st += [("index", self.index), ("topk", self.topk)]
+            st += [("index_topk", self.index_topk)] if self.fused else [("index", self.index), ("topk", self.topk)]
         return st + [("attn", self.attn)]
 
     def step(self, stream=None):

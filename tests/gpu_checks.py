@@ -39,6 +39,24 @@ def _sync():
     torch.cuda.synchronize()
 
 
+def _separate_index_topk(run, rep) -> None:
+    """A step with the fused index + top-k leaves its selection in run.idx.  Run the
+    separate indexer and top-k calls on the same inputs (they fill run.scores, which the
+    checks below compare with the oracle, and run.idx again): the fused selection must be
+    bit-identical to top-k of those scores."""
+    if not run.spec.is_csa or not run.fused:
+        return
+    fused_idx, fused_cnt = run.idx.clone(), run.count.clone()
+    run.index()
+    run.topk()
+    _sync()
+    assert run.read_status() == 0
+    assert torch.equal(fused_idx, run.idx), \
+        f"fused index+top-k differs from the separate calls in {int((fused_idx != run.idx).any(1).sum())} rows"
+    assert torch.equal(fused_cnt, run.count)
+    rep["fused_topk_rows_identical"] = int(fused_idx.shape[0])
+
+
 def check_prefill(spec: wl.Spec, q_sel: Sequence[int] = None, W_x: int = None, report=None, impl: int = 0):
     """Run a prefill workload through the library and compare it with the oracle on the
     queries q_sel (local indices; all queries if None)."""
@@ -48,10 +66,11 @@ def check_prefill(spec: wl.Spec, q_sel: Sequence[int] = None, W_x: int = None, r
     run.step()
     _sync()
     assert run.read_status() == 0, f"device status {run.read_status()}"
+    rep = {} if report is None else report
+    _separate_index_topk(run, rep)
     q_sel = list(range(spec.n_q)) if q_sel is None else list(q_sel)
     orc = OraclePrefill(inp, q_sel, W_x)
     d_n = spec.d_n
-    rep = {} if report is None else report
 
     # compression
     n_c = inp["n_c"]
@@ -202,10 +221,11 @@ def check_decode(spec: wl.Spec, W_x: int = None, report=None, impl: int = 0):
     run.step()
     _sync()
     assert run.read_status() == 0, f"device status {run.read_status()}"
+    rep = {} if report is None else report
+    _separate_index_topk(run, rep)
     orc = OracleDecode(inp, W_x)
     B = spec.num_seqs
     d_n = spec.d_n
-    rep = {} if report is None else report
 
     # decode-time compression of the closed block
     lib_ent = orc.ent_f.copy()

@@ -36,7 +36,12 @@ def test_host_inputs_name_the_stage_that_reads_them():
     assert h["qk_prep_q"][0] is inp["q_raw"]
     assert h["qk_prep_win"][0] is inp["x_new"]
     assert h["compress"][0] is inp["x_tail"] and h["compress"][1] is inp["g_tail"]
-    assert set(map(id, h["index"])) == set(map(id, inp["qI"].values()))
+    # MXFP4 indexer operands: index and top-k run fused, and the indexer queries feed that stage
+    assert r.fused and [n for n, _ in r.stages()][3:] == ["index_topk", "attn"]
+    assert set(map(id, h["index_topk"])) == set(map(id, inp["qI"].values()))
+    r2 = runner.Decode(inp, "cpu", fused=False)
+    assert [n for n, _ in r2.stages()][3:] == ["index", "topk", "attn"]
+    assert set(map(id, r2.host_inputs()["index"])) == set(map(id, inp["qI"].values()))
     assert r.host_outputs() == [r.out, r.lse]
     # prefill: the raw tokens feed both window preparation and compression (two side
     # streams), so they are copied before the fork
