@@ -307,6 +307,74 @@ def hca_attn_query(q: np.ndarray, entries: np.ndarray, n_vis: int, win_rows: np.
 
 
 # =====================================================================================
+# Decode-time cache maintenance
+# =====================================================================================
+E2M1_POS = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])   # codes 0..7
+
+
+def f64_to_e2m1(v: np.ndarray) -> np.ndarray:
+    """float64 -> E2M1 codes (uint8, 4 bits): the nearest E2M1 value, ties to the even
+    code, saturating at +-6 (OCP MX v1.0 conversion with saturation).  Zero is code 0
+    whatever the sign of the input."""
+    a = np.minimum(np.abs(np.asarray(v, dtype=np.float64)), 6.0)
+    d = np.abs(a[..., None] - E2M1_POS)                      # distance to each magnitude
+    best = d.min(axis=-1, keepdims=True)
+    cand = d == best                                           # one or two nearest codes
+    codes = np.arange(8)
+    # among the nearest, the even code (two nearest neighbours differ in the last bit)
+    even = cand & (codes % 2 == 0)
+    pick = np.where(even.any(axis=-1), np.argmax(even, axis=-1), np.argmax(cand, axis=-1))
+    neg = (np.asarray(v) < 0) & (pick > 0)
+    return (pick | (neg.astype(np.int64) << 3)).astype(np.uint8)
+
+
+def f64_to_mxfp4(v: np.ndarray):
+    """float64 [..., d] (d a multiple of 32) -> MXFP4 (codes uint8 [..., d/2] with element 2i
+    in the low nibble, E8M0 scales uint8 [..., d/32]), OCP MX v1.0: per block of 32 the
+    shared scale is X = 2^(floor(log2 amax) - 2), 2 being the largest exponent of E2M1; a
+    block of zeros takes X = 2^0; each element is v / X converted to E2M1."""
+    v = np.asarray(v, dtype=np.float64)
+    d = v.shape[-1]
+    assert d % 32 == 0
+    blk = v.reshape(*v.shape[:-1], d // 32, 32)
+    amax = np.abs(blk).max(axis=-1)
+    _, ex = np.frexp(np.where(amax > 0, amax, 1.0))          # amax = f 2^ex, f in [0.5, 1)
+    e = np.where(amax > 0, ex - 1 - 2, 0)
+    e = np.clip(e, -127, 127)
+    el = f64_to_e2m1(blk / np.ldexp(1.0, e)[..., None]).reshape(*v.shape)
+    codes = (el[..., 0::2] | (el[..., 1::2] << 4)).astype(np.uint8)
+    return codes, (e + 127).astype(np.uint8)
+
+
+def pool_index_keys(k_raw: np.ndarray, g: np.ndarray, m: int, first_block: int = 0, tok_pos0: int = 0,
+                    n_blocks: Optional[int] = None) -> np.ndarray:
+    """Lightning-indexer keys of complete blocks: the same gated pooling as the KV entries
+    (alpha = softmax(g over the block), k = sum alpha_t k_t), with no RMSNorm and no RoPE
+    (the indexer operands are given directly).  k_raw [T, d_I] for positions
+    tok_pos0 .. tok_pos0 + T - 1; returns [n_blocks, d_I] float64."""
+    if n_blocks is None:
+        n_blocks = (tok_pos0 + k_raw.shape[0]) // m - first_block
+    out = np.empty((n_blocks, k_raw.shape[1]), dtype=np.float64)
+    for i in range(n_blocks):
+        r0 = (first_block + i) * m - tok_pos0
+        assert r0 >= 0 and r0 + m <= k_raw.shape[0], "block outside the given token rows"
+        out[i] = pool_block(k_raw[r0:r0 + m], g[r0:r0 + m])
+    return out
+
+
+def ring_slot(pos, R: int):
+    """Window ring buffer of R rows: the prepared row of position `pos` lives in slot pos mod R."""
+    return np.asarray(pos) % R
+
+
+def window_from_ring(ring: np.ndarray, p: int, W: int) -> np.ndarray:
+    """Window rows of a query at p (positions max(0, p-W+1) .. p) read from a ring buffer of
+    R >= W rows, in position order."""
+    ts = list(window_positions(p, W))
+    return ring[ring_slot(np.array(ts, dtype=np.int64), ring.shape[0])] if ts else ring[:0]
+
+
+# =====================================================================================
 # Numbers a test needs about a result
 # =====================================================================================
 def ulp_e4m3(v: np.ndarray) -> np.ndarray:

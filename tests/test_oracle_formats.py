@@ -159,3 +159,56 @@ def test_mxfp4_decode_matches_an_independent_dequantizer_on_every_byte_and_scale
         assert np.array_equal(mine, ref), f"scales {s0}..{s0 + 15}"
     # element 2i in the low nibble: byte 0x61 holds 0.5 (code 1) then 4.0 (code 6)
     assert np.array_equal(O.mxfp4_to_f64(np.full((1, 16), 0x61, np.uint8), np.array([[127]]))[0, :2], [0.5, 4.0])
+
+
+def test_e2m1_encoder_matches_ml_dtypes_rounding():
+    """The oracle's E2M1 conversion (nearest value, ties to the even code, saturating at
+    +-6) against ml_dtypes' float4_e2m1fn cast, on random values and on every tie."""
+    ml_dtypes = pytest.importorskip("ml_dtypes")
+    rng = np.random.default_rng(21)
+    grid = O.e2m1_to_f64(np.arange(8))
+    ties = (grid[:-1] + grid[1:]) / 2
+    v = np.concatenate([rng.standard_normal(20000) * 3, ties, -ties, [0.0, 6.0, 7.99, -7.99, 1e-9]])
+    ref = v.astype(np.float32).astype(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    mine = O.e2m1_to_f64(O.f64_to_e2m1(v))
+    assert np.array_equal(mine, ref)
+    assert np.all(O.f64_to_e2m1(np.array([-0.1, -0.0, 0.0])) == 0)  # zero is code 0
+
+
+def test_mxfp4_encoder_scale_rule_and_elements():
+    """OCP MX v1.0 shared scale X = 2^(floor(log2 amax) - 2) on crafted blocks, a zero block
+    at 2^0, and elements equal to the E2M1 cast of v / X."""
+    ml_dtypes = pytest.importorskip("ml_dtypes")
+    blocks = np.zeros((5, 32))
+    blocks[0, 3] = 1.0          # floor(log2 1) = 0 -> X = 2^-2
+    blocks[1, 0] = -6.0         # 2 -> X = 2^0
+    blocks[2, 31] = 0.3         # -2 -> X = 2^-4
+    blocks[3, 7] = 1000.0       # 9 -> X = 2^7
+    codes, scales = O.f64_to_mxfp4(blocks.reshape(1, 160))
+    assert scales.tolist() == [[125, 127, 123, 134, 127]]
+    rng = np.random.default_rng(22)
+    v = rng.standard_normal((50, 128)) * np.exp2(rng.integers(-6, 6, (50, 1)))
+    codes, scales = O.f64_to_mxfp4(v)
+    X = np.exp2(scales.astype(np.float64) - 127)
+    ref = (v.reshape(50, 4, 32) / X[..., None]).astype(np.float32).astype(ml_dtypes.float4_e2m1fn)
+    assert np.array_equal(O.mxfp4_to_f64(codes, scales), ref.astype(np.float64).reshape(50, 128) * np.repeat(X, 32, -1))
+
+
+def test_mxfp4_encoder_agrees_with_the_input_generator():
+    """Two independent codings of the same rule: the oracle's (numpy distances) and the
+    input generator's (torch bucketize), bit for bit on N(0,1) data."""
+    g = torch.Generator().manual_seed(23)
+    v = torch.randn(300, 128, generator=g)
+    c1, s1 = wl.mxfp4_encode(v)
+    c2, s2 = O.f64_to_mxfp4(v.double().numpy())
+    assert np.array_equal(c1.numpy(), c2) and np.array_equal(s1.numpy(), s2)
+
+
+def test_mxfp4_encoder_roundtrips_representable_values():
+    grid = O.e2m1_to_f64(np.arange(16))
+    rng = np.random.default_rng(24)
+    v = rng.choice(grid, (20, 64)) * 0.125
+    v[:, 0] = 6 * 0.125          # pin each block's amax so X = 2^-3
+    v[:, 32] = -6 * 0.125
+    c, s = O.f64_to_mxfp4(v)
+    assert np.array_equal(O.mxfp4_to_f64(c, s), v)

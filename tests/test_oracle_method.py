@@ -374,3 +374,30 @@ def test_workload_shapes_follow_the_pages():
 def test_mixed_lengths_are_in_range():
     assert len(wl.MIXED_CSA.seq_lens) == 8
     assert all(524288 <= L <= 1048576 for L in wl.MIXED_CSA.seq_lens)
+
+
+# ------------------------------------------------------------------ decode-time cache maintenance
+def test_index_key_pooling_closed_forms():
+    """Indexer keys use the entries' gate: equal gates give the mean, a dominant gate its
+    token, weights e^g / sum e^g in closed form; no normalisation or rotation."""
+    k = RNG.standard_normal((8, 128))
+    np.testing.assert_allclose(O.pool_index_keys(k, np.zeros(8), 4), [k[:4].mean(0), k[4:].mean(0)], rtol=1e-13)
+    g = np.array([0.0, np.log(2.0), np.log(3.0), np.log(4.0)])
+    np.testing.assert_allclose(O.pool_index_keys(np.eye(4), g, 4)[0], np.array([1, 2, 3, 4]) / 10.0, rtol=1e-14)
+    g2 = np.full(8, -50.0)
+    g2[6] = 50.0
+    np.testing.assert_allclose(O.pool_index_keys(k, g2, 4, first_block=1, tok_pos0=0, n_blocks=1)[0], k[6],
+                               rtol=1e-12, atol=1e-30)
+
+
+@pytest.mark.parametrize("R,W", [(128, 128), (192, 128), (16, 16)])
+def test_window_ring_equals_the_linear_window(R, W):
+    """Rows appended one position at a time into slot pos mod R give, for every query
+    position, the same window rows as the linear history."""
+    n = 3 * R + 5
+    rows = RNG.standard_normal((n, 8))
+    ring = np.zeros((R, 8))
+    for p in range(n):
+        ring[O.ring_slot(p, R)] = rows[p]
+        got = O.window_from_ring(ring, p, W)
+        assert np.array_equal(got, rows[max(0, p - W + 1):p + 1])
