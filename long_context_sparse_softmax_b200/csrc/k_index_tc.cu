@@ -493,8 +493,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int bpos = __ffs(word) - 1;
           word &= word - 1;
           const int off = w * 32 + bpos;  // key u * 128 + row' of the range
-          if (alone) out_idx[pos] = jbase + off;
-          else out_c[pos] = make_uint2(order_key(sc[off]), static_cast<uint32_t>(jbase + off));
+          if (pos < K) {  // exactly K bits are set; the guard only matters after a timeout
+            if (alone) out_idx[pos] = jbase + off;
+            else out_c[pos] = make_uint2(order_key(sc[off]), static_cast<uint32_t>(jbase + off));
+          }
           ++pos;
         }
         base += tot;

@@ -521,7 +521,8 @@ __global__ void __launch_bounds__(kMergeThreads) k_topk_merge(int k, int m, int 
   // offsets of the ranges' lists in the concatenation
   int n = 0;
   {
-    const int v = tid < n_chunks ? __ldg(cand_cnt + static_cast<int64_t>(q) * n_chunks + tid) : 0;
+    // a range writes at most k candidates (the clamp only matters after a timeout upstream)
+    const int v = tid < n_chunks ? min(max(__ldg(cand_cnt + static_cast<int64_t>(q) * n_chunks + tid), 0), k) : 0;
     const int ex = scan_cta(v, s_w, &s_total, &n);
     if (tid < n_chunks) s_off[tid] = ex;
     if (tid == 0) s_off[n_chunks] = n;
@@ -625,7 +626,10 @@ __global__ void __launch_bounds__(kMergeThreads) k_topk_merge(int k, int m, int 
   each([&](int i, const uint2* e) {
     const uint32_t key = key_at(i, e);
     const bool eq = !take_all && key == T;
-    if (take_all || key > T || (eq && eq_rank < rem)) out[pos++] = static_cast<int32_t>(__ldg(&e->y));
+    if (take_all || key > T || (eq && eq_rank < rem)) {
+      if (pos < K) out[pos] = static_cast<int32_t>(__ldg(&e->y));
+      ++pos;
+    }
     eq_rank += eq;
   });
 }
