@@ -624,7 +624,10 @@ def oracle_unit(name: str):
         def unit():
             q, _, _ = P.stored(one.q_fmt, O.qk_prep(qr, np.array([p]), one.rope_off, one.d_r), one.d_n)
             if one.is_csa:
-                qI = P.indexer_f64(one.idx_fmt, {k: v.numpy() for k, v in inp["qI"].items()})[0]
+                if one.idx_fmt == O.IDX_MXFP4:
+                    qI = O.mxfp4_to_f64(*O.f64_to_mxfp4(O.bf16_to_f64(inp["qI_raw"].numpy())))[0]
+                else:
+                    qI = P.indexer_f64(one.idx_fmt, {k: v.numpy() for k, v in inp["qI"].items()})[0]
                 kI = P.indexer_f64(one.idx_fmt, {k: v.numpy() for k, v in inp["kI"].items()})
                 idx, _, _ = P.select(qI, kI, inp["w"].numpy().astype(np.float64), p, one.m, one.W, one.k)
             else:
@@ -639,6 +642,13 @@ def oracle_unit(name: str):
     ent, _, _ = P.entries_from_tokens(xfun, inp["g"].numpy().astype(np.float64), spec.m, spec.rope_off, spec.d_r,
                                       spec.kv_fmt, spec.d_n)
     sink = inp["sink"].numpy().astype(np.float64)
+    kI_all = None
+    if spec.is_csa:
+        if spec.idx_fmt == O.IDX_MXFP4:
+            pooled = O.pool_index_keys(O.bf16_to_f64(inp["kI_raw"].numpy()), inp["g"].numpy().astype(np.float64), spec.m)
+            kI_all = O.mxfp4_to_f64(*O.f64_to_mxfp4(pooled))
+        else:
+            kI_all = P.indexer_f64(spec.idx_fmt, {k: v.numpy() for k, v in inp["kI"].items()})
     rng = np.random.default_rng(0)
     qs = rng.integers(0, spec.n_q, 64)
     state = {"i": 0}
@@ -653,13 +663,15 @@ def oracle_unit(name: str):
         qr = P.raw_rows(spec.raw_fmt, inp["q_raw"][i:i + 1].numpy())
         q, _, _ = P.stored(spec.q_fmt, O.qk_prep(qr, np.array([p]), spec.rope_off, spec.d_r), spec.d_n)
         if spec.is_csa:
-            qI = P.indexer_f64(spec.idx_fmt, {k: v[i:i + 1].numpy() for k, v in inp["qI"].items()})[0]
-            kI = P.indexer_f64(spec.idx_fmt, {k: v.numpy() for k, v in inp["kI"].items()})
-            idx, _, _ = P.select(qI, kI, inp["w"].numpy().astype(np.float64), p, spec.m, spec.W, spec.k)
+            if spec.idx_fmt == O.IDX_MXFP4:
+                qI = O.mxfp4_to_f64(*O.f64_to_mxfp4(O.bf16_to_f64(inp["qI_raw"][i:i + 1].numpy())))[0]
+            else:
+                qI = P.indexer_f64(spec.idx_fmt, {k: v[i:i + 1].numpy() for k, v in inp["qI"].items()})[0]
+            idx, _, _ = P.select(qI, kI_all, inp["w"].numpy().astype(np.float64), p, spec.m, spec.W, spec.k)
         else:
             idx = range(O.n_visible(p, spec.m, spec.W, ent.shape[0]))
         return O.sparse_attn_query(q[0], ent, idx, win, ts[0], p, spec.W, sink, spec.scale)
-    return unit, f"{name}: one query per unit (entries compressed once beforehand), float64 oracle"
+    return unit, f"{name}: one query per unit (entries and indexer keys compressed once beforehand), float64 oracle"
 
 
 def cpu_baseline(name: str, budget_s: float):

@@ -266,6 +266,58 @@ lc_status lc_csa_index_topk_decode(const lc_index_topk_args* a, void* stream);
 size_t lc_csa_index_topk_workspace_bytes(const lc_index_topk_args* a, int32_t decode);
 
 /* ---------------------------------------------------------------------------------
+ * mxfp4_quantize — rows of FP32 / BF16 values to OCP MXFP4 (Microscaling Formats v1.0):
+ * per block of 32 elements the E8M0 scale X = 2^(floor(log2 amax) - 2) (a zero block takes
+ * 2^0) and each element v / X converted to E2M1 with round-to-nearest-even, saturating at
+ * +-6; zero is code 0.  Element 2i goes to the low nibble of byte i.  Used for the
+ * indexer queries of each step.  Pages: "解读 DeepSeek V4", "FP4 Quantization-Aware
+ * Training" (the lightning indexer's QK path runs in FP4).
+ * ------------------------------------------------------------------------------- */
+typedef struct lc_mxfp4_quant_args {
+  int64_t n_rows;
+  int32_t d;               /* elements per row: multiple of 32, <= 1024 */
+  int32_t in_fmt;          /* LC_FMT_F32 or LC_FMT_BF16 */
+  const void* x;           /* [n_rows, d] */
+  uint8_t* codes;          /* [n_rows, d/2] */
+  uint8_t* scales;         /* [n_rows, d/32] */
+} lc_mxfp4_quant_args;
+
+lc_status lc_mxfp4_quantize(const lc_mxfp4_quant_args* a, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * csa_index_compress — for each requested complete block j of sequence b, the
+ * lightning-indexer key of entry j: the raw indexer-key rows of the block's m tokens
+ * pooled with the same block-softmax gate as the KV entries (alpha = softmax(g over the
+ * block), k = sum alpha_t k_t; no RMSNorm, no RoPE), quantised to MXFP4 as
+ * lc_mxfp4_quantize does, written at row ent_start[b] + j of codes / scales.  Prefill:
+ * every block; decode: the block the newest token closed.  Pages: "解读 DeepSeek V4" CSA
+ * section (the indexer scores the compressed entries) and FP4 QAT section;
+ * "DeepSeek-V4 论文分析" §5.3, §8.3.
+ * ------------------------------------------------------------------------------- */
+typedef struct lc_index_compress_args {
+  int32_t d_I;             /* key dims: multiple of 32, <= 256 */
+  int32_t m;               /* 1 .. 64 */
+  int32_t num_seqs;
+  int32_t in_fmt;          /* raw key rows: LC_FMT_F32 or LC_FMT_BF16 */
+  int32_t max_blocks;      /* host value: max over b of blk_count[b] */
+  int32_t reserved;
+  const void* x;           /* raw indexer-key rows of the tokens [*, d_I] */
+  const float* g;          /* gate logit of each token row (the KV entries' gates) */
+  const int64_t* tok_row0; /* as in lc_compress_args */
+  const int32_t* tok_pos0;
+  const int32_t* tok_len;
+  const int32_t* blk_first;
+  const int32_t* blk_count;
+  const int64_t* ent_start;
+  uint8_t* codes;          /* [*, d_I/2] */
+  uint8_t* scales;         /* [*, d_I/32] */
+  int32_t* status;         /* optional: LC_DEV_BAD_BLOCK */
+} lc_index_compress_args;
+
+lc_status lc_csa_index_compress_prefill(const lc_index_compress_args* a, void* stream);
+lc_status lc_csa_index_compress_decode(const lc_index_compress_args* a, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * csa_sparse_attn / hca_attn — for each query at p and head h, softmax attention over
  *   CSA: the selected entries idx[q, :] (-1 skipped), HCA: every visible entry,
  * joined with the window rows for positions max(0, p-W+1) .. p and the sink logit
@@ -363,8 +415,8 @@ const char* lc_version(void);
 const char* lc_status_string(lc_status s);
 /* sizeof of the args structs, for bindings to check their mirrors:
  * 0 lc_rows, 1 lc_dims, 2 lc_batch, 3 lc_qk_prep_args, 4 lc_compress_args,
- * 5 lc_index_args, 6 lc_topk_args, 7 lc_attn_args, 8 lc_index_topk_args; other values
- * return 0. */
+ * 5 lc_index_args, 6 lc_topk_args, 7 lc_attn_args, 8 lc_index_topk_args,
+ * 9 lc_mxfp4_quant_args, 10 lc_index_compress_args; other values return 0. */
 size_t lc_struct_size(int32_t which);
 
 #ifdef __cplusplus

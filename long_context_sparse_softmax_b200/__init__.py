@@ -78,6 +78,18 @@ class IndexTopkArgs(ctypes.Structure):
                 ("workspace", c_void_p), ("workspace_bytes", c_size_t)]
 
 
+class Mxfp4QuantArgs(ctypes.Structure):
+    _fields_ = [("n_rows", c_int64), ("d", c_int32), ("in_fmt", c_int32), ("x", c_void_p), ("codes", c_void_p),
+                ("scales", c_void_p)]
+
+
+class IndexCompressArgs(ctypes.Structure):
+    _fields_ = [("d_I", c_int32), ("m", c_int32), ("num_seqs", c_int32), ("in_fmt", c_int32), ("max_blocks", c_int32),
+                ("reserved", c_int32), ("x", c_void_p), ("g", c_void_p), ("tok_row0", c_void_p), ("tok_pos0", c_void_p),
+                ("tok_len", c_void_p), ("blk_first", c_void_p), ("blk_count", c_void_p), ("ent_start", c_void_p),
+                ("codes", c_void_p), ("scales", c_void_p), ("status", c_void_p)]
+
+
 class AttnArgs(ctypes.Structure):
     _fields_ = [("dims", Dims), ("n_q", c_int32), ("k", c_int32), ("m", c_int32), ("W", c_int32), ("W_x", c_int32),
                 ("max_ent", c_int32), ("scale", c_float), ("out_fmt", c_int32), ("q", Rows), ("ent", Rows),
@@ -90,7 +102,8 @@ class AttnArgs(ctypes.Structure):
 LC_IMPL_AUTO, LC_IMPL_TC, LC_IMPL_REF = 0, 2, 3
 
 
-STRUCTS = [Rows, Dims, Batch, QkPrepArgs, CompressArgs, IndexArgs, TopkArgs, AttnArgs, IndexTopkArgs]
+STRUCTS = [Rows, Dims, Batch, QkPrepArgs, CompressArgs, IndexArgs, TopkArgs, AttnArgs, IndexTopkArgs, Mxfp4QuantArgs,
+           IndexCompressArgs]
 
 ENTRY_POINTS = {
     "lc_qk_prep_prefill": QkPrepArgs, "lc_qk_prep_decode": QkPrepArgs,
@@ -99,6 +112,8 @@ ENTRY_POINTS = {
     "lc_csa_index_scores_prefill": IndexArgs, "lc_csa_index_scores_decode": IndexArgs,
     "lc_csa_topk_prefill": TopkArgs, "lc_csa_topk_decode": TopkArgs,
     "lc_csa_index_topk_prefill": IndexTopkArgs, "lc_csa_index_topk_decode": IndexTopkArgs,
+    "lc_mxfp4_quantize": Mxfp4QuantArgs,
+    "lc_csa_index_compress_prefill": IndexCompressArgs, "lc_csa_index_compress_decode": IndexCompressArgs,
     "lc_csa_sparse_attn_prefill": AttnArgs, "lc_csa_sparse_attn_decode": AttnArgs,
     "lc_hca_attn_prefill": AttnArgs, "lc_hca_attn_decode": AttnArgs,
     "lc_csa_sparse_attn_decode_static": AttnArgs,

@@ -116,6 +116,31 @@ lc_status check_index(const lc_index_args* a, bool decode, bool scores) {
   return LC_OK;
 }
 
+lc_status mxfp4_quantize(const lc_mxfp4_quant_args* a, void* stream) {
+  if (!a) return LC_ERR_ARG;
+  if (a->n_rows < 0 || a->d < 32 || a->d > 1024 || a->d % 32) return LC_ERR_ARG;
+  if (a->in_fmt != LC_FMT_F32 && a->in_fmt != LC_FMT_BF16) return LC_ERR_ARG;
+  if (a->n_rows == 0) return LC_OK;
+  if (!a->x || !a->codes || !a->scales) return LC_ERR_ARG;
+  if (!aligned16(a->x) || (reinterpret_cast<uintptr_t>(a->codes) & 15u) || (reinterpret_cast<uintptr_t>(a->scales) & 3u))
+    return LC_ERR_ALIGN;
+  return launched(lc::launch_mxfp4_quantize(*a, static_cast<cudaStream_t>(stream)));
+}
+
+lc_status index_compress(const lc_index_compress_args* a, void* stream) {
+  if (!a) return LC_ERR_ARG;
+  if (a->d_I < 32 || a->d_I > 256 || a->d_I % 32 || a->m < 1 || a->m > 64) return LC_ERR_ARG;
+  if (a->in_fmt != LC_FMT_F32 && a->in_fmt != LC_FMT_BF16) return LC_ERR_ARG;
+  if (a->num_seqs < 0 || a->max_blocks < 0) return LC_ERR_ARG;
+  if (a->num_seqs == 0 || a->max_blocks == 0) return LC_OK;
+  if (!a->x || !a->g || !a->tok_row0 || !a->tok_pos0 || !a->tok_len || !a->blk_first || !a->blk_count ||
+      !a->ent_start || !a->codes || !a->scales)
+    return LC_ERR_ARG;
+  if (!aligned16(a->x) || (reinterpret_cast<uintptr_t>(a->codes) & 15u) || (reinterpret_cast<uintptr_t>(a->scales) & 3u))
+    return LC_ERR_ALIGN;
+  return launched(lc::launch_index_compress(*a, static_cast<cudaStream_t>(stream)));
+}
+
 lc_status index_scores(const lc_index_args* a, void* stream, bool decode) {
   LC_TRY(check_index(a, decode, true));
   if (a->n_q == 0 || a->max_ent == 0) return LC_OK;
@@ -189,6 +214,10 @@ lc_status lc_hca_compress_decode(const lc_compress_args* a, void* stream) { retu
 lc_status lc_csa_index_scores_prefill(const lc_index_args* a, void* stream) { return index_scores(a, stream, false); }
 lc_status lc_csa_index_scores_decode(const lc_index_args* a, void* stream) { return index_scores(a, stream, true); }
 
+lc_status lc_mxfp4_quantize(const lc_mxfp4_quant_args* a, void* stream) { return mxfp4_quantize(a, stream); }
+lc_status lc_csa_index_compress_prefill(const lc_index_compress_args* a, void* stream) { return index_compress(a, stream); }
+lc_status lc_csa_index_compress_decode(const lc_index_compress_args* a, void* stream) { return index_compress(a, stream); }
+
 lc_status lc_csa_index_topk_prefill(const lc_index_topk_args* a, void* stream) { return index_topk(a, stream, false); }
 lc_status lc_csa_index_topk_decode(const lc_index_topk_args* a, void* stream) { return index_topk(a, stream, true); }
 size_t lc_csa_index_topk_workspace_bytes(const lc_index_topk_args* a, int32_t decode) {
@@ -238,6 +267,8 @@ size_t lc_struct_size(int32_t which) {
     case 6: return sizeof(lc_topk_args);
     case 7: return sizeof(lc_attn_args);
     case 8: return sizeof(lc_index_topk_args);
+    case 9: return sizeof(lc_mxfp4_quant_args);
+    case 10: return sizeof(lc_index_compress_args);
     default: return 0;
   }
 }

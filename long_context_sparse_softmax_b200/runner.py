@@ -16,11 +16,13 @@ from typing import Dict, Optional
 
 import torch
 
-from . import (AttnArgs, Batch, CompressArgs, Dims, IndexArgs, IndexTopkArgs, QkPrepArgs, Rows, TopkArgs,
+from . import (AttnArgs, Batch, CompressArgs, Dims, IndexArgs, IndexCompressArgs, IndexTopkArgs, Mxfp4QuantArgs,
+               QkPrepArgs, Rows, TopkArgs,
                LC_FMT_BF16, LC_FMT_E4M3_BF16, LC_FMT_F32, LC_IDX_F32, LC_IDX_MXFP4,
                lc_csa_compress_decode, lc_csa_compress_prefill, lc_csa_index_scores_decode,
                lc_csa_index_scores_prefill, lc_csa_index_topk_decode, lc_csa_index_topk_prefill,
-               lc_csa_index_topk_workspace_bytes, lc_csa_sparse_attn_decode, lc_csa_sparse_attn_prefill,
+               lc_csa_index_topk_workspace_bytes, lc_csa_index_compress_decode, lc_csa_index_compress_prefill,
+               lc_mxfp4_quantize, lc_csa_sparse_attn_decode, lc_csa_sparse_attn_prefill,
                lc_csa_sparse_attn_workspace_bytes, lc_csa_topk_decode, lc_csa_topk_prefill,
                lc_hca_attn_decode, lc_hca_attn_prefill, lc_hca_attn_workspace_bytes,
                lc_hca_compress_decode, lc_hca_compress_prefill, lc_qk_prep_decode, lc_qk_prep_prefill)
@@ -57,33 +59,75 @@ def _round4(n: int) -> int:
 
 
 class _Common:
+    # side stages in groups: a group runs in order on one side stream (its stages share
+    # inputs); groups run concurrently with one another and with the main stages
+    SIDE_GROUPS = (("qk_prep_q",), ("qk_prep_win",), ("compress", "index_compress"))
+
     def dag(self):
-        """The step as three groups: (side, main, after).  `side` (query and window
-        preparation, compression) and `main` (index scores -> top-k) share no buffers and
-        may run concurrently on two streams; `after` (attention) needs both."""
+        """The step as (side groups, main, after).  The side groups (query and window
+        preparation, compression) and `main` (indexer query quantisation, index scores ->
+        top-k) share no buffers that one writes and the other reads in the same step, so
+        they may run concurrently; `after` (attention) needs all of them.  In prefill the
+        indexer keys are compressed on the main stream: the indexer reads them."""
         st = dict(self.stages())
-        side = [(n, st[n]) for n in ("qk_prep_q", "qk_prep_win", "compress") if n in st]
-        main = [(n, st[n]) for n in ("index", "topk", "index_topk") if n in st]
+        main_names = ("index_compress",) if not self.spec.is_decode else ()
+        main_names += ("quant_q", "index", "topk", "index_topk")
+        side = [[(n, st[n]) for n in grp if n in st and n not in main_names] for grp in self.SIDE_GROUPS]
+        side = [g for g in side if g]
+        main = [(n, st[n]) for n in main_names if n in st]
         return side, main, [("attn", st["attn"])]
 
     def host_inputs(self):
         """The device tensors a step reads that a caller refills from the host each step,
         by the stage that first reads them: {stage: [tensors]}.  Tensors that stages on
         different streams share are listed under "_fork" (copied before the fork)."""
-        inp = self.inp
-        qI = list(inp["qI"].values()) if self.spec.is_csa else []
-        if self.spec.is_decode:
+        inp, s = self.inp, self.spec
+        raw = s.is_csa and s.idx_fmt == wl.IDX_MXFP4
+        qI = ([inp["qI_raw"]] if raw else list(inp["qI"].values())) if s.is_csa else []
+        if s.is_decode:
             h = {"qk_prep_q": [inp["q_raw"]], "qk_prep_win": [inp["x_new"]],
                  "compress": [inp["x_tail"], inp["g_tail"]]}
+            if raw:
+                h["index_compress"] = [inp["kI_tail"]]
         else:
             h = {"qk_prep_q": [inp["q_raw"]], "_fork": [inp["x"], inp["g"]]}
+            if raw:
+                h["index_compress"] = [inp["kI_raw"]]
         if qI:
-            h["index_topk" if self.fused else "index"] = qI
+            h["quant_q" if raw else ("index_topk" if self.fused else "index")] = qI
         return h
 
     def host_outputs(self):
         """The step's results a caller reads back: attention output and lse."""
         return [self.out, self.lse]
+
+    def _indexer_buffers(self, n_q: int, n_keys: int, decode: bool):
+        """Indexer operands the step reads: the quantised queries (and, in prefill, the
+        compressed keys) that its own kernels write, or the given FP32 operands."""
+        s, inp, dev = self.spec, self.inp, self.device
+        if s.idx_fmt != wl.IDX_MXFP4:
+            self.qI, self.kI = inp["qI"], inp["kI"]
+            return
+        u8 = dict(dtype=torch.uint8, device=dev)
+        self.qI = {"codes": torch.empty(n_q, s.H_I, s.d_I // 2, **u8), "scales": torch.empty(n_q, s.H_I, s.d_I // 32, **u8)}
+        if decode:
+            self.kI = inp["kI"]
+        else:
+            self.kI = {"codes": torch.empty(max(n_keys, 1), s.d_I // 2, **u8),
+                       "scales": torch.empty(max(n_keys, 1), s.d_I // 32, **u8)}
+        self.a_quant_q = Mxfp4QuantArgs(n_q * s.H_I, s.d_I, LC_FMT_BF16, ptr(inp["qI_raw"]), ptr(self.qI["codes"]),
+                                        ptr(self.qI["scales"]))
+
+    def _index_compress_args(self, x_raw, g, c: Dict[str, torch.Tensor], num_seqs: int, max_blocks: int,
+                             blk_first, blk_count, ent_start) -> IndexCompressArgs:
+        s = self.spec
+        return IndexCompressArgs(s.d_I, s.m, num_seqs, LC_FMT_BF16, max_blocks, 0, ptr(x_raw), ptr(g),
+                                 ptr(c["tok_row0"]), ptr(c["tok_pos0"]), ptr(c["tok_len"]), ptr(blk_first),
+                                 ptr(blk_count), ptr(ent_start), ptr(self.kI["codes"]), ptr(self.kI["scales"]),
+                                 ptr(self.status))
+
+    def quant_q(self, stream=None):
+        lc_mxfp4_quantize(self.a_quant_q, stream)
 
     def step_overlapped(self, main, side, on_stage=None, io=None):
         """One step on several streams: the side stages fork from `main` (stage i on
@@ -111,15 +155,16 @@ class _Common:
                     d.copy_(h, non_blocking=True)
         fork = torch.cuda.Event()
         fork.record(main)
-        used = sides[:len(sd)]
+        used = sides[:min(len(sd), len(sides))]
         for st in used:
             st.wait_event(fork)
         # the critical path is enqueued first, so its CTAs take the SMs before the side
         # streams' do
         for n, f in mn:
             run(n, main, f)
-        for i, (n, f) in enumerate(sd):
-            run(n, sides[i % len(sides)], f)
+        for i, grp in enumerate(sd):
+            for n, f in grp:
+                run(n, sides[i % len(sides)], f)
         for st in used:
             join = torch.cuda.Event()
             join.record(st)
@@ -133,7 +178,7 @@ class _Common:
 
     def _index_args(self, n_q: int, max_ent: int, scores: torch.Tensor) -> IndexArgs:
         s, inp = self.spec, self.inp
-        qI, kI = inp["qI"], inp["kI"]
+        qI, kI = self.qI, self.kI
         mx = s.idx_fmt == wl.IDX_MXFP4
         return IndexArgs(n_q, s.H_I, s.d_I, LC_IDX_MXFP4 if mx else LC_IDX_F32,
                          ptr(qI["codes"] if mx else qI["f32"]), ptr(qI.get("scales")),
@@ -225,6 +270,10 @@ class Prefill(_Common):
         self.out = torch.empty(s.n_q * s.H, s.D, dtype=torch.float32 if s.out_f32 else torch.int16, device=device)
         self.lse = torch.empty(s.n_q * s.H, dtype=torch.float32, device=device)
         if s.is_csa:
+            self._indexer_buffers(s.n_q, n_c, False)
+            if s.idx_fmt == wl.IDX_MXFP4:
+                self.a_index_compress = self._index_compress_args(inp["kI_raw"], inp["g"], c, 1, n_c, c["blk_first"],
+                                                                  c["blk_count"], c["ent_start"])
             self.scores = torch.empty(s.n_q, _round4(n_c), dtype=torch.float32, device=device)
             self.idx = torch.empty(s.n_q, s.k, dtype=torch.int32, device=device)
             self.count = torch.empty(s.n_q, dtype=torch.int32, device=device)
@@ -245,6 +294,9 @@ class Prefill(_Common):
     def compress(self, stream=None):
         (lc_csa_compress_prefill if self.spec.is_csa else lc_hca_compress_prefill)(self.a_compress, stream)
 
+    def index_compress(self, stream=None):
+        lc_csa_index_compress_prefill(self.a_index_compress, stream)
+
     def index(self, stream=None):
         lc_csa_index_scores_prefill(self.a_index, stream)
 
@@ -258,8 +310,11 @@ class Prefill(_Common):
         (lc_csa_sparse_attn_prefill if self.spec.is_csa else lc_hca_attn_prefill)(self.a_attn, stream)
 
     def stages(self):
+        s = self.spec
         st = [("qk_prep_q", self.prep_queries), ("qk_prep_win", self.prep_window), ("compress", self.compress)]
-        if self.spec.is_csa:
+        if s.is_csa:
+            if s.idx_fmt == wl.IDX_MXFP4:
+                st += [("index_compress", self.index_compress), ("quant_q", self.quant_q)]
             st += [("index_topk", self.index_topk)] if self.fused else [("index", self.index), ("topk", self.topk)]
         return st + [("attn", self.attn)]
 
@@ -307,6 +362,11 @@ class Decode(_Common):
         self.out = torch.empty(B * s.H, s.D, dtype=torch.float32 if s.out_f32 else torch.int16, device=device)
         self.lse = torch.empty(B * s.H, dtype=torch.float32, device=device)
         if s.is_csa:
+            self._indexer_buffers(B, sum(n_c), True)
+            if s.idx_fmt == wl.IDX_MXFP4:
+                self.a_index_compress = self._index_compress_args(inp["kI_tail"], inp["g_tail"], c, B, 1,
+                                                                  inp["blk_first"], inp["blk_count"],
+                                                                  inp["batch"]["ent_start"])
             self.scores = torch.empty(B, _round4(max_ent), dtype=torch.float32, device=device)
             self.idx = torch.empty(B, s.k, dtype=torch.int32, device=device)
             self.count = torch.empty(B, dtype=torch.int32, device=device)
@@ -327,6 +387,9 @@ class Decode(_Common):
     def compress(self, stream=None):
         (lc_csa_compress_decode if self.spec.is_csa else lc_hca_compress_decode)(self.a_compress, stream)
 
+    def index_compress(self, stream=None):
+        lc_csa_index_compress_decode(self.a_index_compress, stream)
+
     def index(self, stream=None):
         lc_csa_index_scores_decode(self.a_index, stream)
 
@@ -340,8 +403,11 @@ class Decode(_Common):
         (lc_csa_sparse_attn_decode if self.spec.is_csa else lc_hca_attn_decode)(self.a_attn, stream)
 
     def stages(self):
+        s = self.spec
         st = [("qk_prep_q", self.prep_queries), ("qk_prep_win", self.prep_window), ("compress", self.compress)]
-        if self.spec.is_csa:
+        if s.is_csa:
+            if s.idx_fmt == wl.IDX_MXFP4:
+                st += [("index_compress", self.index_compress), ("quant_q", self.quant_q)]
             st += [("index_topk", self.index_topk)] if self.fused else [("index", self.index), ("topk", self.topk)]
         return st + [("attn", self.attn)]
 

@@ -7,8 +7,8 @@ Two pieces of input preparation do live here, because the path consumes their
 output as given data:
 
 * casts of N(0,1) draws to the storage types (torch's own casts), and
-* MXFP4 encoding of the lightning-indexer queries and keys (the path reads MXFP4
-  bytes; it never quantises).
+* MXFP4 encoding of the indexer keys already in a decode cache (the path quantises the
+  indexer queries and the keys of new blocks itself, from raw BF16 rows).
 
 Shapes follow the DeepSeek-V4 pages: m = 4 (CSA) and m' = 128 (HCA), a 128-token
 window, top-k 512 (Flash) / 1024 (Pro), 576-dim entries with 64 RoPE dims kept in
@@ -237,7 +237,9 @@ def make_prefill(spec: Spec, device="cpu") -> Dict[str, object]:
     """One sequence, raw tokens given; entries and window rows are computed by the path.
 
     Tensors: x [L, D] raw token KV, g [L] gate logits, q_raw [n_q, H, D], the
-    indexer operands qI [n_q, H_I, d_I] and kI [n_c, d_I] (CSA), w [H_I], sink [H].
+    indexer rows (CSA; MXFP4 workloads: raw BF16 qI_raw [n_q, H_I, d_I] and per-token
+    kI_raw [L, d_I], which the path quantises and pools; FP32: qI and kI [n_c, d_I]
+    given directly), w [H_I], sink [H].
     """
     (L,) = spec.seq_lens
     s = spec
@@ -249,8 +251,14 @@ def make_prefill(spec: Spec, device="cpu") -> Dict[str, object]:
     n_c = s.n_entries(L)
     out["n_c"] = n_c
     if s.is_csa:
-        out["qI"] = _indexer_operand(s, "qI", (s.n_q, s.H_I, s.d_I), device)
-        out["kI"] = _indexer_operand(s, "kI", (n_c, s.d_I), device)
+        if s.idx_fmt == IDX_MXFP4:
+            # raw indexer rows: the path quantises the queries and pools + quantises the
+            # keys of every complete block itself
+            out["qI_raw"] = to_bf16_bits(randn(s.seed, "qI", (s.n_q, s.H_I, s.d_I), device))
+            out["kI_raw"] = to_bf16_bits(randn(s.seed, "kI", (L, s.d_I), device))
+        else:
+            out["qI"] = _indexer_operand(s, "qI", (s.n_q, s.H_I, s.d_I), device)
+            out["kI"] = _indexer_operand(s, "kI", (n_c, s.d_I), device)
         out["w"] = rand(s.seed, "w", (s.H_I,), device)
     # positions and the batch descriptor (one sequence)
     q_pos = torch.arange(s.q_first, s.q_first + s.n_q, dtype=torch.int32, device=device)
@@ -278,7 +286,10 @@ def make_decode(spec: Spec, device="cpu") -> Dict[str, object]:
     (nope E4M3 + RoPE BF16, or FP32), prepped window rows [B*W, D] for positions
     L_b - W .. L_b - 1 (BF16 or FP32), indexer keys kI [sum n_c, d_I].  The newest
     block's raw tokens (x_tail [B, m, D], g_tail [B, m]) and the newest token's raw
-    row x_new [B, D] feed the decode-time compression and window preparation.
+    row x_new [B, D] feed the decode-time compression and window preparation.  MXFP4
+    workloads give the query's raw indexer rows (qI_raw [B, H_I, d_I] BF16) and the
+    newest block's raw indexer-key rows (kI_tail [B, m, d_I] BF16) for the step to
+    quantise and pool.
     """
     s = spec
     B = s.num_seqs
@@ -298,7 +309,13 @@ def make_decode(spec: Spec, device="cpu") -> Dict[str, object]:
     out["g_tail"] = randn(s.seed, "g_tail", (B, s.m), device)
     out["sink"] = randn(s.seed, "sink", (s.H,), device)
     if s.is_csa:
-        out["qI"] = _indexer_operand(s, "qI", (B, s.H_I, s.d_I), device)
+        if s.idx_fmt == IDX_MXFP4:
+            # the step quantises the query's raw indexer rows and pools + quantises the
+            # indexer key of the block the newest token closed
+            out["qI_raw"] = to_bf16_bits(randn(s.seed, "qI", (B, s.H_I, s.d_I), device))
+            out["kI_tail"] = to_bf16_bits(randn(s.seed, "kI_tail", (B, s.m, s.d_I), device))
+        else:
+            out["qI"] = _indexer_operand(s, "qI", (B, s.H_I, s.d_I), device)
         out["kI"] = _indexer_operand(s, "kI", (tot, s.d_I), device)
         out["w"] = rand(s.seed, "w", (s.H_I,), device)
     out["q_pos"] = _i32([L - 1 for L in s.seq_lens], device)

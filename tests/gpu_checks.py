@@ -24,7 +24,7 @@ import torch
 from oracle import lc_oracle as O
 from long_context_sparse_softmax_b200 import runner
 from long_context_sparse_softmax_b200 import workloads as wl
-from tests.oracle_ref import (OracleDecode, OraclePrefill, attn_err_in_ulps, attn_ok, np_, out_np,
+from tests.oracle_ref import (OracleDecode, OraclePrefill, attn_err_in_ulps, attn_ok, mxfp4_check, np_, out_np,
                               perturbation_bound, rows_np, stored_check, topk_sets_ok, write_rows)
 
 
@@ -97,16 +97,27 @@ def check_prefill(spec: wl.Spec, q_sel: Sequence[int] = None, W_x: int = None, r
     orc_idx = {}
     if spec.is_csa:
         scores_gpu = np_(run.scores[sel_t])
+        lib_kI = None
+        if spec.idx_fmt == wl.IDX_MXFP4:
+            # indexer queries quantised by the path (exact inputs: bit-exact), keys pooled
+            # and quantised by the path (FP32 pooling: within one grid step)
+            assert np.array_equal(np_(run.qI["codes"][sel_t]), orc.qI_codes), "quantised indexer query codes"
+            assert np.array_equal(np_(run.qI["scales"][sel_t]), orc.qI_scales), "quantised indexer query scales"
+            kc, ks = np_(run.kI["codes"][:n_c]), np_(run.kI["scales"][:n_c])
+            rep["index_keys_flip_frac"] = mxfp4_check(kc, ks, orc.kI_codes, orc.kI_scales, "indexer keys")
+            lib_kI = O.mxfp4_to_f64(kc, ks)
         s_or = {}
         n_diff = 0
         for i, q in enumerate(q_sel):
-            s, bnd = orc.scores(i)
+            # scores on the path's own indexer operands; the selection against the oracle's
+            s, bnd = orc.scores(i, lib_kI)
+            s_o, bnd_o = orc.scores(i) if lib_kI is not None else (s, bnd)
             s_or[i] = s
             g = scores_gpu[i, :s.shape[0]].astype(np.float64)
             assert np.all(np.abs(g - s) <= bnd), f"scores of query {q}: max err {np.max(np.abs(g - s))}"
-            exp_idx[i] = O.topk(s, spec.k)
+            exp_idx[i] = O.topk(s_o, spec.k)
             orc_idx[i] = exp_idx[i]
-            ok_i, nd, why = topk_sets_ok(e2e_idx[i], exp_idx[i], s, spec.k, spec.fp32, bnd)
+            ok_i, nd, why = topk_sets_ok(e2e_idx[i], exp_idx[i], s_o, spec.k, spec.fp32, bnd_o)
             assert ok_i, f"top-k of query {q}: {why}"
             n_diff += nd
         rep["topk_e2e_set_diff"] = n_diff
@@ -250,16 +261,25 @@ def check_decode(spec: wl.Spec, W_x: int = None, report=None, impl: int = 0):
     if spec.is_csa:
         e2e_idx = np_(run.idx)
         scores_gpu = np_(run.scores)
+        lib_kI = None
+        if spec.idx_fmt == wl.IDX_MXFP4:
+            assert np.array_equal(np_(run.qI["codes"]), orc.qI_codes), "quantised indexer query codes"
+            assert np.array_equal(np_(run.qI["scales"]), orc.qI_scales), "quantised indexer query scales"
+            lib_kI = {"codes": np_(run.kI["codes"]), "scales": np_(run.kI["scales"])}
+            for b, (r, c, sc) in orc.new_key.items():
+                mxfp4_check(lib_kI["codes"][r:r + 1], lib_kI["scales"][r:r + 1], c[None], sc[None],
+                            f"indexer key of the block sequence {b} closed")
         s_or = {}
         n_diff = 0
         for b in range(B):
-            s, bnd = orc.scores(b)
+            s, bnd = orc.scores(b, lib_kI)
+            s_o, bnd_o = orc.scores(b) if lib_kI is not None else (s, bnd)
             s_or[b] = s
             g = scores_gpu[b, :s.shape[0]].astype(np.float64)
             assert np.all(np.abs(g - s) <= bnd), f"scores of sequence {b}: max err {np.max(np.abs(g - s))}"
-            exp_idx[b] = O.topk(s, spec.k)
+            exp_idx[b] = O.topk(s_o, spec.k)
             orc_idx[b] = exp_idx[b]
-            ok_b, nd, why = topk_sets_ok(e2e_idx[b], exp_idx[b], s, spec.k, spec.fp32, bnd)
+            ok_b, nd, why = topk_sets_ok(e2e_idx[b], exp_idx[b], s_o, spec.k, spec.fp32, bnd_o)
             assert ok_b, f"top-k of sequence {b}: {why}"
             n_diff += nd
         rep["topk_e2e_set_diff"] = n_diff

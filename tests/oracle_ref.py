@@ -79,6 +79,23 @@ def stored_check(fmt: int, got_f64: np.ndarray, exp_f64: np.ndarray, d_n: int, w
     return frac
 
 
+def mxfp4_check(lib_codes, lib_scales, orc_codes, orc_scales, what: str) -> float:
+    """Acceptance of MXFP4 values the path computed from FP32 intermediates (pooled indexer
+    keys): each element within one E2M1 grid step (at the larger of the two block scales,
+    which differ only where the block maximum sits at a power of two) of the oracle's,
+    and few elements differing at all.  Returns the fraction that differ."""
+    dl = O.mxfp4_to_f64(lib_codes, lib_scales)
+    do = O.mxfp4_to_f64(orc_codes, orc_scales)
+    X = np.repeat(np.exp2(np.maximum(lib_scales, orc_scales).astype(np.float64) - 127), 32, axis=-1)
+    mag = np.maximum(np.abs(dl), np.abs(do)) / X
+    step = np.where(mag < 2, 0.5, np.where(mag < 4, 1.0, 2.0)) * X
+    ok = np.abs(dl - do) <= step + FP32_EVAL_ABS * np.abs(do)
+    assert ok.all(), f"{what}: {(~ok).sum()} elements beyond one grid step"
+    n_diff = int(np.sum(dl != do))
+    assert n_diff <= MAX_FLIP_FRACTION * dl.size + 32, f"{what}: {n_diff} of {dl.size} values differ"
+    return n_diff / dl.size if dl.size else 0.0
+
+
 def rows_np(fmt: int, r: Dict[str, torch.Tensor], sel=None) -> np.ndarray:
     x = r["x"] if sel is None else r["x"][sel]
     rope = r.get("rope")
@@ -217,15 +234,25 @@ class OraclePrefill:
         self.q_f, _, _ = P.stored(s.q_fmt, O.qk_prep(qr, np.array(self.pos), lo, d_r), d_n)
         if s.is_csa:
             sel_t = torch.as_tensor(self.q_sel, device=inp["q_raw"].device)
-            self.qI = P.indexer_f64(s.idx_fmt, idx_operand_np(inp["qI"], sel_t))
-            self.kI = P.indexer_f64(s.idx_fmt, idx_operand_np(inp["kI"]))
+            if s.idx_fmt == O.IDX_MXFP4:
+                # the path quantises the raw indexer queries and pools + quantises the keys
+                self.qI_codes, self.qI_scales = O.f64_to_mxfp4(O.bf16_to_f64(np_(inp["qI_raw"][sel_t])))
+                self.qI = O.mxfp4_to_f64(self.qI_codes, self.qI_scales)
+                pooled = O.pool_index_keys(O.bf16_to_f64(np_(inp["kI_raw"])), g, s.m)
+                self.kI_codes, self.kI_scales = O.f64_to_mxfp4(pooled.reshape(-1, s.d_I))
+                self.kI = O.mxfp4_to_f64(self.kI_codes, self.kI_scales)
+            else:
+                self.qI = P.indexer_f64(s.idx_fmt, idx_operand_np(inp["qI"], sel_t))
+                self.kI = P.indexer_f64(s.idx_fmt, idx_operand_np(inp["kI"]))
             self.w = np_(inp["w"]).astype(np.float64)
 
-    def scores(self, i: int):
-        """Visible scores of sampled query i, and their FP32 error bound."""
+    def scores(self, i: int, kI: np.ndarray = None):
+        """Visible scores of sampled query i, and their FP32 error bound (on the oracle's
+        indexer keys, or on the decoded keys `kI` of another path)."""
         p = self.pos[i]
-        s, n_vis = P.visible_scores(self.qI[i], self.kI, self.w, p, self.s.m, self.W_x)
-        return s, O.score_error_bound(self.qI[i], self.kI[:n_vis], self.w)
+        kI = self.kI if kI is None else kI
+        s, n_vis = P.visible_scores(self.qI[i], kI, self.w, p, self.s.m, self.W_x)
+        return s, O.score_error_bound(self.qI[i], kI[:n_vis], self.w)
 
     def select(self, i: int, s_vis: np.ndarray = None):
         if s_vis is None:
@@ -307,20 +334,39 @@ class OracleDecode:
         qr = P.raw_rows(s.raw_fmt, np_(inp["q_raw"]))
         self.q_f, _, _ = P.stored(s.q_fmt, O.qk_prep(qr, np.array(self.pos), lo, d_r), d_n)
         if s.is_csa:
-            self.qI = P.indexer_f64(s.idx_fmt, idx_operand_np(inp["qI"]))
             kI_np = idx_operand_np(inp["kI"])
+            self.new_key = {}
+            if s.idx_fmt == O.IDX_MXFP4:
+                # the step quantises the query's raw indexer rows ...
+                self.qI_codes, self.qI_scales = O.f64_to_mxfp4(O.bf16_to_f64(np_(inp["qI_raw"])))
+                self.qI = O.mxfp4_to_f64(self.qI_codes, self.qI_scales)
+                # ... and pools + quantises the indexer key of the block the newest token closed
+                kt = O.bf16_to_f64(np_(inp["kI_tail"]))
+                kI_np = {k: v.copy() for k, v in kI_np.items()}
+                for b, L in enumerate(s.seq_lens):
+                    if self.blk_count[b]:
+                        j = L // s.m - 1
+                        key = O.pool_index_keys(kt[b], gt[b], s.m, first_block=j, tok_pos0=L - s.m, n_blocks=1)
+                        c, sc = O.f64_to_mxfp4(key)
+                        r = self.ent_start[b] + j
+                        kI_np["codes"][r], kI_np["scales"][r] = c[0], sc[0]
+                        self.new_key[b] = (r, c[0], sc[0])
+            else:
+                self.qI = P.indexer_f64(s.idx_fmt, idx_operand_np(inp["qI"]))
             self.kI_np = kI_np
             self.w = np_(inp["w"]).astype(np.float64)
 
-    def kI(self, b: int):
+    def kI(self, b: int, kI_np=None):
+        """Decoded indexer keys of sequence b (the oracle's, or another path's kI_np)."""
+        kI_np = self.kI_np if kI_np is None else kI_np
         n0, n = self.ent_start[b], self.n_c[b]
         s = self.s
         if s.idx_fmt == O.IDX_F32:
-            return self.kI_np["f32"][n0:n0 + n].astype(np.float64)
-        return O.mxfp4_to_f64(self.kI_np["codes"][n0:n0 + n], self.kI_np["scales"][n0:n0 + n])
+            return kI_np["f32"][n0:n0 + n].astype(np.float64)
+        return O.mxfp4_to_f64(kI_np["codes"][n0:n0 + n], kI_np["scales"][n0:n0 + n])
 
-    def scores(self, b: int):
-        kI = self.kI(b)
+    def scores(self, b: int, kI_np=None):
+        kI = self.kI(b, kI_np)
         s, n_vis = P.visible_scores(self.qI[b], kI, self.w, self.pos[b], self.s.m, self.W_x)
         return s, O.score_error_bound(self.qI[b], kI[:n_vis], self.w)
 

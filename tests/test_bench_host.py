@@ -36,17 +36,24 @@ def test_host_inputs_name_the_stage_that_reads_them():
     assert h["qk_prep_q"][0] is inp["q_raw"]
     assert h["qk_prep_win"][0] is inp["x_new"]
     assert h["compress"][0] is inp["x_tail"] and h["compress"][1] is inp["g_tail"]
-    # MXFP4 indexer operands: index and top-k run fused, and the indexer queries feed that stage
-    assert r.fused and [n for n, _ in r.stages()][3:] == ["index_topk", "attn"]
-    assert set(map(id, h["index_topk"])) == set(map(id, inp["qI"].values()))
+    # MXFP4 indexer: the step quantises the raw query rows and pools + quantises the key
+    # of the closed block; index and top-k run fused
+    assert r.fused and [n for n, _ in r.stages()][3:] == ["index_compress", "quant_q", "index_topk", "attn"]
+    assert h["quant_q"][0] is inp["qI_raw"] and h["index_compress"][0] is inp["kI_tail"]
+    side, main, after = r.dag()
+    assert [[n for n, _ in g] for g in side] == [["qk_prep_q"], ["qk_prep_win"], ["compress", "index_compress"]]
+    assert [n for n, _ in main] == ["quant_q", "index_topk"] and after[0][0] == "attn"
     r2 = runner.Decode(inp, "cpu", fused=False)
-    assert [n for n, _ in r2.stages()][3:] == ["index", "topk", "attn"]
-    assert set(map(id, r2.host_inputs()["index"])) == set(map(id, inp["qI"].values()))
+    assert [n for n, _ in r2.stages()][3:] == ["index_compress", "quant_q", "index", "topk", "attn"]
     assert r.host_outputs() == [r.out, r.lse]
     # prefill: the raw tokens feed both window preparation and compression (two side
     # streams), so they are copied before the fork
     p = wl.shrink(wl.CSA_PREFILL, name="host_io_prefill", seq_lens=(600,), H=16, k=32, n_q=600)
     ip = wl.make_prefill(p, "cpu")
-    hp = runner.Prefill(ip, "cpu").host_inputs()
+    rp = runner.Prefill(ip, "cpu")
+    hp = rp.host_inputs()
     assert hp["_fork"][0] is ip["x"] and hp["_fork"][1] is ip["g"]
     assert "qk_prep_win" not in hp and "compress" not in hp
+    # prefill compresses the indexer keys on the main stream, before the indexer reads them
+    assert hp["index_compress"][0] is ip["kI_raw"] and hp["quant_q"][0] is ip["qI_raw"]
+    assert [n for n, _ in rp.dag()[1]] == ["index_compress", "quant_q", "index_topk"]

@@ -27,9 +27,10 @@ def _visible(run):
 
 
 def _check(run):
-    """Fused selection against the oracle's top-k of the separate call's scores."""
+    """Fused selection (a whole step: the indexer operands are quantised and pooled by
+    the step's own kernels) against the oracle's top-k of the separate call's scores."""
     k = run.spec.k
-    run.index_topk()
+    run.step()
     torch.cuda.synchronize()
     fused = run.idx.cpu().numpy()
     cnt = run.count.cpu().numpy()
@@ -77,7 +78,7 @@ def test_fused_decode_identical_keys_take_the_lowest_indices():
 
 def test_fused_decode_zero_queries_tie_everywhere():
     def zero_q(inp):
-        inp["qI"]["codes"].zero_()
+        inp["qI_raw"].zero_()
     _check(_decode((40000, 9000), 512, 84, zero_q))
 
 
