@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="launch every call from Python each step "
                     "instead of replaying the step's CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fused", action="store_true", help="run the indexer and top-k as two calls "
+                    "(scores written) instead of the fused index + top-k call")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0)
     ap.add_argument("--attn-impl", default="auto", choices=["auto", "tc", "ref"],
                     help="attention kernel (auto: tcgen05 where it applies, else the FP32 reference kernel)")
@@ -289,14 +291,14 @@ def kernel_traffic(workload: str, stage: str, attn_impl: str):
 # ------------------------------------------------------------------------------------
 # the library arm
 # ------------------------------------------------------------------------------------
-def make_runs(name, device, rank, impl=0):
+def make_runs(name, device, rank, impl=0, fused=None):
     from long_context_sparse_softmax_b200 import runner
     from long_context_sparse_softmax_b200 import workloads as wl
     runs = []
     for spec in wl.WORKLOADS[name]:
         spec = rank_spec(spec, rank)
         inp = (wl.make_decode if spec.is_decode else wl.make_prefill)(spec, device)
-        r = (runner.Decode if spec.is_decode else runner.Prefill)(inp, device, None, impl)
+        r = (runner.Decode if spec.is_decode else runner.Prefill)(inp, device, None, impl, fused)
         runs.append((spec, inp, r))
     return runs
 
@@ -324,7 +326,8 @@ def run_lc(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     pk, pk_kind = peaks()
-    runs = make_runs(args.workload, dev, rank, {"auto": 0, "tc": 2, "ref": 3}[args.attn_impl])
+    runs = make_runs(args.workload, dev, rank, {"auto": 0, "tc": 2, "ref": 3}[args.attn_impl],
+                     False if args.no_fused else None)
     # L2 flush: a 512 MiB write, then a 256 MiB read so that the lines the step evicts are
     # clean (the write alone would leave L2 full of dirty lines whose write-back lands on
     # the first kernel of the step)

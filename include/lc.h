@@ -110,7 +110,12 @@ typedef struct lc_dims {
 /* Ragged batch descriptor: device arrays, one entry per sequence. */
 typedef struct lc_batch {
   int32_t num_seqs;
-  int32_t reserved;
+  int32_t win_ring;         /* host value.  0: window position t of b is row
+                               win_start[b] + (t - win_pos0[b]).  R > 0: the window rows of b
+                               are a ring buffer of R rows, position t in row
+                               win_start[b] + t mod R (R >= W; the tensor-core kernels take
+                               R a multiple of 64).  Either way positions win_pos0[b] ..
+                               win_pos0[b] + win_len[b] - 1 are present. */
   const int32_t* q_start;   /* [num_seqs + 1] queries of b are q_start[b] .. q_start[b+1]-1 */
   const int32_t* q_pos0;    /* [num_seqs] position of the first query of b; query i of b
                                sits at q_pos0[b] + (i - q_start[b]) */

@@ -42,7 +42,7 @@ class Dims(ctypes.Structure):
 
 
 class Batch(ctypes.Structure):
-    _fields_ = [("num_seqs", c_int32), ("reserved", c_int32), ("q_start", c_void_p), ("q_pos0", c_void_p),
+    _fields_ = [("num_seqs", c_int32), ("win_ring", c_int32), ("q_start", c_void_p), ("q_pos0", c_void_p),
                 ("ent_start", c_void_p), ("n_ent", c_void_p), ("win_start", c_void_p), ("win_pos0", c_void_p),
                 ("win_len", c_void_p)]
 

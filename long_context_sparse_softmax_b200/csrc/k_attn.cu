@@ -105,13 +105,14 @@ __global__ void __launch_bounds__(256) k_attn_ref(lc_attn_args a, int sparse) {
   if (a.W > 0) {
     const int wp0 = __ldg(a.batch.win_pos0 + b), wl = __ldg(a.batch.win_len + b);
     const int64_t wr0 = __ldg(a.batch.win_start + b);
+    const int ring = a.batch.win_ring;
     for (int t = max(0, p - a.W + 1); t <= p; ++t) {
       const int r = t - wp0;
       if (r < 0 || r >= wl) {
         if (lane == 0) set_status(a.status, LC_DEV_WINDOW_RANGE);
         continue;
       }
-      attend_row(st, qv, a.win, wr0 + r, D, d_r, lane, a.scale);
+      attend_row(st, qv, a.win, wr0 + (ring > 0 ? t % ring : r), D, d_r, lane, a.scale);
     }
   }
   const float inv = 1.f / st.z;

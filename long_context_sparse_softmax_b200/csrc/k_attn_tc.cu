@@ -291,12 +291,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return j;
     }
-    const int rr = wlo + (s - n_first) - wp0;
+    const int t = wlo + (s - n_first);
+    const int rr = t - wp0;
     if (rr < 0 || rr >= wl) {
       set_status(a.status, LC_DEV_WINDOW_RANGE);
       return -1;
     }
-    return static_cast<int>(kWin) | rr;
+    // row of position t within the sequence's window rows (linear, or a ring buffer)
+    return static_cast<int>(kWin) | (a.batch.win_ring > 0 ? t % a.batch.win_ring : rr);
   };
 
   // ---- set-up: tensor memory, barriers ----

@@ -193,8 +193,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nv = n_visible(p, a.m, a.W_x, n_ent);
   const int64_t ent0 = __ldg(a.batch.ent_start + b);
   const int wlo = a.W > 0 ? max(0, p - a.W + 1) : p + 1;
+  // window slots start at position wbase: wlo, or, for a ring buffer, wlo rounded down to a
+  // multiple of 64, so that every 64-position window tile is 64 consecutive ring rows
+  // (positions below wlo are masked)
+  const int ring = a.batch.win_ring;
+  const int wbase = ring > 0 ? (wlo & ~(kTK - 1)) : wlo;
   const int n_first = sparse ? a.k : nv;
-  const int n_slots = n_first + (p + 1 - wlo);
+  const int n_slots = n_first + (p + 1 - wbase);
   int s_begin, s_end;
   if (!geo.win_own) {
     s_begin = split * geo.sps;
@@ -249,12 +254,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return j;
     }
-    const int rr = wlo + (s - n_first) - wp0;
+    const int t = wbase + (s - n_first);
+    if (t < wlo) return -1;  // ring alignment: before the window
+    const int rr = t - wp0;
     if (rr < 0 || rr >= wl) {
       set_status(a.status, LC_DEV_WINDOW_RANGE);
       return -1;
     }
-    return static_cast<int>(kWin) | rr;
+    return static_cast<int>(kWin) | (ring > 0 ? t % ring : rr);
   };
 
   // ---- set-up ----
@@ -458,7 +465,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ct == 0) {
           const uint32_t wb = su32(&bars.wfull);
           mbar_expect_tx(wb, kTile);
-          const int y = static_cast<int>(wr0) + wlo + (tile_slot0(t) - n_first) - wp0;
+          const int t0 = wbase + (tile_slot0(t) - n_first);  // first position of the tile
+          const int y = static_cast<int>(wr0) + (ring > 0 ? t0 % ring : t0 - wp0);
 #pragma unroll
           for (int cb = 0; cb < kD / 64; ++cb) tma_tile2d(su32(Vt + cb * kBlk), &twin, cb * 64, y, wb);
         }
@@ -788,6 +796,7 @@ bool attn_tc8_supported(const lc_attn_args& a) {
   if (a.dims.D != kD || a.dims.d_r != kDR || a.dims.H % kNR || a.n_ent_rows < 1) return false;
   if (a.q.fmt != LC_FMT_E4M3_BF16 || a.ent.fmt != LC_FMT_E4M3_BF16) return false;
   if (a.W > 0 && (a.win.fmt != LC_FMT_BF16 || a.n_win_rows < 1)) return false;
+  if (a.batch.win_ring > 0 && a.batch.win_ring % kTK) return false;
   auto al = [](const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; };
   if (!al(a.q.x) || !al(a.q.rope) || !al(a.ent.x) || !al(a.ent.rope) || (a.W > 0 && !al(a.win.x))) return false;
   if (!al(a.out) || !al(a.workspace)) return false;
@@ -804,7 +813,9 @@ bool attn_tc8_supported(const lc_attn_args& a) {
 static AttnTc8Geom tc8_geometry(const lc_attn_args& a, bool sparse, bool decode) {
   AttnTc8Geom g{1, 0, 0, 0};
   const int ne = sparse ? a.k : a.max_ent;
-  const int ns = max(ne + a.W, 1);
+  // window slots: W, or up to W + 63 when ring-aligned window tiles start before the window
+  const int wslots = a.W > 0 && a.batch.win_ring > 0 ? a.W + kTK - 1 : a.W;
+  const int ns = max(ne + wslots, 1);
   const int tiles = (ns + kTK - 1) / kTK;
   g.sps = tiles * kTK;
   const int ctas = a.n_q * (a.dims.H / kNR);
@@ -814,7 +825,7 @@ static AttnTc8Geom tc8_geometry(const lc_attn_args& a, bool sparse, bool decode)
     const int per = (tiles + n - 1) / n;
     g.n_split = (tiles + per - 1) / per;
     g.sps = per * kTK;
-    const int te = (ne + kTK - 1) / kTK, tw = (a.W + kTK - 1) / kTK;
+    const int te = (ne + kTK - 1) / kTK, tw = (wslots + kTK - 1) / kTK;
     if (a.W > 0 && n >= 2 && te >= 1) {
       const int per_e = (te + n - 2) / (n - 1);
       // cost in entry-tile units: uniform splits put up to one window tile next to `per`

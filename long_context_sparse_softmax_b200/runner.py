@@ -50,7 +50,8 @@ def rows(fmt: int, r: Dict[str, torch.Tensor]) -> Rows:
 
 
 def batch(bd: Dict[str, torch.Tensor]) -> Batch:
-    return Batch(int(bd["n_ent"].numel()), 0, ptr(bd["q_start"]), ptr(bd["q_pos0"]), ptr(bd["ent_start"]),
+    return Batch(int(bd["n_ent"].numel()), int(bd.get("win_ring", 0)), ptr(bd["q_start"]), ptr(bd["q_pos0"]),
+                 ptr(bd["ent_start"]),
                  ptr(bd["n_ent"]), ptr(bd["win_start"]), ptr(bd["win_pos0"]), ptr(bd["win_len"]))
 
 
@@ -355,7 +356,9 @@ class Decode(_Common):
                                        rows(s.kv_fmt, self.ent), RMS_EPS, ROPE_BASE, ptr(self.status))
         self.a_prep_q = QkPrepArgs(self.dims, B, s.raw_fmt, ptr(inp["q_raw"]), ptr(inp["q_pos"]), None,
                                    rows(s.q_fmt, self.q), RMS_EPS, ROPE_BASE, ptr(self.status))
-        self.win_slot = torch.tensor([b * s.W + (Lb - 1 - max(0, Lb - s.W)) for b, Lb in enumerate(L)], **i64)
+        # the newest token's window row: its ring slot, or the last row of the linear window
+        self.win_slot = torch.tensor([b * s.W + ((Lb - 1) % s.W if s.ring else Lb - 1 - max(0, Lb - s.W))
+                                      for b, Lb in enumerate(L)], **i64)
         self.a_prep_win = QkPrepArgs(Dims(s.D, s.d_r, s.rope_off, 1), B, s.raw_fmt, ptr(inp["x_new"]),
                                      ptr(inp["q_pos"]), ptr(self.win_slot), rows(s.win_fmt, self.win), RMS_EPS,
                                      ROPE_BASE, ptr(self.status))

@@ -62,6 +62,7 @@ class Spec:
     q_first: int = 0
     n_q: int = 0
     overlap: bool = False    # window/compressed overlap reading (W_x = 0)
+    ring: bool = True        # decode: each sequence's window rows are a ring of W rows
 
     @property
     def d_n(self) -> int:
@@ -284,7 +285,8 @@ def make_decode(spec: Spec, device="cpu") -> Dict[str, object]:
 
     Cache tensors are drawn directly in their storage formats: compressed entries
     (nope E4M3 + RoPE BF16, or FP32), prepped window rows [B*W, D] for positions
-    L_b - W .. L_b - 1 (BF16 or FP32), indexer keys kI [sum n_c, d_I].  The newest
+    L_b - W .. L_b - 1 (BF16 or FP32; with spec.ring a ring buffer of W rows per
+    sequence, position t in row b W + t mod W), indexer keys kI [sum n_c, d_I].  The newest
     block's raw tokens (x_tail [B, m, D], g_tail [B, m]) and the newest token's raw
     row x_new [B, D] feed the decode-time compression and window preparation.  MXFP4
     workloads give the query's raw indexer rows (qI_raw [B, H_I, d_I] BF16) and the
@@ -301,7 +303,14 @@ def make_decode(spec: Spec, device="cpu") -> Dict[str, object]:
     out: Dict[str, object] = {"spec": s, "n_c": n_c}
     out["cache"] = _synthetic_cache(s, tot, "cache", device)
     win_rows = B * s.W
-    wv = randn(s.seed, "win", (win_rows, s.D), device)
+    wv = randn(s.seed, "win", (win_rows, s.D), device)   # row b W + i: position win_pos0[b] + i
+    if s.ring:
+        # ring buffer of W rows per sequence: position t in slot t mod W
+        slot = torch.tensor([b * s.W + (max(0, L - s.W) + i) % s.W for b, L in enumerate(s.seq_lens)
+                             for i in range(s.W)], dtype=torch.int64, device=device)
+        ring = torch.empty_like(wv)
+        ring[slot] = wv
+        wv = ring
     out["win"] = wv if s.win_fmt == FMT_F32 else to_bf16_bits(wv)
     out["q_raw"] = _raw_rows(s, "q", (B, s.H, s.D), device)
     out["x_new"] = _raw_rows(s, "x_new", (B, s.D), device)
@@ -327,6 +336,7 @@ def make_decode(spec: Spec, device="cpu") -> Dict[str, object]:
         "win_start": _i64([b * s.W for b in range(B)], device),
         "win_pos0": _i32([max(0, L - s.W) for L in s.seq_lens], device),
         "win_len": _i32([min(s.W, L) for L in s.seq_lens], device),
+        "win_ring": s.W if s.ring and s.W > 0 else 0,
     }
     # the newest block completes at the current token only when m divides L_b
     out["blk_count"] = _i32([1 if L % s.m == 0 else 0 for L in s.seq_lens], device)

@@ -321,8 +321,13 @@ class OracleDecode:
                 f, _, _ = P.stored(s.kv_fmt, y, d_n)
                 self.new_entry[b] = f[0]
                 self.ent_f[self.ent_start[b] + j] = f[0]
-        # window rows: the cached rows, with the newest token prepared from x_new
+        # window rows in position order (read through the ring when the cache is one), with
+        # the newest token prepared from x_new
         self.win_f = O.rows_to_f64(s.win_fmt, np_(inp["win"])).reshape(B, s.W, s.D)
+        if s.ring:
+            for b, L in enumerate(s.seq_lens):
+                p0 = max(0, L - s.W)
+                self.win_f[b] = self.win_f[b][O.ring_slot(np.arange(p0, p0 + s.W), s.W)]
         xn = P.raw_rows(s.raw_fmt, np_(inp["x_new"]))
         self.pos = [L - 1 for L in s.seq_lens]
         newrow, _, _ = P.stored(s.win_fmt, O.qk_prep(xn, np.array(self.pos), lo, d_r), d_n)
