@@ -365,6 +365,9 @@ typedef struct lc_attn_args {
   int32_t n_win_rows;      /* rows of win (every win_start[b] + win_len[b] <= n_win_rows), or 0
                               if unknown; with W > 0 the FP8 tensor-core kernel reads window
                               rows by bulk tensor copies and needs it */
+  int32_t v_nope;          /* 0: the values are the whole D-dim key rows (out [n_q, H, D]);
+                              1: the values are the D - d_r non-RoPE dims of each key row, in
+                              logical order (out [n_q, H, D - d_r]); needs d_r > 0 */
 } lc_attn_args;
 
 /* Attention kernels. */

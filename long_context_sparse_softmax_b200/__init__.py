@@ -96,7 +96,7 @@ class AttnArgs(ctypes.Structure):
                 ("win", Rows), ("idx", c_void_p), ("sink", c_void_p), ("batch", Batch), ("out", c_void_p),
                 ("lse", c_void_p), ("workspace", c_void_p), ("workspace_bytes", c_size_t), ("status", c_void_p),
                 ("impl", c_int32), ("n_ent_rows", c_int32),
-                ("n_win_rows", c_int32)]
+                ("n_win_rows", c_int32), ("v_nope", c_int32)]
 
 
 LC_IMPL_AUTO, LC_IMPL_TC, LC_IMPL_REF = 0, 2, 3

@@ -120,14 +120,22 @@ __global__ void __launch_bounds__(256) k_attn_ref(lc_attn_args a, int sparse) {
   out.fmt = a.out_fmt;
   out.x = a.out;
   out.rope = nullptr;
+  // values: every dim, or (v_nope) the non-RoPE dims, written in logical order
+  const int rope_off = a.dims.rope_off;
+  const int Dv = a.v_nope ? D - d_r : D;
 #pragma unroll
   for (int i = 0; i < kAttnGroups; ++i) {
     const int g = lane + kWarp * i;
     if (g < G) {
+      int d = g << 3;
+      if (a.v_nope) {
+        if (d >= rope_off && d < rope_off + d_r) continue;
+        if (d >= rope_off + d_r) d -= d_r;
+      }
       Vec8 o;
 #pragma unroll
       for (int u = 0; u < 8; ++u) o.v[u] = st.o[i].v[u] * inv;
-      store8(out, qrow, D, d_r, g << 3, o);
+      store8(out, qrow, Dv, 0, d, o);
     }
   }
   if (a.lse && lane == 0) a.lse[qrow] = st.m + logf(st.z);

@@ -31,9 +31,11 @@ __global__ void __launch_bounds__(kCombineThreads) k_attn_combine(lc_attn_args a
                                                                   const float* __restrict__ ws_ml) {
   const int64_t rows = static_cast<int64_t>(a.n_q) * a.dims.H;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kCombineThreads + threadIdx.x;
-  if (t >= rows * kQuads) return;
-  const int64_t row = t / kQuads;
-  const int c4 = static_cast<int>(t % kQuads);
+  const int Dv = a.v_nope ? kAD - a.dims.d_r : kAD;  // output dims (the partial rows keep all kAD)
+  const int nq = Dv / 4;
+  if (t >= rows * nq) return;
+  const int64_t row = t / nq;
+  const int c4 = static_cast<int>(t % nq);
   const int h = static_cast<int>(row % a.dims.H);
   const float sk = __ldg(a.sink + h) * 1.4426950408889634f;
   const float2* ml = reinterpret_cast<const float2*>(ws_ml) + row * n_split;
@@ -81,9 +83,9 @@ __global__ void __launch_bounds__(kCombineThreads) k_attn_combine(lc_attn_args a
     uint2 pk;
     pk.x = pack_bf16(o.x * inv, o.y * inv);
     pk.y = pack_bf16(o.z * inv, o.w * inv);
-    reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + row * kAD)[c4] = pk;
+    reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + row * Dv)[c4] = pk;
   } else {
-    reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * kAD)[c4] =
+    reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * Dv)[c4] =
         make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
   }
   if (a.lse && c4 == 0) a.lse[row] = (M + log2f(Z)) * 0.6931471805599453f;

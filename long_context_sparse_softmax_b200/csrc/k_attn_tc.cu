@@ -263,6 +263,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t wr0 = a.W > 0 ? __ldg(a.batch.win_start + b) : 0;
   const int32_t* idx_row = sparse ? a.idx + static_cast<int64_t>(q) * a.k : nullptr;
   const int64_t row0 = static_cast<int64_t>(q) * H + hg * kNR;  // first output row of the CTA
+  // values: all 576 dims (5 O^T chunks), or (v_nope) the 512 non-RoPE dims (chunks 0-3)
+  const int n_och = a.v_nope ? 4 : 5;
+  const int Dv = a.v_nope ? kDN : kD;
 
   // bounded wait; gives up (and tells the other roles) after kSpin polls
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -399,8 +402,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < kTK / 16; ++kk)
 #pragma unroll
             for (int c = 0; c < 5; ++c)
-              mma_f16(tm + kColO + c * kNR, dv + (c * 2048 + kk * 2 * kG) / 16, dp + kk * 16, c < 4 ? id_o128 : id_o64,
-                      (no > 0) || (kk > 0));
+              if (c < n_och)
+                mma_f16(tm + kColO + c * kNR, dv + (c * 2048 + kk * 2 * kG) / 16, dp + kk * 16,
+                        c < 4 ? id_o128 : id_o64, (no > 0) || (kk > 0));
           mma_commit(su32(&bars.kempty[no & 1]));
           mma_commit(su32(&bars.pempty));
           ++no;
@@ -482,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_bar(1, 128);
         fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 5; ++c)
+        for (int c = 0; c < n_och; ++c)
 #pragma unroll 1
           for (int hh = 0; hh < kNR; hh += 32) {
             uint32_t ov[32];
@@ -543,8 +547,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool f32 = geo.n_split > 1 || a.out_fmt == LC_FMT_F32;
       float* stf = reinterpret_cast<float*>(Ks);
       uint16_t* sth = reinterpret_cast<uint16_t*>(Ks);
+      const int ostr = geo.n_split > 1 ? kD : Dv;  // partial rows keep every dim
 #pragma unroll 1
-      for (int c = 0; c < 5; ++c) {
+      for (int c = 0; c < n_och; ++c) {
         // chunk c < 4: lane L -> dim 128 c + L; chunk 4 (M = 64): lane 32 w + i -> dim 512 + 16 w + i
         const int dim = c < 4 ? c * 128 + warp * 32 + lane : (lane < 16 ? 512 + warp * 16 + lane : -1);
         uint32_t ov[kNR];  // the chunk's 64 head columns, one wait
@@ -561,18 +566,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kNR; ++i) {
           float v = __uint_as_float(ov[i]);
           if (geo.n_split == 1) v *= s_f[i];
-          if (f32) stf[i * kD + dim] = v;
-          else sth[i * kD + dim] = f32_to_bf16_bits(v);
+          if (f32) stf[i * ostr + dim] = v;
+          else sth[i * ostr + dim] = f32_to_bf16_bits(v);
         }
       }
       fence_async_smem();
       named_bar(1, 128);
       if (tid == 0) {
-        const uint32_t bytes = kNR * kD * (f32 ? 4 : 2);
+        const uint32_t bytes = kNR * ostr * (f32 ? 4 : 2);
         void* dst;
         if (geo.n_split > 1) dst = ws_o + (static_cast<int64_t>(split) * a.n_q * H + row0) * kD;
-        else if (a.out_fmt == LC_FMT_F32) dst = static_cast<float*>(a.out) + row0 * kD;
-        else dst = static_cast<uint16_t*>(a.out) + row0 * kD;
+        else if (a.out_fmt == LC_FMT_F32) dst = static_cast<float*>(a.out) + row0 * Dv;
+        else dst = static_cast<uint16_t*>(a.out) + row0 * Dv;
         bulk_store(dst, Ks, bytes);
       }
     }

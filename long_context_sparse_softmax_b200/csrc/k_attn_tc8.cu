@@ -222,6 +222,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t wr0 = a.W > 0 ? __ldg(a.batch.win_start + b) : 0;
   const int32_t* idx_row = sparse ? a.idx + static_cast<int64_t>(q) * a.k : nullptr;
   const int64_t row0 = static_cast<int64_t>(q) * H + hg * kNR;
+  // values: all 576 dims (5 O^T chunks), or (v_nope) the 512 E4M3 dims (chunks 0-3)
+  const int n_och = a.v_nope ? 4 : 5;
+  const int Dv = a.v_nope ? kDN : kD;
 
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
     const uint32_t addr = su32(bar);
@@ -412,16 +415,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < kTK / 16; ++kk)
 #pragma unroll
               for (int c = 0; c < 5; ++c)
-                mma_f16(tm + kColO + c * kNR, dv + (c * 2048 + kk * 2 * kG) / 16, dp + kk * 16,
-                       c < 4 ? id_o128 : id_o64, (no > 0) || (kk > 0));
+                if (c < n_och)
+                  mma_f16(tm + kColO + c * kNR, dv + (c * 2048 + kk * 2 * kG) / 16, dp + kk * 16,
+                          c < 4 ? id_o128 : id_o64, (no > 0) || (kk > 0));
           } else {
             // window tile: V^T straight from the SW128 tile (dims along M, 16 keys per step)
 #pragma unroll
             for (int kk = 0; kk < kTK / 16; ++kk)
 #pragma unroll
               for (int c = 0; c < 5; ++c)
-                mma_f16(tm + kColO + c * kNR, sw128_mn_desc(su32(Vt) + c * 2 * kBlk + kk * 2048, kBlk), dp + kk * 16,
-                       c < 4 ? id_o128 : id_o64, (no > 0) || (kk > 0));
+                if (c < n_och)
+                  mma_f16(tm + kColO + c * kNR, sw128_mn_desc(su32(Vt) + c * 2 * kBlk + kk * 2048, kBlk),
+                          dp + kk * 16, c < 4 ? id_o128 : id_o64, (no > 0) || (kk > 0));
           }
           mma_commit(su32(&bars.vempty));
           mma_commit(su32(&bars.pempty));
@@ -623,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_bar(1, 128);
         fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 5; ++c)
+        for (int c = 0; c < n_och; ++c)
 #pragma unroll 1
           for (int hh = 0; hh < kNR; hh += 32) {
             uint32_t ov[32];
@@ -684,13 +689,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O^T (dims on tensor-memory lanes, heads on columns) straight to global memory:
       // for each head a warp writes 32 consecutive dims, 128 bytes in FP32
       const bool f32 = geo.n_split > 1 || a.out_fmt == LC_FMT_F32;
+      const int ostr = geo.n_split > 1 ? kD : Dv;  // partial rows keep every dim
       float* of = nullptr;
       uint16_t* oh = nullptr;
       if (geo.n_split > 1) of = ws_o + (static_cast<int64_t>(split) * a.n_q * H + row0) * kD;
-      else if (f32) of = static_cast<float*>(a.out) + row0 * kD;
-      else oh = static_cast<uint16_t*>(a.out) + row0 * kD;
+      else if (f32) of = static_cast<float*>(a.out) + row0 * Dv;
+      else oh = static_cast<uint16_t*>(a.out) + row0 * Dv;
 #pragma unroll 1
-      for (int c = 0; c < 5; ++c) {
+      for (int c = 0; c < n_och; ++c) {
         const int dim = c < 4 ? c * 128 + warp * 32 + lane : (lane < 16 ? 512 + warp * 16 + lane : -1);
         uint32_t ov[kNR];
         if (n_tiles > 0) {
@@ -706,8 +712,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kNR; ++i) {
           float v = __uint_as_float(ov[i]);
           if (geo.n_split == 1) v *= s_f[i];
-          if (f32) of[i * kD + dim] = v;
-          else oh[i * kD + dim] = f32_to_bf16_bits(v);
+          if (f32) of[i * ostr + dim] = v;
+          else oh[i * ostr + dim] = f32_to_bf16_bits(v);
         }
       }
     }
@@ -740,7 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar(1, 128);
       const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
 #pragma unroll 1
-      for (int c = 0; c < 5; ++c) {
+      for (int c = 0; c < n_och; ++c) {
         const int dim = c < 4 ? c * 128 + warp * 32 + lane : (lane < 16 ? 512 + warp * 16 + lane : -1);
         uint32_t ov[kNR];
         if (n_tiles > 0) {
@@ -757,8 +763,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     cl.sync();  // every split's scaled O is in its shared memory
-    const int dpc = ((kD + geo.n_split - 1) / geo.n_split + 3) & ~3;
-    const int d0 = min(kD, split * dpc), d1 = min(kD, d0 + dpc);
+    const int dpc = ((Dv + geo.n_split - 1) / geo.n_split + 3) & ~3;
+    const int d0 = min(Dv, split * dpc), d1 = min(Dv, d0 + dpc);
     const int nq4 = (d1 - d0) / 4;
     const float* src[kMaxClusterSplits];
 #pragma unroll
@@ -775,7 +781,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           o.z += v.z;
           o.w += v.w;
         }
-      const int64_t e = (row0 + h) * kD + d;
+      const int64_t e = (row0 + h) * Dv + d;
       if (a.out_fmt == LC_FMT_F32) {
         *reinterpret_cast<float4*>(static_cast<float*>(a.out) + e) = o;
       } else {

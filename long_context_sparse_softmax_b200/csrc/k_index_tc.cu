@@ -378,12 +378,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if constexpr (SELECT) {
       // ================= the range's top K (128 threads; the key ring is idle) =================
-      __shared__ uint32_t s_rng[2][4];
-      __shared__ int s_tmp[4];
-      __shared__ int s_pick[2];
-      __shared__ int s_wcnt[kSelMaxTiles][4];
+      // scratch in the idle key ring (dynamic shared memory, so that the static part stays
+      // small enough for two CTAs per SM)
       uint32_t* hist = reinterpret_cast<uint32_t*>(As);   // [kSelBins]
-      uint32_t* bits = hist + kSelBins;                   // [n_tiles * 4] selection words
+      uint32_t* bits = hist + kSelBins;                   // [kSelMaxTiles * 4] selection words
+      int (*s_wcnt)[4] = reinterpret_cast<int (*)[4]>(bits + kSelMaxTiles * 4);  // [kSelMaxTiles][4]
+      uint32_t (*s_rng)[4] = reinterpret_cast<uint32_t (*)[4]>(s_wcnt + kSelMaxTiles);  // [2][4]
+      int* s_tmp = reinterpret_cast<int*>(s_rng + 2);     // [4]
+      int* s_pick = s_tmp + 4;                            // [2]
       const int q = s_q[0];
       const int jbase = t_begin * kKeys;
       const int n_valid = max(0, min(s_nv[0] - jbase, n_tiles * kKeys));
@@ -557,8 +559,9 @@ IndexGeom index_geometry(const lc_index_args& a, bool decode, bool select) {
               static_cast<size_t>(N) * 4 + 1024;
   if (select) sm += static_cast<size_t>(g.tpc) * kKeys * 4;
   // no more CTAs per SM than its 512 tensor-memory columns hold, so tcgen05.alloc never
-  // waits for another CTA
-  const size_t cap = 227 * 1024 / per_sm - 2048;
+  // waits for another CTA (and no fewer: the static shared memory and the per-CTA
+  // reservation fit in the 3 KB left per CTA)
+  const size_t cap = 227 * 1024 / per_sm - 3072;
   g.smem = sm < cap ? cap : sm;
   return g;
 }

@@ -183,6 +183,7 @@ lc_status attn(const lc_attn_args* a, void* stream, bool sparse, bool decode) {
   if (a->n_q < 0 || a->m < 1 || a->W < 0 || a->W_x < 0 || a->max_ent < 0) return LC_ERR_ARG;
   if (a->out_fmt != LC_FMT_F32 && a->out_fmt != LC_FMT_BF16) return LC_ERR_ARG;
   if (a->batch.win_ring < 0 || (a->batch.win_ring > 0 && a->batch.win_ring < a->W)) return LC_ERR_ARG;
+  if (a->v_nope != 0 && (a->v_nope != 1 || a->dims.d_r <= 0)) return LC_ERR_ARG;
   if (sparse && a->k < 1) return LC_ERR_ARG;
   if (decode && a->n_q != a->batch.num_seqs) return LC_ERR_ARG;
   if (a->impl != LC_IMPL_AUTO && a->impl != LC_IMPL_TC && a->impl != LC_IMPL_REF) return LC_ERR_ARG;

@@ -184,7 +184,8 @@ class _Common:
         return IndexArgs(n_q, s.H_I, s.d_I, LC_IDX_MXFP4 if mx else LC_IDX_F32,
                          ptr(qI["codes"] if mx else qI["f32"]), ptr(qI.get("scales")),
                          ptr(kI["codes"] if mx else kI["f32"]), ptr(kI.get("scales")),
-                         (kI["codes"] if mx else kI["f32"]).shape[0], ptr(inp["w"]), 0, s.m, self.W_x, max_ent, self.batch,
+                         (kI["codes"] if mx else kI["f32"]).shape[0], ptr(inp["w"]), s.H_I if s.w_per_query else 0, s.m,
+                         self.W_x, max_ent, self.batch,
                          ptr(scores), scores.shape[1], ptr(self.status))
 
     def _index_topk_args(self, n_q: int, max_ent: int, decode: bool) -> IndexTopkArgs:
@@ -225,6 +226,7 @@ class _Common:
         a.impl = self.impl
         a.n_ent_rows = int(next(iter(self.ent.values())).shape[0])
         a.n_win_rows = int(self.win["x"].shape[0])
+        a.v_nope = 1 if s.v_nope else 0
         ws = (lc_csa_sparse_attn_workspace_bytes if sparse else lc_hca_attn_workspace_bytes)(a)
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.device)
         a.workspace, a.workspace_bytes = ptr(self.workspace), ws
@@ -268,7 +270,7 @@ class Prefill(_Common):
         self.a_prep_win = QkPrepArgs(Dims(s.D, s.d_r, s.rope_off, 1), n_win, s.raw_fmt, ptr(x_win),
                                      ptr(inp["win_pos"]), None, rows(s.win_fmt, self.win), RMS_EPS, ROPE_BASE,
                                      ptr(self.status))
-        self.out = torch.empty(s.n_q * s.H, s.D, dtype=torch.float32 if s.out_f32 else torch.int16, device=device)
+        self.out = torch.empty(s.n_q * s.H, s.Dv, dtype=torch.float32 if s.out_f32 else torch.int16, device=device)
         self.lse = torch.empty(s.n_q * s.H, dtype=torch.float32, device=device)
         if s.is_csa:
             self._indexer_buffers(s.n_q, n_c, False)
@@ -362,7 +364,7 @@ class Decode(_Common):
         self.a_prep_win = QkPrepArgs(Dims(s.D, s.d_r, s.rope_off, 1), B, s.raw_fmt, ptr(inp["x_new"]),
                                      ptr(inp["q_pos"]), ptr(self.win_slot), rows(s.win_fmt, self.win), RMS_EPS,
                                      ROPE_BASE, ptr(self.status))
-        self.out = torch.empty(B * s.H, s.D, dtype=torch.float32 if s.out_f32 else torch.int16, device=device)
+        self.out = torch.empty(B * s.H, s.Dv, dtype=torch.float32 if s.out_f32 else torch.int16, device=device)
         self.lse = torch.empty(B * s.H, dtype=torch.float32, device=device)
         if s.is_csa:
             self._indexer_buffers(B, sum(n_c), True)

@@ -63,10 +63,17 @@ class Spec:
     n_q: int = 0
     overlap: bool = False    # window/compressed overlap reading (W_x = 0)
     ring: bool = True        # decode: each sequence's window rows are a ring of W rows
+    w_per_query: bool = False  # indexer head weights per query [n_q, H_I] instead of shared [H_I]
+    v_nope: bool = False     # values are the non-RoPE dims of the entries (outputs D - d_r dims)
 
     @property
     def d_n(self) -> int:
         return self.D - self.d_r
+
+    @property
+    def Dv(self) -> int:
+        """Dims of each head's output: the value rows' dims."""
+        return self.D - self.d_r if self.v_nope else self.D
 
     @property
     def scale(self) -> float:
@@ -260,7 +267,7 @@ def make_prefill(spec: Spec, device="cpu") -> Dict[str, object]:
         else:
             out["qI"] = _indexer_operand(s, "qI", (s.n_q, s.H_I, s.d_I), device)
             out["kI"] = _indexer_operand(s, "kI", (n_c, s.d_I), device)
-        out["w"] = rand(s.seed, "w", (s.H_I,), device)
+        out["w"] = rand(s.seed, "w", (s.n_q, s.H_I) if s.w_per_query else (s.H_I,), device)
     # positions and the batch descriptor (one sequence)
     q_pos = torch.arange(s.q_first, s.q_first + s.n_q, dtype=torch.int32, device=device)
     out["q_pos"] = q_pos
@@ -326,7 +333,7 @@ def make_decode(spec: Spec, device="cpu") -> Dict[str, object]:
         else:
             out["qI"] = _indexer_operand(s, "qI", (B, s.H_I, s.d_I), device)
         out["kI"] = _indexer_operand(s, "kI", (tot, s.d_I), device)
-        out["w"] = rand(s.seed, "w", (s.H_I,), device)
+        out["w"] = rand(s.seed, "w", (B, s.H_I) if s.w_per_query else (s.H_I,), device)
     out["q_pos"] = _i32([L - 1 for L in s.seq_lens], device)
     out["batch"] = {
         "q_start": _i32(range(B + 1), device),

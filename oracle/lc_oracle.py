@@ -272,38 +272,47 @@ def window_positions(p: int, W: int) -> range:
     return range(max(0, p - W + 1), p + 1)
 
 
-def attend(q: np.ndarray, keys: np.ndarray, sink: np.ndarray, scale: float):
+def attend(q: np.ndarray, keys: np.ndarray, sink: np.ndarray, scale: float, v_dims=None):
     """Softmax attention of H heads over a shared key set plus a per-head sink.
 
-    q [H, D]; keys [n, D] (values are the same rows); sink [H] (a logit in the
-    denominator only, unscaled).  l = scale * <q_h, key>; M = max(sink_h, max l);
+    q [H, D]; keys [n, D]; the values are the same rows, or their dims v_dims (an index
+    array: the V = non-RoPE-dims variant); sink [H] (a logit in the denominator only,
+    unscaled).  l = scale * <q_h, key>; M = max(sink_h, max l);
     Z = e^(sink_h - M) + sum e^(l - M); o = sum e^(l - M) v / Z; lse = M + ln Z.
     """
     logits = scale * (q @ keys.T)                               # [H, n]
     M = np.maximum(sink, logits.max(axis=1) if keys.shape[0] else -np.inf)
     e = np.exp(logits - M[:, None])
     Z = np.exp(sink - M) + e.sum(axis=1)
-    o = (e @ keys) / Z[:, None]
+    values = keys if v_dims is None else keys[:, v_dims]
+    o = (e @ values) / Z[:, None]
     return o, M + np.log(Z)
 
 
+def nope_dims(D: int, lo: int, d_r: int) -> np.ndarray:
+    """The non-RoPE dims of a D-dim row whose RoPE dims are lo .. lo + d_r - 1, in order
+    (the values of the variant that leaves the RoPE part out of V)."""
+    return np.concatenate([np.arange(0, lo), np.arange(lo + d_r, D)])
+
+
 def sparse_attn_query(q: np.ndarray, entries: np.ndarray, idx: Sequence[int], win_rows: np.ndarray,
-                      win_pos0: int, p: int, W: int, sink: np.ndarray, scale: float):
+                      win_pos0: int, p: int, W: int, sink: np.ndarray, scale: float, v_dims=None):
     """CSA core attention for one query at position p: keys = the selected entries
     (index -1 = padding, skipped) joined with the window tokens p-W+1..p and the sink.
-    win_rows holds prepped window rows for positions win_pos0, win_pos0 + 1, ..."""
+    win_rows holds prepped window rows for positions win_pos0, win_pos0 + 1, ...
+    v_dims: the value dims (None: the whole rows)."""
     sel = [int(j) for j in idx if j >= 0]
     wp = [t - win_pos0 for t in window_positions(p, W)]
     assert all(0 <= r < win_rows.shape[0] for r in wp), "window row missing"
     D = entries.shape[1]
     keys = np.concatenate([entries[sel].reshape(len(sel), D), win_rows[wp].reshape(len(wp), D)], axis=0)
-    return attend(q, keys, sink, scale)
+    return attend(q, keys, sink, scale, v_dims)
 
 
 def hca_attn_query(q: np.ndarray, entries: np.ndarray, n_vis: int, win_rows: np.ndarray,
-                   win_pos0: int, p: int, W: int, sink: np.ndarray, scale: float):
+                   win_pos0: int, p: int, W: int, sink: np.ndarray, scale: float, v_dims=None):
     """HCA attention: every visible entry is selected, no indexer."""
-    return sparse_attn_query(q, entries, range(n_vis), win_rows, win_pos0, p, W, sink, scale)
+    return sparse_attn_query(q, entries, range(n_vis), win_rows, win_pos0, p, W, sink, scale, v_dims)
 
 
 # =====================================================================================

@@ -200,7 +200,8 @@ class _E2E:
         self.worst_path = max(self.worst_path, _ratio(err2, tol2))
         same_sel = not s.is_csa or np.array_equal(np.asarray([v for v in idx_lib if v >= 0]), np.asarray(idx_orc))
         if same_sel:
-            b = perturbation_bound(q_orc, keys(idx_orc), q_lib, keys(idx_lib, ent=ent_lib, win=win_lib), sink, s.scale)
+            b = perturbation_bound(q_orc, keys(idx_orc), q_lib, keys(idx_lib, ent=ent_lib, win=win_lib), sink, s.scale,
+                                   O.nope_dims(s.D, s.rope_off, s.d_r) if s.v_nope else None)
             d = np.abs(o_lib - o_orc)
             assert np.all(d <= b), f"attention (end to end) {what}: intermediates move the result by " \
                                    f"{np.max(d - b)} beyond their perturbation bound"

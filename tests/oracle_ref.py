@@ -115,7 +115,7 @@ def write_rows(r: Dict[str, torch.Tensor], fmt: int, y: np.ndarray, d_n: int, se
 
 def out_np(run, q_sel: Sequence[int]) -> np.ndarray:
     s = run.spec
-    o = run.out.view(-1, s.H, s.D)[torch.as_tensor(list(q_sel), device=run.out.device)]
+    o = run.out.view(-1, s.H, s.Dv)[torch.as_tensor(list(q_sel), device=run.out.device)]
     o = np_(o)
     return o.astype(np.float64) if s.out_f32 else O.bf16_to_f64(o)
 
@@ -141,7 +141,7 @@ def attn_ok(got: np.ndarray, exp: np.ndarray, out_f32: bool):
 
 
 def perturbation_bound(q_a: np.ndarray, keys_a: np.ndarray, q_b: np.ndarray, keys_b: np.ndarray,
-                       sink: np.ndarray, scale: float) -> np.ndarray:
+                       sink: np.ndarray, scale: float, v_dims=None) -> np.ndarray:
     """Bound on |attend(q_b, keys_b) - attend(q_a, keys_a)| per output element [H, D], for
     two inputs with the same keys in the same order whose values differ slightly (the
     library's stored intermediates against the oracle's, one storage grid step apart).
@@ -153,14 +153,16 @@ def perturbation_bound(q_a: np.ndarray, keys_a: np.ndarray, q_b: np.ndarray, key
     la = scale * (q_a @ keys_a.T)
     lb = scale * (q_b @ keys_b.T)
     L = np.max(np.abs(lb - la), axis=1) if keys_a.shape[0] else np.zeros(q_a.shape[0])
-    o_a, lse = O.attend(q_a, keys_a, sink, scale)
+    o_a, lse = O.attend(q_a, keys_a, sink, scale, v_dims)
     p = np.exp(la - lse[:, None])                        # [H, n]
     p_sink = np.exp(sink - lse)                          # [H]
-    dv = np.abs(keys_b - keys_a)                         # [n, D]
+    va = keys_a if v_dims is None else keys_a[:, v_dims]
+    vb = keys_b if v_dims is None else keys_b[:, v_dims]
+    dv = np.abs(vb - va)                                 # [n, Dv]
     g = np.exp(2 * L)[:, None]
     spread = np.empty_like(o_a)
     for h in range(o_a.shape[0]):
-        spread[h] = p[h] @ np.abs(keys_a - o_a[h])
+        spread[h] = p[h] @ np.abs(va - o_a[h])
     bound = g * (p @ dv) + (g - 1) * (spread + p_sink[:, None] * np.abs(o_a))
     return bound * (1 + 1e-9) + 1e-12
 
@@ -208,6 +210,7 @@ class OraclePrefill:
         s: wl.Spec = inp["spec"]
         self.s = s
         self.sink = np_(inp["sink"]).astype(np.float64)
+        self.v_dims = O.nope_dims(s.D, s.rope_off, s.d_r) if s.v_nope else None
         self.W_x = s.W if W_x is None else W_x
         self.q_sel = list(q_sel)
         self.pos = [s.q_first + i for i in self.q_sel]
@@ -251,8 +254,9 @@ class OraclePrefill:
         indexer keys, or on the decoded keys `kI` of another path)."""
         p = self.pos[i]
         kI = self.kI if kI is None else kI
-        s, n_vis = P.visible_scores(self.qI[i], kI, self.w, p, self.s.m, self.W_x)
-        return s, O.score_error_bound(self.qI[i], kI[:n_vis], self.w)
+        w = self.w[self.q_sel[i]] if self.s.w_per_query else self.w
+        s, n_vis = P.visible_scores(self.qI[i], kI, w, p, self.s.m, self.W_x)
+        return s, O.score_error_bound(self.qI[i], kI[:n_vis], w)
 
     def select(self, i: int, s_vis: np.ndarray = None):
         if s_vis is None:
@@ -279,9 +283,9 @@ class OraclePrefill:
         ent = self.ent_f if ent is None else ent
         w0, wr = self.window_block(p, win)
         if s.is_csa:
-            return O.sparse_attn_query(q, ent, idx, wr, w0, p, s.W, self.sink, s.scale)
+            return O.sparse_attn_query(q, ent, idx, wr, w0, p, s.W, self.sink, s.scale, self.v_dims)
         n_vis = O.n_visible(p, s.m, self.W_x, ent.shape[0])
-        return O.hca_attn_query(q, ent, n_vis, wr, w0, p, s.W, self.sink, s.scale)
+        return O.hca_attn_query(q, ent, n_vis, wr, w0, p, s.W, self.sink, s.scale, self.v_dims)
 
     def keys(self, i: int, idx: Sequence[int], ent: np.ndarray = None, win: np.ndarray = None):
         """The key rows attend() uses for sampled query i, in its order (for the
@@ -302,6 +306,7 @@ class OracleDecode:
         self.s = s
         self.W_x = s.W if W_x is None else W_x
         self.sink = np_(inp["sink"]).astype(np.float64)
+        self.v_dims = O.nope_dims(s.D, s.rope_off, s.d_r) if s.v_nope else None
         lo, d_r, d_n = s.rope_off, s.d_r, s.d_n
         B = s.num_seqs
         self.n_c = list(inp["n_c"])
@@ -372,8 +377,9 @@ class OracleDecode:
 
     def scores(self, b: int, kI_np=None):
         kI = self.kI(b, kI_np)
-        s, n_vis = P.visible_scores(self.qI[b], kI, self.w, self.pos[b], self.s.m, self.W_x)
-        return s, O.score_error_bound(self.qI[b], kI[:n_vis], self.w)
+        w = self.w[b] if self.s.w_per_query else self.w
+        s, n_vis = P.visible_scores(self.qI[b], kI, w, self.pos[b], self.s.m, self.W_x)
+        return s, O.score_error_bound(self.qI[b], kI[:n_vis], w)
 
     def entries(self, b: int):
         return self.ent_f[self.ent_start[b]:self.ent_start[b] + self.n_c[b]]
@@ -396,9 +402,9 @@ class OracleDecode:
         e = ent[self.ent_start[b]:self.ent_start[b] + self.n_c[b]]
         wr = self.window_rows(b, win)
         if s.is_csa:
-            return O.sparse_attn_query(q, e, idx, wr, self.win_pos0[b], p, s.W, self.sink, s.scale)
+            return O.sparse_attn_query(q, e, idx, wr, self.win_pos0[b], p, s.W, self.sink, s.scale, self.v_dims)
         n_vis = O.n_visible(p, s.m, self.W_x, self.n_c[b])
-        return O.hca_attn_query(q, e, n_vis, wr, self.win_pos0[b], p, s.W, self.sink, s.scale)
+        return O.hca_attn_query(q, e, n_vis, wr, self.win_pos0[b], p, s.W, self.sink, s.scale, self.v_dims)
 
     def keys(self, b: int, idx: Sequence[int], ent: np.ndarray = None, win: np.ndarray = None):
         """The key rows attend() uses for sequence b, in its order."""

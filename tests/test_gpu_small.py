@@ -102,3 +102,33 @@ def test_small_csa_decode_each_attention_kernel(impl):
 def test_small_hca_decode_each_attention_kernel(impl):
     s = wl.shrink(wl.MIXED_HCA, name="small_hcad_impl", seed=44, seq_lens=(128 * 40 + 3, 900, 128 * 7))
     check_decode(s, impl=impl)
+
+
+def test_per_query_indexer_weights_decode_and_prefill():
+    """Indexer head weights given per query ([n_q, H_I], w_qstride = H_I) instead of shared."""
+    check_decode(wl.shrink(wl.CSA_DECODE, name="wq_decode", seed=45, seq_lens=(3000, 1027, 9000), k=128,
+                           w_per_query=True))
+    check_prefill(wl.shrink(wl.CSA_PREFILL, name="wq_prefill", seed=46, seq_lens=(900,), H=64, k=64, n_q=900,
+                            w_per_query=True), q_sel=range(0, 900, 5))
+
+
+# values without the RoPE dims (outputs of D - d_r dims), on every attention kernel
+@pytest.mark.parametrize("impl", IMPLS)
+def test_nope_values_csa_decode(impl):
+    s = wl.shrink(wl.CSA_DECODE, name="vnope_decode", seed=47, seq_lens=(3000, 1027, 8192, 200), k=256, v_nope=True)
+    check_decode(s, impl=impl)
+
+
+def test_nope_values_csa_decode_few_queries_combine():
+    """Two queries: more key splits than a cluster holds, so the partials are merged by the
+    combine kernel."""
+    check_decode(wl.shrink(wl.CSA_DECODE, name="vnope_combine", seed=48, seq_lens=(20000, 9001), k=512,
+                           v_nope=True))
+
+
+def test_nope_values_prefill_kernels():
+    check_prefill(wl.shrink(wl.CSA_PREFILL, name="vnope_csa_prefill", seed=49, seq_lens=(700,), H=64, k=96, n_q=700,
+                            v_nope=True), q_sel=range(0, 700, 3))
+    check_prefill(wl.shrink(wl.HCA_PREFILL, name="vnope_hca_prefill", seed=50, seq_lens=(128 * 24 + 50,),
+                            q_first=128 * 24 + 50 - 160, n_q=160, v_nope=True))
+    check_prefill(wl.shrink(wl.TINY_CSA_PREFILL, name="vnope_tiny", seed=51, seq_lens=(400,), n_q=400, v_nope=True))

@@ -401,3 +401,28 @@ def test_window_ring_equals_the_linear_window(R, W):
         ring[O.ring_slot(p, R)] = rows[p]
         got = O.window_from_ring(ring, p, W)
         assert np.array_equal(got, rows[max(0, p - W + 1):p + 1])
+
+
+# ------------------------------------------------------------------ values without the RoPE dims
+def test_nope_values_match_sdpa_and_the_full_value_output():
+    """V = the non-RoPE dims: torch SDPA with those value columns, and exactly the non-RoPE
+    columns of the full-V output (same weights)."""
+    H, D, n, lo, d_r = 8, 128, 41, 64, 64
+    q = RNG.standard_normal((H, D)) * 2
+    keys = RNG.standard_normal((n, D))
+    sink = RNG.standard_normal(H)
+    vd = O.nope_dims(D, lo, d_r)
+    assert np.array_equal(vd, np.arange(64))
+    o, lse = O.attend(q, keys, sink, 1 / np.sqrt(D), vd)
+    full, lse_f = O.attend(q, keys, sink, 1 / np.sqrt(D))
+    np.testing.assert_allclose(o, full[:, vd], rtol=1e-13, atol=1e-15)
+    assert np.array_equal(lse, lse_f)
+    K = torch.cat([torch.zeros(1, D, dtype=torch.float64), torch.tensor(keys)], 0)
+    V = K[:, torch.tensor(vd)]
+    mask = torch.zeros(H, 1, n + 1, dtype=torch.float64)
+    mask[:, 0, 0] = torch.tensor(sink)
+    ref = F.scaled_dot_product_attention(torch.tensor(q)[:, None, :], K.expand(H, n + 1, D),
+                                         V.expand(H, n + 1, len(vd)), attn_mask=mask, scale=1 / np.sqrt(D))
+    np.testing.assert_allclose(o, ref[:, 0].numpy(), rtol=1e-12, atol=1e-14)
+    # RoPE dims first in the row (the FP32 layout): the value dims are the rest
+    assert np.array_equal(O.nope_dims(128, 0, 64), np.arange(64, 128))
