@@ -417,6 +417,30 @@ size_t lc_hca_attn_workspace_bytes(const lc_attn_args* a);
 lc_status lc_csa_sparse_attn_decode_static(const lc_attn_args* a, void* stream);
 size_t lc_csa_sparse_attn_decode_static_capacity(void);
 
+/* ---------------------------------------------------------------------------------
+ * grouped_out_proj — the grouped output projection of the attention heads: the H heads of
+ * a query form G groups of H/G consecutive heads, and group g projects the concatenation
+ * of its heads' outputs (K = (H/G) Dv values) to its own d_g output dims:
+ *   y[n, g d_g + c] = sum_k x[n, g K + k] W_g[k, c],  0 <= c < d_g.
+ * Pages: 10100.com analysis §三.1 (CSA and HCA use a grouped output projection to reduce
+ * its cost).  BF16 operands, FP32 accumulation on the tensor cores.
+ * ------------------------------------------------------------------------------- */
+typedef struct lc_out_proj_args {
+  int32_t n_q;             /* queries */
+  int32_t H;               /* heads per query (H % G == 0) */
+  int32_t Dv;              /* output dims per head of the attention */
+  int32_t G;               /* groups */
+  int32_t d_g;             /* output dims per group: multiple of 16 */
+  int32_t out_fmt;         /* LC_FMT_F32 or LC_FMT_BF16 */
+  const void* x;           /* [n_q, H, Dv] BF16: the attention output ((H/G) Dv a multiple of 64) */
+  const void* w;           /* [G, d_g, (H/G) Dv] BF16: W_g transposed (row c of group g holds the
+                              weights of output c) */
+  void* y;                 /* [n_q, G d_g] */
+  int32_t* status;         /* optional: LC_DEV_TIMEOUT */
+} lc_out_proj_args;
+
+lc_status lc_grouped_out_proj(const lc_out_proj_args* a, void* stream);
+
 /* Library version string (static storage). */
 const char* lc_version(void);
 /* Name of a status code (static storage). */
@@ -424,7 +448,8 @@ const char* lc_status_string(lc_status s);
 /* sizeof of the args structs, for bindings to check their mirrors:
  * 0 lc_rows, 1 lc_dims, 2 lc_batch, 3 lc_qk_prep_args, 4 lc_compress_args,
  * 5 lc_index_args, 6 lc_topk_args, 7 lc_attn_args, 8 lc_index_topk_args,
- * 9 lc_mxfp4_quant_args, 10 lc_index_compress_args; other values return 0. */
+ * 9 lc_mxfp4_quant_args, 10 lc_index_compress_args, 11 lc_out_proj_args; other values
+ * return 0. */
 size_t lc_struct_size(int32_t which);
 
 #ifdef __cplusplus

@@ -90,6 +90,11 @@ class IndexCompressArgs(ctypes.Structure):
                 ("codes", c_void_p), ("scales", c_void_p), ("status", c_void_p)]
 
 
+class OutProjArgs(ctypes.Structure):
+    _fields_ = [("n_q", c_int32), ("H", c_int32), ("Dv", c_int32), ("G", c_int32), ("d_g", c_int32), ("out_fmt", c_int32),
+                ("x", c_void_p), ("w", c_void_p), ("y", c_void_p), ("status", c_void_p)]
+
+
 class AttnArgs(ctypes.Structure):
     _fields_ = [("dims", Dims), ("n_q", c_int32), ("k", c_int32), ("m", c_int32), ("W", c_int32), ("W_x", c_int32),
                 ("max_ent", c_int32), ("scale", c_float), ("out_fmt", c_int32), ("q", Rows), ("ent", Rows),
@@ -103,7 +108,7 @@ LC_IMPL_AUTO, LC_IMPL_TC, LC_IMPL_REF = 0, 2, 3
 
 
 STRUCTS = [Rows, Dims, Batch, QkPrepArgs, CompressArgs, IndexArgs, TopkArgs, AttnArgs, IndexTopkArgs, Mxfp4QuantArgs,
-           IndexCompressArgs]
+           IndexCompressArgs, OutProjArgs]
 
 ENTRY_POINTS = {
     "lc_qk_prep_prefill": QkPrepArgs, "lc_qk_prep_decode": QkPrepArgs,
@@ -113,6 +118,7 @@ ENTRY_POINTS = {
     "lc_csa_topk_prefill": TopkArgs, "lc_csa_topk_decode": TopkArgs,
     "lc_csa_index_topk_prefill": IndexTopkArgs, "lc_csa_index_topk_decode": IndexTopkArgs,
     "lc_mxfp4_quantize": Mxfp4QuantArgs,
+    "lc_grouped_out_proj": OutProjArgs,
     "lc_csa_index_compress_prefill": IndexCompressArgs, "lc_csa_index_compress_decode": IndexCompressArgs,
     "lc_csa_sparse_attn_prefill": AttnArgs, "lc_csa_sparse_attn_decode": AttnArgs,
     "lc_hca_attn_prefill": AttnArgs, "lc_hca_attn_decode": AttnArgs,

@@ -15,7 +15,7 @@ ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "liblc.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
-SOURCES = ["lc_abi.cu", "k_prep.cu", "k_index.cu", "k_topk.cu", "k_attn.cu", "k_attn_combine.cu", "k_index_tc.cu", "k_attn_tc.cu", "k_attn_tc8.cu", "k_quant.cu", "lc_noalloc.cu"]
+SOURCES = ["lc_abi.cu", "k_prep.cu", "k_index.cu", "k_topk.cu", "k_attn.cu", "k_attn_combine.cu", "k_index_tc.cu", "k_attn_tc.cu", "k_attn_tc8.cu", "k_quant.cu", "k_outproj.cu", "lc_noalloc.cu"]
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

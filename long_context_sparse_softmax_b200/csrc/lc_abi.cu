@@ -141,6 +141,17 @@ lc_status index_compress(const lc_index_compress_args* a, void* stream) {
   return launched(lc::launch_index_compress(*a, static_cast<cudaStream_t>(stream)));
 }
 
+lc_status out_proj(const lc_out_proj_args* a, void* stream) {
+  if (!a) return LC_ERR_ARG;
+  if (a->n_q < 0 || a->H < 1 || a->G < 1 || a->H % a->G || a->Dv < 1 || a->d_g < 16 || a->d_g % 16) return LC_ERR_ARG;
+  if (a->out_fmt != LC_FMT_F32 && a->out_fmt != LC_FMT_BF16) return LC_ERR_ARG;
+  if ((static_cast<int64_t>(a->H / a->G) * a->Dv) % 64) return LC_ERR_UNSUPPORTED;
+  if (a->n_q == 0) return LC_OK;
+  if (!a->x || !a->w || !a->y) return LC_ERR_ARG;
+  if (!aligned16(a->x) || !aligned16(a->w) || !aligned16(a->y)) return LC_ERR_ALIGN;
+  return launched(lc::launch_out_proj(*a, static_cast<cudaStream_t>(stream)));
+}
+
 lc_status index_scores(const lc_index_args* a, void* stream, bool decode) {
   LC_TRY(check_index(a, decode, true));
   if (a->n_q == 0 || a->max_ent == 0) return LC_OK;
@@ -217,6 +228,7 @@ lc_status lc_csa_index_scores_prefill(const lc_index_args* a, void* stream) { re
 lc_status lc_csa_index_scores_decode(const lc_index_args* a, void* stream) { return index_scores(a, stream, true); }
 
 lc_status lc_mxfp4_quantize(const lc_mxfp4_quant_args* a, void* stream) { return mxfp4_quantize(a, stream); }
+lc_status lc_grouped_out_proj(const lc_out_proj_args* a, void* stream) { return out_proj(a, stream); }
 lc_status lc_csa_index_compress_prefill(const lc_index_compress_args* a, void* stream) { return index_compress(a, stream); }
 lc_status lc_csa_index_compress_decode(const lc_index_compress_args* a, void* stream) { return index_compress(a, stream); }
 
@@ -271,6 +283,7 @@ size_t lc_struct_size(int32_t which) {
     case 8: return sizeof(lc_index_topk_args);
     case 9: return sizeof(lc_mxfp4_quant_args);
     case 10: return sizeof(lc_index_compress_args);
+    case 11: return sizeof(lc_out_proj_args);
     default: return 0;
   }
 }

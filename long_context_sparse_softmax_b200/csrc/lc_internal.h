@@ -14,6 +14,7 @@ cudaError_t launch_qk_prep(const lc_qk_prep_args& a, cudaStream_t st);
 cudaError_t launch_compress(const lc_compress_args& a, bool per_cta, cudaStream_t st);
 cudaError_t launch_mxfp4_quantize(const lc_mxfp4_quant_args& a, cudaStream_t st);
 cudaError_t launch_index_compress(const lc_index_compress_args& a, cudaStream_t st);
+cudaError_t launch_out_proj(const lc_out_proj_args& a, cudaStream_t st);
 cudaError_t launch_index_scores(const lc_index_args& a, bool decode, cudaStream_t st);
 cudaError_t launch_topk(const lc_topk_args& a, bool decode, cudaStream_t st);
 // idx[q, :] = -1 and count[q] = 0 for every query

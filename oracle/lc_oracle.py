@@ -315,6 +315,18 @@ def hca_attn_query(q: np.ndarray, entries: np.ndarray, n_vis: int, win_rows: np.
     return sparse_attn_query(q, entries, range(n_vis), win_rows, win_pos0, p, W, sink, scale, v_dims)
 
 
+def grouped_out_proj(o: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """Grouped output projection (10100.com analysis §三.1): the H heads of each query form G
+    groups of H/G consecutive heads; group g maps the concatenation of its heads' outputs
+    (K = (H/G) Dv values) to its own d_g outputs with its own weights W_g [K, d_g].
+    o [n, H, Dv]; w [G, K, d_g] -> [n, G d_g] (group g's outputs at columns g d_g ..)."""
+    n, H, Dv = o.shape
+    G, K, d_g = w.shape
+    Hg = H // G
+    assert Hg * G == H and Hg * Dv == K
+    return np.concatenate([o[:, g * Hg:(g + 1) * Hg, :].reshape(n, K) @ w[g] for g in range(G)], axis=1)
+
+
 # =====================================================================================
 # Decode-time cache maintenance
 # =====================================================================================

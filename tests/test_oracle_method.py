@@ -426,3 +426,18 @@ def test_nope_values_match_sdpa_and_the_full_value_output():
     np.testing.assert_allclose(o, ref[:, 0].numpy(), rtol=1e-12, atol=1e-14)
     # RoPE dims first in the row (the FP32 layout): the value dims are the rest
     assert np.array_equal(O.nope_dims(128, 0, 64), np.arange(64, 128))
+
+
+# ------------------------------------------------------------------ grouped output projection
+def test_grouped_projection_is_a_block_diagonal_dense_projection():
+    """Grouped projection = the dense projection of the concatenated head outputs by the
+    block-diagonal matrix of the groups' weights (scipy's block_diag, numpy matmul)."""
+    from scipy.linalg import block_diag
+    n, H, Dv, G, d_g = 5, 8, 6, 4, 3
+    o = RNG.standard_normal((n, H, Dv))
+    w = RNG.standard_normal((G, (H // G) * Dv, d_g))
+    ref = o.reshape(n, H * Dv) @ block_diag(*w)
+    np.testing.assert_allclose(O.grouped_out_proj(o, w), ref, rtol=1e-13, atol=1e-13)
+    # one group is the dense projection
+    w1 = RNG.standard_normal((1, H * Dv, 7))
+    np.testing.assert_allclose(O.grouped_out_proj(o, w1), o.reshape(n, -1) @ w1[0], rtol=1e-13)
