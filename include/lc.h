@@ -213,6 +213,10 @@ typedef struct lc_index_args {
   float* scores;           /* [n_q, score_stride] */
   int64_t score_stride;    /* >= max_ent, multiple of 4 */
   int32_t* status;
+  int32_t spin_limit;      /* polls a bounded wait of the MXFP4 kernel makes before it gives up
+                              (LC_DEV_TIMEOUT, results undefined, every copy and MMA in flight
+                              drained before the CTA exits); 0: the default (~2^26) */
+  int32_t reserved;
 } lc_index_args;
 
 lc_status lc_csa_index_scores_prefill(const lc_index_args* a, void* stream);

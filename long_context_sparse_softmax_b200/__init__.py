@@ -64,7 +64,8 @@ class IndexArgs(ctypes.Structure):
     _fields_ = [("n_q", c_int32), ("H_I", c_int32), ("d_I", c_int32), ("fmt", c_int32), ("q", c_void_p),
                 ("q_scale", c_void_p), ("k", c_void_p), ("k_scale", c_void_p), ("n_keys", c_int64), ("w", c_void_p),
                 ("w_qstride", c_int32), ("m", c_int32), ("W_x", c_int32), ("max_ent", c_int32), ("batch", Batch),
-                ("scores", c_void_p), ("score_stride", c_int64), ("status", c_void_p)]
+                ("scores", c_void_p), ("score_stride", c_int64), ("status", c_void_p), ("spin_limit", c_int32),
+                ("reserved", c_int32)]
 
 
 class TopkArgs(ctypes.Structure):

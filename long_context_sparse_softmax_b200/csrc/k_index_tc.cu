@@ -173,15 +173,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int n_tiles = t_end - t_begin;
 
+  // a caller-set limit counts immediate polls (test_wait), so that a small one runs out
+  // for certain; the default counts try_wait polls, which may suspend briefly
+  const long spin = a.spin_limit > 0 ? a.spin_limit : kSpin;
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
     const uint32_t addr = su32(bar);
-    for (long it = 0; it < kSpin; ++it) {
-      if (mbar_test(addr, parity)) return true;
+    for (long it = 0; it < spin; ++it) {
+      if (a.spin_limit > 0 ? mbar_probe(addr, parity) : mbar_test(addr, parity)) return true;
       if ((it & 1023) == 1023 && *reinterpret_cast<volatile int*>(&s_abort)) return false;
     }
     set_status(a.status, LC_DEV_TIMEOUT);
     atomicExch(&s_abort, 1);
     return false;
+  };
+  // before a role ends: the completion of an asynchronous operation it started (a bulk copy
+  // landing, its MMAs finishing) - finite on the hardware, so the default limit applies even
+  // after an abort; giving up here is reported too
+  auto drain = [&](uint64_t* bar, uint32_t parity) {
+    const uint32_t addr = su32(bar);
+    for (long it = 0; it < kSpin; ++it)
+      if (mbar_test(addr, parity)) return;
+    set_status(a.status, LC_DEV_TIMEOUT);
   };
 
   if (warp == 1) {
@@ -227,6 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = 0; u < 4; ++u)
       if (u < n_tiles) sf_load(u, sfw[u]);
     bool go = true;
+    int issued = 0;  // key tiles whose bulk copy this warp started
     for (int it0 = 0; go && it0 < n_tiles; it0 += 4) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -246,9 +259,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint4*>(SFs + s * kKeys + 4 * lane) = make_uint4(sfw[u][0], sfw[u][1], sfw[u][2], sfw[u][3]);
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // the tensor core reads them
         mbar_arrive(full);
+        ++issued;
         if (it + 4 < n_tiles) sf_load(it + 4, sfw[u]);
       }
     }
+    // every copy this warp started has landed before the CTA goes on (after an abort the
+    // shared memory it writes is reused, then released): the last copy into each stage
+    if (lane == 0)
+      for (int it = max(0, issued - kStages); it < issued; ++it) drain(&bars.kfull[it % kStages], (it / kStages) & 1);
+    __syncwarp();
   } else if (warp == 1) {
     // ================= MMA issue (one lane) =================
     if (lane == 0) {
@@ -290,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
           su32(&bars.fin)));
-      wait(&bars.fin, 0);
+      drain(&bars.fin, 0);  // every MMA and scale copy complete before tensor memory is released
     }
   } else {
     // ================= warps 2-5: key scales into tensor memory, epilogue =================
