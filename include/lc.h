@@ -216,7 +216,10 @@ typedef struct lc_index_args {
   int32_t spin_limit;      /* polls a bounded wait of the MXFP4 kernel makes before it gives up
                               (LC_DEV_TIMEOUT, results undefined, every copy and MMA in flight
                               drained before the CTA exits); 0: the default (~2^26) */
-  int32_t reserved;
+  int32_t pdl;             /* 1: programmatic dependent launch - the MXFP4 call may start while
+                              the kernel before it in the stream still runs, and reads q and
+                              q_scale only after that kernel completes; every other input must
+                              be complete before that kernel starts.  0: ordinary ordering */
 } lc_index_args;
 
 lc_status lc_csa_index_scores_prefill(const lc_index_args* a, void* stream);
@@ -234,7 +237,8 @@ typedef struct lc_topk_args {
   int32_t m;
   int32_t W_x;
   int32_t max_ent;         /* host value */
-  int32_t reserved;
+  int32_t pdl;             /* 1: may start while the kernel before it in the stream (the
+                              indexer) runs; reads the scores only after it completes */
   const float* scores;     /* [n_q, score_stride], 16-byte aligned */
   int64_t score_stride;    /* >= max_ent, multiple of 4 */
   lc_batch batch;          /* q_start, q_pos0, n_ent */
@@ -372,6 +376,9 @@ typedef struct lc_attn_args {
   int32_t v_nope;          /* 0: the values are the whole D-dim key rows (out [n_q, H, D]);
                               1: the values are the D - d_r non-RoPE dims of each key row, in
                               logical order (out [n_q, H, D - d_r]); needs d_r > 0 */
+  int32_t pdl;             /* 1: may start while the kernel before it in the stream (the top-k)
+                              runs, and reads idx only after that kernel completes; every other
+                              input must be complete before that kernel starts */
 } lc_attn_args;
 
 /* Attention kernels. */

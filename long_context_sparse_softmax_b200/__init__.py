@@ -65,12 +65,12 @@ class IndexArgs(ctypes.Structure):
                 ("q_scale", c_void_p), ("k", c_void_p), ("k_scale", c_void_p), ("n_keys", c_int64), ("w", c_void_p),
                 ("w_qstride", c_int32), ("m", c_int32), ("W_x", c_int32), ("max_ent", c_int32), ("batch", Batch),
                 ("scores", c_void_p), ("score_stride", c_int64), ("status", c_void_p), ("spin_limit", c_int32),
-                ("reserved", c_int32)]
+                ("pdl", c_int32)]
 
 
 class TopkArgs(ctypes.Structure):
     _fields_ = [("n_q", c_int32), ("k", c_int32), ("m", c_int32), ("W_x", c_int32), ("max_ent", c_int32),
-                ("reserved", c_int32), ("scores", c_void_p), ("score_stride", c_int64), ("batch", Batch),
+                ("pdl", c_int32), ("scores", c_void_p), ("score_stride", c_int64), ("batch", Batch),
                 ("idx", c_void_p), ("count", c_void_p), ("status", c_void_p)]
 
 
@@ -102,7 +102,7 @@ class AttnArgs(ctypes.Structure):
                 ("win", Rows), ("idx", c_void_p), ("sink", c_void_p), ("batch", Batch), ("out", c_void_p),
                 ("lse", c_void_p), ("workspace", c_void_p), ("workspace_bytes", c_size_t), ("status", c_void_p),
                 ("impl", c_int32), ("n_ent_rows", c_int32),
-                ("n_win_rows", c_int32), ("v_nope", c_int32)]
+                ("n_win_rows", c_int32), ("v_nope", c_int32), ("pdl", c_int32)]
 
 
 LC_IMPL_AUTO, LC_IMPL_TC, LC_IMPL_REF = 0, 2, 3

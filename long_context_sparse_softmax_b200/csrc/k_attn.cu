@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(256) k_attn_ref(lc_attn_args a, int sparse) {
   const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
   const int q = blockIdx.x;
   const int H = a.dims.H, D = a.dims.D, d_r = a.dims.d_r;
+  if (a.pdl) asm volatile("griddepcontrol.wait;\n" ::: "memory");  // the previous kernel's top-k
   if (h >= H) return;
   const int b = seq_of_query(a.batch.q_start, a.batch.num_seqs, q);
   const int p = __ldg(a.batch.q_pos0 + b) + (q - __ldg(a.batch.q_start + b));
@@ -177,8 +178,7 @@ cudaError_t launch_attn(const lc_attn_args& a, bool sparse, bool decode, cudaStr
     return launch_attn_combine(a, n_split, st);
   }
   const dim3 grid(a.n_q, (a.dims.H + 7) / 8);
-  k_attn_ref<<<grid, 256, 0, st>>>(a, sparse ? 1 : 0);
-  return cudaGetLastError();
+  return launch_ex(k_attn_ref, grid, dim3(256), 0, st, a.pdl != 0, 1, a, sparse ? 1 : 0);
 }
 
 }  // namespace lc

@@ -242,6 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) TcBars bars;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (a.pdl) pdl_wait();  // the previous kernel's top-k indices (programmatic dependent launch)
   const int n_hg = a.dims.H / kNR;
   const int split = blockIdx.x % geo.n_split;
   const int hg = (blockIdx.x / geo.n_split) % n_hg;
@@ -633,8 +634,8 @@ cudaError_t launch_attn_tc(const lc_attn_args& a, bool sparse, bool decode, cuda
   if (g.n_split > 1) ws_ml = ws_o + static_cast<size_t>(a.n_q) * a.dims.H * g.n_split * kD;
   const int64_t ctas = static_cast<int64_t>(a.n_q) * (a.dims.H / kNR) * g.n_split;
   if (ctas > 0x7fffffff) return cudaErrorInvalidConfiguration;
-  k_attn_tc<<<static_cast<unsigned>(ctas), kThreads, kSmem, st>>>(a, sparse ? 1 : 0, g, ws_o, ws_ml);
-  return cudaGetLastError();
+  return launch_ex(k_attn_tc, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), kSmem, st, a.pdl != 0, 1, a,
+                   sparse ? 1 : 0, g, ws_o, ws_ml);
 }
 
 }  // namespace lc

@@ -317,6 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < n_tiles; ++t) {
       const int cb4 = t & 3;
+      // the top-k indices may be the previous kernel's output (programmatic dependent
+      // launch): the window tiles and Q come in meanwhile
+      if (t == n_wt && a.pdl) pdl_wait();
       // the code buffer of tile t - 4 has been read by its softmax
       bool ok = t < 4 || wait(&bars.cfree[cb4], ((t >> 2) - 1) & 1);
       // raw stage of entry tile e: free once S and the conversion of entry tile e - 2 are
@@ -909,20 +912,9 @@ cudaError_t launch_attn_tc8(const lc_attn_args& a, bool sparse, bool decode, cud
   if (g.n_split > 1 && !g.cluster) ws_ml = ws_o + static_cast<size_t>(a.n_q) * a.dims.H * g.n_split * kD;
   const int64_t ctas = static_cast<int64_t>(a.n_q) * (a.dims.H / kNR) * g.n_split;
   if (ctas > 0x7fffffff) return cudaErrorInvalidConfiguration;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = g.cluster ? g.n_split : 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = g.cluster ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_attn_tc8, tqn, tqr, tkn, tkr, twin, a, sparse ? 1 : 0, decode ? 1 : 0, g, ws_o,
-                            ws_ml);
+  return launch_ex(k_attn_tc8, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), kSmem, st, a.pdl != 0,
+                   g.cluster ? g.n_split : 1, tqn, tqr, tkn, tkr, twin, a, sparse ? 1 : 0, decode ? 1 : 0, g, ws_o,
+                   ws_ml);
 }
 
 }  // namespace lc

@@ -135,6 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int s_q[QPC];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_trigger();  // the merge / top-k after this kernel may start; it waits for our results
   const int qa = blockIdx.x * QPC;
   if (qa >= a.n_q) return;
   // decode: one query per sequence (q_start[b] = b), no search
@@ -161,7 +162,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int t_end = min(t_begin + tiles_per_cta, (nv_max + kKeys - 1) / kKeys);
   if (t_begin >= t_end) {  // uniform over the CTA: nothing allocated yet
     if constexpr (SELECT) {
-      // an empty key range: no candidates (or, alone, an empty selection)
+      // an empty key range: no candidates (or, alone, an empty selection); written only
+      // after the previous kernel, which may still read them, has completed
+      if (a.pdl) pdl_wait();
       if (sel.n_chunks > 1) {
         if (tid == 0) sel.cand_cnt[static_cast<int64_t>(qa) * sel.n_chunks + blockIdx.y] = 0;
       } else {
@@ -317,6 +320,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;                        // tensor-memory lane quadrant of this warp
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const int row = quad * 32 + lane;                 // key row of D this thread reads
+    // the indexer queries may be the previous kernel's output (programmatic dependent
+    // launch): the key tiles above stream in meanwhile
+    if (a.pdl) pdl_wait();
     // query operand (rows n = i * H + h), head weights, query scales
     for (int c = et; c < N * 4; c += 128) {
       const int n = c >> 2, seg = c & 3;
@@ -610,8 +616,8 @@ cudaError_t launch_index_tc(const lc_index_args& a, bool decode, cudaStream_t st
   const dim3 grid(a.n_q, g.n_chunks);
   IdxSelect none{};
   cudaFuncSetAttribute(k_index_tc<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(g.smem));
-  k_index_tc<1, false><<<grid, kThreads, g.smem, st>>>(tk, a, g.tpc, g.tmem_cols, decode ? 1 : 0, none);
-  return cudaGetLastError();
+  return launch_ex(k_index_tc<1, false>, grid, dim3(kThreads), g.smem, st, a.pdl != 0, 1, tk, a, g.tpc, g.tmem_cols,
+                   decode ? 1 : 0, none);
 }
 
 size_t index_topk_workspace(const lc_index_topk_args& a, bool decode) {
@@ -637,8 +643,8 @@ cudaError_t launch_index_topk(const lc_index_topk_args& a, bool decode, cudaStre
   }
   const dim3 grid(a.index.n_q, g.n_chunks);
   cudaFuncSetAttribute(k_index_tc<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(g.smem));
-  k_index_tc<1, true><<<grid, kThreads, g.smem, st>>>(tk, a.index, g.tpc, g.tmem_cols, decode ? 1 : 0, sel);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_ex(k_index_tc<1, true>, grid, dim3(kThreads), g.smem, st, a.index.pdl != 0, 1, tk, a.index,
+                            g.tpc, g.tmem_cols, decode ? 1 : 0, sel);
   if (e != cudaSuccess || g.n_chunks == 1) return e;
   return launch_topk_merge(a, g.n_chunks, sel.cand, sel.cand_cnt, decode, st);
 }

@@ -21,6 +21,7 @@
 #include <cooperative_groups.h>
 
 #include "lc_internal.h"
+#include "lc_ptx.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -62,6 +63,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
   const int rank = static_cast<int>(cl.block_rank());
   const int q = blockIdx.x / C;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_trigger();
+  if (a.pdl) pdl_wait();  // the scores of the indexer before this kernel
   // decode: one query per sequence (q_start[b] = b), no search
   const int b = decode ? q : seq_of_query(a.batch.q_start, a.batch.num_seqs, q);
   const int p = __ldg(a.batch.q_pos0 + b) + (decode ? 0 : q - __ldg(a.batch.q_start + b));
@@ -510,6 +513,8 @@ __global__ void __launch_bounds__(kMergeThreads) k_topk_merge(int k, int m, int 
   __shared__ uint32_t s_rng[2][kMergeWarps];
   const int q = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_trigger();
+  pdl_wait();  // the indexer's candidates (launched right after it, programmatically)
   const int b = decode ? q : seq_of_query(batch.q_start, batch.num_seqs, q);
   const int p = __ldg(batch.q_pos0 + b) + (decode ? 0 : q - __ldg(batch.q_start + b));
   const int nv = n_visible(p, m, W_x, __ldg(batch.n_ent + b));
@@ -641,9 +646,8 @@ cudaError_t launch_topk_merge(const lc_index_topk_args& a, int n_chunks, const u
   const int cached = n_max <= kMergeCache ? 1 : 0;
   const size_t sm = cached ? static_cast<size_t>(n_max) * 4 : 0;
   cudaFuncSetAttribute(k_topk_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, kMergeCache * 4);
-  k_topk_merge<<<a.index.n_q, kMergeThreads, sm, st>>>(a.k, a.index.m, a.index.W_x, a.index.batch, cand, cand_cnt,
-                                                        n_chunks, a.idx, a.count, decode ? 1 : 0, cached);
-  return cudaGetLastError();
+  return launch_ex(k_topk_merge, dim3(a.index.n_q), dim3(kMergeThreads), sm, st, true, 1, a.k, a.index.m, a.index.W_x,
+                   a.index.batch, cand, cand_cnt, n_chunks, a.idx, a.count, decode ? 1 : 0, cached);
 }
 
 __global__ void k_empty_selection(int32_t* idx, int32_t* count, int n_q, int k) {
@@ -677,13 +681,15 @@ cudaError_t launch_topk(const lc_topk_args& a, bool decode, cudaStream_t st) {
   cfg.blockDim = dim3(kTopkThreads);
   cfg.dynamicSmemBytes = sm;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = a.pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, k_topk, a, use_cache, decode ? 1 : 0);
 }
 

@@ -187,6 +187,13 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b,
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization
+// may start while the kernel before it in the stream still runs; pdl_wait() returns once
+// that kernel has completed and its writes are visible (at once when there is none), and
+// pdl_trigger() lets the kernel after this one start early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // 2^x (approximate, flush-to-zero), the softmax exponent
 __device__ __forceinline__ float ex2(float x) {
   float y;

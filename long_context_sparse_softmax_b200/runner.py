@@ -12,6 +12,7 @@ Nothing here computes any part of the method; every step is a kernel of liblc.so
 """
 from __future__ import annotations
 
+import functools
 from typing import Dict, Optional
 
 import torch
@@ -129,6 +130,18 @@ class _Common:
 
     def quant_q(self, stream=None):
         lc_mxfp4_quantize(self.a_quant_q, stream)
+
+    def _index_stages(self):
+        """The indexer and top-k stages of a step.  On the main stream each follows another
+        kernel of the step whose outputs alone it reads after that kernel completes, so it
+        is launched programmatically (its set-up and the loads of its other inputs overlap
+        the previous kernel): the indexer after the query quantisation, the top-k after the
+        indexer, and the attention (see stages()) after the top-k.  Called on their own,
+        the stages launch in plain stream order."""
+        pdl_index = self.spec.idx_fmt == wl.IDX_MXFP4  # quant_q runs right before it
+        if self.fused:
+            return [("index_topk", functools.partial(self.index_topk, pdl=pdl_index))]
+        return [("index", functools.partial(self.index, pdl=pdl_index)), ("topk", functools.partial(self.topk, pdl=True))]
 
     def step_overlapped(self, main, side, on_stage=None, io=None):
         """One step on several streams: the side stages fork from `main` (stage i on
@@ -300,16 +313,21 @@ class Prefill(_Common):
     def index_compress(self, stream=None):
         lc_csa_index_compress_prefill(self.a_index_compress, stream)
 
-    def index(self, stream=None):
+    # pdl: launch programmatically after the previous kernel of the step (see stages())
+    def index(self, stream=None, pdl=False):
+        self.a_index.pdl = int(pdl)
         lc_csa_index_scores_prefill(self.a_index, stream)
 
-    def topk(self, stream=None):
+    def topk(self, stream=None, pdl=False):
+        self.a_topk.pdl = int(pdl)
         lc_csa_topk_prefill(self.a_topk, stream)
 
-    def index_topk(self, stream=None):
+    def index_topk(self, stream=None, pdl=False):
+        self.a_index_topk.index.pdl = int(pdl)
         lc_csa_index_topk_prefill(self.a_index_topk, stream)
 
-    def attn(self, stream=None):
+    def attn(self, stream=None, pdl=False):
+        self.a_attn.pdl = int(pdl)
         (lc_csa_sparse_attn_prefill if self.spec.is_csa else lc_hca_attn_prefill)(self.a_attn, stream)
 
     def stages(self):
@@ -318,8 +336,8 @@ class Prefill(_Common):
         if s.is_csa:
             if s.idx_fmt == wl.IDX_MXFP4:
                 st += [("index_compress", self.index_compress), ("quant_q", self.quant_q)]
-            st += [("index_topk", self.index_topk)] if self.fused else [("index", self.index), ("topk", self.topk)]
-        return st + [("attn", self.attn)]
+            st += self._index_stages()
+        return st + [("attn", functools.partial(self.attn, pdl=s.is_csa))]
 
     def step(self, stream=None):
         for _, f in self.stages():
@@ -395,16 +413,21 @@ class Decode(_Common):
     def index_compress(self, stream=None):
         lc_csa_index_compress_decode(self.a_index_compress, stream)
 
-    def index(self, stream=None):
+    # pdl: launch programmatically after the previous kernel of the step (see stages())
+    def index(self, stream=None, pdl=False):
+        self.a_index.pdl = int(pdl)
         lc_csa_index_scores_decode(self.a_index, stream)
 
-    def topk(self, stream=None):
+    def topk(self, stream=None, pdl=False):
+        self.a_topk.pdl = int(pdl)
         lc_csa_topk_decode(self.a_topk, stream)
 
-    def index_topk(self, stream=None):
+    def index_topk(self, stream=None, pdl=False):
+        self.a_index_topk.index.pdl = int(pdl)
         lc_csa_index_topk_decode(self.a_index_topk, stream)
 
-    def attn(self, stream=None):
+    def attn(self, stream=None, pdl=False):
+        self.a_attn.pdl = int(pdl)
         (lc_csa_sparse_attn_decode if self.spec.is_csa else lc_hca_attn_decode)(self.a_attn, stream)
 
     def stages(self):
@@ -413,8 +436,8 @@ class Decode(_Common):
         if s.is_csa:
             if s.idx_fmt == wl.IDX_MXFP4:
                 st += [("index_compress", self.index_compress), ("quant_q", self.quant_q)]
-            st += [("index_topk", self.index_topk)] if self.fused else [("index", self.index), ("topk", self.topk)]
-        return st + [("attn", self.attn)]
+            st += self._index_stages()
+        return st + [("attn", functools.partial(self.attn, pdl=s.is_csa))]
 
     def step(self, stream=None):
         for _, f in self.stages():
