@@ -149,6 +149,9 @@ def stage_work(spec, inp, run):
             # fused: the keys and queries in, the selection out; no score matrix
             work["index_topk"] = (sum(v * idx_key_b for v in nv) + B * idx_q_b + B * 4 * s.k,
                                   sum(2 * v * s.H_I * s.d_I for v in nv))
+            # raw BF16 indexer rows quantised on the GPU: the query rows, the key of the closed block
+            work["quant_q"] = (B * s.H_I * (2 * s.d_I + idx_key_b), 0)
+            work["index_compress"] = (n_blk * (s.m * (2 * s.d_I + 4) + idx_key_b), 0)
             sel = K
         else:
             sel = nv
@@ -173,6 +176,8 @@ def stage_work(spec, inp, run):
             work["topk"] = (int(nv.sum()) * 4 + s.n_q * 4 * s.k, 0)
             work["index_topk"] = (n_c * idx_key_b + s.n_q * idx_q_b + s.n_q * 4 * s.k,
                                   int(nv.sum()) * 2 * s.H_I * s.d_I)
+            work["quant_q"] = (s.n_q * s.H_I * (2 * s.d_I + idx_key_b), 0)
+            work["index_compress"] = (n_c * (s.m * (2 * s.d_I + 4) + idx_key_b), 0)
             sel = K
         else:
             sel = nv

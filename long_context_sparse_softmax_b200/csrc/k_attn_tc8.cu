@@ -199,7 +199,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ring = a.batch.win_ring;
   const int wbase = ring > 0 ? (wlo & ~(kTK - 1)) : wlo;
   const int n_first = sparse ? a.k : nv;
-  const int n_slots = n_first + (p + 1 - wbase);
+  // the first window slot: right after the entries, or, for a ring, at the next multiple of
+  // 64 (the slots between are dead), so that every window tile starts on a 64-position
+  // boundary whatever split it falls in
+  const int w_slot0 = ring > 0 ? (n_first + kTK - 1) / kTK * kTK : n_first;
+  const int n_slots = w_slot0 + (p + 1 - wbase);
   int s_begin, s_end;
   if (!geo.win_own) {
     s_begin = split * geo.sps;
@@ -214,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // entry tiles cover [s_begin, min(s_end, n_first)), window tiles the rest of the range
   const int e_end = min(s_end, n_first);
   const int n_et = e_end > s_begin ? (e_end - s_begin + kTK - 1) / kTK : 0;
-  const int w_begin = max(s_begin, n_first);
+  const int w_begin = max(s_begin, w_slot0);
   const int n_wt = s_end > w_begin ? (s_end - w_begin + kTK - 1) / kTK : 0;
   const int n_tiles = n_et + n_wt;
   const int wp0 = a.W > 0 ? __ldg(a.batch.win_pos0 + b) : 0;
@@ -257,7 +261,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return j;
     }
-    const int t = wbase + (s - n_first);
+    if (s < w_slot0) return -1;  // dead slots before a ring-aligned window
+    const int t = wbase + (s - w_slot0);
     if (t < wlo) return -1;  // ring alignment: before the window
     const int rr = t - wp0;
     if (rr < 0 || rr >= wl) {
@@ -473,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ct == 0) {
           const uint32_t wb = su32(&bars.wfull);
           mbar_expect_tx(wb, kTile);
-          const int t0 = wbase + (tile_slot0(t) - n_first);  // first position of the tile
+          const int t0 = wbase + (tile_slot0(t) - w_slot0);  // first position of the tile
           const int y = static_cast<int>(wr0) + (ring > 0 ? t0 % ring : t0 - wp0);
 #pragma unroll
           for (int cb = 0; cb < kD / 64; ++cb) tma_tile2d(su32(Vt + cb * kBlk), &twin, cb * 64, y, wb);
@@ -823,8 +828,10 @@ static AttnTc8Geom tc8_geometry(const lc_attn_args& a, bool sparse, bool decode)
   AttnTc8Geom g{1, 0, 0, 0};
   const int ne = sparse ? a.k : a.max_ent;
   // window slots: W, or up to W + 63 when ring-aligned window tiles start before the window
-  const int wslots = a.W > 0 && a.batch.win_ring > 0 ? a.W + kTK - 1 : a.W;
-  const int ns = max(ne + wslots, 1);
+  const bool ring = a.W > 0 && a.batch.win_ring > 0;
+  const int wslots = ring ? a.W + kTK - 1 : a.W;
+  const int ne_pad = ring ? (ne + kTK - 1) / kTK * kTK : ne;  // window slots start on a tile
+  const int ns = max(ne_pad + wslots, 1);
   const int tiles = (ns + kTK - 1) / kTK;
   g.sps = tiles * kTK;
   const int ctas = a.n_q * (a.dims.H / kNR);

@@ -57,3 +57,19 @@ def test_host_inputs_name_the_stage_that_reads_them():
     # prefill compresses the indexer keys on the main stream, before the indexer reads them
     assert hp["index_compress"][0] is ip["kI_raw"] and hp["quant_q"][0] is ip["qI_raw"]
     assert [n for n, _ in rp.dag()[1]] == ["index_compress", "quant_q", "index_topk"]
+
+
+@pytest.mark.parametrize("name", ["csa_decode", "csa_prefill", "hca_prefill", "mixed_decode", "tiny_csa_prefill"])
+@pytest.mark.parametrize("fused", [None, False])
+def test_stage_work_covers_every_stage(name, fused):
+    """The bench counts algorithmic bytes / flops for every stage a step runs."""
+    import dataclasses
+    for spec in wl.WORKLOADS[name]:
+        small = dataclasses.replace(spec, name="sw", seq_lens=tuple(min(L, 3000) for L in spec.seq_lens),
+                                    **({} if spec.is_decode else {"n_q": 64, "q_first": min(spec.seq_lens[0], 3000) - 64}))
+        inp = (wl.make_decode if small.is_decode else wl.make_prefill)(small, "cpu")
+        r = (runner.Decode if small.is_decode else runner.Prefill)(inp, "cpu", fused=fused)
+        work, units = bench.stage_work(small, inp, r)
+        names = [n for n, _ in r.stages()]
+        assert all(n in work for n in names), [n for n in names if n not in work]
+        assert units == (small.num_seqs if small.is_decode else small.n_q)

@@ -90,4 +90,6 @@ def test_indexer_wait_limit_runs_out_cleanly(fused):
         if fused:
             assert torch.equal(run.idx, idx)
         else:
-            assert torch.equal(torch.nan_to_num(run.scores, nan=-1.0), torch.nan_to_num(scores, nan=-1.0))
+            for b, L in enumerate(s.seq_lens):  # the visible columns (the rest is never written)
+                n = O.n_visible(L - 1, s.m, s.W, L // s.m)
+                assert torch.equal(run.scores[b, :n], scores[b, :n])
