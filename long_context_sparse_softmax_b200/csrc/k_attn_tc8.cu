@@ -753,21 +753,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       named_bar(1, 128);
       const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+      // 32 heads at a time: their factors in registers, so that the stores stream (the
+      // compiler cannot tell the factors from the stored rows)
 #pragma unroll 1
-      for (int c = 0; c < n_och; ++c) {
-        const int dim = c < 4 ? c * 128 + warp * 32 + lane : (lane < 16 ? 512 + warp * 16 + lane : -1);
-        uint32_t ov[kNR];
-        if (n_tiles > 0) {
-          tmem_ld32(tm + lane_off + kColO + c * kNR, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
-          tmem_ld32(tm + lane_off + kColO + c * kNR + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
-          tmem_wait_ld();
-        } else {
+      for (int hh = 0; hh < kNR; hh += 32) {
+        float f[32];
 #pragma unroll
-          for (int i = 0; i < kNR; ++i) ov[i] = 0;
+        for (int i = 0; i < 32; ++i) f[i] = s_f[hh + i];
+#pragma unroll 1
+        for (int c = 0; c < n_och; ++c) {
+          const int dim = c < 4 ? c * 128 + warp * 32 + lane : (lane < 16 ? 512 + warp * 16 + lane : -1);
+          uint32_t ov[32];
+          if (n_tiles > 0) {
+            tmem_ld32(tm + lane_off + kColO + c * kNR + hh, ov);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = 0;
+          }
+          if (dim < 0) continue;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) Osm[(hh + i) * kD + dim] = __uint_as_float(ov[i]) * f[i];
         }
-        if (dim < 0) continue;
-#pragma unroll
-        for (int i = 0; i < kNR; ++i) Osm[i * kD + dim] = __uint_as_float(ov[i]) * s_f[i];
       }
     }
     cl.sync();  // every split's scaled O is in its shared memory
@@ -777,25 +784,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float* src[kMaxClusterSplits];
 #pragma unroll
     for (int sp = 0; sp < kMaxClusterSplits; ++sp) src[sp] = sp < geo.n_split ? cl.map_shared_rank(Osm, sp) : Osm;
-    for (int it = tid; it < kNR * nq4; it += kThreads) {
-      const int h = it / nq4, d = d0 + 4 * (it % nq4);
-      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    // kMergeIt outputs per thread at a time, each split's loads for all of them issued
+    // before they are added: the remote loads overlap instead of queueing one by one
+    constexpr int kMergeIt = 6;
+    for (int base = 0; base < kNR * nq4; base += kMergeIt * kThreads) {
+      float4 acc[kMergeIt];
+      int off[kMergeIt];
 #pragma unroll
-      for (int sp = 0; sp < kMaxClusterSplits; ++sp)
-        if (sp < geo.n_split) {
-          const float4 v = *reinterpret_cast<const float4*>(src[sp] + h * kD + d);
-          o.x += v.x;
-          o.y += v.y;
-          o.z += v.z;
-          o.w += v.w;
+      for (int j = 0; j < kMergeIt; ++j) {
+        acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        const int it = base + j * kThreads + tid;
+        off[j] = it < kNR * nq4 ? (it / nq4) * kD + d0 + 4 * (it % nq4) : -1;
+      }
+#pragma unroll
+      for (int sp = 0; sp < kMaxClusterSplits; ++sp) {
+        if (sp >= geo.n_split) break;
+        float4 v[kMergeIt];
+#pragma unroll
+        for (int j = 0; j < kMergeIt; ++j)
+          v[j] = off[j] >= 0 ? *reinterpret_cast<const float4*>(src[sp] + off[j]) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < kMergeIt; ++j) {
+          acc[j].x += v[j].x;
+          acc[j].y += v[j].y;
+          acc[j].z += v[j].z;
+          acc[j].w += v[j].w;
         }
-      const int64_t e = (row0 + h) * Dv + d;
-      if (a.out_fmt == LC_FMT_F32) {
-        *reinterpret_cast<float4*>(static_cast<float*>(a.out) + e) = o;
-      } else {
-        const uint32_t lo = static_cast<uint32_t>(f32_to_bf16_bits(o.x)) | (static_cast<uint32_t>(f32_to_bf16_bits(o.y)) << 16);
-        const uint32_t hi = static_cast<uint32_t>(f32_to_bf16_bits(o.z)) | (static_cast<uint32_t>(f32_to_bf16_bits(o.w)) << 16);
-        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + e) = make_uint2(lo, hi);
+      }
+#pragma unroll
+      for (int j = 0; j < kMergeIt; ++j) {
+        if (off[j] < 0) continue;
+        const int h = off[j] / kD, d = off[j] % kD;
+        const float4 o = acc[j];
+        const int64_t e = (row0 + h) * Dv + d;
+        if (a.out_fmt == LC_FMT_F32) {
+          *reinterpret_cast<float4*>(static_cast<float*>(a.out) + e) = o;
+        } else {
+          const uint32_t lo = static_cast<uint32_t>(f32_to_bf16_bits(o.x)) | (static_cast<uint32_t>(f32_to_bf16_bits(o.y)) << 16);
+          const uint32_t hi = static_cast<uint32_t>(f32_to_bf16_bits(o.z)) | (static_cast<uint32_t>(f32_to_bf16_bits(o.w)) << 16);
+          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + e) = make_uint2(lo, hi);
+        }
       }
     }
     cl.sync();  // no split leaves while another still reads its shared memory

@@ -61,6 +61,7 @@ constexpr uint32_t kColSfb = 16;
 
 constexpr int kSelMaxTiles = 64;    // tiles per CTA in the fused-selection mode (32 KB of scores)
 constexpr int kSelBins = 2048;
+constexpr int kSmallBin = 256;      // the K-th key's first-pass bin is resolved by ranking up to this many
 
 struct IdxBars {
   uint64_t kfull[kStages];   // key tile (expect-tx arrival) and its scale words (32 arrivals) landed
@@ -405,12 +406,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ================= the range's top K (128 threads; the key ring is idle) =================
       // scratch in the idle key ring (dynamic shared memory, so that the static part stays
       // small enough for two CTAs per SM)
-      uint32_t* hist = reinterpret_cast<uint32_t*>(As);   // [kSelBins]
-      uint32_t* bits = hist + kSelBins;                   // [kSelMaxTiles * 4] selection words
-      int (*s_wcnt)[4] = reinterpret_cast<int (*)[4]>(bits + kSelMaxTiles * 4);  // [kSelMaxTiles][4]
-      uint32_t (*s_rng)[4] = reinterpret_cast<uint32_t (*)[4]>(s_wcnt + kSelMaxTiles);  // [2][4]
+      uint32_t* hist4 = reinterpret_cast<uint32_t*>(As);  // [4][kSelBins] per-warp histograms
+      uint32_t* bits = hist4 + 4 * kSelBins;              // [kSelMaxTiles * 4] selection words
+      int (*s_wcnt)[4] = reinterpret_cast<int (*)[4]>(bits + kSelMaxTiles * 4);   // [kSelMaxTiles][4]
+      uint32_t* list_key = reinterpret_cast<uint32_t*>(s_wcnt + kSelMaxTiles);     // [kSmallBin]
+      int* list_off = reinterpret_cast<int*>(list_key + kSmallBin);                // [kSmallBin]
+      uint32_t (*s_rng)[4] = reinterpret_cast<uint32_t (*)[4]>(list_off + kSmallBin);  // [2][4]
       int* s_tmp = reinterpret_cast<int*>(s_rng + 2);     // [4]
-      int* s_pick = s_tmp + 4;                            // [2]
+      int* s_pick = s_tmp + 4;                            // [3]
+      int* s_cnt = s_pick + 3;                            // [1]
+      uint32_t* s_thr = reinterpret_cast<uint32_t*>(s_cnt + 1);  // [2]: Tk, Ts
       const int q = s_q[0];
       const int jbase = t_begin * kKeys;
       const int n_valid = max(0, min(s_nv[0] - jbase, n_tiles * kKeys));
@@ -433,76 +438,123 @@ __global__ void __launch_bounds__(kThreads, 1)
         s_rng[0][quad] = kmin;
         s_rng[1][quad] = kmax;
       }
+      if (row == 0) {
+        *s_cnt = 0;
+        s_thr[0] = 0u;           // every valid key is taken unless a threshold is found
+        s_thr[1] = 0x7fffffffu;
+      }
       named_bar(1, 128);
       const uint32_t umin = min(min(s_rng[0][0], s_rng[0][1]), min(s_rng[0][2], s_rng[0][3]));
       const uint32_t umax = max(max(s_rng[1][0], s_rng[1][1]), max(s_rng[1][2], s_rng[1][3]));
-      // radix passes over rel = key - umin from the top, 11 bits at a time: pfx holds the
-      // bits of the K-th largest rel found so far, rem the keys still to take inside the
-      // bin they select
-      const bool take_all = K == n_valid;
-      uint32_t pfx = 0;
-      int rem = K;
-      int shift = take_all ? 0 : 32 - __clz(static_cast<int>(umax - umin));
+      // The selection is the pair (Tk, Ts): the K-th largest key and the offset of the last
+      // selected key equal to it; offset o is taken iff key > Tk, or key == Tk and o <= Ts.
+      // Radix passes of 11 bits over rel = key - umin (histograms kept per warp, summed per
+      // bin) narrow the bin of the K-th key until it holds at most kSmallBin keys, usually
+      // after one pass; those are ranked exactly (key descending, offset ascending).  A bin
+      // of more than kSmallBin equal keys is ranked in offset order.
+      if (K < n_valid) {
+        uint32_t pfx = 0;
+        int rem = K, in_bin = n_valid;
+        int shift = 32 - __clz(static_cast<int>(umax - umin));
 #pragma unroll 1
-      while (shift > 0) {
-        const int w = min(11, shift);
-        const int hi = shift;
-        shift -= w;
-        const uint32_t bmask = (1u << w) - 1u;
-        for (int i = row; i < kSelBins; i += 128) hist[i] = 0;
-        named_bar(1, 128);
-        for (int u = 0; u < n_tiles; ++u)
-          if (valid(u)) {
-            const uint32_t rel = order_key(sc[u * kKeys + row]) - umin;
-            const uint32_t top = hi >= 32 ? 0u : rel >> hi;
-            if (top == pfx) atomicAdd(&hist[(rel >> shift) & bmask], 1u);
-          }
-        named_bar(1, 128);
-        // descending: thread `row` owns bins 2047 - 16 row - i, i < 16
-        int c[16], sum = 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          c[i] = static_cast<int>(hist[kSelBins - 1 - 16 * row - i]);
-          sum += c[i];
-        }
-        int tot;
-        int run = scan128(sum, quad, lane, s_tmp, &tot);
-        if (run < rem && run + sum >= rem) {
-#pragma unroll 1
-          for (int i = 0; i < 16; ++i) {
-            if (run + c[i] >= rem) {
-              s_pick[0] = kSelBins - 1 - 16 * row - i;
-              s_pick[1] = rem - run;
-              break;
+        while (in_bin > kSmallBin && shift > 0) {
+          const int w = min(11, shift);
+          const int hi = shift;
+          shift -= w;
+          const uint32_t bmask = (1u << w) - 1u;
+          for (int i = row; i < 4 * kSelBins; i += 128) hist4[i] = 0;
+          named_bar(1, 128);
+          for (int u = 0; u < n_tiles; ++u)
+            if (valid(u)) {
+              const uint32_t rel = order_key(sc[u * kKeys + row]) - umin;
+              if ((hi >= 32 ? 0u : rel >> hi) == pfx) atomicAdd(&hist4[quad * kSelBins + ((rel >> shift) & bmask)], 1u);
             }
-            run += c[i];
+          named_bar(1, 128);
+          // descending: thread `row` owns bins 2047 - 16 row - i, i < 16
+          int c[16], sum = 0;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int bin = kSelBins - 1 - 16 * row - i;
+            c[i] = static_cast<int>(hist4[bin] + hist4[kSelBins + bin] + hist4[2 * kSelBins + bin] +
+                                    hist4[3 * kSelBins + bin]);
+            sum += c[i];
+          }
+          int tot;
+          int run = scan128(sum, quad, lane, s_tmp, &tot);
+          if (run < rem && run + sum >= rem) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              if (run < rem && run + c[i] >= rem) {
+                s_pick[0] = kSelBins - 1 - 16 * row - i;
+                s_pick[1] = rem - run;
+                s_pick[2] = c[i];
+              }
+              run += c[i];
+            }
+          }
+          named_bar(1, 128);
+          pfx = (pfx << w) | static_cast<uint32_t>(s_pick[0]);
+          rem = s_pick[1];
+          in_bin = s_pick[2];
+        }
+        if (in_bin <= kSmallBin) {
+          for (int u = 0; u < n_tiles; ++u)
+            if (valid(u)) {
+              const uint32_t key = order_key(sc[u * kKeys + row]);
+              if (shift >= 32 || ((key - umin) >> shift) == pfx) {
+                const int i = atomicAdd(s_cnt, 1);
+                if (i < kSmallBin) {  // exactly in_bin keys arrive here
+                  list_key[i] = key;
+                  list_off[i] = u * kKeys + row;
+                }
+              }
+            }
+          named_bar(1, 128);
+          for (int i = row; i < in_bin; i += 128) {
+            const uint32_t ki = list_key[i];
+            const int oi = list_off[i];
+            int r = 0;
+            for (int j = 0; j < in_bin; ++j) {
+              const uint32_t kj = list_key[j];
+              r += kj > ki || (kj == ki && list_off[j] < oi);
+            }
+            if (r == rem - 1) {
+              s_thr[0] = ki;
+              s_thr[1] = static_cast<uint32_t>(oi);
+            }
+          }
+        } else {
+          // every key of the bin equals T: the rem-th of them in offset order (tile, then row)
+          const uint32_t T = umin + pfx;
+          for (int u = 0; u < n_tiles; ++u) {
+            const bool eq = valid(u) && order_key(sc[u * kKeys + row]) == T;
+            const uint32_t bal = __ballot_sync(0xffffffffu, eq);
+            if (lane == 0) s_wcnt[u][quad] = __popc(bal);
+          }
+          named_bar(1, 128);
+          int eq_before = 0;
+          for (int u = 0; u < n_tiles; ++u) {
+            const bool eq = valid(u) && order_key(sc[u * kKeys + row]) == T;
+            int rank = eq_before + __popc(__ballot_sync(0xffffffffu, eq) & ((1u << lane) - 1u));
+#pragma unroll
+            for (int w = 0; w < 4; ++w) rank += w < quad ? s_wcnt[u][w] : 0;
+            if (eq && rank == rem - 1) {
+              s_thr[0] = T;
+              s_thr[1] = static_cast<uint32_t>(u * kKeys + row);
+            }
+            eq_before += s_wcnt[u][0] + s_wcnt[u][1] + s_wcnt[u][2] + s_wcnt[u][3];
           }
         }
         named_bar(1, 128);
-        pfx = (pfx << w) | static_cast<uint32_t>(s_pick[0]);
-        rem = s_pick[1];
       }
-      const uint32_t T = umin + pfx;
-      // keys equal to T, ranked in index order (u, then row): per-tile warp counts first
+      const uint32_t Tk = s_thr[0];
+      const int Ts = static_cast<int>(s_thr[1]);
       for (int u = 0; u < n_tiles; ++u) {
-        const bool eq = !take_all && valid(u) && order_key(sc[u * kKeys + row]) == T;
-        const uint32_t bal = __ballot_sync(0xffffffffu, eq);
-        if (lane == 0) s_wcnt[u][quad] = __popc(bal);
-      }
-      named_bar(1, 128);
-      int eq_before = 0;
-      for (int u = 0; u < n_tiles; ++u) {
-        const bool v = valid(u);
-        const uint32_t key = v ? order_key(sc[u * kKeys + row]) : 0u;
-        const bool eq = !take_all && v && key == T;
-        // rank among the keys equal to T: earlier tiles, earlier quadrants, earlier lanes
-        int rank = eq_before + __popc(__ballot_sync(0xffffffffu, eq) & ((1u << lane) - 1u));
-#pragma unroll
-        for (int w = 0; w < 4; ++w) rank += w < quad ? s_wcnt[u][w] : 0;
-        const bool pick = v && (take_all || key > T || (eq && rank < rem));
+        const int off = u * kKeys + row;
+        const uint32_t key = valid(u) ? order_key(sc[off]) : 0u;
+        const bool pick = valid(u) && (key > Tk || (key == Tk && off <= Ts));
         const uint32_t word = __ballot_sync(0xffffffffu, pick);
         if (lane == 0) bits[u * 4 + quad] = word;
-        eq_before += s_wcnt[u][0] + s_wcnt[u][1] + s_wcnt[u][2] + s_wcnt[u][3];
       }
       named_bar(1, 128);
       // the selected keys in index order: word w holds keys jbase + 32 w .. + 31

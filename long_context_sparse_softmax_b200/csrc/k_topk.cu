@@ -457,17 +457,28 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(lc_topk_args a, int use_c
 
 // ---------------------------------------------------------------------------------
 // Merge of the fused indexer's candidates (lc_csa_index_topk_* when a query's keys span
-// several CTAs).  Range c of query q left cnt[q][c] candidates (order key, entry index)
-// in ascending index order, at least the range's own top K; the ranges are disjoint and
-// ascending, so the concatenation of their lists is in ascending index order.  One CTA
-// per query selects the K largest keys of the list, ties to the earlier position (the
-// lower index), by radix passes of 11 bits over the keys (held in shared memory when
-// they fit), and writes the selected indices in list order.  Each thread owns a
-// contiguous segment of positions, so the order survives the block-wide scans.
+// several CTAs).  Range c of query q left cnt[q][c] candidates (order key, entry index) in
+// ascending index order in slots c k .. c k + cnt - 1 of the query's [n_chunks][k] block;
+// the ranges are disjoint and ascending, so slot order is index order.  One CTA per query
+// selects the K largest keys, ties to the lower slot, and writes their indices in slot
+// order.  Thread t owns slots t, t + 1024, ... (coalesced loads): up to kMergeRegRounds of
+// them in registers, more in shared memory (kMergeCache keys), beyond that re-read from
+// global memory on each pass.  The selection is the pair (Tk, Ts): the K-th largest key
+// and the slot of the last selected key equal to it; slot s is selected iff key > Tk, or
+// key == Tk and s <= Ts.  Radix passes of 11 bits over rel = key - min narrow the bin that
+// holds the K-th key until it holds at most kSmallBin keys (usually after one pass); those
+// are ranked exactly.  A bin of more than kSmallBin equal keys is ranked in slot order by
+// a block-wide scan, as is the output.
 constexpr int kMergeThreads = 1024;
 constexpr int kMergeWarps = kMergeThreads / 32;
-constexpr int kMergeCache = 48 * 1024;  // keys held in shared memory (192 KB)
-constexpr int kMergeMaxChunks = kMergeThreads;
+constexpr int kMergeRegRounds = 8;        // slots per thread held in registers (n_slots <= 8192)
+constexpr int kMergeCacheKI = 20 * 1024;  // slots whose key and index fit in shared memory
+constexpr int kMergeCacheK = 40 * 1024;   // slots whose key fits in shared memory
+constexpr int kMergeMaxChunks = 1024;
+constexpr int kSmallBin = 256;
+constexpr int kScanRounds = 64;           // slot rounds per block-wide ordering scan
+constexpr int kScanPer = kScanRounds * kMergeWarps / kMergeThreads;
+constexpr int kBatch = 8;                 // rounds whose global loads are issued together
 
 // exclusive prefix of v over the CTA in thread order; *total gets the sum
 __device__ __forceinline__ int scan_cta(int v, int* s_w, int* s_total, int* total) {
@@ -498,22 +509,35 @@ __device__ __forceinline__ int scan_cta(int v, int* s_w, int* s_total, int* tota
   return r;
 }
 
+// R > 0: the slots are held in registers (n_slots <= R * 1024).  R == 0: cache 2 keeps keys
+// and indices in shared memory, cache 1 keys only, cache 0 nothing.
+template <int R>
 __global__ void __launch_bounds__(kMergeThreads) k_topk_merge(int k, int m, int W_x, lc_batch batch,
                                                               const uint2* __restrict__ cand,
                                                               const int* __restrict__ cand_cnt, int n_chunks,
                                                               int32_t* idx, int32_t* count, int decode,
-                                                              int cached) {
+                                                              int cache) {
   static_assert(kMergeWarps == 32, "one warp scans the warp totals");
-  extern __shared__ uint32_t kc[];  // [n] candidate keys (cached)
-  __shared__ int s_off[kMergeMaxChunks + 1];
+  static_assert(R * kMergeWarps <= kMergeThreads, "one scan entry per thread");
+  extern __shared__ uint32_t kc[];
   __shared__ int s_hist[kBins];
+  __shared__ int s_rc[kScanRounds * kMergeWarps];
+  __shared__ uint32_t s_lkey[kSmallBin];
+  __shared__ int s_lslot[kSmallBin];
+  __shared__ int s_cnt[R > 0 ? 1 : kMergeMaxChunks];
   __shared__ int s_w[kMergeWarps];
-  __shared__ int s_total;
-  __shared__ int s_pick[2];
+  __shared__ int s_total, s_lcnt, s_n, s_ts;
+  __shared__ int s_pick[3];
   __shared__ uint32_t s_rng[2][kMergeWarps];
+  __shared__ uint32_t s_tk;
   const int q = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_trigger();
+  for (int i = tid; i < kBins; i += kMergeThreads) s_hist[i] = 0;
+  if (tid == 0) {
+    s_n = 0;
+    s_lcnt = 0;
+  }
   pdl_wait();  // the indexer's candidates (launched right after it, programmatically)
   const int b = decode ? q : seq_of_query(batch.q_start, batch.num_seqs, q);
   const int p = __ldg(batch.q_pos0 + b) + (decode ? 0 : q - __ldg(batch.q_start + b));
@@ -523,131 +547,303 @@ __global__ void __launch_bounds__(kMergeThreads) k_topk_merge(int k, int m, int 
   for (int i = K + tid; i < k; i += kMergeThreads) out[i] = -1;
   if (tid == 0 && count) count[q] = K;
   if (K == 0) return;
-  // offsets of the ranges' lists in the concatenation
-  int n = 0;
-  {
-    // a range writes at most k candidates (the clamp only matters after a timeout upstream)
-    const int v = tid < n_chunks ? min(max(__ldg(cand_cnt + static_cast<int64_t>(q) * n_chunks + tid), 0), k) : 0;
-    const int ex = scan_cta(v, s_w, &s_total, &n);
-    if (tid < n_chunks) s_off[tid] = ex;
-    if (tid == 0) s_off[n_chunks] = n;
-  }
-  __syncthreads();
-  const uint2* cq = cand + static_cast<int64_t>(q) * n_chunks * k;
-  const int seg = (n + kMergeThreads - 1) / kMergeThreads;
-  const int i0 = min(n, tid * seg), i1 = min(n, i0 + seg);
-  int c0 = 0;  // range of position i0: the last c with s_off[c] <= i0
-  {
-    int lo = 0, hi = n_chunks - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_off[mid] <= i0) lo = mid;
-      else hi = mid - 1;
-    }
-    c0 = lo;
-  }
-  // visit the own segment in order: fn(position, candidate)
-  auto each = [&](auto fn) {
-    int c = c0;
-    for (int i = i0; i < i1; ++i) {
-      while (i >= s_off[c + 1]) ++c;
-      fn(i, cq + static_cast<int64_t>(c) * k + (i - s_off[c]));
-    }
+  const int n_slots = n_chunks * k;
+  const int J = (n_slots + kMergeThreads - 1) / kMergeThreads;  // rounds of slots
+  const uint2* cq = cand + static_cast<int64_t>(q) * n_slots;
+  const int* cc = cand_cnt + static_cast<int64_t>(q) * n_chunks;
+  const uint32_t lt = (1u << lane) - 1u;
+  // a range writes at most k candidates (the clamp only matters after a timeout upstream)
+  auto held_g = [&](int slot) {
+    const int c = slot / k;
+    return slot - c * k < min(max(__ldg(cc + c), 0), k);
   };
-  const bool take_all = n <= K;
+  uint32_t key[R > 0 ? R : 1];
+  int id[R > 0 ? R : 1];
+  uint32_t vm = 0;  // R > 0: bit r = round r holds a candidate
+  uint32_t* ks = kc;
+  int* is = reinterpret_cast<int*>(kc + (cache == 2 ? n_slots : 0));
+  uint32_t* vb = kc + (cache == 2 ? 2 * n_slots : cache == 1 ? n_slots : 0);
+  // the key of a slot (R == 0) and whether the slot holds a candidate
+  auto load = [&](int slot, uint32_t& kk) -> bool {
+    if (slot >= n_slots) return false;
+    if (cache) {
+      kk = ks[slot];
+      return (vb[slot >> 5] >> (slot & 31)) & 1u;
+    }
+    const int c = slot / k;
+    if (slot - c * k >= s_cnt[c]) return false;
+    kk = __ldg(&cq[slot].x);
+    return true;
+  };
+  // pass 0: the keys (and indices), their range and count
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  each([&](int i, const uint2* e) {
-    const uint32_t key = __ldg(&e->x);
-    if (cached) kc[i] = key;
-    kmin = min(kmin, key);
-    kmax = max(kmax, key);
-  });
-  auto key_at = [&](int i, const uint2* e) -> uint32_t { return cached ? kc[i] : __ldg(&e->x); };
+  int nmine = 0;
+  if constexpr (R > 0) {
+    bool v[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int slot = r * kMergeThreads + tid;
+      v[r] = slot < n_slots && held_g(slot);
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const uint2 e = v[r] ? __ldg(&cq[r * kMergeThreads + tid]) : make_uint2(0u, 0u);
+      key[r] = e.x;
+      id[r] = static_cast<int>(e.y);
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (v[r]) {
+        vm |= 1u << r;
+        kmin = min(kmin, key[r]);
+        kmax = max(kmax, key[r]);
+        ++nmine;
+      }
+  } else {
+    for (int c = tid; c < n_chunks; c += kMergeThreads) s_cnt[c] = min(max(__ldg(cc + c), 0), k);
+#pragma unroll 1
+    for (int j0 = 0; j0 < J; j0 += kBatch) {
+      uint2 e[kBatch];
+      bool v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int slot = (j0 + u) * kMergeThreads + tid;
+        v[u] = slot < n_slots && held_g(slot);
+        e[u] = v[u] ? __ldg(&cq[slot]) : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int slot = (j0 + u) * kMergeThreads + tid;
+        if (j0 + u < J) {
+          const uint32_t bal = __ballot_sync(0xffffffffu, v[u]);
+          if (cache && slot < n_slots) {
+            ks[slot] = e[u].x;
+            if (cache == 2) is[slot] = static_cast<int>(e[u].y);
+            if (lane == 0) vb[slot >> 5] = bal;
+          }
+        }
+        if (v[u]) {
+          kmin = min(kmin, e[u].x);
+          kmax = max(kmax, e[u].x);
+          ++nmine;
+        }
+      }
+    }
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
     kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    nmine += __shfl_xor_sync(0xffffffffu, nmine, o);
   }
   if (lane == 0) {
     s_rng[0][warp] = kmin;
     s_rng[1][warp] = kmax;
+    atomicAdd(&s_n, nmine);
   }
   __syncthreads();
   uint32_t umin = 0xffffffffu, umax = 0u;
-#pragma unroll 4
+#pragma unroll 8
   for (int w = 0; w < kMergeWarps; ++w) {
     umin = min(umin, s_rng[0][w]);
     umax = max(umax, s_rng[1][w]);
   }
-  // radix passes (see k_topk): pfx = bits of the K-th largest rel = key - umin so far,
-  // rem = keys still to take inside the bin they select
-  uint32_t pfx = 0;
-  int rem = K;
-  int shift = take_all ? 0 : 32 - __clz(static_cast<int>(umax - umin));
+  const int n = s_n;
+  // fn(slot, key) for every candidate this thread owns
+  auto each = [&](auto fn) {
+    if constexpr (R > 0) {
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+        if ((vm >> r) & 1u) fn(r * kMergeThreads + tid, key[r]);
+    } else {
+#pragma unroll 4
+      for (int j = 0; j < J; ++j) {
+        const int slot = j * kMergeThreads + tid;
+        uint32_t kk;
+        if (load(slot, kk)) fn(slot, kk);
+      }
+    }
+  };
+  // slot-order ranks of the candidates where pred(slot, key) holds: fn(slot, rank, index)
+  // (index: the entry index when it is at hand, else -1)
+  auto ordered = [&](auto pred, auto fn) {
+    if constexpr (R > 0) {
+      uint32_t bal[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int slot = r * kMergeThreads + tid;
+        bal[r] = __ballot_sync(0xffffffffu, ((vm >> r) & 1u) && pred(slot, key[r]));
+        if (lane == 0) s_rc[r * kMergeWarps + warp] = __popc(bal[r]);
+      }
+      __syncthreads();
+      const int a0 = tid < R * kMergeWarps ? s_rc[tid] : 0;
+      int tot;
+      const int ex = scan_cta(a0, s_w, &s_total, &tot);
+      if (tid < R * kMergeWarps) s_rc[tid] = ex;
+      __syncthreads();
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+        if ((bal[r] >> lane) & 1u)
+          fn(r * kMergeThreads + tid, s_rc[r * kMergeWarps + warp] + __popc(bal[r] & lt), id[r]);
+    } else {
+      int carry = 0;
 #pragma unroll 1
-  while (shift > 0) {
-    const int w = min(11, shift);
-    const int hi = shift;
-    shift -= w;
-    const uint32_t bmask = (1u << w) - 1u;
-    for (int i = tid; i < kBins; i += kMergeThreads) s_hist[i] = 0;
-    __syncthreads();
-    each([&](int i, const uint2* e) {
-      const uint32_t rel = key_at(i, e) - umin;
-      const uint32_t top = hi >= 32 ? 0u : rel >> hi;
-      if (top == pfx) atomicAdd(&s_hist[(rel >> shift) & bmask], 1);
-    });
-    __syncthreads();
-    // thread t owns bins 2047 - 2t and 2046 - 2t (descending)
-    const int h0 = s_hist[kBins - 1 - 2 * tid], h1 = s_hist[kBins - 2 - 2 * tid];
-    int tot;
-    const int ex = scan_cta(h0 + h1, s_w, &s_total, &tot);
-    if (ex < rem && ex + h0 + h1 >= rem) {
-      const bool upper = ex + h0 >= rem;
-      s_pick[0] = upper ? kBins - 1 - 2 * tid : kBins - 2 - 2 * tid;
-      s_pick[1] = upper ? rem - ex : rem - ex - h0;
+      for (int j0 = 0; j0 < J; j0 += kScanRounds) {
+        const int jn = min(kScanRounds, J - j0);
+#pragma unroll 4
+        for (int j = 0; j < jn; ++j) {
+          const int slot = (j0 + j) * kMergeThreads + tid;
+          uint32_t kk = 0;
+          const bool pr = load(slot, kk) && pred(slot, kk);
+          const uint32_t bal = __ballot_sync(0xffffffffu, pr);
+          if (lane == 0) s_rc[j * kMergeWarps + warp] = __popc(bal);
+        }
+        __syncthreads();
+        int av[kScanPer], sum = 0;
+#pragma unroll
+        for (int i = 0; i < kScanPer; ++i) {
+          const int e = kScanPer * tid + i;
+          av[i] = e < jn * kMergeWarps ? s_rc[e] : 0;
+          sum += av[i];
+        }
+        int tot;
+        int ex = scan_cta(sum, s_w, &s_total, &tot) + carry;
+#pragma unroll
+        for (int i = 0; i < kScanPer; ++i) {
+          const int e = kScanPer * tid + i;
+          if (e < jn * kMergeWarps) s_rc[e] = ex;
+          ex += av[i];
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int j1 = 0; j1 < jn; j1 += kBatch) {
+          int slots[kBatch], ranks[kBatch], ids[kBatch];
+          bool picked[kBatch];
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u) {
+            const int j = j1 + u;
+            slots[u] = (j0 + j) * kMergeThreads + tid;
+            uint32_t kk = 0;
+            picked[u] = j < jn && load(slots[u], kk) && pred(slots[u], kk);
+            const uint32_t bal = __ballot_sync(0xffffffffu, picked[u]);
+            ranks[u] = j < jn ? s_rc[j * kMergeWarps + warp] + __popc(bal & lt) : 0;
+          }
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u)
+            ids[u] = picked[u] ? (cache == 2 ? is[slots[u]] : static_cast<int>(__ldg(&cq[slots[u]].y))) : -1;
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u)
+            if (picked[u]) fn(slots[u], ranks[u], ids[u]);
+        }
+        carry += tot;
+        __syncthreads();
+      }
     }
-    __syncthreads();
-    pfx = (pfx << w) | static_cast<uint32_t>(s_pick[0]);
-    rem = s_pick[1];
-  }
-  const uint32_t T = umin + pfx;
-  // keys equal to T, ranked by position; then the selection's output positions
-  int n_eq = 0;
-  each([&](int i, const uint2* e) { n_eq += !take_all && key_at(i, e) == T; });
-  int tot;
-  int eq_rank = scan_cta(n_eq, s_w, &s_total, &tot);
-  int n_sel = 0;
-  {
-    int r = eq_rank;
-    each([&](int i, const uint2* e) {
-      const uint32_t key = key_at(i, e);
-      const bool eq = !take_all && key == T;
-      n_sel += take_all || key > T || (eq && r < rem);
-      r += eq;
-    });
-  }
-  int pos = scan_cta(n_sel, s_w, &s_total, &tot);
-  each([&](int i, const uint2* e) {
-    const uint32_t key = key_at(i, e);
-    const bool eq = !take_all && key == T;
-    if (take_all || key > T || (eq && eq_rank < rem)) {
-      if (pos < K) out[pos] = static_cast<int32_t>(__ldg(&e->y));
-      ++pos;
+  };
+  if (n <= K) {
+    // every candidate is taken
+    if (tid == 0) {
+      s_tk = 0u;
+      s_ts = 0x7fffffff;
     }
-    eq_rank += eq;
-  });
+  } else {
+    // radix passes inside the bin (pfx over the bits above `shift`) that holds the K-th
+    // largest key; rem = keys still to take inside it, in_bin = keys it holds
+    uint32_t pfx = 0;
+    int rem = K, in_bin = n;
+    int shift = 32 - __clz(static_cast<int>(umax - umin));
+    bool zeroed = true;  // the histogram was cleared before the first barrier
+#pragma unroll 1
+    while (in_bin > kSmallBin && shift > 0) {
+      const int w = min(11, shift);
+      const int hi = shift;
+      shift -= w;
+      const uint32_t bmask = (1u << w) - 1u;
+      if (!zeroed) {
+        for (int i = tid; i < kBins; i += kMergeThreads) s_hist[i] = 0;
+        __syncthreads();
+      }
+      zeroed = false;
+      each([&](int, uint32_t kk) {
+        const uint32_t rel = kk - umin;
+        if ((hi >= 32 ? 0u : rel >> hi) == pfx) atomicAdd(&s_hist[(rel >> shift) & bmask], 1);
+      });
+      __syncthreads();
+      // thread t owns bins 2047 - 2t and 2046 - 2t (descending)
+      const int h0 = s_hist[kBins - 1 - 2 * tid], h1 = s_hist[kBins - 2 - 2 * tid];
+      int tot;
+      const int ex = scan_cta(h0 + h1, s_w, &s_total, &tot);
+      if (ex < rem && ex + h0 + h1 >= rem) {
+        const bool upper = ex + h0 >= rem;
+        s_pick[0] = upper ? kBins - 1 - 2 * tid : kBins - 2 - 2 * tid;
+        s_pick[1] = upper ? rem - ex : rem - ex - h0;
+        s_pick[2] = upper ? h0 : h1;
+      }
+      __syncthreads();
+      pfx = (pfx << w) | static_cast<uint32_t>(s_pick[0]);
+      rem = s_pick[1];
+      in_bin = s_pick[2];
+    }
+    if (in_bin <= kSmallBin) {
+      // rank the bin's keys exactly: (key descending, slot ascending)
+      each([&](int slot, uint32_t kk) {
+        if (shift >= 32 || ((kk - umin) >> shift) == pfx) {
+          const int i = atomicAdd(&s_lcnt, 1);
+          if (i < kSmallBin) {  // exactly in_bin keys arrive here
+            s_lkey[i] = kk;
+            s_lslot[i] = slot;
+          }
+        }
+      });
+      __syncthreads();
+      if (tid < in_bin) {
+        const uint32_t ki = s_lkey[tid];
+        const int si = s_lslot[tid];
+        int r = 0;
+        for (int i = 0; i < in_bin; ++i) {
+          const uint32_t kj = s_lkey[i];
+          r += kj > ki || (kj == ki && s_lslot[i] < si);
+        }
+        if (r == rem - 1) {
+          s_tk = ki;
+          s_ts = si;
+        }
+      }
+    } else {
+      // more than kSmallBin keys equal to Tk: the rem-th of them in slot order
+      const uint32_t T = umin + pfx;
+      if (tid == 0) s_tk = T;
+      ordered([&](int, uint32_t kk) { return kk == T; },
+              [&](int slot, int r, int) {
+                if (r == rem - 1) s_ts = slot;
+              });
+    }
+  }
+  __syncthreads();
+  const uint32_t Tk = s_tk;
+  const int Ts = s_ts;
+  ordered([&](int slot, uint32_t kk) { return kk > Tk || (kk == Tk && slot <= Ts); },
+          [&](int, int r, int e) {
+            if (r < K) out[r] = e;
+          });
 }
 
 cudaError_t launch_topk_merge(const lc_index_topk_args& a, int n_chunks, const uint2* cand, const int* cand_cnt,
                               bool decode, cudaStream_t st) {
   if (n_chunks > kMergeMaxChunks) return cudaErrorInvalidConfiguration;
   const int64_t n_max = static_cast<int64_t>(n_chunks) * a.k;
-  const int cached = n_max <= kMergeCache ? 1 : 0;
-  const size_t sm = cached ? static_cast<size_t>(n_max) * 4 : 0;
-  cudaFuncSetAttribute(k_topk_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, kMergeCache * 4);
-  return launch_ex(k_topk_merge, dim3(a.index.n_q), dim3(kMergeThreads), sm, st, true, 1, a.k, a.index.m, a.index.W_x,
-                   a.index.batch, cand, cand_cnt, n_chunks, a.idx, a.count, decode ? 1 : 0, cached);
+  if (n_max <= static_cast<int64_t>(kMergeRegRounds) * kMergeThreads)
+    return launch_ex(k_topk_merge<kMergeRegRounds>, dim3(a.index.n_q), dim3(kMergeThreads), 0, st, true, 1, a.k,
+                     a.index.m, a.index.W_x, a.index.batch, cand, cand_cnt, n_chunks, a.idx, a.count,
+                     decode ? 1 : 0, 0);
+  const int cache = n_max <= kMergeCacheKI ? 2 : n_max <= kMergeCacheK ? 1 : 0;
+  const size_t words = static_cast<size_t>((n_max + 31) / 32);
+  const size_t sm = cache == 2 ? static_cast<size_t>(n_max) * 8 + words * 4
+                  : cache == 1 ? static_cast<size_t>(n_max) * 4 + words * 4 : 0;
+  cudaFuncSetAttribute(k_topk_merge<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       kMergeCacheK * 4 + kMergeCacheK / 8);
+  return launch_ex(k_topk_merge<0>, dim3(a.index.n_q), dim3(kMergeThreads), sm, st, true, 1, a.k, a.index.m,
+                   a.index.W_x, a.index.batch, cand, cand_cnt, n_chunks, a.idx, a.count, decode ? 1 : 0, cache);
 }
 
 __global__ void k_empty_selection(int32_t* idx, int32_t* count, int n_q, int k) {
