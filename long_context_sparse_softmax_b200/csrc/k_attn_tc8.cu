@@ -155,6 +155,9 @@ struct AttnTc8Geom {
 };
 
 constexpr int kMaxClusterSplits = 8;
+// the receive buffers of the cluster merge (n_split x kNR x ceil(groups / n_split) x 32 floats)
+// fit below the key codes, in the dead tiles
+static_assert((kD / 32 + kMaxClusterSplits - 1) * kNR * 32 * 4 <= kOffCode, "merge buffers fit");
 
 // grid: one CTA per (query, head group, key split), the split index fastest; 320 threads.
 // Partial results of split s go to ws_o rows s * n_q * H + q * H + h (576 floats each) and
@@ -177,7 +180,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ __align__(8) Bars bars;
-  __shared__ float2 s_ml[kNR];  // cluster merge: this split's (max, sum) per head
+  __shared__ float2 s_mlall[kMaxClusterSplits][kNR];  // cluster merge: every split's (max, sum) per head
+  __shared__ float s_sk[kNR];  // the heads' sinks, log2 units
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_hg = a.dims.H / kNR;
@@ -306,6 +310,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   fence_after();
   const uint32_t tm = s_tmem;
+  // cluster: this CTA has started (its shared memory may be written remotely once every
+  // CTA of the cluster has arrived here)
+  if (geo.cluster) asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
 
   if (warp >= 9) {
     // ================= key codes and bulk copies =================
@@ -590,6 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hf = lane >> 4;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const float sl2 = a.scale * 1.4426950408889634f;
+    if (hf == 0) s_sk[r] = __ldg(a.sink + hg * kNR + r) * 1.4426950408889634f;  // read by this thread
     float m_ref = -INFINITY, l_sum = 0.f;
     bool good = true;
     for (int t = 0; t < n_tiles; ++t) {
@@ -676,11 +684,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float l_row = l_sum + __shfl_xor_sync(0xffffffffu, l_sum, 16);
     if (geo.cluster) {
       // this split's (max, sum) per head, for the merge over the cluster below
-      if (hf == 0) s_ml[r] = make_float2(good ? m_ref : -INFINITY, good ? l_row : 0.f);
+      if (hf == 0) s_mlall[split][r] = make_float2(good ? m_ref : -INFINITY, good ? l_row : 0.f);
     } else if (hf == 0) {
-      const int h = hg * kNR + r;
       if (geo.n_split == 1) {
-        const float sk = __ldg(a.sink + h) * 1.4426950408889634f;
+        const float sk = s_sk[r];
         const float M = fmaxf(sk, m_ref);
         const float w = m_ref == -INFINITY ? 0.f : exp2f(m_ref - M);
         const float Z = exp2f(sk - M) + l_row * w;
@@ -728,26 +735,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (geo.cluster) {
     // ================= merge of the key splits over the cluster (every thread) =================
-    // M = max(sink, max_s m_s), Z = e^(sink - M) + sum_s l_s e^(m_s - M) per head; split s
-    // scales its O by e^(m_s - M) / Z into its own shared memory; then split s sums dims
-    // [d0, d1) of every split's scaled O, in split order, and writes them out.
+    // Every transfer is a store into another CTA's shared memory (a remote load would wait
+    // a round trip).  Split s pushes its (m, l) per head to every split; then each split
+    // finds M = max(sink, max_s m_s), Z = e^(sink - M) + sum_s l_s e^(m_s - M) locally,
+    // scales its O by e^(m_s - M) / Z and pushes each 32-dim group of it to the split that
+    // owns the group (split j owns groups [j gp, (j + 1) gp)), which sums the n_split
+    // pieces in split order and writes them out.
     cg::cluster_group cl = cg::this_cluster();
     fence_before();
-    cl.sync();  // every split's (m, l) is published; every role of every split is done
+    __syncthreads();  // this CTA's roles are done: s_mlall[split] is written
+    asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory");  // every CTA has started
+    if (tid < kNR)
+      for (int sp = 0; sp < geo.n_split; ++sp)
+        if (sp != split) cl.map_shared_rank(&s_mlall[split][0], sp)[tid] = s_mlall[split][tid];
+    cl.sync();  // every split's (m, l) is here; every role of every split is done
     fence_after();
-    float* Osm = reinterpret_cast<float*>(smem + kOffRaw);  // [kNR heads][kD dims]
+    const int ngr = Dv / 32;
+    const int gp = (ngr + geo.n_split - 1) / geo.n_split;
+    const int ndj = gp * 32;                       // row length of the receive buffers
+    float* recv = reinterpret_cast<float*>(smem);  // [n_split sources][kNR heads][ndj dims]
     if (warp < 4) {
       const int r = warp * 16 + (lane & 15);
       if ((lane >> 4) == 0) {
-        const float sk = __ldg(a.sink + hg * kNR + r) * 1.4426950408889634f;
+        const float sk = s_sk[r];
         float M = sk;
-        for (int sp = 0; sp < geo.n_split; ++sp) M = fmaxf(M, cl.map_shared_rank(s_ml, sp)[r].x);
+        for (int sp = 0; sp < geo.n_split; ++sp) M = fmaxf(M, s_mlall[sp][r].x);
         float Z = exp2f(sk - M);
         for (int sp = 0; sp < geo.n_split; ++sp) {
-          const float2 v = cl.map_shared_rank(s_ml, sp)[r];
+          const float2 v = s_mlall[sp][r];
           if (v.x != -INFINITY) Z = fmaf(v.y, exp2f(v.x - M), Z);
         }
-        const float mo = s_ml[r].x;
+        const float mo = s_mlall[split][r].x;
         s_f[r] = mo == -INFINITY ? 0.f : exp2f(mo - M) / Z;
         if (split == 0 && a.lse) a.lse[row0 + r] = (M + log2f(Z)) * 0.6931471805599453f;
       }
@@ -772,61 +790,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i) ov[i] = 0;
           }
           if (dim < 0) continue;
+          const int j = (dim >> 5) / gp;
+          float* dst = cl.map_shared_rank(recv, j) + (split * kNR + hh) * ndj + (dim - j * ndj);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) Osm[(hh + i) * kD + dim] = __uint_as_float(ov[i]) * f[i];
+          for (int i = 0; i < 32; ++i) dst[i * ndj] = __uint_as_float(ov[i]) * f[i];
         }
       }
     }
-    cl.sync();  // every split's scaled O is in its shared memory
-    const int dpc = ((Dv + geo.n_split - 1) / geo.n_split + 3) & ~3;
-    const int d0 = min(Dv, split * dpc), d1 = min(Dv, d0 + dpc);
+    cl.sync();  // every split's pieces are in their owners' shared memory
+    // this split's dims [d0, d1): the sum over the sources, in split order
+    const int d0 = min(Dv, split * ndj), d1 = min(Dv, d0 + ndj);
     const int nq4 = (d1 - d0) / 4;
-    const float* src[kMaxClusterSplits];
-#pragma unroll
-    for (int sp = 0; sp < kMaxClusterSplits; ++sp) src[sp] = sp < geo.n_split ? cl.map_shared_rank(Osm, sp) : Osm;
-    // kMergeIt outputs per thread at a time, each split's loads for all of them issued
-    // before they are added: the remote loads overlap instead of queueing one by one
-    constexpr int kMergeIt = 6;
-    for (int base = 0; base < kNR * nq4; base += kMergeIt * kThreads) {
-      float4 acc[kMergeIt];
-      int off[kMergeIt];
-#pragma unroll
-      for (int j = 0; j < kMergeIt; ++j) {
-        acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-        const int it = base + j * kThreads + tid;
-        off[j] = it < kNR * nq4 ? (it / nq4) * kD + d0 + 4 * (it % nq4) : -1;
+    for (int it = tid; it < kNR * nq4; it += kThreads) {
+      const int h = it / nq4, d4 = 4 * (it - h * nq4);
+      float4 acc = *reinterpret_cast<const float4*>(recv + h * ndj + d4);
+      for (int sp = 1; sp < geo.n_split; ++sp) {
+        const float4 v = *reinterpret_cast<const float4*>(recv + (sp * kNR + h) * ndj + d4);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
       }
-#pragma unroll
-      for (int sp = 0; sp < kMaxClusterSplits; ++sp) {
-        if (sp >= geo.n_split) break;
-        float4 v[kMergeIt];
-#pragma unroll
-        for (int j = 0; j < kMergeIt; ++j)
-          v[j] = off[j] >= 0 ? *reinterpret_cast<const float4*>(src[sp] + off[j]) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int j = 0; j < kMergeIt; ++j) {
-          acc[j].x += v[j].x;
-          acc[j].y += v[j].y;
-          acc[j].z += v[j].z;
-          acc[j].w += v[j].w;
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < kMergeIt; ++j) {
-        if (off[j] < 0) continue;
-        const int h = off[j] / kD, d = off[j] % kD;
-        const float4 o = acc[j];
-        const int64_t e = (row0 + h) * Dv + d;
-        if (a.out_fmt == LC_FMT_F32) {
-          *reinterpret_cast<float4*>(static_cast<float*>(a.out) + e) = o;
-        } else {
-          const uint32_t lo = static_cast<uint32_t>(f32_to_bf16_bits(o.x)) | (static_cast<uint32_t>(f32_to_bf16_bits(o.y)) << 16);
-          const uint32_t hi = static_cast<uint32_t>(f32_to_bf16_bits(o.z)) | (static_cast<uint32_t>(f32_to_bf16_bits(o.w)) << 16);
-          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + e) = make_uint2(lo, hi);
-        }
+      const int64_t e = (row0 + h) * Dv + d0 + d4;
+      if (a.out_fmt == LC_FMT_F32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(a.out) + e) = acc;
+      } else {
+        const uint32_t lo = static_cast<uint32_t>(f32_to_bf16_bits(acc.x)) | (static_cast<uint32_t>(f32_to_bf16_bits(acc.y)) << 16);
+        const uint32_t hi = static_cast<uint32_t>(f32_to_bf16_bits(acc.z)) | (static_cast<uint32_t>(f32_to_bf16_bits(acc.w)) << 16);
+        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + e) = make_uint2(lo, hi);
       }
     }
-    cl.sync();  // no split leaves while another still reads its shared memory
   }
   fence_before();
   __syncthreads();

@@ -538,20 +538,33 @@ __global__ void __launch_bounds__(kMergeThreads) k_topk_merge(int k, int m, int 
     s_n = 0;
     s_lcnt = 0;
   }
-  pdl_wait();  // the indexer's candidates (launched right after it, programmatically)
+  // the query's visible entries: step inputs that the indexer does not write
   const int b = decode ? q : seq_of_query(batch.q_start, batch.num_seqs, q);
   const int p = __ldg(batch.q_pos0 + b) + (decode ? 0 : q - __ldg(batch.q_start + b));
   const int nv = n_visible(p, m, W_x, __ldg(batch.n_ent + b));
   const int K = min(k, nv);
   int32_t* out = idx + static_cast<int64_t>(q) * k;
-  for (int i = K + tid; i < k; i += kMergeThreads) out[i] = -1;
-  if (tid == 0 && count) count[q] = K;
-  if (K == 0) return;
   const int n_slots = n_chunks * k;
   const int J = (n_slots + kMergeThreads - 1) / kMergeThreads;  // rounds of slots
   const uint2* cq = cand + static_cast<int64_t>(q) * n_slots;
   const int* cc = cand_cnt + static_cast<int64_t>(q) * n_chunks;
   const uint32_t lt = (1u << lane) - 1u;
+  pdl_wait();  // the indexer's candidates (launched right after it, programmatically)
+  // R > 0: every candidate load at once (a slot past its range's count is read and dropped)
+  uint2 e0[R > 0 ? R : 1];
+  int cn0[R > 0 ? R : 1];
+  if constexpr (R > 0) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int slot = r * kMergeThreads + tid;
+      const bool in = K > 0 && slot < n_slots;
+      cn0[r] = in ? __ldg(cc + slot / k) : 0;
+      e0[r] = in ? __ldg(&cq[slot]) : make_uint2(0u, 0u);
+    }
+  }
+  for (int i = K + tid; i < k; i += kMergeThreads) out[i] = -1;
+  if (tid == 0 && count) count[q] = K;
+  if (K == 0) return;
   // a range writes at most k candidates (the clamp only matters after a timeout upstream)
   auto held_g = [&](int slot) {
     const int c = slot / k;
@@ -579,26 +592,19 @@ __global__ void __launch_bounds__(kMergeThreads) k_topk_merge(int k, int m, int 
   uint32_t kmin = 0xffffffffu, kmax = 0u;
   int nmine = 0;
   if constexpr (R > 0) {
-    bool v[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int slot = r * kMergeThreads + tid;
-      v[r] = slot < n_slots && held_g(slot);
-    }
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const uint2 e = v[r] ? __ldg(&cq[r * kMergeThreads + tid]) : make_uint2(0u, 0u);
-      key[r] = e.x;
-      id[r] = static_cast<int>(e.y);
-    }
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-      if (v[r]) {
+      const bool v = slot < n_slots && slot % k < min(max(cn0[r], 0), k);
+      key[r] = e0[r].x;
+      id[r] = static_cast<int>(e0[r].y);
+      if (v) {
         vm |= 1u << r;
         kmin = min(kmin, key[r]);
         kmax = max(kmax, key[r]);
         ++nmine;
       }
+    }
   } else {
     for (int c = tid; c < n_chunks; c += kMergeThreads) s_cnt[c] = min(max(__ldg(cc + c), 0), k);
 #pragma unroll 1
