@@ -117,7 +117,7 @@ struct IdxSelect {
 // Tensor memory: accumulators at columns [k N, (k + 1) N), k < 3; key scales at 3N + {0, 8};
 // query scales at 3N + 16 (N / 32 columns).
 template <int QPC, bool SELECT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     k_index_tc(const __grid_constant__ CUtensorMap tk, lc_index_args a, int tiles_per_cta, uint32_t tmem_cols,
                int decode, IdxSelect sel) {
   static_assert(!SELECT || QPC == 1, "fused selection takes one query per CTA");
@@ -363,6 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // head weights in registers when one query's heads fill the accumulator (H <= 64);
     // the other epilogue warps wrote part of them: wait for all 128 arrivals first
     const bool weights_ok = __all_sync(0xffffffffu, wait(&bars.bfull, 0));
+    // SELECT: the range of this thread's valid order keys, kept while the scores come in
+    uint32_t sel_kmin = 0xffffffffu, sel_kmax = 0u;
     float wr[64];
     if (QPC == 1) {
 #pragma unroll
@@ -392,7 +394,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         const float s = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-        if constexpr (SELECT) sc[u * kKeys + row] = s;
+        if constexpr (SELECT) {
+          // the order key in place of the score; the selection below reads only keys
+          const uint32_t kk = order_key(s);
+          reinterpret_cast<uint32_t*>(sc)[u * kKeys + row] = kk;
+          if (j < s_nv[0]) {
+            sel_kmin = min(sel_kmin, kk);
+            sel_kmax = max(sel_kmax, kk);
+          }
+        }
         else if (j < s_nv[i]) a.scores[static_cast<int64_t>(s_q[i]) * a.score_stride + j] = s;
       }
       fence_before();
@@ -407,9 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // scratch in the idle key ring (dynamic shared memory, so that the static part stays
       // small enough for two CTAs per SM)
       uint32_t* hist4 = reinterpret_cast<uint32_t*>(As);  // [4][kSelBins] per-warp histograms
-      uint32_t* bits = hist4 + 4 * kSelBins;              // [kSelMaxTiles * 4] selection words
-      int (*s_wcnt)[4] = reinterpret_cast<int (*)[4]>(bits + kSelMaxTiles * 4);   // [kSelMaxTiles][4]
-      uint32_t* list_key = reinterpret_cast<uint32_t*>(s_wcnt + kSelMaxTiles);     // [kSmallBin]
+      int* s_pre = reinterpret_cast<int*>(hist4 + 4 * kSelBins);                   // [kSelMaxTiles * 4]
+      uint32_t* list_key = reinterpret_cast<uint32_t*>(s_pre + kSelMaxTiles * 4);  // [kSmallBin]
       int* list_off = reinterpret_cast<int*>(list_key + kSmallBin);                // [kSmallBin]
       uint32_t (*s_rng)[4] = reinterpret_cast<uint32_t (*)[4]>(list_off + kSmallBin);  // [2][4]
       int* s_tmp = reinterpret_cast<int*>(s_rng + 2);     // [4]
@@ -420,15 +429,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int jbase = t_begin * kKeys;
       const int n_valid = max(0, min(s_nv[0] - jbase, n_tiles * kKeys));
       const int K = min(sel.k, n_valid);
-      auto valid = [&](int u) { return u * kKeys + row < n_valid; };
-      // key range of the valid scores
-      uint32_t kmin = 0xffffffffu, kmax = 0u;
-      for (int u = 0; u < n_tiles; ++u)
-        if (valid(u)) {
-          const uint32_t key = order_key(sc[u * kKeys + row]);
-          kmin = min(kmin, key);
-          kmax = max(kmax, key);
-        }
+      // the valid offsets are a prefix of the range: this thread's are u * 128 + row, u < nu
+      const int nu = n_valid > row ? (n_valid - row + kKeys - 1) / kKeys : 0;
+      // the order keys (written in place of the scores by the epilogue).  The loops below
+      // stay short: this code runs once per launch, and a taken branch into code not yet
+      // fetched stalls on the instruction fetch, so loops unrolled with guarded bodies cost
+      // far more here than they save
+      const uint32_t* key_s = reinterpret_cast<const uint32_t*>(sc);
+      auto key = [&](int u) { return key_s[u * kKeys + row]; };
+      uint32_t kmin = sel_kmin, kmax = sel_kmax;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
@@ -443,6 +452,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         s_thr[0] = 0u;           // every valid key is taken unless a threshold is found
         s_thr[1] = 0x7fffffffu;
       }
+      if (K < n_valid) {
+        uint4* h4 = reinterpret_cast<uint4*>(hist4);
+        for (int i = row; i < kSelBins; i += 128) h4[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
       named_bar(1, 128);
       const uint32_t umin = min(min(s_rng[0][0], s_rng[0][1]), min(s_rng[0][2], s_rng[0][3]));
       const uint32_t umax = max(max(s_rng[1][0], s_rng[1][1]), max(s_rng[1][2], s_rng[1][3]));
@@ -456,28 +469,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pfx = 0;
         int rem = K, in_bin = n_valid;
         int shift = 32 - __clz(static_cast<int>(umax - umin));
+        bool zeroed = true;
 #pragma unroll 1
         while (in_bin > kSmallBin && shift > 0) {
           const int w = min(11, shift);
           const int hi = shift;
           shift -= w;
           const uint32_t bmask = (1u << w) - 1u;
-          for (int i = row; i < 4 * kSelBins; i += 128) hist4[i] = 0;
-          named_bar(1, 128);
-          for (int u = 0; u < n_tiles; ++u)
-            if (valid(u)) {
-              const uint32_t rel = order_key(sc[u * kKeys + row]) - umin;
+          if (!zeroed) {
+            uint4* h4 = reinterpret_cast<uint4*>(hist4);
+            for (int i = row; i < kSelBins; i += 128) h4[i] = make_uint4(0u, 0u, 0u, 0u);
+            named_bar(1, 128);
+          }
+          zeroed = false;
+#pragma unroll 4
+          for (int u = 0; u < nu; ++u) {
+              const uint32_t rel = key(u) - umin;
               if ((hi >= 32 ? 0u : rel >> hi) == pfx) atomicAdd(&hist4[quad * kSelBins + ((rel >> shift) & bmask)], 1u);
             }
           named_bar(1, 128);
           // descending: thread `row` owns bins 2047 - 16 row - i, i < 16
           int c[16], sum = 0;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int bin = kSelBins - 1 - 16 * row - i;
-            c[i] = static_cast<int>(hist4[bin] + hist4[kSelBins + bin] + hist4[2 * kSelBins + bin] +
-                                    hist4[3 * kSelBins + bin]);
-            sum += c[i];
+          for (int i4 = 0; i4 < 4; ++i4) {
+            const int b0 = kSelBins - 16 * row - 4 * i4 - 4;  // bins b0 .. b0 + 3
+            uint4 t = reinterpret_cast<const uint4*>(hist4)[b0 / 4];
+#pragma unroll
+            for (int w4 = 1; w4 < 4; ++w4) {
+              const uint4 x = reinterpret_cast<const uint4*>(hist4 + w4 * kSelBins)[b0 / 4];
+              t.x += x.x;
+              t.y += x.y;
+              t.z += x.z;
+              t.w += x.w;
+            }
+            c[4 * i4] = static_cast<int>(t.w);
+            c[4 * i4 + 1] = static_cast<int>(t.z);
+            c[4 * i4 + 2] = static_cast<int>(t.y);
+            c[4 * i4 + 3] = static_cast<int>(t.x);
+            sum += c[4 * i4] + c[4 * i4 + 1] + c[4 * i4 + 2] + c[4 * i4 + 3];
           }
           int tot;
           int run = scan128(sum, quad, lane, s_tmp, &tot);
@@ -498,15 +527,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           in_bin = s_pick[2];
         }
         if (in_bin <= kSmallBin) {
-          for (int u = 0; u < n_tiles; ++u)
-            if (valid(u)) {
-              const uint32_t key = order_key(sc[u * kKeys + row]);
-              if (shift >= 32 || ((key - umin) >> shift) == pfx) {
-                const int i = atomicAdd(s_cnt, 1);
-                if (i < kSmallBin) {  // exactly in_bin keys arrive here
-                  list_key[i] = key;
-                  list_off[i] = u * kKeys + row;
-                }
+#pragma unroll 4
+          for (int u = 0; u < nu; ++u)
+            if (shift >= 32 || ((key(u) - umin) >> shift) == pfx) {
+              const int i = atomicAdd(s_cnt, 1);
+              if (i < kSmallBin) {  // exactly in_bin keys arrive here
+                list_key[i] = key(u);
+                list_off[i] = u * kKeys + row;
               }
             }
           named_bar(1, 128);
@@ -526,60 +553,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           // every key of the bin equals T: the rem-th of them in offset order (tile, then row)
           const uint32_t T = umin + pfx;
+#pragma unroll 1
           for (int u = 0; u < n_tiles; ++u) {
-            const bool eq = valid(u) && order_key(sc[u * kKeys + row]) == T;
-            const uint32_t bal = __ballot_sync(0xffffffffu, eq);
-            if (lane == 0) s_wcnt[u][quad] = __popc(bal);
-          }
+              const uint32_t bal = __ballot_sync(0xffffffffu, u < nu && key(u) == T);
+              if (lane == 0) s_pre[u * 4 + quad] = __popc(bal);
+            }
           named_bar(1, 128);
           int eq_before = 0;
+#pragma unroll 1
           for (int u = 0; u < n_tiles; ++u) {
-            const bool eq = valid(u) && order_key(sc[u * kKeys + row]) == T;
-            int rank = eq_before + __popc(__ballot_sync(0xffffffffu, eq) & ((1u << lane) - 1u));
+              const bool eq = u < nu && key(u) == T;
+              int rank = eq_before + __popc(__ballot_sync(0xffffffffu, eq) & ((1u << lane) - 1u));
 #pragma unroll
-            for (int w = 0; w < 4; ++w) rank += w < quad ? s_wcnt[u][w] : 0;
-            if (eq && rank == rem - 1) {
-              s_thr[0] = T;
-              s_thr[1] = static_cast<uint32_t>(u * kKeys + row);
+              for (int w = 0; w < 4; ++w) rank += w < quad ? s_pre[u * 4 + w] : 0;
+              if (eq && rank == rem - 1) {
+                s_thr[0] = T;
+                s_thr[1] = static_cast<uint32_t>(u * kKeys + row);
+              }
+              eq_before += s_pre[u * 4] + s_pre[u * 4 + 1] + s_pre[u * 4 + 2] + s_pre[u * 4 + 3];
             }
-            eq_before += s_wcnt[u][0] + s_wcnt[u][1] + s_wcnt[u][2] + s_wcnt[u][3];
-          }
+          named_bar(1, 128);  // s_pre is reused below
         }
         named_bar(1, 128);
       }
       const uint32_t Tk = s_thr[0];
       const int Ts = static_cast<int>(s_thr[1]);
+      // output positions in offset order: the selected keys of each (tile, warp), then a
+      // scan over the (tile, warp) counts in that order
+      uint64_t picks = 0;  // bit u: this thread's key of tile u is selected
+#pragma unroll 4
       for (int u = 0; u < n_tiles; ++u) {
-        const int off = u * kKeys + row;
-        const uint32_t key = valid(u) ? order_key(sc[off]) : 0u;
-        const bool pick = valid(u) && (key > Tk || (key == Tk && off <= Ts));
-        const uint32_t word = __ballot_sync(0xffffffffu, pick);
-        if (lane == 0) bits[u * 4 + quad] = word;
+          const int off = u * kKeys + row;
+          const bool pick = u < nu && (key(u) > Tk || (key(u) == Tk && off <= Ts));
+          picks |= static_cast<uint64_t>(pick) << u;
+          const uint32_t bal = __ballot_sync(0xffffffffu, pick);
+          if (lane == 0) s_pre[u * 4 + quad] = __popc(bal);
+        }
+      named_bar(1, 128);
+      {
+        const int ne = n_tiles * 4;  // <= 256: two entries per thread
+        const int e0 = 2 * row;
+        const int v0 = e0 < ne ? s_pre[e0] : 0, v1 = e0 + 1 < ne ? s_pre[e0 + 1] : 0;
+        int tot;
+        const int ex = scan128(v0 + v1, quad, lane, s_tmp, &tot);
+        if (e0 < ne) s_pre[e0] = ex;
+        if (e0 + 1 < ne) s_pre[e0 + 1] = ex + v0;
       }
       named_bar(1, 128);
-      // the selected keys in index order: word w holds keys jbase + 32 w .. + 31
-      const int n_words = n_tiles * 4;
       const bool alone = sel.n_chunks == 1;
       int32_t* out_idx = alone ? sel.idx + static_cast<int64_t>(q) * sel.k : nullptr;
       uint2* out_c = alone ? nullptr : sel.cand + (static_cast<int64_t>(q) * sel.n_chunks + blockIdx.y) * sel.k;
-      int base = 0;
-      for (int w0 = 0; w0 < n_words; w0 += 128) {
-        const int w = w0 + row;
-        uint32_t word = w < n_words ? bits[w] : 0u;
-        int tot;
-        int pos = base + scan128(__popc(word), quad, lane, s_tmp, &tot);
-        while (word) {
-          const int bpos = __ffs(word) - 1;
-          word &= word - 1;
-          const int off = w * 32 + bpos;  // key u * 128 + row' of the range
-          if (pos < K) {  // exactly K bits are set; the guard only matters after a timeout
+      const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll 4
+      for (int u = 0; u < n_tiles; ++u) {
+          const bool pick = (picks >> u) & 1u;
+          const uint32_t bal = __ballot_sync(0xffffffffu, pick);
+          const int pos = s_pre[u * 4 + quad] + __popc(bal & lt);
+          if (pick && pos < K) {  // exactly K keys are picked; the guard only matters after a timeout
+            const int off = u * kKeys + row;
             if (alone) out_idx[pos] = jbase + off;
-            else out_c[pos] = make_uint2(order_key(sc[off]), static_cast<uint32_t>(jbase + off));
+            else out_c[pos] = make_uint2(key(u), static_cast<uint32_t>(jbase + off));
           }
-          ++pos;
         }
-        base += tot;
-      }
       if (alone) {
         for (int i = K + row; i < sel.k; i += 128) out_idx[i] = -1;
         if (row == 0 && sel.count) sel.count[q] = K;
