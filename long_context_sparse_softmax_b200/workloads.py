@@ -65,6 +65,7 @@ class Spec:
     ring: bool = True        # decode: each sequence's window rows are a ring of W rows
     w_per_query: bool = False  # indexer head weights per query [n_q, H_I] instead of shared [H_I]
     v_nope: bool = False     # values are the non-RoPE dims of the entries (outputs D - d_r dims)
+    out32: bool = False      # FP32 attention outputs with the narrow input formats
 
     @property
     def d_n(self) -> int:
@@ -103,7 +104,7 @@ class Spec:
 
     @property
     def out_f32(self) -> bool:
-        return self.fp32
+        return self.fp32 or self.out32
 
     @property
     def num_seqs(self) -> int:

@@ -132,3 +132,30 @@ def test_nope_values_prefill_kernels():
     check_prefill(wl.shrink(wl.HCA_PREFILL, name="vnope_hca_prefill", seed=50, seq_lens=(128 * 24 + 50,),
                             q_first=128 * 24 + 50 - 160, n_q=160, v_nope=True))
     check_prefill(wl.shrink(wl.TINY_CSA_PREFILL, name="vnope_tiny", seed=51, seq_lens=(400,), n_q=400, v_nope=True))
+
+
+def test_csa_decode_f32_output_cluster_merge():
+    """FP32 outputs of the decode path whose key splits merge over a thread-block cluster
+    (few queries, so each query's keys are split over several CTAs).  The FP32 result must
+    round to the BF16 run's result within one BF16 step (the BF16 run is checked against
+    the oracle by the tests above) and be finite."""
+    import numpy as np
+    import torch
+    from long_context_sparse_softmax_b200 import runner
+    base = wl.shrink(wl.CSA_DECODE, name="f32_out_cluster", seed=42, seq_lens=(3000, 5200, 2100), k=128)
+    inp = wl.make_decode(base, "cuda")
+    r16 = runner.Decode(inp, "cuda")
+    r16.step()
+    inp32 = dict(inp)
+    inp32["spec"] = wl.shrink(base, out32=True)
+    r32 = runner.Decode(inp32, "cuda")
+    r32.step()
+    torch.cuda.synchronize()
+    assert r16.read_status() == 0 and r32.read_status() == 0
+    o16 = (r16.out.to(torch.int32) << 16).view(torch.float32).cpu().numpy().astype(np.float64)
+    o32 = r32.out.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(o32))
+    rms = np.sqrt(np.mean(o32 * o32, axis=-1, keepdims=True))
+    # BF16 rounding (at most 2^-9 relative, round to nearest) of the same FP32 sum; the
+    # margin covers a different summation order
+    assert np.all(np.abs(o16 - o32) <= 2.0 ** -8 * np.abs(o32) + 2.0 ** -12 * rms + 1e-30)
