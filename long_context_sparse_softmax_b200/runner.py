@@ -6,7 +6,9 @@ Prefill (one sequence): prepare queries and window tokens -> compress the contex
 cache): prepare the query and the newest token's window row, compress the block the
 newest token closed, [CSA: index -> top-k] -> attention.  With MXFP4 indexer operands the
 index and top-k stages run fused (lc_csa_index_topk_*: no score matrix) unless the run is
-built with fused=False; the separate calls stay available as index() and topk().
+built with fused=False, or the choice is left open and the fused call's merge would take
+more than FUSED_MAX_CANDIDATES candidates per query; the separate calls stay available as
+index() and topk().
 
 Nothing here computes any part of the method; every step is a kernel of liblc.so.
 """
@@ -201,6 +203,21 @@ class _Common:
                          self.W_x, max_ent, self.batch,
                          ptr(scores), scores.shape[1], ptr(self.status))
 
+    # The fused index + top-k call is the default while its merge takes at most this many
+    # candidates per query (they then stay in registers: measured faster than the separate
+    # score matrix and top-k); past it the separate calls are faster (measured on B200:
+    # 32 ranges x 1024 candidates merged in about 43 us against a 40 us separate top-k).
+    FUSED_MAX_CANDIDATES = 8192
+
+    def _choose_fused(self, fused_arg, n_q: int):
+        """Keep the fused call unless the caller left the choice open and its merge would
+        take more than FUSED_MAX_CANDIDATES candidates per query (the workspace holds them:
+        n_chunks x k pairs of 8 bytes per query)."""
+        if fused_arg is None and self.fused:
+            per_query = self.a_index_topk.workspace_bytes // (8 * max(n_q, 1))
+            if per_query > self.FUSED_MAX_CANDIDATES:
+                self.fused = False
+
     def _index_topk_args(self, n_q: int, max_ent: int, decode: bool) -> IndexTopkArgs:
         """Fused index + top-k into idx / count (the buffers the separate top-k call writes
         and attention reads)."""
@@ -297,6 +314,7 @@ class Prefill(_Common):
             self.a_topk = self._topk_args(s.n_q, n_c)
             if self.fused:
                 self.a_index_topk = self._index_topk_args(s.n_q, n_c, False)
+                self._choose_fused(fused, s.n_q)
         else:
             self.idx = None
         self.a_attn = self._attn_args(s.n_q, n_c, s.is_csa)
@@ -397,6 +415,7 @@ class Decode(_Common):
             self.a_topk = self._topk_args(B, max_ent)
             if self.fused:
                 self.a_index_topk = self._index_topk_args(B, max_ent, True)
+                self._choose_fused(fused, B)
         else:
             self.idx = None
         self.a_attn = self._attn_args(B, max_ent, s.is_csa)
