@@ -87,8 +87,11 @@ enum {
 /* Lightning-indexer operand formats. */
 enum {
   LC_IDX_F32 = 0,          /* FP32 [.., d_I] */
-  LC_IDX_MXFP4 = 3         /* OCP MXFP4: E2M1 codes [.., d_I/2] (element 2i in the low
+  LC_IDX_MXFP4 = 3,        /* OCP MXFP4: E2M1 codes [.., d_I/2] (element 2i in the low
                               nibble, 2i+1 in the high nibble) + E8M0 scales [.., d_I/32] */
+  LC_IDX_MXFP4_QBF16 = 4   /* keys as LC_IDX_MXFP4; queries BF16 [.., d_I], quantised to
+                              MXFP4 inside the call by the rule of lc_mxfp4_quantize (the
+                              same bytes); q_scale is not read */
 };
 
 /* Rows of D logical dims.  In LC_FMT_E4M3_BF16 the logical order is the D - d_r nope
@@ -196,9 +199,10 @@ typedef struct lc_index_args {
   int32_t n_q;
   int32_t H_I;             /* indexer heads (F32: H_I * d_I <= 16384; MXFP4: 32 or 64) */
   int32_t d_I;             /* indexer dims (F32: multiple of 4, <= 256; MXFP4: 128) */
-  int32_t fmt;             /* LC_IDX_F32 or LC_IDX_MXFP4 */
-  const void* q;           /* F32 [n_q, H_I, d_I] or MXFP4 codes [n_q, H_I, d_I/2] */
-  const uint8_t* q_scale;  /* MXFP4: [n_q, H_I, d_I/32], 4-byte aligned */
+  int32_t fmt;             /* LC_IDX_F32, LC_IDX_MXFP4 or LC_IDX_MXFP4_QBF16 */
+  const void* q;           /* F32 [n_q, H_I, d_I], MXFP4 codes [n_q, H_I, d_I/2] or (MXFP4_QBF16)
+                              BF16 [n_q, H_I, d_I] */
+  const uint8_t* q_scale;  /* MXFP4: [n_q, H_I, d_I/32], 4-byte aligned; else unused */
   const void* k;           /* F32 [n_keys, d_I] or MXFP4 codes [n_keys, d_I/2] */
   const uint8_t* k_scale;  /* MXFP4: [n_keys, d_I/32], 4-byte aligned */
   int64_t n_keys;          /* rows of k and k_scale (every ent_start[b] + n_ent[b] <= n_keys);

@@ -24,7 +24,7 @@ LC_OK, LC_ERR_ARG, LC_ERR_ALIGN, LC_ERR_UNSUPPORTED, LC_ERR_WORKSPACE, LC_ERR_LA
 LC_DEV_BAD_INDEX, LC_DEV_WINDOW_RANGE, LC_DEV_BAD_BLOCK, LC_DEV_NONVISIBLE, LC_DEV_TIMEOUT, LC_DEV_RANGE = \
     1, 2, 4, 8, 16, 32
 LC_FMT_F32, LC_FMT_BF16, LC_FMT_E4M3_BF16 = 0, 1, 2
-LC_IDX_F32, LC_IDX_MXFP4 = 0, 3
+LC_IDX_F32, LC_IDX_MXFP4, LC_IDX_MXFP4_QBF16 = 0, 3, 4
 
 
 class LcError(RuntimeError):

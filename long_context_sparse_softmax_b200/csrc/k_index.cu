@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(128) k_index_f32(lc_index_args a) {
 
 cudaError_t launch_index_scores(const lc_index_args& a, bool decode, cudaStream_t st) {
   if (a.n_q == 0 || a.max_ent == 0) return cudaSuccess;
-  if (a.fmt == LC_IDX_MXFP4) return launch_index_tc(a, decode, st);
+  if (a.fmt == LC_IDX_MXFP4 || a.fmt == LC_IDX_MXFP4_QBF16) return launch_index_tc(a, decode, st);
   const dim3 grid(a.n_q, (a.max_ent + 127) / 128);
   const size_t sm = static_cast<size_t>(a.H_I * a.d_I + a.H_I) * sizeof(float);
   cudaFuncSetAttribute(k_index_f32, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));

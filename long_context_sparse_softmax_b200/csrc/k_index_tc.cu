@@ -42,6 +42,7 @@
 #include <cuda.h>
 
 #include "lc_internal.h"
+#include "lc_mxfp4.cuh"
 #include "lc_ptx.cuh"
 
 namespace lc {
@@ -134,6 +135,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   __shared__ __align__(8) IdxBars bars;
   __shared__ int s_nv[QPC];
   __shared__ int s_q[QPC];
+  __shared__ uint32_t s_qsw[QPC * 64];  // MXFP4_QBF16: each query row's scale word
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_trigger();  // the merge / top-k after this kernel may start; it waits for our results
@@ -325,18 +327,45 @@ __global__ void __launch_bounds__(kThreads, 2)
     // launch): the key tiles above stream in meanwhile
     if (a.pdl) pdl_wait();
     // query operand (rows n = i * H + h), head weights, query scales
-    for (int c = et; c < N * 4; c += 128) {
-      const int n = c >> 2, seg = c & 3;
-      const int i = n / H, h = n % H;
-      const int q = s_q[i];
-      const bool ok = q < a.n_q && s_nv[i] > 0;
-      const uint8_t* src = static_cast<const uint8_t*>(a.q) + (static_cast<int64_t>(ok ? q : 0) * H + h) * kRowB + seg * 16;
-      cp_async16(su32(Bs + sw64_off(n, seg)), src, ok);
+    if (a.fmt == LC_IDX_MXFP4_QBF16) {
+      // the BF16 query rows quantised here, by the rule of the standalone quantiser: a warp
+      // takes a row of 128 dims, 4 per lane, into the operand's SW64 layout
+      for (int n = et >> 5; n < N; n += 4) {
+        const int i = n / H, h = n % H;
+        const int q = s_q[i];
+        const bool ok = q < a.n_q && s_nv[i] > 0;
+        float v[4] = {0.f, 0.f, 0.f, 0.f};
+        if (ok) {
+          const uint2 u = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(a.q) +
+                                                               (static_cast<int64_t>(q) * H + h) * kDI) + lane);
+          v[0] = __uint_as_float(u.x << 16);
+          v[1] = __uint_as_float(u.x & 0xffff0000u);
+          v[2] = __uint_as_float(u.y << 16);
+          v[3] = __uint_as_float(u.y & 0xffff0000u);
+        }
+        uint32_t sc;
+        const uint32_t c = mxfp4_quant4(v, &sc);
+        *reinterpret_cast<uint16_t*>(Bs + sw64_off(n, lane >> 3) + 2 * (lane & 7)) = static_cast<uint16_t>(c);
+        // the row's scale word: block b's byte from lane 8 b
+        const uint32_t w = __shfl_sync(0xffffffffu, sc, 0) | (__shfl_sync(0xffffffffu, sc, 8) << 8) |
+                           (__shfl_sync(0xffffffffu, sc, 16) << 16) | (__shfl_sync(0xffffffffu, sc, 24) << 24);
+        if (lane == 0) s_qsw[n] = ok ? w : 0x7f7f7f7fu;
+      }
+    } else {
+      for (int c = et; c < N * 4; c += 128) {
+        const int n = c >> 2, seg = c & 3;
+        const int i = n / H, h = n % H;
+        const int q = s_q[i];
+        const bool ok = q < a.n_q && s_nv[i] > 0;
+        const uint8_t* src = static_cast<const uint8_t*>(a.q) + (static_cast<int64_t>(ok ? q : 0) * H + h) * kRowB + seg * 16;
+        cp_async16(su32(Bs + sw64_off(n, seg)), src, ok);
+      }
     }
     for (int u = et; u < N; u += 128) {
       const int i = u / H, h = u % H;
       ws[u] = __ldg(a.w + static_cast<int64_t>(s_q[i] < a.n_q ? s_q[i] : 0) * a.w_qstride + h);
     }
+    if (a.fmt == LC_IDX_MXFP4_QBF16) named_bar(1, 128);  // every row's scale word is in s_qsw
     {
       uint32_t v[8];
 #pragma unroll
@@ -344,9 +373,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int n = lane + 32 * c;
         uint32_t w = 0x7f7f7f7fu;
         if (n < N) {
-          const int i = n / H, h = n % H;
-          const int q = s_q[i];
-          if (q < a.n_q) w = __ldg(reinterpret_cast<const uint32_t*>(a.q_scale) + static_cast<int64_t>(q) * H + h);
+          if (a.fmt == LC_IDX_MXFP4_QBF16) {
+            w = s_qsw[n];
+          } else {
+            const int i = n / H, h = n % H;
+            const int q = s_q[i];
+            if (q < a.n_q) w = __ldg(reinterpret_cast<const uint32_t*>(a.q_scale) + static_cast<int64_t>(q) * H + h);
+          }
         }
         v[c] = w;
       }

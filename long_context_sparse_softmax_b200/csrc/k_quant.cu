@@ -20,41 +20,22 @@
 #include <cmath>
 
 #include "lc_internal.h"
+#include "lc_mxfp4.cuh"
 
 namespace lc {
 
 namespace {
-
-// Two bytes of E2M1 codes: byte 0 = (v0 low nibble, v1 high), byte 1 = (v2, v3).
-__device__ __forceinline__ uint32_t e2m1x4(float v0, float v1, float v2, float v3) {
-  uint32_t r;
-  asm("{\n.reg .b8 b0, b1;\n"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n"
-      "mov.b32 %0, {b0, b1, b0, b1};\n}\n"
-      : "=r"(r)
-      : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
-  r &= 0xffffu;
-  // negative zero (sign bit over a zero magnitude) -> code 0
-  const uint32_t mag = r & 0x7777u;
-  const uint32_t zero = ~(mag | (mag >> 1) | (mag >> 2)) & 0x1111u;
-  return r & ~(zero << 3);
-}
 
 // Quantise the 4 values of this lane (elements 4 lane .. 4 lane + 3 of a 128-element chunk)
 // and store their 2 code bytes; lane 8 b stores the scale of block b of the chunk.  Every
 // lane of the warp takes part (the block maximum is a shuffle); lanes past the row's end
 // (on = false, whole 8-lane groups) store nothing.
 __device__ __forceinline__ void mxfp4_store(const float (&v)[4], int lane, bool on, uint8_t* codes, uint8_t* scales) {
-  float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-#pragma unroll
-  for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  int e = amax > 0.f ? ilogbf(amax) - 2 : 0;
-  e = min(max(e, -127), 127);
-  const uint32_t c = e2m1x4(ldexpf(v[0], -e), ldexpf(v[1], -e), ldexpf(v[2], -e), ldexpf(v[3], -e));
+  uint32_t sc;
+  const uint32_t c = mxfp4_quant4(v, &sc);
   if (!on) return;
   reinterpret_cast<uint16_t*>(codes)[lane] = static_cast<uint16_t>(c);
-  if ((lane & 7) == 0) scales[lane >> 3] = static_cast<uint8_t>(e + 127);
+  if ((lane & 7) == 0) scales[lane >> 3] = static_cast<uint8_t>(sc);
 }
 
 template <bool kF32In>

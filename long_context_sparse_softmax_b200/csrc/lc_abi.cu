@@ -96,7 +96,7 @@ lc_status check_index(const lc_index_args* a, bool decode, bool scores) {
   if (a->H_I < 1) return LC_ERR_ARG;
   if (a->fmt == LC_IDX_F32) {
     if (a->d_I < 4 || a->d_I % 4 || a->d_I > 256 || a->H_I * a->d_I > 16384) return LC_ERR_UNSUPPORTED;
-  } else if (a->fmt == LC_IDX_MXFP4) {
+  } else if (a->fmt == LC_IDX_MXFP4 || a->fmt == LC_IDX_MXFP4_QBF16) {
     // the tensor-core kernel: 128 dims (two K = 64 block-scaled MMAs), 32 or 64 heads
     if (a->d_I != 128 || (a->H_I != 32 && a->H_I != 64)) return LC_ERR_UNSUPPORTED;
   } else {
@@ -108,10 +108,11 @@ lc_status check_index(const lc_index_args* a, bool decode, bool scores) {
   if (a->n_q == 0 || a->max_ent == 0) return LC_OK;
   LC_TRY(check_batch(a->batch, true, false));
   if (!a->q || !a->k || !a->w || (scores && !a->scores)) return LC_ERR_ARG;
-  if (a->fmt == LC_IDX_MXFP4 && (!a->q_scale || !a->k_scale || a->n_keys < 1 || a->n_keys >= (int64_t{1} << 31)))
-    return LC_ERR_ARG;
-  if (a->fmt == LC_IDX_MXFP4 && ((reinterpret_cast<uintptr_t>(a->q_scale) | reinterpret_cast<uintptr_t>(a->k_scale)) & 3u))
-    return LC_ERR_ALIGN;
+  const bool mx = a->fmt == LC_IDX_MXFP4 || a->fmt == LC_IDX_MXFP4_QBF16;
+  if (mx && (!a->k_scale || a->n_keys < 1 || a->n_keys >= (int64_t{1} << 31))) return LC_ERR_ARG;
+  if (a->fmt == LC_IDX_MXFP4 && !a->q_scale) return LC_ERR_ARG;
+  if (mx && (reinterpret_cast<uintptr_t>(a->k_scale) & 3u)) return LC_ERR_ALIGN;
+  if (a->fmt == LC_IDX_MXFP4 && (reinterpret_cast<uintptr_t>(a->q_scale) & 3u)) return LC_ERR_ALIGN;
   if (!aligned16(a->q) || !aligned16(a->k) || (scores && !aligned16(a->scores))) return LC_ERR_ALIGN;
   return LC_OK;
 }
@@ -162,7 +163,7 @@ lc_status index_topk(const lc_index_topk_args* a, void* stream, bool decode) {
   if (!a) return LC_ERR_ARG;
   if (a->k < 1 || a->k > 2048) return LC_ERR_ARG;
   LC_TRY(check_index(&a->index, decode, false));
-  if (a->index.fmt != LC_IDX_MXFP4) return LC_ERR_UNSUPPORTED;
+  if (a->index.fmt != LC_IDX_MXFP4 && a->index.fmt != LC_IDX_MXFP4_QBF16) return LC_ERR_UNSUPPORTED;
   if (a->index.n_q == 0) return LC_OK;
   if (!a->idx) return LC_ERR_ARG;
   if (a->index.max_ent > 0 && lc::index_geometry(a->index, decode, true).n_chunks > 1024) return LC_ERR_UNSUPPORTED;

@@ -21,7 +21,7 @@ import torch
 
 from . import (AttnArgs, Batch, CompressArgs, Dims, IndexArgs, IndexCompressArgs, IndexTopkArgs, Mxfp4QuantArgs,
                QkPrepArgs, Rows, TopkArgs,
-               LC_FMT_BF16, LC_FMT_E4M3_BF16, LC_FMT_F32, LC_IDX_F32, LC_IDX_MXFP4,
+               LC_FMT_BF16, LC_FMT_E4M3_BF16, LC_FMT_F32, LC_IDX_F32, LC_IDX_MXFP4, LC_IDX_MXFP4_QBF16,
                lc_csa_compress_decode, lc_csa_compress_prefill, lc_csa_index_scores_decode,
                lc_csa_index_scores_prefill, lc_csa_index_topk_decode, lc_csa_index_topk_prefill,
                lc_csa_index_topk_workspace_bytes, lc_csa_index_compress_decode, lc_csa_index_compress_prefill,
@@ -69,8 +69,8 @@ class _Common:
 
     def dag(self):
         """The step as (side groups, main, after).  The side groups (query and window
-        preparation, compression) and `main` (indexer query quantisation, index scores ->
-        top-k) share no buffers that one writes and the other reads in the same step, so
+        preparation, compression) and `main` (decode: indexer query quantisation; index
+        scores -> top-k) share no buffers that one writes and the other reads in the same step, so
         they may run concurrently; `after` (attention) needs all of them.  In prefill the
         indexer keys are compressed on the main stream: the indexer reads them."""
         st = dict(self.stages())
@@ -98,7 +98,7 @@ class _Common:
             if raw:
                 h["index_compress"] = [inp["kI_raw"]]
         if qI:
-            h["quant_q" if raw else ("index_topk" if self.fused else "index")] = qI
+            h["quant_q" if raw and not self.q_in_call else ("index_topk" if self.fused else "index")] = qI
         return h
 
     def host_outputs(self):
@@ -106,8 +106,14 @@ class _Common:
         return [self.out, self.lse]
 
     def _indexer_buffers(self, n_q: int, n_keys: int, decode: bool):
-        """Indexer operands the step reads: the quantised queries (and, in prefill, the
-        compressed keys) that its own kernels write, or the given FP32 operands."""
+        """Indexer operands the step reads: in MXFP4 the queries quantised by the step's
+        quant_q stage and, in prefill, the compressed keys that the step's own kernels
+        write; or the given FP32 operands.  The indexer can quantise BF16 queries itself
+        (LC_IDX_MXFP4_QBF16, q_in_call), but the separate quantiser measured faster in both
+        steps: in decode its short kernel lets the side-stream kernels take their SMs before
+        the indexer fills every SM (in-call: decode step 103 against 92 us), and in prefill
+        each query's rows would be quantised once per key range (in-call: index 27.8 against
+        19.3 ms)."""
         s, inp, dev = self.spec, self.inp, self.device
         if s.idx_fmt != wl.IDX_MXFP4:
             self.qI, self.kI = inp["qI"], inp["kI"]
@@ -131,16 +137,18 @@ class _Common:
                                  ptr(self.status))
 
     def quant_q(self, stream=None):
+        """The indexer queries in MXFP4 by the standalone quantiser (a decode stage)."""
         lc_mxfp4_quantize(self.a_quant_q, stream)
 
     def _index_stages(self):
         """The indexer and top-k stages of a step.  On the main stream each follows another
         kernel of the step whose outputs alone it reads after that kernel completes, so it
         is launched programmatically (its set-up and the loads of its other inputs overlap
-        the previous kernel): the indexer after the query quantisation, the top-k after the
-        indexer, and the attention (see stages()) after the top-k.  Called on their own,
-        the stages launch in plain stream order."""
-        pdl_index = self.spec.idx_fmt == wl.IDX_MXFP4  # quant_q runs right before it
+        the previous kernel): the indexer after the query quantisation (unless it quantises
+        them itself: then the kernel before it may write its keys, and it launches in plain
+        order), the top-k after the indexer, and the attention (see stages()) after the
+        top-k.  Called on their own, the stages launch in plain stream order."""
+        pdl_index = self.spec.idx_fmt == wl.IDX_MXFP4 and not self.q_in_call  # after quant_q
         if self.fused:
             return [("index_topk", functools.partial(self.index_topk, pdl=pdl_index))]
         return [("index", functools.partial(self.index, pdl=pdl_index)), ("topk", functools.partial(self.topk, pdl=True))]
@@ -196,8 +204,13 @@ class _Common:
         s, inp = self.spec, self.inp
         qI, kI = self.qI, self.kI
         mx = s.idx_fmt == wl.IDX_MXFP4
-        return IndexArgs(n_q, s.H_I, s.d_I, LC_IDX_MXFP4 if mx else LC_IDX_F32,
-                         ptr(qI["codes"] if mx else qI["f32"]), ptr(qI.get("scales")),
+        if mx and self.q_in_call:
+            fmt, q, q_scale = LC_IDX_MXFP4_QBF16, ptr(inp["qI_raw"]), None
+        elif mx:
+            fmt, q, q_scale = LC_IDX_MXFP4, ptr(qI["codes"]), ptr(qI["scales"])
+        else:
+            fmt, q, q_scale = LC_IDX_F32, ptr(qI["f32"]), None
+        return IndexArgs(n_q, s.H_I, s.d_I, fmt, q, q_scale,
                          ptr(kI["codes"] if mx else kI["f32"]), ptr(kI.get("scales")),
                          (kI["codes"] if mx else kI["f32"]).shape[0], ptr(inp["w"]), s.H_I if s.w_per_query else 0, s.m,
                          self.W_x, max_ent, self.batch,
@@ -275,6 +288,7 @@ class Prefill(_Common):
         self.impl = impl
         self.spec, self.inp, self.device = s, inp, device
         self.fused = s.is_csa and s.idx_fmt == wl.IDX_MXFP4 if fused is None else fused
+        self.q_in_call = False  # the quant_q stage quantises them (see _indexer_buffers)
         self.W_x = s.W if W_x is None else W_x
         L, n_c = inp["L"], inp["n_c"]
         self.dims = Dims(s.D, s.d_r, s.rope_off, s.H)
@@ -353,7 +367,9 @@ class Prefill(_Common):
         st = [("qk_prep_q", self.prep_queries), ("qk_prep_win", self.prep_window), ("compress", self.compress)]
         if s.is_csa:
             if s.idx_fmt == wl.IDX_MXFP4:
-                st += [("index_compress", self.index_compress), ("quant_q", self.quant_q)]
+                st += [("index_compress", self.index_compress)]
+                if not self.q_in_call:
+                    st += [("quant_q", self.quant_q)]
             st += self._index_stages()
         return st + [("attn", functools.partial(self.attn, pdl=s.is_csa))]
 
@@ -371,6 +387,7 @@ class Decode(_Common):
         self.impl = impl
         self.spec, self.inp, self.device = s, inp, device
         self.fused = s.is_csa and s.idx_fmt == wl.IDX_MXFP4 if fused is None else fused
+        self.q_in_call = False  # the quant_q stage quantises them (see _indexer_buffers)
         self.W_x = s.W if W_x is None else W_x
         B = s.num_seqs
         n_c = inp["n_c"]
@@ -454,7 +471,9 @@ class Decode(_Common):
         st = [("qk_prep_q", self.prep_queries), ("qk_prep_win", self.prep_window), ("compress", self.compress)]
         if s.is_csa:
             if s.idx_fmt == wl.IDX_MXFP4:
-                st += [("index_compress", self.index_compress), ("quant_q", self.quant_q)]
+                st += [("index_compress", self.index_compress)]
+                if not self.q_in_call:
+                    st += [("quant_q", self.quant_q)]
             st += self._index_stages()
         return st + [("attn", functools.partial(self.attn, pdl=s.is_csa))]
 

@@ -99,8 +99,11 @@ def check_prefill(spec: wl.Spec, q_sel: Sequence[int] = None, W_x: int = None, r
         scores_gpu = np_(run.scores[sel_t])
         lib_kI = None
         if spec.idx_fmt == wl.IDX_MXFP4:
-            # indexer queries quantised by the path (exact inputs: bit-exact), keys pooled
+            # indexer queries quantised by the standalone quantiser (exact inputs: bit-exact;
+            # the indexer forms the same bytes itself, see test_gpu_index_topk), keys pooled
             # and quantised by the path (FP32 pooling: within one grid step)
+            run.quant_q()
+            _sync()
             assert np.array_equal(np_(run.qI["codes"][sel_t]), orc.qI_codes), "quantised indexer query codes"
             assert np.array_equal(np_(run.qI["scales"][sel_t]), orc.qI_scales), "quantised indexer query scales"
             kc, ks = np_(run.kI["codes"][:n_c]), np_(run.kI["scales"][:n_c])
@@ -264,6 +267,8 @@ def check_decode(spec: wl.Spec, W_x: int = None, report=None, impl: int = 0):
         scores_gpu = np_(run.scores)
         lib_kI = None
         if spec.idx_fmt == wl.IDX_MXFP4:
+            run.quant_q()
+            _sync()
             assert np.array_equal(np_(run.qI["codes"]), orc.qI_codes), "quantised indexer query codes"
             assert np.array_equal(np_(run.qI["scales"]), orc.qI_scales), "quantised indexer query scales"
             lib_kI = {"codes": np_(run.kI["codes"]), "scales": np_(run.kI["scales"])}

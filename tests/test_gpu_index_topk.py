@@ -99,3 +99,54 @@ def test_fused_prefill_queries_spanning_several_ranges():
     s2 = wl.shrink(wl.CSA_PREFILL, name="index_topk_prefill_early", seed=87, seq_lens=(3000,), H=16, k=256,
                    q_first=0, n_q=3000)
     _check(runner.Prefill(wl.make_prefill(s2, "cuda"), "cuda", fused=True))
+
+
+def test_indexer_quantises_queries_like_the_quantiser():
+    """The MXFP4 indexer call quantises its BF16 queries itself (LC_IDX_MXFP4_QBF16): its
+    scores must be bit-identical to those of the same call fed the standalone quantiser's
+    codes and scales (LC_IDX_MXFP4), in decode and in prefill, including queries that
+    quantise to zero blocks and to saturated codes."""
+    import long_context_sparse_softmax_b200 as lc
+
+    def both(run, decode, n_q, width):
+        run.step()     # every operand the indexer reads (prefill: its compressed keys)
+        run.quant_q()  # the standalone quantiser's codes and scales, into run.qI
+        torch.cuda.synchronize()
+        outs = []
+        for fmt in (lc.LC_IDX_MXFP4_QBF16, lc.LC_IDX_MXFP4):
+            a = type(run.a_index).from_buffer_copy(run.a_index)
+            a.fmt, a.pdl = fmt, 0
+            if fmt == lc.LC_IDX_MXFP4_QBF16:
+                a.q, a.q_scale = run.inp["qI_raw"].data_ptr(), None
+            else:
+                a.q, a.q_scale = run.qI["codes"].data_ptr(), run.qI["scales"].data_ptr()
+            sc = torch.full_like(run.scores, float("nan"))
+            a.scores = sc.data_ptr()
+            (lc.lc_csa_index_scores_decode if decode else lc.lc_csa_index_scores_prefill)(a, None)
+            outs.append(sc)
+        torch.cuda.synchronize()
+        assert run.read_status() == 0
+        for q in range(n_q):
+            n = width(q)
+            assert torch.equal(outs[0][q, :n], outs[1][q, :n]), f"query {q}: in-call quantisation differs"
+
+    def spiky(inp):
+        # BF16 bits (int16): edit through float32 and back, truncating to BF16
+        x = inp["qI_raw"]
+        f = (x.to(torch.int32) << 16).view(torch.float32)
+        f[0, 0, :32] = 0.0              # a zero block
+        f[0, 1, 5] *= 4000.0            # a block whose other values round to 0
+        f[1, 2, :] *= 1e-3
+        x.copy_((f.view(torch.int32) >> 16).to(torch.int16))
+
+    s = wl.shrink(wl.CSA_DECODE, name="qbf16_decode", seed=88, seq_lens=(9000, 20000, 513), k=256)
+    inp = wl.make_decode(s, "cuda")
+    spiky(inp)
+    run = runner.Decode(inp, "cuda", fused=False)
+    nv = _visible(run)
+    both(run, True, len(nv), lambda q: nv[q])
+    sp = wl.shrink(wl.CSA_PREFILL, name="qbf16_prefill", seed=89, seq_lens=(3000,), H=16, k=256, q_first=0,
+                   n_q=700)
+    runp = runner.Prefill(wl.make_prefill(sp, "cuda"), "cuda", fused=False)
+    nvp = _visible(runp)
+    both(runp, False, len(nvp), lambda q: nvp[q])
