@@ -531,6 +531,21 @@ def run_lc(args):
             e_ms += e0.elapsed_time(e1)
         e2e = {"value": weak_throughput(world, units, args.steps, max_over_ranks(e_ms, dev, world)), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "copies": e2e_mode}
+        if graph is not None:
+            # the same, with every C-ABI call (validation, argument marshalling, launch) and
+            # every copy issued from Python each step, as a caller without graphs would
+            barrier()
+            torch.cuda.synchronize()
+            c_ms = 0.0
+            for s in range(args.steps):
+                flush_l2()
+                e0.record(stream)
+                one_step(None, io)
+                e1.record(stream)
+                e1.synchronize()
+                c_ms += e0.elapsed_time(e1)
+            e2e["per_call"] = {"value": weak_throughput(world, units, args.steps, max_over_ranks(c_ms, dev, world)),
+                               "unit": UNIT, "copies": "eager copies and C-ABI calls issued from Python each step"}
 
     # roofline of the dominant kernel (largest share of the step); its duration comes from
     # the headline pass when that pass bracketed it
