@@ -544,8 +544,15 @@ def run_lc(args):
                 e1.record(stream)
                 e1.synchronize()
                 c_ms += e0.elapsed_time(e1)
-            e2e["per_call"] = {"value": weak_throughput(world, units, args.steps, max_over_ranks(c_ms, dev, world)),
-                               "unit": UNIT, "copies": "eager copies and C-ABI calls issued from Python each step"}
+            per_call = {"value": weak_throughput(world, units, args.steps, max_over_ranks(c_ms, dev, world)),
+                        "unit": UNIT, "copies": "eager copies and C-ABI calls issued from Python each step"}
+            # both are the public calls with the host copies timed; the faster is the value
+            # (host-to-device copies inside a graph measured slower than eager ones here)
+            if per_call["value"] > e2e["value"]:
+                e2e["graph"] = {"value": e2e["value"], "unit": UNIT, "copies": e2e["copies"]}
+                e2e["value"], e2e["copies"] = per_call["value"], per_call["copies"]
+            else:
+                e2e["per_call"] = per_call
 
     # roofline of the dominant kernel (largest share of the step); its duration comes from
     # the headline pass when that pass bracketed it

@@ -159,24 +159,29 @@ class _Common:
         attention.  on_stage(name, stream, fn) may wrap each launch (e.g. with timing
         events).  io = (h2d, d2h) adds the host copies: h2d maps a stage (or "_fork") to
         (device, pinned host) pairs copied on that stage's stream just before it, so an
-        upload overlaps the stages before it; d2h holds (pinned host, device) pairs copied
-        on `main` after attention."""
+        upload overlaps the stages before it (the main stream's uploads go first, before
+        the fork); d2h holds (pinned host, device) pairs copied on `main` after attention."""
         import torch
         sd, mn, af = self.dag()
         sides = list(side) if isinstance(side, (list, tuple)) else [side]
         launch = on_stage or (lambda name, stream, fn: fn(stream))
         h2d, d2h = io if io is not None else ({}, [])
 
+        copied = set()
+
         def run(name, stream, fn):
-            if h2d.get(name):
+            if h2d.get(name) and name not in copied:
                 with torch.cuda.stream(stream):
                     for d, h in h2d[name]:
                         d.copy_(h, non_blocking=True)
             launch(name, stream, fn)
-        if h2d.get("_fork"):
-            with torch.cuda.stream(main):
-                for d, h in h2d["_fork"]:
+        # uploads for the critical path go first, before the fork: the side streams' larger
+        # uploads (query rows) queue behind them on the copy engine instead of in front
+        with torch.cuda.stream(main):
+            for name in ["_fork"] + [n for n, _ in mn]:
+                for d, h in h2d.get(name, []):
                     d.copy_(h, non_blocking=True)
+                copied.add(name)
         fork = torch.cuda.Event()
         fork.record(main)
         used = sides[:min(len(sd), len(sides))]
