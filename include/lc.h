@@ -58,7 +58,7 @@ enum {
   LC_OK = 0,
   LC_ERR_ARG = 1,          /* a null pointer, a size out of range, inconsistent shapes */
   LC_ERR_ALIGN = 2,        /* a buffer not 16-byte aligned */
-  LC_ERR_UNSUPPORTED = 3,  /* a format / shape combination this build has no kernel for */
+  LC_ERR_UNSUPPORTED = 3,  /* a format / shape combination the library has no kernel for */
   LC_ERR_WORKSPACE = 4,    /* workspace missing or smaller than *_workspace_bytes() */
   LC_ERR_LAUNCH = 5,       /* the CUDA launch failed */
   LC_ERR_TOO_LARGE = 6     /* the call needs more scratch than the allocation-free entry
