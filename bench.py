@@ -553,6 +553,78 @@ def run_lc(args):
                 e2e["value"], e2e["copies"] = per_call["value"], per_call["copies"]
             else:
                 e2e["per_call"] = per_call
+        if graph is not None:
+            # steps overlapped as a serving loop runs them: three independent sets of
+            # buffers take turns; step i uploads its inputs on one copy stream while step
+            # i - 1 computes, and its results go back on another copy stream while step
+            # i + 1 computes.  Every step's copies and kernels are inside the timed region.
+            # No flush: between two uses of a set the other two sets' steps read about 1.6
+            # times L2's capacity (99 MB each on the decode workload: inputs larger than L2).
+            n_sets = 3
+            sets = [(graph, io)]
+            extra = []
+            for _ in range(n_sets - 1):
+                runs2 = make_runs(args.workload, dev, rank, {"auto": 0, "tc": 2, "ref": 3}[args.attn_impl],
+                                  False if args.no_fused else None)
+                rl2 = [r for _, _, r in runs2]
+                for r in rl2:
+                    r.step(stream)
+                torch.cuda.synchronize()
+                sets.append((capture_step(rl2, stream, side, None), host_io(runs2)))
+                extra.append(runs2)
+            up_st, down_st = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+            done_c = [torch.cuda.Event() for _ in sets]   # the set's last step computed
+            done_d = [torch.cuda.Event() for _ in sets]   # the set's last results read back
+            used = [False] * n_sets
+
+            def pipelined(n):
+                for i in range(n):
+                    k = i % n_sets
+                    g2, io_k = sets[k]
+                    if used[k]:
+                        up_st.wait_event(done_c[k])      # its inputs are no longer read
+                    with torch.cuda.stream(up_st):
+                        for hd, _ in io_k:
+                            for pairs in hd.values():
+                                for d, h in pairs:
+                                    d.copy_(h, non_blocking=True)
+                    up = torch.cuda.Event()
+                    up.record(up_st)
+                    stream.wait_event(up)
+                    if used[k]:
+                        stream.wait_event(done_d[k])     # its outputs were read back
+                    g2.replay()
+                    done_c[k].record(stream)
+                    down_st.wait_event(done_c[k])
+                    with torch.cuda.stream(down_st):
+                        for _, dl in io_k:
+                            for h, d in dl:
+                                h.copy_(d, non_blocking=True)
+                    done_d[k].record(down_st)
+                    used[k] = True
+
+            pipelined(max(n_sets, args.warmup))
+            torch.cuda.synchronize()
+            barrier()
+            p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            p0.record(up_st)
+            stream.wait_event(p0)
+            pipelined(args.steps)
+            for k in range(n_sets):
+                down_st.wait_event(done_d[k])
+            p1.record(down_st)
+            p1.synchronize()
+            pipe = {"value": weak_throughput(world, units, args.steps, max_over_ranks(p0.elapsed_time(p1), dev, world)),
+                    "unit": UNIT, "copies": "overlapped steps: uploads and read-backs on two copy streams "
+                    "overlap the neighbouring steps' kernels (three buffer sets in turn, no L2 flush: the "
+                    "other sets' steps read about 1.6x L2 between two uses of a set)"}
+            prev = {"value": e2e["value"], "unit": UNIT, "copies": e2e["copies"]}
+            if pipe["value"] > e2e["value"]:
+                e2e["serial"] = prev
+                e2e["value"], e2e["copies"] = pipe["value"], pipe["copies"]
+            else:
+                e2e["pipelined"] = pipe
+            del sets, extra
 
     # roofline of the dominant kernel (largest share of the step); its duration comes from
     # the headline pass when that pass bracketed it
