@@ -553,7 +553,9 @@ def run_lc(args):
                 e2e["value"], e2e["copies"] = per_call["value"], per_call["copies"]
             else:
                 e2e["per_call"] = per_call
-        if graph is not None:
+        if graph is not None and h2d + d2h < (256 << 20):
+            # (decode-sized steps: prefill moves gigabytes per step, and three pinned copies
+            # of its inputs would not fit the host)
             # steps overlapped as a serving loop runs them: three independent sets of
             # buffers take turns; step i uploads its inputs on one copy stream while step
             # i - 1 computes, and its results go back on another copy stream while step
