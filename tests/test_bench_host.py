@@ -59,6 +59,20 @@ def test_host_inputs_name_the_stage_that_reads_them():
     assert [n for n, _ in rp.dag()[1]] == ["index_compress", "quant_q", "index_topk"]
 
 
+def test_runner_keeps_fused_topk_only_for_small_merges():
+    """The fused index + top-k call is the default while its merge takes at most
+    FUSED_MAX_CANDIDATES candidates per query (n_chunks x k, read from the call's
+    workspace size); a long two-sequence batch with k = 1024 spreads each query over many
+    key ranges and gets the separate calls; an explicit fused=True is kept."""
+    long_ = wl.shrink(wl.MIXED_CSA, name="fused_choice_long", seq_lens=(200000, 160000), k=1024)
+    inp = wl.make_decode(long_, "cpu")
+    r = runner.Decode(inp, "cpu")
+    assert not r.fused and [n for n, _ in r.stages()][-3:] == ["index", "topk", "attn"]
+    assert runner.Decode(inp, "cpu", fused=True).fused
+    short = wl.shrink(wl.CSA_DECODE, name="fused_choice_short", seq_lens=(4096, 3000), k=512)
+    assert runner.Decode(wl.make_decode(short, "cpu"), "cpu").fused
+
+
 @pytest.mark.parametrize("name", ["csa_decode", "csa_prefill", "hca_prefill", "mixed_decode", "tiny_csa_prefill"])
 @pytest.mark.parametrize("fused", [None, False])
 def test_stage_work_covers_every_stage(name, fused):
