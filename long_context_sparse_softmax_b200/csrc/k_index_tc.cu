@@ -28,17 +28,21 @@
 // The roles meet only at mbarriers.  Every wait is bounded: after ~2^26 polls a role
 // records LC_DEV_TIMEOUT in the status word and sets an abort flag that stops the others.
 //
-// Fused selection (SELECT, lc_csa_index_topk_*): the epilogue keeps the scores of the
-// CTA's key range in shared memory instead of writing them out, and after the last tile
-// its 128 threads select the range's top K = min(k, keys in range) exactly, ties to the
-// lower index: radix passes of 11 bits over the order-preserving keys (relative to the
-// range's smallest) find the K-th largest key T and how many keys equal to T to take;
-// keys equal to T are ranked in index order with warp ballots.  The selection is a
-// bitmap in index order.  With one CTA per query it is the answer (indices written
-// ascending); otherwise the CTA writes its K (key, index) candidates in index order and
-// k_topk_merge picks the final K among every range's candidates.  Every entry of the
-// query's top K is in the top K of its own range, so the result equals csa_topk on the
-// scores this kernel computes.
+// Fused selection (SELECT, lc_csa_index_topk_*): the epilogue keeps the order-preserving
+// keys of its range's scores in shared memory (and each thread's key range) instead of
+// writing the scores out, and after the last tile its 128 threads select the range's top
+// K = min(k, keys in range) exactly, ties to the lower index: radix passes of 11 bits over
+// key - min (per-warp histograms) narrow the bin holding the K-th key until it holds at
+// most kSmallBin keys, which are ranked exactly (more equal keys than that are ranked in
+// index order with warp ballots).  The result is the pair (Tk, Ts): a key is selected iff
+// it is above Tk, or equal to it at an offset up to Ts.  Output positions come from
+// per-(tile, warp) counts and one scan.  With one CTA per query the selection is the
+// answer (indices written ascending); otherwise the CTA writes its K (key, index)
+// candidates in index order and k_topk_merge picks the final K among every range's
+// candidates.  Every entry of the query's top K is in the top K of its own range, so the
+// result equals csa_topk on the scores this kernel computes.  The selection runs once per
+// launch, so its loops stay rolled: a taken branch into code not yet fetched stalls on the
+// instruction fetch, which unrolled loops with guarded bodies multiply.
 #include <cuda.h>
 
 #include "lc_internal.h"
