@@ -21,6 +21,7 @@
 
 #include "lc_internal.h"
 #include "lc_mxfp4.cuh"
+#include "lc_ptx.cuh"
 
 namespace lc {
 
@@ -60,6 +61,9 @@ __device__ __forceinline__ void load4(const void* row, int e, float (&v)[4]) {
 // One warp per row, 8 rows per CTA.
 template <bool kF32In>
 __global__ void __launch_bounds__(256) k_mxfp4_quantize(lc_mxfp4_quant_args a) {
+  // the indexer after this kernel (programmatic dependent launch) may start its set-up and
+  // its key loads now; it reads the codes only once this grid has completed
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (row >= a.n_rows) return;
