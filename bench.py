@@ -364,8 +364,9 @@ def run_lc(args):
     # event times include the wait for SMs the critical path holds)
     crit_names = [f"{i}:{n}" for i, (_, _, r) in enumerate(runs) for part in r.dag()[1:] for n, _ in part]
     # kernels per step: one per call, plus the combine kernel of an attention whose key
-    # splits leave partials in a workspace, plus the merge kernel of a fused index + top-k
-    # whose queries span several indexer CTAs (it then has a candidate workspace)
+    # splits leave partials in a workspace (or, in HCA prefill, the kernel that widens the
+    # entries into that workspace), plus the merge kernel of a fused index + top-k whose
+    # queries span several indexer CTAs (it then has a candidate workspace)
     n_launch = len(stage_names) + sum(1 for (_, _, r) in runs if r.a_attn.workspace_bytes > 0) + \
         sum(1 for (_, _, r) in runs if getattr(r, "fused", False) and r.a_index_topk.workspace_bytes > 0)
     # one stream per side stage: they share no buffers, so none waits for another

@@ -344,7 +344,12 @@ lc_status lc_csa_index_compress_decode(const lc_index_compress_args* a, void* st
  * "DeepSeek-V4 论文分析" §5.4, §六, §七 and §8.4 (sparse core attention).
  * out: [n_q, H, D] in out_fmt (F32 or BF16); lse: [n_q, H] FP32 (optional).
  * The decode variant may split the keys of each query across CTAs; it then needs a
- * workspace of lc_*_workspace_bytes(a) bytes (the prefill variant needs none).
+ * workspace of lc_*_workspace_bytes(a) bytes.  The prefill variants need none.  The HCA
+ * prefill variant takes an optional one of lc_hca_attn_prefill_workspace_bytes(a) bytes
+ * (16-byte aligned; 0 when it does not apply): with BF16 queries it then widens the
+ * entries to F16 once per call instead of once per query, and reads each 64 visible
+ * entries that start on a multiple of 64 in the entry array as one bulk copy.  The
+ * results are the same either way; a smaller workspace is not an error.
  * ------------------------------------------------------------------------------- */
 typedef struct lc_attn_args {
   lc_dims dims;
@@ -404,6 +409,8 @@ lc_status lc_hca_attn_decode(const lc_attn_args* a, void* stream);
 
 size_t lc_csa_sparse_attn_workspace_bytes(const lc_attn_args* a);
 size_t lc_hca_attn_workspace_bytes(const lc_attn_args* a);
+/* F16 image of the n_ent_rows entry rows (needs n_ent_rows > 0), or 0 */
+size_t lc_hca_attn_prefill_workspace_bytes(const lc_attn_args* a);
 
 /* ---------------------------------------------------------------------------------
  * lc_csa_sparse_attn_decode_static — lc_csa_sparse_attn_decode for callers that cannot

@@ -125,7 +125,8 @@ ENTRY_POINTS = {
     "lc_hca_attn_prefill": AttnArgs, "lc_hca_attn_decode": AttnArgs,
     "lc_csa_sparse_attn_decode_static": AttnArgs,
 }
-HELPERS = ["lc_csa_sparse_attn_workspace_bytes", "lc_hca_attn_workspace_bytes", "lc_csa_index_topk_workspace_bytes",
+HELPERS = ["lc_csa_sparse_attn_workspace_bytes", "lc_hca_attn_workspace_bytes", "lc_hca_attn_prefill_workspace_bytes",
+           "lc_csa_index_topk_workspace_bytes",
            "lc_version",
            "lc_status_string", "lc_struct_size", "lc_csa_sparse_attn_decode_static_capacity"]
 
@@ -138,7 +139,8 @@ def _load() -> ctypes.CDLL:
         fn = getattr(so, name)
         fn.argtypes = [ctypes.POINTER(st), c_void_p]
         fn.restype = c_int32
-    for name in ("lc_csa_sparse_attn_workspace_bytes", "lc_hca_attn_workspace_bytes"):
+    for name in ("lc_csa_sparse_attn_workspace_bytes", "lc_hca_attn_workspace_bytes",
+                 "lc_hca_attn_prefill_workspace_bytes"):
         fn = getattr(so, name)
         fn.argtypes = [ctypes.POINTER(AttnArgs)]
         fn.restype = c_size_t
@@ -205,6 +207,10 @@ def lc_csa_sparse_attn_workspace_bytes(args: AttnArgs) -> int:
 
 def lc_hca_attn_workspace_bytes(args: AttnArgs) -> int:
     return int(load().lc_hca_attn_workspace_bytes(ctypes.byref(args)))
+
+
+def lc_hca_attn_prefill_workspace_bytes(args: AttnArgs) -> int:
+    return int(load().lc_hca_attn_prefill_workspace_bytes(ctypes.byref(args)))
 
 
 def lc_csa_index_topk_workspace_bytes(args: IndexTopkArgs, decode: bool) -> int:

@@ -168,6 +168,17 @@ size_t attn_workspace_bytes(const lc_attn_args& a, bool sparse, bool decode) {
   return attn_tc_supported(t) ? attn_tc_workspace(a, sparse, decode) : 0;
 }
 
+// The optional prefill workspace: the F16 image of the entries that the F16-operand kernel
+// reads instead of widening each query's tiles (dense keys, BF16 queries).
+size_t attn_image_bytes(const lc_attn_args& a, bool sparse, bool decode) {
+  if (attn_impl(a) != LC_IMPL_TC) return 0;
+  lc_attn_args t = a;
+  t.out = nullptr;
+  t.workspace = nullptr;
+  if (attn_tc8_supported(t) || !attn_tc_supported(t)) return 0;
+  return attn_tc_image_bytes(a, sparse, decode);
+}
+
 cudaError_t launch_attn(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st) {
   if (a.n_q == 0) return cudaSuccess;
   if (attn_impl(a) == LC_IMPL_TC) {

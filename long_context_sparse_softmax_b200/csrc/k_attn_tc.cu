@@ -208,7 +208,49 @@ __device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_
   asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
 }
 
+// one contiguous global -> shared copy, completing `bytes` on the mbarrier (this CTA only)
+__device__ __forceinline__ void bulk_load(uint8_t* sdst, const void* gsrc, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                   su32(sdst)),
+               "l"(gsrc), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 }  // namespace
+
+// Dense (HCA) prefill: every query of a sequence reads the same entry rows, so they are
+// widened to F16 once per call rather than once per query.  Tile T of the image holds
+// entry rows 64 T .. 64 T + 63 (zeros past n_rows) in the core-matrix layout that
+// tile_copy + tile_convert leave in shared memory, with the same conversions, so a tile
+// loaded from the image is byte for byte the tile a gather would build.  Thread i writes
+// the 16 bytes at image offset 16 i: tile T, row group g, dim chunk c, row r8 of the group.
+__global__ void __launch_bounds__(256) k_attn_f16_tiles(lc_rows ent, int n_rows, int n_tiles,
+                                                         uint8_t* __restrict__ img, int32_t* status) {
+  constexpr int kPer = kTile / 16;  // 16-byte items per tile
+  const int64_t n_items = static_cast<int64_t>(n_tiles) * kPer;
+  const uint8_t* x = static_cast<const uint8_t*>(ent.x);
+  const uint8_t* rope = static_cast<const uint8_t*>(ent.rope);
+  bool big = false;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_items;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int o = static_cast<int>(i % kPer);
+    const int g = o / (8 * (kD / 8)), c = (o / 8) % (kD / 8), r8 = o % 8;
+    const int64_t row = (i / kPer) * kTK + g * 8 + r8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (row < n_rows) {
+      if (ent.fmt == LC_FMT_BF16) {
+        v = bf16x8_f16x8(__ldg(reinterpret_cast<const uint4*>(x + (row * kD + c * 8) * 2)), big);
+      } else if (c < kDN / 8) {
+        const uint2 w = __ldg(reinterpret_cast<const uint2*>(x + row * kDN + c * 8));
+        v = e4m3x8_f16x8(w.x, w.y);
+      } else {
+        v = bf16x8_f16x8(__ldg(reinterpret_cast<const uint4*>(rope + (row * kDR + (c * 8 - kDN)) * 2)), big);
+      }
+    }
+    reinterpret_cast<uint4*>(img)[i] = v;
+  }
+  if (big) set_status(status, LC_DEV_RANGE);
+}
 
 struct AttnTcGeom {
   int n_split;
@@ -228,9 +270,12 @@ struct TcBars {
 
 // grid: one CTA per (query, head group, key split), the split index fastest; 288 threads.
 // Partial results of split s go to ws_o rows s * n_q * H + q * H + h (576 floats each) and
-// ws_ml[2 ((q * H + h) * n_split + s) + {0, 1}] = (m, l).
+// ws_ml[2 ((q * H + h) * n_split + s) + {0, 1}] = (m, l).  img (dense keys only, or null):
+// the entries as F16 tiles (k_attn_f16_tiles), img_tiles of them; a tile of 64 visible
+// entries that starts on a multiple of 64 in the entry array is then one bulk copy.
 __global__ void __launch_bounds__(kThreads, 1)
-    k_attn_tc(lc_attn_args a, int sparse, AttnTcGeom geo, float* __restrict__ ws_o, float* __restrict__ ws_ml) {
+    k_attn_tc(lc_attn_args a, int sparse, AttnTcGeom geo, float* __restrict__ ws_o, float* __restrict__ ws_ml,
+              const uint8_t* __restrict__ img, int img_tiles) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* Qs = smem;                                             // kTile
   uint8_t* Ks = Qs + kTile;                                       // [2][kTile]
@@ -335,6 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int pt = tid - 128, pw = warp - 4;
     const RowSrc src_win = row_src(a.win), src_ent = row_src(a.ent);
     int code_next = pt < kTK ? slot_code(s_begin + pt) : -1;
+    int last_bulk0 = -1, last_bulk1 = -1;  // thread pt = 0: the last tile of stage 0 / 1 it bulk-copied
     for (int t = 0; t < n_tiles; ++t) {
       const int st = t & 1;
       // stage st (and its key codes) is free once O(t - 2) is done: that also means the
@@ -345,6 +391,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (pt < kTK && t + 1 < n_tiles) code_next = slot_code(s_begin + (t + 1) * kTK + pt);
       uint8_t* kt = Ks + st * kTile;
       const int* kc = kcode + st * kTK;
+      // dense keys: slot s is entry s, so 64 visible entries from a multiple of 64 in the
+      // entry array are one image tile
+      const int s0 = s_begin + t * kTK;
+      const int64_t e0 = ent0 + s0;
+      if (img != nullptr && !sparse && s0 + kTK <= nv && e0 % kTK == 0 && e0 / kTK < img_tiles) {
+        if (pt == 0) {
+          mbar_expect_tx(su32(&bars.kfull[st]), kTile);  // this thread's arrival, plus the bytes
+          bulk_load(kt, img + (e0 / kTK) * kTile, kTile, su32(&bars.kfull[st]));
+          (st ? last_bulk1 : last_bulk0) = t;
+        } else {
+          mbar_arrive(su32(&bars.kfull[st]));
+        }
+        continue;
+      }
+      (st ? last_bulk1 : last_bulk0) = -1;  // stage st was released by O(t - 2): its copies have landed
       tile_copy(kt, pw, 4, lane, [&](int r, RowSrc& rs, int64_t& row) {
         const int code = kc[r];
         rs = (code & kWin) ? src_win : src_ent;
@@ -360,6 +421,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_smem();
       mbar_arrive(su32(&bars.kfull[st]));
     }
+    // a role that gave up may leave bulk copies in flight: they land (in bounded time,
+    // from valid memory) before the CTA's shared memory is released
+    if (pt == 0)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int lb = i ? last_bulk1 : last_bulk0;
+        if (lb >= 0) {
+          long it = 0;
+          while (!mbar_test(su32(&bars.kfull[i]), (lb >> 1) & 1) && ++it < kSpin) {
+          }
+          if (it >= kSpin) set_status(a.status, LC_DEV_TIMEOUT);
+        }
+      }
   } else if (warp == 8) {
     // ================= MMA issue (one lane) =================
     if (lane == 0) {
@@ -625,6 +699,13 @@ size_t attn_tc_workspace(const lc_attn_args& a, bool sparse, bool decode) {
   return rows * kD * sizeof(float) + rows * 2 * sizeof(float);
 }
 
+// Dense prefill: the F16 image of every entry row (n_ent_rows of them, in 64-row tiles),
+// built once per call; 0 where it does not apply (CSA, decode, n_ent_rows unknown).
+size_t attn_tc_image_bytes(const lc_attn_args& a, bool sparse, bool decode) {
+  if (sparse || decode || a.n_ent_rows <= 0) return 0;
+  return static_cast<size_t>((a.n_ent_rows + kTK - 1) / kTK) * kTile;
+}
+
 cudaError_t launch_attn_tc(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st, int* n_split_out) {
   const AttnTcGeom g = tc_geometry(a, sparse, decode);
   *n_split_out = g.n_split;
@@ -634,8 +715,24 @@ cudaError_t launch_attn_tc(const lc_attn_args& a, bool sparse, bool decode, cuda
   if (g.n_split > 1) ws_ml = ws_o + static_cast<size_t>(a.n_q) * a.dims.H * g.n_split * kD;
   const int64_t ctas = static_cast<int64_t>(a.n_q) * (a.dims.H / kNR) * g.n_split;
   if (ctas > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  // the image, when the caller's workspace holds it (the prefill variant splits no keys, so
+  // the workspace is otherwise unused)
+  const size_t img_bytes = g.n_split == 1 ? attn_tc_image_bytes(a, sparse, decode) : 0;
+  uint8_t* img = nullptr;
+  int img_tiles = 0;
+  if (img_bytes > 0 && a.workspace && a.workspace_bytes >= img_bytes &&
+      reinterpret_cast<uintptr_t>(a.workspace) % 16 == 0) {
+    img = static_cast<uint8_t*>(a.workspace);
+    img_tiles = (a.n_ent_rows + kTK - 1) / kTK;
+    const int64_t items = static_cast<int64_t>(img_tiles) * (kTile / 16);
+    const int64_t want = (items + 255) / 256, cap = 8LL * sm_count();
+    const int blocks = static_cast<int>(want < cap ? want : cap);
+    k_attn_f16_tiles<<<blocks, 256, 0, st>>>(a.ent, a.n_ent_rows, img_tiles, img, a.status);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   return launch_ex(k_attn_tc, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), kSmem, st, a.pdl != 0, 1, a,
-                   sparse ? 1 : 0, g, ws_o, ws_ml);
+                   sparse ? 1 : 0, g, ws_o, ws_ml, static_cast<const uint8_t*>(img), img_tiles);
 }
 
 }  // namespace lc

@@ -255,6 +255,10 @@ size_t lc_csa_sparse_attn_workspace_bytes(const lc_attn_args* a) {
 size_t lc_hca_attn_workspace_bytes(const lc_attn_args* a) {
   return a ? lc::attn_workspace_bytes(*a, false, true) : 0;
 }
+// Optional workspace of the HCA prefill variant (the F16 image of the entries).
+size_t lc_hca_attn_prefill_workspace_bytes(const lc_attn_args* a) {
+  return a ? lc::attn_image_bytes(*a, false, false) : 0;
+}
 
 const char* lc_version(void) { return "lc 0.1.0 (CSA/HCA attention, sm_100a)"; }
 

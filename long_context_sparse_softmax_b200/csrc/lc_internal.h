@@ -53,10 +53,12 @@ cudaError_t launch_topk(const lc_topk_args& a, bool decode, cudaStream_t st);
 cudaError_t launch_empty_selection(int32_t* idx, int32_t* count, int n_q, int k, cudaStream_t st);
 cudaError_t launch_attn(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st);
 size_t attn_workspace_bytes(const lc_attn_args& a, bool sparse, bool decode);
+size_t attn_image_bytes(const lc_attn_args& a, bool sparse, bool decode);
 bool attn_tc_supported(const lc_attn_args& a);
 int attn_impl(const lc_attn_args& a);
 bool attn_impl_ok(const lc_attn_args& a);
 size_t attn_tc_workspace(const lc_attn_args& a, bool sparse, bool decode);
+size_t attn_tc_image_bytes(const lc_attn_args& a, bool sparse, bool decode);
 cudaError_t launch_attn_tc(const lc_attn_args& a, bool sparse, bool decode, cudaStream_t st, int* n_split);
 cudaError_t launch_attn_combine(const lc_attn_args& a, int n_split, cudaStream_t st);
 bool attn_tc8_supported(const lc_attn_args& a);

@@ -27,7 +27,7 @@ from . import (AttnArgs, Batch, CompressArgs, Dims, IndexArgs, IndexCompressArgs
                lc_csa_index_topk_workspace_bytes, lc_csa_index_compress_decode, lc_csa_index_compress_prefill,
                lc_mxfp4_quantize, lc_csa_sparse_attn_decode, lc_csa_sparse_attn_prefill,
                lc_csa_sparse_attn_workspace_bytes, lc_csa_topk_decode, lc_csa_topk_prefill,
-               lc_hca_attn_decode, lc_hca_attn_prefill, lc_hca_attn_workspace_bytes,
+               lc_hca_attn_decode, lc_hca_attn_prefill, lc_hca_attn_prefill_workspace_bytes, lc_hca_attn_workspace_bytes,
                lc_hca_compress_decode, lc_hca_compress_prefill, lc_qk_prep_decode, lc_qk_prep_prefill)
 from . import workloads as wl
 
@@ -255,7 +255,7 @@ class _Common:
         return TopkArgs(n_q, s.k, s.m, self.W_x, max_ent, 0, ptr(self.scores), self.scores.shape[1], self.batch,
                         ptr(self.idx), ptr(self.count), ptr(self.status))
 
-    def _attn_args(self, n_q: int, max_ent: int, sparse: bool) -> AttnArgs:
+    def _attn_args(self, n_q: int, max_ent: int, sparse: bool, prefill: bool = False) -> AttnArgs:
         s = self.spec
         a = AttnArgs()
         a.dims = self.dims
@@ -275,7 +275,12 @@ class _Common:
         a.n_ent_rows = int(next(iter(self.ent.values())).shape[0])
         a.n_win_rows = int(self.win["x"].shape[0])
         a.v_nope = 1 if s.v_nope else 0
-        ws = (lc_csa_sparse_attn_workspace_bytes if sparse else lc_hca_attn_workspace_bytes)(a)
+        if sparse:
+            ws = lc_csa_sparse_attn_workspace_bytes(a)
+        elif prefill:  # optional: the entries widened to F16 once per call
+            ws = lc_hca_attn_prefill_workspace_bytes(a)
+        else:
+            ws = lc_hca_attn_workspace_bytes(a)
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.device)
         a.workspace, a.workspace_bytes = ptr(self.workspace), ws
         return a
@@ -336,7 +341,7 @@ class Prefill(_Common):
                 self._choose_fused(fused, s.n_q)
         else:
             self.idx = None
-        self.a_attn = self._attn_args(s.n_q, n_c, s.is_csa)
+        self.a_attn = self._attn_args(s.n_q, n_c, s.is_csa, prefill=True)
 
     def prep_queries(self, stream=None):
         lc_qk_prep_prefill(self.a_prep_q, stream)

@@ -159,3 +159,27 @@ def test_csa_decode_f32_output_cluster_merge():
     # BF16 rounding (at most 2^-9 relative, round to nearest) of the same FP32 sum; the
     # margin covers a different summation order
     assert np.all(np.abs(o16 - o32) <= 2.0 ** -8 * np.abs(o32) + 2.0 ** -12 * rms + 1e-30)
+
+
+def test_hca_prefill_entry_image_is_bit_identical():
+    """With its optional workspace, dense prefill widens the entries to F16 once and reads
+    each 64 visible entries as one tile of that image; without it, every query gathers and
+    widens its own tiles.  Both give the same bits.  Here 200 entries give three image
+    tiles, then a gathered tile of the last visible entries and the window."""
+    import torch
+    from long_context_sparse_softmax_b200 import runner
+    L = 128 * 200 + 77
+    s = wl.shrink(wl.HCA_PREFILL, name="hca_image", seed=52, seq_lens=(L,), q_first=L - 96, n_q=96)
+    check_prefill(s, q_sel=range(0, 96, 5))
+    run = runner.Prefill(wl.make_prefill(s, "cuda"), "cuda")
+    n_rows = run.a_attn.n_ent_rows
+    assert n_rows >= 200 and run.a_attn.workspace_bytes == (n_rows + 63) // 64 * 64 * 1152
+    run.step()
+    torch.cuda.synchronize()
+    assert run.read_status() == 0
+    out_img, lse_img = run.out.clone(), run.lse.clone()
+    run.a_attn.workspace_bytes = 0  # the per-query gather path
+    run.attn()
+    torch.cuda.synchronize()
+    assert run.read_status() == 0
+    assert torch.equal(out_img, run.out) and torch.equal(lse_img, run.lse)
