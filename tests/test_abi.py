@@ -116,3 +116,30 @@ def test_binding_raises_on_error_status():
     assert e.value.status == lc.LC_ERR_ARG
     with pytest.raises(TypeError):
         lc.lc_csa_topk_prefill(lc.AttnArgs(), 0)
+
+
+def test_attention_workspace_sizes_on_the_host():
+    """The size queries read only host fields.  HCA prefill with BF16 queries (the
+    F16-operand kernel) offers an F16 image of the entries, 73,728 bytes per 64 entry
+    rows; nothing where that kernel does not run or the entry rows are unknown."""
+    a = lc.AttnArgs()
+    a.dims = lc.Dims(576, 64, 512, 64)
+    a.n_q, a.m, a.W, a.max_ent, a.out_fmt = 4096, 128, 128, 8192, lc.LC_FMT_BF16
+    a.q = lc.Rows(fmt=lc.LC_FMT_BF16)
+    a.ent = lc.Rows(fmt=lc.LC_FMT_E4M3_BF16)
+    a.win = lc.Rows(fmt=lc.LC_FMT_BF16)
+    size = lc.lc_hca_attn_prefill_workspace_bytes
+    a.n_ent_rows = 8192
+    assert size(a) == 128 * 73728
+    a.n_ent_rows = 8193
+    assert size(a) == 129 * 73728
+    a.n_ent_rows = 0
+    assert size(a) == 0
+    a.n_ent_rows = 8192
+    assert lc.lc_hca_attn_workspace_bytes(a) == 0  # decode sizes: 4096 queries split no keys
+    a.impl = lc.LC_IMPL_REF
+    assert size(a) == 0
+    a.impl = lc.LC_IMPL_AUTO
+    a.q = lc.Rows(fmt=lc.LC_FMT_E4M3_BF16)  # E4M3 queries: the E4M3-score kernel
+    a.n_win_rows = 128
+    assert size(a) == 0
