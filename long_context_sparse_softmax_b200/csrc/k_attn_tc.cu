@@ -15,7 +15,9 @@
 //     second chunk.  A conversion pass then widens E4M3 to F16 in place (exact) and rounds
 //     BF16 to F16 in place (exact for magnitudes in [2^-14, 65504], which RMS-normalised
 //     rows stay within; a value beyond 65504 is reported as LC_DEV_RANGE).  F16 rather than
-//     BF16 operands give P 11 significant bits instead of 8;
+//     BF16 operands give P 11 significant bits instead of 8.  Dense prefill, given the
+//     workspace for it, widens the entries once per call into tiles of this layout
+//     (k_attn_f16_tiles); a tile of 64 visible entries is then one bulk copy;
 //   * S = Q K^T: M = 64 heads, N = 64 keys, K = 576, two tensor-memory buffers (M = 64
 //     layout: row r in lane 32 (r / 16) + r % 16; the 16x32bx2 load gives lanes 0-15 of a
 //     warp columns 0-31 and lanes 16-31 columns 32-63 of the same rows);
