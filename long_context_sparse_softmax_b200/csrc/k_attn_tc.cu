@@ -32,12 +32,14 @@
 // is staged in the freed key stages and written by one bulk copy.  A query's keys may be
 // split across CTAs; each split then writes (O, m, l) and k_attn_combine merges them.
 //
-// Warp roles (288 threads): warps 0-3 load Q, turn S into P and write the output (each
+// Warp roles (320 threads): warps 0-3 load Q, turn S into P and write the output (each
 // reaches its own quarter of the tensor-memory lanes); warps 4-7 gather key tiles into a
-// two-stage ring; lane 0 of warp 8 issues the MMAs, whichever of S(t + 1) and O(t) is
-// ready first.  The roles meet only at mbarriers and named barriers, and every mbarrier
-// wait is bounded: a role that gives up sets LC_DEV_TIMEOUT and an abort flag that stops
-// the others at their next wait.
+// two-stage ring; lane 0 of warp 8 issues the S MMAs and lane 0 of warp 9 the O MMAs.  At
+// these shapes the tensor pipe takes an MMA in about 35 cycles, but one thread issues one
+// only every ~53, so two issuers overlap that cost.  The roles meet only at mbarriers and
+// named barriers, and every mbarrier wait is bounded: a role that gives up sets
+// LC_DEV_TIMEOUT and an abort flag that stops the others at their next wait; copies and
+// MMAs already in flight are waited for (bounded) before the CTA exits.
 #include "lc_internal.h"
 #include "lc_ptx.cuh"
 
@@ -59,7 +61,7 @@ constexpr int kNPair = kD / 16;           // chunk pairs per row (36)
 constexpr int kWI = kNPair / 4;           // conversion warp instructions per row group
 constexpr long kSpin = 1L << 26;
 constexpr uint32_t kWin = 1u << 30;
-constexpr int kThreads = 288;
+constexpr int kThreads = 320;
 constexpr float kRescale = 8.f;           // log2 headroom before the reference moves
 constexpr int kColS = 0;                  // S buffers at columns 0 and 64
 constexpr int kColO = 2 * kTK;            // O^T chunk c at 128 + 64 c
@@ -267,7 +269,8 @@ struct TcBars {
   uint64_t sempty[2];  // S buffer read (128 arrivals)
   uint64_t pfull;      // P written (128 arrivals)
   uint64_t pempty;     // P read and O updated (commit)
-  uint64_t fin;        // every MMA complete (commit)
+  uint64_t fin;        // every S MMA complete (commit)
+  uint64_t fin2;       // every O MMA complete (commit)
 };
 
 // grid: one CTA per (query, head group, key split), the split index fastest; 288 threads.
@@ -326,6 +329,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     atomicExch(&s_abort, 1);
     return false;
   };
+  // bounded wait that ignores the abort flag: for copies and MMAs already in flight, which
+  // must land before the CTA releases its tensor memory and exits
+  auto drain = [&](uint64_t* bar, uint32_t parity) {
+    const uint32_t addr = su32(bar);
+    for (long it = 0; it < kSpin; ++it)
+      if (mbar_test(addr, parity)) return;
+    set_status(a.status, LC_DEV_TIMEOUT);
+  };
   // key slot -> entry index j, kWin | window row, or -1 (masked)
   auto slot_code = [&](int s) -> int {
     if (s >= s_end) return -1;
@@ -370,6 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(su32(&bars.pfull), 128);
     mbar_init(su32(&bars.pempty), 1);
     mbar_init(su32(&bars.fin), 1);
+    mbar_init(su32(&bars.fin2), 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n");
   }
   fence_before();
@@ -425,80 +437,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // a role that gave up may leave bulk copies in flight: they land (in bounded time,
     // from valid memory) before the CTA's shared memory is released
-    if (pt == 0)
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int lb = i ? last_bulk1 : last_bulk0;
-        if (lb >= 0) {
-          long it = 0;
-          while (!mbar_test(su32(&bars.kfull[i]), (lb >> 1) & 1) && ++it < kSpin) {
-          }
-          if (it >= kSpin) set_status(a.status, LC_DEV_TIMEOUT);
-        }
-      }
+    if (pt == 0) {
+      if (last_bulk0 >= 0) drain(&bars.kfull[0], (last_bulk0 >> 1) & 1);
+      if (last_bulk1 >= 0) drain(&bars.kfull[1], (last_bulk1 >> 1) & 1);
+    }
   } else if (warp == 8) {
-    // ================= MMA issue (one lane) =================
+    // ================= S MMA issue (one lane) =================
     if (lane == 0) {
-      // F16 operands, FP32 accumulator.  S: M = 64, N = 64, both K-major; O^T: M = 128 (or
-      // 64), N = 64, A (V^T) MN-major
+      // F16 operands, FP32 accumulator.  S: M = 64, N = 64, both K-major
       const uint32_t id_s = (1u << 4) | (static_cast<uint32_t>(kTK >> 3) << 17) |
                             (static_cast<uint32_t>(kNR >> 4) << 24);
+      const uint64_t dq = cm_desc(su32(Qs), 128, kG);
+      // S(ns) once its key stage is full and its S buffer read; S runs at most two tiles
+      // ahead of O (the key stage of S(no + 2) is released by O(no))
+      bool ok = n_tiles == 0 || wait(&bars.qfull, 0);
+      for (int ns = 0; ok && ns < n_tiles; ++ns) {
+        const int st = ns & 1;
+        ok = wait(&bars.kfull[st], (ns >> 1) & 1) && (ns < 2 || wait(&bars.sempty[st], ((ns >> 1) - 1) & 1));
+        if (!ok) break;
+        fence_after();
+        const uint64_t dk = cm_desc(su32(Ks + st * kTile), 128, kG);
+#pragma unroll
+        for (int k = 0; k < kD / 16; ++k)
+          mma_f16(tm + kColS + st * kTK, dq + k * 16, dk + k * 16, id_s, k > 0);
+        mma_commit(su32(&bars.sfull[st]));
+      }
+      mma_commit(su32(&bars.fin));
+      drain(&bars.fin, 0);  // every MMA issued above completes before tensor memory is released
+    }
+  } else if (warp == 9) {
+    // ================= O MMA issue (one lane) =================
+    if (lane == 0) {
+      // O^T: M = 128 (or 64), N = 64, A (V^T) MN-major, P^T K-major
       const uint32_t id_o128 = (1u << 4) | (1u << 15) |
                                (static_cast<uint32_t>(kNR >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
       const uint32_t id_o64 = (1u << 4) | (1u << 15) |
                               (static_cast<uint32_t>(kNR >> 3) << 17) | (static_cast<uint32_t>(64 >> 4) << 24);
-      const uint64_t dq = cm_desc(su32(Qs), 128, kG);
       const uint64_t dp = cm_desc(su32(Ps), 128, (kTK / 8) * 128);
-      // Issue whichever group is ready: S(ns) once its key stage is full and its S buffer
-      // read, O(no) once P(no) is written.  S runs at most two tiles ahead of O (the key
-      // stage of S(no + 2) is released by O(no)).
-      int ns = 0, no = 0;
-      long idle = 0;
-      bool ok = n_tiles == 0 || wait(&bars.qfull, 0);
-      while (ok && no < n_tiles) {
-        bool progressed = false;
-        if (ns < n_tiles) {
-          const int st = ns & 1;
-          if (mbar_probe(su32(&bars.kfull[st]), (ns >> 1) & 1) &&
-              (ns < 2 || mbar_probe(su32(&bars.sempty[st]), ((ns >> 1) - 1) & 1))) {
-            fence_after();
-            const uint64_t dk = cm_desc(su32(Ks + st * kTile), 128, kG);
+      // O(no) once P(no) is written (its S is then complete)
+      for (int no = 0; no < n_tiles; ++no) {
+        if (!wait(&bars.pfull, no & 1)) break;
+        fence_after();
+        // V^T: M = dims (chunk stride 128 B), K = keys (group stride kG)
+        const uint64_t dv = cm_desc(su32(Ks + (no & 1) * kTile), kG, 128);
 #pragma unroll
-            for (int k = 0; k < kD / 16; ++k)
-              mma_f16(tm + kColS + st * kTK, dq + k * 16, dk + k * 16, id_s, k > 0);
-            mma_commit(su32(&bars.sfull[st]));
-            ++ns;
-            progressed = true;
-          }
-        }
-        if (no < ns && mbar_probe(su32(&bars.pfull), no & 1)) {
-          fence_after();
-          // V^T: M = dims (chunk stride 128 B), K = keys (group stride kG); P^T: K-major
-          const uint64_t dv = cm_desc(su32(Ks + (no & 1) * kTile), kG, 128);
+        for (int kk = 0; kk < kTK / 16; ++kk)
 #pragma unroll
-          for (int kk = 0; kk < kTK / 16; ++kk)
-#pragma unroll
-            for (int c = 0; c < 5; ++c)
-              if (c < n_och)
-                mma_f16(tm + kColO + c * kNR, dv + (c * 2048 + kk * 2 * kG) / 16, dp + kk * 16,
-                        c < 4 ? id_o128 : id_o64, (no > 0) || (kk > 0));
-          mma_commit(su32(&bars.kempty[no & 1]));
-          mma_commit(su32(&bars.pempty));
-          ++no;
-          progressed = true;
-        }
-        if (progressed) {
-          idle = 0;
-        } else if (++idle >= kSpin) {
-          set_status(a.status, LC_DEV_TIMEOUT);
-          atomicExch(&s_abort, 1);
-          ok = false;
-        } else if ((idle & 1023) == 0 && *reinterpret_cast<volatile int*>(&s_abort)) {
-          ok = false;
-        }
+          for (int c = 0; c < 5; ++c)
+            if (c < n_och)
+              mma_f16(tm + kColO + c * kNR, dv + (c * 2048 + kk * 2 * kG) / 16, dp + kk * 16,
+                      c < 4 ? id_o128 : id_o64, (no > 0) || (kk > 0));
+        mma_commit(su32(&bars.kempty[no & 1]));
+        mma_commit(su32(&bars.pempty));
       }
-      mma_commit(su32(&bars.fin));
-      wait(&bars.fin, 0);
+      mma_commit(su32(&bars.fin2));
+      drain(&bars.fin2, 0);  // every O MMA completes before tensor memory is released
     }
   } else {
     // ================= warps 0-3: Q, softmax, epilogue =================

@@ -244,6 +244,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     atomicExch(&s_abort, 1);
     return false;
   };
+  // bounded wait that ignores the abort flag: for copies and MMAs already in flight, which
+  // must land before the CTA releases its tensor memory and exits
+  auto drain = [&](uint64_t* bar, uint32_t parity) {
+    const uint32_t addr = su32(bar);
+    for (long it = 0; it < kSpin; ++it)
+      if (mbar_test(addr, parity)) return;
+    set_status(a.status, LC_DEV_TIMEOUT);
+  };
   // first slot of tile t
   // window tiles come first (their rows are on hand while the entry gathers start): tile t
   // is window tile t for t < n_wt, entry tile t - n_wt after that
@@ -327,6 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int cb = 0; cb < 4; ++cb) tma_tile2d(su32(Qn + cb * kBlk), &tqn, cb * 128, static_cast<int>(row0), qb);
       tma_tile2d(su32(Qr), &tqr, 0, static_cast<int>(row0), qb);
     }
+    int e_last0 = -1, e_last1 = -1;  // lane 0: the last entry tile of stage 0 / 1 this warp copied
     for (int t = 0; t < n_tiles; ++t) {
       const int cb4 = t & 3;
       // the top-k indices may be the previous kernel's output (programmatic dependent
@@ -348,7 +357,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (e >= 0) {
         const int st = e & 1;
         const uint32_t kb = su32(&bars.kfull[st]);
-        if (lane == 0) mbar_expect_tx(kb, kRawStage / kCopyWarps);
+        if (lane == 0) {
+          mbar_expect_tx(kb, kRawStage / kCopyWarps);
+          (st ? e_last1 : e_last0) = e;
+        }
         __syncwarp();
         if (lane < 4) {
           // rows 4 g .. 4 g + 3 of the tile, g = 4 cw + lane; a masked key reads row 0 (its
@@ -367,6 +379,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_gather4(su32(stage + kRawN + g * 512), &tkr, 0, rr[0], rr[1], rr[2], rr[3], kb);
         }
       }
+    }
+    // a role that gave up may leave copies in flight: they land before the CTA exits (a
+    // stage's phase also needs the other copy warps' parts, so this wait is bounded too)
+    if (lane == 0) {
+      if (e_last0 >= 0) drain(&bars.kfull[0], (e_last0 >> 1) & 1);
+      if (e_last1 >= 0) drain(&bars.kfull[1], (e_last1 >> 1) & 1);
+      if (cw == 0 && n_tiles > 0) drain(&bars.qfull, 0);
     }
   } else if (warp == 8) {
     // ================= MMA issue (one lane) =================
@@ -463,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       mma_commit(su32(&bars.fin));
-      wait(&bars.fin, 0);
+      drain(&bars.fin, 0);  // every MMA issued above completes before tensor memory is released
     }
   } else if (warp >= 4) {
     // ================= converters: raw or window rows -> F16 tile =================
@@ -471,6 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r8 = ct & 7;     // row within a group of 8 (one quarter warp: 8 rows, one chunk)
     __half2 amax = __float2half2_rn(0.f);
     bool ok = true;
+    int w_last = -1;  // thread ct = 0: the last window tile it copied
     for (int t = 0; ok && t < n_tiles; ++t) {
       if (t < n_wt) {
         // window tile: its rows are consecutive, so it comes as one 64 x 64 BF16 box per 64
@@ -489,6 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int y = static_cast<int>(wr0) + (ring > 0 ? t0 % ring : t0 - wp0);
 #pragma unroll
           for (int cb = 0; cb < kD / 64; ++cb) tma_tile2d(su32(Vt + cb * kBlk), &twin, cb * 64, y, wb);
+          w_last = t;
         }
       }
       if (t == 0 && n_wt > 0) {
@@ -591,6 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (f16_inf(amax)) set_status(a.status, LC_DEV_RANGE);
+    if (ct == 0 && w_last >= 0) drain(&bars.wfull, w_last & 1);  // a window copy in flight lands first
   } else {
     // ================= warps 0-3: softmax, epilogue =================
     const int r = warp * 16 + (lane & 15);
