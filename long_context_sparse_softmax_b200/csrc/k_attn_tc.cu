@@ -273,7 +273,7 @@ struct TcBars {
   uint64_t fin2;       // every O MMA complete (commit)
 };
 
-// grid: one CTA per (query, head group, key split), the split index fastest; 288 threads.
+// grid: one CTA per (query, head group, key split), the split index fastest; 320 threads.
 // Partial results of split s go to ws_o rows s * n_q * H + q * H + h (576 floats each) and
 // ws_ml[2 ((q * H + h) * n_split + s) + {0, 1}] = (m, l).  img (dense keys only, or null):
 // the entries as F16 tiles (k_attn_f16_tiles), img_tiles of them; a tile of 64 visible
